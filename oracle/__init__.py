@@ -1,0 +1,248 @@
+"""Plain float64 CPU oracle for the RAT+ dilated-inference hot path.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline call this package; the CUDA library never imports it and shares no code with it.
+
+The arithmetic lives in ``oracle.c`` (plain loops in float64, one routine per definition);
+this module only builds it, marshals numpy arrays and composes the routines in the order
+the pages give: recurrence over keys and values, RoPE on the recurrence output and on the
+query, then attention over the dilated-plus-window key set.
+
+Sources: "RAT+ Deep Dive" section 2.1 (full-sequence forget-gate recurrence, associative
+scan prefill), section 3.1 table (FLOPs T/D), section 6 (head-wise hybrid); the RAT+
+abstract (dilation D, optional local windows, D-fold KV-cache reduction); RoFormer (RoPE).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_ip = ctypes.POINTER(ctypes.c_int)
+_lp = ctypes.POINTER(ctypes.c_long)
+_bp = ctypes.POINTER(ctypes.c_uint8)
+_L = ctypes.c_long
+
+
+def build(force: bool = False) -> str:
+    """Compile oracle.c into liboracle.so next to it (gcc, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c11",
+                               _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.rat_oracle_recurrence.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp]
+        lib.rat_oracle_rope.argtypes = [_L, _L, _L, _dp, _L, ctypes.c_double]
+        lib.rat_oracle_in_key_set.argtypes = [_L, _L, _L, _L]
+        lib.rat_oracle_in_key_set.restype = ctypes.c_int
+        lib.rat_oracle_key_count.argtypes = [_L, _L, _L]
+        lib.rat_oracle_key_count.restype = ctypes.c_long
+        lib.rat_oracle_dilated_attention.argtypes = [_L, _L, _L, _dp, _dp, _dp, _ip, _L,
+                                                     ctypes.c_double, _lp, _L, _dp]
+        lib.rat_oracle_kv_compress.argtypes = [_L, _L, _L, _L, _L, _bp, _ip, _L, _L, _L, _bp, _bp]
+        lib.rat_oracle_decode_step.argtypes = [_L, _L, _L, _ip, _L, ctypes.c_double,
+                                               ctypes.c_double, _dp, _dp, _dp, _dp, _dp, _dp,
+                                               _dp, _dp, _L, _dp]
+        lib.rat_oracle_threads.restype = ctypes.c_int
+        lib.rat_oracle_set_threads.argtypes = [ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray, kind=_dp):
+    return a.ctypes.data_as(kind)
+
+
+def threads() -> int:
+    return int(_load().rat_oracle_threads())
+
+
+def set_threads(n: int) -> None:
+    _load().rat_oracle_set_threads(int(n))
+
+
+def default_scale(d: int) -> float:
+    """Softmax scale 1/sqrt(d_head) (standard attention; the pages state none)."""
+    return 1.0 / np.sqrt(d)
+
+
+def recurrence(x, a, h0=None):
+    """h_t = g_t h_{t-1} + (1-g_t) x_t, g = sigmoid(a), per channel, over the full sequence.
+
+    x, a: (..., T, d).  h0: (..., d) or None (zeros).  Returns (y, hT) in float64.
+    ("RAT+ Deep Dive" section 2.1, full-sequence recurrence, L = T.)
+    """
+    x = _f64(x)
+    a = _f64(a)
+    assert x.shape == a.shape
+    T, d = x.shape[-2], x.shape[-1]
+    BH = int(np.prod(x.shape[:-2])) if x.ndim > 2 else 1
+    y = np.empty_like(x)
+    hT = np.empty(x.shape[:-2] + (d,), dtype=np.float64)
+    h0p = None
+    if h0 is not None:
+        h0 = _f64(h0)
+        assert h0.shape == hT.shape
+        h0p = _ptr(h0)
+    _load().rat_oracle_recurrence(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(y), _ptr(hT))
+    return y, hT
+
+
+def rope(x, pos0: int = 0, base: float = 10000.0):
+    """Rotate-half RoPE at positions pos0 + t (RoFormer).  Returns a new float64 array."""
+    x = _f64(x).copy()
+    T, d = x.shape[-2], x.shape[-1]
+    BH = int(np.prod(x.shape[:-2])) if x.ndim > 2 else 1
+    _load().rat_oracle_rope(BH, T, d, _ptr(x), int(pos0), float(base))
+    return x
+
+
+def in_key_set(t: int, j: int, D: int, W: int) -> bool:
+    """Is key j in the key set of query t (window (t-We, t] union chunk ends older than it)?"""
+    return bool(_load().rat_oracle_in_key_set(int(t), int(j), int(D), int(W)))
+
+
+def key_count(t: int, D: int, W: int) -> int:
+    """|S(t)| by enumeration."""
+    return int(_load().rat_oracle_key_count(int(t), int(D), int(W)))
+
+
+def _per_bh_dilation(shape_bh, D, D_per_head):
+    B, H = shape_bh
+    if D_per_head is None:
+        Dh = np.full((H,), int(D), dtype=np.int32)
+    else:
+        Dh = np.asarray(D_per_head, dtype=np.int32)
+        assert Dh.shape == (H,)
+    return np.ascontiguousarray(np.tile(Dh, B).astype(np.int32)), Dh
+
+
+def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None):
+    """Causal dilated attention (+ local window, per-head D) over (B, H, T, d) tensors.
+
+    q, k, v are used as given (rotate them first if RoPE is in use).  rows: optional list of
+    query positions; the result then has shape (B, H, len(rows), d).
+    (RAT+ abstract; "RAT+ Deep Dive" section 3.1 table and section 6 head-wise hybrid.)
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, T, d = q.shape
+    Dbh, _ = _per_bh_dilation((B, H), D, D_per_head)
+    if scale is None:
+        scale = default_scale(d)
+    if rows is None:
+        nrows, rp = T, None
+        out = np.empty((B, H, T, d))
+    else:
+        rows_a = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        assert rows_a.min() >= 0 and rows_a.max() < T
+        nrows, rp = len(rows_a), _ptr(rows_a, _lp)
+        out = np.empty((B, H, nrows, d))
+    _load().rat_oracle_dilated_attention(B * H, T, d, _ptr(q), _ptr(k), _ptr(v), _ptr(Dbh, _ip),
+                                         int(W), float(scale), rp, nrows, _ptr(out))
+    return out
+
+
+def layer_prefill(q, k, v, a, D=1, W=0, D_per_head=None, rope_base=0.0, pos0=0, scale=None,
+                  rows=None, h0_k=None, h0_v=None):
+    """The whole prefill path in float64: recurrence -> RoPE -> dilated attention.
+
+    Returns dict(o, k_rec, v_rec, hT_k, hT_v); k_rec is the recurrence output after RoPE
+    (what the cache stores), v_rec the value recurrence output.
+    """
+    k_rec, hT_k = recurrence(k, a, h0_k)
+    v_rec, hT_v = recurrence(v, a, h0_v)
+    qr = _f64(q)
+    if rope_base > 0:
+        k_rec = rope(k_rec, pos0, rope_base)
+        qr = rope(qr, pos0, rope_base)
+    o = dilated_attention(qr, k_rec, v_rec, D=D, W=W, D_per_head=D_per_head, scale=scale, rows=rows)
+    return dict(o=o, k_rec=k_rec, v_rec=v_rec, hT_k=hT_k, hT_v=hT_v)
+
+
+def cache_capacity(Tcap: int, D_per_head) -> np.ndarray:
+    """cap_h = floor(Tcap / D_h): the compressed cache keeps one key per chunk of D."""
+    return np.asarray([Tcap // int(Dh) for Dh in D_per_head], dtype=np.int64)
+
+
+def kv_compress(x, D_per_head, W: int, Tcap: int, pos0: int = 0, dil=None, ring=None):
+    """Bit-exact gather of a (B, H, T, d) tensor of any element type into the cache layout.
+
+    Returns (dil, ring): dil (B, sum_h cap_h, d), ring (B, H, W, d) (or None if W == 0), of
+    x's dtype; existing dil/ring arrays are updated in place (chunked prefill).
+    """
+    x = np.ascontiguousarray(x)
+    B, H, T, d = x.shape
+    Dh = np.ascontiguousarray(np.asarray(D_per_head, dtype=np.int32))
+    total = int(cache_capacity(Tcap, Dh).sum())
+    if dil is None:
+        dil = np.zeros((B, total, d), dtype=x.dtype)
+    if ring is None and W > 0:
+        ring = np.zeros((B, H, W, d), dtype=x.dtype)
+    xb = x.view(np.uint8)
+    _load().rat_oracle_kv_compress(B, H, T, d, x.dtype.itemsize, _ptr(xb, _bp), _ptr(Dh, _ip),
+                                   int(W), int(Tcap), int(pos0), _ptr(dil.view(np.uint8), _bp),
+                                   _ptr(ring.view(np.uint8), _bp) if ring is not None else None)
+    return dil, ring
+
+
+class DecodeState:
+    """Float64 decode oracle: recurrence state plus the full history of k~ and v~.
+
+    Keeping every position is the plain definition (the compressed cache is an optimisation
+    of it); use it on a few (batch, head) slices.  Dbh gives each slice's dilation.
+    """
+
+    def __init__(self, Dbh, d: int, W: int, Tcap: int, rope_base: float = 0.0, scale=None):
+        self.Dbh = np.ascontiguousarray(np.asarray(Dbh, dtype=np.int32))
+        self.BH = len(self.Dbh)
+        self.d, self.W, self.Tcap = d, int(W), int(Tcap)
+        self.rope_base = float(rope_base)
+        self.scale = default_scale(d) if scale is None else float(scale)
+        self.hk = np.zeros((self.BH, d))
+        self.hv = np.zeros((self.BH, d))
+        self.khist = np.zeros((self.BH, self.Tcap, d))
+        self.vhist = np.zeros((self.BH, self.Tcap, d))
+        self.t = 0
+
+    def prefill(self, k, v, a):
+        """Consume a context (BH, T, d) with the sequential recurrence and record history."""
+        k, v, a = _f64(k), _f64(v), _f64(a)
+        T = k.shape[-2]
+        yk, hk = recurrence(k, a, self.hk)
+        yv, hv = recurrence(v, a, self.hv)
+        if self.rope_base > 0:
+            yk = rope(yk, self.t, self.rope_base)
+        self.khist[:, self.t:self.t + T] = yk
+        self.vhist[:, self.t:self.t + T] = yv
+        self.hk, self.hv = np.ascontiguousarray(hk), np.ascontiguousarray(hv)
+        self.t += T
+
+    def step(self, q, k, v, a):
+        """One new token per slice: (BH, d) inputs -> (BH, d) output."""
+        q, k, v, a = _f64(q), _f64(k), _f64(v), _f64(a)
+        o = np.empty((self.BH, self.d))
+        _load().rat_oracle_decode_step(self.BH, self.d, self.t, _ptr(self.Dbh, _ip), self.W,
+                                       self.scale, self.rope_base, _ptr(q), _ptr(k), _ptr(v),
+                                       _ptr(a), _ptr(self.hk), _ptr(self.hv), _ptr(self.khist),
+                                       _ptr(self.vhist), self.Tcap, _ptr(o))
+        self.t += 1
+        return o

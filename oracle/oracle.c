@@ -1,0 +1,294 @@
+/*
+ * oracle.c -- plain, slow, float64 CPU oracle for the RAT+ dilated-inference hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  The tests, the smoke check and the benchmark's CPU-baseline leg
+ * call this code; the library under recurrence_augmented_dilated_b200/ never does, and the two
+ * share no source, header, table or helper.  Every routine is the written-out definition of
+ * what it computes, with no blocking, fusion or reordering: loops in the order of the maths.
+ *
+ * Sources (page title, section):
+ *   [RAT+ Deep Dive]  "RAT+ Deep Dive: A New KV Cache Compression Paradigm ...", section 2.1
+ *                     "Full-Sequence Recurrence" (forget-gate recurrence over the whole
+ *                     sequence, L = T, computed by an associative scan in prefill);
+ *                     section 3.1 table (attention FLOPs T/D); section 6 "Head-Wise Hybrid".
+ *   [RAT+ abstract]   "RAT+: Train Dense, Infer Sparse -- Recurrence Augmented Attention for
+ *                     Dilated Inference", abstract (dilation D cuts attention FLOPs and KV cache
+ *                     by D; optional local windows; hybrid layer/head compositions).
+ *   [RAT abstract]    "RAT: Bridging RNN Efficiency and Attention Accuracy via Chunk-based
+ *                     Sequence Modeling", abstract (recurrence inside chunks, attention across
+ *                     chunk ends).
+ *   [RoFormer]        rotary position embedding, cited by the RAT+ page; rotate-half pairing.
+ *
+ * The recurrence formula itself is lost from the blog's section 2.1 (only "forget-gate
+ * mechanism ... g_l is an input-dependent forget gate, LSTM-like decaying memory" survives);
+ * the form used here is the standard gated EMA  h_t = g_t * h_{t-1} + (1 - g_t) * x_t with
+ * g_t = sigmoid(a_t), elementwise per channel, the same gate for keys and values.
+ *
+ * Readings taken where the pages are silent (each one is listed in the design notes):
+ *   - the gate logit tensor is one (B,H,T,d) tensor shared by K and V;
+ *   - h_{-1} = h0 (zero unless given);
+ *   - key set of query t:  S(t) = { j : t - We < j <= t }  U  { j : j <= t - We, j mod D = D-1 },
+ *     with We = max(W, 1): the query always sees its own recurrence output, the dilated keys
+ *     are the chunk ends (positions D-1, 2D-1, ...) older than the window, the union is disjoint;
+ *   - RoPE is applied to the recurrence output k~ (not to the raw k) and to q, at the absolute
+ *     position pos0 + t, rotate-half pairing (c, c + d/2), theta_c = base^(-2c/d);
+ *   - softmax scale is 1/sqrt(d) unless the caller gives one.
+ *
+ * Build: gcc -O2 -fopenmp -shared -fPIC oracle.c -o liboracle.so -lm  (see build.py).
+ * OpenMP parallelism is over independent (batch, head) slices only.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ---------------------------------------------------------------------------------------- */
+/* Forget gate.  g = sigmoid(a) = 1/(1+e^{-a});  1-g = 1/(1+e^{a}) (computed directly so that
+ * it keeps full relative precision when g is close to 1).                [RAT+ Deep Dive 2.1] */
+static double forget_gate(double a) { return 1.0 / (1.0 + exp(-a)); }
+static double one_minus_gate(double a) { return 1.0 / (1.0 + exp(a)); }
+
+/*
+ * Full-sequence forget-gate recurrence, one tensor at a time.               [RAT+ Deep Dive 2.1]
+ *   x, a, y : [BH][T][d]      h0, hT : [BH][d] (either may be NULL; NULL h0 means zeros)
+ *   h_{-1} = h0;   h_t = g_t * h_{t-1} + (1 - g_t) * x_t;   y_t = h_t;   hT = h_{T-1}.
+ * A sequential loop over t: the definition itself, no scan.
+ */
+void rat_oracle_recurrence(long BH, long T, long d, const double *x, const double *a,
+                           const double *h0, double *y, double *hT)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        for (long c = 0; c < d; ++c) {
+            double h = h0 ? h0[bh * d + c] : 0.0;
+            for (long t = 0; t < T; ++t) {
+                long idx = (bh * T + t) * d + c;
+                double g = forget_gate(a[idx]);
+                double omg = one_minus_gate(a[idx]);
+                h = g * h + omg * x[idx];
+                y[idx] = h;
+            }
+            if (hT) hT[bh * d + c] = h;
+        }
+    }
+}
+
+/*
+ * Rotary position embedding, rotate-half pairing, in place.                  [RoFormer]
+ *   x : [BH][T][d];  position of row t is pos0 + t;  for c < d/2:
+ *   theta_c = base^(-2c/d),  phi = (pos0 + t) * theta_c,
+ *   (x_c, x_{c+d/2}) <- (x_c cos phi - x_{c+d/2} sin phi,  x_{c+d/2} cos phi + x_c sin phi).
+ */
+void rat_oracle_rope(long BH, long T, long d, double *x, long pos0, double base)
+{
+    long half = d / 2;
+#pragma omp parallel for schedule(static)
+    for (long bh = 0; bh < BH; ++bh) {
+        for (long t = 0; t < T; ++t) {
+            double *row = x + (bh * T + t) * d;
+            for (long c = 0; c < half; ++c) {
+                double theta = pow(base, -2.0 * (double)c / (double)d);
+                double phi = (double)(pos0 + t) * theta;
+                double cs = cos(phi), sn = sin(phi);
+                double x1 = row[c], x2 = row[c + half];
+                row[c] = x1 * cs - x2 * sn;
+                row[c + half] = x2 * cs + x1 * sn;
+            }
+        }
+    }
+}
+
+/* Effective window: a query always sees at least itself.                                     */
+static long eff_window(long W) { return W > 1 ? W : 1; }
+
+/*
+ * Membership of key j in the key set of query t (the definition, as a predicate).
+ *                                                     [RAT+ abstract; RAT+ Deep Dive 3.1, 6]
+ */
+int rat_oracle_in_key_set(long t, long j, long D, long W)
+{
+    long We = eff_window(W);
+    if (j < 0 || j > t) return 0;
+    if (j > t - We) return 1;            /* local window, the query's own position included */
+    return (j % D) == (D - 1);           /* dilated key: a chunk end older than the window  */
+}
+
+/* |S(t)|: number of keys query t attends to, counted by enumerating the set.                */
+long rat_oracle_key_count(long t, long D, long W)
+{
+    long n = 0;
+    for (long j = 0; j <= t; ++j) n += rat_oracle_in_key_set(t, j, D, W);
+    return n;
+}
+
+/*
+ * Causal dilated attention with an optional local window and a per-(batch,head) dilation.
+ *                                   [RAT+ abstract; RAT+ Deep Dive 3.1 table, 6 Head-Wise Hybrid]
+ *   q, k, v : [BH][T][d]  (q and k already rotated if RoPE is in use; k, v are the recurrence
+ *                          outputs k~, v~)
+ *   Dbh     : [BH]        dilation of each (batch, head) slice
+ *   rows    : [nrows]     query positions to evaluate (NULL: all T rows, nrows = T)
+ *   o       : [BH][nrows][d]
+ * For each query t:  s_j = scale * <q_t, k_j>  for j in S(t);
+ *                    o_t = sum_j exp(s_j - max s) v_j / sum_j exp(s_j - max s).
+ * S(t) is enumerated as its two parts: the window t-We < j <= t, then the chunk ends
+ * j = D-1, 2D-1, ... with j <= t - We.
+ */
+void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, const double *k,
+                                  const double *v, const int *Dbh, long W, double scale,
+                                  const long *rows, long nrows, double *o)
+{
+    long We = eff_window(W);
+    if (!rows) nrows = T;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        long D = Dbh[bh];
+        long *keys = (long *)malloc(sizeof(long) * (size_t)(T + 1));
+        double *s = (double *)malloc(sizeof(double) * (size_t)(T + 1));
+        for (long r = 0; r < nrows; ++r) {
+            long t = rows ? rows[r] : r;
+            long n = 0;
+            for (long j = (t - We + 1 > 0 ? t - We + 1 : 0); j <= t; ++j) keys[n++] = j;
+            for (long j = D - 1; j <= t - We; j += D) keys[n++] = j;
+            const double *qt = q + (bh * T + t) * d;
+            double mx = -INFINITY;
+            for (long m = 0; m < n; ++m) {
+                const double *kj = k + (bh * T + keys[m]) * d;
+                double dot = 0.0;
+                for (long c = 0; c < d; ++c) dot += qt[c] * kj[c];
+                s[m] = scale * dot;
+                if (s[m] > mx) mx = s[m];
+            }
+            double *ot = o + (bh * nrows + r) * d;
+            for (long c = 0; c < d; ++c) ot[c] = 0.0;
+            double l = 0.0;
+            for (long m = 0; m < n; ++m) {
+                double p = exp(s[m] - mx);
+                const double *vj = v + (bh * T + keys[m]) * d;
+                l += p;
+                for (long c = 0; c < d; ++c) ot[c] += p * vj[c];
+            }
+            for (long c = 0; c < d; ++c) ot[c] /= l;
+        }
+        free(keys);
+        free(s);
+    }
+}
+
+/*
+ * Compressed KV cache build, on raw element bytes (bit-exact gather).      [RAT+ abstract]
+ *   x    : [B][H][T][d] elements of esize bytes: the recurrence outputs of positions
+ *          pos0 .. pos0+T-1
+ *   Dh   : [H] per-head dilation;  cap_h = floor(Tcap / D_h);  off_h = sum_{h' < h} cap_h'
+ *   dil  : [B][sum_h cap_h][d]   entry i of head h = position i*D_h + D_h - 1
+ *   ring : [B][H][W][d]          position p lives in slot p mod W  (ring may be NULL if W == 0)
+ * Every position p of this chunk with p mod D_h = D_h - 1 and p / D_h < cap_h is stored in
+ * dil; every position among the last W of the sequence so far is stored in ring.
+ */
+void rat_oracle_kv_compress(long B, long H, long T, long d, long esize, const uint8_t *x,
+                            const int *Dh, long W, long Tcap, long pos0, uint8_t *dil,
+                            uint8_t *ring)
+{
+    long total_cap = 0;
+    for (long h = 0; h < H; ++h) total_cap += Tcap / Dh[h];
+    long row_bytes = d * esize;
+    for (long b = 0; b < B; ++b) {
+        long off = 0;
+        for (long h = 0; h < H; ++h) {
+            long D = Dh[h], cap = Tcap / D;
+            for (long t = 0; t < T; ++t) {
+                long p = pos0 + t;
+                const uint8_t *src = x + ((b * H + h) * T + t) * row_bytes;
+                if (p % D == D - 1 && p / D < cap)
+                    memcpy(dil + (b * total_cap + off + p / D) * row_bytes, src, (size_t)row_bytes);
+                if (W > 0 && p >= pos0 + T - W)
+                    memcpy(ring + ((b * H + h) * W + p % W) * row_bytes, src, (size_t)row_bytes);
+            }
+            off += cap;
+        }
+    }
+}
+
+/*
+ * One decode step for a new token at absolute position t, per (batch, head) slice.
+ *                                           [RAT+ Deep Dive 2.1; RAT+ abstract; RoFormer]
+ *   q, k, v, a   : [BH][d]          the new token's query, key, value, gate logit
+ *   hk, hv       : [BH][d]          recurrence state (before RoPE), updated in place
+ *   khist, vhist : [BH][Tcap][d]    every earlier k~ (rotated) and v~; row t is written here
+ *   Dbh          : [BH]             dilation per slice
+ *   o            : [BH][d]
+ * State update h = g*h + (1-g)*x for k and v; k~_t = RoPE(h_k, t) (if rope_base > 0); the
+ * query is RoPE(q, t); attention over S(t) exactly as in the prefill definition.
+ */
+void rat_oracle_decode_step(long BH, long d, long t, const int *Dbh, long W, double scale,
+                            double rope_base, const double *q, const double *k, const double *v,
+                            const double *a, double *hk, double *hv, double *khist,
+                            double *vhist, long Tcap, double *o)
+{
+    long We = eff_window(W);
+    long half = d / 2;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        long D = Dbh[bh];
+        double *kt = khist + (bh * Tcap + t) * d;
+        double *vt = vhist + (bh * Tcap + t) * d;
+        double *qr = (double *)malloc(sizeof(double) * (size_t)d);
+        for (long c = 0; c < d; ++c) {
+            long idx = bh * d + c;
+            double g = forget_gate(a[idx]), omg = one_minus_gate(a[idx]);
+            hk[idx] = g * hk[idx] + omg * k[idx];
+            hv[idx] = g * hv[idx] + omg * v[idx];
+            kt[c] = hk[idx];
+            vt[c] = hv[idx];
+            qr[c] = q[idx];
+        }
+        if (rope_base > 0.0) {
+            for (long c = 0; c < half; ++c) {
+                double theta = pow(rope_base, -2.0 * (double)c / (double)d);
+                double phi = (double)t * theta, cs = cos(phi), sn = sin(phi);
+                double x1 = kt[c], x2 = kt[c + half];
+                kt[c] = x1 * cs - x2 * sn;
+                kt[c + half] = x2 * cs + x1 * sn;
+                x1 = qr[c];
+                x2 = qr[c + half];
+                qr[c] = x1 * cs - x2 * sn;
+                qr[c + half] = x2 * cs + x1 * sn;
+            }
+        }
+        long nmax = We + t / D + 2, n = 0;
+        long *keys = (long *)malloc(sizeof(long) * (size_t)nmax);
+        double *s = (double *)malloc(sizeof(double) * (size_t)nmax);
+        for (long j = (t - We + 1 > 0 ? t - We + 1 : 0); j <= t; ++j) keys[n++] = j;
+        for (long j = D - 1; j <= t - We; j += D) keys[n++] = j;
+        double mx = -INFINITY;
+        for (long m = 0; m < n; ++m) {
+            const double *kj = khist + (bh * Tcap + keys[m]) * d;
+            double dot = 0.0;
+            for (long c = 0; c < d; ++c) dot += qr[c] * kj[c];
+            s[m] = scale * dot;
+            if (s[m] > mx) mx = s[m];
+        }
+        double *ot = o + bh * d, l = 0.0;
+        for (long c = 0; c < d; ++c) ot[c] = 0.0;
+        for (long m = 0; m < n; ++m) {
+            double p = exp(s[m] - mx);
+            const double *vj = vhist + (bh * Tcap + keys[m]) * d;
+            l += p;
+            for (long c = 0; c < d; ++c) ot[c] += p * vj[c];
+        }
+        for (long c = 0; c < d; ++c) ot[c] /= l;
+        free(keys);
+        free(s);
+        free(qr);
+    }
+}
+
+/* Number of OpenMP threads the oracle will use (for reporting the CPU baseline's cores).     */
+#ifdef _OPENMP
+#include <omp.h>
+int rat_oracle_threads(void) { return omp_get_max_threads(); }
+void rat_oracle_set_threads(int n) { omp_set_num_threads(n); }
+#else
+int rat_oracle_threads(void) { return 1; }
+void rat_oracle_set_threads(int n) { (void)n; }
+#endif

@@ -1,0 +1,110 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the smoke check.
+
+This module holds no arithmetic of the method: it only draws normal random numbers with a
+seeded torch generator and casts them to the run's dtype.  Both the CUDA library's callers and
+the float64 oracle take their inputs from here.
+
+Workloads (shapes of the pages' 1.5B / 2.6B / 7.6B-model layers; the pages evaluate on
+FineWeb-Edu, LongBench, commonsense and NIAH suites, which these random tensors stand in for):
+
+  tiny_fp32      B1  H2  d64  T256    D4          W0    fp32  gates N(2,1)
+  prefill_1p5b   B4  H16 d128 T4096   D16         W0    bf16  gates N(2,1)   RoPE base 10000
+  window_2p6b    B2  H20 d128 T16384  D64         W128  bf16  gates N(3,1)
+  hybrid_7p6b    B1  H32 d128 T32768  D1 x8, D64 x24  W64  bf16  gates N(2,1.5)
+  decode_7p6b    B32 H32 d128 context 65536, D64 W128, 256 one-token steps, gates N(2,1)
+
+Recipe (prefill): one CPU ``torch.Generator`` seeded with the workload's seed draws float32
+standard normals in the order q, k, v, a (a = mu + sigma * N(0,1)), each (B, H, T, d); the
+results are then cast to the dtype.  Decode: the context k, v, a of slice (b, h) come from a
+generator seeded with (seed, b, h) on the requested device, so one slice can be regenerated
+alone; the per-step tokens come from one CPU generator, drawn as q, k, v, a of shape
+(steps, B, H, d).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import List, Optional
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    d: int
+    T: int
+    D: int = 1
+    W: int = 0
+    D_per_head: Optional[tuple] = None
+    dtype: str = "bf16"
+    gate_mu: float = 2.0
+    gate_sigma: float = 1.0
+    rope_base: float = 0.0
+    seed: int = 0
+    steps: int = 0          # decode steps (decode workloads only)
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    def heads_D(self) -> List[int]:
+        if self.D_per_head is not None:
+            return list(self.D_per_head)
+        return [self.D] * self.H
+
+
+WORKLOADS = {
+    "tiny_fp32": Workload("tiny_fp32", B=1, H=2, d=64, T=256, D=4, W=0, dtype="f32",
+                          gate_mu=2.0, gate_sigma=1.0, seed=0),
+    "prefill_1p5b": Workload("prefill_1p5b", B=4, H=16, d=128, T=4096, D=16, W=0, dtype="bf16",
+                             gate_mu=2.0, gate_sigma=1.0, rope_base=10000.0, seed=1),
+    "window_2p6b": Workload("window_2p6b", B=2, H=20, d=128, T=16384, D=64, W=128, dtype="bf16",
+                            gate_mu=3.0, gate_sigma=1.0, seed=2),
+    "hybrid_7p6b": Workload("hybrid_7p6b", B=1, H=32, d=128, T=32768, W=64,
+                            D_per_head=tuple([1] * 8 + [64] * 24), dtype="bf16",
+                            gate_mu=2.0, gate_sigma=1.5, seed=3),
+    "decode_7p6b": Workload("decode_7p6b", B=32, H=32, d=128, T=65536, D=64, W=128, dtype="bf16",
+                            gate_mu=2.0, gate_sigma=1.0, seed=4, steps=256),
+}
+
+
+def prefill_inputs(w: Workload, B=None, H=None, T=None, seed=None):
+    """q, k, v, a on the CPU in w's dtype, shape (B, H, T, d); sizes may be overridden."""
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    T = w.T if T is None else T
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed if seed is None else seed)
+    shape = (B, H, T, w.d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    a = torch.randn(shape, generator=g, dtype=torch.float32) * w.gate_sigma + w.gate_mu
+    dt = w.torch_dtype
+    return {"q": q.to(dt), "k": k.to(dt), "v": v.to(dt), "a": a.to(dt)}
+
+
+def decode_context_slice(w: Workload, b: int, h: int, device="cpu", T=None):
+    """Context k, v, a of one (batch, head) slice, shape (T, d) each, on `device`."""
+    T = w.T if T is None else T
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed * 1_000_003 + b * 1009 + h + 1)
+    kva = torch.randn((3, T, w.d), generator=g, dtype=torch.float32, device=device)
+    kva[2].mul_(w.gate_sigma).add_(w.gate_mu)
+    return kva.to(w.torch_dtype)
+
+
+def decode_steps(w: Workload, steps=None):
+    """Per-step new tokens q, k, v, a, each (steps, B, H, d), on the CPU in w's dtype."""
+    steps = w.steps if steps is None else steps
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed * 7919 + 17)
+    shape = (steps, w.B, w.H, w.d)
+    q = torch.randn(shape, generator=g, dtype=torch.float32)
+    k = torch.randn(shape, generator=g, dtype=torch.float32)
+    v = torch.randn(shape, generator=g, dtype=torch.float32)
+    a = torch.randn(shape, generator=g, dtype=torch.float32) * w.gate_sigma + w.gate_mu
+    dt = w.torch_dtype
+    return {"q": q.to(dt), "k": k.to(dt), "v": v.to(dt), "a": a.to(dt)}

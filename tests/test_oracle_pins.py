@@ -1,0 +1,299 @@
+"""Pins of the float64 oracle to facts other than itself (CPU only).
+
+Each test checks the oracle against a closed form, a special case that reduces to a textbook
+or library routine (torch's scaled-dot-product attention in float64), an invariant of the
+method, brute force on tiny inputs, or a number the pages print.  The brute-force references
+here are built by slicing and explicit products, not by calling the oracle's own predicate.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(1234)
+
+
+def sdpa(q, k, v, causal=False, scale=None):
+    """Library attention in float64 (torch, CPU)."""
+    tq, tk, tv = (torch.from_numpy(np.ascontiguousarray(x)).double() for x in (q, k, v))
+    return torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal,
+                                                            scale=scale).numpy()
+
+
+def closed_form_recurrence(x, a, h0):
+    """h_t = sum_s (prod_{r=s+1..t} g_r)(1-g_s) x_s + (prod_{r=0..t} g_r) h0, by brute force."""
+    T = x.shape[0]
+    g = 1.0 / (1.0 + np.exp(-a))
+    y = np.zeros_like(x)
+    for t in range(T):
+        acc = np.prod(g[0:t + 1], axis=0) * h0
+        for s in range(t + 1):
+            acc = acc + np.prod(g[s + 1:t + 1], axis=0) * (1.0 - g[s]) * x[s]
+        y[t] = acc
+    return y
+
+
+# ----------------------------------------------------------------------------- recurrence
+# "RAT+ Deep Dive" section 2.1: forget-gate recurrence over the full sequence.
+
+def test_recurrence_matches_closed_form():
+    T, d = 37, 5
+    x = RNG.standard_normal((2, T, d))
+    a = RNG.standard_normal((2, T, d)) * 1.5 + 1.0
+    h0 = RNG.standard_normal((2, d))
+    y, hT = oracle.recurrence(x, a, h0)
+    for bh in range(2):
+        ref = closed_form_recurrence(x[bh], a[bh], h0[bh])
+        np.testing.assert_allclose(y[bh], ref, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(hT[bh], ref[-1], rtol=1e-12, atol=1e-12)
+
+
+def test_recurrence_zero_gate_is_identity():
+    # g = sigmoid(-1e4) = 0 exactly in float64, so h_t = x_t exactly.
+    x = RNG.standard_normal((3, 50, 8))
+    a = np.full_like(x, -1.0e4)
+    h0 = RNG.standard_normal((3, 8))
+    y, _ = oracle.recurrence(x, a, h0)
+    assert np.array_equal(y, x)
+
+
+def test_recurrence_unit_gate_holds_state():
+    # g = 1 exactly: the state never changes, h_t = h0.
+    x = RNG.standard_normal((2, 20, 4))
+    a = np.full_like(x, 1.0e4)
+    h0 = RNG.standard_normal((2, 4))
+    y, hT = oracle.recurrence(x, a, h0)
+    assert np.array_equal(y, np.broadcast_to(h0[:, None, :], y.shape))
+    assert np.array_equal(hT, h0)
+
+
+def test_recurrence_constant_gate_geometric():
+    # constant g = c, x = 1, h0 = 0:  h_t = 1 - c^(t+1).
+    c = 0.9
+    T = 200
+    a = np.full((1, T, 3), math.log(c / (1 - c)))
+    x = np.ones((1, T, 3))
+    y, _ = oracle.recurrence(x, a)
+    ref = 1.0 - c ** (np.arange(T) + 1.0)
+    np.testing.assert_allclose(y[0, :, 0], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_recurrence_associative_scan_any_bracketing():
+    # Prefill by associative scan ("RAT+ Deep Dive" 2.1, 7.3): composing the affine maps
+    # h -> A h + B with a tree of any shape gives the sequential result.
+    T, d = 64, 6
+    x = RNG.standard_normal((T, d))
+    a = RNG.standard_normal((T, d)) + 2.0
+    g = 1.0 / (1.0 + np.exp(-a))
+    A, Bv = g.copy(), (1.0 - g) * x
+    step = 1
+    while step < T:           # Hillis-Steele inclusive scan of (A, B) pairs
+        A2, B2 = A.copy(), Bv.copy()
+        A2[step:] = A[step:] * A[:-step]
+        B2[step:] = A[step:] * Bv[:-step] + Bv[step:]
+        A, Bv = A2, B2
+        step *= 2
+    y, _ = oracle.recurrence(x[None], a[None])
+    np.testing.assert_allclose(y[0], Bv, rtol=1e-12, atol=1e-12)
+
+
+def test_recurrence_chunked_equals_whole():
+    # Chunked prefill: carrying hT of a first part as h0 of the second gives the whole run.
+    x = RNG.standard_normal((2, 90, 7))
+    a = RNG.standard_normal((2, 90, 7)) + 2.0
+    y, hT = oracle.recurrence(x, a)
+    y1, h1 = oracle.recurrence(x[:, :33], a[:, :33])
+    y2, h2 = oracle.recurrence(x[:, 33:], a[:, 33:], h1)
+    np.testing.assert_allclose(np.concatenate([y1, y2], axis=1), y, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(h2, hT, rtol=1e-13, atol=1e-14)
+
+
+# ----------------------------------------------------------------------------- RoPE
+
+def test_rope_matches_complex_rotation():
+    d, T, pos0, base = 16, 9, 1000, 10000.0
+    x = RNG.standard_normal((1, T, d))
+    y = oracle.rope(x, pos0, base)
+    half = d // 2
+    z = x[0, :, :half] + 1j * x[0, :, half:]
+    theta = base ** (-np.arange(half) * 2.0 / d)
+    zr = z * np.exp(1j * (pos0 + np.arange(T))[:, None] * theta[None, :])
+    np.testing.assert_allclose(y[0, :, :half], zr.real, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(y[0, :, half:], zr.imag, rtol=1e-12, atol=1e-12)
+
+
+def test_rope_relative_position_and_identity():
+    d = 32
+    q = RNG.standard_normal((1, 1, d))
+    k = RNG.standard_normal((1, 1, d))
+    assert np.array_equal(oracle.rope(q, 0), q)
+    dots = []
+    for shift in (0, 7, 5000):
+        dots.append(float(np.dot(oracle.rope(q, 40 + shift)[0, 0], oracle.rope(k, 13 + shift)[0, 0])))
+    np.testing.assert_allclose(dots, dots[0], rtol=1e-9)
+
+
+# ----------------------------------------------------------------------------- key set
+# RAT+ abstract and "RAT+ Deep Dive" 3.1: dilation keeps every D-th key.
+
+def closed_form_count(t, D, W):
+    We = max(W, 1)
+    return min(We, t + 1) + max(0, (t - We + 1) // D)
+
+
+@pytest.mark.parametrize("D,W", [(1, 0), (4, 0), (16, 0), (64, 128), (64, 64), (3, 5), (7, 1), (300, 0)])
+def test_key_count_closed_form(D, W):
+    for t in list(range(0, 140)) + [511, 1000, 4095]:
+        assert oracle.key_count(t, D, W) == closed_form_count(t, D, W)
+
+
+def test_key_set_total_tiny_workload():
+    # B1 H2 T256 D4 W0: each head attends to sum_t (1 + floor(t/4)) = 8320 keys; 16640 in all.
+    total = sum(oracle.key_count(t, 4, 0) for t in range(256)) * 2
+    assert total == 16640
+
+
+def test_flops_table_golden():
+    with open(os.path.join(GOLDEN, "flops_table.json")) as f:
+        g = json.load(f)
+    T = g["T"]
+    for row in g["rows"]:
+        assert oracle.key_count(T - 1, row["D"], 0) == row["keys"] == T // row["D"]
+    cap = oracle.cache_capacity(T, [64])
+    assert T // int(cap[0]) == g["kv_reduction_at_D64"]
+
+
+# ----------------------------------------------------------------------------- attention
+
+def rand_qkv(B, H, T, d):
+    return (RNG.standard_normal((B, H, T, d)), RNG.standard_normal((B, H, T, d)),
+            RNG.standard_normal((B, H, T, d)))
+
+
+def test_dense_when_D_is_1():
+    q, k, v = rand_qkv(1, 2, 70, 16)
+    for W in (0, 1, 9, 200):
+        o = oracle.dilated_attention(q, k, v, D=1, W=W)
+        np.testing.assert_allclose(o, sdpa(q, k, v, causal=True), rtol=1e-11, atol=1e-12)
+
+
+def test_dense_when_window_covers_sequence():
+    q, k, v = rand_qkv(2, 1, 50, 8)
+    o = oracle.dilated_attention(q, k, v, D=16, W=50)
+    np.testing.assert_allclose(o, sdpa(q, k, v, causal=True), rtol=1e-11, atol=1e-12)
+
+
+def test_self_only_when_D_exceeds_T():
+    q, k, v = rand_qkv(1, 2, 40, 8)
+    o = oracle.dilated_attention(q, k, v, D=41, W=0)
+    assert np.array_equal(o, v)
+
+
+def test_chunk_end_queries_equal_causal_attention_on_subsampled_sequence():
+    # With W = 0 a query at a chunk end t = mD + D - 1 sees exactly the chunk ends 0..m:
+    # dense causal attention over the stride-D subsequence starting at D - 1.
+    D, T = 8, 96
+    q, k, v = rand_qkv(1, 2, T, 16)
+    rows = np.arange(D - 1, T, D)
+    o = oracle.dilated_attention(q, k, v, D=D, W=0, rows=rows)
+    ref = sdpa(q[:, :, D - 1::D], k[:, :, D - 1::D], v[:, :, D - 1::D], causal=True)
+    np.testing.assert_allclose(o, ref, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("D,W,T", [(4, 0, 64), (8, 5, 77), (16, 16, 130), (3, 1, 40), (64, 10, 200)])
+def test_general_key_set_by_slicing(D, W, T):
+    # Reference built by slicing: chunk ends k[D-1 :: D] older than the window, then the window.
+    d = 8
+    q, k, v = rand_qkv(1, 1, T, d)
+    o = oracle.dilated_attention(q, k, v, D=D, W=W)
+    We = max(W, 1)
+    for t in range(T):
+        lo = max(0, t - We + 1)     # first window position; chunk ends stop before it
+        kk = np.concatenate([k[0, 0, D - 1:lo:D], k[0, 0, lo:t + 1]])
+        vv = np.concatenate([v[0, 0, D - 1:lo:D], v[0, 0, lo:t + 1]])
+        ref = sdpa(q[0, 0, t:t + 1][None], kk[None], vv[None])[0, 0]
+        np.testing.assert_allclose(o[0, 0, t], ref, rtol=1e-11, atol=1e-12)
+
+
+def test_head_hybrid_equals_uniform_runs():
+    # "RAT+ Deep Dive" 6, head-wise hybrid: each head behaves as a uniform-D run of that head.
+    q, k, v = rand_qkv(2, 4, 60, 8)
+    Dh = [1, 1, 4, 16]
+    o = oracle.dilated_attention(q, k, v, W=3, D_per_head=Dh)
+    for h, D in enumerate(Dh):
+        oh = oracle.dilated_attention(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], D=D, W=3)
+        np.testing.assert_array_equal(o[:, h:h + 1], oh)
+
+
+def test_row_subset_equals_full():
+    q, k, v = rand_qkv(1, 2, 90, 8)
+    full = oracle.dilated_attention(q, k, v, D=4, W=6)
+    rows = [0, 5, 44, 89]
+    np.testing.assert_array_equal(oracle.dilated_attention(q, k, v, D=4, W=6, rows=rows),
+                                  full[:, :, rows])
+
+
+# ----------------------------------------------------------------------------- cache build
+
+def tagged(B, H, T, d, dtype=np.float32):
+    x = np.zeros((B, H, T, d), dtype=dtype)
+    x[..., 0] = np.arange(T)[None, None, :]
+    x[..., 1] = (np.arange(B)[:, None] * H + np.arange(H)[None, :])[:, :, None]
+    x[..., 2:] = np.arange(2, d)
+    return x
+
+
+def test_kv_compress_index_layout():
+    B, H, T, d, W = 2, 3, 100, 8, 6
+    Dh = [1, 4, 7]
+    Tcap = 120
+    x = tagged(B, H, T, d)
+    dil, ring = oracle.kv_compress(x, Dh, W, Tcap)
+    caps = [Tcap // D for D in Dh]
+    off = np.concatenate([[0], np.cumsum(caps)])
+    for h, D in enumerate(Dh):
+        n = T // D          # entries present after T positions: floor(T / D)
+        np.testing.assert_array_equal(dil[:, off[h]:off[h] + n], x[:, h, D - 1::D][:, :n])
+        assert np.all(dil[:, off[h] + n:off[h + 1]] == 0)
+        # ring slots read from slot T % W onwards give the last W positions in order
+        order = [(T - W + i) % W for i in range(W)]
+        np.testing.assert_array_equal(ring[:, h, order], x[:, h, T - W:])
+
+
+def test_kv_compress_chunked_equals_whole():
+    B, H, T, d, W, Tcap = 1, 2, 64, 4, 5, 64
+    Dh = [2, 8]
+    x = tagged(B, H, T, d)
+    dil, ring = oracle.kv_compress(x, Dh, W, Tcap)
+    d1, r1 = oracle.kv_compress(x[:, :, :27], Dh, W, Tcap, pos0=0)
+    d2, r2 = oracle.kv_compress(x[:, :, 27:], Dh, W, Tcap, pos0=27, dil=d1, ring=r1)
+    np.testing.assert_array_equal(d2, dil)
+    np.testing.assert_array_equal(r2, ring)
+
+
+# ----------------------------------------------------------------------------- decode
+
+@pytest.mark.parametrize("rope_base", [0.0, 10000.0])
+def test_decode_equals_prefill_rows(rope_base):
+    B, H, T0, steps, d, W = 1, 3, 40, 12, 8, 4
+    Dh = [1, 4, 16]
+    T = T0 + steps
+    q, k, v = rand_qkv(B, H, T, d)
+    a = RNG.standard_normal((B, H, T, d)) + 2.0
+    ref = oracle.layer_prefill(q, k, v, a, D_per_head=Dh, W=W, rope_base=rope_base)
+    st = oracle.DecodeState(np.tile(Dh, B), d, W, Tcap=T, rope_base=rope_base)
+    st.prefill(k[:, :, :T0].reshape(B * H, T0, d), v[:, :, :T0].reshape(B * H, T0, d),
+               a[:, :, :T0].reshape(B * H, T0, d))
+    for s in range(steps):
+        t = T0 + s
+        o = st.step(q[:, :, t].reshape(B * H, d), k[:, :, t].reshape(B * H, d),
+                    v[:, :, t].reshape(B * H, d), a[:, :, t].reshape(B * H, d))
+        np.testing.assert_allclose(o.reshape(B, H, d), ref["o"][:, :, t], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(st.hk.reshape(B, H, d), ref["hT_k"], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(st.hv.reshape(B, H, d), ref["hT_v"], rtol=1e-12, atol=1e-13)
