@@ -1,0 +1,216 @@
+/*
+ * rat.h -- C ABI of the RAT+ dilated-inference hot path on NVIDIA B200 (sm_100a).
+ *
+ * The method ("RAT+: Train Dense, Infer Sparse -- Recurrence Augmented Attention for Dilated
+ * Inference", abstract; "RAT+ Deep Dive" sections 2.1, 3.1 and 6) augments attention with a
+ * full-sequence forget-gate recurrence over keys and values, so that at inference the
+ * attention can be made dilated (every D-th key), optionally with a local window, and mixed
+ * per head.  This library computes, on one GPU:
+ *
+ *   rat_recur_prefill        h_t = g_t h_{t-1} + (1-g_t) x_t,  g = sigmoid(gate logit), per
+ *                            channel, for x = k and x = v with the same gate, over the whole
+ *                            sequence (chunked associative scan); optional RoPE on k~.
+ *   rat_dilated_attn_prefill causal attention of each query t over
+ *                              S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D = D-1 },
+ *                            We = max(W, 1), D per head; optional RoPE on q.
+ *   rat_kv_compress          the D-fold compressed cache: the chunk-end keys/values, the
+ *                            ring of the W most recent ones and the recurrence state.
+ *   rat_dilated_decode       one new token per sequence against that cache.
+ *
+ * Conventions shared by every call
+ *   - Tensors are contiguous, row-major (B, H, T, d) with d innermost, all of one dtype
+ *     (rat_dtype); every pointer must be 16-byte aligned.  d (d_head) is 64 or 128.
+ *   - Device pointers are caller-owned device memory; host pointers are named "host".
+ *     The library allocates no device memory: scratch lives in caller-provided workspaces.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     Its return value reports host-side validation and launch errors only.  Errors found
+ *     on the device (a bounded wait that ran out) are recorded in the workspace and
+ *     returned by rat_sync_status().
+ *   - Recurrence state and all accumulation are float32; bf16 tensors are rounded to
+ *     nearest-even when written.
+ *   - Readings of points the pages leave open: one gate tensor shared by K and V; h_{-1} = 0
+ *     unless h0 is given; the query always sees its own position (We = max(W,1)); dilated keys
+ *     are the chunk ends j = D-1, 2D-1, ...; RoPE (rotate-half pairing (c, c+d/2),
+ *     theta_c = base^(-2c/d)) is applied to k~ after the recurrence, at absolute position
+ *     pos0 + t; softmax scale 1/sqrt(d) unless given.
+ */
+#ifndef RAT_H_
+#define RAT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RAT_API __attribute__((visibility("default")))
+#else
+#define RAT_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes (returned by every entry point, and by rat_sync_status for device errors). */
+typedef enum {
+    RAT_OK = 0,
+    RAT_ERR_INVALID = -1,      /* bad argument: NULL pointer, bad size, misaligned pointer   */
+    RAT_ERR_UNSUPPORTED = -2,  /* valid but not implemented (e.g. d not in {64, 128})       */
+    RAT_ERR_CUDA = -3,         /* a CUDA runtime call or kernel launch failed               */
+    RAT_ERR_TIMEOUT = -4,      /* a bounded device-side wait ran out (workspace not zeroed?) */
+    RAT_ERR_WORKSPACE = -5     /* workspace missing or smaller than the *_workspace_bytes() */
+} rat_status;
+
+/* Element types. */
+typedef enum { RAT_F32 = 0, RAT_BF16 = 1 } rat_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+RAT_API const char *rat_status_string(int status);
+
+/* Library version string, e.g. "rat-b200 0.1 sm_100a". */
+RAT_API const char *rat_version(void);
+
+/* ------------------------------------------------------------------------------------------
+ * Workspaces.
+ * A workspace is caller-owned device memory that holds a 256-byte header (device error word,
+ * launch epoch and CTA tickets) followed by per-call scratch.  Zero it once with
+ * rat_workspace_init() before its first use; afterwards every call leaves it consistent.
+ * Use one workspace per stream and per call kind (prefill recurrence or decode): calls that
+ * share a workspace must not overlap on the GPU.
+ * ---------------------------------------------------------------------------------------- */
+
+/* Zero `ws_bytes` bytes of `ws` on `stream` (cudaMemsetAsync). */
+RAT_API int rat_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/* Synchronise `stream`, then return the first device-side error recorded in workspace `ws`
+ * since the last rat_sync_status() on it (RAT_OK if none) and clear it. */
+RAT_API int rat_sync_status(void *ws, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * rat_recur_prefill -- full-sequence forget-gate recurrence over keys and values.
+ *   "RAT+ Deep Dive" section 2.1 (full-sequence recurrence, L = T, computed in prefill by an
+ *   associative scan; forget gate g input-dependent) and section 7.3 ("parallel prefill by
+ *   associative scan").
+ *
+ *   k, v, gate_logit : device, (B, H, T, d) of dtype          inputs x = k, x = v and a
+ *   h0_k, h0_v       : device, (B, H, d) float32, or NULL     initial state (NULL = zeros)
+ *   k_rec, v_rec     : device, (B, H, T, d) of dtype          outputs k~ (after RoPE, if
+ *                                                            rope_base > 0) and v~
+ *   hT_k, hT_v       : device, (B, H, d) float32, or NULL     final state h_{T-1} (before RoPE)
+ *   pos0             : absolute position of row t = 0 (RoPE angle (pos0 + t) * theta_c)
+ *   rope_base        : > 0 applies RoPE to k~ with this base; <= 0 disables it
+ *   ws, ws_bytes     : workspace of at least rat_recur_workspace_bytes(B, H, T, d, dtype)
+ * Computes g = 1/(1+exp(-a)), 1-g, and h_t = g h_{t-1} + (1-g) x_t in float32 for every
+ * channel.  Outputs may not alias inputs.  T = 0 is a no-op.  The scan carries state between
+ * chunks of the sequence with a bounded-wait decoupled look-back; if that wait runs out the
+ * device error word becomes RAT_ERR_TIMEOUT (see rat_sync_status).
+ * ---------------------------------------------------------------------------------------- */
+RAT_API size_t rat_recur_workspace_bytes(int B, int H, int T, int d, int dtype);
+
+RAT_API int rat_recur_prefill(const void *k, const void *v, const void *gate_logit,
+                      const float *h0_k, const float *h0_v,
+                      void *k_rec, void *v_rec, float *hT_k, float *hT_v,
+                      int B, int H, int T, int d, int dtype,
+                      int64_t pos0, float rope_base,
+                      void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * rat_dilated_attn_prefill -- causal dilated attention with an optional local window and a
+ * per-head dilation, over the recurrence outputs.
+ *   RAT+ abstract (dilation D cuts attention FLOPs and KV cache D-fold; optional local
+ *   windows; hybrid head compositions); "RAT+ Deep Dive" section 3.1 table (FLOPs T/D) and
+ *   section 6 "Head-Wise Hybrid" (different D per head).
+ *
+ *   q             : device, (B, H, T, d) of dtype   queries (RoPE applied inside if rope_base > 0)
+ *   k_rec, v_rec  : device, (B, H, T, d) of dtype   recurrence outputs from rat_recur_prefill
+ *   o             : device, (B, H, T, d) of dtype   output
+ *   D             : dilation of every head (>= 1), used when D_per_head is NULL
+ *   W             : local window (>= 0); the window is the W most recent positions, self
+ *                   included; W = 0 means self only
+ *   D_per_head    : host, int32[H] or NULL          per-head dilation (each >= 1)
+ *   pos0          : absolute position of row 0 (RoPE only)
+ *   rope_base     : > 0 rotates q with this base (k_rec is expected already rotated)
+ *   scale         : softmax scale; <= 0 selects 1/sqrt(d)
+ * For query t of head h:  o_t = sum_{j in S(t)} softmax_j(scale * q^_t . k~_j) v~_j with
+ * S(t) = { t-We < j <= t } U { j <= t-We : j mod D_h = D_h - 1 }, We = max(W, 1).
+ * bf16: QK^T and PV on tcgen05 tensor cores (bf16 operands, float32 accumulation; the
+ * softmax probabilities are rounded to bf16 for PV); float32: CUDA-core FMA throughout.
+ * Needs no workspace; never waits on other CTAs.
+ * ---------------------------------------------------------------------------------------- */
+RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o,
+                             int B, int H, int T, int d, int dtype, int D, int W,
+                             const int32_t *D_per_head, int64_t pos0, float rope_base,
+                             float scale, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Compressed KV cache (RAT+ abstract: dilation reduces the KV cache D-fold; "RAT+ Deep Dive"
+ * section 3.1: "KV cache ... compressed 64x" at D = 64).
+ *
+ * Layout, with cap_h = floor(Tcap / D_h) and off_h = sum_{h' < h} cap_h':
+ *   k_dil, v_dil : device [B][sum_h cap_h][d] of dtype; entry i of head h (row
+ *                  b * sum_h cap_h + off_h + i) holds position i * D_h + D_h - 1
+ *   k_win, v_win : device [B][H][W][d] of dtype; position p is in slot p mod W (NULL if W = 0)
+ *   h_k, h_v     : device [B][H][d] float32 recurrence state after the last position
+ *                  (before RoPE)
+ *   pos          : number of positions consumed so far (the same for every sequence)
+ * The struct itself is host memory; the caller owns every buffer it points to.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct rat_kv_cache {
+    int32_t B, H, d, W;       /* batch, heads, head dim, local window (0 = none)           */
+    int32_t Tcap;             /* maximum number of positions the cache will ever hold      */
+    int32_t dtype;            /* rat_dtype of k_dil, v_dil, k_win, v_win                    */
+    const int32_t *D;         /* host int32[H]: dilation of each head (>= 1)               */
+    void *k_dil, *v_dil;      /* device, see layout above                                  */
+    void *k_win, *v_win;      /* device ring, or NULL when W == 0                          */
+    float *h_k, *h_v;         /* device float32 state                                      */
+    int64_t pos;              /* positions consumed so far                                 */
+} rat_kv_cache;
+
+/* Byte sizes of the buffers a cache with these fields needs (any output may be NULL). */
+RAT_API int rat_kv_cache_bytes(const rat_kv_cache *cache, size_t *dil_bytes, size_t *win_bytes,
+                       size_t *state_bytes);
+
+/* rat_kv_compress -- append T positions of recurrence output to the cache.
+ *   k_rec, v_rec : device (B, H, T, d) of cache->dtype: positions cache->pos .. cache->pos+T-1
+ *   hT_k, hT_v   : device (B, H, d) float32 state after those positions (copied into h_k, h_v)
+ * Writes every position p with p mod D_h = D_h - 1 (and p / D_h < cap_h) to its dil entry, and
+ * the last min(W, T) positions to their ring slots; copies the state; then advances
+ * cache->pos by T on the host.  Bit-exact copies.  Requires cache->pos + T <= Tcap. */
+RAT_API int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, const float *hT_v,
+                    int T, rat_kv_cache *cache, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * rat_dilated_decode -- one new token per sequence against the compressed cache.
+ *   q, k, v, gate_logit : device (B, H, 1, d) of cache->dtype, the token at position t = pos
+ *   o                   : device (B, H, 1, d) of cache->dtype
+ *   rope_base, scale    : as in prefill (rope_base must match the one used for the cache)
+ *   ws, ws_bytes        : workspace of at least rat_decode_workspace_bytes(cache)
+ * Per (b, h): state update h = g h + (1-g) x for k and v; k~_t = RoPE(h_k, t); append k~_t, v~_t
+ * to the dil cache if t mod D_h = D_h - 1 and to ring slot t mod W; then attention of
+ * RoPE(q, t) over the dil entries with position <= t - We, the ring positions
+ * t-We < j < t and the token itself -- the same key set S(t) as in prefill.  Split over the
+ * keys across CTAs, combined by log-sum-exp.  Advances cache->pos by 1 on the host.
+ * Requires pos < Tcap.
+ * ---------------------------------------------------------------------------------------- */
+RAT_API size_t rat_decode_workspace_bytes(const rat_kv_cache *cache);
+
+RAT_API int rat_dilated_decode(const void *q, const void *k, const void *v, const void *gate_logit,
+                       rat_kv_cache *cache, void *o, float rope_base, float scale,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/* Test hook for failure detection (no counterpart in the method): the next rat_recur_prefill
+ * issued from the calling host thread withholds the look-back publication of chunk `chunk`
+ * (chunk index >= 1 along the sequence, in every (b, h)) and bounds each look-back wait by
+ * wait_limit_ns (1 ms .. 2 s).  Its successors' waits run out, the call's results are wrong,
+ * and rat_sync_status() reports RAT_ERR_TIMEOUT; nothing hangs and the context stays usable.
+ * Returns RAT_ERR_INVALID for out-of-range arguments. */
+RAT_API int rat_debug_inject_lookback_fault(int64_t chunk, int64_t wait_limit_ns);
+
+/* Number of keys query t attends to: min(We, t+1) + max(0, floor((t - We + 1) / D)).
+ * Host-only helper used for FLOP and byte accounting. */
+RAT_API int64_t rat_attended_keys(int64_t t, int D, int W);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RAT_H_ */

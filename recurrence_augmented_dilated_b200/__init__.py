@@ -1,0 +1,226 @@
+"""Thin Python binding of librat.so, the C ABI of the RAT+ dilated-inference hot path.
+
+Every function here only marshals arguments (torch tensors -> device pointers, the current
+CUDA stream) and calls the C entry point of the same name; all computation runs in the CUDA
+kernels of librat.so.  There is no fallback: if the library is missing or a call fails, a
+RatError is raised.
+
+Entry points (see include/rat.h for layouts and error behaviour):
+  rat_recur_prefill         forget-gate recurrence over k and v (chunked associative scan)
+  rat_dilated_attn_prefill  causal dilated attention + local window + per-head D
+  rat_kv_compress           build / extend the D-fold compressed KV cache
+  rat_dilated_decode        one token per sequence against that cache
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+import torch
+
+__all__ = [
+    "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
+    "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_dilated_attn_prefill",
+    "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
+    "rat_workspace_init", "rat_sync_status", "rat_attended_keys", "rat_status_string",
+    "Workspace",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "librat.so")
+
+F32, BF16 = 0, 1
+_STATUS = {0: "RAT_OK", -1: "RAT_ERR_INVALID", -2: "RAT_ERR_UNSUPPORTED", -3: "RAT_ERR_CUDA",
+           -4: "RAT_ERR_TIMEOUT", -5: "RAT_ERR_WORKSPACE"}
+
+
+class RatError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (fn, _STATUS.get(status, "?"), status))
+
+
+class KVCache(ctypes.Structure):
+    """Mirror of struct rat_kv_cache (host struct of device pointers)."""
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d", ctypes.c_int32), ("W", ctypes.c_int32),
+        ("Tcap", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("D", ctypes.POINTER(ctypes.c_int32)),
+        ("k_dil", ctypes.c_void_p), ("v_dil", ctypes.c_void_p),
+        ("k_win", ctypes.c_void_p), ("v_win", ctypes.c_void_p),
+        ("h_k", ctypes.c_void_p), ("h_v", ctypes.c_void_p),
+        ("pos", ctypes.c_int64),
+    ]
+
+
+_lib = None
+_vp, _sz, _i, _i64, _f = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_int64, ctypes.c_float
+
+
+def lib():
+    """Load librat.so (raises if it has not been built: there is no other implementation)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise RatError("load librat.so (run recurrence_augmented_dilated_b200.build)", -3)
+        L = ctypes.CDLL(library_path)
+        L.rat_status_string.restype = ctypes.c_char_p
+        L.rat_status_string.argtypes = [_i]
+        L.rat_version.restype = ctypes.c_char_p
+        L.rat_workspace_init.argtypes = [_vp, _sz, _vp]
+        L.rat_sync_status.argtypes = [_vp, _vp]
+        L.rat_recur_workspace_bytes.restype = _sz
+        L.rat_recur_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+        L.rat_recur_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                        _i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
+        L.rat_dilated_attn_prefill.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                               ctypes.POINTER(ctypes.c_int32), _i64, _f, _f, _vp]
+        L.rat_kv_cache_bytes.argtypes = [ctypes.POINTER(KVCache), ctypes.POINTER(_sz),
+                                         ctypes.POINTER(_sz), ctypes.POINTER(_sz)]
+        L.rat_kv_compress.argtypes = [_vp, _vp, _vp, _vp, _i, ctypes.POINTER(KVCache), _vp]
+        L.rat_decode_workspace_bytes.restype = _sz
+        L.rat_decode_workspace_bytes.argtypes = [ctypes.POINTER(KVCache)]
+        L.rat_dilated_decode.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(KVCache), _vp, _f, _f,
+                                         _vp, _sz, _vp]
+        L.rat_debug_inject_lookback_fault.argtypes = [_i64, _i64]
+        L.rat_attended_keys.restype = _i64
+        L.rat_attended_keys.argtypes = [_i64, _i, _i]
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, st: int):
+    if st != 0:
+        raise RatError(fn, st)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise RatError("dtype %s" % t.dtype, -2)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def rat_status_string(status: int) -> str:
+    return lib().rat_status_string(int(status)).decode()
+
+
+def rat_attended_keys(t: int, D: int, W: int) -> int:
+    return int(lib().rat_attended_keys(int(t), int(D), int(W)))
+
+
+class Workspace:
+    """Caller-owned device scratch (a torch uint8 buffer), zeroed once by rat_workspace_init."""
+
+    def __init__(self, nbytes: int, device=None, stream=None):
+        self.nbytes = max(int(nbytes), 256)
+        self.buf = torch.empty(self.nbytes + 256, dtype=torch.uint8, device=device or "cuda")
+        off = (-self.buf.data_ptr()) % 256          # 256-byte aligned view
+        self.view = self.buf[off:off + self.nbytes]
+        rat_workspace_init(self, stream)
+
+    @property
+    def ptr(self):
+        return ctypes.c_void_p(self.view.data_ptr())
+
+
+def rat_workspace_init(ws: Workspace, stream=None):
+    _check("rat_workspace_init", lib().rat_workspace_init(ws.ptr, ws.nbytes, _stream(stream)))
+
+
+def rat_sync_status(ws: Workspace, stream=None) -> int:
+    return int(lib().rat_sync_status(ws.ptr, _stream(stream)))
+
+
+def rat_recur_workspace_bytes(B, H, T, d, dtype) -> int:
+    return int(lib().rat_recur_workspace_bytes(B, H, T, d, dtype))
+
+
+def rat_recur_prefill(k, v, gate_logit, k_rec, v_rec, ws: Workspace, h0_k=None, h0_v=None,
+                      hT_k=None, hT_v=None, pos0: int = 0, rope_base: float = 0.0, stream=None):
+    """k, v, gate_logit -> k_rec, v_rec (all (B, H, T, d)); optional float32 (B, H, d) states."""
+    B, H, T, d = k.shape
+    st = lib().rat_recur_prefill(_ptr(k), _ptr(v), _ptr(gate_logit), _ptr(h0_k), _ptr(h0_v),
+                                 _ptr(k_rec), _ptr(v_rec), _ptr(hT_k), _ptr(hT_v), B, H, T, d,
+                                 _dtype_code(k), int(pos0), float(rope_base), ws.ptr, ws.nbytes,
+                                 _stream(stream))
+    _check("rat_recur_prefill", st)
+
+
+def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,
+                             D_per_head: Optional[Sequence[int]] = None, pos0: int = 0,
+                             rope_base: float = 0.0, scale: float = 0.0, stream=None):
+    """o = dilated attention of q over (k_rec, v_rec); all (B, H, T, d)."""
+    B, H, T, d = q.shape
+    dph = None
+    if D_per_head is not None:
+        dph = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
+    st = lib().rat_dilated_attn_prefill(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), B, H, T, d,
+                                        _dtype_code(q), int(D), int(W), dph, int(pos0),
+                                        float(rope_base), float(scale), _stream(stream))
+    _check("rat_dilated_attn_prefill", st)
+
+
+def make_cache(B, H, d, W, Tcap, dtype: int, D_per_head: Sequence[int], device="cuda"):
+    """Allocate (with torch) the buffers of a compressed cache and return (KVCache, buffers)."""
+    Dh = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
+    c = KVCache(B=B, H=H, d=d, W=W, Tcap=Tcap, dtype=dtype, D=Dh)
+    dil, win, state = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check("rat_kv_cache_bytes", lib().rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(dil),
+                                                          ctypes.byref(win), ctypes.byref(state)))
+    tdt = torch.float32 if dtype == F32 else torch.bfloat16
+    es = 4 if dtype == F32 else 2
+    total = dil.value // (B * d * es)
+    bufs = {
+        "k_dil": torch.zeros((B, total, d), dtype=tdt, device=device),
+        "v_dil": torch.zeros((B, total, d), dtype=tdt, device=device),
+        "k_win": torch.zeros((B, H, max(W, 1), d), dtype=tdt, device=device),
+        "v_win": torch.zeros((B, H, max(W, 1), d), dtype=tdt, device=device),
+        "h_k": torch.zeros((B, H, d), dtype=torch.float32, device=device),
+        "h_v": torch.zeros((B, H, d), dtype=torch.float32, device=device),
+        "D": Dh,
+    }
+    c.k_dil, c.v_dil = bufs["k_dil"].data_ptr(), bufs["v_dil"].data_ptr()
+    c.k_win = bufs["k_win"].data_ptr() if W > 0 else None
+    c.v_win = bufs["v_win"].data_ptr() if W > 0 else None
+    c.h_k, c.h_v = bufs["h_k"].data_ptr(), bufs["h_v"].data_ptr()
+    c.pos = 0
+    return c, bufs
+
+
+def rat_kv_cache_bytes(cache: KVCache):
+    dil, win, state = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check("rat_kv_cache_bytes", lib().rat_kv_cache_bytes(ctypes.byref(cache), ctypes.byref(dil),
+                                                          ctypes.byref(win), ctypes.byref(state)))
+    return dil.value, win.value, state.value
+
+
+def rat_kv_compress(k_rec, v_rec, hT_k, hT_v, cache: KVCache, stream=None):
+    T = k_rec.shape[2]
+    st = lib().rat_kv_compress(_ptr(k_rec), _ptr(v_rec), _ptr(hT_k), _ptr(hT_v), T,
+                               ctypes.byref(cache), _stream(stream))
+    _check("rat_kv_compress", st)
+
+
+def rat_decode_workspace_bytes(cache: KVCache) -> int:
+    return int(lib().rat_decode_workspace_bytes(ctypes.byref(cache)))
+
+
+def rat_dilated_decode(q, k, v, gate_logit, cache: KVCache, o, ws: Workspace,
+                       rope_base: float = 0.0, scale: float = 0.0, stream=None):
+    st = lib().rat_dilated_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit), ctypes.byref(cache),
+                                  _ptr(o), float(rope_base), float(scale), ws.ptr, ws.nbytes,
+                                  _stream(stream))
+    _check("rat_dilated_decode", st)

@@ -1,0 +1,142 @@
+// attn_simt.cu -- causal dilated attention on CUDA cores (float32 path; any d in {64, 128}).
+//
+// RAT+ abstract and "RAT+ Deep Dive" sections 3.1 and 6: query t of head h attends to
+//   S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D_h = D_h - 1 },   We = max(W, 1),
+// the local window (self included) and the chunk ends older than it.  One warp per query:
+// each lane holds d/32 channels of the query and of the running output; for every key of
+// S(t) the warp reduces the dot product with shuffles and applies an online softmax in
+// float32 (exp2 with the scale folded in).  Keys are visited in groups of four so four row
+// loads are in flight at once.  This is the float32 production path (a tensor-core bf16 or
+// tf32 product would not meet float32 accuracy) and a readable GPU statement of the mask.
+#include "common.cuh"
+
+namespace rat {
+
+template <typename E, int CPL> struct RowIO;
+template <> struct RowIO<float, 2> {
+    static RAT_DEVICE void load(const void *p, float *x) {
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(p));
+        x[0] = v.x; x[1] = v.y;
+    }
+    static RAT_DEVICE void store(void *p, const float *x) {
+        *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+    }
+};
+template <> struct RowIO<float, 4> {
+    static RAT_DEVICE void load(const void *p, float *x) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    }
+    static RAT_DEVICE void store(void *p, const float *x) {
+        *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+};
+template <> struct RowIO<__nv_bfloat16, 2> {
+    static RAT_DEVICE void load(const void *p, float *x) {
+        const uint32_t u = __ldg(reinterpret_cast<const unsigned int *>(p));
+        x[0] = bf16_lo(u); x[1] = bf16_hi(u);
+    }
+    static RAT_DEVICE void store(void *p, const float *x) {
+        *reinterpret_cast<uint32_t *>(p) = pack_bf16(x[0], x[1]);
+    }
+};
+template <> struct RowIO<__nv_bfloat16, 4> {
+    static RAT_DEVICE void load(const void *p, float *x) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+        x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+    }
+    static RAT_DEVICE void store(void *p, const float *x) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+    }
+};
+
+RAT_DEVICE float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+template <typename E, int DH>
+__global__ void __launch_bounds__(256) attn_simt_kernel(const __grid_constant__ AttnSimtParams p) {
+    constexpr int CPL = DH / 32;
+    constexpr int EB = sizeof(E);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, h = bh % p.H;
+    const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+    if (t >= p.T) return;
+    const int D = p.Dh[h];
+    const int We = p.W > 1 ? p.W : 1;
+    const uint8_t *kb = static_cast<const uint8_t *>(p.k) + (size_t)bh * p.T * DH * EB + lane * CPL * EB;
+    const uint8_t *vb = static_cast<const uint8_t *>(p.v) + (size_t)bh * p.T * DH * EB + lane * CPL * EB;
+    const size_t qoff = ((size_t)bh * p.T + t) * DH * EB + lane * CPL * EB;
+
+    float q[CPL];
+    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.q) + qoff, q);
+    if (p.rope) {
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) {
+            const int c = lane * CPL + j;
+            float cs, sn;
+            rope_cs(p.pos0 + t, p.theta[c % (DH / 2)], cs, sn);
+            const float partner = __shfl_xor_sync(0xffffffffu, q[j], 16);
+            q[j] = c < DH / 2 ? q[j] * cs - partner * sn : q[j] * cs + partner * sn;
+        }
+    }
+    float m = -INFINITY, l = 0.f, o[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) o[j] = 0.f;
+
+    // the key list: window positions first, then the chunk ends older than the window
+    const int w_lo = max(0, t - We + 1);
+    const int n_win = t - w_lo + 1;
+    const int n_dil = t - We + 1 >= D ? (t - We + 1) / D : 0;   // j = D-1, .., n_dil*D - 1 <= t-We
+    const int n = n_win + n_dil;
+    for (int base = 0; base < n; base += 4) {
+        float kx[4][CPL], vx[4][CPL];
+        int cnt = min(4, n - base);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int idx = base + u;
+            if (u < cnt) {
+                const int j = idx < n_win ? w_lo + idx : (idx - n_win) * D + D - 1;
+                RowIO<E, CPL>::load(kb + (size_t)j * DH * EB, kx[u]);
+                RowIO<E, CPL>::load(vb + (size_t)j * DH * EB, vx[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (u < cnt) {
+                float dot = 0.f;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) dot = fmaf(q[j], kx[u][j], dot);
+                const float s = warp_sum(dot) * p.scale_log2;
+                const float mn = fmaxf(m, s);
+                const float corr = exp2f(m - mn);
+                const float pj = exp2f(s - mn);
+                l = fmaf(l, corr, pj);
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) o[j] = fmaf(o[j], corr, pj * vx[u][j]);
+                m = mn;
+            }
+        }
+    }
+    const float inv = 1.0f / l;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) o[j] *= inv;
+    RowIO<E, CPL>::store(static_cast<uint8_t *>(p.o) + qoff, o);
+}
+
+int launch_attn_simt(const AttnSimtParams &p, int dtype, void *stream) {
+    dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)(p.B * p.H));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == RAT_F32) {
+        if (p.d == 64) attn_simt_kernel<float, 64><<<grid, 256, 0, s>>>(p);
+        else attn_simt_kernel<float, 128><<<grid, 256, 0, s>>>(p);
+    } else {
+        if (p.d == 64) attn_simt_kernel<__nv_bfloat16, 64><<<grid, 256, 0, s>>>(p);
+        else attn_simt_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
+    }
+    return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
+}
+
+}  // namespace rat

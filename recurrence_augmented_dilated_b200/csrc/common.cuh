@@ -1,0 +1,146 @@
+// common.cuh -- small device helpers shared by the kernels of this library (sm_100a only).
+//
+// Hand-written inline PTX for: mbarriers, bulk (TMA) copies, acquire/release flags, the
+// global timer used to bound every wait, bf16 packing, and approximate ex2/rcp.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "internal.h"
+
+#define RAT_DEVICE __device__ __forceinline__
+
+namespace rat {
+
+// ------------------------------------------------------------------------------ elements
+struct f32x4 { float v[4]; };
+
+RAT_DEVICE float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+RAT_DEVICE float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// Round two floats to bf16 (nearest-even) and pack them, lo in bits 0..15.
+RAT_DEVICE uint32_t pack_bf16(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ------------------------------------------------------------------------------ math
+// 2^x and 1/x from the special-function unit (PTX ex2.approx / rcp.approx, flush-to-zero).
+RAT_DEVICE float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+RAT_DEVICE float rcp_approx(float x) {
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Forget gate from its logit: g = 1/(1+e^{-a}) and 1-g = e^{-a}/(1+e^{-a}).
+// For a -> -inf, e^{-a} = inf, g = 0 and the product inf*0 is NaN: fminf maps it to 1 exactly,
+// and also caps rounding of e*g slightly above 1.  For a -> +inf, e = 0, g = 1, 1-g = 0.
+RAT_DEVICE void forget_gate(float a, float &g, float &omg) {
+    const float kLog2e = 1.4426950408889634f;
+    float e = ex2_approx(-a * kLog2e);
+    g = rcp_approx(1.0f + e);
+    omg = fminf(e * g, 1.0f);
+}
+
+// cos/sin of pos * theta for RoPE.  The angle is formed in float64 and reduced by 2*pi with a
+// two-term (Cody-Waite) constant, so positions up to 2^31 keep full single-precision accuracy;
+// the reduced angle in [-pi, pi] goes to the single-precision sincosf.
+RAT_DEVICE void rope_cs(long long pos, double theta, float &c, float &s) {
+    const double kTwoPiHi = 6.283185307179586;          // nearest double to 2*pi
+    const double kTwoPiLo = 2.4492935982947064e-16;     // 2*pi - kTwoPiHi
+    const double kInvTwoPi = 0.15915494309189535;
+    const double ang = (double)pos * theta;
+    const double n = rint(ang * kInvTwoPi);
+    double r = fma(-n, kTwoPiHi, ang);
+    r = fma(-n, kTwoPiLo, r);
+    sincosf((float)r, &s, &c);
+}
+
+// ------------------------------------------------------------------------------ memory order
+RAT_DEVICE uint32_t ld_acquire_gpu(const uint32_t *p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+RAT_DEVICE void st_release_gpu(uint32_t *p, uint32_t v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+RAT_DEVICE uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Record the first device-side error of a launch in the workspace header.
+RAT_DEVICE void record_error(WsHeader *hdr, int code, uint32_t detail) {
+    if (atomicCAS(&hdr->error, 0, code) == 0) hdr->detail = detail;
+}
+
+// ------------------------------------------------------------------------------ smem / mbarrier
+RAT_DEVICE uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+RAT_DEVICE void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(smem_u32(bar)), "r"(count) : "memory");
+}
+RAT_DEVICE void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+RAT_DEVICE void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+                 :: "r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+RAT_DEVICE void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" :: "r"(smem_u32(bar)) : "memory");
+}
+RAT_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier, for at most kWaitLimitNs.  Returns false (and
+// records RAT_ERR_TIMEOUT when hdr is given) if the wait ran out.
+RAT_DEVICE bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, WsHeader *hdr, uint32_t where) {
+    if (mbar_try_wait(bar, parity)) return true;
+    uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (hdr) record_error(hdr, RAT_ERR_TIMEOUT, where);
+            return false;
+        }
+    }
+    return true;
+}
+
+// One-dimensional bulk copy global -> shared (the untiled TMA path), completing on `bar`.
+// Both addresses 16-byte aligned, bytes a multiple of 16.
+RAT_DEVICE void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :: "r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+RAT_DEVICE void ld_shared_v4(const void *p, uint32_t &a, uint32_t &b, uint32_t &c, uint32_t &d) {
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(smem_u32(p)));
+}
+RAT_DEVICE void st_global_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+}  // namespace rat

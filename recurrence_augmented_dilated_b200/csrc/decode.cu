@@ -1,0 +1,281 @@
+// decode.cu -- one new token per sequence against the D-fold compressed KV cache.
+//
+// RAT+ abstract (dilated attention with an optional local window; D-fold smaller KV cache) and
+// "RAT+ Deep Dive" section 2.1 (the recurrence state carries what dilation skips).  For the token
+// at position t of slice (b, h):
+//   1. state update  h_k = g h_k + (1-g) k,  h_v = g h_v + (1-g) v   (float32, g = sigmoid(a));
+//      k~_t = RoPE(h_k, t), v~_t = h_v, both rounded to the cache dtype;
+//   2. append k~_t, v~_t to dil entry (t - D + 1) / D if t mod D = D - 1, and to ring slot t mod W;
+//   3. attention of q^ = RoPE(q, t) over the prefill key set S(t): dil entries whose position
+//      i*D + D - 1 <= t - We, ring positions t - We < j < t, and the token itself.
+// Memory-bound: every key is one 16-byte load per lane for K and one for V.  The keys of a
+// slice are split over `splits` CTAs; each CTA keeps an online softmax per 16-lane group,
+// merges its groups and warps, and writes (max, sum, o) to the workspace; the last CTA of the
+// slice (atomic ticket, no waiting) merges the splits by log-sum-exp and resets the ticket.
+// Split 0 alone does steps 1-2 and adds the token itself to its softmax.
+// No CTA reads what another writes in the same launch: the new dil entry (position t) is never
+// older than the window, and the ring slot written held position t - W, outside the window.
+#include "common.cuh"
+
+namespace rat {
+
+namespace {
+constexpr int kThreads = 128;       // 4 warps; 16 lanes x 8 channels = one d=128 bf16 row
+constexpr int kWarps = kThreads / 32;
+
+RAT_DEVICE void load8(const void *p, float *x) {      // 8 bf16 -> float
+    const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+    x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+    x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
+}
+RAT_DEVICE void load8_cg(const void *p, float *x) {   // same, bypassing L1 (written this launch)
+    const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(p));
+    x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+    x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
+}
+RAT_DEVICE uint4 pack8(const float *x) {
+    return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
+                      pack_bf16(x[6], x[7]));
+}
+}  // namespace
+
+// Template on d: 16 lanes per row for d = 128 (8 bf16 each), 8 lanes for d = 64.
+template <int DH>
+__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int LPR = DH / 8;                 // lanes per key row
+    constexpr int GPW = 32 / LPR;               // key groups per warp
+    constexpr int RB = DH * 2;                  // row bytes (bf16)
+    const int split = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int grp = lane / LPR, cl = lane % LPR;   // key group inside the warp, lane inside row
+    const long long t = p.t;
+    const long long D = p.Dh[h];
+    const long long We = p.W > 1 ? p.W : 1;
+    const long long cap = p.Tcap / D;
+    const bool first_half = cl < LPR / 2;
+
+    // the new token's query, rotated; every lane group holds a copy of its 8 channels
+    float q[8];
+    load8(static_cast<const uint8_t *>(p.q) + (size_t)bh * RB + cl * 16, q);
+    if (p.rope) {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float cs, sn;
+            rope_cs(t, p.theta[(cl * 8 + j) % (DH / 2)], cs, sn);
+            const float partner = __shfl_xor_sync(0xffffffffu, q[j], LPR / 2);
+            q[j] = first_half ? q[j] * cs - partner * sn : q[j] * cs + partner * sn;
+        }
+    }
+
+    // key list of this slice: [0, n_dil) dil entries, then [n_dil, n_dil + n_ring) ring positions
+    long long n_dil = (t - We + 1) >= D ? (t - We + 1) / D : 0;
+    if (n_dil > cap) n_dil = cap;
+    const long long r_lo = max(0ll, t - We + 1);           // first ring position in the window
+    const long long n_ring = t - r_lo;                      // positions r_lo .. t-1
+    const long long n_keys = n_dil + n_ring;
+    const long long k_lo = n_keys * split / p.splits, k_hi = n_keys * (split + 1) / p.splits;
+
+    const uint8_t *kdil = static_cast<const uint8_t *>(p.kdil) + ((size_t)b * p.total_cap + p.off[h]) * RB;
+    const uint8_t *vdil = static_cast<const uint8_t *>(p.vdil) + ((size_t)b * p.total_cap + p.off[h]) * RB;
+    const uint8_t *kwin = p.kwin ? static_cast<const uint8_t *>(p.kwin) + (size_t)bh * p.W * RB : nullptr;
+    const uint8_t *vwin = p.vwin ? static_cast<const uint8_t *>(p.vwin) + (size_t)bh * p.W * RB : nullptr;
+
+    float m = -INFINITY, l = 0.f, o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) o[j] = 0.f;
+
+    // keys of this split: each (warp, group) takes every (kWarps*GPW)-th key, 2 at a time
+    constexpr int kLanesets = kWarps * GPW;
+    const int set = warp * GPW + grp;
+    for (long long base = k_lo + set; base < k_hi; base += 2 * kLanesets) {
+        float kx[2][8], vx[2][8];
+        bool have[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const long long idx = base + (long long)u * kLanesets;
+            have[u] = idx < k_hi;
+            // lanes of a warp may disagree on `have`; loads are predicated, shuffles are not
+            if (have[u]) {
+                const uint8_t *kp, *vp;
+                if (idx < n_dil) {
+                    kp = kdil + (size_t)idx * RB;
+                    vp = vdil + (size_t)idx * RB;
+                } else {
+                    const long long pos = r_lo + (idx - n_dil);
+                    kp = kwin + (size_t)(pos % p.W) * RB;
+                    vp = vwin + (size_t)(pos % p.W) * RB;
+                }
+                load8(kp + cl * 16, kx[u]);
+                load8(vp + cl * 16, vx[u]);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) { kx[u][j] = 0.f; vx[u][j] = 0.f; }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            // the dot-product shuffle needs every lane of the warp: compute, then discard
+            float dot = 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) dot = fmaf(q[j], kx[u][j], dot);
+#pragma unroll
+            for (int off = LPR / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+            if (have[u]) {
+                const float s = dot * p.scale_log2;
+                const float mn = fmaxf(m, s);
+                const float corr = exp2f(m - mn), pj = exp2f(s - mn);
+                l = fmaf(l, corr, pj);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) o[j] = fmaf(o[j], corr, pj * vx[u][j]);
+                m = mn;
+            }
+        }
+    }
+
+    // split 0: recurrence update, cache append, and the token itself as a key (group 0 of warp 0)
+    if (split == 0 && warp == 0) {
+        float kn[8], vn[8], an[8];
+        load8(static_cast<const uint8_t *>(p.k) + (size_t)bh * RB + cl * 16, kn);
+        load8(static_cast<const uint8_t *>(p.v) + (size_t)bh * RB + cl * 16, vn);
+        load8(static_cast<const uint8_t *>(p.a) + (size_t)bh * RB + cl * 16, an);
+        float *hk = p.hk + (size_t)bh * DH + cl * 8;
+        float *hv = p.hv + (size_t)bh * DH + cl * 8;
+        float sk[8], sv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float g, omg;
+            forget_gate(an[j], g, omg);
+            sk[j] = fmaf(g, hk[j], omg * kn[j]);
+            sv[j] = fmaf(g, hv[j], omg * vn[j]);
+        }
+        float kt[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) kt[j] = sk[j];
+        if (p.rope) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float cs, sn;
+                rope_cs(t, p.theta[(cl * 8 + j) % (DH / 2)], cs, sn);
+                const float partner = __shfl_xor_sync(0xffffffffu, sk[j], LPR / 2);
+                kt[j] = first_half ? sk[j] * cs - partner * sn : sk[j] * cs + partner * sn;
+            }
+        }
+        const uint4 kpk = pack8(kt), vpk = pack8(sv);
+        if (grp == 0) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { hk[j] = sk[j]; hv[j] = sv[j]; }
+            if (t % D == D - 1 && t / D < cap) {
+                uint8_t *kd = static_cast<uint8_t *>(p.kdil) + ((size_t)b * p.total_cap + p.off[h] + t / D) * RB;
+                uint8_t *vd = static_cast<uint8_t *>(p.vdil) + ((size_t)b * p.total_cap + p.off[h] + t / D) * RB;
+                *reinterpret_cast<uint4 *>(kd + cl * 16) = kpk;
+                *reinterpret_cast<uint4 *>(vd + cl * 16) = vpk;
+            }
+            if (p.W > 0) {
+                uint8_t *kw = static_cast<uint8_t *>(p.kwin) + ((size_t)bh * p.W + (size_t)(t % p.W)) * RB;
+                uint8_t *vw = static_cast<uint8_t *>(p.vwin) + ((size_t)bh * p.W + (size_t)(t % p.W)) * RB;
+                *reinterpret_cast<uint4 *>(kw + cl * 16) = kpk;
+                *reinterpret_cast<uint4 *>(vw + cl * 16) = vpk;
+            }
+        }
+        // the token itself, as stored in the cache (rounded), attended by lane group 0
+        float kr[8], vr[8];
+        kr[0] = bf16_lo(kpk.x); kr[1] = bf16_hi(kpk.x); kr[2] = bf16_lo(kpk.y); kr[3] = bf16_hi(kpk.y);
+        kr[4] = bf16_lo(kpk.z); kr[5] = bf16_hi(kpk.z); kr[6] = bf16_lo(kpk.w); kr[7] = bf16_hi(kpk.w);
+        vr[0] = bf16_lo(vpk.x); vr[1] = bf16_hi(vpk.x); vr[2] = bf16_lo(vpk.y); vr[3] = bf16_hi(vpk.y);
+        vr[4] = bf16_lo(vpk.z); vr[5] = bf16_hi(vpk.z); vr[6] = bf16_lo(vpk.w); vr[7] = bf16_hi(vpk.w);
+        float dot = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dot = fmaf(q[j], kr[j], dot);
+#pragma unroll
+        for (int off = LPR / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        if (grp == 0) {
+            const float s = dot * p.scale_log2;
+            const float mn = fmaxf(m, s);
+            const float corr = exp2f(m - mn), pj = exp2f(s - mn);
+            l = fmaf(l, corr, pj);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) o[j] = fmaf(o[j], corr, pj * vr[j]);
+            m = mn;
+        }
+    }
+
+    // merge the lane groups of each warp, then the warps, through shared memory
+    __shared__ float s_m[kWarps * 4], s_l[kWarps * 4];
+    __shared__ float s_o[kWarps * 4][DH];
+    s_m[set] = m;            // every lane of the group writes the same value
+    s_l[set] = l;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) s_o[set][cl * 8 + j] = o[j];
+    __syncthreads();
+    // CTA merge: thread c < DH owns channel c
+    if (tid < DH) {
+        float M = -INFINITY;
+        for (int s2 = 0; s2 < kLanesets; ++s2) M = fmaxf(M, s_m[s2]);
+        float L = 0.f, O = 0.f;
+        for (int s2 = 0; s2 < kLanesets; ++s2) {
+            const float w = s_m[s2] == -INFINITY ? 0.f : exp2f(s_m[s2] - M);
+            L = fmaf(s_l[s2], w, L);
+            O = fmaf(s_o[s2][tid], w, O);
+        }
+        p.part_o[((size_t)bh * p.splits + split) * DH + tid] = O;
+        if (tid == 0) {
+            p.part_ml[((size_t)bh * p.splits + split) * 2 + 0] = M;
+            p.part_ml[((size_t)bh * p.splits + split) * 2 + 1] = L;
+        }
+        __threadfence();
+    }
+    __shared__ uint32_t s_last;
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&p.tickets[bh], 1u) == (uint32_t)p.splits - 1;
+    __syncthreads();
+    if (!s_last) return;
+    // last CTA of the slice: merge the splits
+    if (tid < DH) {
+        float M = -INFINITY;
+        for (int s2 = 0; s2 < p.splits; ++s2) M = fmaxf(M, __ldcg(&p.part_ml[((size_t)bh * p.splits + s2) * 2]));
+        float L = 0.f, O = 0.f;
+        for (int s2 = 0; s2 < p.splits; ++s2) {
+            const float ms = __ldcg(&p.part_ml[((size_t)bh * p.splits + s2) * 2]);
+            const float w = ms == -INFINITY ? 0.f : exp2f(ms - M);
+            L = fmaf(__ldcg(&p.part_ml[((size_t)bh * p.splits + s2) * 2 + 1]), w, L);
+            O = fmaf(__ldcg(&p.part_o[((size_t)bh * p.splits + s2) * DH + tid]), w, O);
+        }
+        const float r = O / L;
+        __nv_bfloat16 *out = static_cast<__nv_bfloat16 *>(p.o) + (size_t)bh * DH + tid;
+        *out = __float2bfloat16_rn(r);
+    }
+    if (tid == 0) p.tickets[bh] = 0u;
+}
+
+int decode_splits(int B, int H, int Tcap, const int32_t *Dh, int W) {
+    // aim for about 8 CTAs per SM over the 148 SMs, and at least ~128 keys per split
+    long long max_keys = 0;
+    for (int h = 0; h < H; ++h) {
+        const long long k = Tcap / Dh[h] + W;
+        max_keys = k > max_keys ? k : max_keys;
+    }
+    const long long bh = (long long)B * H;
+    long long s = (148ll * 8 + bh - 1) / bh;
+    const long long by_keys = (max_keys + 127) / 128;
+    if (s > by_keys) s = by_keys;
+    if (s < 1) s = 1;
+    if (s > 64) s = 64;
+    return (int)s;
+}
+
+size_t decode_workspace_bytes(int B, int H, int d, int splits) {
+    const size_t bh = (size_t)B * H;
+    return sizeof(WsHeader) + align256(bh * 4) + align256(bh * splits * 2 * 4) + align256(bh * splits * d * 4);
+}
+
+int launch_decode(const DecodeParams &p, int dtype, void *stream) {
+    if (dtype != RAT_BF16) return RAT_ERR_UNSUPPORTED;
+    dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.H));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p.d == 128) decode_kernel<128><<<grid, kThreads, 0, s>>>(p);
+    else if (p.d == 64) decode_kernel<64><<<grid, kThreads, 0, s>>>(p);
+    else return RAT_ERR_UNSUPPORTED;
+    return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
+}
+
+}  // namespace rat

@@ -1,0 +1,112 @@
+// internal.h -- declarations shared between the C ABI layer and the kernels (not installed).
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/rat.h"
+
+namespace rat {
+
+// Every device-side wait gives up after this long and records RAT_ERR_TIMEOUT.
+constexpr uint64_t kWaitLimitNs = 2000ull * 1000ull * 1000ull;   // 2 s
+
+// First 256 bytes of every workspace.
+struct WsHeader {
+    int error;          // first device-side error of any launch since the last rat_sync_status
+    uint32_t detail;    // where it happened (kernel-specific code)
+    uint32_t epoch;     // launch counter: tags look-back flags so they never need clearing
+    uint32_t ticket;    // CTA ticket dispenser (reset by the last CTA of each launch)
+    uint32_t done;      // CTAs finished in the current launch
+    uint32_t pad[59];
+};
+static_assert(sizeof(WsHeader) == 256, "workspace header must be 256 bytes");
+
+constexpr size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------------------- recurrence
+struct RecurParams {
+    const void *k, *v, *a;
+    const float *h0k, *h0v;
+    void *yk, *yv;
+    float *hTk, *hTv;
+    int BH, T, d, nchunks;
+    long long pos0;
+    int rope;                   // 1: rotate k~
+    WsHeader *hdr;
+    uint32_t *flags;            // [BH * nchunks]
+    float *agg;                 // [BH * nchunks][3][d]   A, Bk, Bv of the chunk
+    float *pre;                 // [BH * nchunks][2][d]   inclusive state Hk, Hv after the chunk
+    double theta[64];           // RoPE frequency theta_c = base^(-2c/d), c < d/2
+    float step_cos[64], step_sin[64];   // cos/sin(theta_c): one-position rotation
+    long long fault_chunk;      // test hook: chunk index that never publishes (-1: none)
+    unsigned long long wait_ns; // bound of each look-back wait
+};
+int recur_chunk_rows(int d, int dtype);
+size_t recur_workspace_bytes(int BH, int T, int d, int dtype);
+int launch_recur(const RecurParams &p, int dtype, void *stream);
+
+// ---------------------------------------------------------------------------- attention
+constexpr int kMaxHeads = 256;
+
+struct AttnSimtParams {
+    const void *q, *k, *v;
+    void *o;
+    int B, H, T, d, W;
+    long long pos0;
+    int rope;
+    float scale_log2;           // softmax scale * log2(e)
+    int Dh[kMaxHeads];
+    double theta[64];
+};
+int launch_attn_simt(const AttnSimtParams &p, int dtype, void *stream);
+
+struct AttnSm100Args {
+    const void *q, *k, *v;
+    void *o;
+    int B, H, T, d, W;
+    long long pos0;
+    int rope;
+    float scale_log2;
+    const int32_t *Dh;          // host [H]
+    double theta[64];
+};
+int launch_attn_sm100(const AttnSm100Args &a, void *stream);
+
+// ---------------------------------------------------------------------------- cache / decode
+struct CompressParams {
+    const void *k, *v;
+    const float *hTk, *hTv;
+    void *kdil, *vdil, *kwin, *vwin;
+    float *hk, *hv;
+    int B, H, T, d, W, Tcap, esize;
+    long long pos0;
+    long long total_cap;
+    int Dh[kMaxHeads];
+    long long off[kMaxHeads];
+};
+int launch_compress(const CompressParams &p, void *stream);
+
+struct DecodeParams {
+    const void *q, *k, *v, *a;
+    void *o;
+    void *kdil, *vdil, *kwin, *vwin;
+    float *hk, *hv;
+    int B, H, d, W, Tcap, splits;
+    long long t;                // position of the new token
+    long long total_cap;
+    int rope;
+    float scale_log2;
+    WsHeader *hdr;
+    uint32_t *tickets;          // [B*H]
+    float *part_ml;             // [B*H][splits][2]  running max (log2 units) and sum
+    float *part_o;              // [B*H][splits][d]
+    int Dh[kMaxHeads];
+    long long off[kMaxHeads];
+    double theta[64];
+};
+int decode_splits(int B, int H, int Tcap, const int32_t *Dh, int W);
+size_t decode_workspace_bytes(int B, int H, int d, int splits);
+int launch_decode(const DecodeParams &p, int dtype, void *stream);
+
+}  // namespace rat

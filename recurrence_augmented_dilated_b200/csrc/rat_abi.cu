@@ -1,0 +1,291 @@
+// rat_abi.cu -- the C ABI: argument validation, workspace carving and kernel dispatch.
+//
+// Every entry point validates on the host and returns a rat_status synchronously; all GPU
+// work is enqueued on the caller's stream.  No entry point allocates device memory.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "internal.h"
+
+using namespace rat;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool supported_d(int d) { return d == 64 || d == 128; }
+bool valid_dtype(int dt) { return dt == RAT_F32 || dt == RAT_BF16; }
+int esize(int dt) { return dt == RAT_F32 ? 4 : 2; }
+
+// theta_c = base^(-2c/d), c < d/2 (RoFormer frequencies), in float64.
+void rope_theta(double base, int d, double *theta) {
+    for (int c = 0; c < d / 2; ++c) theta[c] = std::pow(base, -2.0 * (double)c / (double)d);
+    for (int c = d / 2; c < 64; ++c) theta[c] = 0.0;
+}
+
+long long total_capacity(int H, int Tcap, const int32_t *Dh, long long *off) {
+    long long total = 0;
+    for (int h = 0; h < H; ++h) {
+        if (off) off[h] = total;
+        total += Tcap / Dh[h];
+    }
+    return total;
+}
+
+bool valid_cache(const rat_kv_cache *c) {
+    if (!c || c->B < 1 || c->H < 1 || c->H > kMaxHeads || !supported_d(c->d) || c->W < 0 ||
+        c->Tcap < 1 || !valid_dtype(c->dtype) || !c->D)
+        return false;
+    for (int h = 0; h < c->H; ++h)
+        if (c->D[h] < 1) return false;
+    return true;
+}
+
+// Test hook state: armed by rat_debug_inject_lookback_fault, consumed by the next
+// rat_recur_prefill issued from the same host thread.
+thread_local long long g_fault_chunk = -1;
+thread_local unsigned long long g_fault_wait_ns = 0;
+
+}  // namespace
+
+extern "C" {
+
+int rat_debug_inject_lookback_fault(int64_t chunk, int64_t wait_limit_ns) {
+    if (chunk < 1 || wait_limit_ns < 1000000 || wait_limit_ns > (int64_t)kWaitLimitNs)
+        return RAT_ERR_INVALID;
+    g_fault_chunk = chunk;
+    g_fault_wait_ns = (unsigned long long)wait_limit_ns;
+    return RAT_OK;
+}
+
+const char *rat_status_string(int status) {
+    switch (status) {
+        case RAT_OK: return "RAT_OK";
+        case RAT_ERR_INVALID: return "RAT_ERR_INVALID: invalid argument";
+        case RAT_ERR_UNSUPPORTED: return "RAT_ERR_UNSUPPORTED: unsupported configuration";
+        case RAT_ERR_CUDA: return "RAT_ERR_CUDA: CUDA call or launch failed";
+        case RAT_ERR_TIMEOUT: return "RAT_ERR_TIMEOUT: a bounded device-side wait ran out";
+        case RAT_ERR_WORKSPACE: return "RAT_ERR_WORKSPACE: workspace missing or too small";
+        default: return "unknown rat_status";
+    }
+}
+
+const char *rat_version(void) { return "rat-b200 0.1 sm_100a"; }
+
+int64_t rat_attended_keys(int64_t t, int D, int W) {
+    if (t < 0 || D < 1) return 0;
+    const int64_t We = W > 1 ? W : 1;
+    const int64_t win = We < t + 1 ? We : t + 1;
+    const int64_t older = t - We + 1;
+    return win + (older > 0 ? older / D : 0);
+}
+
+int rat_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws || ws_bytes < sizeof(WsHeader)) return RAT_ERR_WORKSPACE;
+    return cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? RAT_OK : RAT_ERR_CUDA;
+}
+
+int rat_sync_status(void *ws, void *stream) {
+    if (!ws) return RAT_ERR_WORKSPACE;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return RAT_ERR_CUDA;
+    int err = 0;
+    WsHeader *hdr = static_cast<WsHeader *>(ws);
+    if (cudaMemcpy(&err, &hdr->error, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return RAT_ERR_CUDA;
+    if (err != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(&hdr->error, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+            return RAT_ERR_CUDA;
+    }
+    return err;
+}
+
+// ------------------------------------------------------------------------------ recurrence
+size_t rat_recur_workspace_bytes(int B, int H, int T, int d, int dtype) {
+    if (B < 1 || H < 1 || T < 0 || !supported_d(d) || !valid_dtype(dtype)) return 0;
+    return recur_workspace_bytes(B * H, T, d, dtype);
+}
+
+int rat_recur_prefill(const void *k, const void *v, const void *gate_logit, const float *h0_k,
+                      const float *h0_v, void *k_rec, void *v_rec, float *hT_k, float *hT_v,
+                      int B, int H, int T, int d, int dtype, int64_t pos0, float rope_base,
+                      void *ws, size_t ws_bytes, void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype)) return RAT_ERR_INVALID;
+    if (!supported_d(d)) return RAT_ERR_UNSUPPORTED;
+    if (pos0 < 0 || !std::isfinite(rope_base)) return RAT_ERR_INVALID;
+    if (T == 0) return RAT_OK;
+    if (!k || !v || !gate_logit || !k_rec || !v_rec) return RAT_ERR_INVALID;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(gate_logit) || !aligned16(k_rec) ||
+        !aligned16(v_rec))
+        return RAT_ERR_INVALID;
+    if ((long long)B * H * T > (1ll << 40)) return RAT_ERR_UNSUPPORTED;
+    const size_t need = recur_workspace_bytes(B * H, T, d, dtype);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RAT_ERR_WORKSPACE;
+
+    RecurParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k; p.v = v; p.a = gate_logit;
+    p.h0k = h0_k; p.h0v = h0_v;
+    p.yk = k_rec; p.yv = v_rec;
+    p.hTk = hT_k; p.hTv = hT_v;
+    p.BH = B * H; p.T = T; p.d = d;
+    const int tc = recur_chunk_rows(d, dtype);
+    p.nchunks = (T + tc - 1) / tc;
+    p.pos0 = pos0;
+    p.rope = rope_base > 0.f ? 1 : 0;
+    p.fault_chunk = g_fault_chunk;
+    p.wait_ns = g_fault_chunk >= 0 ? g_fault_wait_ns : kWaitLimitNs;
+    g_fault_chunk = -1;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const size_t nch = (size_t)p.BH * p.nchunks;
+    p.hdr = reinterpret_cast<WsHeader *>(w);
+    p.flags = reinterpret_cast<uint32_t *>(w + sizeof(WsHeader));
+    p.agg = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256(nch * 4));
+    p.pre = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256(nch * 4) + align256(nch * 3 * d * 4));
+    if (p.rope) {
+        rope_theta(rope_base, d, p.theta);
+        for (int c = 0; c < 64; ++c) {
+            p.step_cos[c] = (float)std::cos(p.theta[c]);
+            p.step_sin[c] = (float)std::sin(p.theta[c]);
+        }
+    }
+    return launch_recur(p, dtype, stream);
+}
+
+// ------------------------------------------------------------------------------ attention
+int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, int B,
+                             int H, int T, int d, int dtype, int D, int W,
+                             const int32_t *D_per_head, int64_t pos0, float rope_base,
+                             float scale, void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0) return RAT_ERR_INVALID;
+    if (!supported_d(d) || H > kMaxHeads) return RAT_ERR_UNSUPPORTED;
+    if (!std::isfinite(rope_base) || !std::isfinite(scale)) return RAT_ERR_INVALID;
+    if (!D_per_head && D < 1) return RAT_ERR_INVALID;
+    if (D_per_head)
+        for (int h = 0; h < H; ++h)
+            if (D_per_head[h] < 1) return RAT_ERR_INVALID;
+    if (T == 0) return RAT_OK;
+    if (!q || !k_rec || !v_rec || !o) return RAT_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k_rec) || !aligned16(v_rec) || !aligned16(o)) return RAT_ERR_INVALID;
+    if ((long long)B * H > 65535 || T > (1 << 30)) return RAT_ERR_UNSUPPORTED;
+    const float sc = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)d));
+    const float scale_log2 = sc * 1.4426950408889634f;
+
+    int32_t Dh[kMaxHeads];
+    for (int h = 0; h < H; ++h) Dh[h] = D_per_head ? D_per_head[h] : D;
+
+    if (dtype == RAT_BF16 && d == 128) {
+        AttnSm100Args a;
+        std::memset(&a, 0, sizeof(a));
+        a.q = q; a.k = k_rec; a.v = v_rec; a.o = o;
+        a.B = B; a.H = H; a.T = T; a.d = d; a.W = W;
+        a.pos0 = pos0;
+        a.rope = rope_base > 0.f ? 1 : 0;
+        a.scale_log2 = scale_log2;
+        a.Dh = Dh;
+        if (a.rope) rope_theta(rope_base, d, a.theta);
+        return launch_attn_sm100(a, stream);
+    }
+    AttnSimtParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k_rec; p.v = v_rec; p.o = o;
+    p.B = B; p.H = H; p.T = T; p.d = d; p.W = W;
+    p.pos0 = pos0;
+    p.rope = rope_base > 0.f ? 1 : 0;
+    p.scale_log2 = scale_log2;
+    for (int h = 0; h < H; ++h) p.Dh[h] = Dh[h];
+    if (p.rope) rope_theta(rope_base, d, p.theta);
+    return launch_attn_simt(p, dtype, stream);
+}
+
+// ------------------------------------------------------------------------------ cache
+int rat_kv_cache_bytes(const rat_kv_cache *c, size_t *dil_bytes, size_t *win_bytes,
+                       size_t *state_bytes) {
+    if (!valid_cache(c)) return RAT_ERR_INVALID;
+    const size_t row = (size_t)c->d * esize(c->dtype);
+    const long long total = total_capacity(c->H, c->Tcap, c->D, nullptr);
+    if (dil_bytes) *dil_bytes = (size_t)c->B * total * row;
+    if (win_bytes) *win_bytes = (size_t)c->B * c->H * c->W * row;
+    if (state_bytes) *state_bytes = (size_t)c->B * c->H * c->d * sizeof(float);
+    return RAT_OK;
+}
+
+int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, const float *hT_v,
+                    int T, rat_kv_cache *c, void *stream) {
+    if (!valid_cache(c) || T < 0) return RAT_ERR_INVALID;
+    if (c->pos < 0 || c->pos + T > c->Tcap) return RAT_ERR_INVALID;
+    if (T == 0) return RAT_OK;
+    if (!k_rec || !v_rec || !c->k_dil || !c->v_dil || !c->h_k || !c->h_v) return RAT_ERR_INVALID;
+    if (c->W > 0 && (!c->k_win || !c->v_win)) return RAT_ERR_INVALID;
+    if (!aligned16(k_rec) || !aligned16(v_rec) || !aligned16(c->k_dil) || !aligned16(c->v_dil) ||
+        (c->W > 0 && (!aligned16(c->k_win) || !aligned16(c->v_win))))
+        return RAT_ERR_INVALID;
+    if ((long long)c->B * c->H > 65535) return RAT_ERR_UNSUPPORTED;
+    CompressParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k_rec; p.v = v_rec; p.hTk = hT_k; p.hTv = hT_v;
+    p.kdil = c->k_dil; p.vdil = c->v_dil; p.kwin = c->k_win; p.vwin = c->v_win;
+    p.hk = c->h_k; p.hv = c->h_v;
+    p.B = c->B; p.H = c->H; p.T = T; p.d = c->d; p.W = c->W; p.Tcap = c->Tcap;
+    p.esize = esize(c->dtype);
+    p.pos0 = c->pos;
+    for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
+    p.total_cap = total_capacity(c->H, c->Tcap, c->D, p.off);
+    const int st = launch_compress(p, stream);
+    if (st == RAT_OK) c->pos += T;
+    return st;
+}
+
+// ------------------------------------------------------------------------------ decode
+size_t rat_decode_workspace_bytes(const rat_kv_cache *c) {
+    if (!valid_cache(c)) return 0;
+    const int s = decode_splits(c->B, c->H, c->Tcap, c->D, c->W);
+    return decode_workspace_bytes(c->B, c->H, c->d, s);
+}
+
+int rat_dilated_decode(const void *q, const void *k, const void *v, const void *gate_logit,
+                       rat_kv_cache *c, void *o, float rope_base, float scale, void *ws,
+                       size_t ws_bytes, void *stream) {
+    if (!valid_cache(c)) return RAT_ERR_INVALID;
+    if (c->dtype != RAT_BF16) return RAT_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gate_logit || !o) return RAT_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logit) || !aligned16(o))
+        return RAT_ERR_INVALID;
+    if (!c->k_dil || !c->v_dil || !c->h_k || !c->h_v) return RAT_ERR_INVALID;
+    if (c->W > 0 && (!c->k_win || !c->v_win)) return RAT_ERR_INVALID;
+    if (c->pos < 0 || c->pos >= c->Tcap) return RAT_ERR_INVALID;
+    if (!std::isfinite(rope_base) || !std::isfinite(scale)) return RAT_ERR_INVALID;
+    if ((long long)c->B * c->H > 65535) return RAT_ERR_UNSUPPORTED;
+    const int splits = decode_splits(c->B, c->H, c->Tcap, c->D, c->W);
+    const size_t need = decode_workspace_bytes(c->B, c->H, c->d, splits);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RAT_ERR_WORKSPACE;
+
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v; p.a = gate_logit; p.o = o;
+    p.kdil = c->k_dil; p.vdil = c->v_dil; p.kwin = c->k_win; p.vwin = c->v_win;
+    p.hk = c->h_k; p.hv = c->h_v;
+    p.B = c->B; p.H = c->H; p.d = c->d; p.W = c->W; p.Tcap = c->Tcap; p.splits = splits;
+    p.t = c->pos;
+    for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
+    p.total_cap = total_capacity(c->H, c->Tcap, c->D, p.off);
+    p.rope = rope_base > 0.f ? 1 : 0;
+    const float sc = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)c->d));
+    p.scale_log2 = sc * 1.4426950408889634f;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const size_t bh = (size_t)c->B * c->H;
+    p.hdr = reinterpret_cast<WsHeader *>(w);
+    p.tickets = reinterpret_cast<uint32_t *>(w + sizeof(WsHeader));
+    p.part_ml = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256(bh * 4));
+    p.part_o = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256(bh * 4) + align256(bh * splits * 2 * 4));
+    if (p.rope) rope_theta(rope_base, c->d, p.theta);
+    const int st = launch_decode(p, c->dtype, stream);
+    if (st == RAT_OK) c->pos += 1;
+    return st;
+}
+
+}  // extern "C"

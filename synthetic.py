@@ -16,8 +16,8 @@ FineWeb-Edu, LongBench, commonsense and NIAH suites, which these random tensors 
 Recipe (prefill): one CPU ``torch.Generator`` seeded with the workload's seed draws float32
 standard normals in the order q, k, v, a (a = mu + sigma * N(0,1)), each (B, H, T, d); the
 results are then cast to the dtype.  Decode: the context k, v, a of slice (b, h) come from a
-generator seeded with (seed, b, h) on the requested device, so one slice can be regenerated
-alone; the per-step tokens come from one CPU generator, drawn as q, k, v, a of shape
+generator seeded with (seed, b, h, chunk) on the requested device, 8192 positions per chunk,
+so one slice (or one chunk of all slices) can be regenerated alone; the per-step tokens come from one CPU generator, drawn as q, k, v, a of shape
 (steps, B, H, d).
 """
 from __future__ import annotations
@@ -86,14 +86,39 @@ def prefill_inputs(w: Workload, B=None, H=None, T=None, seed=None):
     return {"q": q.to(dt), "k": k.to(dt), "v": v.to(dt), "a": a.to(dt)}
 
 
-def decode_context_slice(w: Workload, b: int, h: int, device="cpu", T=None):
-    """Context k, v, a of one (batch, head) slice, shape (T, d) each, on `device`."""
+CTX_CHUNK = 8192        # context positions drawn per generator call
+
+
+def decode_context_chunk(w: Workload, b: int, h: int, c: int, device="cpu", T=None):
+    """Context k, v, a of slice (b, h) at positions [c*CTX_CHUNK, min((c+1)*CTX_CHUNK, T)),
+    shape (3, rows, d), from a generator seeded with (seed, b, h, c) on `device`."""
     T = w.T if T is None else T
+    lo, hi = c * CTX_CHUNK, min((c + 1) * CTX_CHUNK, T)
     g = torch.Generator(device=device)
-    g.manual_seed(w.seed * 1_000_003 + b * 1009 + h + 1)
-    kva = torch.randn((3, T, w.d), generator=g, dtype=torch.float32, device=device)
+    g.manual_seed(((w.seed * 1_000_003 + b) * 1009 + h) * 4099 + c + 1)
+    kva = torch.randn((3, hi - lo, w.d), generator=g, dtype=torch.float32, device=device)
     kva[2].mul_(w.gate_sigma).add_(w.gate_mu)
     return kva.to(w.torch_dtype)
+
+
+def decode_context_slice(w: Workload, b: int, h: int, device="cpu", T=None):
+    """Whole context k, v, a of one (batch, head) slice, shape (3, T, d)."""
+    T = w.T if T is None else T
+    n = (T + CTX_CHUNK - 1) // CTX_CHUNK
+    return torch.cat([decode_context_chunk(w, b, h, c, device, T) for c in range(n)], dim=1)
+
+
+def decode_context_block(w: Workload, c: int, device="cpu", T=None, B=None, H=None):
+    """Chunk c of the context of every slice: k, v, a each (B, H, rows, d), contiguous."""
+    T = w.T if T is None else T
+    B = w.B if B is None else B
+    H = w.H if H is None else H
+    lo, hi = c * CTX_CHUNK, min((c + 1) * CTX_CHUNK, T)
+    out = torch.empty((3, B, H, hi - lo, w.d), dtype=w.torch_dtype, device=device)
+    for b in range(B):
+        for h in range(H):
+            out[:, b, h] = decode_context_chunk(w, b, h, c, device, T)
+    return out[0], out[1], out[2]
 
 
 def decode_steps(w: Workload, steps=None):

@@ -1,0 +1,156 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every symbol the
+header declares, and validates its arguments before touching the GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import recurrence_augmented_dilated_b200 as rat
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from recurrence_augmented_dilated_b200 import build
+    build.build()
+    return rat.lib()
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"RAT_API\s+[\w\s\*]+?\b(rat_\w+)\s*\(", txt))
+    return names
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_symbols()
+    assert {"rat_recur_prefill", "rat_dilated_attn_prefill", "rat_kv_compress",
+            "rat_dilated_decode"} <= names
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, -5):
+        assert rat.rat_status_string(code).startswith(("RAT_OK", "RAT_ERR"))
+    assert "sm_100a" in L.rat_version().decode()
+
+
+def closed_form_count(t, D, W):
+    We = max(W, 1)
+    return min(We, t + 1) + max(0, (t - We + 1) // D)
+
+
+def test_attended_keys_matches_count(L):
+    for D, W in [(1, 0), (4, 0), (16, 0), (64, 128), (64, 64), (3, 7)]:
+        for t in [0, 1, 2, 63, 64, 127, 128, 1000, 32767]:
+            assert rat.rat_attended_keys(t, D, W) == closed_form_count(t, D, W)
+
+
+def test_recur_validation(L):
+    P = ctypes.c_void_p
+    ws = P(4096 * 256)            # never dereferenced: validation fails first
+    # B < 1
+    assert L.rat_recur_prefill(P(256), P(256), P(256), None, None, P(256), P(256), None, None,
+                               0, 1, 8, 128, 1, 0, 0.0, ws, 1 << 20, None) == -1
+    # d unsupported
+    assert L.rat_recur_prefill(P(256), P(256), P(256), None, None, P(256), P(256), None, None,
+                               1, 1, 8, 96, 1, 0, 0.0, ws, 1 << 20, None) == -2
+    # NULL input
+    assert L.rat_recur_prefill(None, P(256), P(256), None, None, P(256), P(256), None, None,
+                               1, 1, 8, 128, 1, 0, 0.0, ws, 1 << 20, None) == -1
+    # misaligned input
+    assert L.rat_recur_prefill(P(258), P(256), P(256), None, None, P(256), P(256), None, None,
+                               1, 1, 8, 128, 1, 0, 0.0, ws, 1 << 20, None) == -1
+    # workspace too small / missing
+    need = rat.rat_recur_workspace_bytes(1, 1, 8, 128, 1)
+    assert need > 256
+    assert L.rat_recur_prefill(P(256), P(256), P(256), None, None, P(256), P(256), None, None,
+                               1, 1, 8, 128, 1, 0, 0.0, ws, need - 1, None) == -5
+    assert L.rat_recur_prefill(P(256), P(256), P(256), None, None, P(256), P(256), None, None,
+                               1, 1, 8, 128, 1, 0, 0.0, None, need, None) == -5
+    # T == 0 is a no-op
+    assert L.rat_recur_prefill(None, None, None, None, None, None, None, None, None,
+                               1, 1, 0, 128, 1, 0, 0.0, None, 0, None) == 0
+
+
+def test_recur_workspace_grows_with_chunks(L):
+    a = rat.rat_recur_workspace_bytes(1, 1, 128, 128, 1)
+    b = rat.rat_recur_workspace_bytes(1, 1, 129, 128, 1)
+    c = rat.rat_recur_workspace_bytes(4, 16, 4096, 128, 1)
+    assert 256 < a < b < c
+    assert rat.rat_recur_workspace_bytes(0, 1, 8, 128, 1) == 0
+
+
+def test_attn_validation(L):
+    P = ctypes.c_void_p
+    ok = dict(q=P(256), k=P(256), v=P(256), o=P(256))
+    args = lambda **kw: [kw.get(n, ok.get(n)) for n in ("q", "k", "v", "o")]
+    # D < 1 with no per-head table
+    assert L.rat_dilated_attn_prefill(*args(), 1, 1, 8, 128, 1, 0, 0, None, 0, 0.0, 0.0, None) == -1
+    # W < 0
+    assert L.rat_dilated_attn_prefill(*args(), 1, 1, 8, 128, 1, 1, -1, None, 0, 0.0, 0.0, None) == -1
+    # per-head D with a zero
+    Dh = (ctypes.c_int32 * 2)(4, 0)
+    assert L.rat_dilated_attn_prefill(*args(), 1, 2, 8, 128, 1, 1, 0, Dh, 0, 0.0, 0.0, None) == -1
+    # misaligned output
+    assert L.rat_dilated_attn_prefill(*args(o=P(260)), 1, 1, 8, 128, 1, 1, 0, None, 0, 0.0, 0.0, None) == -1
+    # unsupported head dim
+    assert L.rat_dilated_attn_prefill(*args(), 1, 1, 8, 80, 1, 1, 0, None, 0, 0.0, 0.0, None) == -2
+    # too many heads for the per-head table
+    assert L.rat_dilated_attn_prefill(*args(), 1, 300, 8, 128, 1, 1, 0, None, 0, 0.0, 0.0, None) == -2
+
+
+def cache(**kw):
+    D = (ctypes.c_int32 * kw.get("H", 2))(*kw.get("Dlist", [1, 64]))
+    c = rat.KVCache(B=kw.get("B", 2), H=kw.get("H", 2), d=kw.get("d", 128), W=kw.get("W", 16),
+                    Tcap=kw.get("Tcap", 1024), dtype=kw.get("dtype", 1), D=D)
+    c._keep = D
+    return c
+
+
+def test_cache_bytes_layout(L):
+    c = cache()
+    dil, win, state = rat.rat_kv_cache_bytes(c)
+    # cap_h = floor(Tcap / D_h): 1024 + 16 entries per sequence, bf16 rows of 256 bytes
+    assert dil == 2 * (1024 + 16) * 256
+    assert win == 2 * 2 * 16 * 256
+    assert state == 2 * 2 * 128 * 4
+    bad = cache(Dlist=[1, 0])
+    with pytest.raises(rat.RatError):
+        rat.rat_kv_cache_bytes(bad)
+
+
+def test_compress_and_decode_validation(L):
+    P = ctypes.c_void_p
+    c = cache()
+    c.k_dil = c.v_dil = c.k_win = c.v_win = c.h_k = c.h_v = 256
+    # beyond capacity
+    c.pos = 1000
+    assert L.rat_kv_compress(P(256), P(256), None, None, 100, ctypes.byref(c), None) == -1
+    # decode at pos == Tcap
+    c.pos = 1024
+    ws = P(256 * 4096)
+    assert L.rat_dilated_decode(P(256), P(256), P(256), P(256), ctypes.byref(c), P(256), 0.0, 0.0,
+                                ws, 1 << 30, None) == -1
+    # decode with a too-small workspace
+    c.pos = 5
+    need = rat.rat_decode_workspace_bytes(c)
+    assert need > 256
+    assert L.rat_dilated_decode(P(256), P(256), P(256), P(256), ctypes.byref(c), P(256), 0.0, 0.0,
+                                ws, need - 1, None) == -5
+    # fp32 decode is not provided
+    c32 = cache(dtype=0)
+    c32.k_dil = c32.v_dil = c32.k_win = c32.v_win = c32.h_k = c32.h_v = 256
+    assert L.rat_dilated_decode(P(256), P(256), P(256), P(256), ctypes.byref(c32), P(256), 0.0, 0.0,
+                                ws, 1 << 30, None) == -2
+
+
+def test_workspace_init_rejects_null(L):
+    assert L.rat_workspace_init(None, 1024, None) == -5
+    assert L.rat_sync_status(None, None) == -5

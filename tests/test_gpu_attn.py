@@ -1,0 +1,147 @@
+"""GPU parity of rat_dilated_attn_prefill against the float64 oracle.
+
+The attention is checked on its own (q, k~, v~ drawn by the seeded generator and fed to both
+sides) and end to end (GPU recurrence -> GPU attention vs the oracle's recurrence ->
+attention, both from the same raw inputs).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import recurrence_augmented_dilated_b200 as rat
+import synthetic
+from gpu_util import TOL_BF16, TOL_F32, f64, gpu_attn, gpu_recur, rel_err, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def qkv(B, H, T, d, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    return tuple(torch.randn((B, H, T, d), generator=g).to(dtype) for _ in range(3))
+
+
+def check_attn(q, k, v, D=1, W=0, D_per_head=None, rope_base=0.0, pos0=0, rows=None, heads=None,
+               tol=None):
+    o = gpu_attn(q, k, v, D=D, W=W, D_per_head=D_per_head, rope_base=rope_base, pos0=pos0)
+    B, H, T, d = q.shape
+    heads = heads if heads is not None else list(range(H))
+    qs, ks, vs = (f64(x[:, heads]) for x in (q, k, v))
+    Dh = None
+    if D_per_head is not None:
+        Dh = [D_per_head[h] for h in heads]
+    if rope_base > 0:
+        qs = oracle.rope(qs, pos0, rope_base)
+    ref = oracle.dilated_attention(qs, ks, vs, D=D, W=W, D_per_head=Dh, rows=rows)
+    got = o[:, heads]
+    if rows is not None:
+        got = got[:, :, rows]
+    err = rel_err(got, ref)
+    assert err <= (tol if tol is not None else tol_for(q.dtype)), err
+    return o, err
+
+
+@pytest.mark.parametrize("D,W", [(4, 0), (1, 0), (3, 5), (64, 128), (16, 16), (300, 0)])
+@pytest.mark.parametrize("T", [1, 100, 256, 333])
+def test_fp32_cases(D, W, T):
+    q, k, v = qkv(1, 2, T, 64, torch.float32, seed=T * 7 + D)
+    check_attn(q, k, v, D=D, W=W)
+
+
+def test_tiny_fp32_workload():
+    w = synthetic.WORKLOADS["tiny_fp32"]
+    x = synthetic.prefill_inputs(w)
+    kr, vr, _, _ = gpu_recur(x["k"], x["v"], x["a"])
+    o = gpu_attn(x["q"], kr, vr, D=w.D, W=w.W)
+    ref = oracle.layer_prefill(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(x["a"]), D=w.D, W=w.W)
+    assert rel_err(o, ref["o"]) <= TOL_F32
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_fp32_hybrid_heads_and_rope(d):
+    q, k, v = qkv(2, 4, 200, d, torch.float32, seed=d)
+    check_attn(q, k, v, W=7, D_per_head=[1, 4, 16, 64], rope_base=10000.0, pos0=999)
+
+
+BF16_CASES = [
+    # (B, H, T, D, W, D_per_head)
+    (1, 2, 1, 16, 0, None),
+    (1, 2, 127, 16, 0, None),
+    (2, 2, 128, 4, 0, None),
+    (1, 3, 129, 1, 0, None),
+    (1, 2, 300, 16, 0, None),
+    (1, 2, 513, 64, 128, None),
+    (2, 2, 1000, 8, 64, None),
+    (1, 4, 777, 1, 64, [1, 64, 1, 64]),
+    (1, 2, 640, 200, 0, None),
+    (1, 2, 1100, 2, 300, None),
+    (1, 4, 2048, 16, 33, [1, 2, 16, 64]),
+]
+
+
+@pytest.mark.parametrize("B,H,T,D,W,Dph", BF16_CASES)
+def test_bf16_cases(B, H, T, D, W, Dph):
+    q, k, v = qkv(B, H, T, 128, torch.bfloat16, seed=T + 31 * D + W)
+    check_attn(q, k, v, D=D, W=W, D_per_head=Dph)
+
+
+def test_bf16_d64():
+    q, k, v = qkv(1, 2, 300, 64, torch.bfloat16, seed=64)
+    check_attn(q, k, v, D=4, W=3)
+
+
+def test_bf16_rope_query():
+    q, k, v = qkv(1, 2, 700, 128, torch.bfloat16, seed=77)
+    check_attn(q, k, v, D=16, W=0, rope_base=10000.0, pos0=3000)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_self_only_returns_values_exactly(dtype):
+    # D > T and W = 0: every query sees only itself, so o_t = v~_t exactly.
+    q, k, v = qkv(1, 2, 300, 128, dtype, seed=5)
+    o = gpu_attn(q, k, v, D=1000, W=0)
+    assert torch.equal(o.cpu(), v)
+
+
+def test_dense_d1_equals_window_covering_all():
+    q, k, v = qkv(1, 2, 500, 128, torch.bfloat16, seed=8)
+    o1 = gpu_attn(q, k, v, D=1, W=0)
+    o2 = gpu_attn(q, k, v, D=64, W=500)
+    ref = oracle.dilated_attention(f64(q), f64(k), f64(v), D=1, W=0)
+    assert rel_err(o1, ref) <= TOL_BF16 and rel_err(o2, ref) <= TOL_BF16
+
+
+def test_head_hybrid_equals_uniform_runs():
+    q, k, v = qkv(1, 4, 600, 128, torch.bfloat16, seed=9)
+    Dh = [1, 4, 16, 64]
+    o = gpu_attn(q, k, v, W=32, D_per_head=Dh)
+    for h, D in enumerate(Dh):
+        oh = gpu_attn(q[:, h:h + 1].contiguous(), k[:, h:h + 1].contiguous(), v[:, h:h + 1].contiguous(), D=D, W=32)
+        assert torch.equal(o[:, h:h + 1], oh)
+
+
+def sample_rows(T, n=96, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.integers(0, T, size=n).tolist())
+    rows |= {0, 1, 127, 128, 129, T // 2, T - 129, T - 128, T - 2, T - 1}
+    return sorted(r for r in rows if 0 <= r < T)
+
+
+@pytest.mark.parametrize("name", ["prefill_1p5b", "window_2p6b", "hybrid_7p6b"])
+def test_full_size_end_to_end_sampled(name):
+    """Whole prefill (recurrence + attention) at the workload's full size, checked on sampled
+    heads and rows against the oracle's own recurrence and attention."""
+    w = synthetic.WORKLOADS[name]
+    x = synthetic.prefill_inputs(w)
+    kr, vr, _, _ = gpu_recur(x["k"], x["v"], x["a"], rope_base=w.rope_base)
+    o = gpu_attn(x["q"], kr, vr, D=w.D, W=w.W, D_per_head=w.D_per_head, rope_base=w.rope_base)
+    Dh = w.heads_D()
+    heads = sorted({0, w.H - 1, w.H // 2} | ({7, 8} if w.D_per_head else set()))
+    rows = sample_rows(w.T, seed=w.seed)
+    for b in sorted({0, w.B - 1}):
+        sl = lambda t: f64(t[b:b + 1, heads])
+        ref = oracle.layer_prefill(sl(x["q"]), sl(x["k"]), sl(x["v"]), sl(x["a"]),
+                                   D_per_head=[Dh[h] for h in heads], W=w.W, rope_base=w.rope_base,
+                                   rows=rows)
+        err = rel_err(o[b:b + 1, heads][:, :, rows], ref["o"])
+        assert err <= TOL_BF16, (b, err)

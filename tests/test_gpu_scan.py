@@ -1,0 +1,136 @@
+"""GPU parity of rat_recur_prefill (chunked associative scan) against the float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import recurrence_augmented_dilated_b200 as rat
+import synthetic
+from gpu_util import TOL_BF16, TOL_F32, f64, gpu_recur, rel_err, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def check(k, v, a, rope_base=0.0, pos0=0, heads=None, h0=None):
+    """GPU vs oracle on all (b, h) or on `heads` (list of (b, h))."""
+    h0k = h0v = None
+    if h0 is not None:
+        h0k, h0v = (x.cuda() for x in h0)
+    kr, vr, hTk, hTv = gpu_recur(k, v, a, rope_base=rope_base, pos0=pos0, h0k=h0k, h0v=h0v)
+    sel = heads if heads is not None else [(b, h) for b in range(k.shape[0]) for h in range(k.shape[1])]
+    bi = [b for b, _ in sel]
+    hi = [h for _, h in sel]
+    ok_, ov_ = f64(k[bi, hi]), f64(v[bi, hi])
+    oa_ = f64(a[bi, hi])
+    o_h0k = f64(h0[0][bi, hi]) if h0 is not None else None
+    o_h0v = f64(h0[1][bi, hi]) if h0 is not None else None
+    yk, hk = oracle.recurrence(ok_, oa_, o_h0k)
+    yv, hv = oracle.recurrence(ov_, oa_, o_h0v)
+    if rope_base > 0:
+        yk = oracle.rope(yk, pos0, rope_base)
+    tol = tol_for(k.dtype)
+    errs = dict(k=rel_err(kr[bi, hi], yk), v=rel_err(vr[bi, hi], yv), hk=rel_err(hTk[bi, hi], hk),
+                hv=rel_err(hTv[bi, hi], hv))
+    # the float32 state is exact up to float32 rounding even on the bf16 path
+    assert errs["hk"] <= TOL_F32 * (10 if k.dtype == torch.bfloat16 else 1), errs
+    assert errs["hv"] <= TOL_F32 * (10 if k.dtype == torch.bfloat16 else 1), errs
+    assert errs["k"] <= tol and errs["v"] <= tol, errs
+    return errs
+
+
+def inputs(B, H, T, d, dtype, mu=2.0, sigma=1.0, seed=0):
+    w = synthetic.Workload("t", B=B, H=H, d=d, T=T, dtype="f32" if dtype == torch.float32 else "bf16",
+                           gate_mu=mu, gate_sigma=sigma, seed=seed)
+    return synthetic.prefill_inputs(w)
+
+
+def test_tiny_fp32_workload():
+    w = synthetic.WORKLOADS["tiny_fp32"]
+    x = synthetic.prefill_inputs(w)
+    check(x["k"], x["v"], x["a"])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [1, 63, 64, 129, 1000, 2049])
+def test_ragged_lengths(dtype, d, T):
+    x = inputs(2, 3, T, d, dtype, seed=T + d)
+    check(x["k"], x["v"], x["a"])
+
+
+@pytest.mark.parametrize("pos0", [0, 5000, 70000])
+def test_rope_positions(pos0):
+    x = inputs(1, 2, 777, 128, torch.bfloat16, seed=pos0 + 1)
+    check(x["k"], x["v"], x["a"], rope_base=10000.0, pos0=pos0)
+
+
+def test_rope_fp32_precision():
+    x = inputs(1, 2, 300, 64, torch.float32, seed=9)
+    check(x["k"], x["v"], x["a"], rope_base=10000.0, pos0=123456)
+
+
+def test_initial_state_and_chunked_prefill():
+    x = inputs(2, 2, 500, 128, torch.float32, seed=3)
+    g = torch.Generator().manual_seed(5)
+    h0 = (torch.randn((2, 2, 128), generator=g), torch.randn((2, 2, 128), generator=g))
+    check(x["k"], x["v"], x["a"], h0=h0)
+    # two GPU calls chained through hT equal one call
+    k, v, a = (t.cuda() for t in (x["k"], x["v"], x["a"]))
+    kr, vr, hk, hv = gpu_recur(k, v, a)
+    kr1, vr1, hk1, hv1 = gpu_recur(k[:, :, :200].contiguous(), v[:, :, :200].contiguous(), a[:, :, :200].contiguous())
+    kr2, vr2, hk2, hv2 = gpu_recur(k[:, :, 200:].contiguous(), v[:, :, 200:].contiguous(), a[:, :, 200:].contiguous(),
+                                   h0k=hk1, h0v=hv1)
+    assert rel_err(torch.cat([kr1, kr2], 2), kr) <= 1e-5
+    assert rel_err(hk2, hk) <= 1e-5 and rel_err(hv2, hv) <= 1e-5
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_zero_gate_is_identity_exactly(dtype):
+    # logit -1e4: g = 0 and 1-g = 1 exactly, so k~ = k and v~ = v bit for bit
+    x = inputs(1, 2, 300, 128, dtype, seed=11)
+    a = torch.full_like(x["a"], -1.0e4)
+    kr, vr, _, _ = gpu_recur(x["k"], x["v"], a)
+    assert torch.equal(kr.cpu(), x["k"]) and torch.equal(vr.cpu(), x["v"])
+
+
+def test_unit_gate_holds_initial_state():
+    x = inputs(1, 1, 200, 64, torch.float32, seed=12)
+    a = torch.full_like(x["a"], 1.0e4)
+    h0k = torch.randn((1, 1, 64)).cuda()
+    h0v = torch.randn((1, 1, 64)).cuda()
+    kr, vr, hk, hv = gpu_recur(x["k"], x["v"], a, h0k=h0k, h0v=h0v)
+    assert torch.equal(kr[0, 0], h0k[0, 0].expand(200, 64))
+    assert torch.equal(hv, h0v)
+
+
+def test_repeated_launches_reuse_workspace():
+    # the launch epoch lets one workspace serve many calls without clearing
+    x = inputs(2, 4, 1500, 128, torch.bfloat16, seed=21)
+    ws = rat.Workspace(rat.rat_recur_workspace_bytes(2, 4, 1500, 128, 1))
+    first = gpu_recur(x["k"], x["v"], x["a"], ws=ws)[0].cpu()
+    for _ in range(5):
+        again = gpu_recur(x["k"], x["v"], x["a"], ws=ws)[0].cpu()
+        assert torch.equal(again, first)
+
+
+@pytest.mark.parametrize("name", ["prefill_1p5b", "window_2p6b", "hybrid_7p6b"])
+def test_full_size_workloads_sampled_heads(name):
+    w = synthetic.WORKLOADS[name]
+    x = synthetic.prefill_inputs(w)
+    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)]
+    check(x["k"], x["v"], x["a"], rope_base=w.rope_base, heads=heads)
+
+
+def test_lookback_timeout_is_reported():
+    # failure detection: one chunk withholds its publication (test hook); its successors' bounded
+    # waits run out, the device error word reads RAT_ERR_TIMEOUT, and the context stays usable.
+    L = rat.lib()
+    x = inputs(1, 1, 1024, 128, torch.bfloat16, seed=30)
+    L.rat_debug_inject_lookback_fault(2, 20_000_000)      # chunk 2, 20 ms waits, next call only
+    k, v, a = (t.cuda() for t in (x["k"], x["v"], x["a"]))
+    ws = rat.Workspace(rat.rat_recur_workspace_bytes(1, 1, 1024, 128, 1))
+    kr, vr = torch.empty_like(k), torch.empty_like(v)
+    rat.rat_recur_prefill(k, v, a, kr, vr, ws)
+    assert rat.rat_sync_status(ws) == -4
+    # the next call (no fault armed) is correct again
+    check(x["k"], x["v"], x["a"])
