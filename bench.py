@@ -476,13 +476,13 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
-    rank, world, local = dist_setup(args.gpus)
     w = synthetic.WORKLOADS[args.workload]
     metric = "RAT+ layer prefill tokens/s and decode tokens/s at 1 B200; % HBM / tensor roofline"
     peaks, peak_kind = load_peaks()
 
     if args.impl == "reference":
-        if rank != 0:
+        # the CPU oracle runs on rank 0 only; other ranks exit at once without joining a group
+        if int(os.environ.get("RANK", "0")) != 0:
             return 0
         per = []
         desc = cores = None
@@ -506,6 +506,7 @@ def main():
     if not torch.cuda.is_available():
         print(json.dumps({"metric": metric, "error": "no CUDA device"}))
         return 1
+    rank, world, local = dist_setup(args.gpus)
     import recurrence_augmented_dilated_b200 as rat
     rat.lib()       # fail loudly if the library is missing
 

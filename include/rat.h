@@ -134,12 +134,18 @@ RAT_API int rat_recur_prefill(const void *k, const void *v, const void *gate_log
  * S(t) = { t-We < j <= t } U { j <= t-We : j mod D_h = D_h - 1 }, We = max(W, 1).
  * bf16: QK^T and PV on tcgen05 tensor cores (bf16 operands, float32 accumulation; the
  * softmax probabilities are rounded to bf16 for PV); float32: CUDA-core FMA throughout.
- * Needs no workspace; never waits on other CTAs.
+ * Needs no workspace and never waits on other CTAs; its internal pipeline waits are bounded,
+ * and an expired wait is recorded in a library-wide device error word that
+ * rat_attn_sync_status() reads.
  * ---------------------------------------------------------------------------------------- */
 RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o,
                              int B, int H, int T, int d, int dtype, int D, int W,
                              const int32_t *D_per_head, int64_t pos0, float rope_base,
                              float scale, void *stream);
+
+/* Synchronise `stream`, then return (and clear) the first device-side error recorded by the
+ * attention kernel since the last call (RAT_OK if none). */
+RAT_API int rat_attn_sync_status(void *stream);
 
 /* ------------------------------------------------------------------------------------------
  * Compressed KV cache (RAT+ abstract: dilation reduces the KV cache D-fold; "RAT+ Deep Dive"

@@ -23,7 +23,7 @@ __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
-    "rat_workspace_init", "rat_sync_status", "rat_attended_keys", "rat_status_string",
+    "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_attended_keys", "rat_status_string",
     "Workspace",
 ]
 
@@ -84,6 +84,7 @@ def lib():
         L.rat_dilated_decode.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(KVCache), _vp, _f, _f,
                                          _vp, _sz, _vp]
         L.rat_debug_inject_lookback_fault.argtypes = [_i64, _i64]
+        L.rat_attn_sync_status.argtypes = [_vp]
         L.rat_attended_keys.restype = _i64
         L.rat_attended_keys.argtypes = [_i64, _i, _i]
         _lib = L
@@ -142,6 +143,10 @@ def rat_workspace_init(ws: Workspace, stream=None):
 
 def rat_sync_status(ws: Workspace, stream=None) -> int:
     return int(lib().rat_sync_status(ws.ptr, _stream(stream)))
+
+
+def rat_attn_sync_status(stream=None) -> int:
+    return int(lib().rat_attn_sync_status(_stream(stream)))
 
 
 def rat_recur_workspace_bytes(B, H, T, d, dtype) -> int:

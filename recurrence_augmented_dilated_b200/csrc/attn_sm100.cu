@@ -1,19 +1,499 @@
-// attn_sm100.cu -- bf16 dilated attention prefill (tensor-core path; under construction).
+// attn_sm100.cu -- bf16 causal dilated attention prefill on tcgen05 tensor cores (sm_100a).
+//
+// RAT+ abstract ("dilated attention ... optionally with local windows ... hybrid layer/head
+// compositions"); "RAT+ Deep Dive" section 3.1 (attention FLOPs T/D) and section 6 (per-head
+// dilation).  Query t of head h attends to
+//     S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D_h = D_h - 1 },   We = max(W, 1),
+// i.e. its local window (itself included) and the chunk ends older than the window; a head
+// with D_h = 1 is dense causal attention.
+//
+// One CTA computes one 128-query tile of one (b, h) with two key streams:
+//   * the dilated stream -- the chunk ends i*D + D - 1, read through a TMA tensor map whose row
+//     stride is D rows of the recurrence output, so the gather costs nothing but a descriptor;
+//   * the window stream -- the contiguous band of positions the tile's windows cover.
+// Both are cut into blocks of 128 keys.  Per block:
+//   S = Q K^T   (tcgen05.mma, bf16 operands from 128B-swizzled smem, f32 accumulator in TMEM,
+//                double-buffered so the next block's product overlaps this block's softmax);
+//   softmax     (one thread per query row reads its S row from TMEM, masks it to S(t), keeps a
+//                running max and sum; the max is only moved -- and O rescaled in TMEM -- when
+//                it grows by more than 2^8, which keeps the result exact and rescales rare);
+//   O += P V    (P written as bf16 into swizzled smem, V an MN-major smem operand).
+// Roles: warp 0 issues TMA loads (2-stage K/V ring), warp 1 allocates TMEM and issues the
+// MMAs, warps 2-5 do RoPE on Q (in smem), the softmax and the epilogue (O / l -> bf16 -> smem
+// -> TMA store).  Every mbarrier wait is bounded; on expiry the CTA records RAT_ERR_TIMEOUT in
+// a module error word, stops all roles, waits for its own async work and frees TMEM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <cstring>
 
-#include "common.cuh"
+#include "tc.cuh"
 
 namespace rat {
 
+__device__ int g_attn_error;     // first device-side error of the attention kernel
+
+namespace {
+
+constexpr int BM = 128;               // query rows per tile
+constexpr int BN = 128;               // keys per block
+constexpr int DHEAD = 128;
+constexpr int NS = 2;                 // K/V pipeline stages
+constexpr int kThreads = 192;         // warp 0: TMA, warp 1: MMA, warps 2-5: softmax / epilogue
+constexpr uint32_t SUB = 16384;       // one [128 rows][64 bf16] 128B-swizzled sub-tile
+constexpr uint32_t TILE = 2 * SUB;    // one [128][128] bf16 tile
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_K = OFF_Q + TILE;
+constexpr uint32_t OFF_V = OFF_K + NS * TILE;
+constexpr uint32_t OFF_P = OFF_V + NS * TILE;
+constexpr uint32_t SMEM_BYTES = OFF_P + TILE + 1024;   // + slack for 1024-byte alignment
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t COL_S1 = 128;      // S buffers at columns 0 and 128
+constexpr uint32_t COL_O = 256;
+constexpr int kMaxDil = 4;
+constexpr float kRescaleLog2 = 8.0f;  // move the running max only when it grows by > 2^8
+
+struct Params {
+    CUtensorMap tm_q, tm_o, tm_k, tm_v;            // (d, T, B*H) bf16, box (64, 128, 1), 128B swizzle
+    CUtensorMap tm_kd[kMaxDil], tm_vd[kMaxDil];    // chunk ends of one dilation: (d, T/D, B*H)
+    int B, H, T, W, ntiles;
+    long long pos0;
+    int rope;
+    float scale_log2;
+    int head_of[kMaxHeads];   // grid y (mod H) -> head, heaviest (smallest D) first
+    int Dh[kMaxHeads];
+    int dslot[kMaxHeads];     // head -> index into tm_kd / tm_vd (-1 when D == 1)
+    double theta[64];
+};
+
+RAT_DEVICE int floordiv(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
+
+// Key blocks of one tile: nd dilated blocks (compressed indices 128*j ..) then nw window
+// blocks starting at position ws (contiguous).  Dense heads have nd = 0 and ws = 0.
+struct Plan {
+    int nd, nw, ws, D, We;
+    bool dense;
+};
+RAT_DEVICE Plan make_plan(int t0, int D, int W, int T) {
+    Plan pl;
+    pl.D = D;
+    pl.We = W > 1 ? W : 1;
+    pl.dense = D == 1;
+    const int tmax = t0 + BM - 1;
+    if (pl.dense) {
+        pl.nd = 0;
+        pl.ws = 0;
+        pl.nw = (tmax + 1 + BN - 1) / BN;
+    } else {
+        int ndk = tmax - pl.We + 1 >= D ? (tmax - pl.We + 1) / D : 0;  // chunk ends <= tmax - We
+        const int cap = T / D;
+        if (ndk > cap) ndk = cap;
+        pl.nd = (ndk + BN - 1) / BN;
+        pl.ws = t0 - pl.We + 1 > 0 ? t0 - pl.We + 1 : 0;
+        pl.nw = (tmax + 1 - pl.ws + BN - 1) / BN;
+    }
+    return pl;
+}
+
+// Columns [c_lo, c_hi] of block j that query t may attend to.
+RAT_DEVICE void block_range(const Plan &pl, int j, int t, int &c_lo, int &c_hi) {
+    if (j < pl.nd) {
+        // chunk end i = 128 j + c is attended iff i*D + D - 1 <= t - We
+        c_lo = 0;
+        c_hi = floordiv(t - pl.We - pl.D + 1, pl.D) - BN * j;
+    } else {
+        const int base = pl.ws + BN * (j - pl.nd);
+        c_hi = t - base;
+        c_lo = pl.dense ? -(1 << 30) : t - pl.We + 1 - base;
+    }
+}
+
+struct Shared {
+    uint64_t q_full, q_ready, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full, o_ready, fin;
+    uint32_t tmem;
+    volatile int abort;
+};
+
+// Bounded mbarrier wait that also gives up as soon as another role aborted.
+RAT_DEVICE bool wait_bar(Shared &sh, uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    for (;;) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (sh.abort) return false;
+        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            sh.abort = 1;
+            atomicCAS(&g_attn_error, 0, RAT_ERR_TIMEOUT);
+            return false;
+        }
+    }
+}
+
+RAT_DEVICE uint32_t swz(uint32_t row, uint32_t chunk) {   // 128B swizzle inside a sub-tile
+    return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+__global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_constant__ Params p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ Shared sh;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    const int tile = p.ntiles - 1 - (int)blockIdx.x;        // longest tiles first
+    const int t0 = tile * BM;
+    const int b = (int)blockIdx.y / p.H;
+    const int h = p.head_of[(int)blockIdx.y % p.H];
+    const int bh = b * p.H + h;
+    const Plan pl = make_plan(t0, p.Dh[h], p.W, p.T);
+    const int nb = pl.nd + pl.nw;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&sh.q_full, 1);
+        mbar_init(&sh.q_ready, 128);
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(&sh.kv_full[s], 1);
+            mbar_init(&sh.kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sh.s_full[s], 1);
+            mbar_init(&sh.s_free[s], 128);
+        }
+        mbar_init(&sh.p_full, 128);
+        mbar_init(&sh.o_ready, 1);
+        mbar_init(&sh.fin, 1);
+        sh.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tc::tmem_alloc(&sh.tmem, TMEM_COLS);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = sh.tmem;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            const CUtensorMap *mk = pl.dense ? &p.tm_k : &p.tm_kd[max(p.dslot[h], 0)];
+            const CUtensorMap *mv = pl.dense ? &p.tm_v : &p.tm_vd[max(p.dslot[h], 0)];
+            tc::prefetch_tmap(&p.tm_q);
+            tc::prefetch_tmap(mk);
+            tc::prefetch_tmap(&p.tm_k);
+            mbar_arrive_expect_tx(&sh.q_full, TILE);
+            tc::tma_load_3d(smem + OFF_Q, &p.tm_q, 0, t0, bh, &sh.q_full);
+            tc::tma_load_3d(smem + OFF_Q + SUB, &p.tm_q, 64, t0, bh, &sh.q_full);
+            int issued = 0;
+            for (int j = 0; j < nb; ++j) {
+                const int s = j % NS;
+                if (j >= NS && !wait_bar(sh, &sh.kv_empty[s], ((j / NS) - 1) & 1)) break;
+                const CUtensorMap *tk = j < pl.nd ? mk : &p.tm_k;
+                const CUtensorMap *tv = j < pl.nd ? mv : &p.tm_v;
+                const int y = j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd);
+                uint8_t *ks = smem + OFF_K + s * TILE;
+                uint8_t *vs = smem + OFF_V + s * TILE;
+                mbar_arrive_expect_tx(&sh.kv_full[s], 2 * TILE);
+                tc::tma_load_3d(ks, tk, 0, y, bh, &sh.kv_full[s]);
+                tc::tma_load_3d(ks + SUB, tk, 64, y, bh, &sh.kv_full[s]);
+                tc::tma_load_3d(vs, tv, 0, y, bh, &sh.kv_full[s]);
+                tc::tma_load_3d(vs + SUB, tv, 64, y, bh, &sh.kv_full[s]);
+                issued = j + 1;
+            }
+            if (sh.abort) {
+                // let this CTA's own loads land before its shared memory goes away
+                for (int j = max(0, issued - NS); j < issued; ++j) wait_bar(sh, &sh.kv_full[j % NS], (j / NS) & 1);
+                wait_bar(sh, &sh.q_full, 0);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t IDESC_QK = tc::idesc_bf16(BM, BN, 0);      // K^T: K-major B
+            constexpr uint32_t IDESC_PV = tc::idesc_bf16(BM, DHEAD, 1);   // V: MN-major B
+            const uint32_t sq = smem_u32(smem + OFF_Q);
+            const uint32_t sp = smem_u32(smem + OFF_P);
+            bool ok = wait_bar(sh, &sh.q_ready, 0);
+            tc::fence_after_sync();
+            for (int j = 0; ok && j <= nb; ++j) {
+                if (j < nb) {
+                    const int s = j % NS, sb = j & 1;
+                    if (!wait_bar(sh, &sh.kv_full[s], (j / NS) & 1)) break;
+                    if (j >= 2 && !wait_bar(sh, &sh.s_free[sb], ((j >> 1) - 1) & 1)) break;
+                    tc::fence_after_sync();
+                    const uint32_t sk = smem_u32(smem + OFF_K + s * TILE);
+                    for (int kk = 0; kk < DHEAD / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * SUB + (kk & 3) * 32;
+                        tc::mma_bf16_ss(tmem + sb * COL_S1, tc::smem_desc_sw128(sq + off, 16, 1024),
+                                        tc::smem_desc_sw128(sk + off, 16, 1024), IDESC_QK, kk > 0);
+                    }
+                    tc::mma_commit(&sh.s_full[sb]);
+                }
+                if (j >= 1) {
+                    const int jp = j - 1, s = jp % NS;
+                    if (!wait_bar(sh, &sh.p_full, jp & 1)) break;
+                    tc::fence_after_sync();
+                    const uint32_t sv = smem_u32(smem + OFF_V + s * TILE);
+                    for (int kk = 0; kk < BN / 16; ++kk) {
+                        // A = P[:, 16kk .. 16kk+15]  (K-major, 128B swizzle)
+                        const uint32_t aoff = (kk >> 2) * SUB + (kk & 3) * 32;
+                        // B = V[16kk .. 16kk+15, :]  (MN-major: 64-column atoms SUB apart, 8-row groups 1 KiB apart)
+                        const uint32_t boff = kk * 16 * 128;
+                        tc::mma_bf16_ss(tmem + COL_O, tc::smem_desc_sw128(sp + aoff, 16, 1024),
+                                        tc::smem_desc_sw128(sv + boff, SUB, 1024), IDESC_PV,
+                                        (jp > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(&sh.o_ready);
+                    tc::mma_commit(&sh.kv_empty[s]);
+                }
+            }
+            // all MMAs issued by this thread complete before TMEM can be released
+            tc::mma_commit(&sh.fin);
+            const uint64_t t_0 = globaltimer_ns();
+            while (!mbar_try_wait(&sh.fin, 0) && globaltimer_ns() - t_0 < kWaitLimitNs) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int q4 = warp & 3;
+        const int r = q4 * 32 + lane;           // query row in the tile == TMEM lane
+        const int t = t0 + r;
+        const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+        uint8_t *sQ = smem + OFF_Q;
+        uint8_t *sP = smem + OFF_P;
+        bool ok = wait_bar(sh, &sh.q_full, 0);
+        if (ok && p.rope) {
+            // rotate-half RoPE of this row of Q at position pos0 + t: channel c (< 64) pairs with
+            // c + 64, which sits at the same swizzled offset of the second sub-tile
+            const long long pos = p.pos0 + t;
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+                uint4 *p1 = reinterpret_cast<uint4 *>(sQ + swz(r, c));
+                uint4 *p2 = reinterpret_cast<uint4 *>(sQ + SUB + swz(r, c));
+                uint4 u1 = *p1, u2 = *p2;
+                uint32_t a1[4] = {u1.x, u1.y, u1.z, u1.w}, a2[4] = {u2.x, u2.y, u2.z, u2.w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float x1l = bf16_lo(a1[i]), x1h = bf16_hi(a1[i]);
+                    float x2l = bf16_lo(a2[i]), x2h = bf16_hi(a2[i]);
+                    float cl, sl, ch, sh2;
+                    rope_cs(pos, p.theta[c * 8 + 2 * i], cl, sl);
+                    rope_cs(pos, p.theta[c * 8 + 2 * i + 1], ch, sh2);
+                    a1[i] = pack_bf16(x1l * cl - x2l * sl, x1h * ch - x2h * sh2);
+                    a2[i] = pack_bf16(x2l * cl + x1l * sl, x2h * ch + x1h * sh2);
+                }
+                *p1 = make_uint4(a1[0], a1[1], a1[2], a1[3]);
+                *p2 = make_uint4(a2[0], a2[1], a2[2], a2[3]);
+            }
+            tc::fence_proxy_async_smem();
+        }
+        mbar_arrive(&sh.q_ready);
+
+        float m_run = -INFINITY, l_run = 0.f;
+        float sv[BN];
+        int jdone = 0;
+        for (int j = 0; ok && j < nb; ++j) {
+            const int sb = j & 1;
+            if (!wait_bar(sh, &sh.s_full[sb], (j >> 1) & 1)) { ok = false; break; }
+            tc::fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc::tmem_ld32(tl + sb * COL_S1 + 32 * c, reinterpret_cast<uint32_t *>(sv) + 32 * c);
+            tc::tmem_wait_ld();
+            tc::fence_before_sync();
+            mbar_arrive(&sh.s_free[sb]);
+
+            int c_lo, c_hi;
+            block_range(pl, j, t, c_lo, c_hi);
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                const float x = (c >= c_lo && c <= c_hi) ? sv[c] * p.scale_log2 : -INFINITY;
+                sv[c] = x;
+                mx = fmaxf(mx, x);
+            }
+            const float m_new = fmaxf(m_run, mx);
+            const bool resc = m_new > m_run + kRescaleLog2;
+            float alpha = 1.f;
+            if (resc) {
+                alpha = ex2_approx(m_run - m_new);
+                l_run *= alpha;
+                m_run = m_new;
+            }
+            const float mu = m_run == -INFINITY ? 0.f : m_run;
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < BN; ++c) {
+                const float e = ex2_approx(sv[c] - mu);
+                sv[c] = e;
+                sum += e;
+            }
+            l_run += sum;
+            if (j > 0) {
+                // PV of the previous block done: P may be overwritten, O is stable
+                if (!wait_bar(sh, &sh.o_ready, (j - 1) & 1)) { ok = false; break; }
+                if (__any_sync(0xffffffffu, resc)) {
+                    tc::fence_after_sync();
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t o[32];
+                        tc::tmem_ld32(tl + COL_O + 32 * c, o);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                        tc::tmem_st32(tl + COL_O + 32 * c, o);
+                    }
+                    tc::tmem_wait_st();
+                }
+            }
+            // P row -> bf16 -> swizzled smem (keys 0-63 in sub-tile 0, 64-127 in sub-tile 1)
+#pragma unroll
+            for (int ck = 0; ck < 16; ++ck) {
+                const float *e = sv + ck * 8;
+                *reinterpret_cast<uint4 *>(sP + (ck >> 3) * SUB + swz(r, ck & 7)) =
+                    make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
+                               pack_bf16(e[6], e[7]));
+            }
+            tc::fence_proxy_async_smem();
+            tc::fence_before_sync();
+            mbar_arrive(&sh.p_full);
+            jdone = j + 1;
+        }
+        // ---- epilogue: O / l -> bf16 -> smem (Q's tile, no longer read) -> TMA store
+        if (ok && jdone == nb && wait_bar(sh, &sh.o_ready, (nb - 1) & 1)) {
+            tc::fence_after_sync();
+            const float inv = 1.0f / l_run;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+                uint32_t o[32];
+                tc::tmem_ld32(tl + COL_O + 32 * c, o);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int k8 = 0; k8 < 4; ++k8) {
+                    const int col = 32 * c + 8 * k8;
+                    const float *f = reinterpret_cast<const float *>(o) + 8 * k8;
+                    *reinterpret_cast<uint4 *>(sQ + (col >> 6) * SUB + swz(r, (col & 63) >> 3)) =
+                        make_uint4(pack_bf16(f[0] * inv, f[1] * inv), pack_bf16(f[2] * inv, f[3] * inv),
+                                   pack_bf16(f[4] * inv, f[5] * inv), pack_bf16(f[6] * inv, f[7] * inv));
+                }
+            }
+            tc::fence_proxy_async_smem();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (r == 0) {
+                tc::tma_store_3d(&p.tm_o, sQ, 0, t0, bh);
+                tc::tma_store_3d(&p.tm_o, sQ + SUB, 64, t0, bh);
+                tc::tma_store_commit_and_wait();
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 1) tc::tmem_dealloc(tmem, TMEM_COLS);
+}
+
+// ------------------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// (d, rows, BH) bf16 view: row r of slice z at base + (z * slice_stride + r * row_stride) bytes.
+bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t BH, uint64_t row_stride,
+              uint64_t slice_stride) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)DHEAD, rows, BH};
+    cuuint64_t strides[2] = {row_stride, slice_stride};
+    cuuint32_t box[3] = {64, (cuuint32_t)BN, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
 int launch_attn_sm100(const AttnSm100Args &a, void *stream) {
-    AttnSimtParams p;
+    if (a.d != DHEAD) return RAT_ERR_UNSUPPORTED;
+    Params p;          // copied into the launch's parameter space
     std::memset(&p, 0, sizeof(p));
-    p.q = a.q; p.k = a.k; p.v = a.v; p.o = a.o;
-    p.B = a.B; p.H = a.H; p.T = a.T; p.d = a.d; p.W = a.W;
-    p.pos0 = a.pos0; p.rope = a.rope; p.scale_log2 = a.scale_log2;
-    for (int h = 0; h < a.H; ++h) p.Dh[h] = a.Dh[h];
+    const uint64_t BH = (uint64_t)a.B * a.H, T = (uint64_t)a.T;
+    const uint64_t row = DHEAD * 2, slice = T * row;
+    if (!make_map(&p.tm_q, a.q, T, BH, row, slice) || !make_map(&p.tm_o, a.o, T, BH, row, slice) ||
+        !make_map(&p.tm_k, a.k, T, BH, row, slice) || !make_map(&p.tm_v, a.v, T, BH, row, slice))
+        return RAT_ERR_CUDA;
+    // one strided map pair per distinct dilation > 1 that has at least one chunk end
+    int dvals[kMaxDil], nd = 0;
+    for (int h = 0; h < a.H; ++h) {
+        const int D = a.Dh[h];
+        p.Dh[h] = D;
+        p.dslot[h] = -1;
+        if (D == 1) continue;
+        int slot = -1;
+        for (int i = 0; i < nd; ++i)
+            if (dvals[i] == D) slot = i;
+        if (slot < 0) {
+            if (nd == kMaxDil) return RAT_ERR_UNSUPPORTED;
+            slot = nd;
+            dvals[nd++] = D;
+            const uint64_t cap = T / (uint64_t)D;
+            const uint64_t off = (uint64_t)(D - 1) * row;
+            if (cap > 0) {
+                if (!make_map(&p.tm_kd[slot], static_cast<const uint8_t *>(a.k) + off, cap, BH, (uint64_t)D * row, slice) ||
+                    !make_map(&p.tm_vd[slot], static_cast<const uint8_t *>(a.v) + off, cap, BH, (uint64_t)D * row, slice))
+                    return RAT_ERR_CUDA;
+            } else {   // no chunk end inside the sequence: the dilated stream is empty
+                p.tm_kd[slot] = p.tm_k;
+                p.tm_vd[slot] = p.tm_v;
+            }
+        }
+        p.dslot[h] = slot;
+    }
+    // heads with the smallest dilation (most keys) first
+    int order[kMaxHeads];
+    for (int h = 0; h < a.H; ++h) order[h] = h;
+    for (int i = 1; i < a.H; ++i)
+        for (int k = i; k > 0 && a.Dh[order[k]] < a.Dh[order[k - 1]]; --k) {
+            const int tmp = order[k];
+            order[k] = order[k - 1];
+            order[k - 1] = tmp;
+        }
+    for (int h = 0; h < a.H; ++h) p.head_of[h] = order[h];
+    p.B = a.B; p.H = a.H; p.T = a.T; p.W = a.W;
+    p.ntiles = (a.T + BM - 1) / BM;
+    p.pos0 = a.pos0;
+    p.rope = a.rope;
+    p.scale_log2 = a.scale_log2;
     for (int c = 0; c < 64; ++c) p.theta[c] = a.theta[c];
-    return launch_attn_simt(p, RAT_BF16, stream);
+
+    static bool attr = false;
+    if (!attr) {
+        if (cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+            return RAT_ERR_CUDA;
+        attr = true;
+    }
+    dim3 grid((unsigned)p.ntiles, (unsigned)BH);
+    attn_sm100_kernel<<<grid, kThreads, SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
+}
+
+int attn_error_word(void *stream, bool clear) {
+    int v = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return RAT_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_attn_error, sizeof(int)) != cudaSuccess) return RAT_ERR_CUDA;
+    if (v != 0 && clear) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(g_attn_error, &zero, sizeof(int)) != cudaSuccess) return RAT_ERR_CUDA;
+    }
+    return v;
 }
 
 }  // namespace rat

@@ -72,6 +72,7 @@ struct AttnSm100Args {
     double theta[64];
 };
 int launch_attn_sm100(const AttnSm100Args &a, void *stream);
+int attn_error_word(void *stream, bool clear);
 
 // ---------------------------------------------------------------------------- cache / decode
 struct CompressParams {

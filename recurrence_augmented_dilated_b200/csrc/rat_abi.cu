@@ -202,6 +202,8 @@ int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec
     return launch_attn_simt(p, dtype, stream);
 }
 
+int rat_attn_sync_status(void *stream) { return attn_error_word(stream, true); }
+
 // ------------------------------------------------------------------------------ cache
 int rat_kv_cache_bytes(const rat_kv_cache *c, size_t *dil_bytes, size_t *win_bytes,
                        size_t *state_bytes) {
