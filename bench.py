@@ -203,7 +203,7 @@ def algorithmic(w: synthetic.Workload):
 
 
 def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world: int, peaks,
-                peak_kind, with_e2e: bool):
+                peak_kind, with_e2e: bool, min_warmup_s: float = 1.0):
     import recurrence_augmented_dilated_b200 as rat
     dev = torch.device("cuda")
     x = synthetic.prefill_inputs(w, seed=w.seed + 1000 * rank)
@@ -236,7 +236,7 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
     with ClockSampler(torch.cuda.current_device()) as clk:
         t_w = time.perf_counter()
         n_w = 0
-        while n_w < warmup or time.perf_counter() - t_w < 1.0:
+        while n_w < warmup or time.perf_counter() - t_w < min_warmup_s:
             step()
             n_w += 1
             if n_w % 16 == 0:
@@ -473,6 +473,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--all", action="store_true", help="also time the other prefill workloads")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--min-warmup-s", type=float, default=1.0,
+                    help="keep warming up at least this long (clock sampling); 0 under a profiler")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -510,7 +513,8 @@ def main():
     import recurrence_augmented_dilated_b200 as rat
     rat.lib()       # fail loudly if the library is missing
 
-    pre = run_prefill(w, args.steps, args.warmup, rank, world, peaks, peak_kind, with_e2e=True)
+    pre = run_prefill(w, args.steps, args.warmup, rank, world, peaks, peak_kind,
+                      with_e2e=not args.no_e2e, min_warmup_s=args.min_warmup_s)
     kern = pre["kernels"]
     dom_name = max(kern, key=lambda n: kern[n]["ms"])
     dom = kern[dom_name]
@@ -533,7 +537,7 @@ def main():
         "roofline": roof,
         "kernels": kern,
         "clocks": pre["clocks"],
-        "e2e": pre["e2e"],
+        "e2e": pre.get("e2e"),
         "gpu_launches": pre["gpu_launches_per_step"] * args.steps,
     }
     if not args.no_decode:
@@ -543,7 +547,7 @@ def main():
         line["other_workloads"] = []
         for name in ("window_2p6b", "hybrid_7p6b", "tiny_fp32"):
             r = run_prefill(synthetic.WORKLOADS[name], max(3, args.steps // 2), args.warmup, rank,
-                            world, peaks, peak_kind, with_e2e=False)
+                            world, peaks, peak_kind, with_e2e=False, min_warmup_s=args.min_warmup_s)
             line["other_workloads"].append({"workload": name, "tokens_per_s": r["tokens_per_s"],
                                             "ms_per_step": r["ms_per_step"], "kernels": r["kernels"],
                                             "clocks": r["clocks"]})

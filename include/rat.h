@@ -147,6 +147,10 @@ RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const voi
  * attention kernel since the last call (RAT_OK if none). */
 RAT_API int rat_attn_sync_status(void *stream);
 
+/* Tuning knob of the bf16 tensor-core attention: keys per block, 64 (two CTAs per SM) or 128
+ * (one CTA per SM); 0 restores the automatic choice.  Process-wide; RAT_ERR_INVALID otherwise. */
+RAT_API int rat_set_attn_block_keys(int block_keys);
+
 /* ------------------------------------------------------------------------------------------
  * Compressed KV cache (RAT+ abstract: dilation reduces the KV cache D-fold; "RAT+ Deep Dive"
  * section 3.1: "KV cache ... compressed 64x" at D = 64).

@@ -23,7 +23,7 @@ __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
-    "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_attended_keys", "rat_status_string",
+    "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
     "Workspace",
 ]
 
@@ -85,6 +85,7 @@ def lib():
                                          _vp, _sz, _vp]
         L.rat_debug_inject_lookback_fault.argtypes = [_i64, _i64]
         L.rat_attn_sync_status.argtypes = [_vp]
+        L.rat_set_attn_block_keys.argtypes = [_i]
         L.rat_attended_keys.restype = _i64
         L.rat_attended_keys.argtypes = [_i64, _i, _i]
         _lib = L
@@ -147,6 +148,10 @@ def rat_sync_status(ws: Workspace, stream=None) -> int:
 
 def rat_attn_sync_status(stream=None) -> int:
     return int(lib().rat_attn_sync_status(_stream(stream)))
+
+
+def rat_set_attn_block_keys(block_keys: int) -> None:
+    _check("rat_set_attn_block_keys", lib().rat_set_attn_block_keys(int(block_keys)))
 
 
 def rat_recur_workspace_bytes(B, H, T, d, dtype) -> int:

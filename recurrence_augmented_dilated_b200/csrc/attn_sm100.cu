@@ -36,25 +36,34 @@ __device__ int g_attn_error;     // first device-side error of the attention ker
 namespace {
 
 constexpr int BM = 128;               // query rows per tile
-constexpr int BN = 128;               // keys per block
 constexpr int DHEAD = 128;
 constexpr int NS = 2;                 // K/V pipeline stages
 constexpr int kThreads = 192;         // warp 0: TMA, warp 1: MMA, warps 2-5: softmax / epilogue
-constexpr uint32_t SUB = 16384;       // one [128 rows][64 bf16] 128B-swizzled sub-tile
-constexpr uint32_t TILE = 2 * SUB;    // one [128][128] bf16 tile
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + TILE;
-constexpr uint32_t OFF_V = OFF_K + NS * TILE;
-constexpr uint32_t OFF_P = OFF_V + NS * TILE;
-constexpr uint32_t SMEM_BYTES = OFF_P + TILE + 1024;   // + slack for 1024-byte alignment
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_S1 = 128;      // S buffers at columns 0 and 128
-constexpr uint32_t COL_O = 256;
+constexpr uint32_t QSUB = BM * 128;   // one [128 rows][64 bf16] 128B-swizzled sub-tile of Q / O
 constexpr int kMaxDil = 4;
 constexpr float kRescaleLog2 = 8.0f;  // move the running max only when it grows by > 2^8
 
+// Shared-memory / TMEM plan for key blocks of BN keys.
+template <int BN>
+struct Cfg {
+    static constexpr uint32_t KSUB = BN * 128;          // [BN keys][64 bf16] sub-tile
+    static constexpr uint32_t KTILE = 2 * KSUB;         // one K (or V) block: two d-halves
+    static constexpr uint32_t PSUB = BM * 128;          // [128 rows][64 keys] sub-tile of P
+    static constexpr uint32_t OFF_Q = 0;
+    static constexpr uint32_t OFF_K = OFF_Q + 2 * QSUB;
+    static constexpr uint32_t OFF_V = OFF_K + NS * KTILE;
+    static constexpr uint32_t OFF_P = OFF_V + NS * KTILE;
+    static constexpr uint32_t OFF_BAR = OFF_P + (BN / 64) * PSUB;
+    static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
+    static constexpr uint32_t COL_S1 = BN;              // S buffers at columns 0 and BN
+    static constexpr uint32_t COL_O = 2 * BN;           // O: 128 columns after them
+    static constexpr uint32_t TMEM_COLS = BN == 64 ? 256 : 512;
+    static constexpr int MIN_CTAS = BN == 64 ? 2 : 1;   // CTAs resident per SM
+};
+
 struct Params {
-    CUtensorMap tm_q, tm_o, tm_k, tm_v;            // (d, T, B*H) bf16, box (64, 128, 1), 128B swizzle
+    CUtensorMap tm_q, tm_o;                        // (d, T, B*H) bf16, box (64, 128, 1), 128B swizzle
+    CUtensorMap tm_k, tm_v;                        // same tensors, box (64, BN, 1)
     CUtensorMap tm_kd[kMaxDil], tm_vd[kMaxDil];    // chunk ends of one dilation: (d, T/D, B*H)
     int B, H, T, W, ntiles;
     long long pos0;
@@ -74,6 +83,7 @@ struct Plan {
     int nd, nw, ws, D, We;
     bool dense;
 };
+template <int BN>
 RAT_DEVICE Plan make_plan(int t0, int D, int W, int T) {
     Plan pl;
     pl.D = D;
@@ -96,9 +106,10 @@ RAT_DEVICE Plan make_plan(int t0, int D, int W, int T) {
 }
 
 // Columns [c_lo, c_hi] of block j that query t may attend to.
+template <int BN>
 RAT_DEVICE void block_range(const Plan &pl, int j, int t, int &c_lo, int &c_hi) {
     if (j < pl.nd) {
-        // chunk end i = 128 j + c is attended iff i*D + D - 1 <= t - We
+        // chunk end i = BN j + c is attended iff i*D + D - 1 <= t - We
         c_lo = 0;
         c_hi = floordiv(t - pl.We - pl.D + 1, pl.D) - BN * j;
     } else {
@@ -133,10 +144,18 @@ RAT_DEVICE uint32_t swz(uint32_t row, uint32_t chunk) {   // 128B swizzle inside
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
-__global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_constant__ Params p) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ Shared sh;
+template <int BN>
+__global__ void __launch_bounds__(kThreads, Cfg<BN>::MIN_CTAS)
+attn_sm100_kernel(const __grid_constant__ Params p) {
+    using C = Cfg<BN>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    // the 128B-swizzled tiles need a 1024-byte aligned base; every thread sees the same address,
+    // so this early exit is CTA-uniform and happens before any barrier, TMA or TMEM use
+    if (smem_u32(smem) & 1023u) {
+        if (threadIdx.x == 0) atomicCAS(&g_attn_error, 0, RAT_ERR_UNSUPPORTED);
+        return;
+    }
+    Shared &sh = *reinterpret_cast<Shared *>(smem + C::OFF_BAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const int tile = p.ntiles - 1 - (int)blockIdx.x;        // longest tiles first
@@ -144,7 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
     const int b = (int)blockIdx.y / p.H;
     const int h = p.head_of[(int)blockIdx.y % p.H];
     const int bh = b * p.H + h;
-    const Plan pl = make_plan(t0, p.Dh[h], p.W, p.T);
+    const Plan pl = make_plan<BN>(t0, p.Dh[h], p.W, p.T);
     const int nb = pl.nd + pl.nw;
 
     if (threadIdx.x == 0) {
@@ -164,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
         sh.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tc::tmem_alloc(&sh.tmem, TMEM_COLS);
+    if (warp == 1) tc::tmem_alloc(&sh.tmem, C::TMEM_COLS);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -178,9 +197,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
             tc::prefetch_tmap(&p.tm_q);
             tc::prefetch_tmap(mk);
             tc::prefetch_tmap(&p.tm_k);
-            mbar_arrive_expect_tx(&sh.q_full, TILE);
-            tc::tma_load_3d(smem + OFF_Q, &p.tm_q, 0, t0, bh, &sh.q_full);
-            tc::tma_load_3d(smem + OFF_Q + SUB, &p.tm_q, 64, t0, bh, &sh.q_full);
+            mbar_arrive_expect_tx(&sh.q_full, 2 * QSUB);
+            tc::tma_load_3d(smem + C::OFF_Q, &p.tm_q, 0, t0, bh, &sh.q_full);
+            tc::tma_load_3d(smem + C::OFF_Q + QSUB, &p.tm_q, 64, t0, bh, &sh.q_full);
             int issued = 0;
             for (int j = 0; j < nb; ++j) {
                 const int s = j % NS;
@@ -188,13 +207,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
                 const CUtensorMap *tk = j < pl.nd ? mk : &p.tm_k;
                 const CUtensorMap *tv = j < pl.nd ? mv : &p.tm_v;
                 const int y = j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd);
-                uint8_t *ks = smem + OFF_K + s * TILE;
-                uint8_t *vs = smem + OFF_V + s * TILE;
-                mbar_arrive_expect_tx(&sh.kv_full[s], 2 * TILE);
+                uint8_t *ks = smem + C::OFF_K + s * C::KTILE;
+                uint8_t *vs = smem + C::OFF_V + s * C::KTILE;
+                mbar_arrive_expect_tx(&sh.kv_full[s], 2 * C::KTILE);
                 tc::tma_load_3d(ks, tk, 0, y, bh, &sh.kv_full[s]);
-                tc::tma_load_3d(ks + SUB, tk, 64, y, bh, &sh.kv_full[s]);
+                tc::tma_load_3d(ks + C::KSUB, tk, 64, y, bh, &sh.kv_full[s]);
                 tc::tma_load_3d(vs, tv, 0, y, bh, &sh.kv_full[s]);
-                tc::tma_load_3d(vs + SUB, tv, 64, y, bh, &sh.kv_full[s]);
+                tc::tma_load_3d(vs + C::KSUB, tv, 64, y, bh, &sh.kv_full[s]);
                 issued = j + 1;
             }
             if (sh.abort) {
@@ -209,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
         if (lane == 0) {
             constexpr uint32_t IDESC_QK = tc::idesc_bf16(BM, BN, 0);      // K^T: K-major B
             constexpr uint32_t IDESC_PV = tc::idesc_bf16(BM, DHEAD, 1);   // V: MN-major B
-            const uint32_t sq = smem_u32(smem + OFF_Q);
-            const uint32_t sp = smem_u32(smem + OFF_P);
+            const uint32_t sq = smem_u32(smem + C::OFF_Q);
+            const uint32_t sp = smem_u32(smem + C::OFF_P);
             bool ok = wait_bar(sh, &sh.q_ready, 0);
             tc::fence_after_sync();
             for (int j = 0; ok && j <= nb; ++j) {
@@ -219,11 +238,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
                     if (!wait_bar(sh, &sh.kv_full[s], (j / NS) & 1)) break;
                     if (j >= 2 && !wait_bar(sh, &sh.s_free[sb], ((j >> 1) - 1) & 1)) break;
                     tc::fence_after_sync();
-                    const uint32_t sk = smem_u32(smem + OFF_K + s * TILE);
+                    const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::KTILE);
                     for (int kk = 0; kk < DHEAD / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * SUB + (kk & 3) * 32;
-                        tc::mma_bf16_ss(tmem + sb * COL_S1, tc::smem_desc_sw128(sq + off, 16, 1024),
-                                        tc::smem_desc_sw128(sk + off, 16, 1024), IDESC_QK, kk > 0);
+                        // 16 channels of Q (A, K-major) and of K (B, K-major): d-half kk/4, +32 B per step
+                        const uint32_t qoff = (kk >> 2) * QSUB + (kk & 3) * 32;
+                        const uint32_t koff = (kk >> 2) * C::KSUB + (kk & 3) * 32;
+                        tc::mma_bf16_ss(tmem + sb * C::COL_S1, tc::smem_desc_sw128(sq + qoff, 16, 1024),
+                                        tc::smem_desc_sw128(sk + koff, 16, 1024), IDESC_QK, kk > 0);
                     }
                     tc::mma_commit(&sh.s_full[sb]);
                 }
@@ -231,14 +252,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
                     const int jp = j - 1, s = jp % NS;
                     if (!wait_bar(sh, &sh.p_full, jp & 1)) break;
                     tc::fence_after_sync();
-                    const uint32_t sv = smem_u32(smem + OFF_V + s * TILE);
+                    const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KTILE);
                     for (int kk = 0; kk < BN / 16; ++kk) {
-                        // A = P[:, 16kk .. 16kk+15]  (K-major, 128B swizzle)
-                        const uint32_t aoff = (kk >> 2) * SUB + (kk & 3) * 32;
-                        // B = V[16kk .. 16kk+15, :]  (MN-major: 64-column atoms SUB apart, 8-row groups 1 KiB apart)
+                        // A = P[:, 16kk .. 16kk+15]  (K-major, 128B swizzle, 64-key sub-tiles)
+                        const uint32_t aoff = (kk >> 2) * C::PSUB + (kk & 3) * 32;
+                        // B = V[16kk .. 16kk+15, :]  (MN-major: the two 64-channel atoms KSUB apart,
+                        // 8-key groups 1 KiB apart)
                         const uint32_t boff = kk * 16 * 128;
-                        tc::mma_bf16_ss(tmem + COL_O, tc::smem_desc_sw128(sp + aoff, 16, 1024),
-                                        tc::smem_desc_sw128(sv + boff, SUB, 1024), IDESC_PV,
+                        tc::mma_bf16_ss(tmem + C::COL_O, tc::smem_desc_sw128(sp + aoff, 16, 1024),
+                                        tc::smem_desc_sw128(sv + boff, C::KSUB, 1024), IDESC_PV,
                                         (jp > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit(&sh.o_ready);
@@ -258,9 +280,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
         const int r = q4 * 32 + lane;           // query row in the tile == TMEM lane
         const int t = t0 + r;
         const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-        uint8_t *sQ = smem + OFF_Q;
-        uint8_t *sP = smem + OFF_P;
-        bool ok = wait_bar(sh, &sh.q_full, 0);
+        uint8_t *sQ = smem + C::OFF_Q;
+        uint8_t *sP = smem + C::OFF_P;
+        // waits are made warp-uniform: tcgen05.ld/st below are warp-collective
+        bool ok = __all_sync(0xffffffffu, wait_bar(sh, &sh.q_full, 0));
         if (ok && p.rope) {
             // rotate-half RoPE of this row of Q at position pos0 + t: channel c (< 64) pairs with
             // c + 64, which sits at the same swizzled offset of the second sub-tile
@@ -268,7 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
 #pragma unroll 1
             for (int c = 0; c < 8; ++c) {
                 uint4 *p1 = reinterpret_cast<uint4 *>(sQ + swz(r, c));
-                uint4 *p2 = reinterpret_cast<uint4 *>(sQ + SUB + swz(r, c));
+                uint4 *p2 = reinterpret_cast<uint4 *>(sQ + QSUB + swz(r, c));
                 uint4 u1 = *p1, u2 = *p2;
                 uint32_t a1[4] = {u1.x, u1.y, u1.z, u1.w}, a2[4] = {u2.x, u2.y, u2.z, u2.w};
 #pragma unroll
@@ -293,16 +316,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
         int jdone = 0;
         for (int j = 0; ok && j < nb; ++j) {
             const int sb = j & 1;
-            if (!wait_bar(sh, &sh.s_full[sb], (j >> 1) & 1)) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.s_full[sb], (j >> 1) & 1))) { ok = false; break; }
             tc::fence_after_sync();
 #pragma unroll
-            for (int c = 0; c < 4; ++c) tc::tmem_ld32(tl + sb * COL_S1 + 32 * c, reinterpret_cast<uint32_t *>(sv) + 32 * c);
+            for (int c = 0; c < BN / 32; ++c)
+                tc::tmem_ld32(tl + sb * C::COL_S1 + 32 * c, reinterpret_cast<uint32_t *>(sv) + 32 * c);
             tc::tmem_wait_ld();
             tc::fence_before_sync();
             mbar_arrive(&sh.s_free[sb]);
 
             int c_lo, c_hi;
-            block_range(pl, j, t, c_lo, c_hi);
+            block_range<BN>(pl, j, t, c_lo, c_hi);
             float mx = -INFINITY;
 #pragma unroll
             for (int c = 0; c < BN; ++c) {
@@ -329,26 +353,26 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
             l_run += sum;
             if (j > 0) {
                 // PV of the previous block done: P may be overwritten, O is stable
-                if (!wait_bar(sh, &sh.o_ready, (j - 1) & 1)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready, (j - 1) & 1))) { ok = false; break; }
                 if (__any_sync(0xffffffffu, resc)) {
                     tc::fence_after_sync();
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
-                        tc::tmem_ld32(tl + COL_O + 32 * c, o);
+                        tc::tmem_ld32(tl + C::COL_O + 32 * c, o);
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tc::tmem_st32(tl + COL_O + 32 * c, o);
+                        tc::tmem_st32(tl + C::COL_O + 32 * c, o);
                     }
                     tc::tmem_wait_st();
                 }
             }
-            // P row -> bf16 -> swizzled smem (keys 0-63 in sub-tile 0, 64-127 in sub-tile 1)
+            // P row -> bf16 -> swizzled smem (64-key sub-tiles)
 #pragma unroll
-            for (int ck = 0; ck < 16; ++ck) {
+            for (int ck = 0; ck < BN / 8; ++ck) {
                 const float *e = sv + ck * 8;
-                *reinterpret_cast<uint4 *>(sP + (ck >> 3) * SUB + swz(r, ck & 7)) =
+                *reinterpret_cast<uint4 *>(sP + (ck >> 3) * C::PSUB + swz(r, ck & 7)) =
                     make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
                                pack_bf16(e[6], e[7]));
             }
@@ -358,37 +382,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_sm100_kernel(const __grid_co
             jdone = j + 1;
         }
         // ---- epilogue: O / l -> bf16 -> smem (Q's tile, no longer read) -> TMA store
-        if (ok && jdone == nb && wait_bar(sh, &sh.o_ready, (nb - 1) & 1)) {
+        bool have_o = ok && jdone == nb;
+        if (have_o) have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready, (nb - 1) & 1));
+        if (have_o) {
             tc::fence_after_sync();
             const float inv = 1.0f / l_run;
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
-                tc::tmem_ld32(tl + COL_O + 32 * c, o);
+                tc::tmem_ld32(tl + C::COL_O + 32 * c, o);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int k8 = 0; k8 < 4; ++k8) {
                     const int col = 32 * c + 8 * k8;
                     const float *f = reinterpret_cast<const float *>(o) + 8 * k8;
-                    *reinterpret_cast<uint4 *>(sQ + (col >> 6) * SUB + swz(r, (col & 63) >> 3)) =
+                    *reinterpret_cast<uint4 *>(sQ + (col >> 6) * QSUB + swz(r, (col & 63) >> 3)) =
                         make_uint4(pack_bf16(f[0] * inv, f[1] * inv), pack_bf16(f[2] * inv, f[3] * inv),
                                    pack_bf16(f[4] * inv, f[5] * inv), pack_bf16(f[6] * inv, f[7] * inv));
                 }
             }
             tc::fence_proxy_async_smem();
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (r == 0) {
-                tc::tma_store_3d(&p.tm_o, sQ, 0, t0, bh);
-                tc::tma_store_3d(&p.tm_o, sQ + SUB, 64, t0, bh);
-                tc::tma_store_commit_and_wait();
-            }
+        }
+        // all 128 epilogue threads reach this barrier on every path; the store is issued only if
+        // no role aborted (an abort has already recorded RAT_ERR_TIMEOUT)
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (r == 0 && have_o && !sh.abort) {
+            tc::tma_store_3d(&p.tm_o, sQ, 0, t0, bh);
+            tc::tma_store_3d(&p.tm_o, sQ + QSUB, 64, t0, bh);
+            tc::tma_store_commit_and_wait();
         }
     }
 
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 1) tc::tmem_dealloc(tmem, TMEM_COLS);
+    if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 // ------------------------------------------------------------------------------ host side
@@ -404,32 +432,32 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// (d, rows, BH) bf16 view: row r of slice z at base + (z * slice_stride + r * row_stride) bytes.
+// (d, rows, BH) bf16 view: row r of slice z at base + (z * slice_stride + r * row_stride) bytes;
+// box (64 channels, box_rows, 1), 128-byte swizzle, zero fill outside.
 bool make_map(CUtensorMap *m, const void *base, uint64_t rows, uint64_t BH, uint64_t row_stride,
-              uint64_t slice_stride) {
+              uint64_t slice_stride, uint32_t box_rows) {
     auto fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[3] = {(cuuint64_t)DHEAD, rows, BH};
     cuuint64_t strides[2] = {row_stride, slice_stride};
-    cuuint32_t box[3] = {64, (cuuint32_t)BN, 1};
+    cuuint32_t box[3] = {64, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-}  // namespace
-
-int launch_attn_sm100(const AttnSm100Args &a, void *stream) {
-    if (a.d != DHEAD) return RAT_ERR_UNSUPPORTED;
+template <int BN>
+int launch_bn(const AttnSm100Args &a, void *stream) {
+    using C = Cfg<BN>;
     Params p;          // copied into the launch's parameter space
     std::memset(&p, 0, sizeof(p));
     const uint64_t BH = (uint64_t)a.B * a.H, T = (uint64_t)a.T;
     const uint64_t row = DHEAD * 2, slice = T * row;
-    if (!make_map(&p.tm_q, a.q, T, BH, row, slice) || !make_map(&p.tm_o, a.o, T, BH, row, slice) ||
-        !make_map(&p.tm_k, a.k, T, BH, row, slice) || !make_map(&p.tm_v, a.v, T, BH, row, slice))
+    if (!make_map(&p.tm_q, a.q, T, BH, row, slice, BM) || !make_map(&p.tm_o, a.o, T, BH, row, slice, BM) ||
+        !make_map(&p.tm_k, a.k, T, BH, row, slice, BN) || !make_map(&p.tm_v, a.v, T, BH, row, slice, BN))
         return RAT_ERR_CUDA;
-    // one strided map pair per distinct dilation > 1 that has at least one chunk end
+    // one strided map pair per distinct dilation > 1
     int dvals[kMaxDil], nd = 0;
     for (int h = 0; h < a.H; ++h) {
         const int D = a.Dh[h];
@@ -446,8 +474,8 @@ int launch_attn_sm100(const AttnSm100Args &a, void *stream) {
             const uint64_t cap = T / (uint64_t)D;
             const uint64_t off = (uint64_t)(D - 1) * row;
             if (cap > 0) {
-                if (!make_map(&p.tm_kd[slot], static_cast<const uint8_t *>(a.k) + off, cap, BH, (uint64_t)D * row, slice) ||
-                    !make_map(&p.tm_vd[slot], static_cast<const uint8_t *>(a.v) + off, cap, BH, (uint64_t)D * row, slice))
+                if (!make_map(&p.tm_kd[slot], static_cast<const uint8_t *>(a.k) + off, cap, BH, (uint64_t)D * row, slice, BN) ||
+                    !make_map(&p.tm_vd[slot], static_cast<const uint8_t *>(a.v) + off, cap, BH, (uint64_t)D * row, slice, BN))
                     return RAT_ERR_CUDA;
             } else {   // no chunk end inside the sequence: the dilated stream is empty
                 p.tm_kd[slot] = p.tm_k;
@@ -475,13 +503,24 @@ int launch_attn_sm100(const AttnSm100Args &a, void *stream) {
 
     static bool attr = false;
     if (!attr) {
-        if (cudaFuncSetAttribute(attn_sm100_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) != cudaSuccess)
+        if (cudaFuncSetAttribute(attn_sm100_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 C::SMEM_BYTES) != cudaSuccess)
             return RAT_ERR_CUDA;
         attr = true;
     }
     dim3 grid((unsigned)p.ntiles, (unsigned)BH);
-    attn_sm100_kernel<<<grid, kThreads, SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(p);
+    attn_sm100_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
+}
+
+}  // namespace
+
+int g_attn_block_keys = 0;   // 0: automatic; 64 or 128 forces the key-block width
+
+int launch_attn_sm100(const AttnSm100Args &a, void *stream) {
+    if (a.d != DHEAD) return RAT_ERR_UNSUPPORTED;
+    const int bn = g_attn_block_keys ? g_attn_block_keys : 64;
+    return bn == 64 ? launch_bn<64>(a, stream) : launch_bn<128>(a, stream);
 }
 
 int attn_error_word(void *stream, bool clear) {

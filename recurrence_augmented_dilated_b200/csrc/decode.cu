@@ -28,11 +28,6 @@ RAT_DEVICE void load8(const void *p, float *x) {      // 8 bf16 -> float
     x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
     x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
 }
-RAT_DEVICE void load8_cg(const void *p, float *x) {   // same, bypassing L1 (written this launch)
-    const uint4 u = __ldcg(reinterpret_cast<const uint4 *>(p));
-    x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
-    x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
-}
 RAT_DEVICE uint4 pack8(const float *x) {
     return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
                       pack_bf16(x[6], x[7]));
@@ -84,15 +79,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j] = 0.f;
 
-    // keys of this split: each (warp, group) takes every (kWarps*GPW)-th key, 2 at a time
+    // keys of this split: lane set s = warp*GPW + grp takes keys k_lo + s + m*kLanesets, two at a
+    // time.  The loop runs on the warp's first key so every lane of a warp iterates the same
+    // number of times (the dot-product shuffles below need all 32 lanes).
     constexpr int kLanesets = kWarps * GPW;
     const int set = warp * GPW + grp;
-    for (long long base = k_lo + set; base < k_hi; base += 2 * kLanesets) {
+    for (long long base = k_lo + warp * GPW; base < k_hi; base += 2 * kLanesets) {
         float kx[2][8], vx[2][8];
         bool have[2];
 #pragma unroll
         for (int u = 0; u < 2; ++u) {
-            const long long idx = base + (long long)u * kLanesets;
+            const long long idx = base + grp + (long long)u * kLanesets;
             have[u] = idx < k_hi;
             // lanes of a warp may disagree on `have`; loads are predicated, shuffles are not
             if (have[u]) {

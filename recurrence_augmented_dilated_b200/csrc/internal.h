@@ -73,6 +73,7 @@ struct AttnSm100Args {
 };
 int launch_attn_sm100(const AttnSm100Args &a, void *stream);
 int attn_error_word(void *stream, bool clear);
+extern int g_attn_block_keys;
 
 // ---------------------------------------------------------------------------- cache / decode
 struct CompressParams {

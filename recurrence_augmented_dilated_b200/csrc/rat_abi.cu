@@ -204,6 +204,12 @@ int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec
 
 int rat_attn_sync_status(void *stream) { return attn_error_word(stream, true); }
 
+int rat_set_attn_block_keys(int block_keys) {
+    if (block_keys != 0 && block_keys != 64 && block_keys != 128) return RAT_ERR_INVALID;
+    g_attn_block_keys = block_keys;
+    return RAT_OK;
+}
+
 // ------------------------------------------------------------------------------ cache
 int rat_kv_cache_bytes(const rat_kv_cache *c, size_t *dil_bytes, size_t *win_bytes,
                        size_t *state_bytes) {

@@ -15,13 +15,17 @@
 //              publishes its aggregate (A, Bk, Bv) as soon as it has loaded, then walks back
 //              over its predecessors' aggregates until it meets an inclusive state.
 //
-// Data movement: each CTA owns one chunk of TC rows x d channels of one (b, h), i.e. three
-// contiguous byte ranges (a, k, v), fetched with three bulk copies (cp.async.bulk) into shared
-// memory; outputs are written with 16-byte stores, 16 lanes covering one 256-byte row.  The
-// HBM stream is therefore 3 reads + 2 writes per element, the algorithmic minimum.
+// Data movement: a chunk is TC rows x d channels of one (b, h), i.e. three contiguous byte
+// ranges (a, k, v), fetched with three bulk copies (cp.async.bulk) into shared memory.  The
+// kernel is persistent (one CTA per SM) and double-buffered: while a CTA computes one chunk,
+// the bulk copies of its next chunk are in flight.  Outputs are written with 16-byte stores,
+// 16 lanes covering one 256-byte row.  The HBM stream is 3 reads + 2 writes per element, the
+// algorithmic minimum.  The gates of pass 1 stay in registers for pass 2, so each element
+// costs one exp2 and one reciprocal on the special-function unit.
 //
-// Chunk order comes from an atomic ticket (chunk-major: all (b, h) advance together), so every
-// predecessor a CTA waits for has already started; each wait is bounded by kWaitLimitNs and
+// Chunk order comes from an atomic ticket (chunk-major: all (b, h) advance together); a CTA
+// takes its next ticket before finishing the current chunk, and every predecessor it waits
+// for was taken earlier by a resident CTA; each wait is bounded by the caller's limit and
 // records RAT_ERR_TIMEOUT instead of hanging.  Flags carry a launch epoch, so the workspace is
 // never cleared between launches: the last CTA of a launch resets the tickets and bumps the
 // epoch.
@@ -42,7 +46,8 @@ struct ScanCfg {
     static constexpr int TC = SEGS * R;           // rows per chunk
     static constexpr int ROWB = DH * EB;          // bytes per row
     static constexpr int TILEB = TC * ROWB;       // bytes per tensor per chunk (32 KiB)
-    static constexpr int SMEM = 3 * TILEB + NW * 3 * DH * 4;
+    static constexpr int STAGEB = 3 * TILEB;      // a, k, v of one chunk
+    static constexpr int SMEM = 2 * STAGEB + NW * 3 * DH * 4;   // two stages + warp carries
 };
 
 // 16 bytes of a row -> VEC floats.
@@ -93,242 +98,265 @@ RAT_DEVICE uint32_t wait_flag(const uint32_t *f, uint32_t epoch, uint64_t limit_
 }
 
 template <typename E, int DH>
-__global__ void __launch_bounds__(256, 2) recur_kernel(const __grid_constant__ RecurParams p) {
+__global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ RecurParams p) {
     using C = ScanCfg<E, DH>;
     constexpr int VEC = C::VEC, LPR = C::LPR, R = C::R;
     extern __shared__ __align__(128) uint8_t smem[];
-    uint8_t *sa = smem, *sk = smem + C::TILEB, *sv = smem + 2 * C::TILEB;
-    float *sw = reinterpret_cast<float *>(smem + 3 * C::TILEB);   // [NW][3][DH]
-    __shared__ uint64_t bar;
-    __shared__ uint32_t s_ticket, s_epoch;
+    float *sw = reinterpret_cast<float *>(smem + 2 * C::STAGEB);   // [NW][3][DH]
+    __shared__ uint64_t bar[2];
+    __shared__ int s_ticket[2];
+    __shared__ uint32_t s_epoch;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int seg = tid / LPR, cl = tid % LPR, segw = lane / LPR;
     WsHeader *hdr = p.hdr;
+    const int total = p.BH * p.nchunks;
+
+    // issue the three bulk copies of chunk `ticket` into stage `st` (thread 0 only)
+    auto load_chunk = [&](int ticket, int st) {
+        const int c = ticket / p.BH, bh = ticket % p.BH;
+        const int rows = min(C::TC, p.T - c * C::TC);
+        const size_t row0 = (size_t)bh * p.T + (size_t)c * C::TC;
+        const uint32_t bytes = (uint32_t)rows * C::ROWB;
+        uint8_t *s = smem + st * C::STAGEB;
+        mbar_arrive_expect_tx(&bar[st], 3 * bytes);
+        bulk_g2s(s, static_cast<const uint8_t *>(p.a) + row0 * C::ROWB, bytes, &bar[st]);
+        bulk_g2s(s + C::TILEB, static_cast<const uint8_t *>(p.k) + row0 * C::ROWB, bytes, &bar[st]);
+        bulk_g2s(s + 2 * C::TILEB, static_cast<const uint8_t *>(p.v) + row0 * C::ROWB, bytes, &bar[st]);
+    };
 
     if (tid == 0) {
         s_epoch = *reinterpret_cast<volatile uint32_t *>(&hdr->epoch);
-        s_ticket = atomicAdd(&hdr->ticket, 1u);
-        mbar_init(&bar, 1);
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
         fence_mbar_init();
+        const int t0k = (int)atomicAdd(&hdr->ticket, 1u);
+        s_ticket[0] = t0k;
+        if (t0k < total) load_chunk(t0k, 0);
     }
     __syncthreads();
     const uint32_t epoch_raw = s_epoch, epoch = epoch_raw & 0x3fffffffu;
-    const int ticket = (int)s_ticket;
-    const int c = ticket / p.BH, bh = ticket % p.BH;     // chunk-major order
-    const int t0 = c * C::TC;
-    const int rows = min(C::TC, p.T - t0);
-    const size_t chunk_id = (size_t)bh * p.nchunks + c;
-    const size_t row0 = (size_t)bh * p.T + t0;
-    const bool publish = c != p.fault_chunk;            // false only under the test hook
 
-    if (tid == 0) {
-        const uint32_t bytes = (uint32_t)rows * C::ROWB;
-        mbar_arrive_expect_tx(&bar, 3 * bytes);
-        bulk_g2s(sa, static_cast<const uint8_t *>(p.a) + row0 * C::ROWB, bytes, &bar);
-        bulk_g2s(sk, static_cast<const uint8_t *>(p.k) + row0 * C::ROWB, bytes, &bar);
-        bulk_g2s(sv, static_cast<const uint8_t *>(p.v) + row0 * C::ROWB, bytes, &bar);
-    }
-    mbar_wait_bounded(&bar, 0, hdr, 0x100u);
+    for (int it = 0;; ++it) {
+        const int st = it & 1;
+        const int ticket = s_ticket[st];
+        if (ticket >= total) break;
+        // prefetch the next chunk into the other stage (its previous contents were consumed
+        // by the previous iteration, which ended with a block-wide barrier)
+        if (tid == 0) {
+            const int nt = (int)atomicAdd(&hdr->ticket, 1u);
+            s_ticket[st ^ 1] = nt;
+            if (nt < total) load_chunk(nt, st ^ 1);
+        }
+        const int c = ticket / p.BH, bh = ticket % p.BH;     // chunk-major order
+        const int t0 = c * C::TC;
+        const int rows = min(C::TC, p.T - t0);
+        const size_t chunk_id = (size_t)bh * p.nchunks + c;
+        const size_t row0 = (size_t)bh * p.T + t0;
+        const bool publish = c != p.fault_chunk;            // false only under the test hook
+        const uint8_t *sa = smem + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
+        mbar_wait_bounded(&bar[st], (it >> 1) & 1, hdr, 0x100u);
 
-    // ---- pass 1: aggregate of this lane's R rows, per channel
-    float A[VEC], Bk[VEC], Bv[VEC];
+        // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate
+        float G[R][VEC], OG[R][VEC];
+        float A[VEC], Bk[VEC], Bv[VEC];
 #pragma unroll
-    for (int i = 0; i < VEC; ++i) { A[i] = 1.f; Bk[i] = 0.f; Bv[i] = 0.f; }
+        for (int j = 0; j < VEC; ++j) { A[j] = 1.f; Bk[j] = 0.f; Bv[j] = 0.f; }
 #pragma unroll
-    for (int i = 0; i < R; ++i) {
-        const int r = seg * R + i;
-        if (r < rows) {
-            const int off = r * C::ROWB + cl * 16;
+        for (int i = 0; i < R; ++i) {
+            const int r = seg * R + i;
             float xa[VEC], xk[VEC], xv[VEC];
-            Vec<E>::load(sa + off, xa);
-            Vec<E>::load(sk + off, xk);
-            Vec<E>::load(sv + off, xv);
+            if (r < rows) {
+                const int off = r * C::ROWB + cl * 16;
+                Vec<E>::load(sa + off, xa);
+                Vec<E>::load(sk + off, xk);
+                Vec<E>::load(sv + off, xv);
+            } else {        // rows past the end: identity step (g = 1, 1-g = 0)
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) { xa[j] = 1e30f; xk[j] = 0.f; xv[j] = 0.f; }
+            }
 #pragma unroll
             for (int j = 0; j < VEC; ++j) {
-                float g, omg;
-                forget_gate(xa[j], g, omg);
-                A[j] *= g;
-                Bk[j] = fmaf(g, Bk[j], omg * xk[j]);
-                Bv[j] = fmaf(g, Bv[j], omg * xv[j]);
+                forget_gate(xa[j], G[i][j], OG[i][j]);
+                A[j] *= G[i][j];
+                Bk[j] = fmaf(G[i][j], Bk[j], OG[i][j] * xk[j]);
+                Bv[j] = fmaf(G[i][j], Bv[j], OG[i][j] * xv[j]);
             }
         }
-    }
-    // ---- inclusive scan over the segments of this warp (shuffles)
+        // ---- inclusive scan over the segments of this warp (shuffles)
 #pragma unroll
-    for (int sh = 1; sh < C::SPW; sh <<= 1) {
+        for (int sh = 1; sh < C::SPW; sh <<= 1) {
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) {
+                const float pA = __shfl_up_sync(0xffffffffu, A[j], sh * LPR);
+                const float pK = __shfl_up_sync(0xffffffffu, Bk[j], sh * LPR);
+                const float pV = __shfl_up_sync(0xffffffffu, Bv[j], sh * LPR);
+                if (segw >= sh) {
+                    Bk[j] = fmaf(A[j], pK, Bk[j]);
+                    Bv[j] = fmaf(A[j], pV, Bv[j]);
+                    A[j] *= pA;
+                }
+            }
+        }
+        // exclusive prefix of this segment inside its warp
+        float eA[VEC], eK[VEC], eV[VEC];
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
-            float pA = __shfl_up_sync(0xffffffffu, A[j], sh * LPR);
-            float pK = __shfl_up_sync(0xffffffffu, Bk[j], sh * LPR);
-            float pV = __shfl_up_sync(0xffffffffu, Bv[j], sh * LPR);
-            if (segw >= sh) {
-                Bk[j] = fmaf(A[j], pK, Bk[j]);
-                Bv[j] = fmaf(A[j], pV, Bv[j]);
-                A[j] *= pA;
+            eA[j] = __shfl_up_sync(0xffffffffu, A[j], LPR);
+            eK[j] = __shfl_up_sync(0xffffffffu, Bk[j], LPR);
+            eV[j] = __shfl_up_sync(0xffffffffu, Bv[j], LPR);
+            if (segw == 0) { eA[j] = 1.f; eK[j] = 0.f; eV[j] = 0.f; }
+        }
+        if (segw == C::SPW - 1) {
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) {
+                const int ch = cl * VEC + j;
+                sw[(warp * 3 + 0) * DH + ch] = A[j];
+                sw[(warp * 3 + 1) * DH + ch] = Bk[j];
+                sw[(warp * 3 + 2) * DH + ch] = Bv[j];
             }
         }
-    }
-    // exclusive prefix of this segment inside its warp
-    float eA[VEC], eK[VEC], eV[VEC];
+        __syncthreads();
+
+        // ---- chunk aggregate, look-back and carries: one thread per channel
+        if (tid < DH) {
+            const int ch = tid;
+            float cA = 1.f, cK = 0.f, cV = 0.f;
 #pragma unroll
-    for (int j = 0; j < VEC; ++j) {
-        eA[j] = __shfl_up_sync(0xffffffffu, A[j], LPR);
-        eK[j] = __shfl_up_sync(0xffffffffu, Bk[j], LPR);
-        eV[j] = __shfl_up_sync(0xffffffffu, Bv[j], LPR);
-        if (segw == 0) { eA[j] = 1.f; eK[j] = 0.f; eV[j] = 0.f; }
-    }
-    if (segw == C::SPW - 1) {
+            for (int w = 0; w < C::NW; ++w) {
+                const float a = sw[(w * 3 + 0) * DH + ch];
+                cK = fmaf(a, cK, sw[(w * 3 + 1) * DH + ch]);
+                cV = fmaf(a, cV, sw[(w * 3 + 2) * DH + ch]);
+                cA *= a;
+            }
+            float *agg = p.agg + chunk_id * 3 * DH;
+            float *pre = p.pre + chunk_id * 2 * DH;
+            if (c > 0) {
+                agg[ch] = cA;
+                agg[DH + ch] = cK;
+                agg[2 * DH + ch] = cV;
+                __threadfence();
+                asm volatile("bar.sync 1, %0;" :: "r"(DH) : "memory");
+                if (tid == 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 1u);
+            }
+            float Hk = 0.f, Hv = 0.f;     // state entering this chunk
+            if (c == 0) {
+                if (p.h0k) Hk = p.h0k[(size_t)bh * DH + ch];
+                if (p.h0v) Hv = p.h0v[(size_t)bh * DH + ch];
+            } else {
+                float xA = 1.f, xK = 0.f, xV = 0.f;   // composition of chunks j+1 .. c-1
+                for (int j = c - 1; j >= 0; --j) {
+                    const size_t jid = (size_t)bh * p.nchunks + j;
+                    const uint32_t s = wait_flag(p.flags + jid, epoch, p.wait_ns, hdr, 0x200u);
+                    if (s == 2u) {
+                        const float *pj = p.pre + jid * 2 * DH;
+                        Hk = fmaf(xA, __ldcg(pj + ch), xK);
+                        Hv = fmaf(xA, __ldcg(pj + DH + ch), xV);
+                        break;
+                    }
+                    if (s == 0u) break;          // timed out: error recorded, carry zero
+                    const float *aj = p.agg + jid * 3 * DH;
+                    const float a = __ldcg(aj + ch);
+                    xK = fmaf(xA, __ldcg(aj + DH + ch), xK);
+                    xV = fmaf(xA, __ldcg(aj + 2 * DH + ch), xV);
+                    xA *= a;
+                }
+            }
+            const float outK = fmaf(cA, Hk, cK), outV = fmaf(cA, Hv, cV);
+            pre[ch] = outK;
+            pre[DH + ch] = outV;
+            if (c == p.nchunks - 1) {
+                if (p.hTk) p.hTk[(size_t)bh * DH + ch] = outK;
+                if (p.hTv) p.hTv[(size_t)bh * DH + ch] = outV;
+            }
+            __threadfence();
+            // carries entering each warp, written over that warp's aggregate
+            float hK = Hk, hV = Hv;
+#pragma unroll
+            for (int w = 0; w < C::NW; ++w) {
+                const float a = sw[(w * 3 + 0) * DH + ch];
+                const float bk = sw[(w * 3 + 1) * DH + ch];
+                const float bv = sw[(w * 3 + 2) * DH + ch];
+                sw[(w * 3 + 0) * DH + ch] = hK;
+                sw[(w * 3 + 1) * DH + ch] = hV;
+                hK = fmaf(a, hK, bk);
+                hV = fmaf(a, hV, bv);
+            }
+            asm volatile("bar.sync 1, %0;" :: "r"(DH) : "memory");
+            if (tid == 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 2u);
+        }
+        __syncthreads();
+
+        // ---- pass 2: rerun the recurrence from the carry with the kept gates; write k~
+        // (optionally rotated) and v~
+        float hk[VEC], hv[VEC];
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
             const int ch = cl * VEC + j;
-            sw[(warp * 3 + 0) * DH + ch] = A[j];
-            sw[(warp * 3 + 1) * DH + ch] = Bk[j];
-            sw[(warp * 3 + 2) * DH + ch] = Bv[j];
+            const float wk = sw[(warp * 3 + 0) * DH + ch], wv = sw[(warp * 3 + 1) * DH + ch];
+            hk[j] = fmaf(eA[j], wk, eK[j]);
+            hv[j] = fmaf(eA[j], wv, eV[j]);
         }
-    }
-    __syncthreads();
-
-    // ---- chunk aggregate, look-back and carries: one thread per channel
-    if (tid < DH) {
-        const int ch = tid;
-        float cA = 1.f, cK = 0.f, cV = 0.f;
-#pragma unroll
-        for (int w = 0; w < C::NW; ++w) {
-            const float a = sw[(w * 3 + 0) * DH + ch];
-            cK = fmaf(a, cK, sw[(w * 3 + 1) * DH + ch]);
-            cV = fmaf(a, cV, sw[(w * 3 + 2) * DH + ch]);
-            cA *= a;
-        }
-        float *agg = p.agg + chunk_id * 3 * DH;
-        float *pre = p.pre + chunk_id * 2 * DH;
-        if (c > 0) {
-            agg[ch] = cA;
-            agg[DH + ch] = cK;
-            agg[2 * DH + ch] = cV;
-            __threadfence();
-            asm volatile("bar.sync 1, %0;" :: "r"(DH) : "memory");
-            if (tid == 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 1u);
-        }
-        float Hk = 0.f, Hv = 0.f;     // state entering this chunk
-        if (c == 0) {
-            if (p.h0k) Hk = p.h0k[(size_t)bh * DH + ch];
-            if (p.h0v) Hv = p.h0v[(size_t)bh * DH + ch];
-        } else {
-            float xA = 1.f, xK = 0.f, xV = 0.f;   // composition of chunks j+1 .. c-1
-            for (int j = c - 1; j >= 0; --j) {
-                const size_t jid = (size_t)bh * p.nchunks + j;
-                const uint32_t st = wait_flag(p.flags + jid, epoch, p.wait_ns, hdr, 0x200u);
-                if (st == 2u) {
-                    const float *pj = p.pre + jid * 2 * DH;
-                    Hk = fmaf(xA, __ldcg(pj + ch), xK);
-                    Hv = fmaf(xA, __ldcg(pj + DH + ch), xV);
-                    break;
-                }
-                if (st == 0u) break;          // timed out: error recorded, carry zero
-                const float *aj = p.agg + jid * 3 * DH;
-                const float a = __ldcg(aj + ch);
-                xK = fmaf(xA, __ldcg(aj + DH + ch), xK);
-                xV = fmaf(xA, __ldcg(aj + 2 * DH + ch), xV);
-                xA *= a;
-            }
-        }
-        const float outK = fmaf(cA, Hk, cK), outV = fmaf(cA, Hv, cV);
-        pre[ch] = outK;
-        pre[DH + ch] = outV;
-        if (c == p.nchunks - 1) {
-            if (p.hTk) p.hTk[(size_t)bh * DH + ch] = outK;
-            if (p.hTv) p.hTv[(size_t)bh * DH + ch] = outV;
-        }
-        __threadfence();
-        // carries entering each warp, written over that warp's aggregate
-        float hK = Hk, hV = Hv;
-#pragma unroll
-        for (int w = 0; w < C::NW; ++w) {
-            const float a = sw[(w * 3 + 0) * DH + ch];
-            const float bk = sw[(w * 3 + 1) * DH + ch];
-            const float bv = sw[(w * 3 + 2) * DH + ch];
-            sw[(w * 3 + 0) * DH + ch] = hK;
-            sw[(w * 3 + 1) * DH + ch] = hV;
-            hK = fmaf(a, hK, bk);
-            hV = fmaf(a, hV, bv);
-        }
-        asm volatile("bar.sync 1, %0;" :: "r"(DH) : "memory");
-        if (tid == 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 2u);
-    }
-    __syncthreads();
-
-    // ---- pass 2: rerun the recurrence from the carry and write k~ (optionally rotated), v~
-    float hk[VEC], hv[VEC];
-#pragma unroll
-    for (int j = 0; j < VEC; ++j) {
-        const int ch = cl * VEC + j;
-        const float wk = sw[(warp * 3 + 0) * DH + ch], wv = sw[(warp * 3 + 1) * DH + ch];
-        hk[j] = fmaf(eA[j], wk, eK[j]);
-        hv[j] = fmaf(eA[j], wv, eV[j]);
-    }
-    float rc[VEC], rs[VEC], sc[VEC], ss[VEC];
-    const bool first_half = cl < LPR / 2;
-    if (p.rope) {
-        const long long pos = p.pos0 + t0 + seg * R;
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) {
-            const int f = (cl * VEC + j) % (DH / 2);
-            rope_cs(pos, p.theta[f], rc[j], rs[j]);
-            sc[j] = p.step_cos[f];
-            ss[j] = first_half ? -p.step_sin[f] : p.step_sin[f];
-            if (first_half) rs[j] = -rs[j];      // first half: x cos - x' sin
-        }
-    }
-    uint8_t *yk = static_cast<uint8_t *>(p.yk);
-    uint8_t *yv = static_cast<uint8_t *>(p.yv);
-#pragma unroll
-    for (int i = 0; i < R; ++i) {
-        const int r = seg * R + i;
-        const bool valid = r < rows;
-        float xa[VEC], xk[VEC], xv[VEC];
-        if (valid) {
-            const int off = r * C::ROWB + cl * 16;
-            Vec<E>::load(sa + off, xa);
-            Vec<E>::load(sk + off, xk);
-            Vec<E>::load(sv + off, xv);
-        } else {
-#pragma unroll
-            for (int j = 0; j < VEC; ++j) { xa[j] = 0.f; xk[j] = 0.f; xv[j] = 0.f; }
-        }
-        float ok[VEC];
-#pragma unroll
-        for (int j = 0; j < VEC; ++j) {
-            float g, omg;
-            forget_gate(xa[j], g, omg);
-            hk[j] = fmaf(g, hk[j], omg * xk[j]);
-            hv[j] = fmaf(g, hv[j], omg * xv[j]);
-            ok[j] = hk[j];
-        }
-        if (p.rope) {       // uniform across the grid: the shuffles see every lane
+        float rc[VEC], rs[VEC], sc[VEC], ss[VEC];
+        const bool first_half = cl < LPR / 2;
+        if (p.rope) {
+            const long long pos = p.pos0 + t0 + seg * R;
 #pragma unroll
             for (int j = 0; j < VEC; ++j) {
-                const float partner = __shfl_xor_sync(0xffffffffu, hk[j], LPR / 2);
-                ok[j] = fmaf(hk[j], rc[j], partner * rs[j]);
-                // advance the angle by one position: (c + i s) * (cos t + i sin t)
-                const float nc = rc[j] * sc[j] - rs[j] * ss[j];
-                const float ns = rs[j] * sc[j] + rc[j] * ss[j];
-                rc[j] = nc;
-                rs[j] = ns;
+                const int f = (cl * VEC + j) % (DH / 2);
+                rope_cs(pos, p.theta[f], rc[j], rs[j]);
+                sc[j] = p.step_cos[f];
+                ss[j] = first_half ? -p.step_sin[f] : p.step_sin[f];
+                if (first_half) rs[j] = -rs[j];      // first half: x cos - x' sin
             }
         }
-        if (valid) {
-            const size_t go = (row0 + r) * C::ROWB + cl * 16;
-            Vec<E>::store(yk + go, ok);
-            Vec<E>::store(yv + go, hv);
+        uint8_t *yk = static_cast<uint8_t *>(p.yk);
+        uint8_t *yv = static_cast<uint8_t *>(p.yv);
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int r = seg * R + i;
+            const bool valid = r < rows;
+            float xk[VEC], xv[VEC];
+            if (valid) {
+                const int off = r * C::ROWB + cl * 16;
+                Vec<E>::load(sk + off, xk);
+                Vec<E>::load(sv + off, xv);
+            } else {
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) { xk[j] = 0.f; xv[j] = 0.f; }
+            }
+            float ok[VEC];
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) {
+                hk[j] = fmaf(G[i][j], hk[j], OG[i][j] * xk[j]);
+                hv[j] = fmaf(G[i][j], hv[j], OG[i][j] * xv[j]);
+                ok[j] = hk[j];
+            }
+            if (p.rope) {       // uniform across the grid: the shuffles see every lane
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) {
+                    const float partner = __shfl_xor_sync(0xffffffffu, hk[j], LPR / 2);
+                    ok[j] = fmaf(hk[j], rc[j], partner * rs[j]);
+                    // advance the angle by one position: (c + i s) * (cos t + i sin t)
+                    const float nc = rc[j] * sc[j] - rs[j] * ss[j];
+                    const float ns = rs[j] * sc[j] + rc[j] * ss[j];
+                    rc[j] = nc;
+                    rs[j] = ns;
+                }
+            }
+            if (valid) {
+                const size_t go = (row0 + r) * C::ROWB + cl * 16;
+                Vec<E>::store(yk + go, ok);
+                Vec<E>::store(yv + go, hv);
+            }
         }
+        __syncthreads();     // this stage's smem and sw are free for the next chunk
     }
 
     // ---- launch bookkeeping: the last CTA resets the ticket counter and bumps the epoch
     if (tid == 0) {
         __threadfence();
-        const uint32_t total = (uint32_t)p.BH * (uint32_t)p.nchunks;
-        if (atomicAdd(&hdr->done, 1u) == total - 1) {
+        if (atomicAdd(&hdr->done, 1u) == gridDim.x - 1) {
             hdr->ticket = 0;
             hdr->done = 0;
             __threadfence();
@@ -358,7 +386,16 @@ static int launch_one(const RecurParams &p, void *stream) {
             return RAT_ERR_CUDA;
         attr_set = true;
     }
-    const unsigned grid = (unsigned)p.BH * (unsigned)p.nchunks;
+    static int sms = 0;
+    if (!sms) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return RAT_ERR_CUDA;
+    }
+    // persistent: one CTA per SM, each walking chunks in ticket order
+    const long long total = (long long)p.BH * p.nchunks;
+    const unsigned grid = (unsigned)(total < sms ? total : sms);
     kern<<<grid, C::THREADS, C::SMEM, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }

@@ -16,6 +16,14 @@ from gpu_util import TOL_BF16, TOL_F32, f64, gpu_attn, gpu_recur, rel_err, tol_f
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=[64, 128], ids=["bk64", "bk128"])
+def block_keys(request):
+    """Run a tensor-core case with each key-block width of the bf16 kernel."""
+    rat.rat_set_attn_block_keys(request.param)
+    yield request.param
+    rat.rat_set_attn_block_keys(0)
+
+
 def qkv(B, H, T, d, dtype, seed):
     g = torch.Generator().manual_seed(seed)
     return tuple(torch.randn((B, H, T, d), generator=g).to(dtype) for _ in range(3))
@@ -80,7 +88,7 @@ BF16_CASES = [
 
 
 @pytest.mark.parametrize("B,H,T,D,W,Dph", BF16_CASES)
-def test_bf16_cases(B, H, T, D, W, Dph):
+def test_bf16_cases(B, H, T, D, W, Dph, block_keys):
     q, k, v = qkv(B, H, T, 128, torch.bfloat16, seed=T + 31 * D + W)
     check_attn(q, k, v, D=D, W=W, D_per_head=Dph)
 
@@ -90,20 +98,21 @@ def test_bf16_d64():
     check_attn(q, k, v, D=4, W=3)
 
 
-def test_bf16_rope_query():
+def test_bf16_rope_query(block_keys):
     q, k, v = qkv(1, 2, 700, 128, torch.bfloat16, seed=77)
     check_attn(q, k, v, D=16, W=0, rope_base=10000.0, pos0=3000)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-def test_self_only_returns_values_exactly(dtype):
+def test_self_only_returns_values_exactly(dtype, block_keys):
     # D > T and W = 0: every query sees only itself, so o_t = v~_t exactly.
     q, k, v = qkv(1, 2, 300, 128, dtype, seed=5)
     o = gpu_attn(q, k, v, D=1000, W=0)
     assert torch.equal(o.cpu(), v)
+    assert rat.rat_attn_sync_status() == 0
 
 
-def test_dense_d1_equals_window_covering_all():
+def test_dense_d1_equals_window_covering_all(block_keys):
     q, k, v = qkv(1, 2, 500, 128, torch.bfloat16, seed=8)
     o1 = gpu_attn(q, k, v, D=1, W=0)
     o2 = gpu_attn(q, k, v, D=64, W=500)
@@ -111,7 +120,7 @@ def test_dense_d1_equals_window_covering_all():
     assert rel_err(o1, ref) <= TOL_BF16 and rel_err(o2, ref) <= TOL_BF16
 
 
-def test_head_hybrid_equals_uniform_runs():
+def test_head_hybrid_equals_uniform_runs(block_keys):
     q, k, v = qkv(1, 4, 600, 128, torch.bfloat16, seed=9)
     Dh = [1, 4, 16, 64]
     o = gpu_attn(q, k, v, W=32, D_per_head=Dh)
@@ -128,7 +137,7 @@ def sample_rows(T, n=96, seed=0):
 
 
 @pytest.mark.parametrize("name", ["prefill_1p5b", "window_2p6b", "hybrid_7p6b"])
-def test_full_size_end_to_end_sampled(name):
+def test_full_size_end_to_end_sampled(name, block_keys):
     """Whole prefill (recurrence + attention) at the workload's full size, checked on sampled
     heads and rows against the oracle's own recurrence and attention."""
     w = synthetic.WORKLOADS[name]
