@@ -65,13 +65,20 @@ struct Params {
     CUtensorMap tm_q, tm_o;                        // (d, T, B*H) bf16, box (64, 128, 1), 128B swizzle
     CUtensorMap tm_k, tm_v;                        // same tensors, box (64, BN, 1)
     CUtensorMap tm_kd[kMaxDil], tm_vd[kMaxDil];    // chunk ends of one dilation: (d, T/D, B*H)
+    const void *kg, *vg;                           // k~, v~ (the self key when W <= 1)
     int B, H, T, W, ntiles;
     long long pos0;
     int rope;
     float scale_log2;
-    int head_of[kMaxHeads];   // grid y (mod H) -> head, heaviest (smallest D) first
+    int head_of[kMaxHeads];   // heads sorted by dilation, smallest (most keys) first
     int Dh[kMaxHeads];
     int dslot[kMaxHeads];     // head -> index into tm_kd / tm_vd (-1 when D == 1)
+    // work order: groups of heads with equal D, in head_of order; inside a group, tiles from
+    // the last (most keys) to the first, all (b, head) of a tile row together
+    int ngroups;
+    int grp_item0[kMaxHeads + 1];   // first linear block index of each group
+    int grp_head0[kMaxHeads];       // first index into head_of
+    int grp_nheads[kMaxHeads];
     double theta[64];
 };
 
@@ -82,6 +89,7 @@ RAT_DEVICE int floordiv(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) /
 struct Plan {
     int nd, nw, ws, D, We;
     bool dense;
+    bool self_reg;    // We == 1 (dilated head): the self key is handled in registers, no window blocks
 };
 template <int BN>
 RAT_DEVICE Plan make_plan(int t0, int D, int W, int T) {
@@ -89,6 +97,7 @@ RAT_DEVICE Plan make_plan(int t0, int D, int W, int T) {
     pl.D = D;
     pl.We = W > 1 ? W : 1;
     pl.dense = D == 1;
+    pl.self_reg = !pl.dense && pl.We == 1;
     const int tmax = t0 + BM - 1;
     if (pl.dense) {
         pl.nd = 0;
@@ -100,7 +109,7 @@ RAT_DEVICE Plan make_plan(int t0, int D, int W, int T) {
         if (ndk > cap) ndk = cap;
         pl.nd = (ndk + BN - 1) / BN;
         pl.ws = t0 - pl.We + 1 > 0 ? t0 - pl.We + 1 : 0;
-        pl.nw = (tmax + 1 - pl.ws + BN - 1) / BN;
+        pl.nw = pl.self_reg ? 0 : (tmax + 1 - pl.ws + BN - 1) / BN;
     }
     return pl;
 }
@@ -140,6 +149,17 @@ RAT_DEVICE bool wait_bar(Shared &sh, uint64_t *bar, uint32_t parity) {
     }
 }
 
+// cos/sin of pos * theta: angle in float64 reduced by 2*pi (two-term constant), then the
+// special-function-unit sincos on [-pi, pi] (absolute error ~1e-6, far below bf16 rounding).
+RAT_DEVICE void rope_cs_fast(long long pos, double theta, float &c, float &s) {
+    const double kTwoPiHi = 6.283185307179586, kTwoPiLo = 2.4492935982947064e-16;
+    const double ang = (double)pos * theta;
+    const double n = rint(ang * 0.15915494309189535);
+    double r = fma(-n, kTwoPiHi, ang);
+    r = fma(-n, kTwoPiLo, r);
+    __sincosf((float)r, &s, &c);
+}
+
 RAT_DEVICE uint32_t swz(uint32_t row, uint32_t chunk) {   // 128B swizzle inside a sub-tile
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
@@ -158,10 +178,16 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
     Shared &sh = *reinterpret_cast<Shared *>(smem + C::OFF_BAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-    const int tile = p.ntiles - 1 - (int)blockIdx.x;        // longest tiles first
+    // linear block index -> (tile, b, h): longest work first (see Params)
+    const int L = (int)blockIdx.x;
+    int g = 0;
+    while (g + 1 < p.ngroups && L >= p.grp_item0[g + 1]) ++g;
+    const int local = L - p.grp_item0[g];
+    const int per_row = p.B * p.grp_nheads[g];
+    const int tile = p.ntiles - 1 - local / per_row;
     const int t0 = tile * BM;
-    const int b = (int)blockIdx.y / p.H;
-    const int h = p.head_of[(int)blockIdx.y % p.H];
+    const int b = (local % per_row) / p.grp_nheads[g];
+    const int h = p.head_of[p.grp_head0[g] + (local % per_row) % p.grp_nheads[g]];
     const int bh = b * p.H + h;
     const Plan pl = make_plan<BN>(t0, p.Dh[h], p.W, p.T);
     const int nb = pl.nd + pl.nw;
@@ -299,8 +325,8 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                     float x1l = bf16_lo(a1[i]), x1h = bf16_hi(a1[i]);
                     float x2l = bf16_lo(a2[i]), x2h = bf16_hi(a2[i]);
                     float cl, sl, ch, sh2;
-                    rope_cs(pos, p.theta[c * 8 + 2 * i], cl, sl);
-                    rope_cs(pos, p.theta[c * 8 + 2 * i + 1], ch, sh2);
+                    rope_cs_fast(pos, p.theta[c * 8 + 2 * i], cl, sl);
+                    rope_cs_fast(pos, p.theta[c * 8 + 2 * i + 1], ch, sh2);
                     a1[i] = pack_bf16(x1l * cl - x2l * sl, x1h * ch - x2h * sh2);
                     a2[i] = pack_bf16(x2l * cl + x1l * sl, x2h * ch + x1h * sh2);
                 }
@@ -312,6 +338,29 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         mbar_arrive(&sh.q_ready);
 
         float m_run = -INFINITY, l_run = 0.f;
+        float w_self = 0.f;        // weight of the self key when it is kept in registers
+        if (ok && pl.self_reg) {
+            // s_self = q^_t . k~_t with q^ from the (rotated) smem tile and k~_t from global
+            float dot = 0.f;
+            if (t < p.T) {
+                const uint4 *krow = reinterpret_cast<const uint4 *>(
+                    static_cast<const uint8_t *>(p.kg) + ((size_t)bh * p.T + t) * (DHEAD * 2));
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const uint4 kq = __ldg(krow + c);
+                    const uint4 qq = *reinterpret_cast<const uint4 *>(sQ + (c >> 3) * QSUB + swz(r, c & 7));
+                    const uint32_t ku[4] = {kq.x, kq.y, kq.z, kq.w}, qu[4] = {qq.x, qq.y, qq.z, qq.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        dot = fmaf(bf16_lo(qu[i]), bf16_lo(ku[i]), dot);
+                        dot = fmaf(bf16_hi(qu[i]), bf16_hi(ku[i]), dot);
+                    }
+                }
+            }
+            m_run = dot * p.scale_log2;
+            l_run = 1.f;
+            w_self = 1.f;
+        }
         float sv[BN];
         int jdone = 0;
         for (int j = 0; ok && j < nb; ++j) {
@@ -340,6 +389,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             if (resc) {
                 alpha = ex2_approx(m_run - m_new);
                 l_run *= alpha;
+                w_self *= alpha;
                 m_run = m_new;
             }
             const float mu = m_run == -INFINITY ? 0.f : m_run;
@@ -383,15 +433,34 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         }
         // ---- epilogue: O / l -> bf16 -> smem (Q's tile, no longer read) -> TMA store
         bool have_o = ok && jdone == nb;
-        if (have_o) have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready, (nb - 1) & 1));
+        if (have_o && nb > 0) have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready, (nb - 1) & 1));
         if (have_o) {
             tc::fence_after_sync();
             const float inv = 1.0f / l_run;
+            const uint4 *vrow = reinterpret_cast<const uint4 *>(
+                static_cast<const uint8_t *>(p.vg) + ((size_t)bh * p.T + min(t, p.T - 1)) * (DHEAD * 2));
 #pragma unroll 1
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
-                tc::tmem_ld32(tl + C::COL_O + 32 * c, o);
-                tc::tmem_wait_ld();
+                if (nb > 0) {
+                    tc::tmem_ld32(tl + C::COL_O + 32 * c, o);
+                    tc::tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) o[i] = 0u;
+                }
+                if (pl.self_reg) {          // O += w_self * v~_t (the self key's value)
+#pragma unroll
+                    for (int k8 = 0; k8 < 4; ++k8) {
+                        const uint4 vv = __ldg(vrow + 4 * c + k8);
+                        const uint32_t vu[4] = {vv.x, vv.y, vv.z, vv.w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            o[8 * k8 + 2 * i] = __float_as_uint(fmaf(w_self, bf16_lo(vu[i]), __uint_as_float(o[8 * k8 + 2 * i])));
+                            o[8 * k8 + 2 * i + 1] = __float_as_uint(fmaf(w_self, bf16_hi(vu[i]), __uint_as_float(o[8 * k8 + 2 * i + 1])));
+                        }
+                    }
+                }
 #pragma unroll
                 for (int k8 = 0; k8 < 4; ++k8) {
                     const int col = 32 * c + 8 * k8;
@@ -496,6 +565,21 @@ int launch_bn(const AttnSm100Args &a, void *stream) {
     for (int h = 0; h < a.H; ++h) p.head_of[h] = order[h];
     p.B = a.B; p.H = a.H; p.T = a.T; p.W = a.W;
     p.ntiles = (a.T + BM - 1) / BM;
+    p.kg = a.k;
+    p.vg = a.v;
+    p.ngroups = 0;
+    int items = 0;
+    for (int i = 0; i < a.H;) {
+        int k = i;
+        while (k < a.H && a.Dh[order[k]] == a.Dh[order[i]]) ++k;
+        p.grp_item0[p.ngroups] = items;
+        p.grp_head0[p.ngroups] = i;
+        p.grp_nheads[p.ngroups] = k - i;
+        items += p.ntiles * a.B * (k - i);
+        ++p.ngroups;
+        i = k;
+    }
+    p.grp_item0[p.ngroups] = items;
     p.pos0 = a.pos0;
     p.rope = a.rope;
     p.scale_log2 = a.scale_log2;
@@ -508,8 +592,7 @@ int launch_bn(const AttnSm100Args &a, void *stream) {
             return RAT_ERR_CUDA;
         attr = true;
     }
-    dim3 grid((unsigned)p.ntiles, (unsigned)BH);
-    attn_sm100_kernel<BN><<<grid, kThreads, C::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(p);
+    attn_sm100_kernel<BN><<<(unsigned)items, kThreads, C::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 
