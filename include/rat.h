@@ -215,6 +215,26 @@ RAT_API int rat_dilated_decode(const void *q, const void *k, const void *v, cons
  * Returns RAT_ERR_INVALID for out-of-range arguments. */
 RAT_API int rat_debug_inject_lookback_fault(int64_t chunk, int64_t wait_limit_ns);
 
+/* rat_dilated_decode_noalloc -- the same decode step, for callers that cannot allocate.
+ * (The pages have no counterpart: this is a property of the library, not of the method.)
+ * Some callers cannot give the library a device buffer for the decode workspace: their device
+ * memory belongs to a host framework or is planned up front as a fixed arena, and they have no
+ * way to ask for one more allocation.  This entry point allocates nothing; it uses a fixed
+ * 8 MiB scratch array compiled into the library (each GPU that loads the library holds it until
+ * the process exits) and otherwise runs exactly rat_dilated_decode.
+ *   - Arguments and results are those of rat_dilated_decode, without ws / ws_bytes.
+ *   - Returns RAT_ERR_WORKSPACE when rat_decode_workspace_bytes(cache) exceeds 8 MiB (for d = 128
+ *     that is roughly B * H * splits above 16,000).
+ *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
+ *   - Every call shares the one array, which keeps the previous call's contents; each call
+ *     clears its header and tickets on `stream` first.  Calls that overlap on the GPU (other
+ *     streams, other host threads) race on the array and must be serialised by the caller.
+ *   - The array is not reachable by rat_sync_status(); decode has no device-side waits. */
+RAT_API int rat_dilated_decode_noalloc(const void *q, const void *k, const void *v,
+                                       const void *gate_logit, rat_kv_cache *cache, void *o,
+                                       float rope_base, float scale, void *stream);
+
 /* Number of keys query t attends to: min(We, t+1) + max(0, floor((t - We + 1) / D)).
  * Host-only helper used for FLOP and byte accounting. */
 RAT_API int64_t rat_attended_keys(int64_t t, int D, int W);

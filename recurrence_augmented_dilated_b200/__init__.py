@@ -24,7 +24,7 @@ __all__ = [
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
     "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
-    "Workspace",
+    "Workspace", "rat_dilated_decode_noalloc",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -84,6 +84,8 @@ def lib():
         L.rat_dilated_decode.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(KVCache), _vp, _f, _f,
                                          _vp, _sz, _vp]
         L.rat_debug_inject_lookback_fault.argtypes = [_i64, _i64]
+        L.rat_dilated_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(KVCache), _vp,
+                                                 _f, _f, _vp]
         L.rat_attn_sync_status.argtypes = [_vp]
         L.rat_set_attn_block_keys.argtypes = [_i]
         L.rat_attended_keys.restype = _i64
@@ -234,3 +236,13 @@ def rat_dilated_decode(q, k, v, gate_logit, cache: KVCache, o, ws: Workspace,
                                   _ptr(o), float(rope_base), float(scale), ws.ptr, ws.nbytes,
                                   _stream(stream))
     _check("rat_dilated_decode", st)
+
+
+def rat_dilated_decode_noalloc(q, k, v, gate_logit, cache: KVCache, o, rope_base: float = 0.0,
+                               scale: float = 0.0, stream=None):
+    """rat_dilated_decode without a workspace argument: the library's fixed device scratch is used
+    (for callers that cannot allocate; concurrent calls must not overlap on the GPU)."""
+    st = lib().rat_dilated_decode_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit),
+                                          ctypes.byref(cache), _ptr(o), float(rope_base),
+                                          float(scale), _stream(stream))
+    _check("rat_dilated_decode_noalloc", st)

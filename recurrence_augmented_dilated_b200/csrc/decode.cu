@@ -15,6 +15,8 @@
 // Split 0 alone does steps 1-2 and adds the token itself to its softmax.
 // No CTA reads what another writes in the same launch: the new dil entry (position t) is never
 // older than the window, and the ring slot written held position t - W, outside the window.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace rat {
@@ -276,3 +278,55 @@ int launch_decode(const DecodeParams &p, int dtype, void *stream) {
 }
 
 }  // namespace rat
+
+// ------------------------------------------------------------------------------ no-allocation entry
+// A decode call needs a small scratch area (per-split partial results and per-slice tickets).
+// Some callers cannot hand the library a device buffer for it: their device memory is owned by a
+// host framework or planned up front as a fixed arena, and they have no way to obtain an extra
+// allocation.  rat_dilated_decode_noalloc serves them from this fixed array in the library's own
+// device image (every GPU that loads the library holds it until the process exits).
+namespace rat {
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;     // 8 MiB
+constexpr int kNoAllocMaxDevices = 64;
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kNoAllocMaxDevices];   // device address of g_decode_scratch, per device
+}  // namespace
+
+}  // namespace rat
+
+extern "C" int rat_dilated_decode_noalloc(const void *q, const void *k, const void *v,
+                                          const void *gate_logit, rat_kv_cache *cache, void *o,
+                                          float rope_base, float scale, void *stream) {
+    using namespace rat;
+    const size_t need = rat_decode_workspace_bytes(cache);
+    if (need == 0) return RAT_ERR_INVALID;                  // invalid cache description
+    if (need > kNoAllocScratchBytes) return RAT_ERR_WORKSPACE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return RAT_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return RAT_ERR_UNSUPPORTED;
+    void *ptr = nullptr;
+    {
+        // first call on this device: look up the array's device address (host code cannot use
+        // the symbol itself as a device pointer)
+        std::lock_guard<std::mutex> lock(g_scratch_mutex);
+        if (!g_scratch_addr[dev]) {
+            void *a = nullptr;
+            if (cudaGetSymbolAddress(&a, g_decode_scratch) != cudaSuccess || !a) return RAT_ERR_CUDA;
+            g_scratch_addr[dev] = a;
+        }
+        ptr = g_scratch_addr[dev];
+    }
+    // the array keeps the previous call's contents: the header (error word) and the per-slice
+    // tickets must start at zero
+    const size_t bh = (size_t)cache->B * cache->H;
+    if (cudaMemsetAsync(ptr, 0, sizeof(WsHeader) + align256(bh * 4), static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return RAT_ERR_CUDA;
+    return rat_dilated_decode(q, k, v, gate_logit, cache, o, rope_base, scale, ptr, kNoAllocScratchBytes, stream);
+}
+
