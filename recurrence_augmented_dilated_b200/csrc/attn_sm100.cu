@@ -79,6 +79,8 @@ struct Params {
     int grp_item0[kMaxHeads + 1];   // first linear block index of each group
     int grp_head0[kMaxHeads];       // first index into head_of
     int grp_nheads[kMaxHeads];
+    int rope_f32;             // positions small enough for float32 angles (pos0 + T <= 2^13)
+    float theta_f[64];
     double theta[64];
 };
 
@@ -158,6 +160,17 @@ RAT_DEVICE void rope_cs_fast(long long pos, double theta, float &c, float &s) {
     double r = fma(-n, kTwoPiHi, ang);
     r = fma(-n, kTwoPiLo, r);
     __sincosf((float)r, &s, &c);
+}
+
+// Same with a float32 angle; used while pos * theta stays below 2^13 rad, where the float32
+// product is within 2.5e-4 rad of the exact angle (a bf16 query carries 4e-3 relative error).
+RAT_DEVICE void rope_cs_f32(int pos, float theta, float &c, float &s) {
+    const float kTwoPiHi = 6.28318548f, kTwoPiLo = -1.7484555e-7f;   // 2*pi = hi + lo
+    const float ang = (float)pos * theta;
+    const float n = rintf(ang * 0.159154943f);
+    float r = fmaf(-n, kTwoPiHi, ang);
+    r = fmaf(-n, kTwoPiLo, r);
+    __sincosf(r, &s, &c);
 }
 
 RAT_DEVICE uint32_t swz(uint32_t row, uint32_t chunk) {   // 128B swizzle inside a sub-tile
@@ -308,6 +321,15 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
         uint8_t *sQ = smem + C::OFF_Q;
         uint8_t *sP = smem + C::OFF_P;
+        // the self key's row (W <= 1): issue its loads now so they overlap the Q load
+        uint4 kself[16];
+        const bool have_self = pl.self_reg && t < p.T;
+        if (have_self) {
+            const uint4 *krow = reinterpret_cast<const uint4 *>(
+                static_cast<const uint8_t *>(p.kg) + ((size_t)bh * p.T + t) * (DHEAD * 2));
+#pragma unroll
+            for (int c = 0; c < 16; ++c) kself[c] = __ldg(krow + c);
+        }
         // waits are made warp-uniform: tcgen05.ld/st below are warp-collective
         bool ok = __all_sync(0xffffffffu, wait_bar(sh, &sh.q_full, 0));
         if (ok && p.rope) {
@@ -325,8 +347,13 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                     float x1l = bf16_lo(a1[i]), x1h = bf16_hi(a1[i]);
                     float x2l = bf16_lo(a2[i]), x2h = bf16_hi(a2[i]);
                     float cl, sl, ch, sh2;
-                    rope_cs_fast(pos, p.theta[c * 8 + 2 * i], cl, sl);
-                    rope_cs_fast(pos, p.theta[c * 8 + 2 * i + 1], ch, sh2);
+                    if (p.rope_f32) {
+                        rope_cs_f32((int)pos, p.theta_f[c * 8 + 2 * i], cl, sl);
+                        rope_cs_f32((int)pos, p.theta_f[c * 8 + 2 * i + 1], ch, sh2);
+                    } else {
+                        rope_cs_fast(pos, p.theta[c * 8 + 2 * i], cl, sl);
+                        rope_cs_fast(pos, p.theta[c * 8 + 2 * i + 1], ch, sh2);
+                    }
                     a1[i] = pack_bf16(x1l * cl - x2l * sl, x1h * ch - x2h * sh2);
                     a2[i] = pack_bf16(x2l * cl + x1l * sl, x2h * ch + x1h * sh2);
                 }
@@ -342,12 +369,10 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         if (ok && pl.self_reg) {
             // s_self = q^_t . k~_t with q^ from the (rotated) smem tile and k~_t from global
             float dot = 0.f;
-            if (t < p.T) {
-                const uint4 *krow = reinterpret_cast<const uint4 *>(
-                    static_cast<const uint8_t *>(p.kg) + ((size_t)bh * p.T + t) * (DHEAD * 2));
+            if (have_self) {
 #pragma unroll
                 for (int c = 0; c < 16; ++c) {
-                    const uint4 kq = __ldg(krow + c);
+                    const uint4 kq = kself[c];
                     const uint4 qq = *reinterpret_cast<const uint4 *>(sQ + (c >> 3) * QSUB + swz(r, c & 7));
                     const uint32_t ku[4] = {kq.x, kq.y, kq.z, kq.w}, qu[4] = {qq.x, qq.y, qq.z, qq.w};
 #pragma unroll
@@ -376,13 +401,23 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
 
             int c_lo, c_hi;
             block_range<BN>(pl, j, t, c_lo, c_hi);
-            float mx = -INFINITY;
+            // row max of the raw scores (scale > 0 commutes with max), as an 8-way tree; keys
+            // outside S(t) become -inf (only blocks that cut the key set need the mask)
+            float m8[8];
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                const float x = (c >= c_lo && c <= c_hi) ? sv[c] * p.scale_log2 : -INFINITY;
-                sv[c] = x;
-                mx = fmaxf(mx, x);
+            for (int u = 0; u < 8; ++u) m8[u] = -INFINITY;
+            if (c_lo <= 0 && c_hi >= BN - 1) {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
+            } else {
+#pragma unroll
+                for (int c = 0; c < BN; ++c) {
+                    sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
+                    m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
+                }
             }
+            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
             const float m_new = fmaxf(m_run, mx);
             const bool resc = m_new > m_run + kRescaleLog2;
             float alpha = 1.f;
@@ -392,15 +427,17 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                 w_self *= alpha;
                 m_run = m_new;
             }
-            const float mu = m_run == -INFINITY ? 0.f : m_run;
-            float sum = 0.f;
+            const float neg_mu = m_run == -INFINITY ? 0.f : -m_run;
+            float s8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s8[u] = 0.f;
 #pragma unroll
             for (int c = 0; c < BN; ++c) {
-                const float e = ex2_approx(sv[c] - mu);
+                const float e = ex2_approx(fmaf(sv[c], p.scale_log2, neg_mu));   // -inf -> 0
                 sv[c] = e;
-                sum += e;
+                s8[c & 7] += e;
             }
-            l_run += sum;
+            l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
             if (j > 0) {
                 // PV of the previous block done: P may be overwritten, O is stable
                 if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready, (j - 1) & 1))) { ok = false; break; }
@@ -433,13 +470,18 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         }
         // ---- epilogue: O / l -> bf16 -> smem (Q's tile, no longer read) -> TMA store
         bool have_o = ok && jdone == nb;
+        uint4 vself[16];          // the self key's value row, loaded while the last PV runs
+        if (have_o && pl.self_reg) {
+            const uint4 *vrow = reinterpret_cast<const uint4 *>(
+                static_cast<const uint8_t *>(p.vg) + ((size_t)bh * p.T + min(t, p.T - 1)) * (DHEAD * 2));
+#pragma unroll
+            for (int c = 0; c < 16; ++c) vself[c] = __ldg(vrow + c);
+        }
         if (have_o && nb > 0) have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready, (nb - 1) & 1));
         if (have_o) {
             tc::fence_after_sync();
             const float inv = 1.0f / l_run;
-            const uint4 *vrow = reinterpret_cast<const uint4 *>(
-                static_cast<const uint8_t *>(p.vg) + ((size_t)bh * p.T + min(t, p.T - 1)) * (DHEAD * 2));
-#pragma unroll 1
+#pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
                 if (nb > 0) {
@@ -452,7 +494,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                 if (pl.self_reg) {          // O += w_self * v~_t (the self key's value)
 #pragma unroll
                     for (int k8 = 0; k8 < 4; ++k8) {
-                        const uint4 vv = __ldg(vrow + 4 * c + k8);
+                        const uint4 vv = vself[4 * c + k8];
                         const uint32_t vu[4] = {vv.x, vv.y, vv.z, vv.w};
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
@@ -582,8 +624,12 @@ int launch_bn(const AttnSm100Args &a, void *stream) {
     p.grp_item0[p.ngroups] = items;
     p.pos0 = a.pos0;
     p.rope = a.rope;
+    p.rope_f32 = a.pos0 + (long long)a.T <= 8192 ? 1 : 0;
     p.scale_log2 = a.scale_log2;
-    for (int c = 0; c < 64; ++c) p.theta[c] = a.theta[c];
+    for (int c = 0; c < 64; ++c) {
+        p.theta[c] = a.theta[c];
+        p.theta_f[c] = (float)a.theta[c];
+    }
 
     static bool attr = false;
     if (!attr) {

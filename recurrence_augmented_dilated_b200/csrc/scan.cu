@@ -39,15 +39,20 @@ struct ScanCfg {
     static constexpr int VEC = 16 / EB;           // channels per lane (one 16-byte vector)
     static constexpr int LPR = DH / VEC;          // lanes per row
     static constexpr int THREADS = 256;
-    static constexpr int NW = THREADS / 32;       // warps
-    static constexpr int SEGS = THREADS / LPR;    // row segments per chunk
+    static constexpr int NPIPE = 2;               // independent chunk pipelines per CTA
+    static constexpr int PT = THREADS / NPIPE;    // threads per pipeline
+    static constexpr int PW = PT / 32;            // warps per pipeline
+    static constexpr int SEGS = PT / LPR;         // row segments per chunk
     static constexpr int SPW = 32 / LPR;          // segments per warp
     static constexpr int R = 8;                   // rows per segment
     static constexpr int TC = SEGS * R;           // rows per chunk
     static constexpr int ROWB = DH * EB;          // bytes per row
-    static constexpr int TILEB = TC * ROWB;       // bytes per tensor per chunk (32 KiB)
+    static constexpr int TILEB = TC * ROWB;       // bytes per tensor per chunk (16 KiB)
     static constexpr int STAGEB = 3 * TILEB;      // a, k, v of one chunk
-    static constexpr int SMEM = 2 * STAGEB + NW * 3 * DH * 4;   // two stages + warp carries
+    static constexpr int SWB = PW * 3 * DH * 4;   // per-warp aggregates, then carries
+    static constexpr int PIPEB = 2 * STAGEB + SWB + 2 * DH * 4;   // two stages + sw + state in
+    static constexpr int SMEM = NPIPE * PIPEB;
+    static_assert(PT >= DH, "one thread per channel in a pipeline");
 };
 
 // 16 bytes of a row -> VEC floats.
@@ -102,50 +107,61 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
     using C = ScanCfg<E, DH>;
     constexpr int VEC = C::VEC, LPR = C::LPR, R = C::R;
     extern __shared__ __align__(128) uint8_t smem[];
-    float *sw = reinterpret_cast<float *>(smem + 2 * C::STAGEB);   // [NW][3][DH]
-    __shared__ uint64_t bar[2];
-    __shared__ int s_ticket[2];
+    __shared__ uint64_t bar[C::NPIPE][2];
+    __shared__ int s_ticket[C::NPIPE][2];
     __shared__ uint32_t s_epoch;
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int seg = tid / LPR, cl = tid % LPR, segw = lane / LPR;
+    const int tid = threadIdx.x;
+    const int pipe = tid / C::PT, pt = tid % C::PT;              // pipeline and thread in it
+    const int pwarp = pt >> 5, lane = tid & 31;
+    const int seg = pt / LPR, cl = pt % LPR, segw = lane / LPR;
+    const int barid = 1 + pipe;                                   // named barrier of this pipeline
+    uint8_t *pbase = smem + pipe * C::PIPEB;
+    float *sw = reinterpret_cast<float *>(pbase + 2 * C::STAGEB);          // [PW][3][DH]
+    float *sH = reinterpret_cast<float *>(pbase + 2 * C::STAGEB + C::SWB); // [2][DH] state in
     WsHeader *hdr = p.hdr;
     const int total = p.BH * p.nchunks;
 
-    // issue the three bulk copies of chunk `ticket` into stage `st` (thread 0 only)
+    // issue the three bulk copies of chunk `ticket` into stage `st` (thread 0 of the pipeline)
     auto load_chunk = [&](int ticket, int st) {
         const int c = ticket / p.BH, bh = ticket % p.BH;
         const int rows = min(C::TC, p.T - c * C::TC);
         const size_t row0 = (size_t)bh * p.T + (size_t)c * C::TC;
         const uint32_t bytes = (uint32_t)rows * C::ROWB;
-        uint8_t *s = smem + st * C::STAGEB;
-        mbar_arrive_expect_tx(&bar[st], 3 * bytes);
-        bulk_g2s(s, static_cast<const uint8_t *>(p.a) + row0 * C::ROWB, bytes, &bar[st]);
-        bulk_g2s(s + C::TILEB, static_cast<const uint8_t *>(p.k) + row0 * C::ROWB, bytes, &bar[st]);
-        bulk_g2s(s + 2 * C::TILEB, static_cast<const uint8_t *>(p.v) + row0 * C::ROWB, bytes, &bar[st]);
+        uint8_t *s = pbase + st * C::STAGEB;
+        mbar_arrive_expect_tx(&bar[pipe][st], 3 * bytes);
+        bulk_g2s(s, static_cast<const uint8_t *>(p.a) + row0 * C::ROWB, bytes, &bar[pipe][st]);
+        bulk_g2s(s + C::TILEB, static_cast<const uint8_t *>(p.k) + row0 * C::ROWB, bytes, &bar[pipe][st]);
+        bulk_g2s(s + 2 * C::TILEB, static_cast<const uint8_t *>(p.v) + row0 * C::ROWB, bytes, &bar[pipe][st]);
     };
+    auto pipe_sync = [&]() { asm volatile("bar.sync %0, %1;" :: "r"(barid), "r"(C::PT) : "memory"); };
 
     if (tid == 0) {
         s_epoch = *reinterpret_cast<volatile uint32_t *>(&hdr->epoch);
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
+        for (int q = 0; q < C::NPIPE; ++q) {
+            mbar_init(&bar[q][0], 1);
+            mbar_init(&bar[q][1], 1);
+        }
         fence_mbar_init();
-        const int t0k = (int)atomicAdd(&hdr->ticket, 1u);
-        s_ticket[0] = t0k;
-        if (t0k < total) load_chunk(t0k, 0);
     }
     __syncthreads();
     const uint32_t epoch_raw = s_epoch, epoch = epoch_raw & 0x3fffffffu;
+    if (pt == 0) {
+        const int t0k = (int)atomicAdd(&hdr->ticket, 1u);
+        s_ticket[pipe][0] = t0k;
+        if (t0k < total) load_chunk(t0k, 0);
+    }
+    pipe_sync();
 
     for (int it = 0;; ++it) {
         const int st = it & 1;
-        const int ticket = s_ticket[st];
+        const int ticket = s_ticket[pipe][st];
         if (ticket >= total) break;
-        // prefetch the next chunk into the other stage (its previous contents were consumed
-        // by the previous iteration, which ended with a block-wide barrier)
-        if (tid == 0) {
+        // prefetch the next chunk into the other stage (consumed by the previous iteration,
+        // which ended with a pipeline barrier)
+        if (pt == 0) {
             const int nt = (int)atomicAdd(&hdr->ticket, 1u);
-            s_ticket[st ^ 1] = nt;
+            s_ticket[pipe][st ^ 1] = nt;
             if (nt < total) load_chunk(nt, st ^ 1);
         }
         const int c = ticket / p.BH, bh = ticket % p.BH;     // chunk-major order
@@ -154,8 +170,8 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
         const size_t chunk_id = (size_t)bh * p.nchunks + c;
         const size_t row0 = (size_t)bh * p.T + t0;
         const bool publish = c != p.fault_chunk;            // false only under the test hook
-        const uint8_t *sa = smem + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
-        mbar_wait_bounded(&bar[st], (it >> 1) & 1, hdr, 0x100u);
+        const uint8_t *sa = pbase + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
+        mbar_wait_bounded(&bar[pipe][st], (it >> 1) & 1, hdr, 0x100u);
 
         // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate
         float G[R][VEC], OG[R][VEC];
@@ -211,58 +227,91 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
 #pragma unroll
             for (int j = 0; j < VEC; ++j) {
                 const int ch = cl * VEC + j;
-                sw[(warp * 3 + 0) * DH + ch] = A[j];
-                sw[(warp * 3 + 1) * DH + ch] = Bk[j];
-                sw[(warp * 3 + 2) * DH + ch] = Bv[j];
+                sw[(pwarp * 3 + 0) * DH + ch] = A[j];
+                sw[(pwarp * 3 + 1) * DH + ch] = Bk[j];
+                sw[(pwarp * 3 + 2) * DH + ch] = Bv[j];
             }
         }
-        __syncthreads();
+        pipe_sync();
 
-        // ---- chunk aggregate, look-back and carries: one thread per channel
-        if (tid < DH) {
-            const int ch = tid;
-            float cA = 1.f, cK = 0.f, cV = 0.f;
+        // ---- chunk aggregate (one thread per channel), published for the successors
+        float cA = 1.f, cK = 0.f, cV = 0.f;
+        if (pt < DH) {
+            const int ch = pt;
 #pragma unroll
-            for (int w = 0; w < C::NW; ++w) {
+            for (int w = 0; w < C::PW; ++w) {
                 const float a = sw[(w * 3 + 0) * DH + ch];
                 cK = fmaf(a, cK, sw[(w * 3 + 1) * DH + ch]);
                 cV = fmaf(a, cV, sw[(w * 3 + 2) * DH + ch]);
                 cA *= a;
             }
-            float *agg = p.agg + chunk_id * 3 * DH;
-            float *pre = p.pre + chunk_id * 2 * DH;
             if (c > 0) {
+                float *agg = p.agg + chunk_id * 3 * DH;
                 agg[ch] = cA;
                 agg[DH + ch] = cK;
                 agg[2 * DH + ch] = cV;
                 __threadfence();
-                asm volatile("bar.sync 1, %0;" :: "r"(DH) : "memory");
-                if (tid == 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 1u);
             }
-            float Hk = 0.f, Hv = 0.f;     // state entering this chunk
+        }
+        pipe_sync();
+        if (pt == 0 && c > 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 1u);
+
+        // ---- look-back by the pipeline's first warp: state entering this chunk -> sH
+        if (pwarp == 0) {
+            constexpr int CPL = DH / 32;              // channels per lane
+            float Hk[CPL], Hv[CPL];
             if (c == 0) {
-                if (p.h0k) Hk = p.h0k[(size_t)bh * DH + ch];
-                if (p.h0v) Hv = p.h0v[(size_t)bh * DH + ch];
+#pragma unroll
+                for (int u = 0; u < CPL; ++u) {
+                    const int ch = lane + 32 * u;
+                    Hk[u] = p.h0k ? p.h0k[(size_t)bh * DH + ch] : 0.f;
+                    Hv[u] = p.h0v ? p.h0v[(size_t)bh * DH + ch] : 0.f;
+                }
             } else {
-                float xA = 1.f, xK = 0.f, xV = 0.f;   // composition of chunks j+1 .. c-1
+                float xA[CPL], xK[CPL], xV[CPL];      // composition of chunks j+1 .. c-1
+#pragma unroll
+                for (int u = 0; u < CPL; ++u) { xA[u] = 1.f; xK[u] = 0.f; xV[u] = 0.f; Hk[u] = 0.f; Hv[u] = 0.f; }
                 for (int j = c - 1; j >= 0; --j) {
                     const size_t jid = (size_t)bh * p.nchunks + j;
-                    const uint32_t s = wait_flag(p.flags + jid, epoch, p.wait_ns, hdr, 0x200u);
+                    uint32_t s = 0;
+                    if (lane == 0) s = wait_flag(p.flags + jid, epoch, p.wait_ns, hdr, 0x200u);
+                    s = __shfl_sync(0xffffffffu, s, 0);
+                    __syncwarp();
                     if (s == 2u) {
                         const float *pj = p.pre + jid * 2 * DH;
-                        Hk = fmaf(xA, __ldcg(pj + ch), xK);
-                        Hv = fmaf(xA, __ldcg(pj + DH + ch), xV);
+#pragma unroll
+                        for (int u = 0; u < CPL; ++u) {
+                            Hk[u] = fmaf(xA[u], __ldcg(pj + lane + 32 * u), xK[u]);
+                            Hv[u] = fmaf(xA[u], __ldcg(pj + DH + lane + 32 * u), xV[u]);
+                        }
                         break;
                     }
                     if (s == 0u) break;          // timed out: error recorded, carry zero
                     const float *aj = p.agg + jid * 3 * DH;
-                    const float a = __ldcg(aj + ch);
-                    xK = fmaf(xA, __ldcg(aj + DH + ch), xK);
-                    xV = fmaf(xA, __ldcg(aj + 2 * DH + ch), xV);
-                    xA *= a;
+#pragma unroll
+                    for (int u = 0; u < CPL; ++u) {
+                        const int ch = lane + 32 * u;
+                        const float a = __ldcg(aj + ch);
+                        xK[u] = fmaf(xA[u], __ldcg(aj + DH + ch), xK[u]);
+                        xV[u] = fmaf(xA[u], __ldcg(aj + 2 * DH + ch), xV[u]);
+                        xA[u] *= a;
+                    }
                 }
             }
+#pragma unroll
+            for (int u = 0; u < CPL; ++u) {
+                sH[lane + 32 * u] = Hk[u];
+                sH[DH + lane + 32 * u] = Hv[u];
+            }
+        }
+        pipe_sync();
+
+        // ---- inclusive state after the chunk (published) and carries entering each warp
+        if (pt < DH) {
+            const int ch = pt;
+            const float Hk = sH[ch], Hv = sH[DH + ch];
             const float outK = fmaf(cA, Hk, cK), outV = fmaf(cA, Hv, cV);
+            float *pre = p.pre + chunk_id * 2 * DH;
             pre[ch] = outK;
             pre[DH + ch] = outV;
             if (c == p.nchunks - 1) {
@@ -270,10 +319,9 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
                 if (p.hTv) p.hTv[(size_t)bh * DH + ch] = outV;
             }
             __threadfence();
-            // carries entering each warp, written over that warp's aggregate
             float hK = Hk, hV = Hv;
 #pragma unroll
-            for (int w = 0; w < C::NW; ++w) {
+            for (int w = 0; w < C::PW; ++w) {
                 const float a = sw[(w * 3 + 0) * DH + ch];
                 const float bk = sw[(w * 3 + 1) * DH + ch];
                 const float bv = sw[(w * 3 + 2) * DH + ch];
@@ -282,10 +330,9 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
                 hK = fmaf(a, hK, bk);
                 hV = fmaf(a, hV, bv);
             }
-            asm volatile("bar.sync 1, %0;" :: "r"(DH) : "memory");
-            if (tid == 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 2u);
         }
-        __syncthreads();
+        pipe_sync();
+        if (pt == 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 2u);
 
         // ---- pass 2: rerun the recurrence from the carry with the kept gates; write k~
         // (optionally rotated) and v~
@@ -293,7 +340,7 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
 #pragma unroll
         for (int j = 0; j < VEC; ++j) {
             const int ch = cl * VEC + j;
-            const float wk = sw[(warp * 3 + 0) * DH + ch], wv = sw[(warp * 3 + 1) * DH + ch];
+            const float wk = sw[(pwarp * 3 + 0) * DH + ch], wv = sw[(pwarp * 3 + 1) * DH + ch];
             hk[j] = fmaf(eA[j], wk, eK[j]);
             hv[j] = fmaf(eA[j], wv, eV[j]);
         }
@@ -350,13 +397,13 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
                 Vec<E>::store(yv + go, hv);
             }
         }
-        __syncthreads();     // this stage's smem and sw are free for the next chunk
+        pipe_sync();     // this stage's smem and sw are free for the next chunk
     }
 
-    // ---- launch bookkeeping: the last CTA resets the ticket counter and bumps the epoch
-    if (tid == 0) {
+    // ---- launch bookkeeping: the last pipeline resets the ticket counter and bumps the epoch
+    if (pt == 0) {
         __threadfence();
-        if (atomicAdd(&hdr->done, 1u) == gridDim.x - 1) {
+        if (atomicAdd(&hdr->done, 1u) == gridDim.x * C::NPIPE - 1) {
             hdr->ticket = 0;
             hdr->done = 0;
             __threadfence();
@@ -367,7 +414,7 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
 
 int recur_chunk_rows(int d, int dtype) {
     const int eb = dtype == RAT_F32 ? 4 : 2;
-    return (256 / (d * eb / 16)) * 8;
+    return (128 / (d * eb / 16)) * 8;      // (threads per pipeline / lanes per row) x 8 rows
 }
 
 size_t recur_workspace_bytes(int BH, int T, int d, int dtype) {

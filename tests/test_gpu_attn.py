@@ -98,9 +98,11 @@ def test_bf16_d64():
     check_attn(q, k, v, D=4, W=3)
 
 
-def test_bf16_rope_query(block_keys):
+@pytest.mark.parametrize("pos0", [3000, 100000])    # float32 angles below 2^13, float64 above
+def test_bf16_rope_query(block_keys, pos0):
     q, k, v = qkv(1, 2, 700, 128, torch.bfloat16, seed=77)
-    check_attn(q, k, v, D=16, W=0, rope_base=10000.0, pos0=3000)
+    check_attn(q, k, v, D=16, W=0, rope_base=10000.0, pos0=pos0)
+    check_attn(q, k, v, D=4, W=9, rope_base=10000.0, pos0=pos0)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
