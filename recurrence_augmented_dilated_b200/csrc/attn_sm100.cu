@@ -162,17 +162,6 @@ RAT_DEVICE void rope_cs_fast(long long pos, double theta, float &c, float &s) {
     __sincosf((float)r, &s, &c);
 }
 
-// Same with a float32 angle; used while pos * theta stays below 2^13 rad, where the float32
-// product is within 2.5e-4 rad of the exact angle (a bf16 query carries 4e-3 relative error).
-RAT_DEVICE void rope_cs_f32(int pos, float theta, float &c, float &s) {
-    const float kTwoPiHi = 6.28318548f, kTwoPiLo = -1.7484555e-7f;   // 2*pi = hi + lo
-    const float ang = (float)pos * theta;
-    const float n = rintf(ang * 0.159154943f);
-    float r = fmaf(-n, kTwoPiHi, ang);
-    r = fmaf(-n, kTwoPiLo, r);
-    __sincosf(r, &s, &c);
-}
-
 RAT_DEVICE uint32_t swz(uint32_t row, uint32_t chunk) {   // 128B swizzle inside a sub-tile
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }

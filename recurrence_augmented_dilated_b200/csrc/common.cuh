@@ -64,7 +64,27 @@ RAT_DEVICE void rope_cs(long long pos, double theta, float &c, float &s) {
     sincosf((float)r, &s, &c);
 }
 
+// Same with a float32 angle, for positions where pos * theta stays below 2^13 rad: the float32
+// product is then within 2.5e-4 rad of the exact angle, reduced by a two-term float 2*pi, and the
+// special-function-unit sincos is accurate to ~1e-6 on [-pi, pi].  Used only for bf16 outputs.
+RAT_DEVICE void rope_cs_f32(int pos, float theta, float &c, float &s) {
+    const float kTwoPiHi = 6.28318548f, kTwoPiLo = -1.7484555e-7f;   // 2*pi = hi + lo
+    const float ang = (float)pos * theta;
+    const float n = rintf(ang * 0.159154943f);
+    float r = fmaf(-n, kTwoPiHi, ang);
+    r = fmaf(-n, kTwoPiLo, r);
+    __sincosf(r, &s, &c);
+}
+
 // ------------------------------------------------------------------------------ memory order
+RAT_DEVICE uint64_t ld_relaxed_gpu_u64(const uint64_t *p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+RAT_DEVICE void st_relaxed_gpu_u64(uint64_t *p, uint64_t v) {
+    asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
+}
 RAT_DEVICE uint32_t ld_acquire_gpu(const uint32_t *p) {
     uint32_t v;
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");

@@ -81,16 +81,18 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j] = 0.f;
 
-    // keys of this split: lane set s = warp*GPW + grp takes keys k_lo + s + m*kLanesets, two at a
-    // time.  The loop runs on the warp's first key so every lane of a warp iterates the same
-    // number of times (the dot-product shuffles below need all 32 lanes).
+    // keys of this split: lane set s = warp*GPW + grp takes keys k_lo + s + m*kLanesets, KPI at a
+    // time (their K and V rows in flight together, kept as packed bf16).  The loop runs on the
+    // warp's first key so every lane of a warp iterates the same number of times (the
+    // dot-product shuffles below need all 32 lanes).
     constexpr int kLanesets = kWarps * GPW;
+    constexpr int KPI = 4;
     const int set = warp * GPW + grp;
-    for (long long base = k_lo + warp * GPW; base < k_hi; base += 2 * kLanesets) {
-        float kx[2][8], vx[2][8];
-        bool have[2];
+    for (long long base = k_lo + warp * GPW; base < k_hi; base += KPI * kLanesets) {
+        uint4 kr[KPI], vr[KPI];
+        bool have[KPI];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
+        for (int u = 0; u < KPI; ++u) {
             const long long idx = base + grp + (long long)u * kLanesets;
             have[u] = idx < k_hi;
             // lanes of a warp may disagree on `have`; loads are predicated, shuffles are not
@@ -104,30 +106,47 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                     kp = kwin + (size_t)(pos % p.W) * RB;
                     vp = vwin + (size_t)(pos % p.W) * RB;
                 }
-                load8(kp + cl * 16, kx[u]);
-                load8(vp + cl * 16, vx[u]);
+                kr[u] = __ldg(reinterpret_cast<const uint4 *>(kp + cl * 16));
+                vr[u] = __ldg(reinterpret_cast<const uint4 *>(vp + cl * 16));
             } else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) { kx[u][j] = 0.f; vx[u][j] = 0.f; }
+                kr[u] = make_uint4(0u, 0u, 0u, 0u);
+                vr[u] = kr[u];
             }
         }
+        float sc[KPI];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            // the dot-product shuffle needs every lane of the warp: compute, then discard
+        for (int u = 0; u < KPI; ++u) {
+            const uint32_t ku[4] = {kr[u].x, kr[u].y, kr[u].z, kr[u].w};
             float dot = 0.f;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) dot = fmaf(q[j], kx[u][j], dot);
+            for (int i = 0; i < 4; ++i) {
+                dot = fmaf(q[2 * i], bf16_lo(ku[i]), dot);
+                dot = fmaf(q[2 * i + 1], bf16_hi(ku[i]), dot);
+            }
 #pragma unroll
             for (int off = LPR / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-            if (have[u]) {
-                const float s = dot * p.scale_log2;
-                const float mn = fmaxf(m, s);
-                const float corr = exp2f(m - mn), pj = exp2f(s - mn);
-                l = fmaf(l, corr, pj);
+            sc[u] = have[u] ? dot * p.scale_log2 : -INFINITY;
+        }
+        // one rescale for the KPI keys
+        const float mb = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+        const float mn = fmaxf(m, mb);
+        if (mn != -INFINITY) {
+            const float corr = ex2_approx(m - mn);        // m = -inf -> 0
+            l *= corr;
 #pragma unroll
-                for (int j = 0; j < 8; ++j) o[j] = fmaf(o[j], corr, pj * vx[u][j]);
-                m = mn;
+            for (int j = 0; j < 8; ++j) o[j] *= corr;
+#pragma unroll
+            for (int u = 0; u < KPI; ++u) {
+                const float pj = ex2_approx(sc[u] - mn);   // masked keys: -inf -> 0
+                l += pj;
+                const uint32_t vu[4] = {vr[u].x, vr[u].y, vr[u].z, vr[u].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    o[2 * i] = fmaf(pj, bf16_lo(vu[i]), o[2 * i]);
+                    o[2 * i + 1] = fmaf(pj, bf16_hi(vu[i]), o[2 * i + 1]);
+                }
             }
+            m = mn;
         }
     }
 
@@ -247,15 +266,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 }
 
 int decode_splits(int B, int H, int Tcap, const int32_t *Dh, int W) {
-    // aim for about 8 CTAs per SM over the 148 SMs, and at least ~128 keys per split
+    // aim for about 24 CTAs per SM over the 148 SMs, and at least ~64 keys per split
     long long max_keys = 0;
     for (int h = 0; h < H; ++h) {
         const long long k = Tcap / Dh[h] + W;
         max_keys = k > max_keys ? k : max_keys;
     }
     const long long bh = (long long)B * H;
-    long long s = (148ll * 8 + bh - 1) / bh;
-    const long long by_keys = (max_keys + 127) / 128;
+    long long s = (148ll * 24 + bh - 1) / bh;
+    const long long by_keys = (max_keys + 63) / 64;
     if (s > by_keys) s = by_keys;
     if (s < 1) s = 1;
     if (s > 64) s = 64;

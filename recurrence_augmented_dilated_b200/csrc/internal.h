@@ -34,9 +34,12 @@ struct RecurParams {
     long long pos0;
     int rope;                   // 1: rotate k~
     WsHeader *hdr;
-    uint32_t *flags;            // [BH * nchunks]
-    float *agg;                 // [BH * nchunks][3][d]   A, Bk, Bv of the chunk
-    float *pre;                 // [BH * nchunks][2][d]   inclusive state Hk, Hv after the chunk
+    // look-back records, one 64-bit word per value: (launch tag << 32) | float bits, so every
+    // value validates itself and needs no separate flag or fence
+    uint64_t *agg;              // [BH * nchunks][3][d]   A, Bk, Bv of the chunk
+    uint64_t *pre;              // [BH * nchunks][2][d]   inclusive state Hk, Hv after the chunk
+    int rope_f32;               // positions small enough for float32 angles (pos0 + T <= 2^13)
+    float theta_f[64];
     double theta[64];           // RoPE frequency theta_c = base^(-2c/d), c < d/2
     float step_cos[64], step_sin[64];   // cos/sin(theta_c): one-position rotation
     long long fault_chunk;      // test hook: chunk index that never publishes (-1: none)

@@ -143,15 +143,16 @@ int rat_recur_prefill(const void *k, const void *v, const void *gate_logit, cons
     uint8_t *w = static_cast<uint8_t *>(ws);
     const size_t nch = (size_t)p.BH * p.nchunks;
     p.hdr = reinterpret_cast<WsHeader *>(w);
-    p.flags = reinterpret_cast<uint32_t *>(w + sizeof(WsHeader));
-    p.agg = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256(nch * 4));
-    p.pre = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256(nch * 4) + align256(nch * 3 * d * 4));
+    p.agg = reinterpret_cast<uint64_t *>(w + sizeof(WsHeader));
+    p.pre = reinterpret_cast<uint64_t *>(w + sizeof(WsHeader) + align256(nch * 3 * d * 8));
     if (p.rope) {
         rope_theta(rope_base, d, p.theta);
         for (int c = 0; c < 64; ++c) {
+            p.theta_f[c] = (float)p.theta[c];
             p.step_cos[c] = (float)std::cos(p.theta[c]);
             p.step_sin[c] = (float)std::sin(p.theta[c]);
         }
+        p.rope_f32 = (dtype == RAT_BF16 && pos0 + (int64_t)T <= 8192) ? 1 : 0;
     }
     return launch_recur(p, dtype, stream);
 }

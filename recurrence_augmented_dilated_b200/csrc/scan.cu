@@ -84,21 +84,25 @@ template <> struct Vec<__nv_bfloat16> {
     }
 };
 
-// Spin (bounded) until flag f carries this launch's epoch and a non-zero state.
-// Returns the state (1 = aggregate, 2 = inclusive prefix) or 0 if the wait ran out.
-RAT_DEVICE uint32_t wait_flag(const uint32_t *f, uint32_t epoch, uint64_t limit_ns, WsHeader *hdr,
-                              uint32_t where) {
-    uint32_t v = ld_acquire_gpu(f);
-    if ((v >> 2) == epoch && (v & 3u)) return v & 3u;
-    uint64_t t0 = globaltimer_ns();
+// Look-back records: each value is one 64-bit word, (tag << 32) | float bits, written with a
+// single relaxed store; a reader accepts a word only when its tag is this launch's tag, so a
+// value and its validity always travel together.
+RAT_DEVICE uint64_t tagged(uint32_t tag, float v) { return ((uint64_t)tag << 32) | __float_as_uint(v); }
+
+// Wait (bounded) for the tagged word at w; returns false if the wait ran out.
+RAT_DEVICE bool wait_word(const uint64_t *w, uint32_t tag, float &v, uint64_t t_start, uint64_t limit_ns,
+                          WsHeader *hdr) {
     for (;;) {
-        __nanosleep(32);
-        v = ld_acquire_gpu(f);
-        if ((v >> 2) == epoch && (v & 3u)) return v & 3u;
-        if (globaltimer_ns() - t0 > limit_ns) {
-            record_error(hdr, RAT_ERR_TIMEOUT, where);
-            return 0;
+        const uint64_t x = ld_relaxed_gpu_u64(w);
+        if ((uint32_t)(x >> 32) == tag) {
+            v = __uint_as_float((uint32_t)x);
+            return true;
         }
+        if (globaltimer_ns() - t_start > limit_ns) {
+            record_error(hdr, RAT_ERR_TIMEOUT, 0x200u);
+            return false;
+        }
+        __nanosleep(20);
     }
 }
 
@@ -145,7 +149,8 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
         fence_mbar_init();
     }
     __syncthreads();
-    const uint32_t epoch_raw = s_epoch, epoch = epoch_raw & 0x3fffffffu;
+    const uint32_t epoch_raw = s_epoch;
+    const uint32_t tag = (epoch_raw & 0x7fffffffu) | 0x80000000u;   // never 0: a zeroed workspace never matches
     if (pt == 0) {
         const int t0k = (int)atomicAdd(&hdr->ticket, 1u);
         s_ticket[pipe][0] = t0k;
@@ -234,10 +239,11 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
         }
         pipe_sync();
 
-        // ---- chunk aggregate (one thread per channel), published for the successors
-        float cA = 1.f, cK = 0.f, cV = 0.f;
+        // ---- one thread per channel: chunk aggregate (published), look-back for the state
+        // entering the chunk, inclusive state (published), carries entering each warp
         if (pt < DH) {
             const int ch = pt;
+            float cA = 1.f, cK = 0.f, cV = 0.f;
 #pragma unroll
             for (int w = 0; w < C::PW; ++w) {
                 const float a = sw[(w * 3 + 0) * DH + ch];
@@ -245,80 +251,64 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
                 cV = fmaf(a, cV, sw[(w * 3 + 2) * DH + ch]);
                 cA *= a;
             }
-            if (c > 0) {
-                float *agg = p.agg + chunk_id * 3 * DH;
-                agg[ch] = cA;
-                agg[DH + ch] = cK;
-                agg[2 * DH + ch] = cV;
-                __threadfence();
+            if (c > 0 && publish) {
+                uint64_t *agg = p.agg + chunk_id * 3 * DH;
+                st_relaxed_gpu_u64(agg + ch, tagged(tag, cA));
+                st_relaxed_gpu_u64(agg + DH + ch, tagged(tag, cK));
+                st_relaxed_gpu_u64(agg + 2 * DH + ch, tagged(tag, cV));
             }
-        }
-        pipe_sync();
-        if (pt == 0 && c > 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 1u);
-
-        // ---- look-back by the pipeline's first warp: state entering this chunk -> sH
-        if (pwarp == 0) {
-            constexpr int CPL = DH / 32;              // channels per lane
-            float Hk[CPL], Hv[CPL];
+            float Hk = 0.f, Hv = 0.f;     // state entering this chunk
             if (c == 0) {
-#pragma unroll
-                for (int u = 0; u < CPL; ++u) {
-                    const int ch = lane + 32 * u;
-                    Hk[u] = p.h0k ? p.h0k[(size_t)bh * DH + ch] : 0.f;
-                    Hv[u] = p.h0v ? p.h0v[(size_t)bh * DH + ch] : 0.f;
-                }
+                if (p.h0k) Hk = p.h0k[(size_t)bh * DH + ch];
+                if (p.h0v) Hv = p.h0v[(size_t)bh * DH + ch];
             } else {
-                float xA[CPL], xK[CPL], xV[CPL];      // composition of chunks j+1 .. c-1
-#pragma unroll
-                for (int u = 0; u < CPL; ++u) { xA[u] = 1.f; xK[u] = 0.f; xV[u] = 0.f; Hk[u] = 0.f; Hv[u] = 0.f; }
-                for (int j = c - 1; j >= 0; --j) {
+                float xA = 1.f, xK = 0.f, xV = 0.f;   // composition of chunks j+1 .. c-1
+                const uint64_t t_start = globaltimer_ns();
+                bool alive = true;
+                for (int j = c - 1; j >= 0 && alive; --j) {
                     const size_t jid = (size_t)bh * p.nchunks + j;
-                    uint32_t s = 0;
-                    if (lane == 0) s = wait_flag(p.flags + jid, epoch, p.wait_ns, hdr, 0x200u);
-                    s = __shfl_sync(0xffffffffu, s, 0);
-                    __syncwarp();
-                    if (s == 2u) {
-                        const float *pj = p.pre + jid * 2 * DH;
-#pragma unroll
-                        for (int u = 0; u < CPL; ++u) {
-                            Hk[u] = fmaf(xA[u], __ldcg(pj + lane + 32 * u), xK[u]);
-                            Hv[u] = fmaf(xA[u], __ldcg(pj + DH + lane + 32 * u), xV[u]);
+                    const uint64_t *pj = p.pre + jid * 2 * DH;
+                    const uint64_t *aj = p.agg + jid * 3 * DH;
+                    // predecessor j: its inclusive state if published, else its aggregate
+                    for (;;) {
+                        const uint64_t x = ld_relaxed_gpu_u64(pj + ch);
+                        if ((uint32_t)(x >> 32) == tag) {
+                            float hv;
+                            alive = wait_word(pj + DH + ch, tag, hv, t_start, p.wait_ns, hdr);
+                            Hk = fmaf(xA, __uint_as_float((uint32_t)x), xK);
+                            Hv = fmaf(xA, hv, xV);
+                            j = -1;                         // done
+                            break;
                         }
-                        break;
-                    }
-                    if (s == 0u) break;          // timed out: error recorded, carry zero
-                    const float *aj = p.agg + jid * 3 * DH;
-#pragma unroll
-                    for (int u = 0; u < CPL; ++u) {
-                        const int ch = lane + 32 * u;
-                        const float a = __ldcg(aj + ch);
-                        xK[u] = fmaf(xA[u], __ldcg(aj + DH + ch), xK[u]);
-                        xV[u] = fmaf(xA[u], __ldcg(aj + 2 * DH + ch), xV[u]);
-                        xA[u] *= a;
+                        const uint64_t y = ld_relaxed_gpu_u64(aj + ch);
+                        if ((uint32_t)(y >> 32) == tag) {
+                            float bk, bv;
+                            alive = wait_word(aj + DH + ch, tag, bk, t_start, p.wait_ns, hdr) &&
+                                    wait_word(aj + 2 * DH + ch, tag, bv, t_start, p.wait_ns, hdr);
+                            xK = fmaf(xA, bk, xK);
+                            xV = fmaf(xA, bv, xV);
+                            xA *= __uint_as_float((uint32_t)y);
+                            break;                          // next predecessor
+                        }
+                        if (globaltimer_ns() - t_start > p.wait_ns) {
+                            record_error(hdr, RAT_ERR_TIMEOUT, 0x200u);
+                            alive = false;                  // carry zero; error recorded
+                            break;
+                        }
+                        __nanosleep(20);
                     }
                 }
             }
-#pragma unroll
-            for (int u = 0; u < CPL; ++u) {
-                sH[lane + 32 * u] = Hk[u];
-                sH[DH + lane + 32 * u] = Hv[u];
-            }
-        }
-        pipe_sync();
-
-        // ---- inclusive state after the chunk (published) and carries entering each warp
-        if (pt < DH) {
-            const int ch = pt;
-            const float Hk = sH[ch], Hv = sH[DH + ch];
             const float outK = fmaf(cA, Hk, cK), outV = fmaf(cA, Hv, cV);
-            float *pre = p.pre + chunk_id * 2 * DH;
-            pre[ch] = outK;
-            pre[DH + ch] = outV;
+            if (publish) {
+                uint64_t *pre = p.pre + chunk_id * 2 * DH;
+                st_relaxed_gpu_u64(pre + ch, tagged(tag, outK));
+                st_relaxed_gpu_u64(pre + DH + ch, tagged(tag, outV));
+            }
             if (c == p.nchunks - 1) {
                 if (p.hTk) p.hTk[(size_t)bh * DH + ch] = outK;
                 if (p.hTv) p.hTv[(size_t)bh * DH + ch] = outV;
             }
-            __threadfence();
             float hK = Hk, hV = Hv;
 #pragma unroll
             for (int w = 0; w < C::PW; ++w) {
@@ -332,7 +322,6 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
             }
         }
         pipe_sync();
-        if (pt == 0 && publish) st_release_gpu(p.flags + chunk_id, (epoch << 2) | 2u);
 
         // ---- pass 2: rerun the recurrence from the carry with the kept gates; write k~
         // (optionally rotated) and v~
@@ -351,7 +340,8 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
 #pragma unroll
             for (int j = 0; j < VEC; ++j) {
                 const int f = (cl * VEC + j) % (DH / 2);
-                rope_cs(pos, p.theta[f], rc[j], rs[j]);
+                if (p.rope_f32) rope_cs_f32((int)pos, p.theta_f[f], rc[j], rs[j]);
+                else rope_cs(pos, p.theta[f], rc[j], rs[j]);
                 sc[j] = p.step_cos[f];
                 ss[j] = first_half ? -p.step_sin[f] : p.step_sin[f];
                 if (first_half) rs[j] = -rs[j];      // first half: x cos - x' sin
@@ -420,7 +410,7 @@ int recur_chunk_rows(int d, int dtype) {
 size_t recur_workspace_bytes(int BH, int T, int d, int dtype) {
     const size_t tc = (size_t)recur_chunk_rows(d, dtype);
     const size_t nch = (size_t)BH * ((T + tc - 1) / tc);
-    return sizeof(WsHeader) + align256(nch * 4) + align256(nch * 3 * d * 4) + align256(nch * 2 * d * 4);
+    return sizeof(WsHeader) + align256(nch * 3 * d * 8) + align256(nch * 2 * d * 8);
 }
 
 template <typename E, int DH>
