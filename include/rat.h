@@ -147,6 +147,16 @@ RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const voi
  * attention kernel since the last call (RAT_OK if none). */
 RAT_API int rat_attn_sync_status(void *stream);
 
+/* Diagnostic: where the attention kernel's last recorded timeout happened, as
+ * (wait site << 24) | (key block << 8) | phase parity; sites: 1 producer stage-free, 2 MMA
+ * query-ready, 3 MMA stage-full, 4 MMA previous-PV, 5 MMA probabilities-ready, 6 softmax
+ * query-loaded, 7 softmax scores-ready, 8 softmax rescale, 9 epilogue.  0 if none. */
+RAT_API uint32_t rat_attn_error_site(void);
+
+/* Diagnostic: bit s set when a wait at site s (numbering as above) was still in progress when a
+ * CTA of the attention kernel aborted after a timeout. */
+RAT_API uint32_t rat_attn_error_waiting(void);
+
 /* Tuning knob of the bf16 tensor-core attention: keys per block, 64 (two CTAs per SM) or 128
  * (one CTA per SM); 0 restores the automatic choice.  Process-wide; RAT_ERR_INVALID otherwise. */
 RAT_API int rat_set_attn_block_keys(int block_keys);

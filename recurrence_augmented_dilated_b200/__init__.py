@@ -87,6 +87,8 @@ def lib():
         L.rat_dilated_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(KVCache), _vp,
                                                  _f, _f, _vp]
         L.rat_attn_sync_status.argtypes = [_vp]
+        L.rat_attn_error_site.restype = ctypes.c_uint32
+        L.rat_attn_error_waiting.restype = ctypes.c_uint32
         L.rat_set_attn_block_keys.argtypes = [_i]
         L.rat_attended_keys.restype = _i64
         L.rat_attended_keys.argtypes = [_i64, _i, _i]

@@ -32,6 +32,8 @@
 namespace rat {
 
 __device__ int g_attn_error;     // first device-side error of the attention kernel
+__device__ unsigned g_attn_where; // where it happened: (site << 24) | (block << 8) | parity
+__device__ unsigned g_attn_waiting; // bit s set: a wait at site s was in progress when a CTA aborted
 
 namespace {
 
@@ -48,14 +50,14 @@ template <int BN>
 struct Cfg {
     static constexpr uint32_t KSUB = BN * 128;          // [BN keys][64 bf16] sub-tile
     static constexpr uint32_t KTILE = 2 * KSUB;         // one K (or V) block: two d-halves
-    static constexpr uint32_t PSUB = BM * 128;          // [128 rows][64 keys] sub-tile of P
     static constexpr uint32_t OFF_Q = 0;
     static constexpr uint32_t OFF_K = OFF_Q + 2 * QSUB;
     static constexpr uint32_t OFF_V = OFF_K + NS * KTILE;
-    static constexpr uint32_t OFF_P = OFF_V + NS * KTILE;
-    static constexpr uint32_t OFF_BAR = OFF_P + (BN / 64) * PSUB;
+    static constexpr uint32_t OFF_BAR = OFF_V + NS * KTILE;
     static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
-    static constexpr uint32_t COL_S1 = BN;              // S buffers at columns 0 and BN
+    static constexpr uint32_t COL_S1 = BN;              // S buffers at columns 0 and BN; the bf16
+                                                        // P of a block overwrites the first BN/2
+                                                        // columns of its S buffer
     static constexpr uint32_t COL_O = 2 * BN;           // O: 128 columns after them
     static constexpr uint32_t TMEM_COLS = BN == 64 ? 256 : 512;
     static constexpr int MIN_CTAS = BN == 64 ? 2 : 1;   // CTAs resident per SM
@@ -131,21 +133,26 @@ RAT_DEVICE void block_range(const Plan &pl, int j, int t, int &c_lo, int &c_hi) 
 }
 
 struct Shared {
-    uint64_t q_full, q_ready, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full, o_ready, fin;
+    uint64_t q_full, q_ready, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_ready[2], fin;
     uint32_t tmem;
     volatile int abort;
 };
 
-// Bounded mbarrier wait that also gives up as soon as another role aborted.
-RAT_DEVICE bool wait_bar(Shared &sh, uint64_t *bar, uint32_t parity) {
+// Bounded mbarrier wait that also gives up as soon as another role aborted; an expired wait
+// records RAT_ERR_TIMEOUT and its site (see g_attn_where).
+RAT_DEVICE bool wait_bar(Shared &sh, uint64_t *bar, uint32_t parity, uint32_t site = 0, uint32_t blk = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (sh.abort) return false;
+        if (sh.abort) {
+            atomicOr(&g_attn_waiting, 1u << site);
+            return false;
+        }
         if (globaltimer_ns() - t0 > kWaitLimitNs) {
             sh.abort = 1;
-            atomicCAS(&g_attn_error, 0, RAT_ERR_TIMEOUT);
+            if (atomicCAS(&g_attn_error, 0, RAT_ERR_TIMEOUT) == 0)
+                g_attn_where = (site << 24) | ((blk & 0xffffu) << 8) | parity;
             return false;
         }
     }
@@ -201,12 +208,13 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             mbar_init(&sh.kv_full[s], 1);
             mbar_init(&sh.kv_empty[s], 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&sh.s_full[s], 1);
-            mbar_init(&sh.s_free[s], 128);
-        }
-        mbar_init(&sh.p_full, 128);
-        mbar_init(&sh.o_ready, 1);
+        for (int s = 0; s < 2; ++s) mbar_init(&sh.s_full[s], 1);
+        // P of even / odd blocks: the softmax may finish block j while the MMA has not yet
+        // consumed block j-1, but never block j+2 (that needs S(j+2), issued after PV(j))
+        mbar_init(&sh.p_full[0], 128);
+        mbar_init(&sh.p_full[1], 128);
+        mbar_init(&sh.o_ready[0], 1);     // PV of even blocks
+        mbar_init(&sh.o_ready[1], 1);     // PV of odd blocks
         mbar_init(&sh.fin, 1);
         sh.abort = 0;
         fence_mbar_init();
@@ -231,7 +239,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             int issued = 0;
             for (int j = 0; j < nb; ++j) {
                 const int s = j % NS;
-                if (j >= NS && !wait_bar(sh, &sh.kv_empty[s], ((j / NS) - 1) & 1)) break;
+                if (j >= NS && !wait_bar(sh, &sh.kv_empty[s], ((j / NS) - 1) & 1, 1, j)) break;
                 const CUtensorMap *tk = j < pl.nd ? mk : &p.tm_k;
                 const CUtensorMap *tv = j < pl.nd ? mv : &p.tm_v;
                 const int y = j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd);
@@ -257,14 +265,15 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             constexpr uint32_t IDESC_QK = tc::idesc_bf16(BM, BN, 0);      // K^T: K-major B
             constexpr uint32_t IDESC_PV = tc::idesc_bf16(BM, DHEAD, 1);   // V: MN-major B
             const uint32_t sq = smem_u32(smem + C::OFF_Q);
-            const uint32_t sp = smem_u32(smem + C::OFF_P);
-            bool ok = wait_bar(sh, &sh.q_ready, 0);
+            bool ok = wait_bar(sh, &sh.q_ready, 0, 2);
             tc::fence_after_sync();
             for (int j = 0; ok && j <= nb; ++j) {
                 if (j < nb) {
                     const int s = j % NS, sb = j & 1;
-                    if (!wait_bar(sh, &sh.kv_full[s], (j / NS) & 1)) break;
-                    if (j >= 2 && !wait_bar(sh, &sh.s_free[sb], ((j >> 1) - 1) & 1)) break;
+                    if (!wait_bar(sh, &sh.kv_full[s], (j / NS) & 1, 3, j)) break;
+                    // S buffer sb holds P(j-2) until PV(j-2) has read it: wait for that PV to
+                    // complete (this thread issued it, so the barrier is at most one phase ahead)
+                    if (j >= 2 && !wait_bar(sh, &sh.o_ready[(j - 2) & 1], ((j - 2) >> 1) & 1, 4, j)) break;
                     tc::fence_after_sync();
                     const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::KTILE);
                     for (int kk = 0; kk < DHEAD / 16; ++kk) {
@@ -278,20 +287,20 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                 }
                 if (j >= 1) {
                     const int jp = j - 1, s = jp % NS;
-                    if (!wait_bar(sh, &sh.p_full, jp & 1)) break;
+                    if (!wait_bar(sh, &sh.p_full[jp & 1], (jp >> 1) & 1, 5, jp)) break;
                     tc::fence_after_sync();
                     const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KTILE);
+                    const uint32_t pcol = (jp & 1) * C::COL_S1;     // P of block jp, in TMEM
                     for (int kk = 0; kk < BN / 16; ++kk) {
-                        // A = P[:, 16kk .. 16kk+15]  (K-major, 128B swizzle, 64-key sub-tiles)
-                        const uint32_t aoff = (kk >> 2) * C::PSUB + (kk & 3) * 32;
+                        // A = P[:, 16kk .. 16kk+15]: 8 TMEM columns of packed bf16 pairs
                         // B = V[16kk .. 16kk+15, :]  (MN-major: the two 64-channel atoms KSUB apart,
                         // 8-key groups 1 KiB apart)
                         const uint32_t boff = kk * 16 * 128;
-                        tc::mma_bf16_ss(tmem + C::COL_O, tc::smem_desc_sw128(sp + aoff, 16, 1024),
+                        tc::mma_bf16_ts(tmem + C::COL_O, tmem + pcol + kk * 8,
                                         tc::smem_desc_sw128(sv + boff, C::KSUB, 1024), IDESC_PV,
                                         (jp > 0 || kk > 0) ? 1u : 0u);
                     }
-                    tc::mma_commit(&sh.o_ready);
+                    tc::mma_commit(&sh.o_ready[jp & 1]);
                     tc::mma_commit(&sh.kv_empty[s]);
                 }
             }
@@ -309,7 +318,6 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         const int t = t0 + r;
         const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
         uint8_t *sQ = smem + C::OFF_Q;
-        uint8_t *sP = smem + C::OFF_P;
         // the self key's row (W <= 1): issue its loads now so they overlap the Q load
         uint4 kself[16];
         const bool have_self = pl.self_reg && t < p.T;
@@ -320,12 +328,12 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             for (int c = 0; c < 16; ++c) kself[c] = __ldg(krow + c);
         }
         // waits are made warp-uniform: tcgen05.ld/st below are warp-collective
-        bool ok = __all_sync(0xffffffffu, wait_bar(sh, &sh.q_full, 0));
+        bool ok = __all_sync(0xffffffffu, wait_bar(sh, &sh.q_full, 0, 6));
         if (ok && p.rope) {
             // rotate-half RoPE of this row of Q at position pos0 + t: channel c (< 64) pairs with
             // c + 64, which sits at the same swizzled offset of the second sub-tile
             const long long pos = p.pos0 + t;
-#pragma unroll 1
+#pragma unroll
             for (int c = 0; c < 8; ++c) {
                 uint4 *p1 = reinterpret_cast<uint4 *>(sQ + swz(r, c));
                 uint4 *p2 = reinterpret_cast<uint4 *>(sQ + QSUB + swz(r, c));
@@ -379,14 +387,12 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         int jdone = 0;
         for (int j = 0; ok && j < nb; ++j) {
             const int sb = j & 1;
-            if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.s_full[sb], (j >> 1) & 1))) { ok = false; break; }
+            if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.s_full[sb], (j >> 1) & 1, 7, j))) { ok = false; break; }
             tc::fence_after_sync();
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c)
                 tc::tmem_ld32(tl + sb * C::COL_S1 + 32 * c, reinterpret_cast<uint32_t *>(sv) + 32 * c);
             tc::tmem_wait_ld();
-            tc::fence_before_sync();
-            mbar_arrive(&sh.s_free[sb]);
 
             int c_lo, c_hi;
             block_range<BN>(pl, j, t, c_lo, c_hi);
@@ -427,34 +433,34 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                 s8[c & 7] += e;
             }
             l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-            if (j > 0) {
-                // PV of the previous block done: P may be overwritten, O is stable
-                if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready, (j - 1) & 1))) { ok = false; break; }
-                if (__any_sync(0xffffffffu, resc)) {
-                    tc::fence_after_sync();
+            if (j > 0 && __any_sync(0xffffffffu, resc)) {
+                // the running max moved: O must hold PV of every earlier block before rescaling
+                // PV(j-1) completes phase (j-1)/2 of o_ready[(j-1)&1].  PV(j-3) is done (S(j) was
+                // issued after it) and PV(j+1) cannot start before this block's P, so that barrier is
+                // at most one phase ahead of the one waited for: the parity wait is unambiguous.
+                if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready[(j - 1) & 1], ((j - 1) >> 1) & 1, 8, j))) { ok = false; break; }
+                tc::fence_after_sync();
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tc::tmem_ld32(tl + C::COL_O + 32 * c, o);
-                        tc::tmem_wait_ld();
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t o[32];
+                    tc::tmem_ld32(tl + C::COL_O + 32 * c, o);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-                        tc::tmem_st32(tl + C::COL_O + 32 * c, o);
-                    }
-                    tc::tmem_wait_st();
+                    for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+                    tc::tmem_st32(tl + C::COL_O + 32 * c, o);
                 }
             }
-            // P row -> bf16 -> swizzled smem (64-key sub-tiles)
+            // P row -> packed bf16 pairs -> the first BN/2 columns of this block's S buffer
 #pragma unroll
-            for (int ck = 0; ck < BN / 8; ++ck) {
-                const float *e = sv + ck * 8;
-                *reinterpret_cast<uint4 *>(sP + (ck >> 3) * C::PSUB + swz(r, ck & 7)) =
-                    make_uint4(pack_bf16(e[0], e[1]), pack_bf16(e[2], e[3]), pack_bf16(e[4], e[5]),
-                               pack_bf16(e[6], e[7]));
+            for (int c = 0; c < BN / 64; ++c) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) pk[i] = pack_bf16(sv[64 * c + 2 * i], sv[64 * c + 2 * i + 1]);
+                tc::tmem_st32(tl + sb * C::COL_S1 + 32 * c, pk);
             }
-            tc::fence_proxy_async_smem();
+            tc::tmem_wait_st();
             tc::fence_before_sync();
-            mbar_arrive(&sh.p_full);
+            mbar_arrive(&sh.p_full[j & 1]);
             jdone = j + 1;
         }
         // ---- epilogue: O / l -> bf16 -> smem (Q's tile, no longer read) -> TMA store
@@ -466,7 +472,8 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) vself[c] = __ldg(vrow + c);
         }
-        if (have_o && nb > 0) have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready, (nb - 1) & 1));
+        if (have_o && nb > 0)
+            have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready[(nb - 1) & 1], ((nb - 1) >> 1) & 1, 9, nb));
         if (have_o) {
             tc::fence_after_sync();
             const float inv = 1.0f / l_run;
@@ -651,6 +658,18 @@ int attn_error_word(void *stream, bool clear) {
         if (cudaMemcpyToSymbol(g_attn_error, &zero, sizeof(int)) != cudaSuccess) return RAT_ERR_CUDA;
     }
     return v;
+}
+
+unsigned attn_error_where() {
+    unsigned w = 0;
+    if (cudaMemcpyFromSymbol(&w, g_attn_where, sizeof(unsigned)) != cudaSuccess) return 0xffffffffu;
+    return w;
+}
+
+unsigned attn_error_waiting() {
+    unsigned w = 0;
+    if (cudaMemcpyFromSymbol(&w, g_attn_waiting, sizeof(unsigned)) != cudaSuccess) return 0xffffffffu;
+    return w;
 }
 
 }  // namespace rat

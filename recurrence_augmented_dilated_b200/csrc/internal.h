@@ -76,6 +76,8 @@ struct AttnSm100Args {
 };
 int launch_attn_sm100(const AttnSm100Args &a, void *stream);
 int attn_error_word(void *stream, bool clear);
+unsigned attn_error_where();
+unsigned attn_error_waiting();
 extern int g_attn_block_keys;
 
 // ---------------------------------------------------------------------------- cache / decode

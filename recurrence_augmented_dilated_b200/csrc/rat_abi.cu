@@ -205,6 +205,10 @@ int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec
 
 int rat_attn_sync_status(void *stream) { return attn_error_word(stream, true); }
 
+uint32_t rat_attn_error_site(void) { return attn_error_where(); }
+
+uint32_t rat_attn_error_waiting(void) { return attn_error_waiting(); }
+
 int rat_set_attn_block_keys(int block_keys) {
     if (block_keys != 0 && block_keys != 64 && block_keys != 128) return RAT_ERR_INVALID;
     g_attn_block_keys = block_keys;

@@ -54,5 +54,7 @@ def gpu_attn(q, kr, vr, D=1, W=0, D_per_head=None, rope_base=0.0, pos0=0, scale=
     o = torch.empty_like(q)
     rat.rat_dilated_attn_prefill(q, kr, vr, o, D=D, W=W, D_per_head=D_per_head, pos0=pos0,
                                  rope_base=rope_base, scale=scale)
-    torch.cuda.synchronize()
+    st = rat.rat_attn_sync_status()
+    assert st == 0, "attention device error %s at site %#x" % (rat.rat_status_string(st),
+                                                              rat.lib().rat_attn_error_site())
     return o

@@ -156,3 +156,23 @@ def test_full_size_end_to_end_sampled(name, block_keys):
                                    rows=rows)
         err = rel_err(o[b:b + 1, heads][:, :, rows], ref["o"])
         assert err <= TOL_BF16, (b, err)
+
+
+@pytest.mark.parametrize("name", ["prefill_1p5b", "hybrid_7p6b"])
+def test_repeated_launches_no_timeout_and_deterministic(name, block_keys):
+    """Many back-to-back launches at full size: the pipeline's bounded waits never expire (the
+    device error word stays clear) and every launch returns the same bits."""
+    w = synthetic.WORKLOADS[name]
+    x = synthetic.prefill_inputs(w)
+    q, k, v = (x[n].cuda() for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    ref = None
+    for i in range(40 if name == "prefill_1p5b" else 6):
+        rat.rat_dilated_attn_prefill(q, k, v, o, D=w.D, W=w.W, D_per_head=w.D_per_head,
+                                     rope_base=w.rope_base)
+        if ref is None:
+            torch.cuda.synchronize()
+            ref = o.clone()
+    st = rat.rat_attn_sync_status()
+    assert st == 0, hex(rat.lib().rat_attn_error_site())
+    assert torch.equal(o, ref)
