@@ -27,6 +27,44 @@ RAT_DEVICE uint32_t pack_bf16(float lo, float hi) {
     return r;
 }
 
+// ------------------------------------------------------------------------------ float pairs
+// Two float32 lanes in one 64-bit register pair, for the packed f32x2 arithmetic of sm_100
+// (one instruction per pair, IEEE round-to-nearest like the scalar forms).
+typedef unsigned long long f2_t;
+RAT_DEVICE f2_t f2(float lo, float hi) {
+    f2_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+RAT_DEVICE float f2lo(f2_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return lo;
+}
+RAT_DEVICE float f2hi(f2_t v) {
+    float lo, hi;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    return hi;
+}
+RAT_DEVICE f2_t f2_fma(f2_t a, f2_t b, f2_t c) {
+    f2_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+RAT_DEVICE f2_t f2_mul(f2_t a, f2_t b) {
+    f2_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+RAT_DEVICE f2_t f2_add(f2_t a, f2_t b) {
+    f2_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// bf16 pair (low element in bits 0..15) -> float pair, and back (round to nearest even)
+RAT_DEVICE f2_t f2_from_bf16x2(uint32_t u) { return f2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u)); }
+RAT_DEVICE uint32_t f2_to_bf16x2(f2_t v) { return pack_bf16(f2lo(v), f2hi(v)); }
+
 // ------------------------------------------------------------------------------ math
 // 2^x and 1/x from the special-function unit (PTX ex2.approx / rcp.approx, flush-to-zero).
 RAT_DEVICE float ex2_approx(float x) {
@@ -74,6 +112,18 @@ RAT_DEVICE void rope_cs_f32(int pos, float theta, float &c, float &s) {
     float r = fmaf(-n, kTwoPiHi, ang);
     r = fmaf(-n, kTwoPiLo, r);
     __sincosf(r, &s, &c);
+}
+
+// Forget gates of a pair of logits: g = 1/(1+e^{-a}), 1-g = min(e^{-a} g, 1) (see forget_gate).
+RAT_DEVICE void forget_gate2(f2_t a, f2_t &g, f2_t &omg) {
+    const f2_t kNegLog2e = f2(-1.4426950408889634f, -1.4426950408889634f);
+    const f2_t kOne = f2(1.f, 1.f);
+    const f2_t x = f2_mul(a, kNegLog2e);
+    const f2_t e = f2(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
+    const f2_t y = f2_add(e, kOne);
+    g = f2(rcp_approx(f2lo(y)), rcp_approx(f2hi(y)));
+    const f2_t eg = f2_mul(e, g);
+    omg = f2(fminf(f2lo(eg), 1.0f), fminf(f2hi(eg), 1.0f));
 }
 
 // ------------------------------------------------------------------------------ memory order
@@ -137,8 +187,9 @@ RAT_DEVICE bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 RAT_DEVICE bool mbar_wait_bounded(uint64_t *bar, uint32_t parity, WsHeader *hdr, uint32_t where) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = globaltimer_ns();
+    uint32_t tries = 0;
     while (!mbar_try_wait(bar, parity)) {
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        if ((++tries & 15u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
             if (hdr) record_error(hdr, RAT_ERR_TIMEOUT, where);
             return false;
         }

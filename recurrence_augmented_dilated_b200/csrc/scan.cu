@@ -55,32 +55,31 @@ struct ScanCfg {
     static_assert(PT >= DH, "one thread per channel in a pipeline");
 };
 
-// 16 bytes of a row -> VEC floats.
+// 16 bytes of a row <-> VEC/2 float pairs (channels 2q, 2q+1 in pair q).
 template <typename E> struct Vec;
 template <> struct Vec<float> {
-    static constexpr int N = 4;
-    static RAT_DEVICE void load(const uint8_t *s, float *x) {
+    static constexpr int NP = 2;
+    static RAT_DEVICE void load(const uint8_t *s, f2_t *x) {
         uint32_t a, b, c, d;
         ld_shared_v4(s, a, b, c, d);
-        x[0] = __uint_as_float(a); x[1] = __uint_as_float(b);
-        x[2] = __uint_as_float(c); x[3] = __uint_as_float(d);
+        x[0] = f2(__uint_as_float(a), __uint_as_float(b));
+        x[1] = f2(__uint_as_float(c), __uint_as_float(d));
     }
-    static RAT_DEVICE void store(void *g, const float *x) {
-        st_global_v4(g, __float_as_uint(x[0]), __float_as_uint(x[1]), __float_as_uint(x[2]),
-                     __float_as_uint(x[3]));
+    static RAT_DEVICE void store(void *g, const f2_t *x) {
+        st_global_v4(g, __float_as_uint(f2lo(x[0])), __float_as_uint(f2hi(x[0])),
+                     __float_as_uint(f2lo(x[1])), __float_as_uint(f2hi(x[1])));
     }
 };
 template <> struct Vec<__nv_bfloat16> {
-    static constexpr int N = 8;
-    static RAT_DEVICE void load(const uint8_t *s, float *x) {
+    static constexpr int NP = 4;
+    static RAT_DEVICE void load(const uint8_t *s, f2_t *x) {
         uint32_t u[4];
         ld_shared_v4(s, u[0], u[1], u[2], u[3]);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) { x[2 * i] = bf16_lo(u[i]); x[2 * i + 1] = bf16_hi(u[i]); }
+        for (int i = 0; i < 4; ++i) x[i] = f2_from_bf16x2(u[i]);
     }
-    static RAT_DEVICE void store(void *g, const float *x) {
-        st_global_v4(g, pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
-                     pack_bf16(x[6], x[7]));
+    static RAT_DEVICE void store(void *g, const f2_t *x) {
+        st_global_v4(g, f2_to_bf16x2(x[0]), f2_to_bf16x2(x[1]), f2_to_bf16x2(x[2]), f2_to_bf16x2(x[3]));
     }
 };
 
@@ -178,63 +177,69 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
         const uint8_t *sa = pbase + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
         mbar_wait_bounded(&bar[pipe][st], (it >> 1) & 1, hdr, 0x100u);
 
-        // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate
-        float G[R][VEC], OG[R][VEC];
-        float A[VEC], Bk[VEC], Bv[VEC];
+        // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate, on
+        // packed float pairs (channels 2q, 2q+1)
+        constexpr int NP = VEC / 2;
+        const f2_t kOne2 = f2(1.f, 1.f), kZero2 = f2(0.f, 0.f);
+        f2_t G[R][NP], OG[R][NP];
+        f2_t A[NP], Bk[NP], Bv[NP];
 #pragma unroll
-        for (int j = 0; j < VEC; ++j) { A[j] = 1.f; Bk[j] = 0.f; Bv[j] = 0.f; }
+        for (int q = 0; q < NP; ++q) { A[q] = kOne2; Bk[q] = kZero2; Bv[q] = kZero2; }
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             const int r = seg * R + i;
-            float xa[VEC], xk[VEC], xv[VEC];
-            if (r < rows) {
-                const int off = r * C::ROWB + cl * 16;
-                Vec<E>::load(sa + off, xa);
-                Vec<E>::load(sk + off, xk);
-                Vec<E>::load(sv + off, xv);
-            } else {        // rows past the end: identity step (g = 1, 1-g = 0)
+            const int rr = r < rows ? r : rows - 1;          // rows past the end: identity step
+            const int off = rr * C::ROWB + cl * 16;
+            f2_t xa[NP], xk[NP], xv[NP];
+            Vec<E>::load(sa + off, xa);
+            Vec<E>::load(sk + off, xk);
+            Vec<E>::load(sv + off, xv);
 #pragma unroll
-                for (int j = 0; j < VEC; ++j) { xa[j] = 1e30f; xk[j] = 0.f; xv[j] = 0.f; }
-            }
-#pragma unroll
-            for (int j = 0; j < VEC; ++j) {
-                forget_gate(xa[j], G[i][j], OG[i][j]);
-                A[j] *= G[i][j];
-                Bk[j] = fmaf(G[i][j], Bk[j], OG[i][j] * xk[j]);
-                Bv[j] = fmaf(G[i][j], Bv[j], OG[i][j] * xv[j]);
+            for (int q = 0; q < NP; ++q) {
+                forget_gate2(xa[q], G[i][q], OG[i][q]);
+                if (r >= rows) { G[i][q] = kOne2; OG[i][q] = kZero2; }
+                A[q] = f2_mul(A[q], G[i][q]);
+                Bk[q] = f2_fma(G[i][q], Bk[q], f2_mul(OG[i][q], xk[q]));
+                Bv[q] = f2_fma(G[i][q], Bv[q], f2_mul(OG[i][q], xv[q]));
             }
         }
         // ---- inclusive scan over the segments of this warp (shuffles)
 #pragma unroll
         for (int sh = 1; sh < C::SPW; sh <<= 1) {
 #pragma unroll
-            for (int j = 0; j < VEC; ++j) {
-                const float pA = __shfl_up_sync(0xffffffffu, A[j], sh * LPR);
-                const float pK = __shfl_up_sync(0xffffffffu, Bk[j], sh * LPR);
-                const float pV = __shfl_up_sync(0xffffffffu, Bv[j], sh * LPR);
+            for (int q = 0; q < NP; ++q) {
+                const f2_t pA = f2(__shfl_up_sync(0xffffffffu, f2lo(A[q]), sh * LPR),
+                                   __shfl_up_sync(0xffffffffu, f2hi(A[q]), sh * LPR));
+                const f2_t pK = f2(__shfl_up_sync(0xffffffffu, f2lo(Bk[q]), sh * LPR),
+                                   __shfl_up_sync(0xffffffffu, f2hi(Bk[q]), sh * LPR));
+                const f2_t pV = f2(__shfl_up_sync(0xffffffffu, f2lo(Bv[q]), sh * LPR),
+                                   __shfl_up_sync(0xffffffffu, f2hi(Bv[q]), sh * LPR));
                 if (segw >= sh) {
-                    Bk[j] = fmaf(A[j], pK, Bk[j]);
-                    Bv[j] = fmaf(A[j], pV, Bv[j]);
-                    A[j] *= pA;
+                    Bk[q] = f2_fma(A[q], pK, Bk[q]);
+                    Bv[q] = f2_fma(A[q], pV, Bv[q]);
+                    A[q] = f2_mul(A[q], pA);
                 }
             }
         }
         // exclusive prefix of this segment inside its warp
-        float eA[VEC], eK[VEC], eV[VEC];
+        f2_t eA[NP], eK[NP], eV[NP];
 #pragma unroll
-        for (int j = 0; j < VEC; ++j) {
-            eA[j] = __shfl_up_sync(0xffffffffu, A[j], LPR);
-            eK[j] = __shfl_up_sync(0xffffffffu, Bk[j], LPR);
-            eV[j] = __shfl_up_sync(0xffffffffu, Bv[j], LPR);
-            if (segw == 0) { eA[j] = 1.f; eK[j] = 0.f; eV[j] = 0.f; }
+        for (int q = 0; q < NP; ++q) {
+            eA[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(A[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(A[q]), LPR));
+            eK[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(Bk[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(Bk[q]), LPR));
+            eV[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(Bv[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(Bv[q]), LPR));
+            if (segw == 0) { eA[q] = kOne2; eK[q] = kZero2; eV[q] = kZero2; }
         }
         if (segw == C::SPW - 1) {
 #pragma unroll
-            for (int j = 0; j < VEC; ++j) {
-                const int ch = cl * VEC + j;
-                sw[(pwarp * 3 + 0) * DH + ch] = A[j];
-                sw[(pwarp * 3 + 1) * DH + ch] = Bk[j];
-                sw[(pwarp * 3 + 2) * DH + ch] = Bv[j];
+            for (int q = 0; q < NP; ++q) {
+                const int ch = cl * VEC + 2 * q;
+                sw[(pwarp * 3 + 0) * DH + ch] = f2lo(A[q]);
+                sw[(pwarp * 3 + 0) * DH + ch + 1] = f2hi(A[q]);
+                sw[(pwarp * 3 + 1) * DH + ch] = f2lo(Bk[q]);
+                sw[(pwarp * 3 + 1) * DH + ch + 1] = f2hi(Bk[q]);
+                sw[(pwarp * 3 + 2) * DH + ch] = f2lo(Bv[q]);
+                sw[(pwarp * 3 + 2) * DH + ch + 1] = f2hi(Bv[q]);
             }
         }
         pipe_sync();
@@ -264,6 +269,7 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
             } else {
                 float xA = 1.f, xK = 0.f, xV = 0.f;   // composition of chunks j+1 .. c-1
                 const uint64_t t_start = globaltimer_ns();
+                uint32_t spins = 0;
                 bool alive = true;
                 for (int j = c - 1; j >= 0 && alive; --j) {
                     const size_t jid = (size_t)bh * p.nchunks + j;
@@ -290,12 +296,12 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
                             xA *= __uint_as_float((uint32_t)y);
                             break;                          // next predecessor
                         }
-                        if (globaltimer_ns() - t_start > p.wait_ns) {
+                        if ((++spins & 7u) == 0u && globaltimer_ns() - t_start > p.wait_ns) {
                             record_error(hdr, RAT_ERR_TIMEOUT, 0x200u);
                             alive = false;                  // carry zero; error recorded
                             break;
                         }
-                        __nanosleep(20);
+                        __nanosleep(32);
                     }
                 }
             }
@@ -325,26 +331,38 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
 
         // ---- pass 2: rerun the recurrence from the carry with the kept gates; write k~
         // (optionally rotated) and v~
-        float hk[VEC], hv[VEC];
+        f2_t hk[NP], hv[NP];
 #pragma unroll
-        for (int j = 0; j < VEC; ++j) {
-            const int ch = cl * VEC + j;
-            const float wk = sw[(pwarp * 3 + 0) * DH + ch], wv = sw[(pwarp * 3 + 1) * DH + ch];
-            hk[j] = fmaf(eA[j], wk, eK[j]);
-            hv[j] = fmaf(eA[j], wv, eV[j]);
+        for (int q = 0; q < NP; ++q) {
+            const int ch = cl * VEC + 2 * q;
+            const f2_t wk = f2(sw[(pwarp * 3 + 0) * DH + ch], sw[(pwarp * 3 + 0) * DH + ch + 1]);
+            const f2_t wv = f2(sw[(pwarp * 3 + 1) * DH + ch], sw[(pwarp * 3 + 1) * DH + ch + 1]);
+            hk[q] = f2_fma(eA[q], wk, eK[q]);
+            hv[q] = f2_fma(eA[q], wv, eV[q]);
         }
-        float rc[VEC], rs[VEC], sc[VEC], ss[VEC];
+        // RoPE: rotation (rc + i rs) of this lane's channels at its first row, advanced one
+        // position per row by (sc + i ss); the first half of the channels takes x cos - x' sin
+        f2_t rc[NP], rs[NP], sc[NP], ss[NP], nss[NP];
         const bool first_half = cl < LPR / 2;
         if (p.rope) {
             const long long pos = p.pos0 + t0 + seg * R;
 #pragma unroll
-            for (int j = 0; j < VEC; ++j) {
-                const int f = (cl * VEC + j) % (DH / 2);
-                if (p.rope_f32) rope_cs_f32((int)pos, p.theta_f[f], rc[j], rs[j]);
-                else rope_cs(pos, p.theta[f], rc[j], rs[j]);
-                sc[j] = p.step_cos[f];
-                ss[j] = first_half ? -p.step_sin[f] : p.step_sin[f];
-                if (first_half) rs[j] = -rs[j];      // first half: x cos - x' sin
+            for (int q = 0; q < NP; ++q) {
+                float c2[2], s2[2], a2[2], b2[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int f = (cl * VEC + 2 * q + u) % (DH / 2);
+                    if (p.rope_f32) rope_cs_f32((int)pos, p.theta_f[f], c2[u], s2[u]);
+                    else rope_cs(pos, p.theta[f], c2[u], s2[u]);
+                    a2[u] = p.step_cos[f];
+                    b2[u] = first_half ? -p.step_sin[f] : p.step_sin[f];
+                    if (first_half) s2[u] = -s2[u];
+                }
+                rc[q] = f2(c2[0], c2[1]);
+                rs[q] = f2(s2[0], s2[1]);
+                sc[q] = f2(a2[0], a2[1]);
+                ss[q] = f2(b2[0], b2[1]);
+                nss[q] = f2(-b2[0], -b2[1]);
             }
         }
         uint8_t *yk = static_cast<uint8_t *>(p.yk);
@@ -352,36 +370,31 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             const int r = seg * R + i;
-            const bool valid = r < rows;
-            float xk[VEC], xv[VEC];
-            if (valid) {
-                const int off = r * C::ROWB + cl * 16;
-                Vec<E>::load(sk + off, xk);
-                Vec<E>::load(sv + off, xv);
-            } else {
+            const int rr = r < rows ? r : rows - 1;
+            const int off = rr * C::ROWB + cl * 16;
+            f2_t xk[NP], xv[NP];
+            Vec<E>::load(sk + off, xk);
+            Vec<E>::load(sv + off, xv);
+            f2_t ok[NP];
 #pragma unroll
-                for (int j = 0; j < VEC; ++j) { xk[j] = 0.f; xv[j] = 0.f; }
-            }
-            float ok[VEC];
-#pragma unroll
-            for (int j = 0; j < VEC; ++j) {
-                hk[j] = fmaf(G[i][j], hk[j], OG[i][j] * xk[j]);
-                hv[j] = fmaf(G[i][j], hv[j], OG[i][j] * xv[j]);
-                ok[j] = hk[j];
+            for (int q = 0; q < NP; ++q) {
+                hk[q] = f2_fma(G[i][q], hk[q], f2_mul(OG[i][q], xk[q]));
+                hv[q] = f2_fma(G[i][q], hv[q], f2_mul(OG[i][q], xv[q]));
+                ok[q] = hk[q];
             }
             if (p.rope) {       // uniform across the grid: the shuffles see every lane
 #pragma unroll
-                for (int j = 0; j < VEC; ++j) {
-                    const float partner = __shfl_xor_sync(0xffffffffu, hk[j], LPR / 2);
-                    ok[j] = fmaf(hk[j], rc[j], partner * rs[j]);
-                    // advance the angle by one position: (c + i s) * (cos t + i sin t)
-                    const float nc = rc[j] * sc[j] - rs[j] * ss[j];
-                    const float ns = rs[j] * sc[j] + rc[j] * ss[j];
-                    rc[j] = nc;
-                    rs[j] = ns;
+                for (int q = 0; q < NP; ++q) {
+                    const f2_t partner = f2(__shfl_xor_sync(0xffffffffu, f2lo(hk[q]), LPR / 2),
+                                            __shfl_xor_sync(0xffffffffu, f2hi(hk[q]), LPR / 2));
+                    ok[q] = f2_fma(hk[q], rc[q], f2_mul(partner, rs[q]));
+                    // advance one position: (c + i s)(cos t + i sin t)
+                    const f2_t nc = f2_fma(rc[q], sc[q], f2_mul(rs[q], nss[q]));
+                    rs[q] = f2_fma(rs[q], sc[q], f2_mul(rc[q], ss[q]));
+                    rc[q] = nc;
                 }
             }
-            if (valid) {
+            if (r < rows) {
                 const size_t go = (row0 + r) * C::ROWB + cl * 16;
                 Vec<E>::store(yk + go, ok);
                 Vec<E>::store(yv + go, hv);
