@@ -64,10 +64,11 @@ struct Cfg {
 };
 
 struct Params {
-    CUtensorMap tm_q, tm_o;                        // (d, T, B*H) bf16, box (64, 128, 1), 128B swizzle
+    CUtensorMap tm_q;                              // (d, T, B*H) bf16, box (64, 128, 1), 128B swizzle
     CUtensorMap tm_k, tm_v;                        // same tensors, box (64, BN, 1)
     CUtensorMap tm_kd[kMaxDil], tm_vd[kMaxDil];    // chunk ends of one dilation: (d, T/D, B*H)
     const void *kg, *vg;                           // k~, v~ (the self key when W <= 1)
+    void *og;                                      // output, written row by row
     int B, H, T, W, ntiles;
     long long pos0;
     int rope;
@@ -240,6 +241,8 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             for (int j = 0; j < nb; ++j) {
                 const int s = j % NS;
                 if (j >= NS && !wait_bar(sh, &sh.kv_empty[s], ((j / NS) - 1) & 1, 1, j)) break;
+                // with RoPE, stage 1 holds the softmax warps' rotation tables until Q is rotated
+                if (j == 1 && p.rope && !wait_bar(sh, &sh.q_ready, 0, 10, j)) break;
                 const CUtensorMap *tk = j < pl.nd ? mk : &p.tm_k;
                 const CUtensorMap *tv = j < pl.nd ? mv : &p.tm_v;
                 const int y = j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd);
@@ -330,9 +333,30 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         // waits are made warp-uniform: tcgen05.ld/st below are warp-collective
         bool ok = __all_sync(0xffffffffu, wait_bar(sh, &sh.q_full, 0, 6));
         if (ok && p.rope) {
-            // rotate-half RoPE of this row of Q at position pos0 + t: channel c (< 64) pairs with
-            // c + 64, which sits at the same swizzled offset of the second sub-tile
-            const long long pos = p.pos0 + t;
+            // rotate-half RoPE of the Q tile at positions pos0 + t.  Rotation of row 32w + l is
+            // rot(base_w) * rot(l): 128 threads first tabulate rot(l theta_f) for l < 32 and
+            // rot((pos0 + t0 + 32w) theta_f) in the still-unused second K/V stage, then each row
+            // combines one entry of each per frequency.
+            float2 *rel = reinterpret_cast<float2 *>(smem + C::OFF_K + C::KTILE);    // [64 f][32 l]
+            float2 *bas = reinterpret_cast<float2 *>(smem + C::OFF_V + C::KTILE);    // [4 w][64 f]
+            const int i0 = r;                       // 0..127
+#pragma unroll 4
+            for (int k = 0; k < 16; ++k) {
+                const int e = i0 + 128 * k, f = e >> 5, l = e & 31;
+                float cs, sn;
+                rope_cs_f32(l, p.theta_f[f], cs, sn);
+                rel[e] = make_float2(cs, sn);
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int e = i0 + 128 * k, w = e >> 6, f = e & 63;
+                const long long pos = p.pos0 + t0 + 32 * w;
+                float cs, sn;
+                if (p.rope_f32) rope_cs_f32((int)pos, p.theta_f[f], cs, sn);
+                else rope_cs_fast(pos, p.theta[f], cs, sn);
+                bas[w * 64 + f] = make_float2(cs, sn);
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
 #pragma unroll
             for (int c = 0; c < 8; ++c) {
                 uint4 *p1 = reinterpret_cast<uint4 *>(sQ + swz(r, c));
@@ -341,18 +365,18 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                 uint32_t a1[4] = {u1.x, u1.y, u1.z, u1.w}, a2[4] = {u2.x, u2.y, u2.z, u2.w};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    float x1l = bf16_lo(a1[i]), x1h = bf16_hi(a1[i]);
-                    float x2l = bf16_lo(a2[i]), x2h = bf16_hi(a2[i]);
-                    float cl, sl, ch, sh2;
-                    if (p.rope_f32) {
-                        rope_cs_f32((int)pos, p.theta_f[c * 8 + 2 * i], cl, sl);
-                        rope_cs_f32((int)pos, p.theta_f[c * 8 + 2 * i + 1], ch, sh2);
-                    } else {
-                        rope_cs_fast(pos, p.theta[c * 8 + 2 * i], cl, sl);
-                        rope_cs_fast(pos, p.theta[c * 8 + 2 * i + 1], ch, sh2);
+                    float cs[2], sn[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const int f = c * 8 + 2 * i + u;
+                        const float2 b = bas[q4 * 64 + f], rl = rel[f * 32 + lane];
+                        cs[u] = b.x * rl.x - b.y * rl.y;
+                        sn[u] = b.y * rl.x + b.x * rl.y;
                     }
-                    a1[i] = pack_bf16(x1l * cl - x2l * sl, x1h * ch - x2h * sh2);
-                    a2[i] = pack_bf16(x2l * cl + x1l * sl, x2h * ch + x1h * sh2);
+                    const float x1l = bf16_lo(a1[i]), x1h = bf16_hi(a1[i]);
+                    const float x2l = bf16_lo(a2[i]), x2h = bf16_hi(a2[i]);
+                    a1[i] = pack_bf16(x1l * cs[0] - x2l * sn[0], x1h * cs[1] - x2h * sn[1]);
+                    a2[i] = pack_bf16(x2l * cs[0] + x1l * sn[0], x2h * cs[1] + x1h * sn[1]);
                 }
                 *p1 = make_uint4(a1[0], a1[1], a1[2], a1[3]);
                 *p2 = make_uint4(a2[0], a2[1], a2[2], a2[3]);
@@ -463,7 +487,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             mbar_arrive(&sh.p_full[j & 1]);
             jdone = j + 1;
         }
-        // ---- epilogue: O / l -> bf16 -> smem (Q's tile, no longer read) -> TMA store
+        // ---- epilogue: O / l -> bf16 -> global memory, one row per thread
         bool have_o = ok && jdone == nb;
         uint4 vself[16];          // the self key's value row, loaded while the last PV runs
         if (have_o && pl.self_reg) {
@@ -477,6 +501,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         if (have_o) {
             tc::fence_after_sync();
             const float inv = 1.0f / l_run;
+            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.og) + ((size_t)bh * p.T + t) * DHEAD;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
@@ -499,24 +524,16 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                         }
                     }
                 }
+                if (t < p.T && !sh.abort) {   // this row's 256 bytes, straight to global memory
 #pragma unroll
-                for (int k8 = 0; k8 < 4; ++k8) {
-                    const int col = 32 * c + 8 * k8;
-                    const float *f = reinterpret_cast<const float *>(o) + 8 * k8;
-                    *reinterpret_cast<uint4 *>(sQ + (col >> 6) * QSUB + swz(r, (col & 63) >> 3)) =
-                        make_uint4(pack_bf16(f[0] * inv, f[1] * inv), pack_bf16(f[2] * inv, f[3] * inv),
-                                   pack_bf16(f[4] * inv, f[5] * inv), pack_bf16(f[6] * inv, f[7] * inv));
+                    for (int k8 = 0; k8 < 4; ++k8) {
+                        const float *f = reinterpret_cast<const float *>(o) + 8 * k8;
+                        st_global_v4(orow + 32 * c + 8 * k8,
+                                     pack_bf16(f[0] * inv, f[1] * inv), pack_bf16(f[2] * inv, f[3] * inv),
+                                     pack_bf16(f[4] * inv, f[5] * inv), pack_bf16(f[6] * inv, f[7] * inv));
+                    }
                 }
             }
-            tc::fence_proxy_async_smem();
-        }
-        // all 128 epilogue threads reach this barrier on every path; the store is issued only if
-        // no role aborted (an abort has already recorded RAT_ERR_TIMEOUT)
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (r == 0 && have_o && !sh.abort) {
-            tc::tma_store_3d(&p.tm_o, sQ, 0, t0, bh);
-            tc::tma_store_3d(&p.tm_o, sQ + QSUB, 64, t0, bh);
-            tc::tma_store_commit_and_wait();
         }
     }
 
@@ -561,7 +578,7 @@ int launch_bn(const AttnSm100Args &a, void *stream) {
     std::memset(&p, 0, sizeof(p));
     const uint64_t BH = (uint64_t)a.B * a.H, T = (uint64_t)a.T;
     const uint64_t row = DHEAD * 2, slice = T * row;
-    if (!make_map(&p.tm_q, a.q, T, BH, row, slice, BM) || !make_map(&p.tm_o, a.o, T, BH, row, slice, BM) ||
+    if (!make_map(&p.tm_q, a.q, T, BH, row, slice, BM) ||
         !make_map(&p.tm_k, a.k, T, BH, row, slice, BN) || !make_map(&p.tm_v, a.v, T, BH, row, slice, BN))
         return RAT_ERR_CUDA;
     // one strided map pair per distinct dilation > 1
@@ -605,6 +622,7 @@ int launch_bn(const AttnSm100Args &a, void *stream) {
     p.ntiles = (a.T + BM - 1) / BM;
     p.kg = a.k;
     p.vg = a.v;
+    p.og = a.o;
     p.ngroups = 0;
     int items = 0;
     for (int i = 0; i < a.H;) {
