@@ -37,13 +37,13 @@ RAT_DEVICE f2_t f2(float lo, float hi) {
     return r;
 }
 RAT_DEVICE float f2lo(f2_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    float lo;
+    asm("{\n .reg .f32 t;\n mov.b64 {%0, t}, %1;\n}" : "=f"(lo) : "l"(v));
     return lo;
 }
 RAT_DEVICE float f2hi(f2_t v) {
-    float lo, hi;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+    float hi;
+    asm("{\n .reg .f32 t;\n mov.b64 {t, %0}, %1;\n}" : "=f"(hi) : "l"(v));
     return hi;
 }
 RAT_DEVICE f2_t f2_fma(f2_t a, f2_t b, f2_t c) {

@@ -75,10 +75,32 @@ struct AttnSm100Args {
     double theta[64];
 };
 int launch_attn_sm100(const AttnSm100Args &a, void *stream);
+
+// Opt kernel `fn` into `bytes` of dynamic shared memory on the current device, once per device
+// (bit `dev` of *done_mask records it).  Returns a rat_status.
+inline int set_smem_attr(const void *fn, uint32_t bytes, uint64_t *done_mask) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RAT_ERR_CUDA;
+    if (*done_mask >> dev & 1) return RAT_OK;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
+        return RAT_ERR_CUDA;
+    *done_mask |= 1ull << dev;
+    return RAT_OK;
+}
+
+// Number of SMs of the current device (0 on error).
+inline int current_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    return sms;
+}
 int attn_error_word(void *stream, bool clear);
 unsigned attn_error_where();
 unsigned attn_error_waiting();
 extern int g_attn_block_keys;
+extern int g_attn_schedule;
 
 // ---------------------------------------------------------------------------- cache / decode
 struct CompressParams {

@@ -430,19 +430,11 @@ template <typename E, int DH>
 static int launch_one(const RecurParams &p, void *stream) {
     using C = ScanCfg<E, DH>;
     auto kern = recur_kernel<E, DH>;
-    static bool attr_set = false;   // per process; the attribute is per function
-    if (!attr_set) {
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
-            return RAT_ERR_CUDA;
-        attr_set = true;
-    }
-    static int sms = 0;
-    if (!sms) {
-        int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-            return RAT_ERR_CUDA;
-    }
+    static uint64_t attr_done = 0;
+    const int st = set_smem_attr(reinterpret_cast<const void *>(kern), C::SMEM, &attr_done);
+    if (st != RAT_OK) return st;
+    const int sms = current_sm_count();
+    if (sms <= 0) return RAT_ERR_CUDA;
     // persistent: one CTA per SM, each walking chunks in ticket order
     const long long total = (long long)p.BH * p.nchunks;
     const unsigned grid = (unsigned)(total < sms ? total : sms);
