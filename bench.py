@@ -353,7 +353,9 @@ def run_decode(w: synthetic.Workload, steps_timed: int, warmup: int, rank: int, 
         rat.rat_kv_compress(kr, vr, hk2, hv2, cache)
         hk, hv = hk2, hv2
         del k, v, a, kr, vr
+    del ws_r
     torch.cuda.synchronize()
+    torch.cuda.empty_cache()      # only the cache and the step inputs stay on the device
     tok = synthetic.decode_steps(w)
     tq, tk, tv, ta = (tok[n].to(dev).reshape(nsteps, B, H, 1, d) for n in ("q", "k", "v", "a"))
     out = torch.empty((nsteps, B, H, 1, d), dtype=torch.bfloat16, device=dev)

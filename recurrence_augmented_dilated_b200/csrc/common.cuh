@@ -115,16 +115,18 @@ RAT_DEVICE void rope_cs_f32(int pos, float theta, float &c, float &s) {
 }
 
 // Forget gates of a pair of logits: g = 1/(1+e^{-a}), 1-g = min(e^{-a} g, 1) (see forget_gate).
-RAT_DEVICE void forget_gate2(f2_t a, f2_t &g, f2_t &omg) {
+// Forget gate of a pair of logits: g = sigmoid(a) = 1 / (1 + 2^(-a log2 e)).  The
+// complement is formed by gate_complement2 as 1 - g: exact for g >= 1/2 (Sterbenz), within
+// 2^-25 absolute below, and exactly 0 or 1 at the saturated gates.
+RAT_DEVICE f2_t forget_gate2(f2_t a) {
     const f2_t kNegLog2e = f2(-1.4426950408889634f, -1.4426950408889634f);
     const f2_t kOne = f2(1.f, 1.f);
     const f2_t x = f2_mul(a, kNegLog2e);
     const f2_t e = f2(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));
     const f2_t y = f2_add(e, kOne);
-    g = f2(rcp_approx(f2lo(y)), rcp_approx(f2hi(y)));
-    const f2_t eg = f2_mul(e, g);
-    omg = f2(fminf(f2lo(eg), 1.0f), fminf(f2hi(eg), 1.0f));
+    return f2(rcp_approx(f2lo(y)), rcp_approx(f2hi(y)));
 }
+RAT_DEVICE f2_t gate_complement2(f2_t g) { return f2_fma(g, f2(-1.f, -1.f), f2(1.f, 1.f)); }
 
 // ------------------------------------------------------------------------------ memory order
 RAT_DEVICE uint64_t ld_relaxed_gpu_u64(const uint64_t *p) {
@@ -208,6 +210,12 @@ RAT_DEVICE void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, u
 RAT_DEVICE void ld_shared_v4(const void *p, uint32_t &a, uint32_t &b, uint32_t &c, uint32_t &d) {
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(smem_u32(p)));
+}
+RAT_DEVICE void ld_shared_v2(const void *p, uint32_t &a, uint32_t &b) {
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(a), "=r"(b) : "r"(smem_u32(p)));
+}
+RAT_DEVICE void st_global_v2(void *p, uint32_t a, uint32_t b) {
+    asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(p), "r"(a), "r"(b) : "memory");
 }
 RAT_DEVICE void st_global_v4(void *p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d)

@@ -8,20 +8,25 @@
 //     A = prod g,   B = sum_s (prod_{r>s} g_r)(1-g_s) x_s,
 // and (A1,B1) then (A2,B2) = (A2 A1, A2 B1 + B2).  This kernel is that scan, in three levels:
 //
-//   lane     : 8 consecutive rows of one 16-byte channel group, sequentially in registers;
-//   CTA      : the row segments of a chunk combined by warp shuffles, then across the 8 warps
-//              through shared memory;
+//   lane     : R consecutive rows of four channels, sequentially in registers;
+//   CTA      : the row segments of a chunk combined by warp shuffles, then across the warps
+//              of a pipeline through shared memory;
 //   sequence : chunks of the same (b, h) combined by a decoupled look-back -- each chunk
 //              publishes its aggregate (A, Bk, Bv) as soon as it has loaded, then walks back
 //              over its predecessors' aggregates until it meets an inclusive state.
 //
+// Lane layout: lane l of a row holds the channel pairs (2l, 2l+1) and (2l + d/2, 2l+1 + d/2).
+// The two pairs are each other's rotate-half RoPE partners, so the rotation of k~ needs no
+// data from other lanes, and every shared-memory load and global store of a warp touches one
+// contiguous run of bytes.
+//
 // Data movement: a chunk is TC rows x d channels of one (b, h), i.e. three contiguous byte
-// ranges (a, k, v), fetched with three bulk copies (cp.async.bulk) into shared memory.  The
-// kernel is persistent (one CTA per SM) and double-buffered: while a CTA computes one chunk,
-// the bulk copies of its next chunk are in flight.  Outputs are written with 16-byte stores,
-// 16 lanes covering one 256-byte row.  The HBM stream is 3 reads + 2 writes per element, the
-// algorithmic minimum.  The gates of pass 1 stay in registers for pass 2, so each element
-// costs one exp2 and one reciprocal on the special-function unit.
+// ranges (a, k, v) of 16 KiB, fetched with three bulk copies (cp.async.bulk) into shared
+// memory.  The kernel is persistent (one CTA per SM, two independent chunk pipelines) and
+// double-buffered: while a pipeline computes one chunk, the bulk copies of its next chunk are
+// in flight.  The HBM stream is 3 reads + 2 writes per element, the algorithmic minimum.  The
+// gates of pass 1 stay in registers for pass 2, so each element costs one exp2 and one
+// reciprocal on the special-function unit.
 //
 // Chunk order comes from an atomic ticket (chunk-major: all (b, h) advance together); a CTA
 // takes its next ticket before finishing the current chunk, and every predecessor it waits
@@ -36,50 +41,54 @@ namespace rat {
 template <typename E, int DH>
 struct ScanCfg {
     static constexpr int EB = sizeof(E);
-    static constexpr int VEC = 16 / EB;           // channels per lane (one 16-byte vector)
-    static constexpr int LPR = DH / VEC;          // lanes per row
-    static constexpr int THREADS = 256;
+    static constexpr int LPR = DH / 4;            // lanes per row: four channels (two pairs) each
+    static constexpr int HALFB = DH / 2 * EB;     // byte offset of the second half of a row
+    static constexpr int THREADS = 512;
     static constexpr int NPIPE = 2;               // independent chunk pipelines per CTA
     static constexpr int PT = THREADS / NPIPE;    // threads per pipeline
     static constexpr int PW = PT / 32;            // warps per pipeline
     static constexpr int SEGS = PT / LPR;         // row segments per chunk
     static constexpr int SPW = 32 / LPR;          // segments per warp
-    static constexpr int R = 8;                   // rows per segment
-    static constexpr int TC = SEGS * R;           // rows per chunk
     static constexpr int ROWB = DH * EB;          // bytes per row
-    static constexpr int TILEB = TC * ROWB;       // bytes per tensor per chunk (16 KiB)
+    static constexpr int TILEB = 16384;           // bytes per tensor per chunk
+    static constexpr int TC = TILEB / ROWB;       // rows per chunk
+    static constexpr int R = TC / SEGS;           // rows per segment
+    static constexpr int LBW = 2;                 // predecessors read per look-back round
     static constexpr int STAGEB = 3 * TILEB;      // a, k, v of one chunk
     static constexpr int SWB = PW * 3 * DH * 4;   // per-warp aggregates, then carries
-    static constexpr int PIPEB = 2 * STAGEB + SWB + 2 * DH * 4;   // two stages + sw + state in
+    static constexpr int PIPEB = 2 * STAGEB + SWB;
     static constexpr int SMEM = NPIPE * PIPEB;
     static_assert(PT >= DH, "one thread per channel in a pipeline");
+    static_assert(R * SEGS == TC && R >= 1, "whole segments per chunk");
 };
 
-// 16 bytes of a row <-> VEC/2 float pairs (channels 2q, 2q+1 in pair q).
-template <typename E> struct Vec;
-template <> struct Vec<float> {
-    static constexpr int NP = 2;
-    static RAT_DEVICE void load(const uint8_t *s, f2_t *x) {
-        uint32_t a, b, c, d;
-        ld_shared_v4(s, a, b, c, d);
-        x[0] = f2(__uint_as_float(a), __uint_as_float(b));
-        x[1] = f2(__uint_as_float(c), __uint_as_float(d));
+// A lane's two channel pairs of one row: pair 0 at channels (2l, 2l+1), pair 1 at
+// (2l + d/2, 2l+1 + d/2), as float pairs.
+template <typename E> struct Lane;
+template <> struct Lane<float> {
+    template <int HALFB>
+    static RAT_DEVICE void load(const uint8_t *row, int l, f2_t *x) {
+        const uint2 a = *reinterpret_cast<const uint2 *>(row + 8 * l);
+        const uint2 c = *reinterpret_cast<const uint2 *>(row + HALFB + 8 * l);
+        x[0] = f2(__uint_as_float(a.x), __uint_as_float(a.y));
+        x[1] = f2(__uint_as_float(c.x), __uint_as_float(c.y));
     }
-    static RAT_DEVICE void store(void *g, const f2_t *x) {
-        st_global_v4(g, __float_as_uint(f2lo(x[0])), __float_as_uint(f2hi(x[0])),
-                     __float_as_uint(f2lo(x[1])), __float_as_uint(f2hi(x[1])));
+    template <int HALFB>
+    static RAT_DEVICE void store(uint8_t *row, int l, const f2_t *x) {
+        *reinterpret_cast<uint2 *>(row + 8 * l) = make_uint2(__float_as_uint(f2lo(x[0])), __float_as_uint(f2hi(x[0])));
+        *reinterpret_cast<uint2 *>(row + HALFB + 8 * l) = make_uint2(__float_as_uint(f2lo(x[1])), __float_as_uint(f2hi(x[1])));
     }
 };
-template <> struct Vec<__nv_bfloat16> {
-    static constexpr int NP = 4;
-    static RAT_DEVICE void load(const uint8_t *s, f2_t *x) {
-        uint32_t u[4];
-        ld_shared_v4(s, u[0], u[1], u[2], u[3]);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) x[i] = f2_from_bf16x2(u[i]);
+template <> struct Lane<__nv_bfloat16> {
+    template <int HALFB>
+    static RAT_DEVICE void load(const uint8_t *row, int l, f2_t *x) {
+        x[0] = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(row + 4 * l));
+        x[1] = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(row + HALFB + 4 * l));
     }
-    static RAT_DEVICE void store(void *g, const f2_t *x) {
-        st_global_v4(g, f2_to_bf16x2(x[0]), f2_to_bf16x2(x[1]), f2_to_bf16x2(x[2]), f2_to_bf16x2(x[3]));
+    template <int HALFB>
+    static RAT_DEVICE void store(uint8_t *row, int l, const f2_t *x) {
+        *reinterpret_cast<uint32_t *>(row + 4 * l) = f2_to_bf16x2(x[0]);
+        *reinterpret_cast<uint32_t *>(row + HALFB + 4 * l) = f2_to_bf16x2(x[1]);
     }
 };
 
@@ -88,40 +97,25 @@ template <> struct Vec<__nv_bfloat16> {
 // value and its validity always travel together.
 RAT_DEVICE uint64_t tagged(uint32_t tag, float v) { return ((uint64_t)tag << 32) | __float_as_uint(v); }
 
-// Wait (bounded) for the tagged word at w; returns false if the wait ran out.
-RAT_DEVICE bool wait_word(const uint64_t *w, uint32_t tag, float &v, uint64_t t_start, uint64_t limit_ns,
-                          WsHeader *hdr) {
-    for (;;) {
-        const uint64_t x = ld_relaxed_gpu_u64(w);
-        if ((uint32_t)(x >> 32) == tag) {
-            v = __uint_as_float((uint32_t)x);
-            return true;
-        }
-        if (globaltimer_ns() - t_start > limit_ns) {
-            record_error(hdr, RAT_ERR_TIMEOUT, 0x200u);
-            return false;
-        }
-        __nanosleep(20);
-    }
-}
-
 template <typename E, int DH>
-__global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ RecurParams p) {
+__global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const __grid_constant__ RecurParams p) {
     using C = ScanCfg<E, DH>;
-    constexpr int VEC = C::VEC, LPR = C::LPR, R = C::R;
+    constexpr int LPR = C::LPR, R = C::R, HALF = DH / 2, NP = 2;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t bar[C::NPIPE][2];
     __shared__ int s_ticket[C::NPIPE][2];
     __shared__ uint32_t s_epoch;
+    __shared__ float s_theta_f[HALF], s_step_c[HALF], s_step_s[HALF];
+    __shared__ double s_theta[HALF];
 
     const int tid = threadIdx.x;
     const int pipe = tid / C::PT, pt = tid % C::PT;              // pipeline and thread in it
     const int pwarp = pt >> 5, lane = tid & 31;
     const int seg = pt / LPR, cl = pt % LPR, segw = lane / LPR;
+    const int chq[NP] = {2 * cl, 2 * cl + HALF};                   // first channel of each pair
     const int barid = 1 + pipe;                                   // named barrier of this pipeline
     uint8_t *pbase = smem + pipe * C::PIPEB;
     float *sw = reinterpret_cast<float *>(pbase + 2 * C::STAGEB);          // [PW][3][DH]
-    float *sH = reinterpret_cast<float *>(pbase + 2 * C::STAGEB + C::SWB); // [2][DH] state in
     WsHeader *hdr = p.hdr;
     const int total = p.BH * p.nchunks;
 
@@ -139,6 +133,12 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
     };
     auto pipe_sync = [&]() { asm volatile("bar.sync %0, %1;" :: "r"(barid), "r"(C::PT) : "memory"); };
 
+    if (tid < HALF) {           // RoPE tables, read per lane below without divergent constant loads
+        s_theta_f[tid] = p.theta_f[tid];
+        s_theta[tid] = p.theta[tid];
+        s_step_c[tid] = p.step_cos[tid];
+        s_step_s[tid] = p.step_sin[tid];
+    }
     if (tid == 0) {
         s_epoch = *reinterpret_cast<volatile uint32_t *>(&hdr->epoch);
         for (int q = 0; q < C::NPIPE; ++q) {
@@ -177,30 +177,27 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
         const uint8_t *sa = pbase + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
         mbar_wait_bounded(&bar[pipe][st], (it >> 1) & 1, hdr, 0x100u);
 
-        // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate, on
-        // packed float pairs (channels 2q, 2q+1)
-        constexpr int NP = VEC / 2;
+        // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate
         const f2_t kOne2 = f2(1.f, 1.f), kZero2 = f2(0.f, 0.f);
-        f2_t G[R][NP], OG[R][NP];
+        f2_t G[R][NP];           // gates; 1 - g is re-formed where it is used
         f2_t A[NP], Bk[NP], Bv[NP];
 #pragma unroll
         for (int q = 0; q < NP; ++q) { A[q] = kOne2; Bk[q] = kZero2; Bv[q] = kZero2; }
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             const int r = seg * R + i;
-            const int rr = r < rows ? r : rows - 1;          // rows past the end: identity step
-            const int off = rr * C::ROWB + cl * 16;
+            const int off = (r < rows ? r : rows - 1) * C::ROWB;   // rows past the end: identity step
             f2_t xa[NP], xk[NP], xv[NP];
-            Vec<E>::load(sa + off, xa);
-            Vec<E>::load(sk + off, xk);
-            Vec<E>::load(sv + off, xv);
+            Lane<E>::template load<C::HALFB>(sa + off, cl, xa);
+            Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
+            Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
-                forget_gate2(xa[q], G[i][q], OG[i][q]);
-                if (r >= rows) { G[i][q] = kOne2; OG[i][q] = kZero2; }
+                G[i][q] = r < rows ? forget_gate2(xa[q]) : kOne2;
+                const f2_t og = gate_complement2(G[i][q]);
                 A[q] = f2_mul(A[q], G[i][q]);
-                Bk[q] = f2_fma(G[i][q], Bk[q], f2_mul(OG[i][q], xk[q]));
-                Bv[q] = f2_fma(G[i][q], Bv[q], f2_mul(OG[i][q], xv[q]));
+                Bk[q] = f2_fma(G[i][q], Bk[q], f2_mul(og, xk[q]));
+                Bv[q] = f2_fma(G[i][q], Bv[q], f2_mul(og, xv[q]));
             }
         }
         // ---- inclusive scan over the segments of this warp (shuffles)
@@ -225,15 +222,17 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
         f2_t eA[NP], eK[NP], eV[NP];
 #pragma unroll
         for (int q = 0; q < NP; ++q) {
-            eA[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(A[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(A[q]), LPR));
-            eK[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(Bk[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(Bk[q]), LPR));
-            eV[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(Bv[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(Bv[q]), LPR));
-            if (segw == 0) { eA[q] = kOne2; eK[q] = kZero2; eV[q] = kZero2; }
+            if (C::SPW > 1) {
+                eA[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(A[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(A[q]), LPR));
+                eK[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(Bk[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(Bk[q]), LPR));
+                eV[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(Bv[q]), LPR), __shfl_up_sync(0xffffffffu, f2hi(Bv[q]), LPR));
+            }
+            if (C::SPW == 1 || segw == 0) { eA[q] = kOne2; eK[q] = kZero2; eV[q] = kZero2; }
         }
         if (segw == C::SPW - 1) {
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
-                const int ch = cl * VEC + 2 * q;
+                const int ch = chq[q];
                 sw[(pwarp * 3 + 0) * DH + ch] = f2lo(A[q]);
                 sw[(pwarp * 3 + 0) * DH + ch + 1] = f2hi(A[q]);
                 sw[(pwarp * 3 + 1) * DH + ch] = f2lo(Bk[q]);
@@ -267,39 +266,54 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
                 if (p.h0k) Hk = p.h0k[(size_t)bh * DH + ch];
                 if (p.h0v) Hv = p.h0v[(size_t)bh * DH + ch];
             } else {
+                // Walk back from j = c - 1, C::LBW predecessors per round: all five words of each
+                // (inclusive state k, v; aggregate A, Bk, Bv) are read at once, so a round costs one
+                // memory latency.  A predecessor with its inclusive state ends the walk; one with
+                // only its aggregate is composed in and passed; one with neither stops the round,
+                // and the next round re-reads from there.
                 float xA = 1.f, xK = 0.f, xV = 0.f;   // composition of chunks j+1 .. c-1
                 const uint64_t t_start = globaltimer_ns();
                 uint32_t spins = 0;
-                bool alive = true;
-                for (int j = c - 1; j >= 0 && alive; --j) {
-                    const size_t jid = (size_t)bh * p.nchunks + j;
-                    const uint64_t *pj = p.pre + jid * 2 * DH;
-                    const uint64_t *aj = p.agg + jid * 3 * DH;
-                    // predecessor j: its inclusive state if published, else its aggregate
-                    for (;;) {
-                        const uint64_t x = ld_relaxed_gpu_u64(pj + ch);
-                        if ((uint32_t)(x >> 32) == tag) {
-                            float hv;
-                            alive = wait_word(pj + DH + ch, tag, hv, t_start, p.wait_ns, hdr);
-                            Hk = fmaf(xA, __uint_as_float((uint32_t)x), xK);
-                            Hv = fmaf(xA, hv, xV);
-                            j = -1;                         // done
-                            break;
+                int j = c - 1;
+                for (;;) {
+                    uint64_t w[C::LBW][5];
+#pragma unroll
+                    for (int u = 0; u < C::LBW; ++u) {
+                        const size_t jid = (size_t)bh * p.nchunks + max(j - u, 0);
+                        const uint64_t *pj = p.pre + jid * 2 * DH + ch;
+                        const uint64_t *aj = p.agg + jid * 3 * DH + ch;
+                        w[u][0] = ld_relaxed_gpu_u64(pj);
+                        w[u][1] = ld_relaxed_gpu_u64(pj + DH);
+                        w[u][2] = ld_relaxed_gpu_u64(aj);
+                        w[u][3] = ld_relaxed_gpu_u64(aj + DH);
+                        w[u][4] = ld_relaxed_gpu_u64(aj + 2 * DH);
+                    }
+                    bool done = false, stop = false;
+                    int passed = 0;
+#pragma unroll
+                    for (int u = 0; u < C::LBW; ++u) {
+                        if (done || stop || j - u < 0) continue;
+                        auto ok = [&](int e) { return (uint32_t)(w[u][e] >> 32) == tag; };
+                        auto val = [&](int e) { return __uint_as_float((uint32_t)w[u][e]); };
+                        if (ok(0) && ok(1)) {
+                            Hk = fmaf(xA, val(0), xK);
+                            Hv = fmaf(xA, val(1), xV);
+                            done = true;
+                        } else if (ok(2) && ok(3) && ok(4)) {
+                            xK = fmaf(xA, val(3), xK);
+                            xV = fmaf(xA, val(4), xV);
+                            xA *= val(2);
+                            ++passed;
+                        } else {
+                            stop = true;
                         }
-                        const uint64_t y = ld_relaxed_gpu_u64(aj + ch);
-                        if ((uint32_t)(y >> 32) == tag) {
-                            float bk, bv;
-                            alive = wait_word(aj + DH + ch, tag, bk, t_start, p.wait_ns, hdr) &&
-                                    wait_word(aj + 2 * DH + ch, tag, bv, t_start, p.wait_ns, hdr);
-                            xK = fmaf(xA, bk, xK);
-                            xV = fmaf(xA, bv, xV);
-                            xA *= __uint_as_float((uint32_t)y);
-                            break;                          // next predecessor
-                        }
+                    }
+                    if (done) break;
+                    j -= passed;
+                    if (passed == 0) {
                         if ((++spins & 7u) == 0u && globaltimer_ns() - t_start > p.wait_ns) {
                             record_error(hdr, RAT_ERR_TIMEOUT, 0x200u);
-                            alive = false;                  // carry zero; error recorded
-                            break;
+                            break;                          // carry zero; error recorded
                         }
                         __nanosleep(32);
                     }
@@ -334,70 +348,61 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
         f2_t hk[NP], hv[NP];
 #pragma unroll
         for (int q = 0; q < NP; ++q) {
-            const int ch = cl * VEC + 2 * q;
+            const int ch = chq[q];
             const f2_t wk = f2(sw[(pwarp * 3 + 0) * DH + ch], sw[(pwarp * 3 + 0) * DH + ch + 1]);
             const f2_t wv = f2(sw[(pwarp * 3 + 1) * DH + ch], sw[(pwarp * 3 + 1) * DH + ch + 1]);
             hk[q] = f2_fma(eA[q], wk, eK[q]);
             hv[q] = f2_fma(eA[q], wv, eV[q]);
         }
-        // RoPE: rotation (rc + i rs) of this lane's channels at its first row, advanced one
-        // position per row by (sc + i ss); the first half of the channels takes x cos - x' sin
-        f2_t rc[NP], rs[NP], sc[NP], ss[NP], nss[NP];
-        const bool first_half = cl < LPR / 2;
+        // RoPE: angle (rc, rs) of frequencies 2cl, 2cl+1 at this segment's first row, advanced one
+        // position per row by the rotation (sc, ss).  Pair 0 (first half) takes
+        // x cos - x' sin, pair 1 (second half) x' cos + x sin.
+        f2_t rc = kOne2, rs = kZero2, sc = kOne2, ss = kZero2, nss = kZero2;
         if (p.rope) {
             const long long pos = p.pos0 + t0 + seg * R;
+            float c2[2], s2[2];
 #pragma unroll
-            for (int q = 0; q < NP; ++q) {
-                float c2[2], s2[2], a2[2], b2[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int f = (cl * VEC + 2 * q + u) % (DH / 2);
-                    if (p.rope_f32) rope_cs_f32((int)pos, p.theta_f[f], c2[u], s2[u]);
-                    else rope_cs(pos, p.theta[f], c2[u], s2[u]);
-                    a2[u] = p.step_cos[f];
-                    b2[u] = first_half ? -p.step_sin[f] : p.step_sin[f];
-                    if (first_half) s2[u] = -s2[u];
-                }
-                rc[q] = f2(c2[0], c2[1]);
-                rs[q] = f2(s2[0], s2[1]);
-                sc[q] = f2(a2[0], a2[1]);
-                ss[q] = f2(b2[0], b2[1]);
-                nss[q] = f2(-b2[0], -b2[1]);
+            for (int u = 0; u < 2; ++u) {
+                const int f = 2 * cl + u;
+                if (p.rope_f32) rope_cs_f32((int)pos, s_theta_f[f], c2[u], s2[u]);
+                else rope_cs(pos, s_theta[f], c2[u], s2[u]);
             }
+            rc = f2(c2[0], c2[1]);
+            rs = f2(s2[0], s2[1]);
+            sc = f2(s_step_c[2 * cl], s_step_c[2 * cl + 1]);
+            ss = f2(s_step_s[2 * cl], s_step_s[2 * cl + 1]);
+            nss = f2(-s_step_s[2 * cl], -s_step_s[2 * cl + 1]);
         }
+        const f2_t kNegOne2 = f2(-1.f, -1.f);
         uint8_t *yk = static_cast<uint8_t *>(p.yk);
         uint8_t *yv = static_cast<uint8_t *>(p.yv);
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             const int r = seg * R + i;
-            const int rr = r < rows ? r : rows - 1;
-            const int off = rr * C::ROWB + cl * 16;
+            const int off = (r < rows ? r : rows - 1) * C::ROWB;
             f2_t xk[NP], xv[NP];
-            Vec<E>::load(sk + off, xk);
-            Vec<E>::load(sv + off, xv);
-            f2_t ok[NP];
+            Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
+            Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
-                hk[q] = f2_fma(G[i][q], hk[q], f2_mul(OG[i][q], xk[q]));
-                hv[q] = f2_fma(G[i][q], hv[q], f2_mul(OG[i][q], xv[q]));
-                ok[q] = hk[q];
+                const f2_t og = gate_complement2(G[i][q]);
+                hk[q] = f2_fma(G[i][q], hk[q], f2_mul(og, xk[q]));
+                hv[q] = f2_fma(G[i][q], hv[q], f2_mul(og, xv[q]));
             }
-            if (p.rope) {       // uniform across the grid: the shuffles see every lane
-#pragma unroll
-                for (int q = 0; q < NP; ++q) {
-                    const f2_t partner = f2(__shfl_xor_sync(0xffffffffu, f2lo(hk[q]), LPR / 2),
-                                            __shfl_xor_sync(0xffffffffu, f2hi(hk[q]), LPR / 2));
-                    ok[q] = f2_fma(hk[q], rc[q], f2_mul(partner, rs[q]));
-                    // advance one position: (c + i s)(cos t + i sin t)
-                    const f2_t nc = f2_fma(rc[q], sc[q], f2_mul(rs[q], nss[q]));
-                    rs[q] = f2_fma(rs[q], sc[q], f2_mul(rc[q], ss[q]));
-                    rc[q] = nc;
-                }
+            f2_t ok[NP] = {hk[0], hk[1]};
+            if (p.rope) {
+                const f2_t nrs = f2_mul(rs, kNegOne2);
+                ok[0] = f2_fma(hk[1], nrs, f2_mul(hk[0], rc));
+                ok[1] = f2_fma(hk[0], rs, f2_mul(hk[1], rc));
+                // advance one position: (c + i s)(cos t + i sin t)
+                const f2_t nc = f2_fma(rc, sc, f2_mul(rs, nss));
+                rs = f2_fma(rs, sc, f2_mul(rc, ss));
+                rc = nc;
             }
             if (r < rows) {
-                const size_t go = (row0 + r) * C::ROWB + cl * 16;
-                Vec<E>::store(yk + go, ok);
-                Vec<E>::store(yv + go, hv);
+                const size_t go = (row0 + r) * C::ROWB;
+                Lane<E>::template store<C::HALFB>(yk + go, cl, ok);
+                Lane<E>::template store<C::HALFB>(yv + go, cl, hv);
             }
         }
         pipe_sync();     // this stage's smem and sw are free for the next chunk
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(256, 1) recur_kernel(const __grid_constant__ R
 
 int recur_chunk_rows(int d, int dtype) {
     const int eb = dtype == RAT_F32 ? 4 : 2;
-    return (128 / (d * eb / 16)) * 8;      // (threads per pipeline / lanes per row) x 8 rows
+    return 16384 / (d * eb);               // one 16 KiB tile per tensor
 }
 
 size_t recur_workspace_bytes(int BH, int T, int d, int dtype) {
