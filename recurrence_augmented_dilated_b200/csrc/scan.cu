@@ -132,6 +132,21 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
         bulk_g2s(s + 2 * C::TILEB, static_cast<const uint8_t *>(p.v) + row0 * C::ROWB, bytes, &bar[pipe][st]);
     };
     auto pipe_sync = [&]() { asm volatile("bar.sync %0, %1;" :: "r"(barid), "r"(C::PT) : "memory"); };
+    // one look-back round of channel `ch` of (b, h) = bh: predecessors j, j-1, ..., j-LBW+1
+    // (clamped at 0), each its inclusive state (k, v) and its aggregate (A, Bk, Bv)
+    auto read_window = [&](int bh, int j, int ch, uint64_t (&w)[C::LBW][5]) {
+#pragma unroll
+        for (int u = 0; u < C::LBW; ++u) {
+            const size_t jid = (size_t)bh * p.nchunks + max(j - u, 0);
+            const uint64_t *pj = p.pre + jid * 2 * DH + ch;
+            const uint64_t *aj = p.agg + jid * 3 * DH + ch;
+            w[u][0] = ld_relaxed_gpu_u64(pj);
+            w[u][1] = ld_relaxed_gpu_u64(pj + DH);
+            w[u][2] = ld_relaxed_gpu_u64(aj);
+            w[u][3] = ld_relaxed_gpu_u64(aj + DH);
+            w[u][4] = ld_relaxed_gpu_u64(aj + 2 * DH);
+        }
+    };
 
     if (tid < HALF) {           // RoPE tables, read per lane below without divergent constant loads
         s_theta_f[tid] = p.theta_f[tid];
@@ -175,6 +190,10 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
         const size_t row0 = (size_t)bh * p.T + t0;
         const bool publish = c != p.fault_chunk;            // false only under the test hook
         const uint8_t *sa = pbase + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
+        // the first look-back round is issued now and consumed after pass 1, so its memory
+        // latency overlaps the wait for the data and pass 1
+        uint64_t w[C::LBW][5];
+        if (pt < DH && c > 0) read_window(bh, c - 1, pt, w);
         mbar_wait_bounded(&bar[pipe][st], (it >> 1) & 1, hdr, 0x100u);
 
         // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate
@@ -275,19 +294,8 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
                 const uint64_t t_start = globaltimer_ns();
                 uint32_t spins = 0;
                 int j = c - 1;
-                for (;;) {
-                    uint64_t w[C::LBW][5];
-#pragma unroll
-                    for (int u = 0; u < C::LBW; ++u) {
-                        const size_t jid = (size_t)bh * p.nchunks + max(j - u, 0);
-                        const uint64_t *pj = p.pre + jid * 2 * DH + ch;
-                        const uint64_t *aj = p.agg + jid * 3 * DH + ch;
-                        w[u][0] = ld_relaxed_gpu_u64(pj);
-                        w[u][1] = ld_relaxed_gpu_u64(pj + DH);
-                        w[u][2] = ld_relaxed_gpu_u64(aj);
-                        w[u][3] = ld_relaxed_gpu_u64(aj + DH);
-                        w[u][4] = ld_relaxed_gpu_u64(aj + 2 * DH);
-                    }
+                for (bool first = true;; first = false) {
+                    if (!first) read_window(bh, j, ch, w);      // round 0 was read before pass 1
                     bool done = false, stop = false;
                     int passed = 0;
 #pragma unroll
