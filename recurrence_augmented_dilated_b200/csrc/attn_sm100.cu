@@ -25,7 +25,9 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "tc.cuh"
 
@@ -35,6 +37,12 @@ __device__ int g_attn_error;     // first device-side error of the attention ker
 __device__ unsigned g_attn_where; // where it happened: (site << 24) | (block << 8) | parity
 __device__ unsigned g_attn_waiting; // bit s set: a wait at site s was in progress when a CTA aborted
 
+// (cos, sin)(l * theta_f) for l < 32 and the 64 RoPE frequencies, [f][l], formed on the host in
+// float64; the producer copies a launch's table next to Q.  kRelSlots tables per device, one per
+// distinct frequency set in use (replaced round-robin).
+constexpr int kRelSlots = 4;
+__device__ float2 g_rope_rel[kRelSlots][64 * 32];
+
 namespace {
 
 constexpr int BM = 128;               // query rows per tile
@@ -43,7 +51,8 @@ constexpr int NS = 2;                 // K/V pipeline stages
 constexpr int kThreads = 192;         // warp 0: TMA, warp 1: MMA, warps 2-5: softmax / epilogue
 constexpr uint32_t QSUB = BM * 128;   // one [128 rows][64 bf16] 128B-swizzled sub-tile of Q / O
 constexpr int kMaxDil = 4;
-constexpr float kRescaleLog2 = 8.0f;  // move the running max only when it grows by > 2^8
+constexpr float kRescaleLog2 = 8.0f;
+constexpr uint32_t kRelBytes = 64 * 32 * 8;   // the RoPE table g_rope_rel  // move the running max only when it grows by > 2^8
 
 // Shared-memory / TMEM plan for key blocks of BN keys.
 template <int BN>
@@ -86,6 +95,7 @@ struct Params {
     int grp_head0[kMaxHeads];       // first index into head_of
     int grp_nheads[kMaxHeads];
     int rope_f32;             // positions small enough for float32 angles (pos0 + T <= 2^13)
+    const float2 *rope_rel;   // device table [64 f][32 l] of (cos, sin)(l theta_f), see g_rope_rel
     float theta_f[64];
     double theta[64];
 };
@@ -240,9 +250,11 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             tc::prefetch_tmap(&p.tm_q);
             tc::prefetch_tmap(mk);
             tc::prefetch_tmap(&p.tm_k);
-            mbar_arrive_expect_tx(&sh.q_full, 2 * QSUB);
+            mbar_arrive_expect_tx(&sh.q_full, 2 * QSUB + (p.rope ? kRelBytes : 0u));
             tc::tma_load_3d(smem + C::OFF_Q, &p.tm_q, 0, t0, bh, &sh.q_full);
             tc::tma_load_3d(smem + C::OFF_Q + QSUB, &p.tm_q, 64, t0, bh, &sh.q_full);
+            // RoPE: the relative rotation table goes to the second K stage, unused until Q is rotated
+            if (p.rope) bulk_g2s(smem + C::OFF_K + C::KTILE, p.rope_rel, kRelBytes, &sh.q_full);
             int issued = 0;
             for (int j = 0; j < nb; ++j) {
                 const int s = j % NS;
@@ -343,19 +355,13 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         uint4 xrow[16];
         if (self_reg) load_rows(p.kg, xrow);         // k~ of the tile's rows, in flight with Q
         // rotate-half RoPE of the Q tile at positions pos0 + t.  Rotation of row 32w + l is
-        // rot(base_w) * rot(l): while Q is in flight the softmax threads tabulate rot(l theta_f) for
-        // l < 32 and rot((pos0 + t0 + 32w) theta_f) in the still-unused second K/V stage; once Q has
-        // landed each thread rotates its own row.
-        float2 *rel = reinterpret_cast<float2 *>(smem + C::OFF_K + C::KTILE);    // [64 f][32 l]
-        float2 *bas = reinterpret_cast<float2 *>(smem + C::OFF_V + C::KTILE);    // [4 w][64 f]
+        // rot(base_w) * rot(l): rot(l theta_f) for l < 32 arrives with Q (the launch's table, copied
+        // into the still-unused second K stage); while Q is in flight the softmax threads tabulate
+        // rot((pos0 + t0 + 32w) theta_f) in the second V stage; once Q has landed each thread
+        // rotates its own row.
+        const float2 *rel = reinterpret_cast<const float2 *>(smem + C::OFF_K + C::KTILE);  // [64 f][32 l]
+        float2 *bas = reinterpret_cast<float2 *>(smem + C::OFF_V + C::KTILE);              // [4 w][64 f]
         if (p.rope) {
-#pragma unroll 4
-            for (int k = 0; k < 16; ++k) {
-                const int e = r + 128 * k, f = e >> 5, l = e & 31;
-                float cs, sn;
-                rope_cs_f32(l, p.theta_f[f], cs, sn);
-                rel[e] = make_float2(cs, sn);
-            }
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 const int e = r + 128 * k, w = e >> 6, f = e & 63;
@@ -401,26 +407,36 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         float m_run = -INFINITY, l_run = 0.f;
         float w_self = 0.f;        // weight of the self key when it is kept in registers
         if (ok && self_reg) {
-            // s_self = q^_t . k~_t: partial dots over 8 channels per lane, summed over the 16 lanes
-            // of a row, then handed to the lane that owns the row
+            // s_self = q^_t . k~_t: partial dots over 8 channels per lane for the 16 row pairs,
+            // reduced over the 16 lanes of each half-warp by a transposing butterfly (after it,
+            // lane l of half h holds the whole dot of row 2 (l & 15) + h), then handed to the lane
+            // that owns the row
             __syncwarp();          // this warp's rows of q^ are rotated
-            float dot = 0.f;
+            float part[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const uint4 qq = *reinterpret_cast<const uint4 *>(sQ + (xc >> 3) * QSUB + swz(xr + 2 * k, xc & 7));
                 const uint32_t ku[4] = {xrow[k].x, xrow[k].y, xrow[k].z, xrow[k].w};
                 const uint32_t qu[4] = {qq.x, qq.y, qq.z, qq.w};
-                float part = 0.f;
+                float d = 0.f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    part = fmaf(bf16_lo(qu[i]), bf16_lo(ku[i]), part);
-                    part = fmaf(bf16_hi(qu[i]), bf16_hi(ku[i]), part);
+                    d = fmaf(bf16_lo(qu[i]), bf16_lo(ku[i]), d);
+                    d = fmaf(bf16_hi(qu[i]), bf16_hi(ku[i]), d);
                 }
-#pragma unroll
-                for (int o = 8; o >= 1; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-                const float row_dot = __shfl_sync(0xffffffffu, part, (lane & 1) << 4);
-                if ((lane >> 1) == k) dot = row_dot;
+                part[k] = d;
             }
+#pragma unroll
+            for (int o = 8; o >= 1; o >>= 1) {
+                const bool upper = (lane & o) != 0;   // keeps the upper half of its o*2 values
+#pragma unroll
+                for (int i = 0; i < o; ++i) {
+                    const float keep = upper ? part[i + o] : part[i];
+                    const float send = upper ? part[i] : part[i + o];
+                    part[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+                }
+            }
+            const float dot = __shfl_sync(0xffffffffu, part[0], ((lane & 1) << 4) | (lane >> 1));
             m_run = dot * p.scale_log2;
             w_self = 1.f;
         }
@@ -1168,17 +1184,19 @@ int launch_tiles(const Params &p, int items, void *stream) {
 }
 
 template <int BN>
-int launch_bn(const AttnSm100Args &a, void *stream) {
+int launch_bn(const AttnSm100Args &a, const float2 *rel, void *stream) {
     Params p;          // copied into the launch's parameter space
     const int items = fill_params<BN>(p, a);
     if (items < 0) return items;
+    p.rope_rel = rel;
     return a.W <= 1 ? launch_tiles<BN, true>(p, items, stream) : launch_tiles<BN, false>(p, items, stream);
 }
 
-int launch_persistent(const AttnSm100Args &a, void *stream) {
+int launch_persistent(const AttnSm100Args &a, const float2 *rel, void *stream) {
     Params p;
     const int items = fill_params<pk::BN>(p, a);
     if (items < 0) return items;
+    p.rope_rel = rel;
     static uint64_t attr_done = 0;
     const int st = set_smem_attr(reinterpret_cast<const void *>(pk::attn_persist_kernel), pk::SMEM_BYTES, &attr_done);
     if (st != RAT_OK) return st;
@@ -1194,11 +1212,52 @@ int launch_persistent(const AttnSm100Args &a, void *stream) {
 int g_attn_block_keys = 0;   // 0: automatic; 64 or 128 forces the key-block width
 int g_attn_schedule = 0;     // 0: automatic (one CTA per tile), 1: one CTA per tile, 2: persistent
 
+// The device table of a launch's RoPE frequencies: uploaded (stream-ordered) the first time a
+// frequency set is seen on this device, then reused.
+static int rope_rel_table(const double *theta, void *stream, const float2 **out) {
+    struct Slot { double theta[64]; bool valid; };
+    static std::mutex mu;
+    static Slot slots[64][kRelSlots];
+    static float2 *base[64];
+    static int next[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RAT_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!base[dev] && cudaGetSymbolAddress(reinterpret_cast<void **>(&base[dev]), g_rope_rel) != cudaSuccess)
+        return RAT_ERR_CUDA;
+    for (int i = 0; i < kRelSlots; ++i) {
+        if (slots[dev][i].valid && std::memcmp(slots[dev][i].theta, theta, sizeof(double) * 64) == 0) {
+            *out = base[dev] + (size_t)i * 64 * 32;
+            return RAT_OK;
+        }
+    }
+    const int i = next[dev];
+    next[dev] = (i + 1) % kRelSlots;
+    static float2 tab[64 * 32];      // guarded by mu; staged by the copy before it returns
+    for (int f = 0; f < 64; ++f)
+        for (int l = 0; l < 32; ++l) {
+            const double ang = (double)l * theta[f];
+            tab[f * 32 + l] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+        }
+    if (cudaMemcpyToSymbolAsync(g_rope_rel, tab, sizeof(tab), (size_t)i * sizeof(tab), cudaMemcpyHostToDevice,
+                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return RAT_ERR_CUDA;
+    std::memcpy(slots[dev][i].theta, theta, sizeof(double) * 64);
+    slots[dev][i].valid = true;
+    *out = base[dev] + (size_t)i * 64 * 32;
+    return RAT_OK;
+}
+
 int launch_attn_sm100(const AttnSm100Args &a, void *stream) {
     if (a.d != DHEAD) return RAT_ERR_UNSUPPORTED;
-    if (g_attn_schedule == 2 && g_attn_block_keys != 128) return launch_persistent(a, stream);
+    const float2 *rel = nullptr;
+    if (a.rope) {
+        const int st = rope_rel_table(a.theta, stream, &rel);
+        if (st != RAT_OK) return st;
+    }
+    if (g_attn_schedule == 2 && g_attn_block_keys != 128) return launch_persistent(a, rel, stream);
     const int bn = g_attn_block_keys ? g_attn_block_keys : 64;
-    return bn == 64 ? launch_bn<64>(a, stream) : launch_bn<128>(a, stream);
+    return bn == 64 ? launch_bn<64>(a, rel, stream) : launch_bn<128>(a, rel, stream);
 }
 
 int attn_error_word(void *stream, bool clear) {

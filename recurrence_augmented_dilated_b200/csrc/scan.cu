@@ -268,10 +268,10 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
             const int ch = pt;
             float cA = 1.f, cK = 0.f, cV = 0.f;
 #pragma unroll
-            for (int w = 0; w < C::PW; ++w) {
-                const float a = sw[(w * 3 + 0) * DH + ch];
-                cK = fmaf(a, cK, sw[(w * 3 + 1) * DH + ch]);
-                cV = fmaf(a, cV, sw[(w * 3 + 2) * DH + ch]);
+            for (int wp = 0; wp < C::PW; ++wp) {
+                const float a = sw[(wp * 3 + 0) * DH + ch];
+                cK = fmaf(a, cK, sw[(wp * 3 + 1) * DH + ch]);
+                cV = fmaf(a, cV, sw[(wp * 3 + 2) * DH + ch]);
                 cA *= a;
             }
             if (c > 0 && publish) {
@@ -339,12 +339,12 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
             }
             float hK = Hk, hV = Hv;
 #pragma unroll
-            for (int w = 0; w < C::PW; ++w) {
-                const float a = sw[(w * 3 + 0) * DH + ch];
-                const float bk = sw[(w * 3 + 1) * DH + ch];
-                const float bv = sw[(w * 3 + 2) * DH + ch];
-                sw[(w * 3 + 0) * DH + ch] = hK;
-                sw[(w * 3 + 1) * DH + ch] = hV;
+            for (int wp = 0; wp < C::PW; ++wp) {
+                const float a = sw[(wp * 3 + 0) * DH + ch];
+                const float bk = sw[(wp * 3 + 1) * DH + ch];
+                const float bv = sw[(wp * 3 + 2) * DH + ch];
+                sw[(wp * 3 + 0) * DH + ch] = hK;
+                sw[(wp * 3 + 1) * DH + ch] = hV;
                 hK = fmaf(a, hK, bk);
                 hV = fmaf(a, hV, bv);
             }
