@@ -6,13 +6,22 @@
 //   - each chunk end p = i*D_h + D_h - 1 (i < cap_h) to dil entry i of head h, and
 //   - each of the last min(W, T) positions p to ring slot p mod W,
 // for k~ and v~, bit for bit; and copies the final recurrence state into the cache.
-// One CTA per (row block, b*h); 16-byte vector copies, one row per LPR lanes.
+// One CTA per (row block, b*h); 16-byte vector copies, one row per LPR lanes, four rows per
+// thread in flight at once.
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace rat {
 
 __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ CompressParams p) {
-    const int bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
+    // flat grid: per batch row, head h owns CTAs blk0[h] .. blk0[h+1]-1
+    const int per_b = p.blk0[p.H];
+    const int b = (int)blockIdx.x / per_b, rb = (int)blockIdx.x % per_b;
+    int h = 0;
+    while (rb >= p.blk0[h + 1]) ++h;
+    const int bh = b * p.H + h;
+    const int blk = rb - p.blk0[h], nblk = p.blk0[h + 1] - p.blk0[h];
     const long long D = p.Dh[h];
     const long long cap = p.Tcap / D;
     const long long end = p.pos0 + p.T;
@@ -29,12 +38,11 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
 
     const uint8_t *src_k = static_cast<const uint8_t *>(p.k) + (size_t)bh * p.T * row_bytes;
     const uint8_t *src_v = static_cast<const uint8_t *>(p.v) + (size_t)bh * p.T * row_bytes;
-    for (long long job = (long long)blockIdx.x * rows_per_pass + lane_r; job < njobs;
-         job += (long long)gridDim.x * rows_per_pass) {
+    // job -> (source row, destination row) of this (b, h)
+    auto locate = [&](long long job, const uint8_t *&src, uint8_t *&dst) {
         const bool is_v = job >= n_dil + n_ring;
         const long long r = is_v ? job - (n_dil + n_ring) : job;
         long long pos;
-        uint8_t *dst;
         if (r < n_dil) {
             const long long i = i_lo + r;
             pos = i * D + D - 1;
@@ -45,12 +53,30 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
             uint8_t *base = static_cast<uint8_t *>(is_v ? p.vwin : p.kwin);
             dst = base + (((size_t)b * p.H + h) * p.W + (size_t)(pos % p.W)) * row_bytes;
         }
-        const uint8_t *src = (is_v ? src_v : src_k) + (size_t)(pos - p.pos0) * row_bytes;
-        const uint4 val = *reinterpret_cast<const uint4 *>(src + lane_c * 16);
-        *reinterpret_cast<uint4 *>(dst + lane_c * 16) = val;
+        src = (is_v ? src_v : src_k) + (size_t)(pos - p.pos0) * row_bytes;
+    };
+    // kU jobs per thread and trip, their loads issued together before the stores
+    constexpr int kU = 4;
+    const long long stride = (long long)nblk * rows_per_pass;
+    for (long long base = (long long)blk * rows_per_pass + lane_r; base < njobs; base += kU * stride) {
+        uint4 val[kU];
+        uint8_t *dst[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const long long job = base + u * stride;
+            dst[u] = nullptr;
+            if (job < njobs) {
+                const uint8_t *src;
+                locate(job, src, dst[u]);
+                val[u] = *reinterpret_cast<const uint4 *>(src + lane_c * 16);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+            if (dst[u]) *reinterpret_cast<uint4 *>(dst[u] + lane_c * 16) = val[u];
     }
     // recurrence state (float32), once per (b, h)
-    if (blockIdx.x == 0) {
+    if (blk == 0) {
         for (int c = threadIdx.x; c < p.d; c += blockDim.x) {
             if (p.hTk && p.hk != p.hTk) p.hk[(size_t)bh * p.d + c] = p.hTk[(size_t)bh * p.d + c];
             if (p.hTv && p.hv != p.hTv) p.hv[(size_t)bh * p.d + c] = p.hTv[(size_t)bh * p.d + c];
@@ -58,21 +84,25 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
     }
 }
 
-int launch_compress(const CompressParams &p, void *stream) {
-    // enough CTAs per (b, h) to cover its dil rows in a few passes
-    long long max_rows = 0;
+int launch_compress(const CompressParams &p_in, void *stream) {
+    // CTAs per head: enough for about kU rows per thread, at least one (it copies the state)
+    CompressParams p = p_in;
+    const int rows_per_pass = 256 / (p.d * p.esize / 16);
+    int acc = 0;
     for (int h = 0; h < p.H; ++h) {
         const long long D = p.Dh[h];
-        const long long n = min((p.pos0 + p.T) / D, p.Tcap / D) - p.pos0 / D;
-        max_rows = n > max_rows ? n : max_rows;
+        const long long n_dil = std::max(0ll, std::min((p.pos0 + p.T) / D, p.Tcap / D) - p.pos0 / D);
+        const long long n_ring = p.W > 0 ? std::min(p.W, p.T) : 0;     // the last min(W, T) positions
+        const long long jobs = 2 * (n_dil + n_ring);
+        long long n = (jobs + rows_per_pass * 4 - 1) / (rows_per_pass * 4);
+        n = std::max(1ll, std::min(n, 4096ll));
+        p.blk0[h] = acc;
+        acc += (int)n;
     }
-    max_rows = 2 * (max_rows + p.W);
-    const int rows_per_pass = 256 / (p.d * p.esize / 16);
-    long long gx = (max_rows + rows_per_pass * 4 - 1) / (rows_per_pass * 4);
-    if (gx < 1) gx = 1;
-    if (gx > 1024) gx = 1024;
-    dim3 grid((unsigned)gx, (unsigned)(p.B * p.H));
-    compress_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    p.blk0[p.H] = acc;
+    const long long grid = (long long)acc * p.B;
+    if (grid > 0x7fffffffll) return RAT_ERR_UNSUPPORTED;
+    compress_kernel<<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 

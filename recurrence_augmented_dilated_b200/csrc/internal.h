@@ -113,6 +113,7 @@ struct CompressParams {
     long long total_cap;
     int Dh[kMaxHeads];
     long long off[kMaxHeads];
+    int blk0[kMaxHeads + 1];    // filled by launch_compress: first CTA of head h within a batch row
 };
 int launch_compress(const CompressParams &p, void *stream);
 

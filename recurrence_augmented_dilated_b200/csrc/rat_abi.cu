@@ -243,7 +243,6 @@ int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, con
     if (!aligned16(k_rec) || !aligned16(v_rec) || !aligned16(c->k_dil) || !aligned16(c->v_dil) ||
         (c->W > 0 && (!aligned16(c->k_win) || !aligned16(c->v_win))))
         return RAT_ERR_INVALID;
-    if ((long long)c->B * c->H > 65535) return RAT_ERR_UNSUPPORTED;
     CompressParams p;
     std::memset(&p, 0, sizeof(p));
     p.k = k_rec; p.v = v_rec; p.hTk = hT_k; p.hTv = hT_v;
