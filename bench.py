@@ -303,7 +303,15 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
         res["kernels"][name] = e
     res["algorithmic"] = alg
     if with_e2e:
-        res["e2e"] = run_e2e(w, steps, warmup, step, x, (q, k, v, a), o, world)
+        o_ref = o.clone()
+        res["e2e"] = run_e2e(w, steps, warmup, x, {"q": q, "k": k, "v": v, "a": a, "kr": kr, "vr": vr,
+                                                  "o": o, "hk": hk, "hv": hv}, world)
+        # the host-buffer path must reproduce the device path's output (up to the rounding order
+        # of the scan's look-back)
+        diff = (res["e2e"].pop("out").float() - o_ref.cpu().float()).abs().max().item()
+        scale = o_ref.float().abs().max().item()
+        if not diff <= 1e-2 * max(scale, 1e-30):
+            raise RuntimeError("end-to-end output differs from the device path: %g" % diff)
     return res
 
 
@@ -315,34 +323,77 @@ class _Null:
         return False
 
 
-def run_e2e(w, steps, warmup, step, x, dev_inputs, o, world):
-    """Same step through the public API with host buffers: H2D of q, k, v, a from pinned memory
-    and D2H of the output inside the timed region."""
-    host = [x[n].pin_memory() for n in ("q", "k", "v", "a")]
+def run_e2e(w, steps, warmup, x, dev, world):
+    """The layer step through the public API from host buffers: for each batch row, the H2D copy
+    of its q, k, v, a from pinned memory, the three calls, and the D2H copy of its output, on
+    three streams (copy in, compute, copy out) so that one row's copies overlap another row's
+    compute. Every copy of the step is inside the timed region."""
+    import recurrence_augmented_dilated_b200 as rat
+    names = ("q", "k", "v", "a")
+    host = {n: x[n].pin_memory() for n in names}
+    o, kr, vr, hk, hv = dev["o"], dev["kr"], dev["vr"], dev["hk"], dev["hv"]
     out_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    stream = torch.cuda.current_stream()
+    B, H, T, d = o.shape
+    dtc = rat.F32 if w.dtype == "f32" else rat.BF16
+    Dph = list(w.D_per_head) if w.D_per_head else None
+    # one cache and one scan workspace per batch row (calls on one row never overlap themselves)
+    caches = [rat.make_cache(1, H, d, w.W, T, dtc, w.heads_D()) for _ in range(B)]
+    ws = [rat.Workspace(rat.rat_recur_workspace_bytes(1, H, T, d, dtc)) for _ in range(B)]
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(B)]
+    ev_comp = [torch.cuda.Event() for _ in range(B)]
+    ev_out = [torch.cuda.Event() for _ in range(B)]
 
     def e2e_step():
-        for hsrc, dst in zip(host, dev_inputs):
-            dst.copy_(hsrc, non_blocking=True)
-        step()
-        out_host.copy_(o, non_blocking=True)
+        for b in range(B):
+            r = slice(b, b + 1)
+            s_in.wait_event(ev_comp[b])          # the previous step's row b no longer needs its inputs
+            with torch.cuda.stream(s_in):
+                for n in names:
+                    dev[n][r].copy_(host[n][r], non_blocking=True)
+                ev_in[b].record(s_in)
+            s_comp.wait_event(ev_in[b])
+            s_comp.wait_event(ev_out[b])         # the previous step's row b output has been read
+            with torch.cuda.stream(s_comp):
+                rat.rat_recur_prefill(dev["k"][r], dev["v"][r], dev["a"][r], kr[r], vr[r], ws[b],
+                                      hT_k=hk[r], hT_v=hv[r], rope_base=w.rope_base)
+                rat.rat_dilated_attn_prefill(dev["q"][r], kr[r], vr[r], o[r], D=w.D, W=w.W,
+                                             D_per_head=Dph, rope_base=w.rope_base)
+                cache = caches[b][0]
+                cache.pos = 0
+                rat.rat_kv_compress(kr[r], vr[r], hk[r], hv[r], cache)
+                ev_comp[b].record(s_comp)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                out_host[r].copy_(o[r], non_blocking=True)
+                ev_out[b].record(s_out)
 
+    cur = torch.cuda.current_stream()
     for _ in range(max(1, warmup)):
         e2e_step()
     torch.cuda.synchronize()
+    for b in range(B):
+        if rat.rat_sync_status(ws[b]) != 0:
+            raise RuntimeError("device error in the end-to-end leg")
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e0.record(cur)
+    for s_ in (s_in, s_comp, s_out):
+        s_.wait_event(e0)
     for _ in range(steps):
         e2e_step()
-    e1.record(stream)
+    done = torch.cuda.Event()
+    done.record(s_out)
+    cur.wait_event(done)
+    e1.record(cur)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
-    h2d = sum(t.numel() * t.element_size() for t in host)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = out_host.numel() * out_host.element_size()
     return {"value": world * w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "method": "per batch row: H2D, recurrence + attention + compress, D2H on three streams",
+            "out": out_host}
 
 
 def run_decode(w: synthetic.Workload, steps_timed: int, warmup: int, rank: int, world: int, peaks,
