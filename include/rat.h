@@ -161,11 +161,6 @@ RAT_API uint32_t rat_attn_error_waiting(void);
  * (one CTA per SM); 0 restores the automatic choice.  Process-wide; RAT_ERR_INVALID otherwise. */
 RAT_API int rat_set_attn_block_keys(int block_keys);
 
-/* Tuning knob of the bf16 tensor-core attention schedule: 0 (automatic) and 1 run one CTA per
- * 128-query tile; 2 runs one persistent CTA per SM that prepares the next tile's queries and
- * writes the previous tile's output while the current tile's key blocks run (64-key blocks).
- * Block width 128 always uses one CTA per tile.  Process-wide; RAT_ERR_INVALID otherwise. */
-RAT_API int rat_set_attn_schedule(int schedule);
 
 /* ------------------------------------------------------------------------------------------
  * Compressed KV cache (RAT+ abstract: dilation reduces the KV cache D-fold; "RAT+ Deep Dive"

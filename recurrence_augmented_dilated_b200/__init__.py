@@ -23,7 +23,7 @@ __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
-    "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_set_attn_schedule", "rat_attended_keys", "rat_status_string",
+    "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
     "Workspace", "rat_dilated_decode_noalloc",
 ]
 
@@ -90,7 +90,6 @@ def lib():
         L.rat_attn_error_site.restype = ctypes.c_uint32
         L.rat_attn_error_waiting.restype = ctypes.c_uint32
         L.rat_set_attn_block_keys.argtypes = [_i]
-        L.rat_set_attn_schedule.argtypes = [_i]
         L.rat_attended_keys.restype = _i64
         L.rat_attended_keys.argtypes = [_i64, _i, _i]
         _lib = L
@@ -157,10 +156,6 @@ def rat_attn_sync_status(stream=None) -> int:
 
 def rat_set_attn_block_keys(block_keys: int) -> None:
     _check("rat_set_attn_block_keys", lib().rat_set_attn_block_keys(int(block_keys)))
-
-
-def rat_set_attn_schedule(schedule: int) -> None:
-    _check("rat_set_attn_schedule", lib().rat_set_attn_schedule(int(schedule)))
 
 
 def rat_recur_workspace_bytes(B, H, T, d, dtype) -> int:

@@ -583,490 +583,6 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
     if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
-// ============================================================================ persistent variant
-// One CTA per SM walks a strided share of the (longest-first) tile list.  Warp 0 issues TMA
-// loads (Q double-buffered, 3-stage K/V ring), warp 1 the MMAs over a flat sequence of key blocks
-// that crosses tile boundaries, warps 2-5 (softmax) handle only the key blocks, and warps 6-9
-// (prologue / epilogue) rotate and score the self key of tile i+1 and write out tile i while
-// the softmax works.  TMEM: two S buffers (P aliased in their first half) and one O accumulator
-// per tile slot.  Every mbarrier is either per slot (one phase per tile of that slot) or
-// alternates with the parity of the global block index, so no waiter can find a barrier two
-// phases ahead of the phase it waits for.
-namespace pk {
-constexpr int BN = 64;
-constexpr int NSTG = 3;
-constexpr int kThreadsP = 320;
-constexpr uint32_t KSUB = BN * 128;              // [64 keys][64 bf16] sub-tile
-constexpr uint32_t KTILE = 2 * KSUB;
-constexpr uint32_t OFF_Q = 0;                    // Q[2]: 2 x 32 KiB
-constexpr uint32_t OFF_K = 4 * QSUB;             // K ring: 3 x 16 KiB
-constexpr uint32_t OFF_V = OFF_K + NSTG * KTILE; // V ring: 3 x 16 KiB
-constexpr uint32_t OFF_REL = OFF_V + NSTG * KTILE;   // rot(l theta_f), [64 f][32 l] float2
-constexpr uint32_t OFF_BAS = OFF_REL + 16384;        // rot(row-group base), [2 slot][4 w][64 f] float2
-constexpr uint32_t OFF_STAT = OFF_BAS + 4096;        // per-row handoff floats (see below)
-constexpr uint32_t OFF_BAR = OFF_STAT + 4096;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 512;
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_O = 128;                  // O of slot a at 128 + 128 a; S(g) at 64 (g & 1)
-
-struct Bars {
-    uint64_t q_full[2], q_ready[2], q_empty[2];
-    uint64_t kv_full[NSTG], kv_empty[NSTG];
-    uint64_t s_full[2], p_full[2], o_ready[2];
-    uint64_t tile_done[2], o_done[2], o_free[2];
-    uint64_t fin;
-    uint32_t tmem;
-    volatile int abort;
-};
-static_assert(sizeof(Bars) <= 512, "barrier block");
-
-RAT_DEVICE bool pwait(Bars &sh, uint64_t *bar, uint32_t parity, uint32_t site, uint32_t blk = 0) {
-    if (mbar_try_wait(bar, parity)) return true;
-    const uint64_t t0 = globaltimer_ns();
-    for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if (sh.abort) {
-            atomicOr(&g_attn_waiting, 1u << site);
-            return false;
-        }
-        if (globaltimer_ns() - t0 > kWaitLimitNs) {
-            sh.abort = 1;
-            if (atomicCAS(&g_attn_error, 0, RAT_ERR_TIMEOUT) == 0)
-                g_attn_where = (site << 24) | ((blk & 0xffffu) << 8) | parity;
-            return false;
-        }
-    }
-}
-
-struct Item {
-    int t0, b, h, bh;
-    Plan pl;
-    int nb;
-};
-RAT_DEVICE Item decode_item(const Params &p, int L) {
-    int g = 0;
-    while (g + 1 < p.ngroups && L >= p.grp_item0[g + 1]) ++g;
-    const int local = L - p.grp_item0[g];
-    const int per_row = p.B * p.grp_nheads[g];
-    Item it;
-    const int tile = p.ntiles - 1 - local / per_row;
-    it.t0 = tile * BM;
-    it.b = (local % per_row) / p.grp_nheads[g];
-    it.h = p.head_of[p.grp_head0[g] + (local % per_row) % p.grp_nheads[g]];
-    it.bh = it.b * p.H + it.h;
-    it.pl = make_plan<BN>(it.t0, p.Dh[it.h], p.W, p.T);
-    it.nb = it.pl.nd + it.pl.nw;
-    return it;
-}
-
-__global__ void __launch_bounds__(kThreadsP, 1) attn_persist_kernel(const __grid_constant__ Params p) {
-    extern __shared__ __align__(1024) uint8_t smem[];
-    if (smem_u32(smem) & 1023u) {
-        if (threadIdx.x == 0) atomicCAS(&g_attn_error, 0, RAT_ERR_UNSUPPORTED);
-        return;
-    }
-    Bars &sh = *reinterpret_cast<Bars *>(smem + OFF_BAR);
-    float *init_m = reinterpret_cast<float *>(smem + OFF_STAT);          // [2][128] self score
-    float *fin_st = init_m + 256;                                         // [2][3][128] m, l, w
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int total = p.grp_item0[p.ngroups];
-    const int G = gridDim.x;
-
-    if (threadIdx.x == 0) {
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&sh.q_full[a], 1);
-            mbar_init(&sh.q_ready[a], 128);
-            mbar_init(&sh.q_empty[a], 1);
-            mbar_init(&sh.s_full[a], 1);
-            mbar_init(&sh.p_full[a], 128);
-            mbar_init(&sh.o_ready[a], 1);
-            mbar_init(&sh.tile_done[a], 128);
-            mbar_init(&sh.o_done[a], 1);
-            mbar_init(&sh.o_free[a], 128);
-        }
-        for (int s = 0; s < NSTG; ++s) {
-            mbar_init(&sh.kv_full[s], 1);
-            mbar_init(&sh.kv_empty[s], 1);
-        }
-        mbar_init(&sh.fin, 1);
-        sh.abort = 0;
-        fence_mbar_init();
-    }
-    if (warp == 1) tc::tmem_alloc(&sh.tmem, TMEM_COLS);
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = sh.tmem;
-
-    if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
-        if (lane == 0) {
-            tc::prefetch_tmap(&p.tm_q);
-            tc::prefetch_tmap(&p.tm_k);
-            int g = 0;
-            bool ok = true;
-            for (int i = 0; ok; ++i) {
-                const int L = (int)blockIdx.x + i * G;
-                if (L >= total) break;
-                const Item it = decode_item(p, L);
-                const int a = i & 1;
-                // Q(i) replaces Q(i-2) once every S MMA of tile i-2 has completed
-                if (i >= 2 && !pwait(sh, &sh.q_empty[a], ((i >> 1) - 1) & 1, 11, i)) break;
-                mbar_arrive_expect_tx(&sh.q_full[a], 2 * QSUB);
-                tc::tma_load_3d(smem + OFF_Q + a * 2 * QSUB, &p.tm_q, 0, it.t0, it.bh, &sh.q_full[a]);
-                tc::tma_load_3d(smem + OFF_Q + a * 2 * QSUB + QSUB, &p.tm_q, 64, it.t0, it.bh, &sh.q_full[a]);
-                const CUtensorMap *mk = it.pl.dense ? &p.tm_k : &p.tm_kd[max(p.dslot[it.h], 0)];
-                const CUtensorMap *mv = it.pl.dense ? &p.tm_v : &p.tm_vd[max(p.dslot[it.h], 0)];
-                for (int j = 0; j < it.nb; ++j, ++g) {
-                    const int s = g % NSTG;
-                    if (g >= NSTG && !pwait(sh, &sh.kv_empty[s], ((g / NSTG) - 1) & 1, 12, g)) { ok = false; break; }
-                    const CUtensorMap *tk = j < it.pl.nd ? mk : &p.tm_k;
-                    const CUtensorMap *tv = j < it.pl.nd ? mv : &p.tm_v;
-                    const int y = j < it.pl.nd ? BN * j : it.pl.ws + BN * (j - it.pl.nd);
-                    uint8_t *ks = smem + OFF_K + s * KTILE;
-                    uint8_t *vs = smem + OFF_V + s * KTILE;
-                    mbar_arrive_expect_tx(&sh.kv_full[s], 2 * KTILE);
-                    tc::tma_load_3d(ks, tk, 0, y, it.bh, &sh.kv_full[s]);
-                    tc::tma_load_3d(ks + KSUB, tk, 64, y, it.bh, &sh.kv_full[s]);
-                    tc::tma_load_3d(vs, tv, 0, y, it.bh, &sh.kv_full[s]);
-                    tc::tma_load_3d(vs + KSUB, tv, 64, y, it.bh, &sh.kv_full[s]);
-                }
-            }
-            if (sh.abort) {     // let this CTA's own loads land before its shared memory goes away
-                for (int s = 0; s < NSTG; ++s) pwait(sh, &sh.kv_full[s], 0, 0);
-            }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t IDESC_QK = tc::idesc_bf16(BM, BN, 0);
-            constexpr uint32_t IDESC_PV = tc::idesc_bf16(BM, DHEAD, 1);
-            // the PV of the previous block, issued after the next S so the two overlap
-            bool have_pv = false;
-            int pv_g = 0, pv_a = 0, pv_tile = 0;
-            bool pv_first = false, pv_last = false;
-            bool ok = true;
-            auto issue_pv = [&]() -> bool {
-                if (!pwait(sh, &sh.p_full[pv_g & 1], (pv_g >> 1) & 1, 13, pv_g)) return false;
-                if (pv_first && pv_tile >= 2 && !pwait(sh, &sh.o_free[pv_a], ((pv_tile >> 1) - 1) & 1, 14, pv_tile))
-                    return false;
-                tc::fence_after_sync();
-                const int s = pv_g % NSTG;
-                const uint32_t sv = smem_u32(smem + OFF_V + s * KTILE);
-                const uint32_t pcol = (pv_g & 1) * BN;
-                for (int kk = 0; kk < BN / 16; ++kk)
-                    tc::mma_bf16_ts(tmem + COL_O + pv_a * 128, tmem + pcol + kk * 8,
-                                    tc::smem_desc_sw128(sv + kk * 16 * 128, KSUB, 1024), IDESC_PV,
-                                    (pv_first && kk == 0) ? 0u : 1u);
-                tc::mma_commit(&sh.o_ready[pv_g & 1]);
-                tc::mma_commit(&sh.kv_empty[s]);
-                if (pv_last) tc::mma_commit(&sh.o_done[pv_a]);
-                have_pv = false;
-                return true;
-            };
-            int g = 0;
-            for (int i = 0; ok; ++i) {
-                const int L = (int)blockIdx.x + i * G;
-                if (L >= total) break;
-                const Item it = decode_item(p, L);
-                const int a = i & 1;
-                if (!pwait(sh, &sh.q_ready[a], (i >> 1) & 1, 15, i)) break;
-                tc::fence_after_sync();
-                const uint32_t sq = smem_u32(smem + OFF_Q + a * 2 * QSUB);
-                for (int j = 0; j < it.nb; ++j, ++g) {
-                    const int s = g % NSTG;
-                    if (!pwait(sh, &sh.kv_full[s], (g / NSTG) & 1, 16, g)) { ok = false; break; }
-                    // S buffer g&1 holds P(g-2) until PV(g-2) has completed
-                    if (g >= 2 && !pwait(sh, &sh.o_ready[g & 1], ((g - 2) >> 1) & 1, 17, g)) { ok = false; break; }
-                    tc::fence_after_sync();
-                    const uint32_t sk = smem_u32(smem + OFF_K + s * KTILE);
-                    for (int kk = 0; kk < DHEAD / 16; ++kk) {
-                        const uint32_t qoff = (kk >> 2) * QSUB + (kk & 3) * 32;
-                        const uint32_t koff = (kk >> 2) * KSUB + (kk & 3) * 32;
-                        tc::mma_bf16_ss(tmem + (g & 1) * BN, tc::smem_desc_sw128(sq + qoff, 16, 1024),
-                                        tc::smem_desc_sw128(sk + koff, 16, 1024), IDESC_QK, kk > 0);
-                    }
-                    tc::mma_commit(&sh.s_full[g & 1]);
-                    if (j == it.nb - 1) tc::mma_commit(&sh.q_empty[a]);
-                    if (have_pv && !issue_pv()) { ok = false; break; }
-                    have_pv = true;
-                    pv_g = g; pv_a = a; pv_tile = i;
-                    pv_first = j == 0;
-                    pv_last = j == it.nb - 1;
-                }
-                if (ok && it.nb == 0) {
-                    // a tile without key blocks keeps the per-slot phases in step
-                    tc::mma_commit(&sh.q_empty[a]);
-                    if (have_pv && !issue_pv()) break;
-                    if (i >= 2 && !pwait(sh, &sh.o_free[a], ((i >> 1) - 1) & 1, 14, i)) break;
-                    tc::mma_commit(&sh.o_done[a]);
-                }
-            }
-            if (ok && have_pv) issue_pv();
-            tc::mma_commit(&sh.fin);
-            const uint64_t t_0 = globaltimer_ns();
-            while (!mbar_try_wait(&sh.fin, 0) && globaltimer_ns() - t_0 < kWaitLimitNs) {
-            }
-        }
-        __syncwarp();
-    } else if (warp < 6) {
-        // ------------------------------------------------------------ softmax (key blocks)
-        const int q4 = warp & 3;
-        const int r = q4 * 32 + lane;
-        const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-        float sv[BN];
-        int g = 0;
-        bool ok = true;
-        for (int i = 0; ok; ++i) {
-            const int L = (int)blockIdx.x + i * G;
-            if (L >= total) break;
-            const Item it = decode_item(p, L);
-            const int a = i & 1;
-            const int t = it.t0 + r;
-            if (!__all_sync(0xffffffffu, pwait(sh, &sh.q_ready[a], (i >> 1) & 1, 18, i))) break;
-            float m_run = -INFINITY, l_run = 0.f, w_self = 0.f;
-            if (it.pl.self_reg) {
-                m_run = init_m[a * 128 + r];
-                l_run = 1.f;
-                w_self = 1.f;
-            }
-            for (int j = 0; j < it.nb; ++j, ++g) {
-                if (!__all_sync(0xffffffffu, pwait(sh, &sh.s_full[g & 1], (g >> 1) & 1, 19, g))) { ok = false; break; }
-                tc::fence_after_sync();
-#pragma unroll
-                for (int c = 0; c < BN / 32; ++c)
-                    tc::tmem_ld32(tl + (g & 1) * BN + 32 * c, reinterpret_cast<uint32_t *>(sv) + 32 * c);
-                tc::tmem_wait_ld();
-                int c_lo, c_hi;
-                block_range<BN>(it.pl, j, t, c_lo, c_hi);
-                float m8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) m8[u] = -INFINITY;
-                if (c_lo <= 0 && c_hi >= BN - 1) {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < BN; ++c) {
-                        sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
-                        m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
-                    }
-                }
-                const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
-                const float m_new = fmaxf(m_run, mx);
-                const bool resc = m_new > m_run + kRescaleLog2;
-                float alpha = 1.f;
-                if (resc) {
-                    alpha = ex2_approx(m_run - m_new);
-                    l_run *= alpha;
-                    w_self *= alpha;
-                    m_run = m_new;
-                }
-                const float neg_mu = m_run == -INFINITY ? 0.f : -m_run;
-                float s8[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) s8[u] = 0.f;
-#pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    const float e = ex2_approx(fmaf(sv[c], p.scale_log2, neg_mu));
-                    sv[c] = e;
-                    s8[c & 7] += e;
-                }
-                l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-                if (j > 0 && __any_sync(0xffffffffu, resc)) {
-                    // PV(g-1) (same tile) completes phase (g-1)/2 of o_ready[(g-1)&1]
-                    if (!__all_sync(0xffffffffu, pwait(sh, &sh.o_ready[(g - 1) & 1], ((g - 1) >> 1) & 1, 20, g))) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after_sync();
-#pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
-                        uint32_t o[32];
-                        tc::tmem_ld32(tl + COL_O + a * 128 + 32 * c, o);
-                        tc::tmem_wait_ld();
-#pragma unroll
-                        for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-                        tc::tmem_st32(tl + COL_O + a * 128 + 32 * c, o);
-                    }
-                }
-                {
-                    uint32_t pk[32];
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) pk[k] = pack_bf16(sv[2 * k], sv[2 * k + 1]);
-                    tc::tmem_st32(tl + (g & 1) * BN, pk);
-                }
-                tc::tmem_wait_st();
-                tc::fence_before_sync();
-                mbar_arrive(&sh.p_full[g & 1]);
-            }
-            if (!ok) break;
-            fin_st[(a * 3 + 0) * 128 + r] = m_run;
-            fin_st[(a * 3 + 1) * 128 + r] = l_run;
-            fin_st[(a * 3 + 2) * 128 + r] = w_self;
-            mbar_arrive(&sh.tile_done[a]);
-        }
-    } else {
-        // ------------------------------------------------------------ prologue / epilogue
-        const int q4 = warp & 3;
-        const int r = q4 * 32 + lane;
-        const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-        float2 *rel = reinterpret_cast<float2 *>(smem + OFF_REL);
-        float2 *bas = reinterpret_cast<float2 *>(smem + OFF_BAS);
-        if (p.rope) {            // rot(l theta_f) for l < 32: the same for every tile
-#pragma unroll 4
-            for (int k = 0; k < 16; ++k) {
-                const int e = r + 128 * k, f = e >> 5, l = e & 31;
-                float cs, sn;
-                rope_cs_f32(l, p.theta_f[f], cs, sn);
-                rel[e] = make_float2(cs, sn);
-            }
-        }
-        bool ok = true;
-        auto prologue = [&](int i) -> bool {
-            const int L = (int)blockIdx.x + i * G;
-            const Item it = decode_item(p, L);
-            const int a = i & 1;
-            const int t = it.t0 + r;
-            uint8_t *sQ = smem + OFF_Q + a * 2 * QSUB;
-            uint4 kself[16];
-            const bool have_self = it.pl.self_reg && t < p.T;
-            if (have_self) {
-                const uint4 *krow = reinterpret_cast<const uint4 *>(
-                    static_cast<const uint8_t *>(p.kg) + ((size_t)it.bh * p.T + t) * (DHEAD * 2));
-#pragma unroll
-                for (int c = 0; c < 16; ++c) kself[c] = __ldg(krow + c);
-            }
-            if (p.rope) {
-#pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int e = r + 128 * k, w = e >> 6, f = e & 63;
-                    const long long pos = p.pos0 + it.t0 + 32 * w;
-                    float cs, sn;
-                    if (p.rope_f32) rope_cs_f32((int)pos, p.theta_f[f], cs, sn);
-                    else rope_cs_fast(pos, p.theta[f], cs, sn);
-                    bas[(a * 4 + w) * 64 + f] = make_float2(cs, sn);
-                }
-            }
-            if (!__all_sync(0xffffffffu, pwait(sh, &sh.q_full[a], (i >> 1) & 1, 21, i))) return false;
-            if (p.rope) {
-                asm volatile("bar.sync 1, 128;" ::: "memory");     // bas (and rel) complete
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint4 *p1 = reinterpret_cast<uint4 *>(sQ + swz(r, c));
-                    uint4 *p2 = reinterpret_cast<uint4 *>(sQ + QSUB + swz(r, c));
-                    uint4 u1 = *p1, u2 = *p2;
-                    uint32_t a1[4] = {u1.x, u1.y, u1.z, u1.w}, a2[4] = {u2.x, u2.y, u2.z, u2.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        float cs[2], sn[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int f = c * 8 + 2 * k + u;
-                            const float2 b = bas[(a * 4 + q4) * 64 + f], rl = rel[f * 32 + lane];
-                            cs[u] = b.x * rl.x - b.y * rl.y;
-                            sn[u] = b.y * rl.x + b.x * rl.y;
-                        }
-                        const float x1l = bf16_lo(a1[k]), x1h = bf16_hi(a1[k]);
-                        const float x2l = bf16_lo(a2[k]), x2h = bf16_hi(a2[k]);
-                        a1[k] = pack_bf16(x1l * cs[0] - x2l * sn[0], x1h * cs[1] - x2h * sn[1]);
-                        a2[k] = pack_bf16(x2l * cs[0] + x1l * sn[0], x2h * cs[1] + x1h * sn[1]);
-                    }
-                    *p1 = make_uint4(a1[0], a1[1], a1[2], a1[3]);
-                    *p2 = make_uint4(a2[0], a2[1], a2[2], a2[3]);
-                }
-            }
-            float dot = 0.f;
-            if (have_self) {
-#pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const uint4 kq = kself[c];
-                    const uint4 qq = *reinterpret_cast<const uint4 *>(sQ + (c >> 3) * QSUB + swz(r, c & 7));
-                    const uint32_t ku[4] = {kq.x, kq.y, kq.z, kq.w}, qu[4] = {qq.x, qq.y, qq.z, qq.w};
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        dot = fmaf(bf16_lo(qu[k]), bf16_lo(ku[k]), dot);
-                        dot = fmaf(bf16_hi(qu[k]), bf16_hi(ku[k]), dot);
-                    }
-                }
-            }
-            init_m[a * 128 + r] = dot * p.scale_log2;
-            tc::fence_proxy_async_smem();
-            mbar_arrive(&sh.q_ready[a]);
-            return true;
-        };
-        auto epilogue = [&](int i) -> bool {
-            const int L = (int)blockIdx.x + i * G;
-            const Item it = decode_item(p, L);
-            const int a = i & 1;
-            const int t = it.t0 + r;
-            uint4 vself[16];
-            if (it.pl.self_reg) {
-                const uint4 *vrow = reinterpret_cast<const uint4 *>(
-                    static_cast<const uint8_t *>(p.vg) + ((size_t)it.bh * p.T + min(t, p.T - 1)) * (DHEAD * 2));
-#pragma unroll
-                for (int c = 0; c < 16; ++c) vself[c] = __ldg(vrow + c);
-            }
-            if (!__all_sync(0xffffffffu, pwait(sh, &sh.tile_done[a], (i >> 1) & 1, 22, i))) return false;
-            if (!__all_sync(0xffffffffu, pwait(sh, &sh.o_done[a], (i >> 1) & 1, 23, i))) return false;
-            tc::fence_after_sync();
-            const float l_run = fin_st[(a * 3 + 1) * 128 + r];
-            const float w_self = fin_st[(a * 3 + 2) * 128 + r];
-            const float inv = 1.0f / l_run;
-            __nv_bfloat16 *orow = static_cast<__nv_bfloat16 *>(p.og) + ((size_t)it.bh * p.T + t) * DHEAD;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                uint32_t o[32];
-                if (it.nb > 0) {
-                    tc::tmem_ld32(tl + COL_O + a * 128 + 32 * c, o);
-                    tc::tmem_wait_ld();
-                } else {
-#pragma unroll
-                    for (int k = 0; k < 32; ++k) o[k] = 0u;
-                }
-                if (it.pl.self_reg) {
-#pragma unroll
-                    for (int k8 = 0; k8 < 4; ++k8) {
-                        const uint4 vv = vself[4 * c + k8];
-                        const uint32_t vu[4] = {vv.x, vv.y, vv.z, vv.w};
-#pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            o[8 * k8 + 2 * k] = __float_as_uint(fmaf(w_self, bf16_lo(vu[k]), __uint_as_float(o[8 * k8 + 2 * k])));
-                            o[8 * k8 + 2 * k + 1] = __float_as_uint(fmaf(w_self, bf16_hi(vu[k]), __uint_as_float(o[8 * k8 + 2 * k + 1])));
-                        }
-                    }
-                }
-                if (t < p.T && !sh.abort) {
-#pragma unroll
-                    for (int k8 = 0; k8 < 4; ++k8) {
-                        const float *f = reinterpret_cast<const float *>(o) + 8 * k8;
-                        st_global_v4(orow + 32 * c + 8 * k8,
-                                     pack_bf16(f[0] * inv, f[1] * inv), pack_bf16(f[2] * inv, f[3] * inv),
-                                     pack_bf16(f[4] * inv, f[5] * inv), pack_bf16(f[6] * inv, f[7] * inv));
-                    }
-                }
-            }
-            tc::fence_before_sync();
-            mbar_arrive(&sh.o_free[a]);
-            return true;
-        };
-        if ((int)blockIdx.x < total) ok = prologue(0);
-        for (int i = 0; ok; ++i) {
-            const int L = (int)blockIdx.x + i * G;
-            if (L >= total) break;
-            if (L + G < total && !prologue(i + 1)) break;
-            if (!epilogue(i)) break;
-        }
-    }
-
-    tc::fence_before_sync();
-    __syncthreads();
-    tc::fence_after_sync();
-    if (warp == 1) tc::tmem_dealloc(tmem, TMEM_COLS);
-}
-}  // namespace pk
 
 // ------------------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1192,25 +708,10 @@ int launch_bn(const AttnSm100Args &a, const float2 *rel, void *stream) {
     return a.W <= 1 ? launch_tiles<BN, true>(p, items, stream) : launch_tiles<BN, false>(p, items, stream);
 }
 
-int launch_persistent(const AttnSm100Args &a, const float2 *rel, void *stream) {
-    Params p;
-    const int items = fill_params<pk::BN>(p, a);
-    if (items < 0) return items;
-    p.rope_rel = rel;
-    static uint64_t attr_done = 0;
-    const int st = set_smem_attr(reinterpret_cast<const void *>(pk::attn_persist_kernel), pk::SMEM_BYTES, &attr_done);
-    if (st != RAT_OK) return st;
-    const int sms = current_sm_count();
-    if (sms <= 0) return RAT_ERR_CUDA;
-    const int grid = items < sms ? items : sms;
-    pk::attn_persist_kernel<<<(unsigned)grid, pk::kThreadsP, pk::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(p);
-    return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
-}
 
 }  // namespace
 
 int g_attn_block_keys = 0;   // 0: automatic; 64 or 128 forces the key-block width
-int g_attn_schedule = 0;     // 0: automatic (one CTA per tile), 1: one CTA per tile, 2: persistent
 
 // The device table of a launch's RoPE frequencies: uploaded (stream-ordered) the first time a
 // frequency set is seen on this device, then reused.
@@ -1255,7 +756,6 @@ int launch_attn_sm100(const AttnSm100Args &a, void *stream) {
         const int st = rope_rel_table(a.theta, stream, &rel);
         if (st != RAT_OK) return st;
     }
-    if (g_attn_schedule == 2 && g_attn_block_keys != 128) return launch_persistent(a, rel, stream);
     const int bn = g_attn_block_keys ? g_attn_block_keys : 64;
     return bn == 64 ? launch_bn<64>(a, rel, stream) : launch_bn<128>(a, rel, stream);
 }

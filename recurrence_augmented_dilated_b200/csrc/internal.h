@@ -100,7 +100,6 @@ int attn_error_word(void *stream, bool clear);
 unsigned attn_error_where();
 unsigned attn_error_waiting();
 extern int g_attn_block_keys;
-extern int g_attn_schedule;
 
 // ---------------------------------------------------------------------------- cache / decode
 struct CompressParams {

@@ -209,11 +209,6 @@ uint32_t rat_attn_error_site(void) { return attn_error_where(); }
 
 uint32_t rat_attn_error_waiting(void) { return attn_error_waiting(); }
 
-int rat_set_attn_schedule(int schedule) {
-    if (schedule < 0 || schedule > 2) return RAT_ERR_INVALID;
-    g_attn_schedule = schedule;
-    return RAT_OK;
-}
 
 int rat_set_attn_block_keys(int block_keys) {
     if (block_keys != 0 && block_keys != 64 && block_keys != 128) return RAT_ERR_INVALID;

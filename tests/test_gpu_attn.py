@@ -16,16 +16,12 @@ from gpu_util import TOL_BF16, TOL_F32, f64, gpu_attn, gpu_recur, rel_err, tol_f
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(params=[(0, 2), (64, 1), (128, 1)], ids=["persistent", "bk64", "bk128"])
+@pytest.fixture(params=[64, 128], ids=["bk64", "bk128"])
 def block_keys(request):
-    """Run a tensor-core case with each kernel of the bf16 path: the persistent kernel and the
-    one-CTA-per-tile kernel with 64- and 128-key blocks."""
-    bk, sched = request.param
-    rat.rat_set_attn_block_keys(bk)
-    rat.rat_set_attn_schedule(sched)
+    """Run a tensor-core case with both key-block widths of the bf16 path."""
+    rat.rat_set_attn_block_keys(request.param)
     yield request.param
     rat.rat_set_attn_block_keys(0)
-    rat.rat_set_attn_schedule(0)
 
 
 def qkv(B, H, T, d, dtype, seed):
