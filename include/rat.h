@@ -148,9 +148,10 @@ RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const voi
 RAT_API int rat_attn_sync_status(void *stream);
 
 /* Diagnostic: where the attention kernel's last recorded timeout happened, as
- * (wait site << 24) | (key block << 8) | phase parity; sites: 1 producer stage-free, 2 MMA
- * query-ready, 3 MMA stage-full, 4 MMA previous-PV, 5 MMA probabilities-ready, 6 softmax
- * query-loaded, 7 softmax scores-ready, 8 softmax rescale, 9 epilogue.  0 if none. */
+ * (wait site << 24) | (key block << 8) | phase parity; sites: 1 producer K-stage-free, 2 MMA
+ * query-ready, 3 MMA K-stage-full, 4 MMA previous-PV, 5 MMA probabilities-ready, 6 softmax
+ * query-loaded, 7 softmax scores-ready, 8 softmax rescale, 9 epilogue, 10 producer
+ * query-rotated, 11 producer V-stage-free, 12 MMA V-stage-full.  0 if none. */
 RAT_API uint32_t rat_attn_error_site(void);
 
 /* Diagnostic: bit s set when a wait at site s (numbering as above) was still in progress when a

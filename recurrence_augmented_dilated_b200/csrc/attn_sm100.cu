@@ -147,10 +147,13 @@ RAT_DEVICE void block_range(const Plan &pl, int j, int t, int &c_lo, int &c_hi) 
 }
 
 struct Shared {
-    uint64_t q_full, q_ready, kv_full[NS], kv_empty[NS], s_full[2], p_full[2], o_ready[2], fin;
+    // K and V of a stage have separate lifetimes: K is free once S has read it, V once PV has
+    uint64_t q_full, q_ready, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS];
+    uint64_t s_full[2], p_full[2], o_ready[2], fin;
     uint32_t tmem;
     volatile int abort;
 };
+static_assert(sizeof(Shared) <= 256, "barriers fit the 256 bytes reserved after the tiles");
 
 // Bounded mbarrier wait that also gives up as soon as another role aborted; an expired wait
 // records RAT_ERR_TIMEOUT and its site (see g_attn_where).
@@ -169,6 +172,13 @@ RAT_DEVICE bool wait_bar(Shared &sh, uint64_t *bar, uint32_t parity, uint32_t si
                 g_attn_where = (site << 24) | ((blk & 0xffffu) << 8) | parity;
             return false;
         }
+    }
+}
+
+// Bounded wait that ignores aborts: a role draining its own asynchronous copies before exit.
+RAT_DEVICE void wait_drain(uint64_t *bar, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kWaitLimitNs) {
     }
 }
 
@@ -222,8 +232,10 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         mbar_init(&sh.q_full, 1);
         mbar_init(&sh.q_ready, 128);
         for (int s = 0; s < NS; ++s) {
-            mbar_init(&sh.kv_full[s], 1);
-            mbar_init(&sh.kv_empty[s], 1);
+            mbar_init(&sh.k_full[s], 1);
+            mbar_init(&sh.v_full[s], 1);
+            mbar_init(&sh.k_empty[s], 1);
+            mbar_init(&sh.v_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) mbar_init(&sh.s_full[s], 1);
         // P of even / odd blocks: the softmax may finish block j while the MMA has not yet
@@ -255,28 +267,39 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             tc::tma_load_3d(smem + C::OFF_Q + QSUB, &p.tm_q, 64, t0, bh, &sh.q_full);
             // RoPE: the relative rotation table goes to the second K stage, unused until Q is rotated
             if (p.rope) bulk_g2s(smem + C::OFF_K + C::KTILE, p.rope_rel, kRelBytes, &sh.q_full);
-            int issued = 0;
-            for (int j = 0; j < nb; ++j) {
-                const int s = j % NS;
-                if (j >= NS && !wait_bar(sh, &sh.kv_empty[s], ((j / NS) - 1) & 1, 1, j)) break;
-                // with RoPE, stage 1 holds the softmax warps' rotation tables until Q is rotated
-                if (j == 1 && p.rope && !wait_bar(sh, &sh.q_ready, 0, 10, j)) break;
-                const CUtensorMap *tk = j < pl.nd ? mk : &p.tm_k;
-                const CUtensorMap *tv = j < pl.nd ? mv : &p.tm_v;
-                const int y = j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd);
-                uint8_t *ks = smem + C::OFF_K + s * C::KTILE;
-                uint8_t *vs = smem + C::OFF_V + s * C::KTILE;
-                mbar_arrive_expect_tx(&sh.kv_full[s], 2 * C::KTILE);
-                tc::tma_load_3d(ks, tk, 0, y, bh, &sh.kv_full[s]);
-                tc::tma_load_3d(ks + C::KSUB, tk, 64, y, bh, &sh.kv_full[s]);
-                tc::tma_load_3d(vs, tv, 0, y, bh, &sh.kv_full[s]);
-                tc::tma_load_3d(vs + C::KSUB, tv, 64, y, bh, &sh.kv_full[s]);
-                issued = j + 1;
+            // K runs one block ahead of V: S(j) needs K(j) long before PV(j) needs V(j), and a K
+            // stage frees up as soon as its S has completed
+            auto row_of = [&](int j) { return j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd); };
+            int k_issued = 0, v_issued = 0;
+            for (int j = 0; j <= nb; ++j) {
+                if (j < nb) {
+                    const int s = j % NS;
+                    if (j >= NS && !wait_bar(sh, &sh.k_empty[s], ((j / NS) - 1) & 1, 1, j)) break;
+                    // with RoPE, stage 1 holds the softmax warps' rotation tables until Q is rotated
+                    if (j == 1 && p.rope && !wait_bar(sh, &sh.q_ready, 0, 10, j)) break;
+                    const CUtensorMap *tk = j < pl.nd ? mk : &p.tm_k;
+                    uint8_t *ks = smem + C::OFF_K + s * C::KTILE;
+                    mbar_arrive_expect_tx(&sh.k_full[s], C::KTILE);
+                    tc::tma_load_3d(ks, tk, 0, row_of(j), bh, &sh.k_full[s]);
+                    tc::tma_load_3d(ks + C::KSUB, tk, 64, row_of(j), bh, &sh.k_full[s]);
+                    k_issued = j + 1;
+                }
+                if (j >= 1) {
+                    const int jv = j - 1, s = jv % NS;
+                    if (jv >= NS && !wait_bar(sh, &sh.v_empty[s], ((jv / NS) - 1) & 1, 11, jv)) break;
+                    const CUtensorMap *tv = jv < pl.nd ? mv : &p.tm_v;
+                    uint8_t *vs = smem + C::OFF_V + s * C::KTILE;
+                    mbar_arrive_expect_tx(&sh.v_full[s], C::KTILE);
+                    tc::tma_load_3d(vs, tv, 0, row_of(jv), bh, &sh.v_full[s]);
+                    tc::tma_load_3d(vs + C::KSUB, tv, 64, row_of(jv), bh, &sh.v_full[s]);
+                    v_issued = jv + 1;
+                }
             }
             if (sh.abort) {
                 // let this CTA's own loads land before its shared memory goes away
-                for (int j = max(0, issued - NS); j < issued; ++j) wait_bar(sh, &sh.kv_full[j % NS], (j / NS) & 1);
-                wait_bar(sh, &sh.q_full, 0);
+                for (int j = max(0, k_issued - NS); j < k_issued; ++j) wait_drain(&sh.k_full[j % NS], (j / NS) & 1);
+                for (int j = max(0, v_issued - NS); j < v_issued; ++j) wait_drain(&sh.v_full[j % NS], (j / NS) & 1);
+                wait_drain(&sh.q_full, 0);
             }
         }
         __syncwarp();
@@ -291,7 +314,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             for (int j = 0; ok && j <= nb; ++j) {
                 if (j < nb) {
                     const int s = j % NS, sb = j & 1;
-                    if (!wait_bar(sh, &sh.kv_full[s], (j / NS) & 1, 3, j)) break;
+                    if (!wait_bar(sh, &sh.k_full[s], (j / NS) & 1, 3, j)) break;
                     // S buffer sb holds P(j-2) until PV(j-2) has read it: wait for that PV to
                     // complete (this thread issued it, so the barrier is at most one phase ahead)
                     if (j >= 2 && !wait_bar(sh, &sh.o_ready[(j - 2) & 1], ((j - 2) >> 1) & 1, 4, j)) break;
@@ -305,10 +328,12 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                                         tc::smem_desc_sw128(sk + koff, 16, 1024), IDESC_QK, kk > 0);
                     }
                     tc::mma_commit(&sh.s_full[sb]);
+                    tc::mma_commit(&sh.k_empty[s]);
                 }
                 if (j >= 1) {
                     const int jp = j - 1, s = jp % NS;
                     if (!wait_bar(sh, &sh.p_full[jp & 1], (jp >> 1) & 1, 5, jp)) break;
+                    if (!wait_bar(sh, &sh.v_full[s], (jp / NS) & 1, 12, jp)) break;
                     tc::fence_after_sync();
                     const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KTILE);
                     const uint32_t pcol = (jp & 1) * C::COL_S1;     // P of block jp, in TMEM
@@ -322,7 +347,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                                         (jp > 0 || kk > 0) ? 1u : 0u);
                     }
                     tc::mma_commit(&sh.o_ready[jp & 1]);
-                    tc::mma_commit(&sh.kv_empty[s]);
+                    tc::mma_commit(&sh.v_empty[s]);
                 }
             }
             // all MMAs issued by this thread complete before TMEM can be released
