@@ -483,18 +483,14 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             float m8[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) m8[u] = -INFINITY;
-            if (c_lo <= 0 && c_hi >= BN - 1) {
+            if (!(c_lo <= 0 && c_hi >= BN - 1)) {
 #pragma unroll
-                for (int c = 0; c < BN; ++c) m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
-            } else {
-#pragma unroll
-                for (int c = 0; c < BN; ++c) {
-                    sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
-                    m8[c & 7] = fmaxf(m8[c & 7], sv[c]);
-                }
+                for (int c = 0; c < BN; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
             }
-            const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7]))) * p.scale_log2;
+#pragma unroll
+            for (int c = 0; c < BN; c += 2) m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], sv[c], sv[c + 1]);
+            const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                                   fmaxf(m8[6], m8[7])) * p.scale_log2;
             const float m_new = fmaxf(m_run, mx);
             const bool resc = m_new > m_run + kRescaleLog2;
             float alpha = 1.f;
@@ -505,16 +501,21 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                 m_run = m_new;
             }
             const float neg_mu = m_run == -INFINITY ? 0.f : -m_run;
-            float s8[8];
+            // exponents and row sum on float pairs (columns 2i, 2i+1)
+            const f2_t sc2 = f2(p.scale_log2, p.scale_log2), mu2 = f2(neg_mu, neg_mu);
+            f2_t s4[4];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) s8[u] = 0.f;
+            for (int u = 0; u < 4; ++u) s4[u] = f2(0.f, 0.f);
 #pragma unroll
-            for (int c = 0; c < BN; ++c) {
-                const float e = ex2_approx(fmaf(sv[c], p.scale_log2, neg_mu));   // -inf -> 0
-                sv[c] = e;
-                s8[c & 7] += e;
+            for (int i = 0; i < BN / 2; ++i) {
+                const f2_t x = f2_fma(f2(sv[2 * i], sv[2 * i + 1]), sc2, mu2);
+                const f2_t e = f2(ex2_approx(f2lo(x)), ex2_approx(f2hi(x)));    // -inf -> 0
+                sv[2 * i] = f2lo(e);
+                sv[2 * i + 1] = f2hi(e);
+                s4[i & 3] = f2_add(s4[i & 3], e);
             }
-            l_run += ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+            const f2_t s2 = f2_add(f2_add(s4[0], s4[1]), f2_add(s4[2], s4[3]));
+            l_run += f2lo(s2) + f2hi(s2);
             if (j > 0 && __any_sync(0xffffffffu, resc)) {
                 // the running max moved: O must hold PV of every earlier block before rescaling.
                 // PV(j-1) completes phase (j-1)/2 of o_ready[(j-1)&1].  PV(j-3) is done (S(j) was

@@ -62,6 +62,12 @@ RAT_DEVICE f2_t f2_add(f2_t a, f2_t b) {
     return d;
 }
 // bf16 pair (low element in bits 0..15) -> float pair, and back (round to nearest even)
+// max(a, b, c) in one instruction (three-input max.f32, sm_100).
+RAT_DEVICE float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
 RAT_DEVICE f2_t f2_from_bf16x2(uint32_t u) { return f2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u)); }
 RAT_DEVICE uint32_t f2_to_bf16x2(f2_t v) { return pack_bf16(f2lo(v), f2hi(v)); }
 
