@@ -267,7 +267,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 
 int decode_splits(int B, int H, int Tcap, const int32_t *Dh, int W) {
     // aim for about 12 CTAs per SM over the 148 SMs, and at least ~64 keys per split (measured on
-    // the 32 x 32-slice, 1151-key workload: 2 splits per slice beat 1, 3, 4, 6 and 8)
+    // the 32 x 32-slice, 1151-key workload: 2 splits per slice beat 1, 3, 4, 5 and 7)
     long long max_keys = 0;
     for (int h = 0; h < H; ++h) {
         const long long k = Tcap / Dh[h] + W;
