@@ -47,6 +47,7 @@ def _load():
     if _lib is None:
         lib = ctypes.CDLL(build())
         lib.rat_oracle_recurrence.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp]
+        lib.rat_oracle_recurrence_reset.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _L, _L]
         lib.rat_oracle_rope.argtypes = [_L, _L, _L, _dp, _L, ctypes.c_double]
         lib.rat_oracle_in_key_set.argtypes = [_L, _L, _L, _L]
         lib.rat_oracle_in_key_set.restype = ctypes.c_int
@@ -85,11 +86,13 @@ def default_scale(d: int) -> float:
     return 1.0 / np.sqrt(d)
 
 
-def recurrence(x, a, h0=None):
+def recurrence(x, a, h0=None, pos0: int = 0, reset_every: int = 0):
     """h_t = g_t h_{t-1} + (1-g_t) x_t, g = sigmoid(a), per channel, over the full sequence.
 
     x, a: (..., T, d).  h0: (..., d) or None (zeros).  Returns (y, hT) in float64.
-    ("RAT+ Deep Dive" section 2.1, full-sequence recurrence, L = T.)
+    ("RAT+ Deep Dive" section 2.1, full-sequence recurrence, L = T.)  With reset_every = L > 0
+    the state is zeroed before every absolute position pos0 + t that is a multiple of L: the
+    predecessor RAT's chunk-local recurrence (same section; the RAT paper's abstract).
     """
     x = _f64(x)
     a = _f64(a)
@@ -103,7 +106,11 @@ def recurrence(x, a, h0=None):
         h0 = _f64(h0)
         assert h0.shape == hT.shape
         h0p = _ptr(h0)
-    _load().rat_oracle_recurrence(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(y), _ptr(hT))
+    if reset_every and int(reset_every) > 0:
+        _load().rat_oracle_recurrence_reset(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(y), _ptr(hT),
+                                            int(pos0), int(reset_every))
+    else:
+        _load().rat_oracle_recurrence(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(y), _ptr(hT))
     return y, hT
 
 
@@ -162,14 +169,15 @@ def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None)
 
 
 def layer_prefill(q, k, v, a, D=1, W=0, D_per_head=None, rope_base=0.0, pos0=0, scale=None,
-                  rows=None, h0_k=None, h0_v=None):
+                  rows=None, h0_k=None, h0_v=None, reset_every=0):
     """The whole prefill path in float64: recurrence -> RoPE -> dilated attention.
 
     Returns dict(o, k_rec, v_rec, hT_k, hT_v); k_rec is the recurrence output after RoPE
-    (what the cache stores), v_rec the value recurrence output.
+    (what the cache stores), v_rec the value recurrence output.  reset_every > 0 selects the
+    chunk-local recurrence (see recurrence()).
     """
-    k_rec, hT_k = recurrence(k, a, h0_k)
-    v_rec, hT_v = recurrence(v, a, h0_v)
+    k_rec, hT_k = recurrence(k, a, h0_k, pos0=pos0, reset_every=reset_every)
+    v_rec, hT_v = recurrence(v, a, h0_v, pos0=pos0, reset_every=reset_every)
     qr = _f64(q)
     if rope_base > 0:
         k_rec = rope(k_rec, pos0, rope_base)
@@ -211,7 +219,8 @@ class DecodeState:
     of it); use it on a few (batch, head) slices.  Dbh gives each slice's dilation.
     """
 
-    def __init__(self, Dbh, d: int, W: int, Tcap: int, rope_base: float = 0.0, scale=None):
+    def __init__(self, Dbh, d: int, W: int, Tcap: int, rope_base: float = 0.0, scale=None,
+                 reset_every: int = 0):
         self.Dbh = np.ascontiguousarray(np.asarray(Dbh, dtype=np.int32))
         self.BH = len(self.Dbh)
         self.d, self.W, self.Tcap = d, int(W), int(Tcap)
@@ -222,13 +231,14 @@ class DecodeState:
         self.khist = np.zeros((self.BH, self.Tcap, d))
         self.vhist = np.zeros((self.BH, self.Tcap, d))
         self.t = 0
+        self.reset_every = int(reset_every)     # > 0: chunk-local recurrence (state zeroed at t % L == 0)
 
     def prefill(self, k, v, a):
         """Consume a context (BH, T, d) with the sequential recurrence and record history."""
         k, v, a = _f64(k), _f64(v), _f64(a)
         T = k.shape[-2]
-        yk, hk = recurrence(k, a, self.hk)
-        yv, hv = recurrence(v, a, self.hv)
+        yk, hk = recurrence(k, a, self.hk, pos0=self.t, reset_every=self.reset_every)
+        yv, hv = recurrence(v, a, self.hv, pos0=self.t, reset_every=self.reset_every)
         if self.rope_base > 0:
             yk = rope(yk, self.t, self.rope_base)
         self.khist[:, self.t:self.t + T] = yk
@@ -239,6 +249,9 @@ class DecodeState:
     def step(self, q, k, v, a):
         """One new token per slice: (BH, d) inputs -> (BH, d) output."""
         q, k, v, a = _f64(q), _f64(k), _f64(v), _f64(a)
+        if self.reset_every > 0 and self.t % self.reset_every == 0:
+            self.hk[:] = 0.0                    # a new block starts at this position
+            self.hv[:] = 0.0
         o = np.empty((self.BH, self.d))
         _load().rat_oracle_decode_step(self.BH, self.d, self.t, _ptr(self.Dbh, _ip), self.W,
                                        self.scale, self.rope_base, _ptr(q), _ptr(k), _ptr(v),

@@ -74,6 +74,34 @@ void rat_oracle_recurrence(long BH, long T, long d, const double *x, const doubl
 }
 
 /*
+ * Chunk-local recurrence of the predecessor RAT ("RAT+ Deep Dive" section 2.1: the original RAT
+ * splits the sequence into blocks of size L and each token recurses only within its block; the
+ * RAT paper's abstract: recurrence within each chunk).  Same step as above, but the state is
+ * set to zero before every absolute position p = pos0 + t with p mod L == 0 (L > 0), so each
+ * block of L positions starts from an empty state.  h0 is the state before pos0 (dropped when
+ * pos0 itself starts a block).
+ */
+void rat_oracle_recurrence_reset(long BH, long T, long d, const double *x, const double *a,
+                                 const double *h0, double *y, double *hT, long pos0, long L)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        for (long c = 0; c < d; ++c) {
+            double h = h0 ? h0[bh * d + c] : 0.0;
+            for (long t = 0; t < T; ++t) {
+                long idx = (bh * T + t) * d + c;
+                if ((pos0 + t) % L == 0) h = 0.0;        /* a new block starts here */
+                double g = forget_gate(a[idx]);
+                double omg = one_minus_gate(a[idx]);
+                h = g * h + omg * x[idx];
+                y[idx] = h;
+            }
+            if (hT) hT[bh * d + c] = h;
+        }
+    }
+}
+
+/*
  * Rotary position embedding, rotate-half pairing, in place.                  [RoFormer]
  *   x : [BH][T][d];  position of row t is pos0 + t;  for c < d/2:
  *   theta_c = base^(-2c/d),  phi = (pos0 + t) * theta_c,

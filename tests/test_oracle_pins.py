@@ -116,6 +116,63 @@ def test_recurrence_chunked_equals_whole():
 
 # ----------------------------------------------------------------------------- RoPE
 
+@pytest.mark.parametrize("pos0,L", [(7, 100), (3, 64)])
+def test_reset_outside_the_sequence_is_the_full_recurrence(pos0, L):
+    # no block boundary in pos0 .. pos0+T-1: identical operations, identical bits
+    x, a = RNG.standard_normal((3, 50, 5)), RNG.standard_normal((3, 50, 5))
+    h0 = RNG.standard_normal((3, 5))
+    y0, hT0 = oracle.recurrence(x, a, h0)
+    y1, hT1 = oracle.recurrence(x, a, h0, pos0=pos0, reset_every=L)
+    assert np.array_equal(y0, y1) and np.array_equal(hT0, hT1)
+
+
+def test_reset_every_position_keeps_only_the_input_term():
+    # L = 1: every step starts from an empty state, h_t = (1 - g_t) x_t
+    x, a = RNG.standard_normal((2, 40, 4)), 3 * RNG.standard_normal((2, 40, 4))
+    y, _ = oracle.recurrence(x, a, RNG.standard_normal((2, 4)), pos0=5, reset_every=1)
+    g = 1.0 / (1.0 + np.exp(-a))
+    np.testing.assert_allclose(y, (1.0 - g) * x, rtol=1e-14, atol=1e-15)
+
+
+@pytest.mark.parametrize("pos0,L", [(0, 16), (5, 16), (13, 7), (64, 64)])
+def test_reset_equals_independent_blocks(pos0, L):
+    # the chunk-local recurrence is the full recurrence run separately on every block of L
+    # positions, from zero at each block start (and from h0 for a block already under way)
+    T = 90
+    x, a = RNG.standard_normal((2, T, 3)), RNG.standard_normal((2, T, 3))
+    h0 = RNG.standard_normal((2, 3))
+    y, hT = oracle.recurrence(x, a, h0, pos0=pos0, reset_every=L)
+    want = np.empty_like(y)
+    t = 0
+    h = h0
+    while t < T:
+        if (pos0 + t) % L == 0:
+            h = np.zeros_like(h0)
+        end = min(T, t + L - (pos0 + t) % L)      # up to the next block start
+        ys, h = oracle.recurrence(x[:, t:end], a[:, t:end], h)
+        want[:, t:end] = ys
+        t = end
+    assert np.array_equal(y, want) and np.array_equal(hT, h)
+
+
+def test_reset_brute_force_sum():
+    # y_t = sum over s in t's block (s <= t) of (prod_{r=s+1..t} g_r)(1-g_s) x_s, plus the carried
+    # h0 term when t's block began before pos0
+    T, L, pos0 = 23, 6, 4
+    x, a = RNG.standard_normal((1, T, 2)), RNG.standard_normal((1, T, 2))
+    h0 = RNG.standard_normal((1, 2))
+    y, _ = oracle.recurrence(x, a, h0, pos0=pos0, reset_every=L)
+    g = 1.0 / (1.0 + np.exp(-a[0]))
+    for t in range(T):
+        start = t - ((pos0 + t) % L)              # first position of t's block (may be < 0)
+        acc = np.zeros(2)
+        for s_ in range(max(start, 0), t + 1):
+            acc += np.prod(g[s_ + 1:t + 1], axis=0) * (1 - g[s_]) * x[0, s_]
+        if start < 0:
+            acc += np.prod(g[0:t + 1], axis=0) * h0[0]
+        np.testing.assert_allclose(y[0, t], acc, rtol=1e-12, atol=1e-13)
+
+
 def test_rope_matches_complex_rotation():
     d, T, pos0, base = 16, 9, 1000, 10000.0
     x = RNG.standard_normal((1, T, d))
@@ -279,15 +336,15 @@ def test_kv_compress_chunked_equals_whole():
 
 # ----------------------------------------------------------------------------- decode
 
-@pytest.mark.parametrize("rope_base", [0.0, 10000.0])
-def test_decode_equals_prefill_rows(rope_base):
+@pytest.mark.parametrize("rope_base,reset", [(0.0, 0), (10000.0, 0), (10000.0, 8)])
+def test_decode_equals_prefill_rows(rope_base, reset):
     B, H, T0, steps, d, W = 1, 3, 40, 12, 8, 4
     Dh = [1, 4, 16]
     T = T0 + steps
     q, k, v = rand_qkv(B, H, T, d)
     a = RNG.standard_normal((B, H, T, d)) + 2.0
-    ref = oracle.layer_prefill(q, k, v, a, D_per_head=Dh, W=W, rope_base=rope_base)
-    st = oracle.DecodeState(np.tile(Dh, B), d, W, Tcap=T, rope_base=rope_base)
+    ref = oracle.layer_prefill(q, k, v, a, D_per_head=Dh, W=W, rope_base=rope_base, reset_every=reset)
+    st = oracle.DecodeState(np.tile(Dh, B), d, W, Tcap=T, rope_base=rope_base, reset_every=reset)
     st.prefill(k[:, :, :T0].reshape(B * H, T0, d), v[:, :, :T0].reshape(B * H, T0, d),
                a[:, :, :T0].reshape(B * H, T0, d))
     for s in range(steps):
