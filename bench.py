@@ -218,7 +218,7 @@ class ProfiledRegion:
 
 
 def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world: int, peaks,
-                peak_kind, with_e2e: bool, min_warmup_s: float = 1.0):
+                peak_kind, with_e2e: bool, min_warmup_s: float = 1.0, reset_every: int = 0):
     import recurrence_augmented_dilated_b200 as rat
     dev = torch.device("cuda")
     x = synthetic.prefill_inputs(w, seed=w.seed + 1000 * rank)
@@ -236,7 +236,12 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
     def step(timer=None, qq=q, kk=k, vv=v, aa=a):
         span = timer.span if timer else (lambda n: _Null())
         with span("recur"):
-            rat.rat_recur_prefill(kk, vv, aa, kr, vr, ws, hT_k=hk, hT_v=hv, rope_base=w.rope_base)
+            if reset_every > 0:
+                rat.rat_recur_prefill_local(kk, vv, aa, kr, vr, ws, reset_every, hT_k=hk, hT_v=hv,
+                                            rope_base=w.rope_base)
+            else:
+                rat.rat_recur_prefill(kk, vv, aa, kr, vr, ws, hT_k=hk, hT_v=hv,
+                                      rope_base=w.rope_base)
         with span("attn"):
             rat.rat_dilated_attn_prefill(qq, kr, vr, o, D=w.D, W=w.W, D_per_head=Dph,
                                          rope_base=w.rope_base)
@@ -563,6 +568,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--all", action="store_true", help="also time the other prefill workloads")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--reset-every", type=int, default=0,
+                    help="L > 0: the chunk-local recurrence (restart every L positions) in the "
+                         "prefill step instead of the full-sequence one")
     ap.add_argument("--min-warmup-s", type=float, default=1.0,
                     help="keep warming up at least this long (clock sampling); 0 under a profiler")
     args = ap.parse_args()
@@ -603,11 +611,13 @@ def main():
     rat.lib()       # fail loudly if the library is missing
 
     pre = run_prefill(w, args.steps, args.warmup, rank, world, peaks, peak_kind,
-                      with_e2e=not args.no_e2e, min_warmup_s=args.min_warmup_s)
+                      with_e2e=not args.no_e2e and args.reset_every == 0,
+                      min_warmup_s=args.min_warmup_s, reset_every=args.reset_every)
     kern = pre["kernels"]
     src_of = {"recur": "scan.cu", "attn": "attn_sm100.cu", "compress": "compress.cu"}
     for n in kern:      # DRAM bytes per launch from the committed ncu capture (null if stale)
-        kern[n]["traffic"] = recorded_traffic(src_of[n], w.name)
+        kern[n]["traffic"] = recorded_traffic(
+            src_of[n], w.name + ("_L%d" % args.reset_every if args.reset_every and n == "recur" else ""))
     dom_name = max(kern, key=lambda n: kern[n]["ms"])
     dom = kern[dom_name]
     roof = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
@@ -621,7 +631,9 @@ def main():
         "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "D": w.D, "W": w.W,
                    "D_per_head": list(w.D_per_head) if w.D_per_head else None,
                    "rope_base": w.rope_base, "gates": [w.gate_mu, w.gate_sigma],
-                   "step": "rat_recur_prefill + rat_dilated_attn_prefill + rat_kv_compress",
+                   "step": "%s + rat_dilated_attn_prefill + rat_kv_compress" % (
+                       "rat_recur_prefill" if args.reset_every == 0 else
+                       "rat_recur_prefill_local(L=%d)" % args.reset_every),
                    "l2": "inputs larger than L2 (q, k, v, a = %d MB per rank)" % (
                        4 * w.B * w.H * w.T * w.d * (2 if w.dtype == "bf16" else 4) // 2**20),
                    "parallelism": "replicas: dp%d over (batch) with no collective" % world},

@@ -10,6 +10,8 @@
  *   rat_recur_prefill        h_t = g_t h_{t-1} + (1-g_t) x_t,  g = sigmoid(gate logit), per
  *                            channel, for x = k and x = v with the same gate, over the whole
  *                            sequence (chunked associative scan); optional RoPE on k~.
+ *   rat_recur_prefill_local  the same recurrence restarted every L positions (RAT's
+ *                            chunk-local form).
  *   rat_dilated_attn_prefill causal attention of each query t over
  *                              S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D = D-1 },
  *                            We = max(W, 1), D per head; optional RoPE on q.
@@ -114,6 +116,31 @@ RAT_API int rat_recur_prefill(const void *k, const void *v, const void *gate_log
                       void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------------------------
+ * rat_recur_prefill_local -- the chunk-local recurrence of RAT: the sequence is cut into blocks
+ * of L positions and the recurrence runs inside each block only.
+ *   Abstract of "RAT: Bridging RNN Efficiency and Attention Accuracy via Chunk-based Sequence
+ *   Modeling" (recurrence within each chunk, attention across chunks) and "RAT+ Deep Dive"
+ *   section 2.1 (original RAT: blocks of size L = D, each token recurs within its own block).
+ *
+ *   Arguments as rat_recur_prefill, plus
+ *   L : block length (>= 1).  Blocks are aligned to absolute positions: the state is set to 0
+ *       before every position p = pos0 + t with p mod L = 0, i.e.
+ *         h_t = (1-g_t) x_t                 if (pos0 + t) mod L = 0
+ *         h_t = g_t h_{t-1} + (1-g_t) x_t   otherwise.
+ *       h0_k, h0_v therefore reach only the positions before the first block start; with
+ *       pos0 mod L = 0 they are ignored.  hT_k, hT_v are the state after position T-1 (the
+ *       value a following call or rat_dilated_decode continues from).
+ *   Returns RAT_ERR_INVALID for L < 1; everything else as rat_recur_prefill.  A block start at
+ *   a chunk boundary of the scan removes that chunk's look-back wait.
+ * ---------------------------------------------------------------------------------------- */
+RAT_API int rat_recur_prefill_local(const void *k, const void *v, const void *gate_logit,
+                            const float *h0_k, const float *h0_v,
+                            void *k_rec, void *v_rec, float *hT_k, float *hT_v,
+                            int B, int H, int T, int d, int dtype,
+                            int64_t pos0, int64_t L, float rope_base,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------
  * rat_dilated_attn_prefill -- causal dilated attention with an optional local window and a
  * per-head dilation, over the recurrence outputs.
  *   RAT+ abstract (dilation D cuts attention FLOPs and KV cache D-fold; optional local
@@ -174,6 +201,9 @@ RAT_API int rat_set_attn_block_keys(int block_keys);
  *   h_k, h_v     : device [B][H][d] float32 recurrence state after the last position
  *                  (before RoPE)
  *   pos          : number of positions consumed so far (the same for every sequence)
+ *   reset_every  : 0 for the full-sequence recurrence of RAT+; L > 0 for the chunk-local
+ *                  recurrence of RAT (state dropped before every position p with p mod L = 0,
+ *                  as in rat_recur_prefill_local); read by rat_dilated_decode
  * The struct itself is host memory; the caller owns every buffer it points to.
  * ---------------------------------------------------------------------------------------- */
 typedef struct rat_kv_cache {
@@ -185,6 +215,7 @@ typedef struct rat_kv_cache {
     void *k_win, *v_win;      /* device ring, or NULL when W == 0                          */
     float *h_k, *h_v;         /* device float32 state                                      */
     int64_t pos;              /* positions consumed so far                                 */
+    int64_t reset_every;      /* recurrence block length L, or 0 (full sequence); >= 0     */
 } rat_kv_cache;
 
 /* Byte sizes of the buffers a cache with these fields needs (any output may be NULL). */
@@ -206,7 +237,8 @@ RAT_API int rat_kv_compress(const void *k_rec, const void *v_rec, const float *h
  *   o                   : device (B, H, 1, d) of cache->dtype
  *   rope_base, scale    : as in prefill (rope_base must match the one used for the cache)
  *   ws, ws_bytes        : workspace of at least rat_decode_workspace_bytes(cache)
- * Per (b, h): state update h = g h + (1-g) x for k and v; k~_t = RoPE(h_k, t); append k~_t, v~_t
+ * Per (b, h): state update h = g h + (1-g) x for k and v (h taken as 0 first when
+ * cache->reset_every = L > 0 and t mod L = 0); k~_t = RoPE(h_k, t); append k~_t, v~_t
  * to the dil cache if t mod D_h = D_h - 1 and to ring slot t mod W; then attention of
  * RoPE(q, t) over the dil entries with position <= t - We, the ring positions
  * t-We < j < t and the token itself -- the same key set S(t) as in prefill.  Split over the

@@ -21,7 +21,8 @@ import torch
 
 __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
-    "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_dilated_attn_prefill",
+    "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_recur_prefill_local",
+    "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
     "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
     "Workspace", "rat_dilated_decode_noalloc",
@@ -50,7 +51,7 @@ class KVCache(ctypes.Structure):
         ("k_dil", ctypes.c_void_p), ("v_dil", ctypes.c_void_p),
         ("k_win", ctypes.c_void_p), ("v_win", ctypes.c_void_p),
         ("h_k", ctypes.c_void_p), ("h_v", ctypes.c_void_p),
-        ("pos", ctypes.c_int64),
+        ("pos", ctypes.c_int64), ("reset_every", ctypes.c_int64),
     ]
 
 
@@ -74,6 +75,8 @@ def lib():
         L.rat_recur_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.rat_recur_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
+        L.rat_recur_prefill_local.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                              _i, _i, _i, _i, _i, _i64, _i64, _f, _vp, _sz, _vp]
         L.rat_dilated_attn_prefill.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
                                                ctypes.POINTER(ctypes.c_int32), _i64, _f, _f, _vp]
         L.rat_kv_cache_bytes.argtypes = [ctypes.POINTER(KVCache), ctypes.POINTER(_sz),
@@ -173,6 +176,18 @@ def rat_recur_prefill(k, v, gate_logit, k_rec, v_rec, ws: Workspace, h0_k=None, 
     _check("rat_recur_prefill", st)
 
 
+def rat_recur_prefill_local(k, v, gate_logit, k_rec, v_rec, ws: Workspace, L: int,
+                            h0_k=None, h0_v=None, hT_k=None, hT_v=None, pos0: int = 0,
+                            rope_base: float = 0.0, stream=None):
+    """rat_recur_prefill restarted before every absolute position that is a multiple of L."""
+    B, H, T, d = k.shape
+    st = lib().rat_recur_prefill_local(_ptr(k), _ptr(v), _ptr(gate_logit), _ptr(h0_k),
+                                       _ptr(h0_v), _ptr(k_rec), _ptr(v_rec), _ptr(hT_k),
+                                       _ptr(hT_v), B, H, T, d, _dtype_code(k), int(pos0), int(L),
+                                       float(rope_base), ws.ptr, ws.nbytes, _stream(stream))
+    _check("rat_recur_prefill_local", st)
+
+
 def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,
                              D_per_head: Optional[Sequence[int]] = None, pos0: int = 0,
                              rope_base: float = 0.0, scale: float = 0.0, stream=None):
@@ -187,10 +202,12 @@ def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,
     _check("rat_dilated_attn_prefill", st)
 
 
-def make_cache(B, H, d, W, Tcap, dtype: int, D_per_head: Sequence[int], device="cuda"):
-    """Allocate (with torch) the buffers of a compressed cache and return (KVCache, buffers)."""
+def make_cache(B, H, d, W, Tcap, dtype: int, D_per_head: Sequence[int], device="cuda",
+               reset_every: int = 0):
+    """Allocate (with torch) the buffers of a compressed cache and return (KVCache, buffers).
+    reset_every = L > 0 selects the chunk-local recurrence for the decode steps."""
     Dh = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
-    c = KVCache(B=B, H=H, d=d, W=W, Tcap=Tcap, dtype=dtype, D=Dh)
+    c = KVCache(B=B, H=H, d=d, W=W, Tcap=Tcap, dtype=dtype, D=Dh, reset_every=int(reset_every))
     dil, win, state = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     _check("rat_kv_cache_bytes", lib().rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(dil),
                                                           ctypes.byref(win), ctypes.byref(state)))

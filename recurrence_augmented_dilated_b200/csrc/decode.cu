@@ -4,7 +4,9 @@
 // "RAT+ Deep Dive" section 2.1 (the recurrence state carries what dilation skips).  For the token
 // at position t of slice (b, h):
 //   1. state update  h_k = g h_k + (1-g) k,  h_v = g h_v + (1-g) v   (float32, g = sigmoid(a));
-//      k~_t = RoPE(h_k, t), v~_t = h_v, both rounded to the cache dtype;
+//      k~_t = RoPE(h_k, t), v~_t = h_v, both rounded to the cache dtype; with the chunk-local
+//      recurrence of RAT (abstract of "RAT: Bridging RNN Efficiency and Attention Accuracy"),
+//      h is dropped first when t is a multiple of the block length L;
 //   2. append k~_t, v~_t to dil entry (t - D + 1) / D if t mod D = D - 1, and to ring slot t mod W;
 //   3. attention of q^ = RoPE(q, t) over the prefill key set S(t): dil entries whose position
 //      i*D + D - 1 <= t - We, ring positions t - We < j < t, and the token itself.
@@ -158,13 +160,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         load8(static_cast<const uint8_t *>(p.a) + (size_t)bh * RB + cl * 16, an);
         float *hk = p.hk + (size_t)bh * DH + cl * 8;
         float *hv = p.hv + (size_t)bh * DH + cl * 8;
+        // chunk-local recurrence: the state is dropped before every position that starts a block
+        const bool fresh = p.reset > 0 && t % p.reset == 0;
         float sk[8], sv[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             float g, omg;
             forget_gate(an[j], g, omg);
-            sk[j] = fmaf(g, hk[j], omg * kn[j]);
-            sv[j] = fmaf(g, hv[j], omg * vn[j]);
+            sk[j] = fresh ? omg * kn[j] : fmaf(g, hk[j], omg * kn[j]);
+            sv[j] = fresh ? omg * vn[j] : fmaf(g, hv[j], omg * vn[j]);
         }
         float kt[8];
 #pragma unroll

@@ -44,6 +44,7 @@ struct RecurParams {
     float step_cos[64], step_sin[64];   // cos/sin(theta_c): one-position rotation
     long long fault_chunk;      // test hook: chunk index that never publishes (-1: none)
     unsigned long long wait_ns; // bound of each look-back wait
+    long long reset;            // > 0: state zeroed before every position that is a multiple (chunk-local recurrence)
 };
 int recur_chunk_rows(int d, int dtype);
 size_t recur_workspace_bytes(int BH, int T, int d, int dtype);
@@ -123,6 +124,7 @@ struct DecodeParams {
     float *hk, *hv;
     int B, H, d, W, Tcap, splits;
     long long t;                // position of the new token
+    long long reset;            // > 0: state dropped before every position that is a multiple
     long long total_cap;
     int rope;
     float scale_log2;

@@ -36,7 +36,7 @@ long long total_capacity(int H, int Tcap, const int32_t *Dh, long long *off) {
 
 bool valid_cache(const rat_kv_cache *c) {
     if (!c || c->B < 1 || c->H < 1 || c->H > kMaxHeads || !supported_d(c->d) || c->W < 0 ||
-        c->Tcap < 1 || !valid_dtype(c->dtype) || !c->D)
+        c->Tcap < 1 || !valid_dtype(c->dtype) || !c->D || c->reset_every < 0)
         return false;
     for (int h = 0; h < c->H; ++h)
         if (c->D[h] < 1) return false;
@@ -110,11 +110,16 @@ size_t rat_recur_workspace_bytes(int B, int H, int T, int d, int dtype) {
     return recur_workspace_bytes(B * H, T, d, dtype);
 }
 
-int rat_recur_prefill(const void *k, const void *v, const void *gate_logit, const float *h0_k,
-                      const float *h0_v, void *k_rec, void *v_rec, float *hT_k, float *hT_v,
-                      int B, int H, int T, int d, int dtype, int64_t pos0, float rope_base,
-                      void *ws, size_t ws_bytes, void *stream) {
-    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype)) return RAT_ERR_INVALID;
+}  // extern "C"
+
+namespace {
+// Both recurrence entry points: reset_every = 0 is the full-sequence recurrence, L > 0 drops
+// the state before every absolute position that is a multiple of L.
+int recur_prefill(const void *k, const void *v, const void *gate_logit, const float *h0_k,
+                  const float *h0_v, void *k_rec, void *v_rec, float *hT_k, float *hT_v, int B,
+                  int H, int T, int d, int dtype, int64_t pos0, int64_t reset_every,
+                  float rope_base, void *ws, size_t ws_bytes, void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || reset_every < 0) return RAT_ERR_INVALID;
     if (!supported_d(d)) return RAT_ERR_UNSUPPORTED;
     if (pos0 < 0 || !std::isfinite(rope_base)) return RAT_ERR_INVALID;
     if (T == 0) return RAT_OK;
@@ -136,6 +141,7 @@ int rat_recur_prefill(const void *k, const void *v, const void *gate_logit, cons
     const int tc = recur_chunk_rows(d, dtype);
     p.nchunks = (T + tc - 1) / tc;
     p.pos0 = pos0;
+    p.reset = reset_every;
     p.rope = rope_base > 0.f ? 1 : 0;
     p.fault_chunk = g_fault_chunk;
     p.wait_ns = g_fault_chunk >= 0 ? g_fault_wait_ns : kWaitLimitNs;
@@ -155,6 +161,27 @@ int rat_recur_prefill(const void *k, const void *v, const void *gate_logit, cons
         p.rope_f32 = (dtype == RAT_BF16 && pos0 + (int64_t)T <= 8192) ? 1 : 0;
     }
     return launch_recur(p, dtype, stream);
+}
+}  // namespace
+
+extern "C" {
+
+int rat_recur_prefill(const void *k, const void *v, const void *gate_logit, const float *h0_k,
+                      const float *h0_v, void *k_rec, void *v_rec, float *hT_k, float *hT_v,
+                      int B, int H, int T, int d, int dtype, int64_t pos0, float rope_base,
+                      void *ws, size_t ws_bytes, void *stream) {
+    return recur_prefill(k, v, gate_logit, h0_k, h0_v, k_rec, v_rec, hT_k, hT_v, B, H, T, d,
+                         dtype, pos0, 0, rope_base, ws, ws_bytes, stream);
+}
+
+int rat_recur_prefill_local(const void *k, const void *v, const void *gate_logit,
+                            const float *h0_k, const float *h0_v, void *k_rec, void *v_rec,
+                            float *hT_k, float *hT_v, int B, int H, int T, int d, int dtype,
+                            int64_t pos0, int64_t L, float rope_base, void *ws, size_t ws_bytes,
+                            void *stream) {
+    if (L < 1) return RAT_ERR_INVALID;
+    return recur_prefill(k, v, gate_logit, h0_k, h0_v, k_rec, v_rec, hT_k, hT_v, B, H, T, d,
+                         dtype, pos0, L, rope_base, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------------------ attention
@@ -284,6 +311,7 @@ int rat_dilated_decode(const void *q, const void *k, const void *v, const void *
     p.hk = c->h_k; p.hv = c->h_v;
     p.B = c->B; p.H = c->H; p.d = c->d; p.W = c->W; p.Tcap = c->Tcap; p.splits = splits;
     p.t = c->pos;
+    p.reset = c->reset_every;
     for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
     p.total_cap = total_capacity(c->H, c->Tcap, c->D, p.off);
     p.rope = rope_base > 0.f ? 1 : 0;

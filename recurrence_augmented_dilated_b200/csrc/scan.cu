@@ -97,7 +97,9 @@ template <> struct Lane<__nv_bfloat16> {
 // value and its validity always travel together.
 RAT_DEVICE uint64_t tagged(uint32_t tag, float v) { return ((uint64_t)tag << 32) | __float_as_uint(v); }
 
-template <typename E, int DH>
+// RESET: the chunk-local form (p.reset > 0) is a separate instantiation, so the full-sequence
+// scan carries none of its per-row tests.
+template <typename E, int DH, bool RESET>
 __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const __grid_constant__ RecurParams p) {
     using C = ScanCfg<E, DH>;
     constexpr int LPR = C::LPR, R = C::R, HALF = DH / 2, NP = 2;
@@ -190,10 +192,25 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
         const size_t row0 = (size_t)bh * p.T + t0;
         const bool publish = c != p.fault_chunk;            // false only under the test hook
         const uint8_t *sa = pbase + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
+        // chunk-local recurrence: bit i of rmask marks row seg*R + i as the first of a block
+        // (the carried state is dropped there); a chunk that starts a block needs no carry
+        uint32_t rmask = 0;
+        bool fresh = false;
+        if (RESET) {
+            const long long m = (p.pos0 + t0 + seg * R) % p.reset;
+            const long long off = m == 0 ? 0 : p.reset - m;               // rows to the next block start
+            const int lim = min(R, rows - seg * R);       // rows past the end keep the identity step
+            if (off < lim) {
+                const int step = p.reset < R ? (int)p.reset : R;          // beyond R: one start at most
+#pragma unroll 1
+                for (int i = (int)off; i < lim; i += step) rmask |= 1u << i;
+            }
+            fresh = (p.pos0 + t0) % p.reset == 0;
+        }
         // the first look-back round is issued now and consumed after pass 1, so its memory
         // latency overlaps the wait for the data and pass 1
         uint64_t w[C::LBW][5];
-        if (pt < DH && c > 0) read_window(bh, c - 1, pt, w);
+        if (pt < DH && c > 0 && !fresh) read_window(bh, c - 1, pt, w);
         mbar_wait_bounded(&bar[pipe][st], (it >> 1) & 1, hdr, 0x100u);
 
         // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate
@@ -210,6 +227,10 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
             Lane<E>::template load<C::HALFB>(sa + off, cl, xa);
             Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
             Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
+            if (RESET && ((rmask >> i) & 1)) {        // a block starts at this row: the state before it is dropped
+#pragma unroll
+                for (int q = 0; q < NP; ++q) { A[q] = kZero2; Bk[q] = kZero2; Bv[q] = kZero2; }
+            }
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
                 G[i][q] = r < rows ? forget_gate2(xa[q]) : kOne2;
@@ -284,6 +305,8 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
             if (c == 0) {
                 if (p.h0k) Hk = p.h0k[(size_t)bh * DH + ch];
                 if (p.h0v) Hv = p.h0v[(size_t)bh * DH + ch];
+            } else if (fresh) {
+                // the chunk starts a block: the state before it is dropped, nothing to wait for
             } else {
                 // Walk back from j = c - 1, C::LBW predecessors per round: all five words of each
                 // (inclusive state k, v; aggregate A, Bk, Bv) are read at once, so a round costs one
@@ -312,6 +335,11 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
                             xV = fmaf(xA, val(4), xV);
                             xA *= val(2);
                             ++passed;
+                            if (RESET && xA == 0.f) {   // a block starts in between: older state is dropped
+                                Hk = xK;
+                                Hv = xV;
+                                done = true;
+                            }
                         } else {
                             stop = true;
                         }
@@ -391,6 +419,10 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
             f2_t xk[NP], xv[NP];
             Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
             Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
+            if (RESET && ((rmask >> i) & 1)) {
+#pragma unroll
+                for (int q = 0; q < NP; ++q) { hk[q] = kZero2; hv[q] = kZero2; }
+            }
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
                 const f2_t og = gate_complement2(G[i][q]);
@@ -442,9 +474,9 @@ size_t recur_workspace_bytes(int BH, int T, int d, int dtype) {
 template <typename E, int DH>
 static int launch_one(const RecurParams &p, void *stream) {
     using C = ScanCfg<E, DH>;
-    auto kern = recur_kernel<E, DH>;
-    static uint64_t attr_done = 0;
-    const int st = set_smem_attr(reinterpret_cast<const void *>(kern), C::SMEM, &attr_done);
+    auto kern = p.reset > 0 ? recur_kernel<E, DH, true> : recur_kernel<E, DH, false>;
+    static uint64_t attr_done[2] = {0, 0};
+    const int st = set_smem_attr(reinterpret_cast<const void *>(kern), C::SMEM, &attr_done[p.reset > 0]);
     if (st != RAT_OK) return st;
     const int sms = current_sm_count();
     if (sms <= 0) return RAT_ERR_CUDA;

@@ -30,8 +30,9 @@ def rel_err(x, r) -> float:
     return float(np.max(np.abs(x - r))) / (den if den > 0 else 1.0)
 
 
-def gpu_recur(k, v, a, rope_base=0.0, pos0=0, h0k=None, h0v=None, ws=None):
-    """Run rat_recur_prefill on device copies; returns (k_rec, v_rec, hT_k, hT_v) on device."""
+def gpu_recur(k, v, a, rope_base=0.0, pos0=0, h0k=None, h0v=None, ws=None, reset_every=0):
+    """Run rat_recur_prefill (rat_recur_prefill_local when reset_every > 0) on device copies;
+    returns (k_rec, v_rec, hT_k, hT_v) on device."""
     dev = torch.device("cuda")
     k, v, a = (x.to(dev) for x in (k, v, a))
     B, H, T, d = k.shape
@@ -41,8 +42,12 @@ def gpu_recur(k, v, a, rope_base=0.0, pos0=0, h0k=None, h0v=None, ws=None):
     hTv = torch.empty_like(hTk)
     if ws is None:
         ws = rat.Workspace(rat.rat_recur_workspace_bytes(B, H, T, d, 0 if k.dtype == torch.float32 else 1))
-    rat.rat_recur_prefill(k, v, a, kr, vr, ws, h0_k=h0k, h0_v=h0v, hT_k=hTk, hT_v=hTv, pos0=pos0,
-                          rope_base=rope_base)
+    if reset_every > 0:
+        rat.rat_recur_prefill_local(k, v, a, kr, vr, ws, reset_every, h0_k=h0k, h0_v=h0v,
+                                    hT_k=hTk, hT_v=hTv, pos0=pos0, rope_base=rope_base)
+    else:
+        rat.rat_recur_prefill(k, v, a, kr, vr, ws, h0_k=h0k, h0_v=h0v, hT_k=hTk, hT_v=hTv,
+                              pos0=pos0, rope_base=rope_base)
     st = rat.rat_sync_status(ws)
     assert st == 0, rat.rat_status_string(st)
     return kr, vr, hTk, hTv

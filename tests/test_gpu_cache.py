@@ -78,7 +78,7 @@ def test_compress_chunked_equals_whole():
         assert torch.equal(b1[n], b2[n]), n
 
 
-def run_decode(w, T0, steps, heads_check, B=None, H=None, rope_base=0.0):
+def run_decode(w, T0, steps, heads_check, B=None, H=None, rope_base=0.0, reset_every=0):
     """GPU: prefill a T0-token context, compress, then decode `steps` tokens.
     Oracle: the same from the same raw inputs on the (b, h) slices in heads_check."""
     B = w.B if B is None else B
@@ -87,13 +87,14 @@ def run_decode(w, T0, steps, heads_check, B=None, H=None, rope_base=0.0):
     Dh = w.heads_D()[:H]
     Tcap = T0 + steps
     dev = torch.device("cuda")
-    cache, bufs = rat.make_cache(B, H, d, W, Tcap, rat.BF16, Dh)
+    cache, bufs = rat.make_cache(B, H, d, W, Tcap, rat.BF16, Dh, reset_every=reset_every)
     hk = torch.zeros((B, H, d), dtype=torch.float32, device=dev)
     hv = torch.zeros_like(hk)
     nchunks = (T0 + synthetic.CTX_CHUNK - 1) // synthetic.CTX_CHUNK
     for c in range(nchunks):     # chunked prefill of the context: state carried, cache appended
         k, v, a = synthetic.decode_context_block(w, c, device=dev, T=T0, B=B, H=H)
-        kr, vr, hk, hv = gpu_recur(k, v, a, rope_base=rope_base, pos0=cache.pos, h0k=hk, h0v=hv)
+        kr, vr, hk, hv = gpu_recur(k, v, a, rope_base=rope_base, pos0=cache.pos, h0k=hk, h0v=hv,
+                                   reset_every=reset_every)
         rat.rat_kv_compress(kr, vr, hk, hv, cache)
         del k, v, a, kr, vr
     tok = synthetic.decode_steps(w, steps)
@@ -109,7 +110,8 @@ def run_decode(w, T0, steps, heads_check, B=None, H=None, rope_base=0.0):
     assert cache.pos == Tcap
     got = torch.stack(outs)[:, :, :, 0]            # (steps, B, H, d)
     # oracle on the checked slices
-    st = oracle.DecodeState([Dh[h] for _, h in heads_check], d, W, Tcap, rope_base=rope_base)
+    st = oracle.DecodeState([Dh[h] for _, h in heads_check], d, W, Tcap, rope_base=rope_base,
+                            reset_every=reset_every)
     ctx = [synthetic.decode_context_slice(w, b, h, device=dev, T=T0) for b, h in heads_check]
     st.prefill(np.stack([f64(x[0]) for x in ctx]), np.stack([f64(x[1]) for x in ctx]),
                np.stack([f64(x[2]) for x in ctx]))
@@ -143,5 +145,18 @@ def test_decode_no_window():
 def test_decode_full_size_sampled():
     w = synthetic.WORKLOADS["decode_7p6b"]
     err, herr = run_decode(w, T0=w.T, steps=8, heads_check=[(0, 0), (w.B - 1, w.H - 1), (5, 17)])
+    assert err <= TOL_BF16, err
+    assert herr <= 1e-3, herr
+
+
+@pytest.mark.parametrize("L", [1, 16, 50])
+def test_decode_local_recurrence(L):
+    # RAT's chunk-local recurrence in decode: the context ends inside a block (100 mod L != 0 for
+    # L = 16, 50) and the decoded tokens cross block starts; L = 16 equals the largest head's D
+    w = synthetic.Workload("dec_local", B=2, H=3, d=128, T=0, W=8, D_per_head=(1, 4, 16),
+                           dtype="bf16", seed=42)
+    heads = [(b, h) for b in range(2) for h in range(3)]
+    err, herr = run_decode(w, T0=100, steps=40, heads_check=heads, rope_base=10000.0,
+                           reset_every=L)
     assert err <= TOL_BF16, err
     assert herr <= 1e-3, herr

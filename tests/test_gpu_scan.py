@@ -11,12 +11,13 @@ from gpu_util import TOL_BF16, TOL_F32, f64, gpu_recur, rel_err, tol_for
 pytestmark = pytest.mark.gpu
 
 
-def check(k, v, a, rope_base=0.0, pos0=0, heads=None, h0=None):
+def check(k, v, a, rope_base=0.0, pos0=0, heads=None, h0=None, reset_every=0):
     """GPU vs oracle on all (b, h) or on `heads` (list of (b, h))."""
     h0k = h0v = None
     if h0 is not None:
         h0k, h0v = (x.cuda() for x in h0)
-    kr, vr, hTk, hTv = gpu_recur(k, v, a, rope_base=rope_base, pos0=pos0, h0k=h0k, h0v=h0v)
+    kr, vr, hTk, hTv = gpu_recur(k, v, a, rope_base=rope_base, pos0=pos0, h0k=h0k, h0v=h0v,
+                                 reset_every=reset_every)
     sel = heads if heads is not None else [(b, h) for b in range(k.shape[0]) for h in range(k.shape[1])]
     bi = [b for b, _ in sel]
     hi = [h for _, h in sel]
@@ -24,8 +25,8 @@ def check(k, v, a, rope_base=0.0, pos0=0, heads=None, h0=None):
     oa_ = f64(a[bi, hi])
     o_h0k = f64(h0[0][bi, hi]) if h0 is not None else None
     o_h0v = f64(h0[1][bi, hi]) if h0 is not None else None
-    yk, hk = oracle.recurrence(ok_, oa_, o_h0k)
-    yv, hv = oracle.recurrence(ov_, oa_, o_h0v)
+    yk, hk = oracle.recurrence(ok_, oa_, o_h0k, pos0=pos0, reset_every=reset_every)
+    yv, hv = oracle.recurrence(ov_, oa_, o_h0v, pos0=pos0, reset_every=reset_every)
     if rope_base > 0:
         yk = oracle.rope(yk, pos0, rope_base)
     tol = tol_for(k.dtype)
@@ -134,3 +135,60 @@ def test_lookback_timeout_is_reported():
     assert rat.rat_sync_status(ws) == -4
     # the next call (no fault armed) is correct again
     check(x["k"], x["v"], x["a"])
+
+
+# ---- chunk-local recurrence (RAT: the state restarts every L positions)
+# The scan's chunk holds 32 (float32, d 128), 64 (float32 d 64, bf16 d 128) or 128 (bf16 d 64)
+# rows, split into segments of 4 or 8 rows per lane; L is chosen below, equal to and above those
+# sizes, as a divisor and a non-divisor of them, and beyond the sequence.
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("L", [1, 3, 8, 16, 37, 64, 128, 200, 5000])
+def test_local_recurrence(dtype, d, L):
+    x = inputs(2, 2, 1100, d, dtype, seed=L + d)
+    check(x["k"], x["v"], x["a"], reset_every=L)
+
+
+@pytest.mark.parametrize("pos0", [5, 63, 64, 1000003])
+def test_local_recurrence_offsets_and_initial_state(pos0):
+    # blocks are aligned to absolute positions; h0 reaches only the rows before the first start
+    x = inputs(2, 2, 700, 128, torch.float32, seed=pos0 % 97)
+    g = torch.Generator().manual_seed(pos0 % 89)
+    h0 = (torch.randn((2, 2, 128), generator=g), torch.randn((2, 2, 128), generator=g))
+    for L in (16, 64, 100):
+        check(x["k"], x["v"], x["a"], pos0=pos0, h0=h0, reset_every=L, rope_base=10000.0)
+
+
+def test_local_recurrence_chained_equals_whole():
+    # float32 outputs: the two forms differ only in float32 rounding order, which can flip a
+    # bf16 rounding
+    x = inputs(1, 3, 900, 128, torch.float32, seed=77)
+    k, v, a = (t.cuda() for t in (x["k"], x["v"], x["a"]))
+    L = 48
+    kr, vr, hk, hv = gpu_recur(k, v, a, reset_every=L)
+    cut = 301
+    parts = [slice(0, cut), slice(cut, 900)]
+    kr1, vr1, hk1, hv1 = gpu_recur(*(t[:, :, parts[0]].contiguous() for t in (k, v, a)), reset_every=L)
+    kr2, vr2, hk2, hv2 = gpu_recur(*(t[:, :, parts[1]].contiguous() for t in (k, v, a)), reset_every=L,
+                                   pos0=cut, h0k=hk1, h0v=hv1)
+    assert rel_err(torch.cat([kr1, kr2], 2), kr) <= 1e-5
+    assert rel_err(torch.cat([vr1, vr2], 2), vr) <= 1e-5
+    assert rel_err(hk2, hk) <= 1e-5 and rel_err(hv2, hv) <= 1e-5
+
+
+def test_local_recurrence_block_one_is_the_input_term():
+    # L = 1: every row starts a block, so k~_t = (1 - g_t) k_t exactly as the kernel rounds it
+    # (one float32 product of the gate complement and the input)
+    x = inputs(1, 2, 257, 64, torch.float32, seed=5)
+    kr, vr, hk, _ = gpu_recur(x["k"], x["v"], x["a"], reset_every=1)
+    ref = oracle.recurrence(f64(x["k"]), f64(x["a"]), reset_every=1)[0]
+    assert rel_err(kr, ref) <= TOL_F32
+    assert rel_err(hk, ref[..., -1, :]) <= TOL_F32
+
+
+def test_local_recurrence_full_size_sampled_heads():
+    # the prefill_1p5b workload (B 4, H 16, T 4096, d 128, bf16, RoPE) with RAT's chunk size 16
+    w = synthetic.WORKLOADS["prefill_1p5b"]
+    x = synthetic.prefill_inputs(w)
+    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)]
+    check(x["k"], x["v"], x["a"], rope_base=w.rope_base, heads=heads, reset_every=16)
