@@ -48,6 +48,7 @@ def _load():
         lib = ctypes.CDLL(build())
         lib.rat_oracle_recurrence.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp]
         lib.rat_oracle_recurrence_reset.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _L, _L]
+        lib.rat_oracle_recurrence_window.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _L, _dp]
         lib.rat_oracle_rope.argtypes = [_L, _L, _L, _dp, _L, ctypes.c_double]
         lib.rat_oracle_in_key_set.argtypes = [_L, _L, _L, _L]
         lib.rat_oracle_in_key_set.restype = ctypes.c_int
@@ -112,6 +113,28 @@ def recurrence(x, a, h0=None, pos0: int = 0, reset_every: int = 0):
     else:
         _load().rat_oracle_recurrence(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(y), _ptr(hT))
     return y, hT
+
+
+def recurrence_window(x, a, Lw: int = 64, prev_x=None, prev_a=None):
+    """Fixed-window recurrence: y_t is the forget-gate recurrence restarted from zero at
+    t - Lw + 1 and run to t ("RAT+ Deep Dive" section 2.1, recurrence window L* = 64).
+
+    x, a: (..., T, d).  prev_x, prev_a: (..., Lw, d), the Lw positions before row 0, or None
+    (the window is clipped at row 0).  Returns y in float64.
+    """
+    x = _f64(x)
+    a = _f64(a)
+    assert x.shape == a.shape and int(Lw) >= 1
+    T, d = x.shape[-2], x.shape[-1]
+    BH = int(np.prod(x.shape[:-2])) if x.ndim > 2 else 1
+    y = np.empty_like(x)
+    px = pa = None
+    if prev_x is not None:
+        prev_x, prev_a = _f64(prev_x), _f64(prev_a)
+        assert prev_x.shape == x.shape[:-2] + (int(Lw), d) and prev_a.shape == prev_x.shape
+        px, pa = _ptr(prev_x), _ptr(prev_a)
+    _load().rat_oracle_recurrence_window(BH, T, d, _ptr(x), _ptr(a), px, pa, int(Lw), _ptr(y))
+    return y
 
 
 def rope(x, pos0: int = 0, base: float = 10000.0):

@@ -102,6 +102,42 @@ void rat_oracle_recurrence_reset(long BH, long T, long d, const double *x, const
 }
 
 /*
+ * Fixed-window recurrence of RAT+ ("RAT+ Deep Dive" section 2.1: every token's recurrence looks
+ * back a fixed L* = 64 tokens, independent of the dilation).  Read as: the state at t is the
+ * forget-gate recurrence started from zero at position t - Lw + 1 and run to t,
+ *   y_t = sum_{s = t-Lw+1}^{t} ( prod_{r = s+1}^{t} g_r ) (1 - g_s) x_s,
+ * evaluated here by that restarted sequential loop for every t (O(T Lw) per channel).  Rows
+ * before the sequence come from prev_x / prev_a ([BH][Lw][d]: the Lw positions just before row 0,
+ * oldest first) when given; without them the window is clipped at row 0.
+ */
+void rat_oracle_recurrence_window(long BH, long T, long d, const double *x, const double *a,
+                                  const double *prev_x, const double *prev_a, long Lw, double *y)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        for (long c = 0; c < d; ++c) {
+            for (long t = 0; t < T; ++t) {
+                double h = 0.0;
+                for (long s = t - Lw + 1; s <= t; ++s) {
+                    double xs, as;
+                    if (s >= 0) {
+                        xs = x[(bh * T + s) * d + c];
+                        as = a[(bh * T + s) * d + c];
+                    } else if (prev_x && s >= -Lw) {
+                        xs = prev_x[(bh * Lw + (Lw + s)) * d + c];
+                        as = prev_a[(bh * Lw + (Lw + s)) * d + c];
+                    } else {
+                        continue;           /* before the known sequence: clipped */
+                    }
+                    h = forget_gate(as) * h + one_minus_gate(as) * xs;
+                }
+                y[(bh * T + t) * d + c] = h;
+            }
+        }
+    }
+}
+
+/*
  * Rotary position embedding, rotate-half pairing, in place.                  [RoFormer]
  *   x : [BH][T][d];  position of row t is pos0 + t;  for c < d/2:
  *   theta_c = base^(-2c/d),  phi = (pos0 + t) * theta_c,

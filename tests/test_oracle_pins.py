@@ -173,6 +173,73 @@ def test_reset_brute_force_sum():
         np.testing.assert_allclose(y[0, t], acc, rtol=1e-12, atol=1e-13)
 
 
+# ---- fixed-window recurrence (each state covers the last Lw positions only)
+def test_window_longer_than_the_sequence_is_the_full_recurrence():
+    # no position ever leaves the window: the full recurrence from a zero state
+    x, a = RNG.standard_normal((2, 40, 3)), RNG.standard_normal((2, 40, 3))
+    y = oracle.recurrence_window(x, a, Lw=40)
+    want, _ = oracle.recurrence(x, a)
+    np.testing.assert_allclose(y, want, rtol=1e-13, atol=1e-14)
+    np.testing.assert_array_equal(oracle.recurrence_window(x, a, Lw=1000), y)
+
+
+def test_window_of_one_is_the_input_term():
+    x, a = RNG.standard_normal((2, 30, 4)), 3 * RNG.standard_normal((2, 30, 4))
+    y = oracle.recurrence_window(x, a, Lw=1)
+    g = 1.0 / (1.0 + np.exp(-a))
+    np.testing.assert_allclose(y, (1.0 - g) * x, rtol=1e-14, atol=1e-15)
+
+
+@pytest.mark.parametrize("Lw", [4, 7, 16])
+def test_window_at_block_ends_equals_the_chunk_local_recurrence(Lw):
+    # at t = m Lw + Lw - 1 the window is exactly block m of the chunk-local form
+    T = 5 * Lw + 3
+    x, a = RNG.standard_normal((2, T, 3)), RNG.standard_normal((2, T, 3))
+    y = oracle.recurrence_window(x, a, Lw=Lw)
+    loc, _ = oracle.recurrence(x, a, reset_every=Lw)
+    ends = np.arange(Lw - 1, T, Lw)
+    np.testing.assert_allclose(y[:, ends], loc[:, ends], rtol=1e-13, atol=1e-14)
+    # before the first block ends the clipped window is the plain recurrence from row 0
+    np.testing.assert_allclose(y[:, :Lw], loc[:, :Lw], rtol=1e-13, atol=1e-14)
+
+
+def test_window_is_full_state_minus_the_decayed_old_state():
+    # y_t = h_t - (prod_{r=t-Lw+1..t} g_r) h_{t-Lw} with h the full recurrence: a different formula
+    T, Lw = 60, 9
+    x, a = RNG.standard_normal((2, T, 3)), RNG.standard_normal((2, T, 3))
+    y = oracle.recurrence_window(x, a, Lw=Lw)
+    h, _ = oracle.recurrence(x, a)
+    g = 1.0 / (1.0 + np.exp(-a))
+    for t in range(Lw, T):
+        want = h[:, t] - np.prod(g[:, t - Lw + 1:t + 1], axis=1) * h[:, t - Lw]
+        np.testing.assert_allclose(y[:, t], want, rtol=1e-9, atol=1e-11)
+
+
+def test_window_brute_force_sum_with_history():
+    # explicit weighted sum over the window, the positions before row 0 taken from prev
+    T, Lw = 11, 5
+    x, a = RNG.standard_normal((1, T, 2)), RNG.standard_normal((1, T, 2))
+    px, pa = RNG.standard_normal((1, Lw, 2)), RNG.standard_normal((1, Lw, 2))
+    y = oracle.recurrence_window(x, a, Lw=Lw, prev_x=px, prev_a=pa)
+    xs = np.concatenate([px[0], x[0]])
+    gs = 1.0 / (1.0 + np.exp(-np.concatenate([pa[0], a[0]])))
+    for t in range(T):
+        u = t + Lw                                   # index into the joined sequence
+        acc = np.zeros(2)
+        for s_ in range(u - Lw + 1, u + 1):
+            acc += np.prod(gs[s_ + 1:u + 1], axis=0) * (1 - gs[s_]) * xs[s_]
+        np.testing.assert_allclose(y[0, t], acc, rtol=1e-12, atol=1e-13)
+
+
+def test_window_history_equals_the_joined_sequence():
+    T, Lw = 37, 8
+    x, a = RNG.standard_normal((3, T, 2)), RNG.standard_normal((3, T, 2))
+    px, pa = RNG.standard_normal((3, Lw, 2)), RNG.standard_normal((3, Lw, 2))
+    y = oracle.recurrence_window(x, a, Lw=Lw, prev_x=px, prev_a=pa)
+    joined = oracle.recurrence_window(np.concatenate([px, x], 1), np.concatenate([pa, a], 1), Lw=Lw)
+    np.testing.assert_array_equal(y, joined[:, Lw:])
+
+
 def test_rope_matches_complex_rotation():
     d, T, pos0, base = 16, 9, 1000, 10000.0
     x = RNG.standard_normal((1, T, d))
