@@ -218,7 +218,8 @@ class ProfiledRegion:
 
 
 def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world: int, peaks,
-                peak_kind, with_e2e: bool, min_warmup_s: float = 1.0, reset_every: int = 0):
+                peak_kind, with_e2e: bool, min_warmup_s: float = 1.0, reset_every: int = 0,
+                window: int = 0):
     import recurrence_augmented_dilated_b200 as rat
     dev = torch.device("cuda")
     x = synthetic.prefill_inputs(w, seed=w.seed + 1000 * rank)
@@ -236,7 +237,9 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
     def step(timer=None, qq=q, kk=k, vv=v, aa=a):
         span = timer.span if timer else (lambda n: _Null())
         with span("recur"):
-            if reset_every > 0:
+            if window > 0:
+                rat.rat_recur_prefill_window(kk, vv, aa, kr, vr, ws, window, rope_base=w.rope_base)
+            elif reset_every > 0:
                 rat.rat_recur_prefill_local(kk, vv, aa, kr, vr, ws, reset_every, hT_k=hk, hT_v=hv,
                                             rope_base=w.rope_base)
             else:
@@ -571,6 +574,9 @@ def main():
     ap.add_argument("--reset-every", type=int, default=0,
                     help="L > 0: the chunk-local recurrence (restart every L positions) in the "
                          "prefill step instead of the full-sequence one")
+    ap.add_argument("--window", type=int, default=0,
+                    help="Lw > 0: the fixed-window recurrence (each state over the last Lw "
+                         "positions) in the prefill step")
     ap.add_argument("--min-warmup-s", type=float, default=1.0,
                     help="keep warming up at least this long (clock sampling); 0 under a profiler")
     args = ap.parse_args()
@@ -611,13 +617,16 @@ def main():
     rat.lib()       # fail loudly if the library is missing
 
     pre = run_prefill(w, args.steps, args.warmup, rank, world, peaks, peak_kind,
-                      with_e2e=not args.no_e2e and args.reset_every == 0,
-                      min_warmup_s=args.min_warmup_s, reset_every=args.reset_every)
+                      with_e2e=not args.no_e2e and args.reset_every == 0 and args.window == 0,
+                      min_warmup_s=args.min_warmup_s, reset_every=args.reset_every,
+                      window=args.window)
     kern = pre["kernels"]
-    src_of = {"recur": "scan.cu", "attn": "attn_sm100.cu", "compress": "compress.cu"}
+    src_of = {"recur": "window.cu" if args.window else "scan.cu", "attn": "attn_sm100.cu",
+              "compress": "compress.cu"}
+    variant = ("_L%d" % args.reset_every if args.reset_every else
+               "_window%d" % args.window if args.window else "")
     for n in kern:      # DRAM bytes per launch from the committed ncu capture (null if stale)
-        kern[n]["traffic"] = recorded_traffic(
-            src_of[n], w.name + ("_L%d" % args.reset_every if args.reset_every and n == "recur" else ""))
+        kern[n]["traffic"] = recorded_traffic(src_of[n], w.name + (variant if n == "recur" else ""))
     dom_name = max(kern, key=lambda n: kern[n]["ms"])
     dom = kern[dom_name]
     roof = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
@@ -632,8 +641,9 @@ def main():
                    "D_per_head": list(w.D_per_head) if w.D_per_head else None,
                    "rope_base": w.rope_base, "gates": [w.gate_mu, w.gate_sigma],
                    "step": "%s + rat_dilated_attn_prefill + rat_kv_compress" % (
-                       "rat_recur_prefill" if args.reset_every == 0 else
-                       "rat_recur_prefill_local(L=%d)" % args.reset_every),
+                       "rat_recur_prefill_window(Lw=%d)" % args.window if args.window else
+                       "rat_recur_prefill_local(L=%d)" % args.reset_every if args.reset_every else
+                       "rat_recur_prefill"),
                    "l2": "inputs larger than L2 (q, k, v, a = %d MB per rank)" % (
                        4 * w.B * w.H * w.T * w.d * (2 if w.dtype == "bf16" else 4) // 2**20),
                    "parallelism": "replicas: dp%d over (batch) with no collective" % world},

@@ -12,6 +12,8 @@
  *                            sequence (chunked associative scan); optional RoPE on k~.
  *   rat_recur_prefill_local  the same recurrence restarted every L positions (RAT's
  *                            chunk-local form).
+ *   rat_recur_prefill_window the same recurrence over a fixed window of the last Lw = 64
+ *                            positions (RAT+'s L*).
  *   rat_dilated_attn_prefill causal attention of each query t over
  *                              S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D = D-1 },
  *                            We = max(W, 1), D per head; optional RoPE on q.
@@ -139,6 +141,36 @@ RAT_API int rat_recur_prefill_local(const void *k, const void *v, const void *ga
                             int B, int H, int T, int d, int dtype,
                             int64_t pos0, int64_t L, float rope_base,
                             void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * rat_recur_prefill_window -- the fixed-window recurrence of RAT+: each state covers only the
+ * last Lw positions.
+ *   "RAT+ Deep Dive" section 2.1 (a fixed recurrence window L* = 64, looking back 64 tokens
+ *   from the current one, computed in parallel in prefill).  Read as: the state at t is the
+ *   recurrence restarted from zero at t - Lw + 1,
+ *     y_t = sum_{s = t-Lw+1}^{t} ( prod_{r = s+1}^{t} g_r ) (1 - g_s) x_s,   g = sigmoid(a),
+ *   for x = k and x = v with the same gate, in float32; k~ = RoPE(y^k) when rope_base > 0.
+ *
+ *   k, v, gate_logit : device, (B, H, T, d) of dtype          inputs
+ *   prev_k, prev_v, prev_gate_logit
+ *                    : device, (B, H, Lw, d) of dtype, or all three NULL: the Lw positions just
+ *                      before row 0 (oldest first), so that a sequence can be continued; NULL
+ *                      clips the window at row 0
+ *   k_rec, v_rec     : device, (B, H, T, d) of dtype          outputs k~, v~
+ *   pos0             : absolute position of row 0 (RoPE only)
+ *   Lw               : window length; 64 (the pages' L*) is the supported value
+ *                      (RAT_ERR_UNSUPPORTED otherwise, RAT_ERR_INVALID below 1)
+ *   ws, ws_bytes     : workspace of at least 256 bytes, 256-byte aligned (its header receives
+ *                      device-side errors; see rat_sync_status)
+ * There is no initial or final state: the window makes the state a function of the last Lw
+ * inputs.  Outputs may not alias inputs.  T = 0 is a no-op.  No CTA waits for another (the
+ * segmented form is computed block by block), so the call has no look-back.
+ * ---------------------------------------------------------------------------------------- */
+RAT_API int rat_recur_prefill_window(const void *k, const void *v, const void *gate_logit,
+                             const void *prev_k, const void *prev_v, const void *prev_gate_logit,
+                             void *k_rec, void *v_rec, int B, int H, int T, int d, int dtype,
+                             int64_t pos0, int64_t Lw, float rope_base,
+                             void *ws, size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------------------------
  * rat_dilated_attn_prefill -- causal dilated attention with an optional local window and a

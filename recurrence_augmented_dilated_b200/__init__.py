@@ -22,6 +22,7 @@ import torch
 __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_recur_prefill_local",
+    "rat_recur_prefill_window",
     "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
     "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
@@ -75,6 +76,8 @@ def lib():
         L.rat_recur_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.rat_recur_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
+        L.rat_recur_prefill_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                               _i, _i, _i, _i, _i, _i64, _i64, _f, _vp, _sz, _vp]
         L.rat_recur_prefill_local.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                               _i, _i, _i, _i, _i, _i64, _i64, _f, _vp, _sz, _vp]
         L.rat_dilated_attn_prefill.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
@@ -186,6 +189,20 @@ def rat_recur_prefill_local(k, v, gate_logit, k_rec, v_rec, ws: Workspace, L: in
                                        _ptr(hT_v), B, H, T, d, _dtype_code(k), int(pos0), int(L),
                                        float(rope_base), ws.ptr, ws.nbytes, _stream(stream))
     _check("rat_recur_prefill_local", st)
+
+
+def rat_recur_prefill_window(k, v, gate_logit, k_rec, v_rec, ws: Workspace, Lw: int = 64,
+                             prev_k=None, prev_v=None, prev_gate_logit=None, pos0: int = 0,
+                             rope_base: float = 0.0, stream=None):
+    """Fixed-window recurrence: each state restarted Lw positions back; optional (B, H, Lw, d)
+    history rows before row 0."""
+    B, H, T, d = k.shape
+    st = lib().rat_recur_prefill_window(_ptr(k), _ptr(v), _ptr(gate_logit), _ptr(prev_k),
+                                        _ptr(prev_v), _ptr(prev_gate_logit), _ptr(k_rec),
+                                        _ptr(v_rec), B, H, T, d, _dtype_code(k), int(pos0),
+                                        int(Lw), float(rope_base), ws.ptr, ws.nbytes,
+                                        _stream(stream))
+    _check("rat_recur_prefill_window", st)
 
 
 def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,

@@ -46,6 +46,22 @@ struct RecurParams {
     unsigned long long wait_ns; // bound of each look-back wait
     long long reset;            // > 0: state zeroed before every position that is a multiple (chunk-local recurrence)
 };
+// fixed-window recurrence: each state restarted kWindowRows positions back
+constexpr int kWindowRows = 64;
+struct WindowParams {
+    const void *k, *v, *a;
+    const void *pk, *pv, *pa;   // [BH][kWindowRows][d] positions before row 0, or all null
+    void *yk, *yv;
+    int BH, T, d, nblk;         // nblk = ceil(T / kWindowRows)
+    long long pos0;
+    int rope, rope_f32;
+    WsHeader *hdr;
+    float theta_f[64];
+    double theta[64];
+    float step_cos[64], step_sin[64];
+};
+int launch_window(const WindowParams &p, int dtype, void *stream);
+
 int recur_chunk_rows(int d, int dtype);
 size_t recur_workspace_bytes(int BH, int T, int d, int dtype);
 int launch_recur(const RecurParams &p, int dtype, void *stream);

@@ -174,6 +174,47 @@ int rat_recur_prefill(const void *k, const void *v, const void *gate_logit, cons
                          dtype, pos0, 0, rope_base, ws, ws_bytes, stream);
 }
 
+int rat_recur_prefill_window(const void *k, const void *v, const void *gate_logit,
+                             const void *prev_k, const void *prev_v, const void *prev_gate_logit,
+                             void *k_rec, void *v_rec, int B, int H, int T, int d, int dtype,
+                             int64_t pos0, int64_t Lw, float rope_base, void *ws, size_t ws_bytes,
+                             void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || Lw < 1) return RAT_ERR_INVALID;
+    if (!supported_d(d) || Lw != kWindowRows) return RAT_ERR_UNSUPPORTED;
+    if (pos0 < 0 || !std::isfinite(rope_base)) return RAT_ERR_INVALID;
+    const int nprev = (prev_k != nullptr) + (prev_v != nullptr) + (prev_gate_logit != nullptr);
+    if (nprev != 0 && nprev != 3) return RAT_ERR_INVALID;
+    if (T == 0) return RAT_OK;
+    if (!k || !v || !gate_logit || !k_rec || !v_rec) return RAT_ERR_INVALID;
+    if (!aligned16(k) || !aligned16(v) || !aligned16(gate_logit) || !aligned16(k_rec) ||
+        !aligned16(v_rec) || (nprev && (!aligned16(prev_k) || !aligned16(prev_v) ||
+                                        !aligned16(prev_gate_logit))))
+        return RAT_ERR_INVALID;
+    if ((long long)B * H * T > (1ll << 40)) return RAT_ERR_UNSUPPORTED;
+    if (!ws || ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return RAT_ERR_WORKSPACE;
+    WindowParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k; p.v = v; p.a = gate_logit;
+    p.pk = prev_k; p.pv = prev_v; p.pa = prev_gate_logit;
+    p.yk = k_rec; p.yv = v_rec;
+    p.BH = B * H; p.T = T; p.d = d;
+    p.nblk = (T + kWindowRows - 1) / kWindowRows;
+    p.pos0 = pos0;
+    p.rope = rope_base > 0.f ? 1 : 0;
+    p.hdr = static_cast<WsHeader *>(ws);
+    if (p.rope) {
+        rope_theta(rope_base, d, p.theta);
+        for (int c = 0; c < 64; ++c) {
+            p.theta_f[c] = (float)p.theta[c];
+            p.step_cos[c] = (float)std::cos(p.theta[c]);
+            p.step_sin[c] = (float)std::sin(p.theta[c]);
+        }
+        p.rope_f32 = (dtype == RAT_BF16 && pos0 + (int64_t)T <= 8192) ? 1 : 0;
+    }
+    return launch_window(p, dtype, stream);
+}
+
 int rat_recur_prefill_local(const void *k, const void *v, const void *gate_logit,
                             const float *h0_k, const float *h0_v, void *k_rec, void *v_rec,
                             float *hT_k, float *hT_v, int B, int H, int T, int d, int dtype,

@@ -62,36 +62,6 @@ struct ScanCfg {
     static_assert(R * SEGS == TC && R >= 1, "whole segments per chunk");
 };
 
-// A lane's two channel pairs of one row: pair 0 at channels (2l, 2l+1), pair 1 at
-// (2l + d/2, 2l+1 + d/2), as float pairs.
-template <typename E> struct Lane;
-template <> struct Lane<float> {
-    template <int HALFB>
-    static RAT_DEVICE void load(const uint8_t *row, int l, f2_t *x) {
-        const uint2 a = *reinterpret_cast<const uint2 *>(row + 8 * l);
-        const uint2 c = *reinterpret_cast<const uint2 *>(row + HALFB + 8 * l);
-        x[0] = f2(__uint_as_float(a.x), __uint_as_float(a.y));
-        x[1] = f2(__uint_as_float(c.x), __uint_as_float(c.y));
-    }
-    template <int HALFB>
-    static RAT_DEVICE void store(uint8_t *row, int l, const f2_t *x) {
-        *reinterpret_cast<uint2 *>(row + 8 * l) = make_uint2(__float_as_uint(f2lo(x[0])), __float_as_uint(f2hi(x[0])));
-        *reinterpret_cast<uint2 *>(row + HALFB + 8 * l) = make_uint2(__float_as_uint(f2lo(x[1])), __float_as_uint(f2hi(x[1])));
-    }
-};
-template <> struct Lane<__nv_bfloat16> {
-    template <int HALFB>
-    static RAT_DEVICE void load(const uint8_t *row, int l, f2_t *x) {
-        x[0] = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(row + 4 * l));
-        x[1] = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(row + HALFB + 4 * l));
-    }
-    template <int HALFB>
-    static RAT_DEVICE void store(uint8_t *row, int l, const f2_t *x) {
-        *reinterpret_cast<uint32_t *>(row + 4 * l) = f2_to_bf16x2(x[0]);
-        *reinterpret_cast<uint32_t *>(row + HALFB + 4 * l) = f2_to_bf16x2(x[1]);
-    }
-};
-
 // Look-back records: each value is one 64-bit word, (tag << 32) | float bits, written with a
 // single relaxed store; a reader accepts a word only when its tag is this launch's tag, so a
 // value and its validity always travel together.

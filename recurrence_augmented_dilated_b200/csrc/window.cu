@@ -1,0 +1,363 @@
+// window.cu -- fixed-window forget-gate recurrence over keys and values (prefill).
+//
+// "RAT+ Deep Dive", section 2.1: RAT+ gives every token a recurrence window of a fixed L* = 64
+// tokens, whatever the dilation.  Read as: the state at t is the recurrence h <- g h + (1-g) x
+// (g = sigmoid(logit), per channel, x = k and x = v) restarted from zero at t - Lw + 1,
+//     y_t = sum_{s = t-Lw+1}^{t} (prod_{r = s+1}^{t} g_r) (1 - g_s) x_s,     Lw = 64.
+//
+// Segmented form, no subtraction of an older state.  Cut the rows into blocks of Lw aligned at
+// row 0.  For t = c Lw + j (row j of block c) the window is the tail of block c-1 from its row
+// j + 1 followed by the head of block c up to t, so
+//     y_t = F_c(t) + P_c(t) U_{c-1}(j + 1),
+//   F_c(t)   : the recurrence from zero at the first row of block c, at t;
+//   P_c(t)   : the product of block c's gates up to t;
+//   U_{c}(i) : the recurrence from zero at row i of block c, at the block's last row
+//              (U_c(Lw) = 0): a suffix quantity, formed by a backward pass over block c after
+//              its forward pass and kept in registers for block c + 1.
+// No CTA waits for another: the flattened (b, h, block) sequence is cut into one contiguous
+// range per CTA, walked in order; the block before a range (or the history rows before row 0)
+// is read once more to form its U.
+//
+// Lane layout as in the full-sequence scan: lane l holds the channel pairs (2l, 2l+1) and
+// (2l + d/2, 2l+1 + d/2), the rotate-half RoPE partners.  The 512 threads of a CTA cover one
+// block: d/4 lanes per row and 512/(d/4) segments of R consecutive rows (R = 4 for d = 128,
+// 2 for d = 64).  A segment's aggregate (A = prod g, B = sum ...) goes to shared memory; one
+// thread per channel forms the exclusive prefix (for F, P) and suffix (for U) over the
+// segments.  Blocks stream through a ring of shared-memory stages filled by bulk copies
+// (cp.async.bulk) two blocks ahead.  HBM traffic: 3 reads + 2 writes per element, plus one
+// extra block per range.
+#include "common.cuh"
+
+namespace rat {
+
+namespace {
+
+template <typename E, int DH>
+struct WinCfg {
+    static constexpr int EB = sizeof(E);
+    static constexpr int LW = kWindowRows;              // window = block rows
+    static constexpr int THREADS = 512;
+    static constexpr int LPR = DH / 4;                  // lanes per row
+    static constexpr int SEGS = THREADS / LPR;          // row segments per block
+    static constexpr int R = LW / SEGS;                 // rows per segment
+    static constexpr int ROWB = DH * EB;
+    static constexpr int HALFB = ROWB / 2;
+    static constexpr int TILEB = LW * ROWB;             // one tensor of one block
+    static constexpr int STAGEB = 3 * TILEB;            // a, k, v
+    static constexpr int XB = SEGS * 3 * DH * 4;        // one [SEGS][3][DH] float table
+    static constexpr int FIT = (200 * 1024 - 2 * XB) / STAGEB;
+    static constexpr int NST = FIT >= 3 ? 3 : (FIT >= 1 ? FIT : 1);   // stages in the ring
+    static constexpr int SMEM = NST * STAGEB + 2 * XB;
+    static_assert(R * SEGS == LW && R >= 1, "whole segments per block");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+// The items a CTA walks: for each block of its range, first (when needed) the block before it
+// -- only to form U -- then the block itself.  Producer and consumers each step through the
+// same sequence with their own cursor.
+struct Cursor {
+    long long f;          // next flattened block index
+    bool prep_done;       // the extra block before f has been returned
+};
+struct Item {
+    int bh, c;            // c = -1: the history rows before row 0
+    bool prep;            // true: only U is formed
+};
+
+RAT_DEVICE bool next_item(Cursor &cur, long long f0, long long f1, int nblk, bool has_prev,
+                          Item &it) {
+    if (cur.f >= f1) return false;
+    it.bh = (int)(cur.f / nblk);
+    const int c = (int)(cur.f % nblk);
+    const bool need = (cur.f == f0 && c > 0) || (c == 0 && has_prev);
+    if (need && !cur.prep_done) {
+        it.c = c - 1;
+        it.prep = true;
+        cur.prep_done = true;
+        return true;
+    }
+    it.c = c;
+    it.prep = false;
+    cur.prep_done = false;
+    ++cur.f;
+    return true;
+}
+
+}  // namespace
+
+template <typename E, int DH>
+__global__ void __launch_bounds__(WinCfg<E, DH>::THREADS, 1)
+window_kernel(const __grid_constant__ WindowParams p) {
+    using C = WinCfg<E, DH>;
+    constexpr int LPR = C::LPR, R = C::R, HALF = DH / 2, NP = 2;
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t bar[C::NST];
+    __shared__ float s_theta_f[HALF], s_step_c[HALF], s_step_s[HALF];
+    __shared__ double s_theta[HALF];
+
+    const int tid = threadIdx.x;
+    const int seg = tid / LPR, cl = tid % LPR;
+    const int chq[NP] = {2 * cl, 2 * cl + HALF};                // first channel of each pair
+    float *X = reinterpret_cast<float *>(smem + C::NST * C::STAGEB);   // [SEGS][3][DH]
+    float *S = X + C::SEGS * 3 * DH;                                  // [SEGS][3][DH]
+    const long long total = (long long)p.BH * p.nblk;
+    const long long f0 = total * blockIdx.x / gridDim.x;
+    const long long f1 = total * (blockIdx.x + 1) / gridDim.x;
+    const bool has_prev = p.pk != nullptr;
+    const f2_t kOne2 = f2(1.f, 1.f), kZero2 = f2(0.f, 0.f), kNegOne2 = f2(-1.f, -1.f);
+
+    // three bulk copies (a, k, v) of one item into stage st (thread 0)
+    auto load_item = [&](const Item &it, int st) {
+        const uint8_t *ga, *gk, *gv;
+        int rows;
+        if (it.c < 0) {
+            const size_t o = (size_t)it.bh * C::LW * C::ROWB;
+            ga = static_cast<const uint8_t *>(p.pa) + o;
+            gk = static_cast<const uint8_t *>(p.pk) + o;
+            gv = static_cast<const uint8_t *>(p.pv) + o;
+            rows = C::LW;
+        } else {
+            rows = min(C::LW, p.T - it.c * C::LW);
+            const size_t o = ((size_t)it.bh * p.T + (size_t)it.c * C::LW) * C::ROWB;
+            ga = static_cast<const uint8_t *>(p.a) + o;
+            gk = static_cast<const uint8_t *>(p.k) + o;
+            gv = static_cast<const uint8_t *>(p.v) + o;
+        }
+        const uint32_t bytes = (uint32_t)rows * C::ROWB;
+        uint8_t *s = smem + st * C::STAGEB;
+        mbar_arrive_expect_tx(&bar[st], 3 * bytes);
+        bulk_g2s(s, ga, bytes, &bar[st]);
+        bulk_g2s(s + C::TILEB, gk, bytes, &bar[st]);
+        bulk_g2s(s + 2 * C::TILEB, gv, bytes, &bar[st]);
+    };
+
+    if (tid < HALF) {
+        s_theta_f[tid] = p.theta_f[tid];
+        s_theta[tid] = p.theta[tid];
+        s_step_c[tid] = p.step_cos[tid];
+        s_step_s[tid] = p.step_sin[tid];
+    }
+    if (tid == 0) {
+        for (int s = 0; s < C::NST; ++s) mbar_init(&bar[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    Cursor pc{f0, false};                 // producer cursor, NST - 1 items ahead (thread 0)
+    if (tid == 0) {
+        for (int s = 0; s < C::NST - 1; ++s) {
+            Item nx;
+            if (!next_item(pc, f0, f1, p.nblk, has_prev, nx)) break;
+            load_item(nx, s);
+        }
+    }
+
+    f2_t Uk[R][NP], Uv[R][NP];            // U of the block before the current one, my rows
+    int u_bh = -1, u_c = -2;              // the block those U belong to
+    bool dead = false;                    // a copy never arrived: skip the rest (error recorded)
+    Cursor cc{f0, false};
+    Item it;
+    for (int k = 0; next_item(cc, f0, f1, p.nblk, has_prev, it); ++k) {
+        const int st = k % C::NST;
+        if (tid == 0 && !dead) {          // refill the stage the previous item released
+            Item nx;
+            if (next_item(pc, f0, f1, p.nblk, has_prev, nx)) load_item(nx, (k + C::NST - 1) % C::NST);
+        }
+        if (!dead && !mbar_wait_bounded(&bar[st], (uint32_t)(k / C::NST) & 1u, p.hdr, 0x300u))
+            dead = true;
+        const int rows = it.c < 0 ? C::LW : min(C::LW, p.T - it.c * C::LW);
+        const uint8_t *sa = smem + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
+
+        // ---- forward pass over my R rows: gates (kept) and the segment aggregate from zero
+        f2_t G[R][NP];
+        f2_t A[NP] = {kOne2, kOne2}, Bk[NP] = {kZero2, kZero2}, Bv[NP] = {kZero2, kZero2};
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int r = seg * R + i;
+            const int off = (r < rows ? r : rows - 1) * C::ROWB;
+            f2_t xa[NP], xk[NP], xv[NP];
+            Lane<E>::template load<C::HALFB>(sa + off, cl, xa);
+            Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
+            Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                G[i][q] = r < rows ? forget_gate2(xa[q]) : kOne2;     // past the end: identity
+                const f2_t og = gate_complement2(G[i][q]);
+                A[q] = f2_mul(A[q], G[i][q]);
+                Bk[q] = f2_fma(G[i][q], Bk[q], f2_mul(og, xk[q]));
+                Bv[q] = f2_fma(G[i][q], Bv[q], f2_mul(og, xv[q]));
+            }
+        }
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            float *x = X + seg * 3 * DH + chq[q];
+            x[0] = f2lo(A[q]);           x[1] = f2hi(A[q]);
+            x[DH] = f2lo(Bk[q]);         x[DH + 1] = f2hi(Bk[q]);
+            x[2 * DH] = f2lo(Bv[q]);     x[2 * DH + 1] = f2hi(Bv[q]);
+        }
+        __syncthreads();
+
+        // ---- one thread per channel: exclusive suffix (segments after s) into S, exclusive
+        // prefix (segments before s) over X in place
+        if (tid < DH) {
+            const int ch = tid;
+            float sA = 1.f, sK = 0.f, sV = 0.f;
+#pragma unroll 4
+            for (int s = C::SEGS - 1; s >= 0; --s) {
+                float *o = S + s * 3 * DH + ch;
+                const float *x = X + s * 3 * DH + ch;
+                o[0] = sA;
+                o[DH] = sK;
+                o[2 * DH] = sV;
+                sK = fmaf(sA, x[DH], sK);
+                sV = fmaf(sA, x[2 * DH], sV);
+                sA *= x[0];
+            }
+            if (!it.prep) {
+                float pA = 1.f, pK = 0.f, pV = 0.f;
+#pragma unroll 4
+                for (int s = 0; s < C::SEGS; ++s) {
+                    float *x = X + s * 3 * DH + ch;
+                    const float a = x[0], bk = x[DH], bv = x[2 * DH];
+                    x[0] = pA;
+                    x[DH] = pK;
+                    x[2 * DH] = pV;
+                    pK = fmaf(a, pK, bk);
+                    pV = fmaf(a, pV, bv);
+                    pA *= a;
+                }
+            }
+        }
+        __syncthreads();
+
+        // ---- outputs y_t = F(t) + P(t) U(j + 1) of my rows, k~ rotated
+        if (!it.prep) {
+            const bool useU = u_bh == it.bh && u_c == it.c - 1;
+            f2_t Fk[NP], Fv[NP], Pp[NP];
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const float *x = X + seg * 3 * DH + chq[q];
+                Pp[q] = f2(x[0], x[1]);
+                Fk[q] = f2(x[DH], x[DH + 1]);
+                Fv[q] = f2(x[2 * DH], x[2 * DH + 1]);
+            }
+            f2_t rc = kOne2, rs = kZero2, sc = kOne2, ss = kZero2, nss = kZero2;
+            if (p.rope) {
+                const long long pos = p.pos0 + (long long)it.c * C::LW + seg * R;
+                float c2[2], s2[2];
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int f = 2 * cl + u;
+                    if (p.rope_f32) rope_cs_f32((int)pos, s_theta_f[f], c2[u], s2[u]);
+                    else rope_cs(pos, s_theta[f], c2[u], s2[u]);
+                }
+                rc = f2(c2[0], c2[1]);
+                rs = f2(s2[0], s2[1]);
+                sc = f2(s_step_c[2 * cl], s_step_c[2 * cl + 1]);
+                ss = f2(s_step_s[2 * cl], s_step_s[2 * cl + 1]);
+                nss = f2(-s_step_s[2 * cl], -s_step_s[2 * cl + 1]);
+            }
+            uint8_t *yk = static_cast<uint8_t *>(p.yk);
+            uint8_t *yv = static_cast<uint8_t *>(p.yv);
+            const size_t row0 = (size_t)it.bh * p.T + (size_t)it.c * C::LW;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const int r = seg * R + i;
+                const int off = (r < rows ? r : rows - 1) * C::ROWB;
+                f2_t xk[NP], xv[NP], hk[NP], hv[NP];
+                Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
+                Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
+#pragma unroll
+                for (int q = 0; q < NP; ++q) {
+                    const f2_t og = gate_complement2(G[i][q]);
+                    Fk[q] = f2_fma(G[i][q], Fk[q], f2_mul(og, xk[q]));
+                    Fv[q] = f2_fma(G[i][q], Fv[q], f2_mul(og, xv[q]));
+                    Pp[q] = f2_mul(Pp[q], G[i][q]);
+                    hk[q] = useU ? f2_fma(Pp[q], Uk[i][q], Fk[q]) : Fk[q];
+                    hv[q] = useU ? f2_fma(Pp[q], Uv[i][q], Fv[q]) : Fv[q];
+                }
+                f2_t ok[NP] = {hk[0], hk[1]};
+                if (p.rope) {
+                    const f2_t nrs = f2_mul(rs, kNegOne2);
+                    ok[0] = f2_fma(hk[1], nrs, f2_mul(hk[0], rc));
+                    ok[1] = f2_fma(hk[0], rs, f2_mul(hk[1], rc));
+                    const f2_t nc = f2_fma(rc, sc, f2_mul(rs, nss));     // advance one position
+                    rs = f2_fma(rs, sc, f2_mul(rc, ss));
+                    rc = nc;
+                }
+                if (r < rows && !dead) {
+                    const size_t go = (row0 + r) * C::ROWB;
+                    Lane<E>::template store<C::HALFB>(yk + go, cl, ok);
+                    Lane<E>::template store<C::HALFB>(yv + go, cl, hv);
+                }
+            }
+        }
+
+        // ---- U of this block for the next one (a full block: only the last may be partial):
+        // U(seg R + i + 1) = As * W(i + 1) + Bs, W(j) = the recurrence from zero at my row j to
+        // my last row, (As, Bs) = the segments after mine
+        if (it.c + 1 < p.nblk) {
+            f2_t sA[NP], sK[NP], sV[NP];
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const float *o = S + seg * 3 * DH + chq[q];
+                sA[q] = f2(o[0], o[1]);
+                sK[q] = f2(o[DH], o[DH + 1]);
+                sV[q] = f2(o[2 * DH], o[2 * DH + 1]);
+            }
+            f2_t wk[NP] = {kZero2, kZero2}, wv[NP] = {kZero2, kZero2}, pr[NP] = {kOne2, kOne2};
+#pragma unroll
+            for (int i = R - 1; i >= 0; --i) {
+#pragma unroll
+                for (int q = 0; q < NP; ++q) {
+                    Uk[i][q] = f2_fma(sA[q], wk[q], sK[q]);
+                    Uv[i][q] = f2_fma(sA[q], wv[q], sV[q]);
+                }
+                if (i > 0) {
+                    const int off = (seg * R + i) * C::ROWB;
+                    f2_t xk[NP], xv[NP];
+                    Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
+                    Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const f2_t og = gate_complement2(G[i][q]);
+                        wk[q] = f2_fma(pr[q], f2_mul(og, xk[q]), wk[q]);
+                        wv[q] = f2_fma(pr[q], f2_mul(og, xv[q]), wv[q]);
+                        pr[q] = f2_mul(pr[q], G[i][q]);
+                    }
+                }
+            }
+            u_bh = it.bh;
+            u_c = it.c;
+        }
+        __syncthreads();        // the stage and the X / S tables are free for the next item
+    }
+}
+
+template <typename E, int DH>
+static int launch_one(const WindowParams &p, void *stream) {
+    using C = WinCfg<E, DH>;
+    auto kern = window_kernel<E, DH>;
+    static uint64_t attr_done = 0;
+    const int st = set_smem_attr(reinterpret_cast<const void *>(kern), C::SMEM, &attr_done);
+    if (st != RAT_OK) return st;
+    const int sms = current_sm_count();
+    if (sms <= 0) return RAT_ERR_CUDA;
+    // one CTA per SM, each a contiguous range of blocks (ranges differ by at most one block)
+    const long long total = (long long)p.BH * p.nblk;
+    const unsigned grid = (unsigned)(total < sms ? total : sms);
+    kern<<<grid, C::THREADS, C::SMEM, static_cast<cudaStream_t>(stream)>>>(p);
+    return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
+}
+
+int launch_window(const WindowParams &p, int dtype, void *stream) {
+    if (dtype == RAT_F32) {
+        if (p.d == 64) return launch_one<float, 64>(p, stream);
+        if (p.d == 128) return launch_one<float, 128>(p, stream);
+    } else {
+        if (p.d == 64) return launch_one<__nv_bfloat16, 64>(p, stream);
+        if (p.d == 128) return launch_one<__nv_bfloat16, 128>(p, stream);
+    }
+    return RAT_ERR_UNSUPPORTED;
+}
+
+}  // namespace rat

@@ -79,6 +79,33 @@ def test_recur_validation(L):
                                1, 1, 0, 128, 1, 0, 0.0, None, 0, None) == 0
 
 
+def test_local_and_window_validation(L):
+    P = ctypes.c_void_p
+    ws = P(4096 * 256)
+    need = rat.rat_recur_workspace_bytes(1, 1, 8, 128, 1)
+    # chunk-local: the block length must be at least 1
+    assert L.rat_recur_prefill_local(P(256), P(256), P(256), None, None, P(256), P(256), None,
+                                     None, 1, 1, 8, 128, 1, 0, 0, 0.0, ws, need, None) == -1
+    assert L.rat_recur_prefill_local(P(256), P(256), P(256), None, None, P(256), P(256), None,
+                                     None, 1, 1, 8, 128, 1, 0, -3, 0.0, ws, need, None) == -1
+    assert L.rat_recur_prefill_local(None, None, None, None, None, None, None, None, None,
+                                     1, 1, 0, 128, 1, 0, 16, 0.0, None, 0, None) == 0
+    args = lambda Lw, prev=(None, None, None), ws_=ws, wsb=256, T=8: (
+        P(256), P(256), P(256), *prev, P(256), P(256), 1, 1, T, 128, 1, 0, Lw, 0.0, ws_, wsb, None)
+    # window: below 1 invalid, other lengths than 64 unsupported
+    assert L.rat_recur_prefill_window(*args(0)) == -1
+    assert L.rat_recur_prefill_window(*args(32)) == -2
+    # history rows: all three or none
+    assert L.rat_recur_prefill_window(*args(64, prev=(P(256), None, None))) == -1
+    assert L.rat_recur_prefill_window(*args(64, prev=(P(256), P(256), P(258)))) == -1
+    # workspace header missing, too small or misaligned
+    assert L.rat_recur_prefill_window(*args(64, ws_=None)) == -5
+    assert L.rat_recur_prefill_window(*args(64, wsb=255)) == -5
+    assert L.rat_recur_prefill_window(*args(64, ws_=P(4096 * 256 + 16))) == -5
+    # T == 0 is a no-op
+    assert L.rat_recur_prefill_window(*args(64, T=0)) == 0
+
+
 def test_recur_workspace_grows_with_chunks(L):
     a = rat.rat_recur_workspace_bytes(1, 1, 128, 128, 1)
     b = rat.rat_recur_workspace_bytes(1, 1, 129, 128, 1)
@@ -149,6 +176,15 @@ def test_compress_and_decode_validation(L):
     c32.k_dil = c32.v_dil = c32.k_win = c32.v_win = c32.h_k = c32.h_v = 256
     assert L.rat_dilated_decode(P(256), P(256), P(256), P(256), ctypes.byref(c32), P(256), 0.0, 0.0,
                                 ws, 1 << 30, None) == -2
+
+
+def test_cache_rejects_negative_block_length(L):
+    c = cache()
+    c.reset_every = -1
+    sz = ctypes.c_size_t()
+    assert L.rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(sz), None, None) == -1
+    c.reset_every = 16
+    assert L.rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(sz), None, None) == 0
 
 
 def test_workspace_init_rejects_null(L):

@@ -192,3 +192,85 @@ def test_local_recurrence_full_size_sampled_heads():
     x = synthetic.prefill_inputs(w)
     heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)]
     check(x["k"], x["v"], x["a"], rope_base=w.rope_base, heads=heads, reset_every=16)
+
+
+# ---- fixed-window recurrence (each state covers the last 64 positions)
+def gpu_window(k, v, a, prev=None, pos0=0, rope_base=0.0):
+    dev = torch.device("cuda")
+    k, v, a = (x.to(dev) for x in (k, v, a))
+    kr, vr = torch.empty_like(k), torch.empty_like(v)
+    ws = rat.Workspace(256)
+    pk = pv = pa = None
+    if prev is not None:
+        pk, pv, pa = (x.to(dev) for x in prev)
+    rat.rat_recur_prefill_window(k, v, a, kr, vr, ws, 64, prev_k=pk, prev_v=pv,
+                                 prev_gate_logit=pa, pos0=pos0, rope_base=rope_base)
+    st = rat.rat_sync_status(ws)
+    assert st == 0, rat.rat_status_string(st)
+    return kr, vr
+
+
+def check_window(k, v, a, prev=None, pos0=0, rope_base=0.0, heads=None):
+    kr, vr = gpu_window(k, v, a, prev=prev, pos0=pos0, rope_base=rope_base)
+    sel = heads if heads is not None else [(b, h) for b in range(k.shape[0]) for h in range(k.shape[1])]
+    bi = [b for b, _ in sel]
+    hi = [h for _, h in sel]
+    px = pv = pa = None
+    if prev is not None:
+        px, pv, pa = (f64(x[bi, hi]) for x in prev)
+    oa = f64(a[bi, hi])
+    yk = oracle.recurrence_window(f64(k[bi, hi]), oa, 64, prev_x=px, prev_a=pa)
+    yv = oracle.recurrence_window(f64(v[bi, hi]), oa, 64, prev_x=pv, prev_a=pa)
+    if rope_base > 0:
+        yk = oracle.rope(yk, pos0, rope_base)
+    tol = tol_for(k.dtype)
+    errs = dict(k=rel_err(kr[bi, hi], yk), v=rel_err(vr[bi, hi], yv))
+    assert errs["k"] <= tol and errs["v"] <= tol, errs
+    return errs
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 1000, 2049])
+def test_window_recurrence(dtype, d, T):
+    # B 2 x H 4 x 33 blocks at T = 2049 is more blocks than SMs: CTA ranges span several blocks
+    # and cross (b, h) boundaries
+    x = inputs(2, 4, T, d, dtype, seed=T + 3 * d)
+    check_window(x["k"], x["v"], x["a"])
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_window_history_rows_and_rope(dtype):
+    x = inputs(2, 3, 777, 128, dtype, seed=17)
+    p = inputs(2, 3, 64, 128, dtype, seed=18)
+    prev = (p["k"], p["v"], p["a"])
+    check_window(x["k"], x["v"], x["a"], prev=prev, pos0=5000, rope_base=10000.0)
+
+
+def test_window_continues_a_sequence():
+    # two calls, the second given the last 64 rows of the first as history, equal one call
+    x = inputs(1, 2, 640, 128, torch.float32, seed=23)
+    k, v, a = (t.cuda() for t in (x["k"], x["v"], x["a"]))
+    kr, vr = gpu_window(k, v, a)
+    cut = 320
+    kr1, vr1 = gpu_window(*(t[:, :, :cut].contiguous() for t in (k, v, a)))
+    prev = tuple(t[:, :, cut - 64:cut].contiguous() for t in (k, v, a))
+    kr2, vr2 = gpu_window(*(t[:, :, cut:].contiguous() for t in (k, v, a)), prev=prev)
+    assert rel_err(torch.cat([kr1, kr2], 2), kr) <= 1e-5
+    assert rel_err(torch.cat([vr1, vr2], 2), vr) <= 1e-5
+
+
+def test_window_short_sequence_is_the_full_recurrence():
+    # T <= 64 without history: no position ever leaves the window
+    x = inputs(2, 2, 64, 128, torch.float32, seed=29)
+    kr, vr = gpu_window(x["k"], x["v"], x["a"])
+    kf, vf, _, _ = gpu_recur(x["k"], x["v"], x["a"])
+    assert rel_err(kr, kf) <= 1e-5 and rel_err(vr, vf) <= 1e-5
+
+
+def test_window_full_size_sampled_heads():
+    # the prefill_1p5b workload (B 4, H 16, T 4096, d 128, bf16, RoPE)
+    w = synthetic.WORKLOADS["prefill_1p5b"]
+    x = synthetic.prefill_inputs(w)
+    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2), (1, 7)]
+    check_window(x["k"], x["v"], x["a"], rope_base=w.rope_base, heads=heads)
