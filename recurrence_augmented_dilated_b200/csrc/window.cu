@@ -5,15 +5,21 @@
 // (g = sigmoid(logit), per channel, x = k and x = v) restarted from zero at t - Lw + 1,
 //     y_t = sum_{s = t-Lw+1}^{t} (prod_{r = s+1}^{t} g_r) (1 - g_s) x_s,     Lw = 64.
 //
-// Segmented form, no subtraction of an older state.  Cut the rows into blocks of Lw aligned at
-// row 0.  For t = c Lw + j (row j of block c) the window is the tail of block c-1 from its row
-// j + 1 followed by the head of block c up to t, so
+// Segmented form.  Cut the rows into blocks of Lw aligned at row 0.  For t = c Lw + j (row j
+// of block c) the window is the tail of block c-1 from its row j + 1 followed by the head of
+// block c up to t, so
 //     y_t = F_c(t) + P_c(t) U_{c-1}(j + 1),
 //   F_c(t)   : the recurrence from zero at the first row of block c, at t;
 //   P_c(t)   : the product of block c's gates up to t;
-//   U_{c}(i) : the recurrence from zero at row i of block c, at the block's last row
-//              (U_c(Lw) = 0): a suffix quantity, formed by a backward pass over block c after
-//              its forward pass and kept in registers for block c + 1.
+//   U_c(i)   : the recurrence from zero at row i of block c, at the block's last row
+//              (U_c(Lw) = 0), kept in registers for block c + 1.  Since the whole block's
+//              recurrence E_c splits at row j into Pa_c(j) F_c(j) + U_c(j + 1), with Pa_c(j) the
+//              product of the gates after row j, U comes out of the same forward pass as
+//              U_c(j + 1) = E_c - Pa_c(j) F_c(j).  Both terms are sums over this block's rows
+//              with weights that sum to at most 1, so the difference is exact to a few units in
+//              the last place of the block's largest input; no state older than one block is
+//              ever subtracted (subtracting the decayed full-sequence state instead would carry
+//              the rounding of the whole history).
 // No CTA waits for another: the flattened (b, h, block) sequence is cut into one contiguous
 // range per CTA, walked in order; the block before a range (or the history rows before row 0)
 // is read once more to form its U.
@@ -21,9 +27,10 @@
 // Lane layout as in the full-sequence scan: lane l holds the channel pairs (2l, 2l+1) and
 // (2l + d/2, 2l+1 + d/2), the rotate-half RoPE partners.  The 512 threads of a CTA cover one
 // block: d/4 lanes per row and 512/(d/4) segments of R consecutive rows (R = 4 for d = 128,
-// 2 for d = 64).  A segment's aggregate (A = prod g, B = sum ...) goes to shared memory; one
-// thread per channel forms the exclusive prefix (for F, P) and suffix (for U) over the
-// segments.  Blocks stream through a ring of shared-memory stages filled by bulk copies
+// 2 for d = 64).  Per block: a forward pass over each segment's rows forms its aggregate
+// (A = prod g, B = sum ...); one thread per channel combines them through shared memory into
+// each segment's carry (exclusive prefix), the block total and the gate product of the later
+// segments; a second forward pass from the carry writes the outputs and U.  Blocks stream through a ring of shared-memory stages filled by bulk copies
 // (cp.async.bulk) two blocks ahead.  HBM traffic: 3 reads + 2 writes per element, plus one
 // extra block per range.
 #include "common.cuh"
@@ -44,10 +51,12 @@ struct WinCfg {
     static constexpr int HALFB = ROWB / 2;
     static constexpr int TILEB = LW * ROWB;             // one tensor of one block
     static constexpr int STAGEB = 3 * TILEB;            // a, k, v
-    static constexpr int XB = SEGS * 3 * DH * 4;        // one [SEGS][3][DH] float table
-    static constexpr int FIT = (200 * 1024 - 2 * XB) / STAGEB;
+    // [SEGS + 1][3][DH] aggregates -> exclusive prefixes (+ block total), [SEGS][DH] suffix
+    // gate products
+    static constexpr int XB = (SEGS + 1) * 3 * DH * 4 + SEGS * DH * 4;
+    static constexpr int FIT = (200 * 1024 - XB) / STAGEB;
     static constexpr int NST = FIT >= 3 ? 3 : (FIT >= 1 ? FIT : 1);   // stages in the ring
-    static constexpr int SMEM = NST * STAGEB + 2 * XB;
+    static constexpr int SMEM = NST * STAGEB + XB;
     static_assert(R * SEGS == LW && R >= 1, "whole segments per block");
     static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -57,6 +66,7 @@ struct WinCfg {
 // same sequence with their own cursor.
 struct Cursor {
     long long f;          // next flattened block index
+    int bh, c;            // its slice and block
     bool prep_done;       // the extra block before f has been returned
 };
 struct Item {
@@ -64,22 +74,34 @@ struct Item {
     bool prep;            // true: only U is formed
 };
 
+RAT_DEVICE Cursor cursor_at(long long f, int nblk) {
+    Cursor cur;
+    cur.f = f;
+    cur.bh = (int)(f / nblk);
+    cur.c = (int)(f % nblk);
+    cur.prep_done = false;
+    return cur;
+}
+
 RAT_DEVICE bool next_item(Cursor &cur, long long f0, long long f1, int nblk, bool has_prev,
                           Item &it) {
     if (cur.f >= f1) return false;
-    it.bh = (int)(cur.f / nblk);
-    const int c = (int)(cur.f % nblk);
-    const bool need = (cur.f == f0 && c > 0) || (c == 0 && has_prev);
+    it.bh = cur.bh;
+    const bool need = (cur.f == f0 && cur.c > 0) || (cur.c == 0 && has_prev);
     if (need && !cur.prep_done) {
-        it.c = c - 1;
+        it.c = cur.c - 1;
         it.prep = true;
         cur.prep_done = true;
         return true;
     }
-    it.c = c;
+    it.c = cur.c;
     it.prep = false;
     cur.prep_done = false;
     ++cur.f;
+    if (++cur.c == nblk) {
+        cur.c = 0;
+        ++cur.bh;
+    }
     return true;
 }
 
@@ -98,8 +120,8 @@ window_kernel(const __grid_constant__ WindowParams p) {
     const int tid = threadIdx.x;
     const int seg = tid / LPR, cl = tid % LPR;
     const int chq[NP] = {2 * cl, 2 * cl + HALF};                // first channel of each pair
-    float *X = reinterpret_cast<float *>(smem + C::NST * C::STAGEB);   // [SEGS][3][DH]
-    float *S = X + C::SEGS * 3 * DH;                                  // [SEGS][3][DH]
+    float *X = reinterpret_cast<float *>(smem + C::NST * C::STAGEB);   // [SEGS + 1][3][DH]
+    float *S = X + (C::SEGS + 1) * 3 * DH;                            // [SEGS][DH]
     const long long total = (long long)p.BH * p.nblk;
     const long long f0 = total * blockIdx.x / gridDim.x;
     const long long f1 = total * (blockIdx.x + 1) / gridDim.x;
@@ -142,7 +164,7 @@ window_kernel(const __grid_constant__ WindowParams p) {
         fence_mbar_init();
     }
     __syncthreads();
-    Cursor pc{f0, false};                 // producer cursor, NST - 1 items ahead (thread 0)
+    Cursor pc = cursor_at(f0, p.nblk);    // producer cursor, NST - 1 items ahead (thread 0)
     if (tid == 0) {
         for (int s = 0; s < C::NST - 1; ++s) {
             Item nx;
@@ -154,7 +176,7 @@ window_kernel(const __grid_constant__ WindowParams p) {
     f2_t Uk[R][NP], Uv[R][NP];            // U of the block before the current one, my rows
     int u_bh = -1, u_c = -2;              // the block those U belong to
     bool dead = false;                    // a copy never arrived: skip the rest (error recorded)
-    Cursor cc{f0, false};
+    Cursor cc = cursor_at(f0, p.nblk);
     Item it;
     for (int k = 0; next_item(cc, f0, f1, p.nblk, has_prev, it); ++k) {
         const int st = k % C::NST;
@@ -196,85 +218,118 @@ window_kernel(const __grid_constant__ WindowParams p) {
         }
         __syncthreads();
 
-        // ---- one thread per channel: exclusive suffix (segments after s) into S, exclusive
-        // prefix (segments before s) over X in place
+        // ---- one thread per channel: product of the gates of the segments after s into S,
+        // exclusive prefixes (segments before s) over X in place, the block total in X[SEGS]
         if (tid < DH) {
             const int ch = tid;
-            float sA = 1.f, sK = 0.f, sV = 0.f;
-#pragma unroll 4
-            for (int s = C::SEGS - 1; s >= 0; --s) {
-                float *o = S + s * 3 * DH + ch;
-                const float *x = X + s * 3 * DH + ch;
-                o[0] = sA;
-                o[DH] = sK;
-                o[2 * DH] = sV;
-                sK = fmaf(sA, x[DH], sK);
-                sV = fmaf(sA, x[2 * DH], sV);
-                sA *= x[0];
+            constexpr int GS = DH == 128 ? 8 : 4;      // segments loaded ahead of the chain
+            float sA = 1.f;
+#pragma unroll 1
+            for (int g0 = C::SEGS - GS; g0 >= 0; g0 -= GS) {
+                float xa[GS];
+#pragma unroll
+                for (int u = 0; u < GS; ++u) xa[u] = X[(g0 + u) * 3 * DH + ch];
+#pragma unroll
+                for (int u = GS - 1; u >= 0; --u) {
+                    S[(g0 + u) * DH + ch] = sA;
+                    sA *= xa[u];
+                }
             }
-            if (!it.prep) {
-                float pA = 1.f, pK = 0.f, pV = 0.f;
-#pragma unroll 4
-                for (int s = 0; s < C::SEGS; ++s) {
-                    float *x = X + s * 3 * DH + ch;
-                    const float a = x[0], bk = x[DH], bv = x[2 * DH];
+            float pA = 1.f, pK = 0.f, pV = 0.f;
+#pragma unroll 1
+            for (int g0 = 0; g0 < C::SEGS; g0 += GS) {
+                float xa[GS], xk[GS], xv[GS];
+#pragma unroll
+                for (int u = 0; u < GS; ++u) {
+                    const float *x = X + (g0 + u) * 3 * DH + ch;
+                    xa[u] = x[0];
+                    xk[u] = x[DH];
+                    xv[u] = x[2 * DH];
+                }
+#pragma unroll
+                for (int u = 0; u < GS; ++u) {
+                    float *x = X + (g0 + u) * 3 * DH + ch;
                     x[0] = pA;
                     x[DH] = pK;
                     x[2 * DH] = pV;
-                    pK = fmaf(a, pK, bk);
-                    pV = fmaf(a, pV, bv);
-                    pA *= a;
+                    pK = fmaf(xa[u], pK, xk[u]);
+                    pV = fmaf(xa[u], pV, xv[u]);
+                    pA *= xa[u];
                 }
             }
+            float *x = X + C::SEGS * 3 * DH + ch;
+            x[0] = pA;
+            x[DH] = pK;
+            x[2 * DH] = pV;
         }
         __syncthreads();
 
-        // ---- outputs y_t = F(t) + P(t) U(j + 1) of my rows, k~ rotated
-        if (!it.prep) {
-            const bool useU = u_bh == it.bh && u_c == it.c - 1;
-            f2_t Fk[NP], Fv[NP], Pp[NP];
+        // ---- forward over my rows again from the segment's carry: F and P, the outputs
+        // y = F + P U(j + 1) (k~ rotated), and U of this block for the next one,
+        //     U(j + 1) = E - Pa(j) F(j),
+        // E = the block total, Pa(j) = the product of the block's gates after row j.  E and
+        // Pa F are both sums over this block's rows with weights summing to at most 1, so the
+        // difference is exact to a few units of the block's largest input.
+        const bool needU = it.c + 1 < p.nblk;           // a next block of this slice exists
+        if (!it.prep && !(u_bh == it.bh && u_c == it.c - 1)) {
+#pragma unroll
+            for (int i = 0; i < R; ++i)
+#pragma unroll
+                for (int q = 0; q < NP; ++q) { Uk[i][q] = kZero2; Uv[i][q] = kZero2; }
+        }
+        f2_t Fk[NP], Fv[NP], Pp[NP], Ek[NP], Ev[NP], npa[R][NP];
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            const float *x = X + seg * 3 * DH + chq[q];
+            Pp[q] = f2(x[0], x[1]);
+            Fk[q] = f2(x[DH], x[DH + 1]);
+            Fv[q] = f2(x[2 * DH], x[2 * DH + 1]);
+            const float *e = X + C::SEGS * 3 * DH + chq[q];
+            Ek[q] = f2(e[DH], e[DH + 1]);
+            Ev[q] = f2(e[2 * DH], e[2 * DH + 1]);
+            const float *o = S + seg * DH + chq[q];
+            npa[R - 1][q] = f2(-o[0], -o[1]);           // minus the gates after my last row
+#pragma unroll
+            for (int i = R - 2; i >= 0; --i) npa[i][q] = f2_mul(npa[i + 1][q], G[i + 1][q]);
+        }
+        f2_t rc = kOne2, rs = kZero2, sc = kOne2, ss = kZero2, nss = kZero2;
+        if (p.rope && !it.prep) {
+            const long long pos = p.pos0 + (long long)it.c * C::LW + seg * R;
+            float c2[2], s2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int f = 2 * cl + u;
+                if (p.rope_f32) rope_cs_f32((int)pos, s_theta_f[f], c2[u], s2[u]);
+                else rope_cs(pos, s_theta[f], c2[u], s2[u]);
+            }
+            rc = f2(c2[0], c2[1]);
+            rs = f2(s2[0], s2[1]);
+            sc = f2(s_step_c[2 * cl], s_step_c[2 * cl + 1]);
+            ss = f2(s_step_s[2 * cl], s_step_s[2 * cl + 1]);
+            nss = f2(-s_step_s[2 * cl], -s_step_s[2 * cl + 1]);
+        }
+        uint8_t *yk = static_cast<uint8_t *>(p.yk);
+        uint8_t *yv = static_cast<uint8_t *>(p.yv);
+        const size_t row0 = (size_t)it.bh * p.T + (size_t)it.c * C::LW;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int r = seg * R + i;
+            const int off = (r < rows ? r : rows - 1) * C::ROWB;
+            f2_t xk[NP], xv[NP], hk[NP], hv[NP];
+            Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
+            Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
-                const float *x = X + seg * 3 * DH + chq[q];
-                Pp[q] = f2(x[0], x[1]);
-                Fk[q] = f2(x[DH], x[DH + 1]);
-                Fv[q] = f2(x[2 * DH], x[2 * DH + 1]);
+                const f2_t og = gate_complement2(G[i][q]);
+                Fk[q] = f2_fma(G[i][q], Fk[q], f2_mul(og, xk[q]));
+                Fv[q] = f2_fma(G[i][q], Fv[q], f2_mul(og, xv[q]));
+                Pp[q] = f2_mul(Pp[q], G[i][q]);
+                hk[q] = f2_fma(Pp[q], Uk[i][q], Fk[q]);
+                hv[q] = f2_fma(Pp[q], Uv[i][q], Fv[q]);
+                Uk[i][q] = f2_fma(npa[i][q], Fk[q], Ek[q]);
+                Uv[i][q] = f2_fma(npa[i][q], Fv[q], Ev[q]);
             }
-            f2_t rc = kOne2, rs = kZero2, sc = kOne2, ss = kZero2, nss = kZero2;
-            if (p.rope) {
-                const long long pos = p.pos0 + (long long)it.c * C::LW + seg * R;
-                float c2[2], s2[2];
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    const int f = 2 * cl + u;
-                    if (p.rope_f32) rope_cs_f32((int)pos, s_theta_f[f], c2[u], s2[u]);
-                    else rope_cs(pos, s_theta[f], c2[u], s2[u]);
-                }
-                rc = f2(c2[0], c2[1]);
-                rs = f2(s2[0], s2[1]);
-                sc = f2(s_step_c[2 * cl], s_step_c[2 * cl + 1]);
-                ss = f2(s_step_s[2 * cl], s_step_s[2 * cl + 1]);
-                nss = f2(-s_step_s[2 * cl], -s_step_s[2 * cl + 1]);
-            }
-            uint8_t *yk = static_cast<uint8_t *>(p.yk);
-            uint8_t *yv = static_cast<uint8_t *>(p.yv);
-            const size_t row0 = (size_t)it.bh * p.T + (size_t)it.c * C::LW;
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-                const int r = seg * R + i;
-                const int off = (r < rows ? r : rows - 1) * C::ROWB;
-                f2_t xk[NP], xv[NP], hk[NP], hv[NP];
-                Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
-                Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
-#pragma unroll
-                for (int q = 0; q < NP; ++q) {
-                    const f2_t og = gate_complement2(G[i][q]);
-                    Fk[q] = f2_fma(G[i][q], Fk[q], f2_mul(og, xk[q]));
-                    Fv[q] = f2_fma(G[i][q], Fv[q], f2_mul(og, xv[q]));
-                    Pp[q] = f2_mul(Pp[q], G[i][q]);
-                    hk[q] = useU ? f2_fma(Pp[q], Uk[i][q], Fk[q]) : Fk[q];
-                    hv[q] = useU ? f2_fma(Pp[q], Uv[i][q], Fv[q]) : Fv[q];
-                }
+            if (!it.prep) {
                 f2_t ok[NP] = {hk[0], hk[1]};
                 if (p.rope) {
                     const f2_t nrs = f2_mul(rs, kNegOne2);
@@ -291,41 +346,7 @@ window_kernel(const __grid_constant__ WindowParams p) {
                 }
             }
         }
-
-        // ---- U of this block for the next one (a full block: only the last may be partial):
-        // U(seg R + i + 1) = As * W(i + 1) + Bs, W(j) = the recurrence from zero at my row j to
-        // my last row, (As, Bs) = the segments after mine
-        if (it.c + 1 < p.nblk) {
-            f2_t sA[NP], sK[NP], sV[NP];
-#pragma unroll
-            for (int q = 0; q < NP; ++q) {
-                const float *o = S + seg * 3 * DH + chq[q];
-                sA[q] = f2(o[0], o[1]);
-                sK[q] = f2(o[DH], o[DH + 1]);
-                sV[q] = f2(o[2 * DH], o[2 * DH + 1]);
-            }
-            f2_t wk[NP] = {kZero2, kZero2}, wv[NP] = {kZero2, kZero2}, pr[NP] = {kOne2, kOne2};
-#pragma unroll
-            for (int i = R - 1; i >= 0; --i) {
-#pragma unroll
-                for (int q = 0; q < NP; ++q) {
-                    Uk[i][q] = f2_fma(sA[q], wk[q], sK[q]);
-                    Uv[i][q] = f2_fma(sA[q], wv[q], sV[q]);
-                }
-                if (i > 0) {
-                    const int off = (seg * R + i) * C::ROWB;
-                    f2_t xk[NP], xv[NP];
-                    Lane<E>::template load<C::HALFB>(sk + off, cl, xk);
-                    Lane<E>::template load<C::HALFB>(sv + off, cl, xv);
-#pragma unroll
-                    for (int q = 0; q < NP; ++q) {
-                        const f2_t og = gate_complement2(G[i][q]);
-                        wk[q] = f2_fma(pr[q], f2_mul(og, xk[q]), wk[q]);
-                        wv[q] = f2_fma(pr[q], f2_mul(og, xv[q]), wv[q]);
-                        pr[q] = f2_mul(pr[q], G[i][q]);
-                    }
-                }
-            }
+        if (needU) {
             u_bh = it.bh;
             u_c = it.c;
         }
