@@ -503,6 +503,109 @@ def run_decode(w: synthetic.Workload, steps_timed: int, warmup: int, rank: int, 
     }
 
 
+def run_decode_paged(w: synthetic.Workload, steps_timed: int, warmup: int, rank: int, world: int,
+                     peaks, peak_kind, page_entries: int = 64):
+    """Ragged decode: the sequences of the batch hold different context lengths
+    (synthetic.ragged_lengths), in a paged compressed cache; every sequence decodes w.steps
+    tokens at its own position.  The steps of a repetition replay as one CUDA graph (positions
+    advance on the device)."""
+    import recurrence_augmented_dilated_b200 as rat
+    dev = torch.device("cuda")
+    B, H, d, W = w.B, w.H, w.d, w.W
+    nsteps = w.steps
+    lengths = synthetic.ragged_lengths(w)
+    Dh = w.heads_D()
+    cap = (max(lengths) + nsteps) // min(Dh) + 1
+    max_pages = (cap + page_entries - 1) // page_entries
+    n_pages = B * H * max_pages
+    g = torch.Generator().manual_seed(w.seed)
+    table = torch.randperm(n_pages, generator=g).to(torch.int32).reshape(B, H, max_pages)
+    cache, bufs = rat.make_paged_cache(B, H, d, W, rat.BF16, Dh, page_entries, n_pages,
+                                       table.contiguous().to(dev))
+    ws_c = rat.Workspace(256)
+    ws_r = rat.Workspace(rat.rat_recur_workspace_bytes(1, H, synthetic.CTX_CHUNK, d, rat.BF16))
+    for b, T in enumerate(lengths):
+        hk = torch.zeros((1, H, d), dtype=torch.float32, device=dev)
+        hv = torch.zeros_like(hk)
+        for c in range((T + synthetic.CTX_CHUNK - 1) // synthetic.CTX_CHUNK):
+            kva = torch.stack([synthetic.decode_context_chunk(w, b, h, c, dev, T) for h in range(H)], 1)
+            k, v, a = (kva[i].unsqueeze(0).contiguous() for i in range(3))
+            kr, vr = torch.empty_like(k), torch.empty_like(v)
+            hk2, hv2 = torch.empty_like(hk), torch.empty_like(hv)
+            pos0 = c * synthetic.CTX_CHUNK
+            rat.rat_recur_prefill(k, v, a, kr, vr, ws_r, h0_k=hk, h0_v=hv, hT_k=hk2, hT_v=hv2,
+                                  pos0=pos0, rope_base=w.rope_base)
+            rat.rat_paged_kv_compress(kr, vr, hk2, hv2, b, pos0, cache, ws_c)
+            hk, hv = hk2, hv2
+    if rat.rat_sync_status(ws_c) != 0:
+        raise RuntimeError("paged compress reported an error")
+    del ws_r
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    tok = synthetic.decode_steps(w)
+    tq, tk, tv, ta = (tok[n].to(dev).reshape(nsteps, B, H, 1, d) for n in ("q", "k", "v", "a"))
+    out = torch.empty((nsteps, B, H, 1, d), dtype=torch.bfloat16, device=dev)
+    ws = rat.Workspace(rat.rat_paged_decode_workspace_bytes(cache))
+    snap = {n: bufs[n].clone() for n in ("h_k", "h_v", "k_win", "v_win", "pos")}
+
+    def reset():
+        for n in snap:
+            bufs[n].copy_(snap[n])
+
+    reset()
+    torch.cuda.synchronize()
+    s_cap = torch.cuda.Stream()
+    s_cap.wait_stream(torch.cuda.current_stream())
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s_cap):
+        with torch.cuda.graph(gr, stream=s_cap):
+            for s in range(nsteps):
+                rat.rat_dilated_decode_paged(tq[s], tk[s], tv[s], ta[s], cache, out[s], ws,
+                                             rope_base=w.rope_base)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        reset()
+        gr.replay()
+    torch.cuda.synchronize()
+    st = rat.rat_sync_status(ws)
+    if st != 0:
+        raise RuntimeError("paged decode device error " + rat.rat_status_string(st))
+    if bufs["pos"].cpu().tolist() != [T + nsteps for T in lengths]:
+        raise RuntimeError("paged decode positions did not advance")
+    times = []
+    barrier(world)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(steps_timed):
+            reset()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            gr.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+    ms_total = max_over_ranks(sum(times) / len(times), world)
+    ms_step = ms_total / nsteps
+    rows = 0
+    for T in lengths:
+        for D in Dh:
+            for s in range(nsteps):
+                rows += rat.rat_attended_keys(T + s, D, W) - 1
+    step_bytes = 2 * (rows / nsteps) * d * 2
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9
+    return {
+        "workload": w.name + "_ragged_paged", "metric": "decode tokens/s", "unit": "tokens/s",
+        "value": world * B * nsteps / (ms_total / 1e3), "ms_per_token_step": ms_step,
+        "context_lengths": [min(lengths), max(lengths)], "page_entries": page_entries,
+        "steps_per_repetition": nsteps, "repetitions": steps_timed, "cuda_graph": True,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "of": peak_kind,
+                     "traffic": recorded_traffic("decode.cu", w.name + "_ragged_paged")},
+        "clocks": clk.summary(),
+        "gpu_launches": nsteps * steps_timed,
+    }
+
+
 # ----------------------------------------------------------------------------- oracle (CPU)
 def oracle_sample(w: synthetic.Workload, budget_s: float = 12.0):
     """Time the float64 oracle on whole (b, h) slices of w (recurrence + RoPE + attention over
@@ -574,6 +677,8 @@ def main():
     ap.add_argument("--reset-every", type=int, default=0,
                     help="L > 0: the chunk-local recurrence (restart every L positions) in the "
                          "prefill step instead of the full-sequence one")
+    ap.add_argument("--decode-paged", action="store_true",
+                    help="also time ragged decode (context lengths T/2 .. T) on a paged cache")
     ap.add_argument("--window", type=int, default=0,
                     help="Lw > 0: the fixed-window recurrence (each state over the last Lw "
                          "positions) in the prefill step")
@@ -656,6 +761,10 @@ def main():
     if not args.no_decode:
         dw = synthetic.WORKLOADS["decode_7p6b"]
         line["decode"] = run_decode(dw, max(1, min(args.steps, 10)), 3, rank, world, peaks, peak_kind)
+    if args.decode_paged:
+        dw = synthetic.WORKLOADS["decode_7p6b"]
+        line["decode_paged"] = run_decode_paged(dw, max(1, min(args.steps, 10)), 3, rank, world,
+                                                peaks, peak_kind)
     if args.all:
         line["other_workloads"] = []
         for name in ("window_2p6b", "hybrid_7p6b", "tiny_fp32"):

@@ -20,6 +20,7 @@
  *   rat_kv_compress          the D-fold compressed cache: the chunk-end keys/values, the
  *                            ring of the W most recent ones and the recurrence state.
  *   rat_dilated_decode       one new token per sequence against that cache.
+ *   rat_dilated_decode_paged the same over a paged cache, every sequence at its own position.
  *
  * Conventions shared by every call
  *   - Tensors are contiguous, row-major (B, H, T, d) with d innermost, all of one dtype
@@ -282,6 +283,68 @@ RAT_API size_t rat_decode_workspace_bytes(const rat_kv_cache *cache);
 RAT_API int rat_dilated_decode(const void *q, const void *k, const void *v, const void *gate_logit,
                        rat_kv_cache *cache, void *o, float rope_base, float scale,
                        void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * Paged compressed cache with per-sequence positions, for serving: sequences of different
+ * lengths decode in one launch.  The content is that of rat_kv_cache (the pages' D-fold
+ * compressed cache: chunk-end entries, the window ring, the recurrence state); how it is laid
+ * out in memory is this library's (the pages describe no memory management).
+ *
+ *   k_pool, v_pool : device [n_pages][page_entries][d] of dtype
+ *   page_table     : device int32 [B][H][max_pages]: dil entry i of slice (b, h) -- position
+ *                    i*D_h + D_h - 1 -- is row page_table[b][h][i / page_entries] * page_entries
+ *                    + (i mod page_entries) of the pool.  Every table entry that a call reaches
+ *                    must name a page in [0, n_pages); one that does not is skipped and records
+ *                    RAT_ERR_INVALID in the workspace header (see rat_sync_status).
+ *   k_win, v_win   : device [B][H][W][d] ring, position p in slot p mod W (NULL if W = 0)
+ *   h_k, h_v       : device float32 [B][H][d], each sequence's state after its last position
+ *   pos            : device int64 [B], positions consumed by each sequence: set by
+ *                    rat_paged_kv_compress, advanced by one on the device by every
+ *                    rat_dilated_decode_paged (so a captured CUDA graph of decode steps replays
+ *                    with the positions moving)
+ *   page_entries   : a power of two; a slice holds at most max_pages * page_entries dil entries
+ *                    (positions beyond are attended through the window only while in it, as in
+ *                    rat_kv_cache with Tcap = max_pages * page_entries * D_h)
+ *   reset_every    : as in rat_kv_cache
+ * The struct is host memory; the caller owns every buffer and fills the page table.
+ * ---------------------------------------------------------------------------------------- */
+typedef struct rat_paged_kv_cache {
+    int32_t B, H, d, W;       /* batch, heads, head dim, local window (0 = none)           */
+    int32_t dtype;            /* rat_dtype of the pools and the ring                        */
+    int32_t page_entries;     /* dil entries per page (power of two)                        */
+    int32_t max_pages;        /* page-table entries per (b, h) slice                        */
+    int32_t n_pages;          /* pages in each pool                                         */
+    const int32_t *D;         /* host int32[H]: dilation of each head (>= 1)               */
+    void *k_pool, *v_pool;    /* device pools, see above                                    */
+    const int32_t *page_table;/* device int32 [B][H][max_pages]                             */
+    void *k_win, *v_win;      /* device ring, or NULL when W == 0                          */
+    float *h_k, *h_v;         /* device float32 state                                      */
+    int64_t *pos;             /* device int64 [B]                                           */
+    int64_t reset_every;      /* recurrence block length L, or 0 (full sequence)           */
+} rat_paged_kv_cache;
+
+/* rat_paged_kv_compress -- append positions pos0 .. pos0+T-1 of sequence b to a paged cache.
+ *   k_rec, v_rec : device (1, H, T, d) of cache->dtype, recurrence outputs of those positions
+ *   hT_k, hT_v   : device (1, H, d) float32 state after them (copied into the cache's slot b)
+ *   ws, ws_bytes : workspace of at least 256 bytes, 256-byte aligned (error header)
+ * Writes every position p with p mod D_h = D_h - 1 (and p / D_h below the slice capacity) to its
+ * pool row, the last min(W, T) positions to their ring slots, the state, and pos[b] = pos0 + T
+ * (on the device, in stream order).  Bit-exact copies.  0 <= b < B; pos0 >= 0. */
+RAT_API int rat_paged_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k,
+                          const float *hT_v, int T, int b, int64_t pos0,
+                          rat_paged_kv_cache *cache, void *ws, size_t ws_bytes, void *stream);
+
+/* rat_dilated_decode_paged -- rat_dilated_decode for every sequence b at its own position
+ * t_b = pos[b] (read on the device), over the paged cache, then pos[b] = t_b + 1.  Arguments,
+ * results and numerics as rat_dilated_decode; ws of at least rat_paged_decode_workspace_bytes.
+ * When t_b mod D_h = D_h - 1 the table must name a page for entry t_b / D_h below the slice
+ * capacity; otherwise the entry is not stored and RAT_ERR_INVALID is recorded. */
+RAT_API size_t rat_paged_decode_workspace_bytes(const rat_paged_kv_cache *cache);
+
+RAT_API int rat_dilated_decode_paged(const void *q, const void *k, const void *v,
+                             const void *gate_logit, rat_paged_kv_cache *cache, void *o,
+                             float rope_base, float scale, void *ws, size_t ws_bytes,
+                             void *stream);
 
 /* Test hook for failure detection (no counterpart in the method): the next rat_recur_prefill
  * issued from the calling host thread withholds the look-back publication of chunk `chunk`

@@ -26,7 +26,8 @@ __all__ = [
     "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
     "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
-    "Workspace", "rat_dilated_decode_noalloc",
+    "Workspace", "rat_dilated_decode_noalloc", "PagedKVCache", "make_paged_cache",
+    "rat_paged_kv_compress", "rat_paged_decode_workspace_bytes", "rat_dilated_decode_paged",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -53,6 +54,21 @@ class KVCache(ctypes.Structure):
         ("k_win", ctypes.c_void_p), ("v_win", ctypes.c_void_p),
         ("h_k", ctypes.c_void_p), ("h_v", ctypes.c_void_p),
         ("pos", ctypes.c_int64), ("reset_every", ctypes.c_int64),
+    ]
+
+
+class PagedKVCache(ctypes.Structure):
+    """Mirror of struct rat_paged_kv_cache (host struct of device pointers)."""
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d", ctypes.c_int32), ("W", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("page_entries", ctypes.c_int32), ("max_pages", ctypes.c_int32),
+        ("n_pages", ctypes.c_int32),
+        ("D", ctypes.POINTER(ctypes.c_int32)),
+        ("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+        ("page_table", ctypes.c_void_p),
+        ("k_win", ctypes.c_void_p), ("v_win", ctypes.c_void_p),
+        ("h_k", ctypes.c_void_p), ("h_v", ctypes.c_void_p),
+        ("pos", ctypes.c_void_p), ("reset_every", ctypes.c_int64),
     ]
 
 
@@ -92,6 +108,12 @@ def lib():
         L.rat_debug_inject_lookback_fault.argtypes = [_i64, _i64]
         L.rat_dilated_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(KVCache), _vp,
                                                  _f, _f, _vp]
+        L.rat_paged_kv_compress.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i64,
+                                             ctypes.POINTER(PagedKVCache), _vp, _sz, _vp]
+        L.rat_paged_decode_workspace_bytes.restype = _sz
+        L.rat_paged_decode_workspace_bytes.argtypes = [ctypes.POINTER(PagedKVCache)]
+        L.rat_dilated_decode_paged.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(PagedKVCache),
+                                               _vp, _f, _f, _vp, _sz, _vp]
         L.rat_attn_sync_status.argtypes = [_vp]
         L.rat_attn_error_site.restype = ctypes.c_uint32
         L.rat_attn_error_waiting.restype = ctypes.c_uint32
@@ -282,3 +304,56 @@ def rat_dilated_decode_noalloc(q, k, v, gate_logit, cache: KVCache, o, rope_base
                                           ctypes.byref(cache), _ptr(o), float(rope_base),
                                           float(scale), _stream(stream))
     _check("rat_dilated_decode_noalloc", st)
+
+
+def make_paged_cache(B, H, d, W, dtype: int, D_per_head: Sequence[int], page_entries: int,
+                     n_pages: int, page_table, device="cuda", reset_every: int = 0):
+    """Allocate (with torch) the pools, ring, state and positions of a paged cache around a
+    caller-filled int32 page table (B, H, max_pages) on the device; returns (PagedKVCache,
+    buffers)."""
+    Dh = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
+    tdt = torch.float32 if dtype == F32 else torch.bfloat16
+    assert page_table.dtype == torch.int32 and page_table.is_contiguous()
+    assert tuple(page_table.shape[:2]) == (B, H)
+    bufs = {
+        "k_pool": torch.zeros((n_pages, page_entries, d), dtype=tdt, device=device),
+        "v_pool": torch.zeros((n_pages, page_entries, d), dtype=tdt, device=device),
+        "k_win": torch.zeros((B, H, max(W, 1), d), dtype=tdt, device=device),
+        "v_win": torch.zeros((B, H, max(W, 1), d), dtype=tdt, device=device),
+        "h_k": torch.zeros((B, H, d), dtype=torch.float32, device=device),
+        "h_v": torch.zeros((B, H, d), dtype=torch.float32, device=device),
+        "pos": torch.zeros((B,), dtype=torch.int64, device=device),
+        "page_table": page_table, "D": Dh,
+    }
+    c = PagedKVCache(B=B, H=H, d=d, W=W, dtype=dtype, page_entries=page_entries,
+                     max_pages=int(page_table.shape[2]), n_pages=n_pages, D=Dh,
+                     reset_every=int(reset_every))
+    c.k_pool, c.v_pool = bufs["k_pool"].data_ptr(), bufs["v_pool"].data_ptr()
+    c.page_table = page_table.data_ptr()
+    c.k_win = bufs["k_win"].data_ptr() if W > 0 else None
+    c.v_win = bufs["v_win"].data_ptr() if W > 0 else None
+    c.h_k, c.h_v = bufs["h_k"].data_ptr(), bufs["h_v"].data_ptr()
+    c.pos = bufs["pos"].data_ptr()
+    return c, bufs
+
+
+def rat_paged_kv_compress(k_rec, v_rec, hT_k, hT_v, b: int, pos0: int, cache: PagedKVCache,
+                          ws: Workspace, stream=None):
+    """Append positions pos0 .. pos0+T-1 of sequence b ((1, H, T, d) tensors) to a paged cache."""
+    T = k_rec.shape[2]
+    st = lib().rat_paged_kv_compress(_ptr(k_rec), _ptr(v_rec), _ptr(hT_k), _ptr(hT_v), T, int(b),
+                                     int(pos0), ctypes.byref(cache), ws.ptr, ws.nbytes,
+                                     _stream(stream))
+    _check("rat_paged_kv_compress", st)
+
+
+def rat_paged_decode_workspace_bytes(cache: PagedKVCache) -> int:
+    return int(lib().rat_paged_decode_workspace_bytes(ctypes.byref(cache)))
+
+
+def rat_dilated_decode_paged(q, k, v, gate_logit, cache: PagedKVCache, o, ws: Workspace,
+                             rope_base: float = 0.0, scale: float = 0.0, stream=None):
+    st = lib().rat_dilated_decode_paged(_ptr(q), _ptr(k), _ptr(v), _ptr(gate_logit),
+                                        ctypes.byref(cache), _ptr(o), float(rope_base),
+                                        float(scale), ws.ptr, ws.nbytes, _stream(stream))
+    _check("rat_dilated_decode_paged", st)

@@ -189,7 +189,7 @@ RAT_DEVICE uint64_t globaltimer_ns() {
 
 // Record the first device-side error of a launch in the workspace header.
 RAT_DEVICE void record_error(WsHeader *hdr, int code, uint32_t detail) {
-    if (atomicCAS(&hdr->error, 0, code) == 0) hdr->detail = detail;
+    if (hdr && atomicCAS(&hdr->error, 0, code) == 0) hdr->detail = detail;
 }
 
 // ------------------------------------------------------------------------------ smem / mbarrier

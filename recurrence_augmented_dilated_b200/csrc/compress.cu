@@ -7,7 +7,8 @@
 //   - each of the last min(W, T) positions p to ring slot p mod W,
 // for k~ and v~, bit for bit; and copies the final recurrence state into the cache.
 // One CTA per (row block, b*h); 16-byte vector copies, one row per LPR lanes, four rows per
-// thread in flight at once.
+// thread in flight at once.  The paged form (one sequence per call) writes the dil entries into
+// the pool rows the page table names, and sets the sequence's position.
 #include <algorithm>
 
 #include "common.cuh"
@@ -20,10 +21,12 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
     const int b = (int)blockIdx.x / per_b, rb = (int)blockIdx.x % per_b;
     int h = 0;
     while (rb >= p.blk0[h + 1]) ++h;
-    const int bh = b * p.H + h;
+    const int bh = b * p.H + h;                                  // input slice
+    const bool paged = p.page_table != nullptr;
+    const int bhc = paged ? p.seq * p.H + h : bh;                // cache slice
     const int blk = rb - p.blk0[h], nblk = p.blk0[h + 1] - p.blk0[h];
     const long long D = p.Dh[h];
-    const long long cap = p.Tcap / D;
+    const long long cap = paged ? (long long)p.max_pages << p.page_shift : p.Tcap / D;
     const long long end = p.pos0 + p.T;
     const long long i_lo = p.pos0 / D;                       // first chunk end >= pos0
     const long long i_hi = min(end / D, cap);                // chunk ends < end, within capacity
@@ -47,11 +50,21 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
             const long long i = i_lo + r;
             pos = i * D + D - 1;
             uint8_t *base = static_cast<uint8_t *>(is_v ? p.vdil : p.kdil);
-            dst = base + ((size_t)b * p.total_cap + p.off[h] + i) * row_bytes;
+            if (paged) {
+                const int32_t pg = p.page_table[(size_t)bhc * p.max_pages + (i >> p.page_shift)];
+                if ((uint32_t)pg < (uint32_t)p.n_pages) {
+                    dst = base + (((size_t)pg << p.page_shift) + (size_t)(i & ((1ll << p.page_shift) - 1))) * row_bytes;
+                } else {
+                    dst = nullptr;                      // no such page: skipped, error recorded
+                    record_error(p.hdr, RAT_ERR_INVALID, 0x500u);
+                }
+            } else {
+                dst = base + ((size_t)b * p.total_cap + p.off[h] + i) * row_bytes;
+            }
         } else {
             pos = r_lo + (r - n_dil);
             uint8_t *base = static_cast<uint8_t *>(is_v ? p.vwin : p.kwin);
-            dst = base + (((size_t)b * p.H + h) * p.W + (size_t)(pos % p.W)) * row_bytes;
+            dst = base + ((size_t)bhc * p.W + (size_t)(pos % p.W)) * row_bytes;
         }
         src = (is_v ? src_v : src_k) + (size_t)(pos - p.pos0) * row_bytes;
     };
@@ -68,7 +81,7 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
             if (job < njobs) {
                 const uint8_t *src;
                 locate(job, src, dst[u]);
-                val[u] = *reinterpret_cast<const uint4 *>(src + lane_c * 16);
+                if (dst[u]) val[u] = *reinterpret_cast<const uint4 *>(src + lane_c * 16);
             }
         }
 #pragma unroll
@@ -78,9 +91,10 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
     // recurrence state (float32), once per (b, h)
     if (blk == 0) {
         for (int c = threadIdx.x; c < p.d; c += blockDim.x) {
-            if (p.hTk && p.hk != p.hTk) p.hk[(size_t)bh * p.d + c] = p.hTk[(size_t)bh * p.d + c];
-            if (p.hTv && p.hv != p.hTv) p.hv[(size_t)bh * p.d + c] = p.hTv[(size_t)bh * p.d + c];
+            if (p.hTk && p.hk != p.hTk) p.hk[(size_t)bhc * p.d + c] = p.hTk[(size_t)bh * p.d + c];
+            if (p.hTv && p.hv != p.hTv) p.hv[(size_t)bhc * p.d + c] = p.hTv[(size_t)bh * p.d + c];
         }
+        if (paged && p.seq_pos && h == 0 && threadIdx.x == 0) p.seq_pos[p.seq] = end;
     }
 }
 
@@ -91,7 +105,8 @@ int launch_compress(const CompressParams &p_in, void *stream) {
     int acc = 0;
     for (int h = 0; h < p.H; ++h) {
         const long long D = p.Dh[h];
-        const long long n_dil = std::max(0ll, std::min((p.pos0 + p.T) / D, p.Tcap / D) - p.pos0 / D);
+        const long long cap = p.page_table ? (long long)p.max_pages << p.page_shift : p.Tcap / D;
+        const long long n_dil = std::max(0ll, std::min((p.pos0 + p.T) / D, cap) - p.pos0 / D);
         const long long n_ring = p.W > 0 ? std::min(p.W, p.T) : 0;     // the last min(W, T) positions
         const long long jobs = 2 * (n_dil + n_ring);
         long long n = (jobs + rows_per_pass * 4 - 1) / (rows_per_pass * 4);

@@ -38,8 +38,10 @@ RAT_DEVICE uint4 pack8(const float *x) {
 }
 }  // namespace
 
-// Template on d: 16 lanes per row for d = 128 (8 bf16 each), 8 lanes for d = 64.
-template <int DH>
+// Template on d: 16 lanes per row for d = 128 (8 bf16 each), 8 lanes for d = 64.  PAGED: the
+// dilated entries live in pages of a pool found through a page table, and every sequence has
+// its own position (read from seq_pos, advanced by the last CTA of the sequence).
+template <int DH, bool PAGED>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int LPR = DH / 8;                 // lanes per key row
     constexpr int GPW = 32 / LPR;               // key groups per warp
@@ -47,10 +49,23 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     const int split = blockIdx.x, bh = blockIdx.y, b = bh / p.H, h = bh % p.H;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int grp = lane / LPR, cl = lane % LPR;   // key group inside the warp, lane inside row
-    const long long t = p.t;
+    const long long t = PAGED ? p.seq_pos[b] : p.t;
     const long long D = p.Dh[h];
     const long long We = p.W > 1 ? p.W : 1;
-    const long long cap = p.Tcap / D;
+    const long long cap = PAGED ? (long long)p.max_pages << p.page_shift : p.Tcap / D;
+    // pool row of dil entry idx of this slice; a page index outside the pool marks the entry
+    // missing (and records the error) instead of reading outside the pool
+    const int32_t *ptab = PAGED ? p.page_table + (size_t)bh * p.max_pages : nullptr;
+    auto dil_row = [&](long long idx, bool &ok) -> size_t {
+        if (!PAGED) {
+            ok = true;
+            return (size_t)b * p.total_cap + p.off[h] + idx;
+        }
+        const int32_t pg = __ldg(ptab + (idx >> p.page_shift));
+        ok = (uint32_t)pg < (uint32_t)p.n_pages;
+        if (!ok) record_error(p.hdr, RAT_ERR_INVALID, 0x400u);
+        return ((size_t)(ok ? pg : 0) << p.page_shift) + (size_t)(idx & ((1ll << p.page_shift) - 1));
+    };
     const bool first_half = cl < LPR / 2;
 
     // the new token's query, rotated; every lane group holds a copy of its 8 channels
@@ -74,8 +89,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     const long long n_keys = n_dil + n_ring;
     const long long k_lo = n_keys * split / p.splits, k_hi = n_keys * (split + 1) / p.splits;
 
-    const uint8_t *kdil = static_cast<const uint8_t *>(p.kdil) + ((size_t)b * p.total_cap + p.off[h]) * RB;
-    const uint8_t *vdil = static_cast<const uint8_t *>(p.vdil) + ((size_t)b * p.total_cap + p.off[h]) * RB;
+    // paged: the pools; otherwise this slice's first entry
+    const size_t dil0 = PAGED ? 0 : ((size_t)b * p.total_cap + p.off[h]) * RB;
+    const uint8_t *kdil = static_cast<const uint8_t *>(p.kdil) + dil0;
+    const uint8_t *vdil = static_cast<const uint8_t *>(p.vdil) + dil0;
     const uint8_t *kwin = p.kwin ? static_cast<const uint8_t *>(p.kwin) + (size_t)bh * p.W * RB : nullptr;
     const uint8_t *vwin = p.vwin ? static_cast<const uint8_t *>(p.vwin) + (size_t)bh * p.W * RB : nullptr;
 
@@ -101,8 +118,16 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
             if (have[u]) {
                 const uint8_t *kp, *vp;
                 if (idx < n_dil) {
-                    kp = kdil + (size_t)idx * RB;
-                    vp = vdil + (size_t)idx * RB;
+                    if constexpr (PAGED) {
+                        bool ok;
+                        const size_t row = dil_row(idx, ok);
+                        have[u] = ok;
+                        kp = kdil + row * RB;
+                        vp = vdil + row * RB;
+                    } else {
+                        kp = kdil + (size_t)idx * RB;
+                        vp = vdil + (size_t)idx * RB;
+                    }
                 } else {
                     const long long pos = r_lo + (idx - n_dil);
                     kp = kwin + (size_t)(pos % p.W) * RB;
@@ -111,6 +136,10 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                 kr[u] = __ldg(reinterpret_cast<const uint4 *>(kp + cl * 16));
                 vr[u] = __ldg(reinterpret_cast<const uint4 *>(vp + cl * 16));
             } else {
+                kr[u] = make_uint4(0u, 0u, 0u, 0u);
+                vr[u] = kr[u];
+            }
+            if (PAGED && !have[u]) {            // an entry without a page
                 kr[u] = make_uint4(0u, 0u, 0u, 0u);
                 vr[u] = kr[u];
             }
@@ -186,11 +215,19 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         if (grp == 0) {
 #pragma unroll
             for (int j = 0; j < 8; ++j) { hk[j] = sk[j]; hv[j] = sv[j]; }
-            if (t % D == D - 1 && t / D < cap) {
-                uint8_t *kd = static_cast<uint8_t *>(p.kdil) + ((size_t)b * p.total_cap + p.off[h] + t / D) * RB;
-                uint8_t *vd = static_cast<uint8_t *>(p.vdil) + ((size_t)b * p.total_cap + p.off[h] + t / D) * RB;
-                *reinterpret_cast<uint4 *>(kd + cl * 16) = kpk;
-                *reinterpret_cast<uint4 *>(vd + cl * 16) = vpk;
+            if (t % D == D - 1) {
+                bool ok = t / D < cap;
+                if (ok) {
+                    const size_t row = dil_row(t / D, ok);
+                    if (ok) {
+                        uint8_t *kd = static_cast<uint8_t *>(p.kdil) + row * RB;
+                        uint8_t *vd = static_cast<uint8_t *>(p.vdil) + row * RB;
+                        *reinterpret_cast<uint4 *>(kd + cl * 16) = kpk;
+                        *reinterpret_cast<uint4 *>(vd + cl * 16) = vpk;
+                    }
+                } else if (PAGED) {
+                    record_error(p.hdr, RAT_ERR_INVALID, 0x401u);     // no page for the entry
+                }
             }
             if (p.W > 0) {
                 uint8_t *kw = static_cast<uint8_t *>(p.kwin) + ((size_t)bh * p.W + (size_t)(t % p.W)) * RB;
@@ -248,7 +285,18 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     }
     __shared__ uint32_t s_last;
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&p.tickets[bh], 1u) == (uint32_t)p.splits - 1;
+    if (tid == 0) {
+        s_last = atomicAdd(&p.tickets[bh], 1u) == (uint32_t)p.splits - 1;
+        if (PAGED) {
+            // every CTA of the sequence has read its position (at its start): the last one to
+            // finish advances it for the next step and rearms the ticket
+            const uint32_t n = (uint32_t)(p.H * p.splits);
+            if (atomicAdd(&p.seq_ticket[b], 1u) == n - 1) {
+                p.seq_ticket[b] = 0u;
+                p.seq_pos[b] = t + 1;
+            }
+        }
+    }
     __syncthreads();
     if (!s_last) return;
     // last CTA of the slice: merge the splits
@@ -270,13 +318,17 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 }
 
 int decode_splits(int B, int H, int Tcap, const int32_t *Dh, int W) {
-    // aim for about 12 CTAs per SM over the 148 SMs, and at least ~64 keys per split (measured on
-    // the 32 x 32-slice, 1151-key workload: 2 splits per slice beat 1, 3, 4, 5 and 7)
     long long max_keys = 0;
     for (int h = 0; h < H; ++h) {
         const long long k = Tcap / Dh[h] + W;
         max_keys = k > max_keys ? k : max_keys;
     }
+    return decode_splits_for_keys(B, H, max_keys);
+}
+
+int decode_splits_for_keys(int B, int H, long long max_keys) {
+    // aim for about 12 CTAs per SM over the 148 SMs, and at least ~64 keys per split (measured on
+    // the 32 x 32-slice, 1151-key workload: 2 splits per slice beat 1, 3, 4, 5 and 7)
     const long long bh = (long long)B * H;
     long long s = (148ll * 12 + bh - 1) / bh;
     const long long by_keys = (max_keys + 63) / 64;
@@ -286,17 +338,21 @@ int decode_splits(int B, int H, int Tcap, const int32_t *Dh, int W) {
     return (int)s;
 }
 
+// header, per-slice tickets, per-split (max, sum) and o partials, per-sequence tickets
 size_t decode_workspace_bytes(int B, int H, int d, int splits) {
     const size_t bh = (size_t)B * H;
-    return sizeof(WsHeader) + align256(bh * 4) + align256(bh * splits * 2 * 4) + align256(bh * splits * d * 4);
+    return sizeof(WsHeader) + align256(bh * 4) + align256(bh * splits * 2 * 4) +
+           align256(bh * splits * d * 4) + align256((size_t)B * 4);
 }
 
-int launch_decode(const DecodeParams &p, int dtype, void *stream) {
+int launch_decode(const DecodeParams &p, int dtype, void *stream, bool paged) {
     if (dtype != RAT_BF16) return RAT_ERR_UNSUPPORTED;
     dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.H));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (p.d == 128) decode_kernel<128><<<grid, kThreads, 0, s>>>(p);
-    else if (p.d == 64) decode_kernel<64><<<grid, kThreads, 0, s>>>(p);
+    if (p.d == 128 && !paged) decode_kernel<128, false><<<grid, kThreads, 0, s>>>(p);
+    else if (p.d == 64 && !paged) decode_kernel<64, false><<<grid, kThreads, 0, s>>>(p);
+    else if (p.d == 128) decode_kernel<128, true><<<grid, kThreads, 0, s>>>(p);
+    else if (p.d == 64) decode_kernel<64, true><<<grid, kThreads, 0, s>>>(p);
     else return RAT_ERR_UNSUPPORTED;
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }

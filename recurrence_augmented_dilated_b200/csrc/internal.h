@@ -130,6 +130,13 @@ struct CompressParams {
     int Dh[kMaxHeads];
     long long off[kMaxHeads];
     int blk0[kMaxHeads + 1];    // filled by launch_compress: first CTA of head h within a batch row
+    // paged cache (page_table non-null): the input holds one sequence (B = 1), stored as
+    // sequence `seq` of the cache; dil entry i of head h goes to pool row
+    // page_table[seq * H + h][i >> page_shift] * page_entries + (i & (page_entries - 1))
+    const int32_t *page_table;
+    int page_shift, max_pages, n_pages, seq;
+    long long *seq_pos;         // [B] set to pos0 + T for sequence seq
+    WsHeader *hdr;              // receives RAT_ERR_INVALID for a page index outside the pool
 };
 int launch_compress(const CompressParams &p, void *stream);
 
@@ -151,9 +158,17 @@ struct DecodeParams {
     int Dh[kMaxHeads];
     long long off[kMaxHeads];
     double theta[64];
+    // paged cache with per-sequence positions (launch_decode with paged = true): kdil / vdil are
+    // the page pools, entry i of slice (b, h) is row page_table[bh][i >> page_shift] *
+    // page_entries + (i & (page_entries - 1)) of the pool
+    long long *seq_pos;         // [B] position of sequence b's new token; advanced by the kernel
+    uint32_t *seq_ticket;       // [B] CTAs of sequence b finished (the last one advances seq_pos)
+    const int32_t *page_table;  // [B * H][max_pages]
+    int page_shift, max_pages, n_pages;
 };
 int decode_splits(int B, int H, int Tcap, const int32_t *Dh, int W);
+int decode_splits_for_keys(int B, int H, long long max_keys);
 size_t decode_workspace_bytes(int B, int H, int d, int splits);
-int launch_decode(const DecodeParams &p, int dtype, void *stream);
+int launch_decode(const DecodeParams &p, int dtype, void *stream, bool paged = false);
 
 }  // namespace rat

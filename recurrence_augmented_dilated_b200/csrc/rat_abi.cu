@@ -43,6 +43,27 @@ bool valid_cache(const rat_kv_cache *c) {
     return true;
 }
 
+bool valid_paged_cache(const rat_paged_kv_cache *c) {
+    if (!c || c->B < 1 || c->H < 1 || c->H > kMaxHeads || !supported_d(c->d) || c->W < 0 ||
+        !valid_dtype(c->dtype) || !c->D || c->reset_every < 0 || c->page_entries < 1 ||
+        (c->page_entries & (c->page_entries - 1)) != 0 || c->max_pages < 1 || c->n_pages < 1)
+        return false;
+    if ((long long)c->max_pages * c->page_entries > (1ll << 40)) return false;
+    for (int h = 0; h < c->H; ++h)
+        if (c->D[h] < 1) return false;
+    if (!c->k_pool || !c->v_pool || !c->page_table || !c->h_k || !c->h_v || !c->pos) return false;
+    if (!aligned16(c->k_pool) || !aligned16(c->v_pool)) return false;
+    if (c->W > 0 && (!c->k_win || !c->v_win || !aligned16(c->k_win) || !aligned16(c->v_win)))
+        return false;
+    return true;
+}
+
+int log2_exact(int x) {
+    int s = 0;
+    while ((1 << s) < x) ++s;
+    return s;
+}
+
 // Test hook state: armed by rat_debug_inject_lookback_fault, consumed by the next
 // rat_recur_prefill issued from the same host thread.
 thread_local long long g_fault_chunk = -1;
@@ -326,6 +347,86 @@ size_t rat_decode_workspace_bytes(const rat_kv_cache *c) {
     if (!valid_cache(c)) return 0;
     const int s = decode_splits(c->B, c->H, c->Tcap, c->D, c->W);
     return decode_workspace_bytes(c->B, c->H, c->d, s);
+}
+
+// ------------------------------------------------------------------------------ paged cache
+int rat_paged_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k,
+                          const float *hT_v, int T, int b, int64_t pos0,
+                          rat_paged_kv_cache *c, void *ws, size_t ws_bytes, void *stream) {
+    if (!valid_paged_cache(c) || T < 0 || b < 0 || b >= c->B || pos0 < 0) return RAT_ERR_INVALID;
+    if (!ws || ws_bytes < sizeof(WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255u))
+        return RAT_ERR_WORKSPACE;
+    if (T == 0) return RAT_OK;
+    if (!k_rec || !v_rec || !aligned16(k_rec) || !aligned16(v_rec)) return RAT_ERR_INVALID;
+    CompressParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k_rec; p.v = v_rec; p.hTk = hT_k; p.hTv = hT_v;
+    p.kdil = c->k_pool; p.vdil = c->v_pool; p.kwin = c->k_win; p.vwin = c->v_win;
+    p.hk = c->h_k; p.hv = c->h_v;
+    p.B = 1; p.H = c->H; p.T = T; p.d = c->d; p.W = c->W;
+    p.esize = esize(c->dtype);
+    p.pos0 = pos0;
+    for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
+    p.page_table = c->page_table;
+    p.page_shift = log2_exact(c->page_entries);
+    p.max_pages = c->max_pages;
+    p.n_pages = c->n_pages;
+    p.seq = b;
+    p.seq_pos = reinterpret_cast<long long *>(c->pos);
+    p.hdr = static_cast<WsHeader *>(ws);
+    return launch_compress(p, stream);
+}
+
+size_t rat_paged_decode_workspace_bytes(const rat_paged_kv_cache *c) {
+    if (!valid_paged_cache(c)) return 0;
+    const long long keys = (long long)c->max_pages * c->page_entries + c->W;
+    return decode_workspace_bytes(c->B, c->H, c->d, decode_splits_for_keys(c->B, c->H, keys));
+}
+
+int rat_dilated_decode_paged(const void *q, const void *k, const void *v, const void *gate_logit,
+                             rat_paged_kv_cache *c, void *o, float rope_base, float scale,
+                             void *ws, size_t ws_bytes, void *stream) {
+    if (!valid_paged_cache(c)) return RAT_ERR_INVALID;
+    if (c->dtype != RAT_BF16) return RAT_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !gate_logit || !o) return RAT_ERR_INVALID;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logit) || !aligned16(o))
+        return RAT_ERR_INVALID;
+    if (!std::isfinite(rope_base) || !std::isfinite(scale)) return RAT_ERR_INVALID;
+    if ((long long)c->B * c->H > 65535) return RAT_ERR_UNSUPPORTED;
+    const long long keys = (long long)c->max_pages * c->page_entries + c->W;
+    const int splits = decode_splits_for_keys(c->B, c->H, keys);
+    const size_t need = decode_workspace_bytes(c->B, c->H, c->d, splits);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RAT_ERR_WORKSPACE;
+
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k; p.v = v; p.a = gate_logit; p.o = o;
+    p.kdil = c->k_pool; p.vdil = c->v_pool; p.kwin = c->k_win; p.vwin = c->v_win;
+    p.hk = c->h_k; p.hv = c->h_v;
+    p.B = c->B; p.H = c->H; p.d = c->d; p.W = c->W; p.splits = splits;
+    p.reset = c->reset_every;
+    for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
+    p.rope = rope_base > 0.f ? 1 : 0;
+    const float sc = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)c->d));
+    p.scale_log2 = sc * 1.4426950408889634f;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    const size_t bh = (size_t)c->B * c->H;
+    p.hdr = reinterpret_cast<WsHeader *>(w);
+    size_t off = sizeof(WsHeader);
+    p.tickets = reinterpret_cast<uint32_t *>(w + off);
+    off += align256(bh * 4);
+    p.part_ml = reinterpret_cast<float *>(w + off);
+    off += align256(bh * splits * 2 * 4);
+    p.part_o = reinterpret_cast<float *>(w + off);
+    off += align256(bh * splits * c->d * 4);
+    p.seq_ticket = reinterpret_cast<uint32_t *>(w + off);
+    p.seq_pos = reinterpret_cast<long long *>(c->pos);
+    p.page_table = c->page_table;
+    p.page_shift = log2_exact(c->page_entries);
+    p.max_pages = c->max_pages;
+    p.n_pages = c->n_pages;
+    if (p.rope) rope_theta(rope_base, c->d, p.theta);
+    return launch_decode(p, c->dtype, stream, true);
 }
 
 int rat_dilated_decode(const void *q, const void *k, const void *v, const void *gate_logit,

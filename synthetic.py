@@ -121,6 +121,13 @@ def decode_context_block(w: Workload, c: int, device="cpu", T=None, B=None, H=No
     return out[0], out[1], out[2]
 
 
+def ragged_lengths(w: Workload) -> List[int]:
+    """Context lengths of the ragged decode batch: sequence b holds T/2 + (T/2) b / (B-1)
+    positions, evenly spread from half the workload's context to all of it."""
+    half = w.T // 2
+    return [half + (half * b) // max(w.B - 1, 1) for b in range(w.B)]
+
+
 def decode_steps(w: Workload, steps=None):
     """Per-step new tokens q, k, v, a, each (steps, B, H, d), on the CPU in w's dtype."""
     steps = w.steps if steps is None else steps

@@ -187,6 +187,49 @@ def test_cache_rejects_negative_block_length(L):
     assert L.rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(sz), None, None) == 0
 
 
+def paged(**kw):
+    D = (ctypes.c_int32 * kw.get("H", 2))(*kw.get("Dlist", [1, 64]))
+    c = rat.PagedKVCache(B=kw.get("B", 2), H=kw.get("H", 2), d=kw.get("d", 128), W=kw.get("W", 16),
+                         dtype=kw.get("dtype", 1), page_entries=kw.get("pe", 64),
+                         max_pages=kw.get("max_pages", 8), n_pages=kw.get("n_pages", 32), D=D)
+    c._keep = D
+    c.k_pool = c.v_pool = c.k_win = c.v_win = c.h_k = c.h_v = c.pos = c.page_table = 256
+    return c
+
+
+def test_paged_validation(L):
+    P = ctypes.c_void_p
+    ws = P(256 * 4096)
+    ok = paged()
+    need = rat.rat_paged_decode_workspace_bytes(ok)
+    assert need > 256
+    args = lambda c, wsb=need: (P(256), P(256), P(256), P(256), ctypes.byref(c), P(256), 0.0, 0.0,
+                                ws, wsb, None)
+    # page_entries must be a power of two; pool and table sizes at least 1
+    for bad in (paged(pe=48), paged(pe=0), paged(max_pages=0), paged(n_pages=0)):
+        assert rat.rat_paged_decode_workspace_bytes(bad) == 0
+        assert L.rat_dilated_decode_paged(*args(bad)) == -1
+    # missing page table or positions
+    c = paged()
+    c.page_table = None
+    assert L.rat_dilated_decode_paged(*args(c)) == -1
+    c = paged()
+    c.pos = None
+    assert L.rat_dilated_decode_paged(*args(c)) == -1
+    # float32 decode is not provided; the workspace must be large enough
+    assert L.rat_dilated_decode_paged(*args(paged(dtype=0))) == -2
+    assert L.rat_dilated_decode_paged(*args(ok, need - 1)) == -5
+    # compress: sequence index in range, workspace header present
+    assert L.rat_paged_kv_compress(P(256), P(256), None, None, 8, 2, 0, ctypes.byref(ok), ws, 256,
+                                   None) == -1
+    assert L.rat_paged_kv_compress(P(256), P(256), None, None, 8, 0, -1, ctypes.byref(ok), ws, 256,
+                                   None) == -1
+    assert L.rat_paged_kv_compress(P(256), P(256), None, None, 8, 0, 0, ctypes.byref(ok), None, 256,
+                                   None) == -5
+    assert L.rat_paged_kv_compress(None, None, None, None, 0, 0, 0, ctypes.byref(ok), ws, 256,
+                                   None) == 0
+
+
 def test_workspace_init_rejects_null(L):
     assert L.rat_workspace_init(None, 1024, None) == -5
     assert L.rat_sync_status(None, None) == -5
