@@ -49,6 +49,8 @@ def _load():
         lib.rat_oracle_recurrence.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp]
         lib.rat_oracle_recurrence_reset.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _L, _L]
         lib.rat_oracle_recurrence_window.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _L, _dp]
+        lib.rat_oracle_recurrence_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _dp,
+                                                       _dp, _dp]
         lib.rat_oracle_rope.argtypes = [_L, _L, _L, _dp, _L, ctypes.c_double]
         lib.rat_oracle_in_key_set.argtypes = [_L, _L, _L, _L]
         lib.rat_oracle_in_key_set.restype = ctypes.c_int
@@ -144,6 +146,57 @@ def rope(x, pos0: int = 0, base: float = 10000.0):
     BH = int(np.prod(x.shape[:-2])) if x.ndim > 2 else 1
     _load().rat_oracle_rope(BH, T, d, _ptr(x), int(pos0), float(base))
     return x
+
+
+def rope_transpose(y, pos0: int = 0, base: float = 10000.0):
+    """The transpose (= inverse) of the rotate-half rotation: each pair (c, c + d/2) turned by
+    -(pos0 + t) theta_c.  The backward of y = RoPE(h) is dh = RoPE^T(dy)."""
+    y = _f64(y)
+    T, d = y.shape[-2], y.shape[-1]
+    half = d // 2
+    theta = base ** (-2.0 * np.arange(half) / d)
+    ang = (pos0 + np.arange(T))[:, None] * theta[None, :]
+    c, s = np.cos(ang), np.sin(ang)
+    y1, y2 = y[..., :half], y[..., half:]
+    return np.concatenate([y1 * c + y2 * s, y2 * c - y1 * s], axis=-1)
+
+
+def recurrence_backward(x, a, dy, h0=None, dhT=None):
+    """Reverse-mode derivative of recurrence(x, a, h0) (the full-sequence form): returns
+    (dx, dg, dh0) for upstream gradients dy of the outputs and dhT of the final state; dg is
+    the gradient with respect to the gate value g = sigmoid(a)."""
+    x, a, dy = _f64(x), _f64(a), _f64(dy)
+    assert x.shape == a.shape == dy.shape
+    T, d = x.shape[-2], x.shape[-1]
+    BH = int(np.prod(x.shape[:-2])) if x.ndim > 2 else 1
+    dx, dg = np.empty_like(x), np.empty_like(x)
+    dh0 = np.empty(x.shape[:-2] + (d,), dtype=np.float64)
+    h0p = None
+    if h0 is not None:
+        h0 = _f64(h0)
+        h0p = _ptr(h0)
+    dhTp = None
+    if dhT is not None:
+        dhT = _f64(dhT)
+        dhTp = _ptr(dhT)
+    _load().rat_oracle_recurrence_backward(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(dy), dhTp,
+                                           _ptr(dx), _ptr(dg), _ptr(dh0))
+    return dx, dg, dh0
+
+
+def recurrence_layer_backward(k, v, a, dk_rec, dv_rec, h0k=None, h0v=None, dhTk=None, dhTv=None,
+                              pos0: int = 0, rope_base: float = 0.0):
+    """Backward of the prefill recurrence step (k~ = RoPE(h^k), v~ = h^v, one gate for both):
+    returns (dk, dv, da, dh0k, dh0v).  The gate is shared, so its gradient sums the k and v
+    parts, through dg/da = g (1 - g)."""
+    ek = rope_transpose(dk_rec, pos0, rope_base) if rope_base > 0 else _f64(dk_rec)
+    dk, dgk, dh0k = recurrence_backward(k, a, ek, h0k, dhTk)
+    dv, dgv, dh0v = recurrence_backward(v, a, dv_rec, h0v, dhTv)
+    a = _f64(a)
+    with np.errstate(over="ignore"):        # saturated logits: exp -> inf gives g = 0 or 1
+        g = 1.0 / (1.0 + np.exp(-a))
+        omg = 1.0 / (1.0 + np.exp(a))
+    return dk, dv, g * omg * (dgk + dgv), dh0k, dh0v
 
 
 def in_key_set(t: int, j: int, D: int, W: int) -> bool:

@@ -138,6 +138,44 @@ void rat_oracle_recurrence_window(long BH, long T, long d, const double *x, cons
 }
 
 /*
+ * Backward of the forget-gate recurrence above (its reverse-mode derivative), for one of x = k
+ * or x = v.  With dy_t = dL/dy_t the upstream gradient of the outputs y_t = h_t and dhT =
+ * dL/dh_{T-1} an extra gradient of the final state (NULL: none), the total gradient of the
+ * state runs backwards,
+ *   mu_{T-1} = dy_{T-1} + dhT,      mu_t = dy_t + g_{t+1} mu_{t+1},
+ * and gives  dL/dx_t = (1 - g_t) mu_t,   dL/dg_t = mu_t (h_{t-1} - x_t)  (h_{-1} = h0),
+ *            dL/dh0 = g_0 mu_0.
+ * h is recomputed by the forward loop; dg is the gradient with respect to the gate value g
+ * (the caller applies dg/da = g (1 - g) and sums the k and v parts, which share the gate).
+ */
+void rat_oracle_recurrence_backward(long BH, long T, long d, const double *x, const double *a,
+                                    const double *h0, const double *dy, const double *dhT,
+                                    double *dx, double *dg, double *dh0)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        double *h = (double *)malloc((size_t)(T + 1) * sizeof(double));  /* h[t+1] = h_t */
+        for (long c = 0; c < d; ++c) {
+            h[0] = h0 ? h0[bh * d + c] : 0.0;
+            for (long t = 0; t < T; ++t) {
+                long idx = (bh * T + t) * d + c;
+                h[t + 1] = forget_gate(a[idx]) * h[t] + one_minus_gate(a[idx]) * x[idx];
+            }
+            double mu = dhT ? dhT[bh * d + c] : 0.0;     /* gradient arriving from t + 1 */
+            for (long t = T - 1; t >= 0; --t) {
+                long idx = (bh * T + t) * d + c;
+                mu += dy[idx];                               /* total dL/dh_t */
+                dx[idx] = one_minus_gate(a[idx]) * mu;
+                dg[idx] = mu * (h[t] - x[idx]);
+                mu *= forget_gate(a[idx]);                   /* dL/dh_{t-1} through h_t */
+            }
+            if (dh0) dh0[bh * d + c] = mu;
+        }
+        free(h);
+    }
+}
+
+/*
  * Rotary position embedding, rotate-half pairing, in place.                  [RoFormer]
  *   x : [BH][T][d];  position of row t is pos0 + t;  for c < d/2:
  *   theta_c = base^(-2c/d),  phi = (pos0 + t) * theta_c,

@@ -240,6 +240,104 @@ def test_window_history_equals_the_joined_sequence():
     np.testing.assert_array_equal(y, joined[:, Lw:])
 
 
+# ---- backward of the recurrence step
+def _torch_layer(k, v, a, h0k, h0v, pos0, base):
+    """The forward step written with torch float64 ops, for autograd to differentiate."""
+    import torch
+    T, d = k.shape[-2], k.shape[-1]
+    g = torch.sigmoid(a)
+    hk, hv = h0k, h0v
+    yk, yv = [], []
+    for t in range(T):
+        hk = g[..., t, :] * hk + (1 - g[..., t, :]) * k[..., t, :]
+        hv = g[..., t, :] * hv + (1 - g[..., t, :]) * v[..., t, :]
+        yk.append(hk)
+        yv.append(hv)
+    yk, yv = torch.stack(yk, -2), torch.stack(yv, -2)
+    if base > 0:
+        half = d // 2
+        theta = base ** (-2.0 * torch.arange(half, dtype=torch.float64) / d)
+        ang = (pos0 + torch.arange(T, dtype=torch.float64))[:, None] * theta[None, :]
+        c, s_ = torch.cos(ang), torch.sin(ang)
+        y1, y2 = yk[..., :half], yk[..., half:]
+        yk = torch.cat([y1 * c - y2 * s_, y2 * c + y1 * s_], -1)
+    return yk, yv, hk, hv
+
+
+@pytest.mark.parametrize("base,pos0", [(0.0, 0), (10000.0, 37)])
+def test_backward_matches_autograd(base, pos0):
+    import torch
+    shp = (2, 9, 6)
+    k, v, a = (torch.tensor(RNG.standard_normal(shp), requires_grad=True) for _ in range(3))
+    h0k, h0v = (torch.tensor(RNG.standard_normal((2, 6)), requires_grad=True) for _ in range(2))
+    dyk, dyv = RNG.standard_normal(shp), RNG.standard_normal(shp)
+    dhk, dhv = RNG.standard_normal((2, 6)), RNG.standard_normal((2, 6))
+    yk, yv, hk, hv = _torch_layer(k, v, a, h0k, h0v, pos0, base)
+    loss = ((yk * torch.tensor(dyk)).sum() + (yv * torch.tensor(dyv)).sum() +
+            (hk * torch.tensor(dhk)).sum() + (hv * torch.tensor(dhv)).sum())
+    loss.backward()
+    dk, dv, da, dh0k, dh0v = oracle.recurrence_layer_backward(
+        k.detach().numpy(), v.detach().numpy(), a.detach().numpy(), dyk, dyv,
+        h0k.detach().numpy(), h0v.detach().numpy(), dhk, dhv, pos0=pos0, rope_base=base)
+    for mine, ref in ((dk, k.grad), (dv, v.grad), (da, a.grad), (dh0k, h0k.grad), (dh0v, h0v.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_finite_differences():
+    # central differences of L = <dy, y(k, a, h0)> + <dhT, hT> on single elements
+    T, d = 7, 3
+    x, a = RNG.standard_normal((1, T, d)), RNG.standard_normal((1, T, d))
+    h0, dy, dhT = RNG.standard_normal((1, d)), RNG.standard_normal((1, T, d)), RNG.standard_normal((1, d))
+
+    def L(x_, a_, h0_):
+        y, hT = oracle.recurrence(x_, a_, h0_)
+        return float((y * dy).sum() + (hT * dhT).sum())
+
+    dx, dg, dh0 = oracle.recurrence_backward(x, a, dy, h0, dhT)
+    g = 1.0 / (1.0 + np.exp(-a))
+    da = dg * g * (1 - g)
+    eps = 1e-6
+    for (t, c) in ((0, 0), (3, 1), (6, 2)):
+        for arr, grad in ((x, dx), (a, da)):
+            p_, m_ = arr.copy(), arr.copy()
+            p_[0, t, c] += eps
+            m_[0, t, c] -= eps
+            args_p = (p_, a, h0) if arr is x else (x, p_, h0)
+            args_m = (m_, a, h0) if arr is x else (x, m_, h0)
+            fd = (L(*args_p) - L(*args_m)) / (2 * eps)
+            assert abs(fd - grad[0, t, c]) <= 1e-7 * max(1.0, abs(fd)), (t, c, fd, grad[0, t, c])
+    for c in range(d):
+        p_, m_ = h0.copy(), h0.copy()
+        p_[0, c] += eps
+        m_[0, c] -= eps
+        fd = (L(x, a, p_) - L(x, a, m_)) / (2 * eps)
+        assert abs(fd - dh0[0, c]) <= 1e-7 * max(1.0, abs(fd))
+
+
+def test_backward_is_the_adjoint_of_the_linear_map():
+    # at fixed gates and h0 = 0, x -> y is linear: <dy, y(x)> = <dx(dy), x> exactly
+    x, a, dy = (RNG.standard_normal((3, 40, 4)) for _ in range(3))
+    y, _ = oracle.recurrence(x, a)
+    dx, _, _ = oracle.recurrence_backward(x, a, dy)
+    lhs, rhs = float((dy * y).sum()), float((dx * x).sum())
+    assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), 1.0)
+
+
+def test_backward_zero_gate_passes_the_gradient_through():
+    # g = 0: y = x, so dx = dy exactly and the gate gets no gradient (g (1 - g) = 0)
+    x, dy = RNG.standard_normal((2, 20, 3)), RNG.standard_normal((2, 20, 3))
+    a = np.full_like(x, -1.0e4)
+    dk, dv, da, dh0k, _ = oracle.recurrence_layer_backward(x, x, a, dy, dy)
+    assert np.array_equal(dk, dy) and np.array_equal(dv, dy)
+    assert np.all(da == 0.0) and np.all(dh0k == 0.0)
+
+
+def test_rope_transpose_inverts_rope():
+    x = RNG.standard_normal((2, 11, 8))
+    np.testing.assert_allclose(oracle.rope_transpose(oracle.rope(x, 123, 500.0), 123, 500.0), x,
+                               rtol=1e-12, atol=1e-13)
+
+
 def test_rope_matches_complex_rotation():
     d, T, pos0, base = 16, 9, 1000, 10000.0
     x = RNG.standard_normal((1, T, d))
