@@ -14,6 +14,7 @@
  *                            chunk-local form).
  *   rat_recur_prefill_window the same recurrence over a fixed window of the last Lw = 64
  *                            positions (RAT+'s L*).
+ *   rat_recur_backward       gradients of rat_recur_prefill's step.
  *   rat_dilated_attn_prefill causal attention of each query t over
  *                              S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D = D-1 },
  *                            We = max(W, 1), D per head; optional RoPE on q.
@@ -142,6 +143,41 @@ RAT_API int rat_recur_prefill_local(const void *k, const void *v, const void *ga
                             int B, int H, int T, int d, int dtype,
                             int64_t pos0, int64_t L, float rope_base,
                             void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * rat_recur_backward -- gradients of the prefill recurrence step (rat_recur_prefill, the
+ * full-sequence form), for training with dilated inference in view ("RAT+ Deep Dive" section
+ * 2.2: training mixes dense and dilated samples, which needs this step's derivative).
+ *   The reverse-mode derivative of h_t = g_t h_{t-1} + (1-g_t) x_t, k~ = RoPE(h^k), v~ = h^v:
+ *     mu_t = e_t + g_{t+1} mu_{t+1},  mu_{T-1} = e_{T-1} + dhT,
+ *     e^k_t = RoPE_t^T(dk~_t), e^v_t = dv~_t,
+ *     dk_t = (1-g_t) mu^k_t,  dv_t = (1-g_t) mu^v_t,
+ *     dgate_t = g_t (1-g_t) [mu^k_t (h^k_{t-1} - k_t) + mu^v_t (h^v_{t-1} - v_t)],
+ *     dh0 = g_0 mu_0,   with h^k = RoPE^T(k~), h^v = v~ read from the forward outputs.
+ *
+ *   k, v, gate_logit : device, (B, H, T, d) of dtype          the forward inputs
+ *   h0_k, h0_v       : device, (B, H, d) float32, or NULL     the forward initial state
+ *   k_rec, v_rec     : device, (B, H, T, d) of dtype          the forward outputs k~, v~
+ *   dk_rec, dv_rec   : device, (B, H, T, d) of dtype          upstream gradients of k~, v~
+ *   dhT_k, dhT_v     : device, (B, H, d) float32, or NULL     upstream gradient of the final
+ *                                                            state (NULL: zero)
+ *   dk, dv, dgate_logit : device, (B, H, T, d) of dtype       outputs
+ *   dh0_k, dh0_v     : device, (B, H, d) float32, or NULL     gradient of the initial state
+ *   pos0, rope_base  : as given to rat_recur_prefill
+ *   ws, ws_bytes     : workspace of at least rat_recur_backward_workspace_bytes(B, H, T, d)
+ * float32 arithmetic; bf16 outputs rounded once.  h_{t-1} is taken from the stored (rounded)
+ * forward outputs, as a memory-saving training step would.  Outputs may not alias inputs.
+ * T = 0 is a no-op.  Three launches (chunk reduce, carry, output); no device-side waits.
+ * ---------------------------------------------------------------------------------------- */
+RAT_API size_t rat_recur_backward_workspace_bytes(int B, int H, int T, int d);
+
+RAT_API int rat_recur_backward(const void *k, const void *v, const void *gate_logit,
+                       const float *h0_k, const float *h0_v, const void *k_rec,
+                       const void *v_rec, const void *dk_rec, const void *dv_rec,
+                       const float *dhT_k, const float *dhT_v, void *dk, void *dv,
+                       void *dgate_logit, float *dh0_k, float *dh0_v, int B, int H, int T,
+                       int d, int dtype, int64_t pos0, float rope_base, void *ws,
+                       size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------------------------
  * rat_recur_prefill_window -- the fixed-window recurrence of RAT+: each state covers only the

@@ -22,7 +22,7 @@ import torch
 __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_recur_prefill_local",
-    "rat_recur_prefill_window",
+    "rat_recur_prefill_window", "rat_recur_backward", "rat_recur_backward_workspace_bytes",
     "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
     "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
@@ -92,6 +92,9 @@ def lib():
         L.rat_recur_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.rat_recur_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
+        L.rat_recur_backward_workspace_bytes.restype = _sz
+        L.rat_recur_backward_workspace_bytes.argtypes = [_i, _i, _i, _i]
+        L.rat_recur_backward.argtypes = [_vp] * 16 + [_i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
         L.rat_recur_prefill_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                _i, _i, _i, _i, _i, _i64, _i64, _f, _vp, _sz, _vp]
         L.rat_recur_prefill_local.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -211,6 +214,25 @@ def rat_recur_prefill_local(k, v, gate_logit, k_rec, v_rec, ws: Workspace, L: in
                                        _ptr(hT_v), B, H, T, d, _dtype_code(k), int(pos0), int(L),
                                        float(rope_base), ws.ptr, ws.nbytes, _stream(stream))
     _check("rat_recur_prefill_local", st)
+
+
+def rat_recur_backward_workspace_bytes(B, H, T, d) -> int:
+    return int(lib().rat_recur_backward_workspace_bytes(B, H, T, d))
+
+
+def rat_recur_backward(k, v, gate_logit, k_rec, v_rec, dk_rec, dv_rec, dk, dv, dgate_logit,
+                       ws: Workspace, h0_k=None, h0_v=None, dhT_k=None, dhT_v=None, dh0_k=None,
+                       dh0_v=None, pos0: int = 0, rope_base: float = 0.0, stream=None):
+    """Gradients of the prefill recurrence step: dk, dv, dgate_logit (all (B, H, T, d)) and,
+    if given, dh0_k, dh0_v (float32 (B, H, d))."""
+    B, H, T, d = k.shape
+    st = lib().rat_recur_backward(_ptr(k), _ptr(v), _ptr(gate_logit), _ptr(h0_k), _ptr(h0_v),
+                                  _ptr(k_rec), _ptr(v_rec), _ptr(dk_rec), _ptr(dv_rec),
+                                  _ptr(dhT_k), _ptr(dhT_v), _ptr(dk), _ptr(dv),
+                                  _ptr(dgate_logit), _ptr(dh0_k), _ptr(dh0_v), B, H, T, d,
+                                  _dtype_code(k), int(pos0), float(rope_base), ws.ptr, ws.nbytes,
+                                  _stream(stream))
+    _check("rat_recur_backward", st)
 
 
 def rat_recur_prefill_window(k, v, gate_logit, k_rec, v_rec, ws: Workspace, Lw: int = 64,

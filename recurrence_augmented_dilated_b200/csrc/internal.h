@@ -62,6 +62,28 @@ struct WindowParams {
 };
 int launch_window(const WindowParams &p, int dtype, void *stream);
 
+// backward of the recurrence step (reduce, carry and output launches over 64-row chunks)
+constexpr int kBwdRows = 64;
+struct RecurBwdParams {
+    const void *k, *v, *a;          // forward inputs
+    const void *yk, *yv;            // forward outputs k~ (rotated), v~
+    const void *dyk, *dyv;          // upstream gradients of k~, v~
+    const float *h0k, *h0v;         // initial state, or null
+    const float *dhTk, *dhTv;       // gradient of the final state, or null
+    void *dk, *dv, *da;             // outputs
+    float *dh0k, *dh0v;             // gradient of the initial state, or null
+    float *agg;                     // [BH][nch][3][d]  A, Bk, Bv of each chunk (reverse map)
+    float *carry;                   // [BH][nch][2][d]  gradient entering each chunk from the right
+    int BH, T, d, nch;
+    long long pos0;
+    int rope, rope_f32;
+    float theta_f[64];
+    double theta[64];
+    float step_cos[64], step_sin[64];
+};
+size_t recur_bwd_workspace_bytes(int BH, int T, int d);
+int launch_recur_bwd(const RecurBwdParams &p, int dtype, void *stream);
+
 int recur_chunk_rows(int d, int dtype);
 size_t recur_workspace_bytes(int BH, int T, int d, int dtype);
 int launch_recur(const RecurParams &p, int dtype, void *stream);

@@ -1,0 +1,110 @@
+"""GPU parity of rat_recur_backward (gradients of the prefill recurrence step) against the
+float64 oracle's reverse loop."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import recurrence_augmented_dilated_b200 as rat
+import synthetic
+from gpu_util import TOL_BF16, TOL_F32, f64, gpu_recur, rel_err, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def inputs(B, H, T, d, dtype, seed=0, mu=2.0, sigma=1.0):
+    w = synthetic.Workload("b", B=B, H=H, d=d, T=T, dtype="f32" if dtype == torch.float32 else "bf16",
+                           gate_mu=mu, gate_sigma=sigma, seed=seed)
+    return synthetic.prefill_inputs(w)
+
+
+def gpu_backward(x, dyk, dyv, h0=None, dhT=None, pos0=0, rope_base=0.0):
+    dev = torch.device("cuda")
+    k, v, a = (x[n].to(dev) for n in ("k", "v", "a"))
+    B, H, T, d = k.shape
+    h0k = h0v = dhk = dhv = None
+    if h0 is not None:
+        h0k, h0v = (t.to(dev) for t in h0)
+    if dhT is not None:
+        dhk, dhv = (t.to(dev) for t in dhT)
+    kr, vr, _, _ = gpu_recur(k, v, a, rope_base=rope_base, pos0=pos0, h0k=h0k, h0v=h0v)
+    dk, dv, da = torch.empty_like(k), torch.empty_like(v), torch.empty_like(a)
+    dh0k = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+    dh0v = torch.empty_like(dh0k)
+    ws = rat.Workspace(rat.rat_recur_backward_workspace_bytes(B, H, T, d))
+    rat.rat_recur_backward(k, v, a, kr, vr, dyk.to(dev), dyv.to(dev), dk, dv, da, ws,
+                           h0_k=h0k, h0_v=h0v, dhT_k=dhk, dhT_v=dhv, dh0_k=dh0k, dh0_v=dh0v,
+                           pos0=pos0, rope_base=rope_base)
+    assert rat.rat_sync_status(ws) == 0
+    return dk, dv, da, dh0k, dh0v
+
+
+def check(x, dyk, dyv, h0=None, dhT=None, pos0=0, rope_base=0.0, heads=None):
+    got = gpu_backward(x, dyk, dyv, h0, dhT, pos0, rope_base)
+    B, H = x["k"].shape[:2]
+    sel = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    bi, hi = [b for b, _ in sel], [h for _, h in sel]
+    pick = lambda t: None if t is None else f64(t[bi, hi])
+    ref = oracle.recurrence_layer_backward(
+        pick(x["k"]), pick(x["v"]), pick(x["a"]), pick(dyk), pick(dyv),
+        None if h0 is None else pick(h0[0]), None if h0 is None else pick(h0[1]),
+        None if dhT is None else pick(dhT[0]), None if dhT is None else pick(dhT[1]),
+        pos0=pos0, rope_base=rope_base)
+    tol = tol_for(x["k"].dtype)
+    names = ("dk", "dv", "da", "dh0k", "dh0v")
+    errs = {n: rel_err(g[bi, hi], r) for n, g, r in zip(names, got, ref)}
+    for n in names:
+        assert errs[n] <= tol, errs
+    return errs
+
+
+def grads(B, H, T, d, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn((B, H, T, d), generator=g).to(dtype),
+            torch.randn((B, H, T, d), generator=g).to(dtype))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 200, 1000])
+def test_backward_ragged_lengths(dtype, d, T):
+    x = inputs(2, 3, T, d, dtype, seed=T + d)
+    dyk, dyv = grads(2, 3, T, d, dtype, seed=T)
+    check(x, dyk, dyv)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("pos0", [0, 5000])
+def test_backward_state_gradients_and_rope(dtype, pos0):
+    x = inputs(2, 2, 333, 128, dtype, seed=pos0 + 3)
+    dyk, dyv = grads(2, 2, 333, 128, dtype, seed=9)
+    g = torch.Generator().manual_seed(11)
+    h0 = (torch.randn((2, 2, 128), generator=g), torch.randn((2, 2, 128), generator=g))
+    dhT = (torch.randn((2, 2, 128), generator=g), torch.randn((2, 2, 128), generator=g))
+    check(x, dyk, dyv, h0=h0, dhT=dhT, pos0=pos0, rope_base=10000.0)
+
+
+def test_backward_slow_gates():
+    # gates near 1 carry the gradient far back (logits around 5: g ~ 0.993)
+    x = inputs(1, 2, 1500, 128, torch.float32, seed=4, mu=5.0, sigma=0.5)
+    dyk, dyv = grads(1, 2, 1500, 128, torch.float32, seed=5)
+    check(x, dyk, dyv)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_backward_zero_gate_passes_the_gradient_through(dtype):
+    # g = 0 exactly: k~ = k, so dk = dk~ bit for bit and the gate gets no gradient
+    x = inputs(1, 2, 300, 128, dtype, seed=12)
+    x["a"] = torch.full_like(x["a"], -1.0e4)
+    dyk, dyv = grads(1, 2, 300, 128, dtype, seed=13)
+    dk, dv, da, dh0k, _ = gpu_backward(x, dyk, dyv)
+    assert torch.equal(dk.cpu(), dyk) and torch.equal(dv.cpu(), dyv)
+    assert torch.count_nonzero(da).item() == 0 and torch.count_nonzero(dh0k).item() == 0
+
+
+def test_backward_full_size_sampled_heads():
+    # the prefill_1p5b workload (B 4, H 16, T 4096, d 128, bf16, RoPE)
+    w = synthetic.WORKLOADS["prefill_1p5b"]
+    x = synthetic.prefill_inputs(w)
+    dyk, dyv = grads(w.B, w.H, w.T, w.d, torch.bfloat16, seed=21)
+    check(x, dyk, dyv, rope_base=w.rope_base, heads=[(0, 0), (w.B - 1, w.H - 1), (2, 5)])
