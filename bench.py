@@ -606,6 +606,53 @@ def run_decode_paged(w: synthetic.Workload, steps_timed: int, warmup: int, rank:
     }
 
 
+def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, peaks, peak_kind):
+    """Backward of the recurrence step on the prefill workload: the forward outputs and
+    upstream gradients are resident; each timed step is one rat_recur_backward call."""
+    import recurrence_augmented_dilated_b200 as rat
+    dev = torch.device("cuda")
+    x = synthetic.prefill_inputs(w)
+    k, v, a = (x[n].to(dev) for n in ("k", "v", "a"))
+    B, H, T, d = k.shape
+    dtc = rat.F32 if w.dtype == "f32" else rat.BF16
+    kr, vr = torch.empty_like(k), torch.empty_like(v)
+    ws_f = rat.Workspace(rat.rat_recur_workspace_bytes(B, H, T, d, dtc))
+    rat.rat_recur_prefill(k, v, a, kr, vr, ws_f, rope_base=w.rope_base)
+    g = torch.Generator(device=dev).manual_seed(w.seed + 77)
+    dyk = torch.randn(k.shape, generator=g, device=dev).to(k.dtype)
+    dyv = torch.randn(k.shape, generator=g, device=dev).to(k.dtype)
+    dk, dv, da = torch.empty_like(k), torch.empty_like(v), torch.empty_like(a)
+    ws = rat.Workspace(rat.rat_recur_backward_workspace_bytes(B, H, T, d))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rat.rat_recur_backward(k, v, a, kr, vr, dyk, dyv, dk, dv, da, ws, rope_base=w.rope_base)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if rat.rat_sync_status(ws) != 0:
+        raise RuntimeError("backward device error")
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    eb = 2 if w.dtype == "bf16" else 4
+    nbytes = 10 * B * H * T * d * eb       # read k, v, a, k~, v~, dk~, dv~; write dk, dv, da
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name, "step": "rat_recur_backward (3 launches)", "ms": ms,
+            "tokens_per_s": world * B * T / (ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "of": peak_kind,
+                         "algorithmic_bytes": nbytes},
+            "clocks": clk.summary(), "gpu_launches": 3 * steps}
+
+
 # ----------------------------------------------------------------------------- oracle (CPU)
 def oracle_sample(w: synthetic.Workload, budget_s: float = 12.0):
     """Time the float64 oracle on whole (b, h) slices of w (recurrence + RoPE + attention over
@@ -679,6 +726,8 @@ def main():
                          "prefill step instead of the full-sequence one")
     ap.add_argument("--decode-paged", action="store_true",
                     help="also time ragged decode (context lengths T/2 .. T) on a paged cache")
+    ap.add_argument("--backward", action="store_true",
+                    help="also time the backward of the recurrence step on the workload")
     ap.add_argument("--window", type=int, default=0,
                     help="Lw > 0: the fixed-window recurrence (each state over the last Lw "
                          "positions) in the prefill step")
@@ -761,6 +810,8 @@ def main():
     if not args.no_decode:
         dw = synthetic.WORKLOADS["decode_7p6b"]
         line["decode"] = run_decode(dw, max(1, min(args.steps, 10)), 3, rank, world, peaks, peak_kind)
+    if args.backward:
+        line["backward"] = run_backward(w, args.steps, args.warmup, world, peaks, peak_kind)
     if args.decode_paged:
         dw = synthetic.WORKLOADS["decode_7p6b"]
         line["decode_paged"] = run_decode_paged(dw, max(1, min(args.steps, 10)), 3, rank, world,

@@ -33,7 +33,8 @@ struct BwdCfg {
     static constexpr int SPW = 32 / LPR;               // chunk streams per warp
     static constexpr int ROWB = DH * (int)sizeof(E);
     static constexpr int HALFB = ROWB / 2;
-    static constexpr int U = sizeof(E) == 2 ? 4 : 2;   // rows whose loads are issued together
+    static constexpr int U = sizeof(E) == 2 ? 3 : 2;   // rows loaded together (output pass)
+    static constexpr int UR = sizeof(E) == 2 ? 4 : 2;  // rows loaded together (reduce pass)
     static constexpr int THREADS = 256;
     static constexpr int SPB = THREADS / 32 * SPW;     // chunk streams per CTA
 };
@@ -73,7 +74,7 @@ RAT_DEVICE void step_back(f2_t &c, f2_t &s, f2_t sc, f2_t ss) {
 template <typename E, int DH>
 __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS) bwd_reduce_kernel(const __grid_constant__ RecurBwdParams p) {
     using C = BwdCfg<E, DH>;
-    constexpr int NP = 2, U = C::U;
+    constexpr int NP = 2, U = C::UR;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int cl = lane % C::LPR;
     const long long stream = ((long long)blockIdx.x * (C::THREADS / 32) + warp) * C::SPW + lane / C::LPR;
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(128) bwd_carry_kernel(const __grid_constant__ 
 }
 
 template <typename E, int DH>
-__global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS) bwd_out_kernel(const __grid_constant__ RecurBwdParams p) {
+__global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS, 2) bwd_out_kernel(const __grid_constant__ RecurBwdParams p) {
     using C = BwdCfg<E, DH>;
     constexpr int NP = 2, U = C::U;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
