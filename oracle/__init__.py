@@ -49,6 +49,9 @@ def _load():
         lib.rat_oracle_recurrence.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp]
         lib.rat_oracle_recurrence_reset.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _L, _L]
         lib.rat_oracle_recurrence_window.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _L, _dp]
+        lib.rat_oracle_dilated_attention_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp,
+                                                              _ip, _L, ctypes.c_double, _dp,
+                                                              _dp, _dp]
         lib.rat_oracle_recurrence_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _dp,
                                                        _dp, _dp]
         lib.rat_oracle_rope.argtypes = [_L, _L, _L, _dp, _L, ctypes.c_double]
@@ -242,6 +245,27 @@ def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None)
     _load().rat_oracle_dilated_attention(B * H, T, d, _ptr(q), _ptr(k), _ptr(v), _ptr(Dbh, _ip),
                                          int(W), float(scale), rp, nrows, _ptr(out))
     return out
+
+
+def dilated_attention_backward(q, k, v, dO, D=1, W=0, D_per_head=None, scale=None,
+                               rope_base=0.0, pos0=0):
+    """Reverse-mode derivative of dilated_attention for upstream gradients dO: returns
+    (dq, dk, dv) in float64.  With rope_base > 0, q is rotated at positions pos0 + t first (as
+    the attention does) and dq is the gradient with respect to the unrotated q (RoPE^T applied);
+    k and v are the recurrence outputs k~, v~ as stored (k~ already rotated)."""
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, H, T, d = q.shape
+    Dbh, _ = _per_bh_dilation((B, H), D, D_per_head)
+    if scale is None:
+        scale = default_scale(d)
+    qh = rope(q, pos0, rope_base) if rope_base > 0 else q
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    _load().rat_oracle_dilated_attention_backward(B * H, T, d, _ptr(qh), _ptr(k), _ptr(v),
+                                                  _ptr(dO), _ptr(Dbh, _ip), int(W), float(scale),
+                                                  _ptr(dq), _ptr(dk), _ptr(dv))
+    if rope_base > 0:
+        dq = rope_transpose(dq, pos0, rope_base)
+    return dq, dk, dv
 
 
 def layer_prefill(q, k, v, a, D=1, W=0, D_per_head=None, rope_base=0.0, pos0=0, scale=None,

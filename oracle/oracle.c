@@ -278,6 +278,77 @@ void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, cons
 }
 
 /*
+ * Backward of the dilated attention above (its reverse-mode derivative), for upstream
+ * gradients dO of the outputs.  Per query t, with p_j the softmax weights over S(t) and
+ * o_t = sum_j p_j v_j:
+ *   dv_j += p_j dO_t;   dp_j = <dO_t, v_j>;   ds_j = p_j (dp_j - <dO_t, o_t>);
+ *   dq_t  = scale * sum_j ds_j k_j;   dk_j += scale * ds_j q_t.
+ * q, k as used by the attention (already rotated); dq, dk, dv are accumulated into arrays the
+ * caller zeroes.  o_t is recomputed here from the definition.
+ */
+void rat_oracle_dilated_attention_backward(long BH, long T, long d, const double *q,
+                                           const double *k, const double *v, const double *dO,
+                                           const int *Dbh, long W, double scale, double *dq,
+                                           double *dk, double *dv)
+{
+    long We = eff_window(W);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {           /* slices are independent: no shared writes */
+        long D = Dbh[bh];
+        long *keys = (long *)malloc(sizeof(long) * (size_t)(T + 1));
+        double *p = (double *)malloc(sizeof(double) * (size_t)(T + 1));
+        double *ot = (double *)malloc(sizeof(double) * (size_t)d);
+        for (long t = 0; t < T; ++t) {
+            long n = 0;
+            for (long j = (t - We + 1 > 0 ? t - We + 1 : 0); j <= t; ++j) keys[n++] = j;
+            for (long j = D - 1; j <= t - We; j += D) keys[n++] = j;
+            const double *qt = q + (bh * T + t) * d;
+            const double *gt = dO + (bh * T + t) * d;
+            double mx = -INFINITY;
+            for (long m = 0; m < n; ++m) {
+                const double *kj = k + (bh * T + keys[m]) * d;
+                double dot = 0.0;
+                for (long c = 0; c < d; ++c) dot += qt[c] * kj[c];
+                p[m] = scale * dot;
+                if (p[m] > mx) mx = p[m];
+            }
+            double l = 0.0;
+            for (long m = 0; m < n; ++m) {
+                p[m] = exp(p[m] - mx);
+                l += p[m];
+            }
+            for (long c = 0; c < d; ++c) ot[c] = 0.0;
+            for (long m = 0; m < n; ++m) {
+                p[m] /= l;
+                const double *vj = v + (bh * T + keys[m]) * d;
+                for (long c = 0; c < d; ++c) ot[c] += p[m] * vj[c];
+            }
+            double delta = 0.0;                          /* <dO_t, o_t> */
+            for (long c = 0; c < d; ++c) delta += gt[c] * ot[c];
+            double *dqt = dq + (bh * T + t) * d;
+            for (long m = 0; m < n; ++m) {
+                long j = keys[m];
+                const double *kj = k + (bh * T + j) * d;
+                const double *vj = v + (bh * T + j) * d;
+                double dp = 0.0;
+                for (long c = 0; c < d; ++c) dp += gt[c] * vj[c];
+                double ds = p[m] * (dp - delta);
+                double *dkj = dk + (bh * T + j) * d;
+                double *dvj = dv + (bh * T + j) * d;
+                for (long c = 0; c < d; ++c) {
+                    dqt[c] += scale * ds * kj[c];
+                    dkj[c] += scale * ds * qt[c];
+                    dvj[c] += p[m] * gt[c];
+                }
+            }
+        }
+        free(keys);
+        free(p);
+        free(ot);
+    }
+}
+
+/*
  * Compressed KV cache build, on raw element bytes (bit-exact gather).      [RAT+ abstract]
  *   x    : [B][H][T][d] elements of esize bytes: the recurrence outputs of positions
  *          pos0 .. pos0+T-1

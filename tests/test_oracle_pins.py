@@ -338,6 +338,83 @@ def test_rope_transpose_inverts_rope():
                                rtol=1e-12, atol=1e-13)
 
 
+# ---- backward of the dilated attention
+def _torch_attention(q, k, v, D, W, scale):
+    """Masked softmax attention in torch float64, the mask built from the key-set definition,
+    for autograd to differentiate."""
+    import torch
+    T = q.shape[-2]
+    mask = torch.tensor([[oracle.in_key_set(t, j, D, W) for j in range(T)] for t in range(T)])
+    s = scale * (q @ k.transpose(-1, -2))
+    s = s.masked_fill(~mask, float("-inf"))
+    return torch.softmax(s, -1) @ v
+
+
+@pytest.mark.parametrize("D,W,T", [(1, 0, 12), (4, 0, 19), (3, 5, 17), (8, 1, 30)])
+def test_attention_backward_matches_autograd(D, W, T):
+    import torch
+    shp = (2, T, 8)
+    q, k, v = (torch.tensor(RNG.standard_normal(shp), requires_grad=True) for _ in range(3))
+    dO = RNG.standard_normal(shp)
+    o = _torch_attention(q, k, v, D, W, 0.4)
+    (o * torch.tensor(dO)).sum().backward()
+    dq, dk, dv = oracle.dilated_attention_backward(q.detach().numpy()[None], k.detach().numpy()[None],
+                                                   v.detach().numpy()[None], dO[None], D=D, W=W,
+                                                   scale=0.4)
+    for mine, ref in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
+        np.testing.assert_allclose(mine[0], ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_backward_rope_and_head_dilations():
+    # per-head D and the RoPE of q: autograd through rotate-half written in torch
+    import torch
+    B, H, T, d, base, pos0 = 1, 2, 15, 8, 100.0, 9
+    q, k, v = (torch.tensor(RNG.standard_normal((B, H, T, d)), requires_grad=True) for _ in range(3))
+    dO = RNG.standard_normal((B, H, T, d))
+    half = d // 2
+    theta = base ** (-2.0 * torch.arange(half, dtype=torch.float64) / d)
+    ang = (pos0 + torch.arange(T, dtype=torch.float64))[:, None] * theta[None, :]
+    c, s_ = torch.cos(ang), torch.sin(ang)
+    qh = torch.cat([q[..., :half] * c - q[..., half:] * s_, q[..., half:] * c + q[..., :half] * s_], -1)
+    Dh = [2, 5]
+    o = torch.stack([_torch_attention(qh[:, h], k[:, h], v[:, h], Dh[h], 3, 0.5) for h in range(H)], 1)
+    (o * torch.tensor(dO)).sum().backward()
+    dq, dk, dv = oracle.dilated_attention_backward(q.detach().numpy(), k.detach().numpy(),
+                                                   v.detach().numpy(), dO, W=3, D_per_head=Dh,
+                                                   scale=0.5, rope_base=base, pos0=pos0)
+    for mine, ref in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_attention_backward_finite_differences():
+    B, H, T, d, D, W = 1, 1, 10, 4, 3, 2
+    q, k, v, dO = (RNG.standard_normal((B, H, T, d)) for _ in range(4))
+
+    def L(q_, k_, v_):
+        return float((oracle.dilated_attention(q_, k_, v_, D=D, W=W) * dO).sum())
+
+    dq, dk, dv = oracle.dilated_attention_backward(q, k, v, dO, D=D, W=W)
+    eps = 1e-6
+    for arr, grad, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        for (t, c) in ((0, 0), (5, 2), (9, 3)):
+            p_, m_ = arr.copy(), arr.copy()
+            p_[0, 0, t, c] += eps
+            m_[0, 0, t, c] -= eps
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = p_, m_
+            fd = (L(*args_p) - L(*args_m)) / (2 * eps)
+            assert abs(fd - grad[0, 0, t, c]) <= 1e-7 * max(1.0, abs(fd)), (which, t, c)
+
+
+def test_attention_backward_single_key_passes_dv_only():
+    # D > T, W = 0: every query sees only itself, o = v exactly: dv = dO, dq = dk = 0
+    q, k, v, dO = (RNG.standard_normal((1, 2, 9, 4)) for _ in range(4))
+    dq, dk, dv = oracle.dilated_attention_backward(q, k, v, dO, D=100, W=0)
+    np.testing.assert_array_equal(dv, dO)
+    assert np.all(dq == 0.0) and np.all(dk == 0.0)
+
+
 def test_rope_matches_complex_rotation():
     d, T, pos0, base = 16, 9, 1000, 10000.0
     x = RNG.standard_normal((1, T, d))
