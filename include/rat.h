@@ -18,6 +18,7 @@
  *   rat_dilated_attn_prefill causal attention of each query t over
  *                              S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D = D-1 },
  *                            We = max(W, 1), D per head; optional RoPE on q.
+ *   rat_dilated_attn_backward gradients of rat_dilated_attn_prefill.
  *   rat_kv_compress          the D-fold compressed cache: the chunk-end keys/values, the
  *                            ring of the W most recent ones and the recurrence state.
  *   rat_dilated_decode       one new token per sequence against that cache.
@@ -242,6 +243,32 @@ RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const voi
 /* Synchronise `stream`, then return (and clear) the first device-side error recorded by the
  * attention kernel since the last call (RAT_OK if none). */
 RAT_API int rat_attn_sync_status(void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * rat_dilated_attn_backward -- gradients of rat_dilated_attn_prefill (training with dilated
+ * samples: "RAT+ Deep Dive" section 2.2 trains half the samples with D = 1 and half with
+ * D = 64, which needs this derivative for every D).
+ *   With p_t the softmax weights of query t over S(t) and q^ = RoPE(q):
+ *     dp_tj = <dO_t, v~_j>,  ds_tj = p_tj (dp_tj - <dO_t, o_t>),
+ *     dq = RoPE^T(scale sum_j ds_tj k~_j),  dk~_j = scale sum_t ds_tj q^_t,
+ *     dv~_j = sum_t p_tj dO_t.
+ *   q, k_rec, v_rec, o : device (B, H, T, d) of dtype     the forward's inputs and output
+ *   dO                 : device (B, H, T, d) of dtype     upstream gradient of o
+ *   dq, dk_rec, dv_rec : device (B, H, T, d) of dtype     outputs (dk_rec, dv_rec are the
+ *                        gradients of k~, v~: the dk_rec, dv_rec inputs of rat_recur_backward)
+ *   D, W, D_per_head, pos0, rope_base, scale : as given to rat_dilated_attn_prefill
+ *   ws, ws_bytes       : workspace of at least rat_dilated_attn_backward_workspace_bytes
+ * CUDA-core kernels with float32 accumulation: the softmax denominators are recomputed (not
+ * taken from the forward), q^ is rounded to the dtype as the forward's operand is, outputs are
+ * rounded once.  Three launches (prep, dq, dk~ and dv~); no device-side waits.
+ * ---------------------------------------------------------------------------------------- */
+RAT_API size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int dtype);
+
+RAT_API int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_rec,
+                              const void *o, const void *dO, void *dq, void *dk_rec,
+                              void *dv_rec, int B, int H, int T, int d, int dtype, int D, int W,
+                              const int32_t *D_per_head, int64_t pos0, float rope_base,
+                              float scale, void *ws, size_t ws_bytes, void *stream);
 
 /* Diagnostic: where the attention kernel's last recorded timeout happened, as
  * (wait site << 24) | (key block << 8) | phase parity; sites: 1 producer K-stage-free, 2 MMA

@@ -23,6 +23,7 @@ __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_recur_prefill_local",
     "rat_recur_prefill_window", "rat_recur_backward", "rat_recur_backward_workspace_bytes",
+    "rat_dilated_attn_backward", "rat_dilated_attn_backward_workspace_bytes",
     "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
     "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
@@ -92,6 +93,11 @@ def lib():
         L.rat_recur_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.rat_recur_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                         _i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
+        L.rat_dilated_attn_backward_workspace_bytes.restype = _sz
+        L.rat_dilated_attn_backward_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
+        L.rat_dilated_attn_backward.argtypes = [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _i,
+                                                            ctypes.POINTER(ctypes.c_int32), _i64,
+                                                            _f, _f, _vp, _sz, _vp]
         L.rat_recur_backward_workspace_bytes.restype = _sz
         L.rat_recur_backward_workspace_bytes.argtypes = [_i, _i, _i, _i]
         L.rat_recur_backward.argtypes = [_vp] * 16 + [_i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
@@ -261,6 +267,27 @@ def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,
                                         _dtype_code(q), int(D), int(W), dph, int(pos0),
                                         float(rope_base), float(scale), _stream(stream))
     _check("rat_dilated_attn_prefill", st)
+
+
+def rat_dilated_attn_backward_workspace_bytes(B, H, T, d, dtype) -> int:
+    return int(lib().rat_dilated_attn_backward_workspace_bytes(B, H, T, d, dtype))
+
+
+def rat_dilated_attn_backward(q, k_rec, v_rec, o, dO, dq, dk_rec, dv_rec, ws: Workspace,
+                              D: int = 1, W: int = 0, D_per_head: Optional[Sequence[int]] = None,
+                              pos0: int = 0, rope_base: float = 0.0, scale: float = 0.0,
+                              stream=None):
+    """Gradients of rat_dilated_attn_prefill: dq, dk_rec, dv_rec (all (B, H, T, d))."""
+    B, H, T, d = q.shape
+    dph = None
+    if D_per_head is not None:
+        dph = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
+    st = lib().rat_dilated_attn_backward(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), _ptr(dO),
+                                         _ptr(dq), _ptr(dk_rec), _ptr(dv_rec), B, H, T, d,
+                                         _dtype_code(q), int(D), int(W), dph, int(pos0),
+                                         float(rope_base), float(scale), ws.ptr, ws.nbytes,
+                                         _stream(stream))
+    _check("rat_dilated_attn_backward", st)
 
 
 def make_cache(B, H, d, W, Tcap, dtype: int, D_per_head: Sequence[int], device="cuda",

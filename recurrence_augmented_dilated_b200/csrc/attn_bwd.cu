@@ -1,0 +1,238 @@
+// attn_bwd.cu -- backward of the causal dilated attention (CUDA cores, float32 accumulation).
+//
+// The forward (RAT+ abstract; "RAT+ Deep Dive" sections 3.1 and 6): query t of head h attends
+//   S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D_h = D_h - 1 },   We = max(W, 1),
+// o_t = sum_{j in S(t)} p_tj v_j,  p_t = softmax_j(scale <q^_t, k~_j>),  q^ = RoPE(q).
+// Its reverse-mode derivative, for upstream gradients dO:
+//   dp_tj = <dO_t, v_j>,   ds_tj = p_tj (dp_tj - <dO_t, o_t>),
+//   dq^_t = scale sum_j ds_tj k~_j,   dk~_j = scale sum_t ds_tj q^_t,   dv_j = sum_t p_tj dO_t,
+//   dq = RoPE^T(dq^).
+// Three launches, one warp per row, each lane holding d/32 consecutive channels:
+//   prep : q^ = RoPE(q) (rounded to the dtype, as the attention's operand) and <dO_t, o_t>;
+//   dq   : per query, the key set walked twice -- once for the softmax denominator (kept for
+//          the next launch), once for dq;
+//   dkv  : per key, the queries whose key set holds it walked once: the window t in
+//          [j, j + We - 1], and, for a chunk end (j mod D = D - 1), every t >= j + We.
+// Each (query, key) pair is recomputed in both gradient launches; p comes from the stored
+// denominator, so the two launches agree.  This is the plain CUDA-core path of the backward:
+// dot products are warp reductions, four rows' loads in flight per warp.
+#include "common.cuh"
+
+namespace rat {
+
+namespace {
+
+// rotate-half RoPE of a lane's CPL channels (partner channel c +- d/2 lives 16 lanes away);
+// sign = +1 for the rotation, -1 for its transpose
+template <int DH>
+RAT_DEVICE void rope_lane(const AttnBwdParams &p, long long pos, int lane, float sign, float *x) {
+    constexpr int CPL = DH / 32;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+        const int c = lane * CPL + j;
+        float cs, sn;
+        rope_cs(pos, p.theta[c % (DH / 2)], cs, sn);
+        sn *= sign;
+        const float partner = __shfl_xor_sync(0xffffffffu, x[j], 16);
+        x[j] = c < DH / 2 ? x[j] * cs - partner * sn : x[j] * cs + partner * sn;
+    }
+}
+
+}  // namespace
+
+template <typename E, int DH>
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constant__ AttnBwdParams p) {
+    constexpr int CPL = DH / 32, EB = sizeof(E);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= p.T) return;
+    const size_t off = ((size_t)bh * p.T + t) * DH * EB + lane * CPL * EB;
+    float q[CPL], o[CPL], g[CPL];
+    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.q) + off, q);
+    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.o) + off, o);
+    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.dO) + off, g);
+    if (p.rope) rope_lane<DH>(p, p.pos0 + t, lane, 1.f, q);
+    RowIO<E, CPL>::store(static_cast<uint8_t *>(p.qh) + off, q);
+    float dot = 0.f;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) dot = fmaf(g[j], o[j], dot);
+    dot = warp_sum(dot);
+    if (lane == 0) p.delta[(size_t)bh * p.T + t] = dot;
+}
+
+template <typename E, int DH>
+__global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const __grid_constant__ AttnBwdParams p) {
+    constexpr int CPL = DH / 32, EB = sizeof(E);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, h = bh % p.H;
+    const int t = blockIdx.x * 8 + warp;
+    if (t >= p.T) return;
+    const int D = p.Dh[h];
+    const int We = p.W > 1 ? p.W : 1;
+    const size_t row = (size_t)bh * p.T;
+    const uint8_t *kb = static_cast<const uint8_t *>(p.k) + row * DH * EB + lane * CPL * EB;
+    const uint8_t *vb = static_cast<const uint8_t *>(p.v) + row * DH * EB + lane * CPL * EB;
+    const size_t off = (row + t) * DH * EB + lane * CPL * EB;
+    float q[CPL], g[CPL];
+    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.qh) + off, q);
+    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.dO) + off, g);
+    const float delta = p.delta[row + t];
+
+    const int w_lo = max(0, t - We + 1);
+    const int n_win = t - w_lo + 1;
+    const int n_dil = t - We + 1 >= D ? (t - We + 1) / D : 0;
+    const int n = n_win + n_dil;
+    auto key = [&](int idx) { return idx < n_win ? w_lo + idx : (idx - n_win) * D + D - 1; };
+
+    // pass 1: the softmax denominator (log2 units)
+    float m = -INFINITY, l = 0.f;
+    for (int base = 0; base < n; base += 4) {
+        float kx[4][CPL];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (base + u < n) RowIO<E, CPL>::load(kb + (size_t)key(base + u) * DH * EB, kx[u]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (base + u < n) {
+                float dot = 0.f;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) dot = fmaf(q[j], kx[u][j], dot);
+                const float s = warp_sum(dot) * p.scale_log2;
+                const float mn = fmaxf(m, s);
+                l = fmaf(l, exp2f(m - mn), exp2f(s - mn));
+                m = mn;
+            }
+        }
+    }
+    const float lse = m + log2f(l);
+    // pass 2: dq^ = scale sum_j p_j (<dO, v_j> - delta) k_j
+    float dq[CPL];
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) dq[j] = 0.f;
+    for (int base = 0; base < n; base += 4) {
+        float kx[4][CPL], vx[4][CPL];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (base + u < n) {
+                const size_t jr = (size_t)key(base + u) * DH * EB;
+                RowIO<E, CPL>::load(kb + jr, kx[u]);
+                RowIO<E, CPL>::load(vb + jr, vx[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (base + u < n) {
+                float sd = 0.f, pd = 0.f;
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) {
+                    sd = fmaf(q[j], kx[u][j], sd);
+                    pd = fmaf(g[j], vx[u][j], pd);
+                }
+                sd = warp_sum(sd);
+                pd = warp_sum(pd);
+                const float pj = exp2f(sd * p.scale_log2 - lse);
+                const float ds = pj * (pd - delta);
+#pragma unroll
+                for (int j = 0; j < CPL; ++j) dq[j] = fmaf(ds, kx[u][j], dq[j]);
+            }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) dq[j] *= p.scale;
+    if (p.rope) rope_lane<DH>(p, p.pos0 + t, lane, -1.f, dq);
+    RowIO<E, CPL>::store(static_cast<uint8_t *>(p.dq) + off, dq);
+    if (lane == 0) p.lse[row + t] = lse;
+}
+
+template <typename E, int DH>
+__global__ void __launch_bounds__(256) attn_bwd_dkv_kernel(const __grid_constant__ AttnBwdParams p) {
+    constexpr int CPL = DH / 32, EB = sizeof(E);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, h = bh % p.H;
+    // key j; the oldest keys, which have the most queries, are in the first CTAs
+    const int j = blockIdx.x * 8 + warp;
+    if (j >= p.T) return;
+    const int D = p.Dh[h];
+    const int We = p.W > 1 ? p.W : 1;
+    const size_t row = (size_t)bh * p.T;
+    const size_t off = (row + j) * DH * EB + lane * CPL * EB;
+    float kx[CPL], vx[CPL];
+    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.k) + off, kx);
+    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.v) + off, vx);
+    const uint8_t *qb = static_cast<const uint8_t *>(p.qh) + row * DH * EB + lane * CPL * EB;
+    const uint8_t *gb = static_cast<const uint8_t *>(p.dO) + row * DH * EB + lane * CPL * EB;
+
+    // queries holding key j: t in [j, j + We - 1] (window), then t >= j + We (chunk end)
+    const int n_win = min(We, p.T - j);
+    const int n_dil = (j % D == D - 1) ? max(0, p.T - (j + We)) : 0;
+    const int n = n_win + n_dil;
+    float dk[CPL], dv[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) { dk[c] = 0.f; dv[c] = 0.f; }
+    for (int base = 0; base < n; base += 4) {
+        float qx[4][CPL], gx[4][CPL], lse[4], dl[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (base + u < n) {
+                const int t = j + base + u;             // both parts are contiguous from j
+                RowIO<E, CPL>::load(qb + (size_t)t * DH * EB, qx[u]);
+                RowIO<E, CPL>::load(gb + (size_t)t * DH * EB, gx[u]);
+                lse[u] = p.lse[row + t];
+                dl[u] = p.delta[row + t];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (base + u < n) {
+                float sd = 0.f, pd = 0.f;
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    sd = fmaf(qx[u][c], kx[c], sd);
+                    pd = fmaf(gx[u][c], vx[c], pd);
+                }
+                sd = warp_sum(sd);
+                pd = warp_sum(pd);
+                const float pj = exp2f(sd * p.scale_log2 - lse[u]);
+                const float ds = pj * (pd - dl[u]);
+#pragma unroll
+                for (int c = 0; c < CPL; ++c) {
+                    dk[c] = fmaf(ds, qx[u][c], dk[c]);
+                    dv[c] = fmaf(pj, gx[u][c], dv[c]);
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) dk[c] *= p.scale;
+    RowIO<E, CPL>::store(static_cast<uint8_t *>(p.dk) + off, dk);
+    RowIO<E, CPL>::store(static_cast<uint8_t *>(p.dv) + off, dv);
+}
+
+size_t attn_bwd_workspace_bytes(int B, int H, int T, int d, int dtype) {
+    const size_t rows = (size_t)B * H * T;
+    return sizeof(WsHeader) + align256(rows * d * (dtype == RAT_F32 ? 4 : 2)) + 2 * align256(rows * 4);
+}
+
+template <typename E, int DH>
+static int launch_bwd(const AttnBwdParams &p, cudaStream_t s) {
+    dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)(p.B * p.H));
+    attn_bwd_prep_kernel<E, DH><<<grid, 256, 0, s>>>(p);
+    attn_bwd_dq_kernel<E, DH><<<grid, 256, 0, s>>>(p);
+    attn_bwd_dkv_kernel<E, DH><<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
+}
+
+int launch_attn_bwd(const AttnBwdParams &p, int dtype, void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (dtype == RAT_F32) {
+        if (p.d == 64) return launch_bwd<float, 64>(p, s);
+        if (p.d == 128) return launch_bwd<float, 128>(p, s);
+    } else {
+        if (p.d == 64) return launch_bwd<__nv_bfloat16, 64>(p, s);
+        if (p.d == 128) return launch_bwd<__nv_bfloat16, 128>(p, s);
+    }
+    return RAT_ERR_UNSUPPORTED;
+}
+
+}  // namespace rat

@@ -102,6 +102,51 @@ template <> struct Lane<__nv_bfloat16> {
     }
 };
 
+// CPL consecutive channels of one row per lane (the CUDA-core attention kernels), as floats.
+template <typename E, int CPL> struct RowIO;
+template <> struct RowIO<float, 2> {
+    static RAT_DEVICE void load(const void *p, float *x) {
+        const float2 v = __ldg(reinterpret_cast<const float2 *>(p));
+        x[0] = v.x; x[1] = v.y;
+    }
+    static RAT_DEVICE void store(void *p, const float *x) {
+        *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+    }
+};
+template <> struct RowIO<float, 4> {
+    static RAT_DEVICE void load(const void *p, float *x) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(p));
+        x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+    }
+    static RAT_DEVICE void store(void *p, const float *x) {
+        *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+};
+template <> struct RowIO<__nv_bfloat16, 2> {
+    static RAT_DEVICE void load(const void *p, float *x) {
+        const uint32_t u = __ldg(reinterpret_cast<const unsigned int *>(p));
+        x[0] = bf16_lo(u); x[1] = bf16_hi(u);
+    }
+    static RAT_DEVICE void store(void *p, const float *x) {
+        *reinterpret_cast<uint32_t *>(p) = pack_bf16(x[0], x[1]);
+    }
+};
+template <> struct RowIO<__nv_bfloat16, 4> {
+    static RAT_DEVICE void load(const void *p, float *x) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+        x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+    }
+    static RAT_DEVICE void store(void *p, const float *x) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]));
+    }
+};
+
+RAT_DEVICE float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
 // ------------------------------------------------------------------------------ math
 // 2^x and 1/x from the special-function unit (PTX ex2.approx / rcp.approx, flush-to-zero).
 RAT_DEVICE float ex2_approx(float x) {

@@ -162,6 +162,23 @@ struct CompressParams {
 };
 int launch_compress(const CompressParams &p, void *stream);
 
+// backward of the dilated attention (CUDA cores, float32 accumulation)
+struct AttnBwdParams {
+    const void *q, *k, *v, *o, *dO;
+    void *dq, *dk, *dv;
+    void *qh;                   // workspace [B*H][T][d] of dtype: RoPE(q) as the attention uses it
+    float *lse;                 // workspace [B*H][T]: log2 of each query's softmax denominator
+    float *delta;               // workspace [B*H][T]: <dO_t, o_t>
+    int B, H, T, d, W;
+    long long pos0;
+    int rope;
+    float scale, scale_log2;
+    int Dh[kMaxHeads];
+    double theta[64];
+};
+size_t attn_bwd_workspace_bytes(int B, int H, int T, int d, int dtype);
+int launch_attn_bwd(const AttnBwdParams &p, int dtype, void *stream);
+
 struct DecodeParams {
     const void *q, *k, *v, *a;
     void *o;

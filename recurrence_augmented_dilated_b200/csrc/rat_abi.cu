@@ -337,6 +337,51 @@ int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec
     return launch_attn_simt(p, dtype, stream);
 }
 
+size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int dtype) {
+    if (B < 1 || H < 1 || T < 0 || !supported_d(d) || !valid_dtype(dtype)) return 0;
+    return attn_bwd_workspace_bytes(B, H, T, d, dtype);
+}
+
+int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_rec, const void *o,
+                              const void *dO, void *dq, void *dk_rec, void *dv_rec, int B, int H,
+                              int T, int d, int dtype, int D, int W, const int32_t *D_per_head,
+                              int64_t pos0, float rope_base, float scale, void *ws,
+                              size_t ws_bytes, void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0) return RAT_ERR_INVALID;
+    if (!supported_d(d) || H > kMaxHeads) return RAT_ERR_UNSUPPORTED;
+    if (!std::isfinite(rope_base) || !std::isfinite(scale)) return RAT_ERR_INVALID;
+    if (!D_per_head && D < 1) return RAT_ERR_INVALID;
+    if (D_per_head)
+        for (int h = 0; h < H; ++h)
+            if (D_per_head[h] < 1) return RAT_ERR_INVALID;
+    if (T == 0) return RAT_OK;
+    const void *req[] = {q, k_rec, v_rec, o, dO, dq, dk_rec, dv_rec};
+    for (const void *x : req)
+        if (!x || !aligned16(x)) return RAT_ERR_INVALID;
+    if ((long long)B * H > 65535 || T > (1 << 30)) return RAT_ERR_UNSUPPORTED;
+    const size_t need = attn_bwd_workspace_bytes(B, H, T, d, dtype);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RAT_ERR_WORKSPACE;
+    AttnBwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = q; p.k = k_rec; p.v = v_rec; p.o = o; p.dO = dO;
+    p.dq = dq; p.dk = dk_rec; p.dv = dv_rec;
+    const size_t rows = (size_t)B * H * T;
+    uint8_t *w = static_cast<uint8_t *>(ws) + sizeof(WsHeader);
+    p.qh = w;
+    w += align256(rows * d * (dtype == RAT_F32 ? 4 : 2));
+    p.lse = reinterpret_cast<float *>(w);
+    w += align256(rows * 4);
+    p.delta = reinterpret_cast<float *>(w);
+    p.B = B; p.H = H; p.T = T; p.d = d; p.W = W;
+    p.pos0 = pos0;
+    p.rope = rope_base > 0.f ? 1 : 0;
+    p.scale = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)d));
+    p.scale_log2 = p.scale * 1.4426950408889634f;
+    for (int h = 0; h < H; ++h) p.Dh[h] = D_per_head ? D_per_head[h] : D;
+    if (p.rope) rope_theta(rope_base, d, p.theta);
+    return launch_attn_bwd(p, dtype, stream);
+}
+
 int rat_attn_sync_status(void *stream) { return attn_error_word(stream, true); }
 
 uint32_t rat_attn_error_site(void) { return attn_error_where(); }

@@ -1,0 +1,68 @@
+"""GPU parity of rat_dilated_attn_backward (gradients of the dilated attention) against the
+float64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import recurrence_augmented_dilated_b200 as rat
+import synthetic
+from gpu_util import TOL_BF16, TOL_F32, f64, gpu_attn, rel_err, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def run(B, H, T, d, dtype, D=1, W=0, D_per_head=None, rope_base=0.0, pos0=0, seed=0, heads=None,
+        x=None):
+    if x is None:
+        w = synthetic.Workload("ab", B=B, H=H, d=d, T=T, dtype="f32" if dtype == torch.float32 else "bf16",
+                               seed=seed)
+        x = synthetic.prefill_inputs(w)
+    dev = torch.device("cuda")
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))     # k, v stand in for k~, v~
+    g = torch.Generator().manual_seed(seed + 1)
+    dO = torch.randn(q.shape, generator=g).to(dtype)
+    o = gpu_attn(q, k, v, D=D, W=W, D_per_head=D_per_head, rope_base=rope_base, pos0=pos0)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = rat.Workspace(rat.rat_dilated_attn_backward_workspace_bytes(B, H, T, d, 0 if dtype == torch.float32 else 1))
+    rat.rat_dilated_attn_backward(q, k, v, o, dO.to(dev), dq, dk, dv, ws, D=D, W=W,
+                                  D_per_head=D_per_head, pos0=pos0, rope_base=rope_base)
+    torch.cuda.synchronize()
+    sel = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    errs = {}
+    for b, h in sel:
+        Dh = [D_per_head[h]] if D_per_head is not None else None
+        ref = oracle.dilated_attention_backward(
+            f64(x["q"][b:b + 1, h:h + 1]), f64(x["k"][b:b + 1, h:h + 1]), f64(x["v"][b:b + 1, h:h + 1]),
+            f64(dO[b:b + 1, h:h + 1]), D=D, W=W, D_per_head=Dh, rope_base=rope_base, pos0=pos0)
+        for n, got, r in zip(("dq", "dk", "dv"), (dq, dk, dv), ref):
+            errs[(b, h, n)] = rel_err(got[b, h], r[0, 0])
+    tol = tol_for(dtype)
+    worst = max(errs.values())
+    assert worst <= tol, {k_: v_ for k_, v_ in errs.items() if v_ > tol}
+    return worst
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("D,W", [(1, 0), (4, 0), (16, 0), (4, 8), (64, 128), (7, 3)])
+def test_attention_backward_key_sets(dtype, d, D, W):
+    run(1, 2, 300, d, dtype, D=D, W=W, seed=D * 10 + W)
+
+
+@pytest.mark.parametrize("T", [1, 2, 65, 129])
+def test_attention_backward_short_and_ragged(T):
+    run(2, 2, T, 128, torch.bfloat16, D=4, W=2, seed=T)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_attention_backward_rope_and_head_hybrid(dtype):
+    run(1, 4, 257, 128, dtype, D_per_head=[1, 4, 16, 64], W=8, rope_base=10000.0, pos0=4000, seed=3)
+
+
+def test_attention_backward_full_size_sampled_heads():
+    # the prefill_1p5b workload (B 4, H 16, T 4096, d 128, D 16, RoPE), two heads checked whole
+    w = synthetic.WORKLOADS["prefill_1p5b"]
+    x = synthetic.prefill_inputs(w)
+    run(w.B, w.H, w.T, w.d, torch.bfloat16, D=w.D, W=w.W, rope_base=w.rope_base, x=x,
+        heads=[(0, 0), (w.B - 1, w.H - 1)], seed=5)
