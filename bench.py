@@ -645,12 +645,46 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     eb = 2 if w.dtype == "bf16" else 4
     nbytes = 10 * B * H * T * d * eb       # read k, v, a, k~, v~, dk~, dv~; write dk, dv, da
     achieved = nbytes / (ms * 1e-3) / 1e9
-    return {"workload": w.name, "step": "rat_recur_backward (3 launches)", "ms": ms,
-            "tokens_per_s": world * B * T / (ms * 1e-3),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "of": peak_kind,
-                         "algorithmic_bytes": nbytes},
-            "clocks": clk.summary(), "gpu_launches": 3 * steps}
+    res = {"workload": w.name, "step": "rat_recur_backward (3 launches)", "ms": ms,
+           "tokens_per_s": world * B * T / (ms * 1e-3),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "of": peak_kind,
+                        "algorithmic_bytes": nbytes},
+           "clocks": clk.summary(), "gpu_launches": 3 * steps}
+    # attention backward on the same shapes: q, k~, v~, o, dO resident
+    q = x["q"].to(dev)
+    o = torch.empty_like(q)
+    Dph = list(w.D_per_head) if w.D_per_head else None
+    rat.rat_dilated_attn_prefill(q, kr, vr, o, D=w.D, W=w.W, D_per_head=Dph, rope_base=w.rope_base)
+    dO = torch.randn(q.shape, generator=g, device=dev).to(q.dtype)
+    dq, dkr, dvr = torch.empty_like(q), torch.empty_like(kr), torch.empty_like(vr)
+    ws_a = rat.Workspace(rat.rat_dilated_attn_backward_workspace_bytes(B, H, T, d, dtc))
+
+    def astep():
+        rat.rat_dilated_attn_backward(q, kr, vr, o, dO, dq, dkr, dvr, ws_a, D=w.D, W=w.W,
+                                      D_per_head=Dph, rope_base=w.rope_base)
+
+    for _ in range(warmup):
+        astep()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0.record(stream)
+    for _ in range(steps):
+        astep()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ams = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+    abytes = 8 * B * H * T * d * eb        # read q, k~, v~, o, dO; write dq, dk~, dv~
+    pairs = sum(rat.rat_attended_keys(t, D_, w.W) for D_ in w.heads_D() for t in range(T)) * B
+    aflops = 10 * d * pairs                 # per pair: recomputed score, dp, dq, dk, dv
+    a_ach = abytes / (ams * 1e-3) / 1e9
+    res["attention"] = {"step": "rat_dilated_attn_backward (3 CUDA-core launches)", "ms": ams,
+                        "roofline": {"bound": "hbm", "achieved": a_ach, "peak": peaks["hbm_gbs"],
+                                     "unit": "GB/s", "frac": a_ach / peaks["hbm_gbs"],
+                                     "of": peak_kind, "algorithmic_bytes": abytes,
+                                     "tflops": aflops / (ams * 1e-3) / 1e12},
+                        "gpu_launches": 3 * steps}
+    return res
 
 
 # ----------------------------------------------------------------------------- oracle (CPU)
