@@ -15,6 +15,8 @@
 
 namespace rat {
 
+// PAGED: the paged form (one sequence per call, dil entries through the page table)
+template <bool PAGED>
 __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ CompressParams p) {
     // flat grid: per batch row, head h owns CTAs blk0[h] .. blk0[h+1]-1
     const int per_b = p.blk0[p.H];
@@ -22,7 +24,7 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
     int h = 0;
     while (rb >= p.blk0[h + 1]) ++h;
     const int bh = b * p.H + h;                                  // input slice
-    const bool paged = p.page_table != nullptr;
+    constexpr bool paged = PAGED;
     const int bhc = paged ? p.seq * p.H + h : bh;                // cache slice
     const int blk = rb - p.blk0[h], nblk = p.blk0[h + 1] - p.blk0[h];
     const long long D = p.Dh[h];
@@ -50,7 +52,7 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
             const long long i = i_lo + r;
             pos = i * D + D - 1;
             uint8_t *base = static_cast<uint8_t *>(is_v ? p.vdil : p.kdil);
-            if (paged) {
+            if constexpr (PAGED) {
                 const int32_t pg = p.page_table[(size_t)bhc * p.max_pages + (i >> p.page_shift)];
                 if ((uint32_t)pg < (uint32_t)p.n_pages) {
                     dst = base + (((size_t)pg << p.page_shift) + (size_t)(i & ((1ll << p.page_shift) - 1))) * row_bytes;
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
             if (job < njobs) {
                 const uint8_t *src;
                 locate(job, src, dst[u]);
-                if (dst[u]) val[u] = *reinterpret_cast<const uint4 *>(src + lane_c * 16);
+                if (!PAGED || dst[u]) val[u] = *reinterpret_cast<const uint4 *>(src + lane_c * 16);
             }
         }
 #pragma unroll
@@ -117,7 +119,8 @@ int launch_compress(const CompressParams &p_in, void *stream) {
     p.blk0[p.H] = acc;
     const long long grid = (long long)acc * p.B;
     if (grid > 0x7fffffffll) return RAT_ERR_UNSUPPORTED;
-    compress_kernel<<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    if (p.page_table) compress_kernel<true><<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+    else compress_kernel<false><<<(unsigned)grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 
