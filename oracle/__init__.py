@@ -50,7 +50,7 @@ def _load():
         lib.rat_oracle_recurrence_reset.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _L, _L]
         lib.rat_oracle_recurrence_window.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _L, _dp]
         lib.rat_oracle_dilated_attention_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp,
-                                                              _ip, _L, ctypes.c_double, _dp,
+                                                              _ip, _L, _L, ctypes.c_double, _dp,
                                                               _dp, _dp]
         lib.rat_oracle_recurrence_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _dp,
                                                        _dp, _dp]
@@ -59,10 +59,14 @@ def _load():
         lib.rat_oracle_in_key_set.restype = ctypes.c_int
         lib.rat_oracle_key_count.argtypes = [_L, _L, _L]
         lib.rat_oracle_key_count.restype = ctypes.c_long
-        lib.rat_oracle_dilated_attention.argtypes = [_L, _L, _L, _dp, _dp, _dp, _ip, _L,
+        lib.rat_oracle_in_key_set_sinks.argtypes = [_L, _L, _L, _L, _L]
+        lib.rat_oracle_in_key_set_sinks.restype = ctypes.c_int
+        lib.rat_oracle_key_count_sinks.argtypes = [_L, _L, _L, _L]
+        lib.rat_oracle_key_count_sinks.restype = ctypes.c_long
+        lib.rat_oracle_dilated_attention.argtypes = [_L, _L, _L, _dp, _dp, _dp, _ip, _L, _L,
                                                      ctypes.c_double, _lp, _L, _dp]
         lib.rat_oracle_kv_compress.argtypes = [_L, _L, _L, _L, _L, _bp, _ip, _L, _L, _L, _bp, _bp]
-        lib.rat_oracle_decode_step.argtypes = [_L, _L, _L, _ip, _L, ctypes.c_double,
+        lib.rat_oracle_decode_step.argtypes = [_L, _L, _L, _ip, _L, _L, ctypes.c_double,
                                                ctypes.c_double, _dp, _dp, _dp, _dp, _dp, _dp,
                                                _dp, _dp, _L, _dp]
         lib.rat_oracle_threads.restype = ctypes.c_int
@@ -202,13 +206,18 @@ def recurrence_layer_backward(k, v, a, dk_rec, dv_rec, h0k=None, h0v=None, dhTk=
     return dk, dv, g * omg * (dgk + dgv), dh0k, dh0v
 
 
-def in_key_set(t: int, j: int, D: int, W: int) -> bool:
-    """Is key j in the key set of query t (window (t-We, t] union chunk ends older than it)?"""
+def in_key_set(t: int, j: int, D: int, W: int, n_sink: int = 0) -> bool:
+    """Is key j in the key set of query t (window (t-We, t] union chunk ends older than it,
+    union the first n_sink positions)?"""
+    if n_sink:
+        return bool(_load().rat_oracle_in_key_set_sinks(int(t), int(j), int(D), int(W), int(n_sink)))
     return bool(_load().rat_oracle_in_key_set(int(t), int(j), int(D), int(W)))
 
 
-def key_count(t: int, D: int, W: int) -> int:
+def key_count(t: int, D: int, W: int, n_sink: int = 0) -> int:
     """|S(t)| by enumeration."""
+    if n_sink:
+        return int(_load().rat_oracle_key_count_sinks(int(t), int(D), int(W), int(n_sink)))
     return int(_load().rat_oracle_key_count(int(t), int(D), int(W)))
 
 
@@ -222,12 +231,14 @@ def _per_bh_dilation(shape_bh, D, D_per_head):
     return np.ascontiguousarray(np.tile(Dh, B).astype(np.int32)), Dh
 
 
-def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None):
+def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None, n_sink=0):
     """Causal dilated attention (+ local window, per-head D) over (B, H, T, d) tensors.
 
     q, k, v are used as given (rotate them first if RoPE is in use).  rows: optional list of
-    query positions; the result then has shape (B, H, len(rows), d).
-    (RAT+ abstract; "RAT+ Deep Dive" section 3.1 table and section 6 head-wise hybrid.)
+    query positions; the result then has shape (B, H, len(rows), d).  n_sink > 0 adds the first
+    n_sink positions to every key set (StreamingLLM attention sinks).
+    (RAT+ abstract; "RAT+ Deep Dive" section 3.1 table and section 6 head-wise and layer-wise
+    hybrids.)
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, T, d = q.shape
@@ -243,12 +254,12 @@ def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None)
         nrows, rp = len(rows_a), _ptr(rows_a, _lp)
         out = np.empty((B, H, nrows, d))
     _load().rat_oracle_dilated_attention(B * H, T, d, _ptr(q), _ptr(k), _ptr(v), _ptr(Dbh, _ip),
-                                         int(W), float(scale), rp, nrows, _ptr(out))
+                                         int(W), int(n_sink), float(scale), rp, nrows, _ptr(out))
     return out
 
 
 def dilated_attention_backward(q, k, v, dO, D=1, W=0, D_per_head=None, scale=None,
-                               rope_base=0.0, pos0=0):
+                               rope_base=0.0, pos0=0, n_sink=0):
     """Reverse-mode derivative of dilated_attention for upstream gradients dO: returns
     (dq, dk, dv) in float64.  With rope_base > 0, q is rotated at positions pos0 + t first (as
     the attention does) and dq is the gradient with respect to the unrotated q (RoPE^T applied);
@@ -261,7 +272,8 @@ def dilated_attention_backward(q, k, v, dO, D=1, W=0, D_per_head=None, scale=Non
     qh = rope(q, pos0, rope_base) if rope_base > 0 else q
     dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
     _load().rat_oracle_dilated_attention_backward(B * H, T, d, _ptr(qh), _ptr(k), _ptr(v),
-                                                  _ptr(dO), _ptr(Dbh, _ip), int(W), float(scale),
+                                                  _ptr(dO), _ptr(Dbh, _ip), int(W), int(n_sink),
+                                                  float(scale),
                                                   _ptr(dq), _ptr(dk), _ptr(dv))
     if rope_base > 0:
         dq = rope_transpose(dq, pos0, rope_base)
@@ -269,7 +281,7 @@ def dilated_attention_backward(q, k, v, dO, D=1, W=0, D_per_head=None, scale=Non
 
 
 def layer_prefill(q, k, v, a, D=1, W=0, D_per_head=None, rope_base=0.0, pos0=0, scale=None,
-                  rows=None, h0_k=None, h0_v=None, reset_every=0):
+                  rows=None, h0_k=None, h0_v=None, reset_every=0, n_sink=0):
     """The whole prefill path in float64: recurrence -> RoPE -> dilated attention.
 
     Returns dict(o, k_rec, v_rec, hT_k, hT_v); k_rec is the recurrence output after RoPE
@@ -282,7 +294,8 @@ def layer_prefill(q, k, v, a, D=1, W=0, D_per_head=None, rope_base=0.0, pos0=0, 
     if rope_base > 0:
         k_rec = rope(k_rec, pos0, rope_base)
         qr = rope(qr, pos0, rope_base)
-    o = dilated_attention(qr, k_rec, v_rec, D=D, W=W, D_per_head=D_per_head, scale=scale, rows=rows)
+    o = dilated_attention(qr, k_rec, v_rec, D=D, W=W, D_per_head=D_per_head, scale=scale, rows=rows,
+                          n_sink=n_sink)
     return dict(o=o, k_rec=k_rec, v_rec=v_rec, hT_k=hT_k, hT_v=hT_v)
 
 
@@ -320,7 +333,7 @@ class DecodeState:
     """
 
     def __init__(self, Dbh, d: int, W: int, Tcap: int, rope_base: float = 0.0, scale=None,
-                 reset_every: int = 0):
+                 reset_every: int = 0, n_sink: int = 0):
         self.Dbh = np.ascontiguousarray(np.asarray(Dbh, dtype=np.int32))
         self.BH = len(self.Dbh)
         self.d, self.W, self.Tcap = d, int(W), int(Tcap)
@@ -332,6 +345,7 @@ class DecodeState:
         self.vhist = np.zeros((self.BH, self.Tcap, d))
         self.t = 0
         self.reset_every = int(reset_every)     # > 0: chunk-local recurrence (state zeroed at t % L == 0)
+        self.n_sink = int(n_sink)               # attention sinks: the first n_sink positions
 
     def prefill(self, k, v, a):
         """Consume a context (BH, T, d) with the sequential recurrence and record history."""
@@ -354,7 +368,7 @@ class DecodeState:
             self.hv[:] = 0.0
         o = np.empty((self.BH, self.d))
         _load().rat_oracle_decode_step(self.BH, self.d, self.t, _ptr(self.Dbh, _ip), self.W,
-                                       self.scale, self.rope_base, _ptr(q), _ptr(k), _ptr(v),
+                                       self.n_sink, self.scale, self.rope_base, _ptr(q), _ptr(k), _ptr(v),
                                        _ptr(a), _ptr(self.hk), _ptr(self.hv), _ptr(self.khist),
                                        _ptr(self.vhist), self.Tcap, _ptr(o))
         self.t += 1

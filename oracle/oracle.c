@@ -204,22 +204,47 @@ void rat_oracle_rope(long BH, long T, long d, double *x, long pos0, double base)
 static long eff_window(long W) { return W > 1 ? W : 1; }
 
 /*
- * Membership of key j in the key set of query t (the definition, as a predicate).
+ * Membership of key j in the key set of query t (the definition, as a predicate), with
+ * n_sink attention sinks: the first n_sink positions, always attended (StreamingLLM layers,
+ * "RAT+ Deep Dive" section 6 layer-wise hybrid).  n_sink = 0 is the RAT+ key set.
  *                                                     [RAT+ abstract; RAT+ Deep Dive 3.1, 6]
  */
-int rat_oracle_in_key_set(long t, long j, long D, long W)
+int rat_oracle_in_key_set_sinks(long t, long j, long D, long W, long n_sink)
 {
     long We = eff_window(W);
     if (j < 0 || j > t) return 0;
     if (j > t - We) return 1;            /* local window, the query's own position included */
+    if (j < n_sink) return 1;            /* attention sink                                   */
     return (j % D) == (D - 1);           /* dilated key: a chunk end older than the window  */
 }
 
+int rat_oracle_in_key_set(long t, long j, long D, long W)
+{
+    return rat_oracle_in_key_set_sinks(t, j, D, W, 0);
+}
+
 /* |S(t)|: number of keys query t attends to, counted by enumerating the set.                */
-long rat_oracle_key_count(long t, long D, long W)
+long rat_oracle_key_count_sinks(long t, long D, long W, long n_sink)
 {
     long n = 0;
-    for (long j = 0; j <= t; ++j) n += rat_oracle_in_key_set(t, j, D, W);
+    for (long j = 0; j <= t; ++j) n += rat_oracle_in_key_set_sinks(t, j, D, W, n_sink);
+    return n;
+}
+
+long rat_oracle_key_count(long t, long D, long W) { return rat_oracle_key_count_sinks(t, D, W, 0); }
+
+/*
+ * S(t) listed in the order the loops below use: the window t-We < j <= t, then the chunk ends
+ * j = D-1, 2D-1, ... with j <= t-We, then the sinks j < n_sink older than the window that are not
+ * chunk ends (each key once).  Returns |S(t)|.
+ */
+static long list_keys(long t, long D, long We, long n_sink, long *keys)
+{
+    long n = 0;
+    for (long j = (t - We + 1 > 0 ? t - We + 1 : 0); j <= t; ++j) keys[n++] = j;
+    for (long j = D - 1; j <= t - We; j += D) keys[n++] = j;
+    for (long j = 0; j < n_sink && j <= t - We; ++j)
+        if (j % D != D - 1) keys[n++] = j;
     return n;
 }
 
@@ -237,8 +262,8 @@ long rat_oracle_key_count(long t, long D, long W)
  * j = D-1, 2D-1, ... with j <= t - We.
  */
 void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, const double *k,
-                                  const double *v, const int *Dbh, long W, double scale,
-                                  const long *rows, long nrows, double *o)
+                                  const double *v, const int *Dbh, long W, long n_sink,
+                                  double scale, const long *rows, long nrows, double *o)
 {
     long We = eff_window(W);
     if (!rows) nrows = T;
@@ -249,9 +274,7 @@ void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, cons
         double *s = (double *)malloc(sizeof(double) * (size_t)(T + 1));
         for (long r = 0; r < nrows; ++r) {
             long t = rows ? rows[r] : r;
-            long n = 0;
-            for (long j = (t - We + 1 > 0 ? t - We + 1 : 0); j <= t; ++j) keys[n++] = j;
-            for (long j = D - 1; j <= t - We; j += D) keys[n++] = j;
+            long n = list_keys(t, D, We, n_sink, keys);
             const double *qt = q + (bh * T + t) * d;
             double mx = -INFINITY;
             for (long m = 0; m < n; ++m) {
@@ -288,8 +311,8 @@ void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, cons
  */
 void rat_oracle_dilated_attention_backward(long BH, long T, long d, const double *q,
                                            const double *k, const double *v, const double *dO,
-                                           const int *Dbh, long W, double scale, double *dq,
-                                           double *dk, double *dv)
+                                           const int *Dbh, long W, long n_sink, double scale,
+                                           double *dq, double *dk, double *dv)
 {
     long We = eff_window(W);
 #pragma omp parallel for schedule(dynamic, 1)
@@ -299,9 +322,7 @@ void rat_oracle_dilated_attention_backward(long BH, long T, long d, const double
         double *p = (double *)malloc(sizeof(double) * (size_t)(T + 1));
         double *ot = (double *)malloc(sizeof(double) * (size_t)d);
         for (long t = 0; t < T; ++t) {
-            long n = 0;
-            for (long j = (t - We + 1 > 0 ? t - We + 1 : 0); j <= t; ++j) keys[n++] = j;
-            for (long j = D - 1; j <= t - We; j += D) keys[n++] = j;
+            long n = list_keys(t, D, We, n_sink, keys);
             const double *qt = q + (bh * T + t) * d;
             const double *gt = dO + (bh * T + t) * d;
             double mx = -INFINITY;
@@ -393,7 +414,8 @@ void rat_oracle_kv_compress(long B, long H, long T, long d, long esize, const ui
  * State update h = g*h + (1-g)*x for k and v; k~_t = RoPE(h_k, t) (if rope_base > 0); the
  * query is RoPE(q, t); attention over S(t) exactly as in the prefill definition.
  */
-void rat_oracle_decode_step(long BH, long d, long t, const int *Dbh, long W, double scale,
+void rat_oracle_decode_step(long BH, long d, long t, const int *Dbh, long W, long n_sink,
+                            double scale,
                             double rope_base, const double *q, const double *k, const double *v,
                             const double *a, double *hk, double *hv, double *khist,
                             double *vhist, long Tcap, double *o)
@@ -428,11 +450,10 @@ void rat_oracle_decode_step(long BH, long d, long t, const int *Dbh, long W, dou
                 qr[c + half] = x2 * cs + x1 * sn;
             }
         }
-        long nmax = We + t / D + 2, n = 0;
+        long nmax = We + t / D + n_sink + 2;
         long *keys = (long *)malloc(sizeof(long) * (size_t)nmax);
         double *s = (double *)malloc(sizeof(double) * (size_t)nmax);
-        for (long j = (t - We + 1 > 0 ? t - We + 1 : 0); j <= t; ++j) keys[n++] = j;
-        for (long j = D - 1; j <= t - We; j += D) keys[n++] = j;
+        long n = list_keys(t, D, We, n_sink, keys);
         double mx = -INFINITY;
         for (long m = 0; m < n; ++m) {
             const double *kj = khist + (bh * Tcap + keys[m]) * d;

@@ -415,6 +415,54 @@ def test_attention_backward_single_key_passes_dv_only():
     assert np.all(dq == 0.0) and np.all(dk == 0.0)
 
 
+# ---- attention sinks (StreamingLLM layers)
+@pytest.mark.parametrize("D,W,n_sink", [(10**6, 8, 4), (10**6, 1, 3), (4, 0, 6), (3, 5, 7)])
+def test_sink_key_count_closed_form(D, W, n_sink):
+    We = max(W, 1)
+    for t in range(60):
+        lim = min(n_sink, max(0, t - We + 1))          # sinks older than the window
+        dil = max(0, (t - We + 1) // D) if t - We + 1 >= D else 0
+        want = min(We, t + 1) + dil + lim - lim // D    # sinks that are chunk ends count once
+        assert oracle.key_count(t, D, W, n_sink) == want, (t, D, W, n_sink)
+
+
+def test_streaming_attention_equals_masked_sdpa():
+    # no chunk ends (D beyond T): the key set is the window plus the first n_sink positions
+    import torch
+    B, H, T, d, W, n_sink = 1, 2, 40, 8, 6, 4
+    q, k, v = (RNG.standard_normal((B, H, T, d)) for _ in range(3))
+    o = oracle.dilated_attention(q, k, v, D=10**6, W=W, n_sink=n_sink, scale=0.3)
+    t_ = torch.arange(T)[:, None]
+    j_ = torch.arange(T)[None, :]
+    mask = (j_ <= t_) & ((j_ > t_ - W) | (j_ < n_sink))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q), torch.tensor(k), torch.tensor(v), attn_mask=mask, scale=0.3)
+    np.testing.assert_allclose(o, ref.numpy(), rtol=1e-11, atol=1e-12)
+
+
+def test_sinks_that_are_chunk_ends_change_nothing():
+    # D = 1: every position is already a chunk end, so sinks add no key
+    q, k, v = (RNG.standard_normal((1, 2, 30, 4)) for _ in range(3))
+    a = oracle.dilated_attention(q, k, v, D=1, W=3)
+    b = oracle.dilated_attention(q, k, v, D=1, W=3, n_sink=5)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_decode_with_sinks_equals_prefill_rows():
+    T0, steps, d, W, n_sink = 20, 15, 8, 3, 4
+    Dh = [1, 4, 10**6]
+    H = len(Dh)
+    T = T0 + steps
+    q, k, v, a = (RNG.standard_normal((1, H, T, d)) for _ in range(4))
+    full = oracle.layer_prefill(q, k, v, a, D_per_head=Dh, W=W, rope_base=100.0, n_sink=n_sink)["o"]
+    st = oracle.DecodeState(Dh, d, W, T, rope_base=100.0, n_sink=n_sink)
+    st.prefill(k[0, :, :T0], v[0, :, :T0], a[0, :, :T0])
+    for s_ in range(steps):
+        t = T0 + s_
+        o = st.step(q[0, :, t], k[0, :, t], v[0, :, t], a[0, :, t])
+        np.testing.assert_allclose(o, full[0, :, t], rtol=1e-10, atol=1e-12)
+
+
 def test_rope_matches_complex_rotation():
     d, T, pos0, base = 16, 9, 1000, 10000.0
     x = RNG.standard_normal((1, T, d))
