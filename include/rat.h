@@ -240,6 +240,19 @@ RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const voi
                              const int32_t *D_per_head, int64_t pos0, float rope_base,
                              float scale, void *stream);
 
+/* rat_dilated_attn_prefill_sinks -- the same attention with attention sinks: the first n_sink
+ * positions join every key set (StreamingLLM layers; "RAT+ Deep Dive" section 6, layer-wise
+ * hybrid: "odd layers StreamingLLM").  Each key counts once (a sink already in the window or a
+ * chunk end is not repeated).  A StreamingLLM layer is D larger than any position (no chunk
+ * ends), W its window, n_sink its sinks; sinks also combine with dilation.
+ *   Arguments as rat_dilated_attn_prefill, plus n_sink >= 0 (0: exactly
+ *   rat_dilated_attn_prefill).  Calls with n_sink > 0 run the CUDA-core kernel (float32
+ *   arithmetic) for both dtypes. */
+RAT_API int rat_dilated_attn_prefill_sinks(const void *q, const void *k_rec, const void *v_rec,
+                             void *o, int B, int H, int T, int d, int dtype, int D, int W,
+                             const int32_t *D_per_head, int n_sink, int64_t pos0,
+                             float rope_base, float scale, void *stream);
+
 /* Synchronise `stream`, then return (and clear) the first device-side error recorded by the
  * attention kernel since the last call (RAT_OK if none). */
 RAT_API int rat_attn_sync_status(void *stream);
@@ -256,7 +269,8 @@ RAT_API int rat_attn_sync_status(void *stream);
  *   dO                 : device (B, H, T, d) of dtype     upstream gradient of o
  *   dq, dk_rec, dv_rec : device (B, H, T, d) of dtype     outputs (dk_rec, dv_rec are the
  *                        gradients of k~, v~: the dk_rec, dv_rec inputs of rat_recur_backward)
- *   D, W, D_per_head, pos0, rope_base, scale : as given to rat_dilated_attn_prefill
+ *   D, W, D_per_head, n_sink, pos0, rope_base, scale : as given to the forward
+ *                        (rat_dilated_attn_prefill_sinks; n_sink = 0 without sinks)
  *   ws, ws_bytes       : workspace of at least rat_dilated_attn_backward_workspace_bytes
  * CUDA-core kernels with float32 accumulation: the softmax denominators are recomputed (not
  * taken from the forward), q^ is rounded to the dtype as the forward's operand is, outputs are
@@ -267,8 +281,9 @@ RAT_API size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, in
 RAT_API int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_rec,
                               const void *o, const void *dO, void *dq, void *dk_rec,
                               void *dv_rec, int B, int H, int T, int d, int dtype, int D, int W,
-                              const int32_t *D_per_head, int64_t pos0, float rope_base,
-                              float scale, void *ws, size_t ws_bytes, void *stream);
+                              const int32_t *D_per_head, int n_sink, int64_t pos0,
+                              float rope_base, float scale, void *ws, size_t ws_bytes,
+                              void *stream);
 
 /* Diagnostic: where the attention kernel's last recorded timeout happened, as
  * (wait site << 24) | (key block << 8) | phase parity; sites: 1 producer K-stage-free, 2 MMA
@@ -297,6 +312,8 @@ RAT_API int rat_set_attn_block_keys(int block_keys);
  *   h_k, h_v     : device [B][H][d] float32 recurrence state after the last position
  *                  (before RoPE)
  *   pos          : number of positions consumed so far (the same for every sequence)
+ *   k_sink, v_sink : device [B][H][n_sink][d] of dtype: positions 0 .. n_sink-1 (attention
+ *                  sinks, attended by every later token as in rat_dilated_attn_prefill_sinks)
  *   reset_every  : 0 for the full-sequence recurrence of RAT+; L > 0 for the chunk-local
  *                  recurrence of RAT (state dropped before every position p with p mod L = 0,
  *                  as in rat_recur_prefill_local); read by rat_dilated_decode
@@ -312,6 +329,8 @@ typedef struct rat_kv_cache {
     float *h_k, *h_v;         /* device float32 state                                      */
     int64_t pos;              /* positions consumed so far                                 */
     int64_t reset_every;      /* recurrence block length L, or 0 (full sequence); >= 0     */
+    int32_t n_sink;           /* attention sinks kept (first positions); 0 = none          */
+    void *k_sink, *v_sink;    /* device [B][H][n_sink][d] of dtype, or NULL when n_sink == 0 */
 } rat_kv_cache;
 
 /* Byte sizes of the buffers a cache with these fields needs (any output may be NULL). */
@@ -321,8 +340,9 @@ RAT_API int rat_kv_cache_bytes(const rat_kv_cache *cache, size_t *dil_bytes, siz
 /* rat_kv_compress -- append T positions of recurrence output to the cache.
  *   k_rec, v_rec : device (B, H, T, d) of cache->dtype: positions cache->pos .. cache->pos+T-1
  *   hT_k, hT_v   : device (B, H, d) float32 state after those positions (copied into h_k, h_v)
- * Writes every position p with p mod D_h = D_h - 1 (and p / D_h < cap_h) to its dil entry, and
- * the last min(W, T) positions to their ring slots; copies the state; then advances
+ * Writes every position p with p mod D_h = D_h - 1 (and p / D_h < cap_h) to its dil entry, the
+ * last min(W, T) positions to their ring slots and positions below n_sink to the sink rows;
+ * copies the state; then advances
  * cache->pos by T on the host.  Bit-exact copies.  Requires cache->pos + T <= Tcap. */
 RAT_API int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, const float *hT_v,
                     int T, rat_kv_cache *cache, void *stream);
@@ -335,9 +355,10 @@ RAT_API int rat_kv_compress(const void *k_rec, const void *v_rec, const float *h
  *   ws, ws_bytes        : workspace of at least rat_decode_workspace_bytes(cache)
  * Per (b, h): state update h = g h + (1-g) x for k and v (h taken as 0 first when
  * cache->reset_every = L > 0 and t mod L = 0); k~_t = RoPE(h_k, t); append k~_t, v~_t
- * to the dil cache if t mod D_h = D_h - 1 and to ring slot t mod W; then attention of
- * RoPE(q, t) over the dil entries with position <= t - We, the ring positions
- * t-We < j < t and the token itself -- the same key set S(t) as in prefill.  Split over the
+ * to the dil cache if t mod D_h = D_h - 1, to ring slot t mod W and to the sink rows if
+ * t < n_sink; then attention of RoPE(q, t) over the dil entries with position <= t - We, the
+ * ring positions t-We < j < t, the sinks older than the window that are not chunk ends, and the
+ * token itself -- the same key set S(t) as in prefill.  Split over the
  * keys across CTAs, combined by log-sum-exp.  Advances cache->pos by 1 on the host.
  * Requires pos < Tcap.
  * ---------------------------------------------------------------------------------------- */

@@ -55,6 +55,7 @@ class KVCache(ctypes.Structure):
         ("k_win", ctypes.c_void_p), ("v_win", ctypes.c_void_p),
         ("h_k", ctypes.c_void_p), ("h_v", ctypes.c_void_p),
         ("pos", ctypes.c_int64), ("reset_every", ctypes.c_int64),
+        ("n_sink", ctypes.c_int32), ("k_sink", ctypes.c_void_p), ("v_sink", ctypes.c_void_p),
     ]
 
 
@@ -96,8 +97,11 @@ def lib():
         L.rat_dilated_attn_backward_workspace_bytes.restype = _sz
         L.rat_dilated_attn_backward_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.rat_dilated_attn_backward.argtypes = [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _i,
-                                                            ctypes.POINTER(ctypes.c_int32), _i64,
-                                                            _f, _f, _vp, _sz, _vp]
+                                                            ctypes.POINTER(ctypes.c_int32), _i,
+                                                            _i64, _f, _f, _vp, _sz, _vp]
+        L.rat_dilated_attn_prefill_sinks.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                                     _i, ctypes.POINTER(ctypes.c_int32), _i,
+                                                     _i64, _f, _f, _vp]
         L.rat_recur_backward_workspace_bytes.restype = _sz
         L.rat_recur_backward_workspace_bytes.argtypes = [_i, _i, _i, _i]
         L.rat_recur_backward.argtypes = [_vp] * 16 + [_i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
@@ -257,12 +261,21 @@ def rat_recur_prefill_window(k, v, gate_logit, k_rec, v_rec, ws: Workspace, Lw: 
 
 def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,
                              D_per_head: Optional[Sequence[int]] = None, pos0: int = 0,
-                             rope_base: float = 0.0, scale: float = 0.0, stream=None):
-    """o = dilated attention of q over (k_rec, v_rec); all (B, H, T, d)."""
+                             rope_base: float = 0.0, scale: float = 0.0, stream=None,
+                             n_sink: int = 0):
+    """o = dilated attention of q over (k_rec, v_rec); all (B, H, T, d).  n_sink > 0 adds the
+    first n_sink positions to every key set (rat_dilated_attn_prefill_sinks)."""
     B, H, T, d = q.shape
     dph = None
     if D_per_head is not None:
         dph = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
+    if n_sink:
+        st = lib().rat_dilated_attn_prefill_sinks(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), B, H,
+                                                  T, d, _dtype_code(q), int(D), int(W), dph,
+                                                  int(n_sink), int(pos0), float(rope_base),
+                                                  float(scale), _stream(stream))
+        _check("rat_dilated_attn_prefill_sinks", st)
+        return
     st = lib().rat_dilated_attn_prefill(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), B, H, T, d,
                                         _dtype_code(q), int(D), int(W), dph, int(pos0),
                                         float(rope_base), float(scale), _stream(stream))
@@ -276,26 +289,28 @@ def rat_dilated_attn_backward_workspace_bytes(B, H, T, d, dtype) -> int:
 def rat_dilated_attn_backward(q, k_rec, v_rec, o, dO, dq, dk_rec, dv_rec, ws: Workspace,
                               D: int = 1, W: int = 0, D_per_head: Optional[Sequence[int]] = None,
                               pos0: int = 0, rope_base: float = 0.0, scale: float = 0.0,
-                              stream=None):
-    """Gradients of rat_dilated_attn_prefill: dq, dk_rec, dv_rec (all (B, H, T, d))."""
+                              stream=None, n_sink: int = 0):
+    """Gradients of rat_dilated_attn_prefill(_sinks): dq, dk_rec, dv_rec (all (B, H, T, d))."""
     B, H, T, d = q.shape
     dph = None
     if D_per_head is not None:
         dph = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
     st = lib().rat_dilated_attn_backward(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), _ptr(dO),
                                          _ptr(dq), _ptr(dk_rec), _ptr(dv_rec), B, H, T, d,
-                                         _dtype_code(q), int(D), int(W), dph, int(pos0),
-                                         float(rope_base), float(scale), ws.ptr, ws.nbytes,
-                                         _stream(stream))
+                                         _dtype_code(q), int(D), int(W), dph, int(n_sink),
+                                         int(pos0), float(rope_base), float(scale), ws.ptr,
+                                         ws.nbytes, _stream(stream))
     _check("rat_dilated_attn_backward", st)
 
 
 def make_cache(B, H, d, W, Tcap, dtype: int, D_per_head: Sequence[int], device="cuda",
-               reset_every: int = 0):
+               reset_every: int = 0, n_sink: int = 0):
     """Allocate (with torch) the buffers of a compressed cache and return (KVCache, buffers).
-    reset_every = L > 0 selects the chunk-local recurrence for the decode steps."""
+    reset_every = L > 0 selects the chunk-local recurrence for the decode steps; n_sink > 0
+    keeps the first n_sink positions as attention sinks."""
     Dh = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
-    c = KVCache(B=B, H=H, d=d, W=W, Tcap=Tcap, dtype=dtype, D=Dh, reset_every=int(reset_every))
+    c = KVCache(B=B, H=H, d=d, W=W, Tcap=Tcap, dtype=dtype, D=Dh, reset_every=int(reset_every),
+                n_sink=int(n_sink))
     dil, win, state = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     _check("rat_kv_cache_bytes", lib().rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(dil),
                                                           ctypes.byref(win), ctypes.byref(state)))
@@ -309,12 +324,16 @@ def make_cache(B, H, d, W, Tcap, dtype: int, D_per_head: Sequence[int], device="
         "v_win": torch.zeros((B, H, max(W, 1), d), dtype=tdt, device=device),
         "h_k": torch.zeros((B, H, d), dtype=torch.float32, device=device),
         "h_v": torch.zeros((B, H, d), dtype=torch.float32, device=device),
+        "k_sink": torch.zeros((B, H, max(n_sink, 1), d), dtype=tdt, device=device),
+        "v_sink": torch.zeros((B, H, max(n_sink, 1), d), dtype=tdt, device=device),
         "D": Dh,
     }
     c.k_dil, c.v_dil = bufs["k_dil"].data_ptr(), bufs["v_dil"].data_ptr()
     c.k_win = bufs["k_win"].data_ptr() if W > 0 else None
     c.v_win = bufs["v_win"].data_ptr() if W > 0 else None
     c.h_k, c.h_v = bufs["h_k"].data_ptr(), bufs["h_v"].data_ptr()
+    c.k_sink = bufs["k_sink"].data_ptr() if n_sink > 0 else None
+    c.v_sink = bufs["v_sink"].data_ptr() if n_sink > 0 else None
     c.pos = 0
     return c, bufs
 

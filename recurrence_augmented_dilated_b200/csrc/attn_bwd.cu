@@ -2,6 +2,7 @@
 //
 // The forward (RAT+ abstract; "RAT+ Deep Dive" sections 3.1 and 6): query t of head h attends
 //   S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D_h = D_h - 1 },   We = max(W, 1),
+// plus, with n_sink > 0, the first n_sink positions (attention sinks, each key once),
 // o_t = sum_{j in S(t)} p_tj v_j,  p_t = softmax_j(scale <q^_t, k~_j>),  q^ = RoPE(q).
 // Its reverse-mode derivative, for upstream gradients dO:
 //   dp_tj = <dO_t, v_j>,   ds_tj = p_tj (dp_tj - <dO_t, o_t>),
@@ -82,8 +83,15 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const __grid_constant_
     const int w_lo = max(0, t - We + 1);
     const int n_win = t - w_lo + 1;
     const int n_dil = t - We + 1 >= D ? (t - We + 1) / D : 0;
-    const int n = n_win + n_dil;
-    auto key = [&](int idx) { return idx < n_win ? w_lo + idx : (idx - n_win) * D + D - 1; };
+    const int s_lim = min(p.n_sink, max(0, t - We + 1));     // sinks that are not chunk ends
+    const int n_snk = D > 1 ? s_lim - s_lim / D : 0;
+    const int n = n_win + n_dil + n_snk;
+    auto key = [&](int idx) {
+        if (idx < n_win) return w_lo + idx;
+        if (idx < n_win + n_dil) return (idx - n_win) * D + D - 1;
+        const int s = idx - n_win - n_dil;
+        return s + s / (D - 1);
+    };
 
     // pass 1: the softmax denominator (log2 units)
     float m = -INFINITY, l = 0.f;
@@ -163,9 +171,9 @@ __global__ void __launch_bounds__(256) attn_bwd_dkv_kernel(const __grid_constant
     const uint8_t *qb = static_cast<const uint8_t *>(p.qh) + row * DH * EB + lane * CPL * EB;
     const uint8_t *gb = static_cast<const uint8_t *>(p.dO) + row * DH * EB + lane * CPL * EB;
 
-    // queries holding key j: t in [j, j + We - 1] (window), then t >= j + We (chunk end)
+    // queries holding key j: t in [j, j + We - 1] (window), then t >= j + We (chunk end or sink)
     const int n_win = min(We, p.T - j);
-    const int n_dil = (j % D == D - 1) ? max(0, p.T - (j + We)) : 0;
+    const int n_dil = (j % D == D - 1 || j < p.n_sink) ? max(0, p.T - (j + We)) : 0;
     const int n = n_win + n_dil;
     float dk[CPL], dv[CPL];
 #pragma unroll

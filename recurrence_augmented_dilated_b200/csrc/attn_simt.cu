@@ -2,7 +2,9 @@
 //
 // RAT+ abstract and "RAT+ Deep Dive" sections 3.1 and 6: query t of head h attends to
 //   S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D_h = D_h - 1 },   We = max(W, 1),
-// the local window (self included) and the chunk ends older than it.  One warp per query:
+// the local window (self included) and the chunk ends older than it; with n_sink > 0 also the
+// first n_sink positions (StreamingLLM's attention sinks, section 6's layer-wise hybrid), each
+// key once.  This kernel is also the path for every call with sinks.  One warp per query:
 // each lane holds d/32 channels of the query and of the running output; for every key of
 // S(t) the warp reduces the dot product with shuffles and applies an online softmax in
 // float32 (exp2 with the scale folded in).  Keys are visited in groups of four so four row
@@ -42,11 +44,15 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const __grid_constant__ 
 #pragma unroll
     for (int j = 0; j < CPL; ++j) o[j] = 0.f;
 
-    // the key list: window positions first, then the chunk ends older than the window
+    // the key list: window positions first, then the chunk ends older than the window, then
+    // the sinks older than the window that are not chunk ends (sink s is position
+    // s + s / (D-1): the D-1 non-chunk-ends of each chunk in turn)
     const int w_lo = max(0, t - We + 1);
     const int n_win = t - w_lo + 1;
     const int n_dil = t - We + 1 >= D ? (t - We + 1) / D : 0;   // j = D-1, .., n_dil*D - 1 <= t-We
-    const int n = n_win + n_dil;
+    const int s_lim = min(p.n_sink, max(0, t - We + 1));
+    const int n_snk = D > 1 ? s_lim - s_lim / D : 0;
+    const int n = n_win + n_dil + n_snk;
     for (int base = 0; base < n; base += 4) {
         float kx[4][CPL], vx[4][CPL];
         int cnt = min(4, n - base);
@@ -54,7 +60,13 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const __grid_constant__ 
         for (int u = 0; u < 4; ++u) {
             const int idx = base + u;
             if (u < cnt) {
-                const int j = idx < n_win ? w_lo + idx : (idx - n_win) * D + D - 1;
+                int j;
+                if (idx < n_win) j = w_lo + idx;
+                else if (idx < n_win + n_dil) j = (idx - n_win) * D + D - 1;
+                else {
+                    const int s = idx - n_win - n_dil;
+                    j = s + s / (D - 1);
+                }
                 RowIO<E, CPL>::load(kb + (size_t)j * DH * EB, kx[u]);
                 RowIO<E, CPL>::load(vb + (size_t)j * DH * EB, vx[u]);
             }

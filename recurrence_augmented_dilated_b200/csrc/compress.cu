@@ -5,6 +5,7 @@
 // (b, h) this kernel copies
 //   - each chunk end p = i*D_h + D_h - 1 (i < cap_h) to dil entry i of head h, and
 //   - each of the last min(W, T) positions p to ring slot p mod W,
+//   - each position p < n_sink to sink row p (attention sinks),
 // for k~ and v~, bit for bit; and copies the final recurrence state into the cache.
 // One CTA per (row block, b*h); 16-byte vector copies, one row per LPR lanes, four rows per
 // thread in flight at once.  The paged form (one sequence per call) writes the dil entries into
@@ -35,18 +36,20 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
     const long long n_dil = max(0ll, i_hi - i_lo);
     const long long r_lo = max(p.pos0, end - (long long)p.W);  // ring positions [r_lo, end)
     const long long n_ring = p.W > 0 ? end - r_lo : 0;
+    const long long n_sk = max(0ll, min(end, (long long)p.n_sink) - p.pos0);   // sink rows
     const int row_bytes = p.d * p.esize;
     const int lpr = row_bytes / 16;                          // lanes per row
     const int rows_per_pass = blockDim.x / lpr;
     const int lane_r = threadIdx.x / lpr, lane_c = threadIdx.x % lpr;
-    const long long njobs = 2 * (n_dil + n_ring);            // (k, v) x (dil rows + ring rows)
+    const long long per = n_dil + n_ring + n_sk;            // rows of one tensor
+    const long long njobs = 2 * per;                          // (k, v) x (dil + ring + sink rows)
 
     const uint8_t *src_k = static_cast<const uint8_t *>(p.k) + (size_t)bh * p.T * row_bytes;
     const uint8_t *src_v = static_cast<const uint8_t *>(p.v) + (size_t)bh * p.T * row_bytes;
     // job -> (source row, destination row) of this (b, h)
     auto locate = [&](long long job, const uint8_t *&src, uint8_t *&dst) {
-        const bool is_v = job >= n_dil + n_ring;
-        const long long r = is_v ? job - (n_dil + n_ring) : job;
+        const bool is_v = job >= per;
+        const long long r = is_v ? job - per : job;
         long long pos;
         if (r < n_dil) {
             const long long i = i_lo + r;
@@ -63,10 +66,14 @@ __global__ void __launch_bounds__(256) compress_kernel(const __grid_constant__ C
             } else {
                 dst = base + ((size_t)b * p.total_cap + p.off[h] + i) * row_bytes;
             }
-        } else {
+        } else if (r < n_dil + n_ring) {
             pos = r_lo + (r - n_dil);
             uint8_t *base = static_cast<uint8_t *>(is_v ? p.vwin : p.kwin);
             dst = base + ((size_t)bhc * p.W + (size_t)(pos % p.W)) * row_bytes;
+        } else {
+            pos = p.pos0 + (r - n_dil - n_ring);
+            uint8_t *base = static_cast<uint8_t *>(is_v ? p.vsink : p.ksink);
+            dst = base + ((size_t)bhc * p.n_sink + (size_t)pos) * row_bytes;
         }
         src = (is_v ? src_v : src_k) + (size_t)(pos - p.pos0) * row_bytes;
     };
@@ -110,7 +117,8 @@ int launch_compress(const CompressParams &p_in, void *stream) {
         const long long cap = p.page_table ? (long long)p.max_pages << p.page_shift : p.Tcap / D;
         const long long n_dil = std::max(0ll, std::min((p.pos0 + p.T) / D, cap) - p.pos0 / D);
         const long long n_ring = p.W > 0 ? std::min(p.W, p.T) : 0;     // the last min(W, T) positions
-        const long long jobs = 2 * (n_dil + n_ring);
+        const long long n_sk = std::max(0ll, std::min(p.pos0 + p.T, (long long)p.n_sink) - p.pos0);
+        const long long jobs = 2 * (n_dil + n_ring + n_sk);
         long long n = (jobs + rows_per_pass * 4 - 1) / (rows_per_pass * 4);
         n = std::max(1ll, std::min(n, 4096ll));
         p.blk0[h] = acc;

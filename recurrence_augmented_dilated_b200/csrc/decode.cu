@@ -41,7 +41,8 @@ RAT_DEVICE uint4 pack8(const float *x) {
 // Template on d: 16 lanes per row for d = 128 (8 bf16 each), 8 lanes for d = 64.  PAGED: the
 // dilated entries live in pages of a pool found through a page table, and every sequence has
 // its own position (read from seq_pos, advanced by the last CTA of the sequence).
-template <int DH, bool PAGED>
+// SINKS: the first n_sink positions are kept in sink rows and join every key set.
+template <int DH, bool PAGED, bool SINKS>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int LPR = DH / 8;                 // lanes per key row
     constexpr int GPW = 32 / LPR;               // key groups per warp
@@ -81,12 +82,19 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         }
     }
 
-    // key list of this slice: [0, n_dil) dil entries, then [n_dil, n_dil + n_ring) ring positions
+    // key list of this slice: [0, n_dil) dil entries, then [n_dil, n_dil + n_ring) ring
+    // positions, then (SINKS) the sinks older than the window that are not chunk ends (sink s is
+    // position s + s / (D-1))
     long long n_dil = (t - We + 1) >= D ? (t - We + 1) / D : 0;
     if (n_dil > cap) n_dil = cap;
     const long long r_lo = max(0ll, t - We + 1);           // first ring position in the window
     const long long n_ring = t - r_lo;                      // positions r_lo .. t-1
-    const long long n_keys = n_dil + n_ring;
+    long long n_snk = 0;
+    if constexpr (SINKS) {
+        const long long s_lim = min((long long)p.n_sink, r_lo);
+        n_snk = D > 1 ? s_lim - s_lim / D : 0;
+    }
+    const long long n_keys = n_dil + n_ring + n_snk;
     const long long k_lo = n_keys * split / p.splits, k_hi = n_keys * (split + 1) / p.splits;
 
     // paged: the pools; otherwise this slice's first entry
@@ -128,10 +136,15 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                         kp = kdil + (size_t)idx * RB;
                         vp = vdil + (size_t)idx * RB;
                     }
-                } else {
+                } else if (!SINKS || idx < n_dil + n_ring) {
                     const long long pos = r_lo + (idx - n_dil);
                     kp = kwin + (size_t)(pos % p.W) * RB;
                     vp = vwin + (size_t)(pos % p.W) * RB;
+                } else {
+                    const long long s = idx - n_dil - n_ring;
+                    const size_t row = (size_t)bh * p.n_sink + (size_t)(s + s / (D - 1));
+                    kp = static_cast<const uint8_t *>(p.ksink) + row * RB;
+                    vp = static_cast<const uint8_t *>(p.vsink) + row * RB;
                 }
                 kr[u] = __ldg(reinterpret_cast<const uint4 *>(kp + cl * 16));
                 vr[u] = __ldg(reinterpret_cast<const uint4 *>(vp + cl * 16));
@@ -228,6 +241,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                 } else if (PAGED) {
                     record_error(p.hdr, RAT_ERR_INVALID, 0x401u);     // no page for the entry
                 }
+            }
+            if (SINKS && t < p.n_sink) {
+                uint8_t *ks = static_cast<uint8_t *>(p.ksink) + ((size_t)bh * p.n_sink + (size_t)t) * RB;
+                uint8_t *vs = static_cast<uint8_t *>(p.vsink) + ((size_t)bh * p.n_sink + (size_t)t) * RB;
+                *reinterpret_cast<uint4 *>(ks + cl * 16) = kpk;
+                *reinterpret_cast<uint4 *>(vs + cl * 16) = vpk;
             }
             if (p.W > 0) {
                 uint8_t *kw = static_cast<uint8_t *>(p.kwin) + ((size_t)bh * p.W + (size_t)(t % p.W)) * RB;
@@ -349,11 +368,19 @@ int launch_decode(const DecodeParams &p, int dtype, void *stream, bool paged) {
     if (dtype != RAT_BF16) return RAT_ERR_UNSUPPORTED;
     dim3 grid((unsigned)p.splits, (unsigned)(p.B * p.H));
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (p.d == 128 && !paged) decode_kernel<128, false><<<grid, kThreads, 0, s>>>(p);
-    else if (p.d == 64 && !paged) decode_kernel<64, false><<<grid, kThreads, 0, s>>>(p);
-    else if (p.d == 128) decode_kernel<128, true><<<grid, kThreads, 0, s>>>(p);
-    else if (p.d == 64) decode_kernel<64, true><<<grid, kThreads, 0, s>>>(p);
-    else return RAT_ERR_UNSUPPORTED;
+    const bool sinks = p.n_sink > 0;
+    if (paged && sinks) return RAT_ERR_UNSUPPORTED;
+    if (p.d == 128) {
+        if (paged) decode_kernel<128, true, false><<<grid, kThreads, 0, s>>>(p);
+        else if (sinks) decode_kernel<128, false, true><<<grid, kThreads, 0, s>>>(p);
+        else decode_kernel<128, false, false><<<grid, kThreads, 0, s>>>(p);
+    } else if (p.d == 64) {
+        if (paged) decode_kernel<64, true, false><<<grid, kThreads, 0, s>>>(p);
+        else if (sinks) decode_kernel<64, false, true><<<grid, kThreads, 0, s>>>(p);
+        else decode_kernel<64, false, false><<<grid, kThreads, 0, s>>>(p);
+    } else {
+        return RAT_ERR_UNSUPPORTED;
+    }
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 

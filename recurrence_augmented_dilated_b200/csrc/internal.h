@@ -98,6 +98,7 @@ struct AttnSimtParams {
     long long pos0;
     int rope;
     float scale_log2;           // softmax scale * log2(e)
+    int n_sink;                 // attention sinks: the first n_sink positions join every key set
     int Dh[kMaxHeads];
     double theta[64];
 };
@@ -159,6 +160,8 @@ struct CompressParams {
     int page_shift, max_pages, n_pages, seq;
     long long *seq_pos;         // [B] set to pos0 + T for sequence seq
     WsHeader *hdr;              // receives RAT_ERR_INVALID for a page index outside the pool
+    void *ksink, *vsink;        // [B][H][n_sink][d]: positions below n_sink (attention sinks)
+    int n_sink;
 };
 int launch_compress(const CompressParams &p, void *stream);
 
@@ -169,7 +172,7 @@ struct AttnBwdParams {
     void *qh;                   // workspace [B*H][T][d] of dtype: RoPE(q) as the attention uses it
     float *lse;                 // workspace [B*H][T]: log2 of each query's softmax denominator
     float *delta;               // workspace [B*H][T]: <dO_t, o_t>
-    int B, H, T, d, W;
+    int B, H, T, d, W, n_sink;
     long long pos0;
     int rope;
     float scale, scale_log2;
@@ -204,6 +207,8 @@ struct DecodeParams {
     uint32_t *seq_ticket;       // [B] CTAs of sequence b finished (the last one advances seq_pos)
     const int32_t *page_table;  // [B * H][max_pages]
     int page_shift, max_pages, n_pages;
+    void *ksink, *vsink;        // [B * H][n_sink][d]: positions 0 .. n_sink-1 (attention sinks)
+    int n_sink;
 };
 int decode_splits(int B, int H, int Tcap, const int32_t *Dh, int W);
 int decode_splits_for_keys(int B, int H, long long max_keys);

@@ -36,7 +36,7 @@ long long total_capacity(int H, int Tcap, const int32_t *Dh, long long *off) {
 
 bool valid_cache(const rat_kv_cache *c) {
     if (!c || c->B < 1 || c->H < 1 || c->H > kMaxHeads || !supported_d(c->d) || c->W < 0 ||
-        c->Tcap < 1 || !valid_dtype(c->dtype) || !c->D || c->reset_every < 0)
+        c->Tcap < 1 || !valid_dtype(c->dtype) || !c->D || c->reset_every < 0 || c->n_sink < 0)
         return false;
     for (int h = 0; h < c->H; ++h)
         if (c->D[h] < 1) return false;
@@ -292,11 +292,14 @@ int rat_recur_prefill_local(const void *k, const void *v, const void *gate_logit
 }
 
 // ------------------------------------------------------------------------------ attention
-int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, int B,
-                             int H, int T, int d, int dtype, int D, int W,
-                             const int32_t *D_per_head, int64_t pos0, float rope_base,
-                             float scale, void *stream) {
-    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0) return RAT_ERR_INVALID;
+}  // extern "C"
+
+namespace {
+int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, int B, int H,
+                 int T, int d, int dtype, int D, int W, const int32_t *D_per_head, int n_sink,
+                 int64_t pos0, float rope_base, float scale, void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0 || n_sink < 0)
+        return RAT_ERR_INVALID;
     if (!supported_d(d) || H > kMaxHeads) return RAT_ERR_UNSUPPORTED;
     if (!std::isfinite(rope_base) || !std::isfinite(scale)) return RAT_ERR_INVALID;
     if (!D_per_head && D < 1) return RAT_ERR_INVALID;
@@ -313,7 +316,7 @@ int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec
     int32_t Dh[kMaxHeads];
     for (int h = 0; h < H; ++h) Dh[h] = D_per_head ? D_per_head[h] : D;
 
-    if (dtype == RAT_BF16 && d == 128) {
+    if (dtype == RAT_BF16 && d == 128 && n_sink == 0) {
         AttnSm100Args a;
         std::memset(&a, 0, sizeof(a));
         a.q = q; a.k = k_rec; a.v = v_rec; a.o = o;
@@ -332,9 +335,29 @@ int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec
     p.pos0 = pos0;
     p.rope = rope_base > 0.f ? 1 : 0;
     p.scale_log2 = scale_log2;
+    p.n_sink = n_sink;
     for (int h = 0; h < H; ++h) p.Dh[h] = Dh[h];
     if (p.rope) rope_theta(rope_base, d, p.theta);
     return launch_attn_simt(p, dtype, stream);
+}
+}  // namespace
+
+extern "C" {
+
+int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, int B,
+                             int H, int T, int d, int dtype, int D, int W,
+                             const int32_t *D_per_head, int64_t pos0, float rope_base,
+                             float scale, void *stream) {
+    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, 0, pos0,
+                        rope_base, scale, stream);
+}
+
+int rat_dilated_attn_prefill_sinks(const void *q, const void *k_rec, const void *v_rec, void *o,
+                                   int B, int H, int T, int d, int dtype, int D, int W,
+                                   const int32_t *D_per_head, int n_sink, int64_t pos0,
+                                   float rope_base, float scale, void *stream) {
+    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, n_sink, pos0,
+                        rope_base, scale, stream);
 }
 
 size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int dtype) {
@@ -345,9 +368,10 @@ size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int
 int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_rec, const void *o,
                               const void *dO, void *dq, void *dk_rec, void *dv_rec, int B, int H,
                               int T, int d, int dtype, int D, int W, const int32_t *D_per_head,
-                              int64_t pos0, float rope_base, float scale, void *ws,
+                              int n_sink, int64_t pos0, float rope_base, float scale, void *ws,
                               size_t ws_bytes, void *stream) {
-    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0) return RAT_ERR_INVALID;
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0 || n_sink < 0)
+        return RAT_ERR_INVALID;
     if (!supported_d(d) || H > kMaxHeads) return RAT_ERR_UNSUPPORTED;
     if (!std::isfinite(rope_base) || !std::isfinite(scale)) return RAT_ERR_INVALID;
     if (!D_per_head && D < 1) return RAT_ERR_INVALID;
@@ -372,7 +396,7 @@ int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_re
     p.lse = reinterpret_cast<float *>(w);
     w += align256(rows * 4);
     p.delta = reinterpret_cast<float *>(w);
-    p.B = B; p.H = H; p.T = T; p.d = d; p.W = W;
+    p.B = B; p.H = H; p.T = T; p.d = d; p.W = W; p.n_sink = n_sink;
     p.pos0 = pos0;
     p.rope = rope_base > 0.f ? 1 : 0;
     p.scale = scale > 0.f ? scale : (float)(1.0 / std::sqrt((double)d));
@@ -414,6 +438,8 @@ int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, con
     if (T == 0) return RAT_OK;
     if (!k_rec || !v_rec || !c->k_dil || !c->v_dil || !c->h_k || !c->h_v) return RAT_ERR_INVALID;
     if (c->W > 0 && (!c->k_win || !c->v_win)) return RAT_ERR_INVALID;
+    if (c->n_sink > 0 && (!c->k_sink || !c->v_sink || !aligned16(c->k_sink) || !aligned16(c->v_sink)))
+        return RAT_ERR_INVALID;
     if (!aligned16(k_rec) || !aligned16(v_rec) || !aligned16(c->k_dil) || !aligned16(c->v_dil) ||
         (c->W > 0 && (!aligned16(c->k_win) || !aligned16(c->v_win))))
         return RAT_ERR_INVALID;
@@ -425,6 +451,7 @@ int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, con
     p.B = c->B; p.H = c->H; p.T = T; p.d = c->d; p.W = c->W; p.Tcap = c->Tcap;
     p.esize = esize(c->dtype);
     p.pos0 = c->pos;
+    p.ksink = c->k_sink; p.vsink = c->v_sink; p.n_sink = c->n_sink;
     for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
     p.total_cap = total_capacity(c->H, c->Tcap, c->D, p.off);
     const int st = launch_compress(p, stream);
@@ -529,6 +556,8 @@ int rat_dilated_decode(const void *q, const void *k, const void *v, const void *
         return RAT_ERR_INVALID;
     if (!c->k_dil || !c->v_dil || !c->h_k || !c->h_v) return RAT_ERR_INVALID;
     if (c->W > 0 && (!c->k_win || !c->v_win)) return RAT_ERR_INVALID;
+    if (c->n_sink > 0 && (!c->k_sink || !c->v_sink || !aligned16(c->k_sink) || !aligned16(c->v_sink)))
+        return RAT_ERR_INVALID;
     if (c->pos < 0 || c->pos >= c->Tcap) return RAT_ERR_INVALID;
     if (!std::isfinite(rope_base) || !std::isfinite(scale)) return RAT_ERR_INVALID;
     if ((long long)c->B * c->H > 65535) return RAT_ERR_UNSUPPORTED;
@@ -544,6 +573,7 @@ int rat_dilated_decode(const void *q, const void *k, const void *v, const void *
     p.B = c->B; p.H = c->H; p.d = c->d; p.W = c->W; p.Tcap = c->Tcap; p.splits = splits;
     p.t = c->pos;
     p.reset = c->reset_every;
+    p.ksink = c->k_sink; p.vsink = c->v_sink; p.n_sink = c->n_sink;
     for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
     p.total_cap = total_capacity(c->H, c->Tcap, c->D, p.off);
     p.rope = rope_base > 0.f ? 1 : 0;

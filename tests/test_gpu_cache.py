@@ -78,7 +78,7 @@ def test_compress_chunked_equals_whole():
         assert torch.equal(b1[n], b2[n]), n
 
 
-def run_decode(w, T0, steps, heads_check, B=None, H=None, rope_base=0.0, reset_every=0):
+def run_decode(w, T0, steps, heads_check, B=None, H=None, rope_base=0.0, reset_every=0, n_sink=0):
     """GPU: prefill a T0-token context, compress, then decode `steps` tokens.
     Oracle: the same from the same raw inputs on the (b, h) slices in heads_check."""
     B = w.B if B is None else B
@@ -87,7 +87,8 @@ def run_decode(w, T0, steps, heads_check, B=None, H=None, rope_base=0.0, reset_e
     Dh = w.heads_D()[:H]
     Tcap = T0 + steps
     dev = torch.device("cuda")
-    cache, bufs = rat.make_cache(B, H, d, W, Tcap, rat.BF16, Dh, reset_every=reset_every)
+    cache, bufs = rat.make_cache(B, H, d, W, Tcap, rat.BF16, Dh, reset_every=reset_every,
+                                 n_sink=n_sink)
     hk = torch.zeros((B, H, d), dtype=torch.float32, device=dev)
     hv = torch.zeros_like(hk)
     nchunks = (T0 + synthetic.CTX_CHUNK - 1) // synthetic.CTX_CHUNK
@@ -111,7 +112,7 @@ def run_decode(w, T0, steps, heads_check, B=None, H=None, rope_base=0.0, reset_e
     got = torch.stack(outs)[:, :, :, 0]            # (steps, B, H, d)
     # oracle on the checked slices
     st = oracle.DecodeState([Dh[h] for _, h in heads_check], d, W, Tcap, rope_base=rope_base,
-                            reset_every=reset_every)
+                            reset_every=reset_every, n_sink=n_sink)
     ctx = [synthetic.decode_context_slice(w, b, h, device=dev, T=T0) for b, h in heads_check]
     st.prefill(np.stack([f64(x[0]) for x in ctx]), np.stack([f64(x[1]) for x in ctx]),
                np.stack([f64(x[2]) for x in ctx]))
