@@ -52,6 +52,8 @@ def _load():
         lib.rat_oracle_dilated_attention_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp,
                                                               _ip, _L, _L, ctypes.c_double, _dp,
                                                               _dp, _dp]
+        lib.rat_oracle_topk_attention.argtypes = [_L, _L, _L, _dp, _dp, _dp, _ip, _L, _L, _L,
+                                                  ctypes.c_double, _dp]
         lib.rat_oracle_recurrence_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _dp,
                                                        _dp, _dp]
         lib.rat_oracle_rope.argtypes = [_L, _L, _L, _dp, _L, ctypes.c_double]
@@ -255,6 +257,21 @@ def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None,
         out = np.empty((B, H, nrows, d))
     _load().rat_oracle_dilated_attention(B * H, T, d, _ptr(q), _ptr(k), _ptr(v), _ptr(Dbh, _ip),
                                          int(W), int(n_sink), float(scale), rp, nrows, _ptr(out))
+    return out
+
+
+def topk_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, n_sink=0, top_k=0):
+    """Dilated attention plus the top_k chunks (scored by their chunk-end keys) attended at
+    every position ("RAT+ Deep Dive" section 4, dilation combined with top-k selection).
+    q, k, v as in dilated_attention; returns (B, H, T, d) in float64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, T, d = q.shape
+    Dbh, _ = _per_bh_dilation((B, H), D, D_per_head)
+    if scale is None:
+        scale = default_scale(d)
+    out = np.empty((B, H, T, d))
+    _load().rat_oracle_topk_attention(B * H, T, d, _ptr(q), _ptr(k), _ptr(v), _ptr(Dbh, _ip),
+                                      int(W), int(n_sink), int(top_k), float(scale), _ptr(out))
     return out
 
 

@@ -301,6 +301,71 @@ void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, cons
 }
 
 /*
+ * Dilated attention with top-k chunk selection ("RAT+ Deep Dive" section 4: dilation combined
+ * with top-k block selection, "dilation provides global coverage while top-k increases local
+ * density").  Read as: the blocks are the dilation's chunks c = [cD, cD + D - 1]; a chunk wholly
+ * older than the window (cD + D - 1 <= t - We) is scored by its chunk-end key,
+ * s_c = scale * <q_t, k_{cD+D-1}>; the top_k highest-scoring chunks (ties: the earlier chunk)
+ * are attended at every position, on top of S(t) (and the sinks), each key once.
+ * Arguments as rat_oracle_dilated_attention (all rows), plus top_k >= 0.
+ */
+void rat_oracle_topk_attention(long BH, long T, long d, const double *q, const double *k,
+                               const double *v, const int *Dbh, long W, long n_sink, long top_k,
+                               double scale, double *o)
+{
+    long We = eff_window(W);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        long D = Dbh[bh];
+        long *keys = (long *)malloc(sizeof(long) * (size_t)(T + 1));
+        double *s = (double *)malloc(sizeof(double) * (size_t)(T + 1));
+        double *cs = (double *)malloc(sizeof(double) * (size_t)(T / D + 1));
+        char *taken = (char *)malloc((size_t)(T / D + 1));
+        for (long t = 0; t < T; ++t) {
+            long n = list_keys(t, D, We, n_sink, keys);
+            const double *qt = q + (bh * T + t) * d;
+            long nc = t - We + 1 >= D ? (t - We + 1) / D : 0;       /* candidate chunks */
+            for (long c = 0; c < nc; ++c) {
+                const double *kj = k + (bh * T + c * D + D - 1) * d;
+                double dot = 0.0;
+                for (long x = 0; x < d; ++x) dot += qt[x] * kj[x];
+                cs[c] = scale * dot;
+                taken[c] = 0;
+            }
+            for (long r = 0; r < top_k && r < nc; ++r) {            /* r-th best: a plain scan */
+                long best = -1;
+                for (long c = 0; c < nc; ++c)
+                    if (!taken[c] && (best < 0 || cs[c] > cs[best])) best = c;
+                taken[best] = 1;
+                for (long j = best * D; j < best * D + D - 1; ++j)
+                    if (j >= n_sink) keys[n++] = j;                 /* sinks are listed already */
+            }
+            double mx = -INFINITY;
+            for (long m = 0; m < n; ++m) {
+                const double *kj = k + (bh * T + keys[m]) * d;
+                double dot = 0.0;
+                for (long x = 0; x < d; ++x) dot += qt[x] * kj[x];
+                s[m] = scale * dot;
+                if (s[m] > mx) mx = s[m];
+            }
+            double *ot = o + (bh * T + t) * d, l = 0.0;
+            for (long x = 0; x < d; ++x) ot[x] = 0.0;
+            for (long m = 0; m < n; ++m) {
+                double p = exp(s[m] - mx);
+                const double *vj = v + (bh * T + keys[m]) * d;
+                l += p;
+                for (long x = 0; x < d; ++x) ot[x] += p * vj[x];
+            }
+            for (long x = 0; x < d; ++x) ot[x] /= l;
+        }
+        free(keys);
+        free(s);
+        free(cs);
+        free(taken);
+    }
+}
+
+/*
  * Backward of the dilated attention above (its reverse-mode derivative), for upstream
  * gradients dO of the outputs.  Per query t, with p_j the softmax weights over S(t) and
  * o_t = sum_j p_j v_j:

@@ -463,6 +463,44 @@ def test_decode_with_sinks_equals_prefill_rows():
         np.testing.assert_allclose(o, full[0, :, t], rtol=1e-10, atol=1e-12)
 
 
+# ---- top-k chunk selection combined with dilation
+def test_topk_zero_is_the_dilated_attention():
+    q, k, v = (RNG.standard_normal((1, 2, 50, 8)) for _ in range(3))
+    a = oracle.dilated_attention(q, k, v, D=4, W=3, n_sink=2)
+    b = oracle.topk_attention(q, k, v, D=4, W=3, n_sink=2, top_k=0)
+    np.testing.assert_array_equal(a, b)
+
+
+def test_topk_with_unit_chunks_adds_nothing():
+    # D = 1: a chunk is its own chunk end, already a key
+    q, k, v = (RNG.standard_normal((1, 2, 40, 8)) for _ in range(3))
+    np.testing.assert_allclose(oracle.topk_attention(q, k, v, D=1, W=2, top_k=5),
+                               oracle.dilated_attention(q, k, v, D=1, W=2), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("D,W,n_sink,top_k", [(4, 3, 0, 2), (5, 1, 3, 3), (8, 8, 0, 100)])
+def test_topk_equals_masked_sdpa_with_argsort_selection(D, W, n_sink, top_k):
+    # the selection by a library sort of the chunk scores, the mask built from it, SDPA over it
+    import torch
+    T, d, scale = 60, 8, 0.35
+    q, k, v = (RNG.standard_normal((1, 1, T, d)) for _ in range(3))
+    We = max(W, 1)
+    mask = np.zeros((T, T), dtype=bool)
+    for t in range(T):
+        for j in range(t + 1):
+            mask[t, j] = oracle.in_key_set(t, j, D, W, n_sink)
+        nc = (t - We + 1) // D if t - We + 1 >= D else 0
+        if nc:
+            sc = np.array([scale * q[0, 0, t] @ k[0, 0, c * D + D - 1] for c in range(nc)])
+            order = np.argsort(-sc, kind="stable")[:top_k]      # ties: the earlier chunk
+            for c in order:
+                mask[t, c * D:c * D + D] = True
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(q), torch.tensor(k), torch.tensor(v), attn_mask=torch.tensor(mask), scale=scale)
+    got = oracle.topk_attention(q, k, v, D=D, W=W, n_sink=n_sink, top_k=top_k, scale=scale)
+    np.testing.assert_allclose(got, ref.numpy(), rtol=1e-11, atol=1e-12)
+
+
 def test_rope_matches_complex_rotation():
     d, T, pos0, base = 16, 9, 1000, 10000.0
     x = RNG.standard_normal((1, T, d))
