@@ -253,6 +253,21 @@ RAT_API int rat_dilated_attn_prefill_sinks(const void *q, const void *k_rec, con
                              const int32_t *D_per_head, int n_sink, int64_t pos0,
                              float rope_base, float scale, void *stream);
 
+/* rat_dilated_attn_prefill_topk -- the attention with top-k chunk selection combined with the
+ * dilation ("RAT+ Deep Dive" section 4: "dilation provides global coverage while top-k increases
+ * local density").  Read as: the blocks are the dilation's chunks [cD, cD + D - 1]; each chunk
+ * wholly older than the window (cD + D - 1 <= t - We) is scored by its chunk-end key (the
+ * recurrence state that sums the chunk up), s_c = scale <q^_t, k~_{cD+D-1}>; every position of
+ * the top_k best chunks (ties: the earlier chunk) joins S(t) and the sinks, each key once.
+ *   Arguments as rat_dilated_attn_prefill_sinks, plus top_k in [0, 16] (RAT_ERR_UNSUPPORTED
+ *   above 16).  Runs the CUDA-core kernel (float32 arithmetic) for both dtypes.  The selection
+ *   is taken on float32 scores: where two chunk scores tie to within float32 rounding, either
+ *   may be taken.  Prefill only: a decode step would need the uncompressed cache. */
+RAT_API int rat_dilated_attn_prefill_topk(const void *q, const void *k_rec, const void *v_rec,
+                             void *o, int B, int H, int T, int d, int dtype, int D, int W,
+                             const int32_t *D_per_head, int n_sink, int top_k, int64_t pos0,
+                             float rope_base, float scale, void *stream);
+
 /* Synchronise `stream`, then return (and clear) the first device-side error recorded by the
  * attention kernel since the last call (RAT_OK if none). */
 RAT_API int rat_attn_sync_status(void *stream);

@@ -102,6 +102,9 @@ def lib():
         L.rat_dilated_attn_prefill_sinks.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                                      _i, ctypes.POINTER(ctypes.c_int32), _i,
                                                      _i64, _f, _f, _vp]
+        L.rat_dilated_attn_prefill_topk.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
+                                                    _i, ctypes.POINTER(ctypes.c_int32), _i, _i,
+                                                    _i64, _f, _f, _vp]
         L.rat_recur_backward_workspace_bytes.restype = _sz
         L.rat_recur_backward_workspace_bytes.argtypes = [_i, _i, _i, _i]
         L.rat_recur_backward.argtypes = [_vp] * 16 + [_i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
@@ -262,13 +265,21 @@ def rat_recur_prefill_window(k, v, gate_logit, k_rec, v_rec, ws: Workspace, Lw: 
 def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,
                              D_per_head: Optional[Sequence[int]] = None, pos0: int = 0,
                              rope_base: float = 0.0, scale: float = 0.0, stream=None,
-                             n_sink: int = 0):
+                             n_sink: int = 0, top_k: int = 0):
     """o = dilated attention of q over (k_rec, v_rec); all (B, H, T, d).  n_sink > 0 adds the
-    first n_sink positions to every key set (rat_dilated_attn_prefill_sinks)."""
+    first n_sink positions to every key set (rat_dilated_attn_prefill_sinks); top_k > 0 adds
+    the top_k chunks by their chunk-end scores (rat_dilated_attn_prefill_topk)."""
     B, H, T, d = q.shape
     dph = None
     if D_per_head is not None:
         dph = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
+    if top_k:
+        st = lib().rat_dilated_attn_prefill_topk(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), B, H,
+                                                 T, d, _dtype_code(q), int(D), int(W), dph,
+                                                 int(n_sink), int(top_k), int(pos0),
+                                                 float(rope_base), float(scale), _stream(stream))
+        _check("rat_dilated_attn_prefill_topk", st)
+        return
     if n_sink:
         st = lib().rat_dilated_attn_prefill_sinks(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), B, H,
                                                   T, d, _dtype_code(q), int(D), int(W), dph,

@@ -99,6 +99,7 @@ struct AttnSimtParams {
     int rope;
     float scale_log2;           // softmax scale * log2(e)
     int n_sink;                 // attention sinks: the first n_sink positions join every key set
+    int top_k;                  // chunks (scored by their chunk-end keys) attended in full, <= 16
     int Dh[kMaxHeads];
     double theta[64];
 };

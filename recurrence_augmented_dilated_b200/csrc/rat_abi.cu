@@ -297,9 +297,11 @@ int rat_recur_prefill_local(const void *k, const void *v, const void *gate_logit
 namespace {
 int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, int B, int H,
                  int T, int d, int dtype, int D, int W, const int32_t *D_per_head, int n_sink,
-                 int64_t pos0, float rope_base, float scale, void *stream) {
-    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0 || n_sink < 0)
+                 int top_k, int64_t pos0, float rope_base, float scale, void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0 || n_sink < 0 ||
+        top_k < 0)
         return RAT_ERR_INVALID;
+    if (top_k > 16) return RAT_ERR_UNSUPPORTED;
     if (!supported_d(d) || H > kMaxHeads) return RAT_ERR_UNSUPPORTED;
     if (!std::isfinite(rope_base) || !std::isfinite(scale)) return RAT_ERR_INVALID;
     if (!D_per_head && D < 1) return RAT_ERR_INVALID;
@@ -316,7 +318,7 @@ int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, i
     int32_t Dh[kMaxHeads];
     for (int h = 0; h < H; ++h) Dh[h] = D_per_head ? D_per_head[h] : D;
 
-    if (dtype == RAT_BF16 && d == 128 && n_sink == 0) {
+    if (dtype == RAT_BF16 && d == 128 && n_sink == 0 && top_k == 0) {
         AttnSm100Args a;
         std::memset(&a, 0, sizeof(a));
         a.q = q; a.k = k_rec; a.v = v_rec; a.o = o;
@@ -336,6 +338,7 @@ int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, i
     p.rope = rope_base > 0.f ? 1 : 0;
     p.scale_log2 = scale_log2;
     p.n_sink = n_sink;
+    p.top_k = top_k;
     for (int h = 0; h < H; ++h) p.Dh[h] = Dh[h];
     if (p.rope) rope_theta(rope_base, d, p.theta);
     return launch_attn_simt(p, dtype, stream);
@@ -348,7 +351,7 @@ int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec
                              int H, int T, int d, int dtype, int D, int W,
                              const int32_t *D_per_head, int64_t pos0, float rope_base,
                              float scale, void *stream) {
-    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, 0, pos0,
+    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, 0, 0, pos0,
                         rope_base, scale, stream);
 }
 
@@ -356,8 +359,16 @@ int rat_dilated_attn_prefill_sinks(const void *q, const void *k_rec, const void 
                                    int B, int H, int T, int d, int dtype, int D, int W,
                                    const int32_t *D_per_head, int n_sink, int64_t pos0,
                                    float rope_base, float scale, void *stream) {
-    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, n_sink, pos0,
+    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, n_sink, 0, pos0,
                         rope_base, scale, stream);
+}
+
+int rat_dilated_attn_prefill_topk(const void *q, const void *k_rec, const void *v_rec, void *o,
+                                  int B, int H, int T, int d, int dtype, int D, int W,
+                                  const int32_t *D_per_head, int n_sink, int top_k, int64_t pos0,
+                                  float rope_base, float scale, void *stream) {
+    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, n_sink, top_k,
+                        pos0, rope_base, scale, stream);
 }
 
 size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int dtype) {
