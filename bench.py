@@ -182,15 +182,25 @@ def barrier(world: int):
 
 
 # ----------------------------------------------------------------------------- our arm
-def algorithmic(w: synthetic.Workload):
-    """Algorithmic bytes / FLOPs of one launch of each kernel on workload w."""
+def algorithmic(w: synthetic.Workload, n_sink: int = 0, top_k: int = 0):
+    """Algorithmic bytes / FLOPs of one launch of each kernel on workload w (with n_sink
+    attention sinks and top_k selected chunks added to every key set)."""
     import recurrence_augmented_dilated_b200 as rat
     eb = 4 if w.dtype == "f32" else 2
     N = w.B * w.H * w.T * w.d
+    We = max(w.W, 1)
     keys = 0
     for D in w.heads_D():
         # sum over queries of |S(t)| (closed form per t, summed in C by the library helper)
         keys += sum(rat.rat_attended_keys(t, D, w.W) for t in range(w.T))
+        for t in range(w.T):
+            lim = min(n_sink, max(0, t - We + 1))           # sinks older than the window
+            keys += lim - lim // D if D > 1 else 0
+            n_dil = (t - We + 1) // D if t - We + 1 >= D else 0
+            if top_k and D > 1:
+                # the positions of the selected chunks, less those that are sinks already
+                # (counted at most: every selected chunk taken in full)
+                keys += min(top_k, n_dil) * (D - 1)
     keys *= w.B
     cache_rows = sum(w.T // D for D in w.heads_D()) * w.B + w.B * w.H * min(w.W, w.T)
     return {
@@ -219,7 +229,7 @@ class ProfiledRegion:
 
 def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world: int, peaks,
                 peak_kind, with_e2e: bool, min_warmup_s: float = 1.0, reset_every: int = 0,
-                window: int = 0):
+                window: int = 0, n_sink: int = 0, top_k: int = 0):
     import recurrence_augmented_dilated_b200 as rat
     dev = torch.device("cuda")
     x = synthetic.prefill_inputs(w, seed=w.seed + 1000 * rank)
@@ -247,7 +257,7 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
                                       rope_base=w.rope_base)
         with span("attn"):
             rat.rat_dilated_attn_prefill(qq, kr, vr, o, D=w.D, W=w.W, D_per_head=Dph,
-                                         rope_base=w.rope_base)
+                                         rope_base=w.rope_base, n_sink=n_sink, top_k=top_k)
         cache.pos = 0
         with span("compress"):
             rat.rat_kv_compress(kr, vr, hk, hv, cache)
@@ -281,7 +291,7 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
     st = rat.rat_sync_status(ws)
     if st != 0:
         raise RuntimeError("device error " + rat.rat_status_string(st))
-    alg = algorithmic(w)
+    alg = algorithmic(w, n_sink, top_k)
     res = {
         "ms_per_step": ms_max,
         "tokens_per_s": world * B * T / (ms_max / 1e3),
@@ -762,6 +772,10 @@ def main():
                     help="also time ragged decode (context lengths T/2 .. T) on a paged cache")
     ap.add_argument("--backward", action="store_true",
                     help="also time the backward of the recurrence step on the workload")
+    ap.add_argument("--sinks", type=int, default=0,
+                    help="n > 0: the first n positions join every key set (attention sinks)")
+    ap.add_argument("--top-k", type=int, default=0,
+                    help="k > 0: the k best chunks (by chunk-end score) are attended in full")
     ap.add_argument("--window", type=int, default=0,
                     help="Lw > 0: the fixed-window recurrence (each state over the last Lw "
                          "positions) in the prefill step")
@@ -805,11 +819,13 @@ def main():
     rat.lib()       # fail loudly if the library is missing
 
     pre = run_prefill(w, args.steps, args.warmup, rank, world, peaks, peak_kind,
-                      with_e2e=not args.no_e2e and args.reset_every == 0 and args.window == 0,
+                      with_e2e=(not args.no_e2e and args.reset_every == 0 and args.window == 0 and
+                                args.sinks == 0 and args.top_k == 0),
                       min_warmup_s=args.min_warmup_s, reset_every=args.reset_every,
-                      window=args.window)
+                      window=args.window, n_sink=args.sinks, top_k=args.top_k)
     kern = pre["kernels"]
-    src_of = {"recur": "window.cu" if args.window else "scan.cu", "attn": "attn_sm100.cu",
+    src_of = {"recur": "window.cu" if args.window else "scan.cu",
+              "attn": "attn_simt.cu" if (args.sinks or args.top_k) else "attn_sm100.cu",
               "compress": "compress.cu"}
     variant = ("_L%d" % args.reset_every if args.reset_every else
                "_window%d" % args.window if args.window else "")
@@ -828,10 +844,14 @@ def main():
         "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "D": w.D, "W": w.W,
                    "D_per_head": list(w.D_per_head) if w.D_per_head else None,
                    "rope_base": w.rope_base, "gates": [w.gate_mu, w.gate_sigma],
-                   "step": "%s + rat_dilated_attn_prefill + rat_kv_compress" % (
+                   "step": "%s + %s + rat_kv_compress" % (
                        "rat_recur_prefill_window(Lw=%d)" % args.window if args.window else
                        "rat_recur_prefill_local(L=%d)" % args.reset_every if args.reset_every else
-                       "rat_recur_prefill"),
+                       "rat_recur_prefill",
+                       "rat_dilated_attn_prefill_topk(n_sink=%d, top_k=%d)" % (args.sinks, args.top_k)
+                       if args.top_k else
+                       "rat_dilated_attn_prefill_sinks(n_sink=%d)" % args.sinks if args.sinks else
+                       "rat_dilated_attn_prefill"),
                    "l2": "inputs larger than L2 (q, k, v, a = %d MB per rank)" % (
                        4 * w.B * w.H * w.T * w.d * (2 if w.dtype == "bf16" else 4) // 2**20),
                    "parallelism": "replicas: dp%d over (batch) with no collective" % world},
