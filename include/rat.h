@@ -246,8 +246,9 @@ RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const voi
  * chunk end is not repeated).  A StreamingLLM layer is D larger than any position (no chunk
  * ends), W its window, n_sink its sinks; sinks also combine with dilation.
  *   Arguments as rat_dilated_attn_prefill, plus n_sink >= 0 (0: exactly
- *   rat_dilated_attn_prefill).  Calls with n_sink > 0 run the CUDA-core kernel (float32
- *   arithmetic) for both dtypes. */
+ *   rat_dilated_attn_prefill).  bf16 with d = 128, n_sink <= 64 and no chunk end among the sinks
+ *   (every head has D = 1 or D > n_sink) runs the tensor-core kernel with the sinks as one more
+ *   key block; other calls run the CUDA-core kernel (float32 arithmetic). */
 RAT_API int rat_dilated_attn_prefill_sinks(const void *q, const void *k_rec, const void *v_rec,
                              void *o, int B, int H, int T, int d, int dtype, int D, int W,
                              const int32_t *D_per_head, int n_sink, int64_t pos0,

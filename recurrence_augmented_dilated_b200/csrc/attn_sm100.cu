@@ -95,6 +95,7 @@ struct Params {
     int grp_head0[kMaxHeads];       // first index into head_of
     int grp_nheads[kMaxHeads];
     int rope_f32;             // positions small enough for float32 angles (pos0 + T <= 2^13)
+    int n_sink;               // attention sinks (n_sink < D of every dilated head, <= BN)
     const float2 *rope_rel;   // device table [64 f][32 l] of (cos, sin)(l theta_f), see g_rope_rel
     float theta_f[64];
     double theta[64];
@@ -102,21 +103,26 @@ struct Params {
 
 RAT_DEVICE int floordiv(int a, int b) { return a >= 0 ? a / b : -((-a + b - 1) / b); }
 
-// Key blocks of one tile: nd dilated blocks (compressed indices 128*j ..) then nw window
-// blocks starting at position ws (contiguous).  Dense heads have nd = 0 and ws = 0.
+// Key blocks of one tile: ns sink blocks (0 or 1: positions 0 .. n_sink-1), nd dilated blocks
+// (compressed indices BN*j ..), then nw window blocks starting at position ws (contiguous).
+// Dense heads have ns = nd = 0 and ws = 0.  Sinks come here only when no chunk end is a sink
+// (n_sink < D) and n_sink <= BN, so the three sets stay disjoint with contiguous columns.
 struct Plan {
-    int nd, nw, ws, D, We;
+    int ns, nd, nw, ws, D, We, n_sink;
     bool dense;
     bool self_reg;    // We == 1 (dilated head): the self key is handled in registers, no window blocks
 };
 template <int BN>
-RAT_DEVICE Plan make_plan(int t0, int D, int W, int T) {
+RAT_DEVICE Plan make_plan(int t0, int D, int W, int T, int n_sink) {
     Plan pl;
     pl.D = D;
     pl.We = W > 1 ? W : 1;
     pl.dense = D == 1;
     pl.self_reg = !pl.dense && pl.We == 1;
+    pl.n_sink = n_sink;
     const int tmax = t0 + BM - 1;
+    // a sink block when some query of the tile has a sink older than its window
+    pl.ns = (!pl.dense && n_sink > 0 && tmax - pl.We + 1 > 0) ? 1 : 0;
     if (pl.dense) {
         pl.nd = 0;
         pl.ws = 0;
@@ -135,6 +141,13 @@ RAT_DEVICE Plan make_plan(int t0, int D, int W, int T) {
 // Columns [c_lo, c_hi] of block j that query t may attend to.
 template <int BN>
 RAT_DEVICE void block_range(const Plan &pl, int j, int t, int &c_lo, int &c_hi) {
+    if (j < pl.ns) {
+        // sinks older than the window: positions 0 .. min(n_sink, t - We + 1) - 1
+        c_lo = 0;
+        c_hi = min(pl.n_sink, t - pl.We + 1) - 1;
+        return;
+    }
+    j -= pl.ns;
     if (j < pl.nd) {
         // chunk end i = BN j + c is attended iff i*D + D - 1 <= t - We
         c_lo = 0;
@@ -224,9 +237,9 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
     const int b = (local % per_row) / p.grp_nheads[g];
     const int h = p.head_of[p.grp_head0[g] + (local % per_row) % p.grp_nheads[g]];
     const int bh = b * p.H + h;
-    const Plan pl = make_plan<BN>(t0, p.Dh[h], p.W, p.T);
+    const Plan pl = make_plan<BN>(t0, p.Dh[h], p.W, p.T, p.n_sink);
     const bool self_reg = SELF && pl.self_reg;      // pl.self_reg implies W <= 1, hence SELF
-    const int nb = pl.nd + pl.nw;
+    const int nb = pl.ns + pl.nd + pl.nw;
 
     if (threadIdx.x == 0) {
         mbar_init(&sh.q_full, 1);
@@ -269,7 +282,14 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             if (p.rope) bulk_g2s(smem + C::OFF_K + C::KTILE, p.rope_rel, kRelBytes, &sh.q_full);
             // K runs one block ahead of V: S(j) needs K(j) long before PV(j) needs V(j), and a K
             // stage frees up as soon as its S has completed
-            auto row_of = [&](int j) { return j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd); };
+            // first key row of block j: the sinks at row 0, a dilated block in the compressed
+            // view, a window block in the plain one
+            auto row_of = [&](int j) {
+                if (j < pl.ns) return 0;
+                j -= pl.ns;
+                return j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd);
+            };
+            auto dil_blk = [&](int j) { return j >= pl.ns && j - pl.ns < pl.nd; };
             int k_issued = 0, v_issued = 0;
             for (int j = 0; j <= nb; ++j) {
                 if (j < nb) {
@@ -277,7 +297,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                     if (j >= NS && !wait_bar(sh, &sh.k_empty[s], ((j / NS) - 1) & 1, 1, j)) break;
                     // with RoPE, stage 1 holds the softmax warps' rotation tables until Q is rotated
                     if (j == 1 && p.rope && !wait_bar(sh, &sh.q_ready, 0, 10, j)) break;
-                    const CUtensorMap *tk = j < pl.nd ? mk : &p.tm_k;
+                    const CUtensorMap *tk = dil_blk(j) ? mk : &p.tm_k;
                     uint8_t *ks = smem + C::OFF_K + s * C::KTILE;
                     mbar_arrive_expect_tx(&sh.k_full[s], C::KTILE);
                     tc::tma_load_3d(ks, tk, 0, row_of(j), bh, &sh.k_full[s]);
@@ -287,7 +307,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                 if (j >= 1) {
                     const int jv = j - 1, s = jv % NS;
                     if (jv >= NS && !wait_bar(sh, &sh.v_empty[s], ((jv / NS) - 1) & 1, 11, jv)) break;
-                    const CUtensorMap *tv = jv < pl.nd ? mv : &p.tm_v;
+                    const CUtensorMap *tv = dil_blk(jv) ? mv : &p.tm_v;
                     uint8_t *vs = smem + C::OFF_V + s * C::KTILE;
                     mbar_arrive_expect_tx(&sh.v_full[s], C::KTILE);
                     tc::tma_load_3d(vs, tv, 0, row_of(jv), bh, &sh.v_full[s]);
@@ -706,6 +726,7 @@ int fill_params(Params &p, const AttnSm100Args &a) {
     p.pos0 = a.pos0;
     p.rope = a.rope;
     p.rope_f32 = a.pos0 + (long long)a.T <= 8192 ? 1 : 0;
+    p.n_sink = a.n_sink;
     p.scale_log2 = a.scale_log2;
     for (int c = 0; c < 64; ++c) {
         p.theta[c] = a.theta[c];

@@ -113,6 +113,7 @@ struct AttnSm100Args {
     int rope;
     float scale_log2;
     const int32_t *Dh;          // host [H]
+    int n_sink;                 // attention sinks; the caller ensures n_sink < D (D > 1) and <= 64
     double theta[64];
 };
 int launch_attn_sm100(const AttnSm100Args &a, void *stream);

@@ -318,7 +318,11 @@ int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, i
     int32_t Dh[kMaxHeads];
     for (int h = 0; h < H; ++h) Dh[h] = D_per_head ? D_per_head[h] : D;
 
-    if (dtype == RAT_BF16 && d == 128 && n_sink == 0 && top_k == 0) {
+    // the tensor-core kernel takes sinks as one extra key block when no chunk end is a sink
+    bool sinks_fit = n_sink <= 64;
+    for (int h = 0; h < H; ++h)
+        if (Dh[h] > 1 && Dh[h] <= n_sink) sinks_fit = false;
+    if (dtype == RAT_BF16 && d == 128 && top_k == 0 && (n_sink == 0 || sinks_fit)) {
         AttnSm100Args a;
         std::memset(&a, 0, sizeof(a));
         a.q = q; a.k = k_rec; a.v = v_rec; a.o = o;
@@ -327,6 +331,7 @@ int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, i
         a.rope = rope_base > 0.f ? 1 : 0;
         a.scale_log2 = scale_log2;
         a.Dh = Dh;
+        a.n_sink = n_sink;
         if (a.rope) rope_theta(rope_base, d, a.theta);
         return launch_attn_sm100(a, stream);
     }
