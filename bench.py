@@ -242,10 +242,13 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
     cache, bufs = rat.make_cache(B, H, d, w.W, T, dtc, w.heads_D())
     ws = rat.Workspace(rat.rat_recur_workspace_bytes(B, H, T, d, dtc))
     stream = torch.cuda.current_stream()
+    side = torch.cuda.Stream()          # the cache append runs beside the attention
+    side_timer = EventTimer(side)
     Dph = list(w.D_per_head) if w.D_per_head else None
 
     def step(timer=None, qq=q, kk=k, vv=v, aa=a):
         span = timer.span if timer else (lambda n: _Null())
+        sspan = side_timer.span if timer else (lambda n: _Null())
         with span("recur"):
             if window > 0:
                 rat.rat_recur_prefill_window(kk, vv, aa, kr, vr, ws, window, rope_base=w.rope_base)
@@ -255,12 +258,17 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
             else:
                 rat.rat_recur_prefill(kk, vv, aa, kr, vr, ws, hT_k=hk, hT_v=hv,
                                       rope_base=w.rope_base)
+        # the attention and the cache append both read only the recurrence outputs: the append
+        # runs on a second stream while the attention runs, and the step ends when both have
+        side.wait_stream(stream)
+        cache.pos = 0
+        with torch.cuda.stream(side):
+            with sspan("compress"):
+                rat.rat_kv_compress(kr, vr, hk, hv, cache, stream=side)
         with span("attn"):
             rat.rat_dilated_attn_prefill(qq, kr, vr, o, D=w.D, W=w.W, D_per_head=Dph,
                                          rope_base=w.rope_base, n_sink=n_sink, top_k=top_k)
-        cache.pos = 0
-        with span("compress"):
-            rat.rat_kv_compress(kr, vr, hk, hv, cache)
+        stream.wait_stream(side)
 
     timer = EventTimer(stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -288,6 +296,7 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
     ms = e0.elapsed_time(e1) / steps
     ms_max = max_over_ranks(ms, world)
     kern = timer.mean_ms()
+    kern.update(side_timer.mean_ms())
     st = rat.rat_sync_status(ws)
     if st != 0:
         raise RuntimeError("device error " + rat.rat_status_string(st))
@@ -302,7 +311,7 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
     hbm = peaks["hbm_gbs"]
     tc = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     for name, t in kern.items():
-        e = {"ms": t, "share": t / sum(kern.values())}
+        e = {"ms": t, "share_of_kernel_time": t / sum(kern.values())}
         if name == "recur":
             e.update(bound="hbm", achieved=alg["recur_bytes"] / (t * 1e-3) / 1e9, peak=hbm, unit="GB/s")
         elif name == "attn":
@@ -315,7 +324,10 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
             else:
                 e.update(bound="tensor", achieved=tfs, peak=tc, unit="TFLOP/s", gbs=gbs)
         elif name == "compress":
-            e.update(bound="hbm", achieved=alg["compress_bytes"] / (t * 1e-3) / 1e9, peak=hbm, unit="GB/s")
+            # launched beside the attention: the span runs from its launch until the attention
+            # leaves it SM slots, so it is not the kernel's own duration
+            e.update(bound="hbm", achieved=alg["compress_bytes"] / (t * 1e-3) / 1e9, peak=hbm, unit="GB/s",
+                     overlapped_with="attn")
         e["frac"] = e["achieved"] / e["peak"]
         e["of"] = peak_kind
         res["kernels"][name] = e
@@ -831,7 +843,8 @@ def main():
                "_window%d" % args.window if args.window else "")
     for n in kern:      # DRAM bytes per launch from the committed ncu capture (null if stale)
         kern[n]["traffic"] = recorded_traffic(src_of[n], w.name + (variant if n == "recur" else ""))
-    dom_name = max(kern, key=lambda n: kern[n]["ms"])
+    # the dominant kernel of the step (the cache append overlaps the attention)
+    dom_name = max((n for n in kern if not kern[n].get("overlapped_with")), key=lambda n: kern[n]["ms"])
     dom = kern[dom_name]
     roof = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
             "unit": dom["unit"], "frac": dom["frac"], "of": peak_kind, "kernel": dom_name,
@@ -844,7 +857,7 @@ def main():
         "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "D": w.D, "W": w.W,
                    "D_per_head": list(w.D_per_head) if w.D_per_head else None,
                    "rope_base": w.rope_base, "gates": [w.gate_mu, w.gate_sigma],
-                   "step": "%s + %s + rat_kv_compress" % (
+                   "step": "%s + %s + rat_kv_compress (on a second stream, beside the attention)" % (
                        "rat_recur_prefill_window(Lw=%d)" % args.window if args.window else
                        "rat_recur_prefill_local(L=%d)" % args.reset_every if args.reset_every else
                        "rat_recur_prefill",

@@ -288,21 +288,6 @@ RAT_DEVICE void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, u
         :: "r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
-// One-dimensional bulk copy shared -> global (the untiled TMA store), in the current bulk
-// group.  Both addresses 16-byte aligned, bytes a multiple of 16.  Generic-proxy writes to the
-// source must be made visible first (fence_proxy_async_shared by the writers, then a barrier).
-RAT_DEVICE void bulk_s2g(void *gmem_dst, const void *smem_src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
-                 :: "l"(gmem_dst), "r"(smem_u32(smem_src)), "r"(bytes) : "memory");
-}
-RAT_DEVICE void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Wait until at most N of this thread's most recent bulk groups still read their source.
-template <int N>
-RAT_DEVICE void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read %0;" :: "n"(N) : "memory"); }
-// Wait until all of this thread's bulk groups have completed.
-RAT_DEVICE void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-RAT_DEVICE void fence_proxy_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
 RAT_DEVICE void ld_shared_v4(const void *p, uint32_t &a, uint32_t &b, uint32_t &c, uint32_t &d) {
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(smem_u32(p)));
