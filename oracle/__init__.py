@@ -66,7 +66,7 @@ def _load():
         lib.rat_oracle_key_count_sinks.argtypes = [_L, _L, _L, _L]
         lib.rat_oracle_key_count_sinks.restype = ctypes.c_long
         lib.rat_oracle_dilated_attention.argtypes = [_L, _L, _L, _dp, _dp, _dp, _ip, _L, _L,
-                                                     ctypes.c_double, _lp, _L, _dp]
+                                                     ctypes.c_double, _lp, _L, _dp, _dp]
         lib.rat_oracle_kv_compress.argtypes = [_L, _L, _L, _L, _L, _bp, _ip, _L, _L, _L, _bp, _bp]
         lib.rat_oracle_decode_step.argtypes = [_L, _L, _L, _ip, _L, _L, ctypes.c_double,
                                                ctypes.c_double, _dp, _dp, _dp, _dp, _dp, _dp,
@@ -233,14 +233,15 @@ def _per_bh_dilation(shape_bh, D, D_per_head):
     return np.ascontiguousarray(np.tile(Dh, B).astype(np.int32)), Dh
 
 
-def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None, n_sink=0):
+def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None, n_sink=0,
+                      return_lse=False):
     """Causal dilated attention (+ local window, per-head D) over (B, H, T, d) tensors.
 
     q, k, v are used as given (rotate them first if RoPE is in use).  rows: optional list of
     query positions; the result then has shape (B, H, len(rows), d).  n_sink > 0 adds the first
     n_sink positions to every key set (StreamingLLM attention sinks).
     (RAT+ abstract; "RAT+ Deep Dive" section 3.1 table and section 6 head-wise and layer-wise
-    hybrids.)
+    hybrids.)  return_lse: also return log2 of each row's softmax denominator, (B, H, rows).
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, H, T, d = q.shape
@@ -255,9 +256,11 @@ def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None,
         assert rows_a.min() >= 0 and rows_a.max() < T
         nrows, rp = len(rows_a), _ptr(rows_a, _lp)
         out = np.empty((B, H, nrows, d))
+    lse = np.empty(out.shape[:-1]) if return_lse else None
     _load().rat_oracle_dilated_attention(B * H, T, d, _ptr(q), _ptr(k), _ptr(v), _ptr(Dbh, _ip),
-                                         int(W), int(n_sink), float(scale), rp, nrows, _ptr(out))
-    return out
+                                         int(W), int(n_sink), float(scale), rp, nrows, _ptr(out),
+                                         _ptr(lse) if return_lse else None)
+    return (out, lse) if return_lse else out
 
 
 def topk_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, n_sink=0, top_k=0):

@@ -256,6 +256,8 @@ static long list_keys(long t, long D, long We, long n_sink, long *keys)
  *   Dbh     : [BH]        dilation of each (batch, head) slice
  *   rows    : [nrows]     query positions to evaluate (NULL: all T rows, nrows = T)
  *   o       : [BH][nrows][d]
+ *   lse     : [BH][nrows] or NULL: log2 of sum_j exp(s_j), the softmax denominator in base-2
+ *             units (what the backward needs to rebuild the weights)
  * For each query t:  s_j = scale * <q_t, k_j>  for j in S(t);
  *                    o_t = sum_j exp(s_j - max s) v_j / sum_j exp(s_j - max s).
  * S(t) is enumerated as its two parts: the window t-We < j <= t, then the chunk ends
@@ -263,7 +265,8 @@ static long list_keys(long t, long D, long We, long n_sink, long *keys)
  */
 void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, const double *k,
                                   const double *v, const int *Dbh, long W, long n_sink,
-                                  double scale, const long *rows, long nrows, double *o)
+                                  double scale, const long *rows, long nrows, double *o,
+                                  double *lse)
 {
     long We = eff_window(W);
     if (!rows) nrows = T;
@@ -294,6 +297,8 @@ void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, cons
                 for (long c = 0; c < d; ++c) ot[c] += p * vj[c];
             }
             for (long c = 0; c < d; ++c) ot[c] /= l;
+            /* log2 of the softmax denominator sum_j 2^(s_j log2 e): (max s + ln l) / ln 2 */
+            if (lse) lse[bh * nrows + r] = (mx + log(l)) / log(2.0);
         }
         free(keys);
         free(s);

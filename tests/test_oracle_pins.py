@@ -501,6 +501,18 @@ def test_topk_equals_masked_sdpa_with_argsort_selection(D, W, n_sink, top_k):
     np.testing.assert_allclose(got, ref.numpy(), rtol=1e-11, atol=1e-12)
 
 
+def test_attention_lse_is_the_log_partition():
+    # log2 sum_j exp(s_j) over the key set, by a library logsumexp over the masked scores
+    from scipy.special import logsumexp
+    T, d, D, W, scale = 33, 8, 4, 3, 0.4
+    q, k, v = (RNG.standard_normal((1, 1, T, d)) for _ in range(3))
+    _, lse = oracle.dilated_attention(q, k, v, D=D, W=W, n_sink=2, scale=scale, return_lse=True)
+    for t in range(T):
+        keys = [j for j in range(t + 1) if oracle.in_key_set(t, j, D, W, 2)]
+        sc = scale * (k[0, 0, keys] @ q[0, 0, t])
+        assert abs(lse[0, 0, t] - logsumexp(sc) / np.log(2.0)) <= 1e-12
+
+
 def test_rope_matches_complex_rotation():
     d, T, pos0, base = 16, 9, 1000, 10000.0
     x = RNG.standard_normal((1, T, d))
