@@ -677,14 +677,16 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     q = x["q"].to(dev)
     o = torch.empty_like(q)
     Dph = list(w.D_per_head) if w.D_per_head else None
-    rat.rat_dilated_attn_prefill(q, kr, vr, o, D=w.D, W=w.W, D_per_head=Dph, rope_base=w.rope_base)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)    # saved by the forward
+    rat.rat_dilated_attn_prefill(q, kr, vr, o, D=w.D, W=w.W, D_per_head=Dph, rope_base=w.rope_base,
+                                 lse=lse)
     dO = torch.randn(q.shape, generator=g, device=dev).to(q.dtype)
     dq, dkr, dvr = torch.empty_like(q), torch.empty_like(kr), torch.empty_like(vr)
     ws_a = rat.Workspace(rat.rat_dilated_attn_backward_workspace_bytes(B, H, T, d, dtc))
 
     def astep():
         rat.rat_dilated_attn_backward(q, kr, vr, o, dO, dq, dkr, dvr, ws_a, D=w.D, W=w.W,
-                                      D_per_head=Dph, rope_base=w.rope_base)
+                                      D_per_head=Dph, rope_base=w.rope_base, lse=lse)
 
     for _ in range(warmup):
         astep()
@@ -700,7 +702,8 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     pairs = sum(rat.rat_attended_keys(t, D_, w.W) for D_ in w.heads_D() for t in range(T)) * B
     aflops = 10 * d * pairs                 # per pair: recomputed score, dp, dq, dk, dv
     a_ach = abytes / (ams * 1e-3) / 1e9
-    res["attention"] = {"step": "rat_dilated_attn_backward (3 CUDA-core launches)", "ms": ams,
+    res["attention"] = {"step": "rat_dilated_attn_backward (3 CUDA-core launches, the forward's "
+                                "log-sum-exp given)", "ms": ams,
                         "roofline": {"bound": "hbm", "achieved": a_ach, "peak": peaks["hbm_gbs"],
                                      "unit": "GB/s", "frac": a_ach / peaks["hbm_gbs"],
                                      "of": peak_kind, "algorithmic_bytes": abytes,

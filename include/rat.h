@@ -274,6 +274,28 @@ RAT_API int rat_dilated_attn_prefill_topk(const void *q, const void *k_rec, cons
 RAT_API int rat_attn_sync_status(void *stream);
 
 /* ------------------------------------------------------------------------------------------
+ * rat_dilated_attn_prefill_ex -- the attention with every option of this library.
+ *   Arguments as rat_dilated_attn_prefill, plus opt (NULL: no option):
+ *     n_sink : attention sinks (as rat_dilated_attn_prefill_sinks)
+ *     top_k  : chunks attended in full (as rat_dilated_attn_prefill_topk)
+ *     lse    : device float32 [B][H][T] output, or NULL: log2 of each query's softmax
+ *              denominator, log2 sum_j 2^(s_j log2 e) with s_j = scale <q^_t, k~_j> -- the
+ *              value rat_dilated_attn_backward takes to rebuild the weights (4-byte aligned)
+ *   Dispatch as for the other entry points (tensor cores for bf16, d = 128 when the options
+ *   allow it).
+ * ---------------------------------------------------------------------------------------- */
+typedef struct rat_attn_options {
+    int32_t n_sink;           /* attention sinks, >= 0                                     */
+    int32_t top_k;            /* chunks attended in full, 0 .. 16                          */
+    float *lse;               /* optional output, see above                                */
+} rat_attn_options;
+
+RAT_API int rat_dilated_attn_prefill_ex(const void *q, const void *k_rec, const void *v_rec,
+                             void *o, int B, int H, int T, int d, int dtype, int D, int W,
+                             const int32_t *D_per_head, int64_t pos0, float rope_base,
+                             float scale, const rat_attn_options *opt, void *stream);
+
+/* ------------------------------------------------------------------------------------------
  * rat_dilated_attn_backward -- gradients of rat_dilated_attn_prefill (training with dilated
  * samples: "RAT+ Deep Dive" section 2.2 trains half the samples with D = 1 and half with
  * D = 64, which needs this derivative for every D).
@@ -287,19 +309,21 @@ RAT_API int rat_attn_sync_status(void *stream);
  *                        gradients of k~, v~: the dk_rec, dv_rec inputs of rat_recur_backward)
  *   D, W, D_per_head, n_sink, pos0, rope_base, scale : as given to the forward
  *                        (rat_dilated_attn_prefill_sinks; n_sink = 0 without sinks)
+ *   lse                : device float32 [B][H][T], the forward's rat_attn_options.lse output,
+ *                        or NULL (the denominators are then recomputed: one more walk over
+ *                        every key set)
  *   ws, ws_bytes       : workspace of at least rat_dilated_attn_backward_workspace_bytes
- * CUDA-core kernels with float32 accumulation: the softmax denominators are recomputed (not
- * taken from the forward), q^ is rounded to the dtype as the forward's operand is, outputs are
- * rounded once.  Three launches (prep, dq, dk~ and dv~); no device-side waits.
+ * CUDA-core kernels with float32 accumulation: q^ is rounded to the dtype as the forward's
+ * operand is, outputs are rounded once.  Three launches (prep, dq, dk~ and dv~); no device-side waits.
  * ---------------------------------------------------------------------------------------- */
 RAT_API size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int dtype);
 
 RAT_API int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_rec,
                               const void *o, const void *dO, void *dq, void *dk_rec,
                               void *dv_rec, int B, int H, int T, int d, int dtype, int D, int W,
-                              const int32_t *D_per_head, int n_sink, int64_t pos0,
-                              float rope_base, float scale, void *ws, size_t ws_bytes,
-                              void *stream);
+                              const int32_t *D_per_head, int n_sink, const float *lse,
+                              int64_t pos0, float rope_base, float scale, void *ws,
+                              size_t ws_bytes, void *stream);
 
 /* Diagnostic: where the attention kernel's last recorded timeout happened, as
  * (wait site << 24) | (key block << 8) | phase parity; sites: 1 producer K-stage-free, 2 MMA

@@ -27,7 +27,7 @@ __all__ = [
     "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
     "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
-    "Workspace", "rat_dilated_decode_noalloc", "PagedKVCache", "make_paged_cache",
+    "Workspace", "rat_dilated_decode_noalloc", "PagedKVCache", "make_paged_cache", "AttnOptions",
     "rat_paged_kv_compress", "rat_paged_decode_workspace_bytes", "rat_dilated_decode_paged",
 ]
 
@@ -57,6 +57,11 @@ class KVCache(ctypes.Structure):
         ("pos", ctypes.c_int64), ("reset_every", ctypes.c_int64),
         ("n_sink", ctypes.c_int32), ("k_sink", ctypes.c_void_p), ("v_sink", ctypes.c_void_p),
     ]
+
+
+class AttnOptions(ctypes.Structure):
+    """Mirror of struct rat_attn_options."""
+    _fields_ = [("n_sink", ctypes.c_int32), ("top_k", ctypes.c_int32), ("lse", ctypes.c_void_p)]
 
 
 class PagedKVCache(ctypes.Structure):
@@ -98,7 +103,10 @@ def lib():
         L.rat_dilated_attn_backward_workspace_bytes.argtypes = [_i, _i, _i, _i, _i]
         L.rat_dilated_attn_backward.argtypes = [_vp] * 8 + [_i, _i, _i, _i, _i, _i, _i,
                                                             ctypes.POINTER(ctypes.c_int32), _i,
-                                                            _i64, _f, _f, _vp, _sz, _vp]
+                                                            _vp, _i64, _f, _f, _vp, _sz, _vp]
+        L.rat_dilated_attn_prefill_ex.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
+                                                  ctypes.POINTER(ctypes.c_int32), _i64, _f, _f,
+                                                  ctypes.POINTER(AttnOptions), _vp]
         L.rat_dilated_attn_prefill_sinks.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i,
                                                      _i, ctypes.POINTER(ctypes.c_int32), _i,
                                                      _i64, _f, _f, _vp]
@@ -265,14 +273,24 @@ def rat_recur_prefill_window(k, v, gate_logit, k_rec, v_rec, ws: Workspace, Lw: 
 def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,
                              D_per_head: Optional[Sequence[int]] = None, pos0: int = 0,
                              rope_base: float = 0.0, scale: float = 0.0, stream=None,
-                             n_sink: int = 0, top_k: int = 0):
+                             n_sink: int = 0, top_k: int = 0, lse=None):
     """o = dilated attention of q over (k_rec, v_rec); all (B, H, T, d).  n_sink > 0 adds the
     first n_sink positions to every key set (rat_dilated_attn_prefill_sinks); top_k > 0 adds
-    the top_k chunks by their chunk-end scores (rat_dilated_attn_prefill_topk)."""
+    the top_k chunks by their chunk-end scores (rat_dilated_attn_prefill_topk); lse, a float32
+    (B, H, T) tensor, receives log2 of every row's softmax denominator
+    (rat_dilated_attn_prefill_ex)."""
     B, H, T, d = q.shape
     dph = None
     if D_per_head is not None:
         dph = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
+    if lse is not None:
+        opt = AttnOptions(n_sink=int(n_sink), top_k=int(top_k), lse=lse.data_ptr())
+        st = lib().rat_dilated_attn_prefill_ex(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), B, H, T,
+                                               d, _dtype_code(q), int(D), int(W), dph, int(pos0),
+                                               float(rope_base), float(scale), ctypes.byref(opt),
+                                               _stream(stream))
+        _check("rat_dilated_attn_prefill_ex", st)
+        return
     if top_k:
         st = lib().rat_dilated_attn_prefill_topk(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), B, H,
                                                  T, d, _dtype_code(q), int(D), int(W), dph,
@@ -300,8 +318,9 @@ def rat_dilated_attn_backward_workspace_bytes(B, H, T, d, dtype) -> int:
 def rat_dilated_attn_backward(q, k_rec, v_rec, o, dO, dq, dk_rec, dv_rec, ws: Workspace,
                               D: int = 1, W: int = 0, D_per_head: Optional[Sequence[int]] = None,
                               pos0: int = 0, rope_base: float = 0.0, scale: float = 0.0,
-                              stream=None, n_sink: int = 0):
-    """Gradients of rat_dilated_attn_prefill(_sinks): dq, dk_rec, dv_rec (all (B, H, T, d))."""
+                              stream=None, n_sink: int = 0, lse=None):
+    """Gradients of rat_dilated_attn_prefill(_sinks): dq, dk_rec, dv_rec (all (B, H, T, d));
+    lse: the forward's (B, H, T) float32 output, or None (recomputed)."""
     B, H, T, d = q.shape
     dph = None
     if D_per_head is not None:
@@ -309,8 +328,8 @@ def rat_dilated_attn_backward(q, k_rec, v_rec, o, dO, dq, dk_rec, dv_rec, ws: Wo
     st = lib().rat_dilated_attn_backward(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), _ptr(dO),
                                          _ptr(dq), _ptr(dk_rec), _ptr(dv_rec), B, H, T, d,
                                          _dtype_code(q), int(D), int(W), dph, int(n_sink),
-                                         int(pos0), float(rope_base), float(scale), ws.ptr,
-                                         ws.nbytes, _stream(stream))
+                                         _ptr(lse), int(pos0), float(rope_base), float(scale),
+                                         ws.ptr, ws.nbytes, _stream(stream))
     _check("rat_dilated_attn_backward", st)
 
 

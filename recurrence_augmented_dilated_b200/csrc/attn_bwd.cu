@@ -93,9 +93,9 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const __grid_constant_
         return s + s / (D - 1);
     };
 
-    // pass 1: the softmax denominator (log2 units)
+    // pass 1: the softmax denominator (log2 units), unless the forward's is given
     float m = -INFINITY, l = 0.f;
-    for (int base = 0; base < n; base += 4) {
+    for (int base = 0; base < (p.lse_given ? 0 : n); base += 4) {
         float kx[4][CPL];
 #pragma unroll
         for (int u = 0; u < 4; ++u)
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const __grid_constant_
             }
         }
     }
-    const float lse = m + log2f(l);
+    const float lse = p.lse_given ? p.lse[row + t] : m + log2f(l);
     // pass 2: dq^ = scale sum_j p_j (<dO, v_j> - delta) k_j
     float dq[CPL];
 #pragma unroll
@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const __grid_constant_
     for (int j = 0; j < CPL; ++j) dq[j] *= p.scale;
     if (p.rope) rope_lane<DH>(p, p.pos0 + t, lane, -1.f, dq);
     RowIO<E, CPL>::store(static_cast<uint8_t *>(p.dq) + off, dq);
-    if (lane == 0) p.lse[row + t] = lse;
+    if (lane == 0 && !p.lse_given) p.lse[row + t] = lse;
 }
 
 template <typename E, int DH>

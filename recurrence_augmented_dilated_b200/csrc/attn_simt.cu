@@ -141,6 +141,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const __grid_constant__ 
 #pragma unroll
     for (int j = 0; j < CPL; ++j) o[j] *= inv;
     RowIO<E, CPL>::store(static_cast<uint8_t *>(p.o) + qoff, o);
+    if (p.lse && lane == 0) p.lse[(size_t)bh * p.T + t] = m + log2f(l);
 }
 
 int launch_attn_simt(const AttnSimtParams &p, int dtype, void *stream) {

@@ -96,6 +96,7 @@ struct Params {
     int grp_nheads[kMaxHeads];
     int rope_f32;             // positions small enough for float32 angles (pos0 + T <= 2^13)
     int n_sink;               // attention sinks (n_sink < D of every dilated head, <= BN)
+    float *lse;               // [B*H][T] or null: log2 of each row's softmax denominator
     const float2 *rope_rel;   // device table [64 f][32 l] of (cos, sin)(l theta_f), see g_rope_rel
     float theta_f[64];
     double theta[64];
@@ -582,6 +583,8 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             }
             tc::fence_after_sync();
             const float inv = 1.0f / (l_run + w_self);
+            // the row's softmax denominator, for the backward (m_run is in log2-scaled units)
+            if (p.lse && t < p.T) p.lse[(size_t)bh * p.T + t] = m_run + log2f(l_run + w_self);
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
@@ -727,6 +730,7 @@ int fill_params(Params &p, const AttnSm100Args &a) {
     p.rope = a.rope;
     p.rope_f32 = a.pos0 + (long long)a.T <= 8192 ? 1 : 0;
     p.n_sink = a.n_sink;
+    p.lse = a.lse;
     p.scale_log2 = a.scale_log2;
     for (int c = 0; c < 64; ++c) {
         p.theta[c] = a.theta[c];

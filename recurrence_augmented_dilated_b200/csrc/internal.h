@@ -100,6 +100,7 @@ struct AttnSimtParams {
     float scale_log2;           // softmax scale * log2(e)
     int n_sink;                 // attention sinks: the first n_sink positions join every key set
     int top_k;                  // chunks (scored by their chunk-end keys) attended in full, <= 16
+    float *lse;                 // [B*H][T] or null: log2 of each row's softmax denominator
     int Dh[kMaxHeads];
     double theta[64];
 };
@@ -114,6 +115,7 @@ struct AttnSm100Args {
     float scale_log2;
     const int32_t *Dh;          // host [H]
     int n_sink;                 // attention sinks; the caller ensures n_sink < D (D > 1) and <= 64
+    float *lse;                 // [B*H][T] or null: log2 of each row's softmax denominator
     double theta[64];
 };
 int launch_attn_sm100(const AttnSm100Args &a, void *stream);
@@ -172,7 +174,9 @@ struct AttnBwdParams {
     const void *q, *k, *v, *o, *dO;
     void *dq, *dk, *dv;
     void *qh;                   // workspace [B*H][T][d] of dtype: RoPE(q) as the attention uses it
-    float *lse;                 // workspace [B*H][T]: log2 of each query's softmax denominator
+    float *lse;                 // [B*H][T]: log2 of each query's softmax denominator (workspace,
+                                // or the forward's output when lse_given)
+    int lse_given;              // 1: lse holds the forward's values, the dq launch skips its pass 1
     float *delta;               // workspace [B*H][T]: <dO_t, o_t>
     int B, H, T, d, W, n_sink;
     long long pos0;

@@ -297,7 +297,8 @@ int rat_recur_prefill_local(const void *k, const void *v, const void *gate_logit
 namespace {
 int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, int B, int H,
                  int T, int d, int dtype, int D, int W, const int32_t *D_per_head, int n_sink,
-                 int top_k, int64_t pos0, float rope_base, float scale, void *stream) {
+                 int top_k, float *lse, int64_t pos0, float rope_base, float scale,
+                 void *stream) {
     if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0 || n_sink < 0 ||
         top_k < 0)
         return RAT_ERR_INVALID;
@@ -332,6 +333,7 @@ int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, i
         a.scale_log2 = scale_log2;
         a.Dh = Dh;
         a.n_sink = n_sink;
+        a.lse = lse;
         if (a.rope) rope_theta(rope_base, d, a.theta);
         return launch_attn_sm100(a, stream);
     }
@@ -344,6 +346,7 @@ int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, i
     p.scale_log2 = scale_log2;
     p.n_sink = n_sink;
     p.top_k = top_k;
+    p.lse = lse;
     for (int h = 0; h < H; ++h) p.Dh[h] = Dh[h];
     if (p.rope) rope_theta(rope_base, d, p.theta);
     return launch_attn_simt(p, dtype, stream);
@@ -356,16 +359,16 @@ int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec
                              int H, int T, int d, int dtype, int D, int W,
                              const int32_t *D_per_head, int64_t pos0, float rope_base,
                              float scale, void *stream) {
-    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, 0, 0, pos0,
-                        rope_base, scale, stream);
+    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, 0, 0, nullptr,
+                        pos0, rope_base, scale, stream);
 }
 
 int rat_dilated_attn_prefill_sinks(const void *q, const void *k_rec, const void *v_rec, void *o,
                                    int B, int H, int T, int d, int dtype, int D, int W,
                                    const int32_t *D_per_head, int n_sink, int64_t pos0,
                                    float rope_base, float scale, void *stream) {
-    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, n_sink, 0, pos0,
-                        rope_base, scale, stream);
+    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, n_sink, 0,
+                        nullptr, pos0, rope_base, scale, stream);
 }
 
 int rat_dilated_attn_prefill_topk(const void *q, const void *k_rec, const void *v_rec, void *o,
@@ -373,7 +376,19 @@ int rat_dilated_attn_prefill_topk(const void *q, const void *k_rec, const void *
                                   const int32_t *D_per_head, int n_sink, int top_k, int64_t pos0,
                                   float rope_base, float scale, void *stream) {
     return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, n_sink, top_k,
-                        pos0, rope_base, scale, stream);
+                        nullptr, pos0, rope_base, scale, stream);
+}
+
+int rat_dilated_attn_prefill_ex(const void *q, const void *k_rec, const void *v_rec, void *o,
+                                int B, int H, int T, int d, int dtype, int D, int W,
+                                const int32_t *D_per_head, int64_t pos0, float rope_base,
+                                float scale, const rat_attn_options *opt, void *stream) {
+    if (!opt)
+        return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, 0, 0, nullptr,
+                            pos0, rope_base, scale, stream);
+    if (opt->lse && (reinterpret_cast<uintptr_t>(opt->lse) & 3u)) return RAT_ERR_INVALID;
+    return attn_prefill(q, k_rec, v_rec, o, B, H, T, d, dtype, D, W, D_per_head, opt->n_sink,
+                        opt->top_k, opt->lse, pos0, rope_base, scale, stream);
 }
 
 size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int dtype) {
@@ -384,8 +399,8 @@ size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int
 int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_rec, const void *o,
                               const void *dO, void *dq, void *dk_rec, void *dv_rec, int B, int H,
                               int T, int d, int dtype, int D, int W, const int32_t *D_per_head,
-                              int n_sink, int64_t pos0, float rope_base, float scale, void *ws,
-                              size_t ws_bytes, void *stream) {
+                              int n_sink, const float *lse, int64_t pos0, float rope_base,
+                              float scale, void *ws, size_t ws_bytes, void *stream) {
     if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || W < 0 || pos0 < 0 || n_sink < 0)
         return RAT_ERR_INVALID;
     if (!supported_d(d) || H > kMaxHeads) return RAT_ERR_UNSUPPORTED;
@@ -409,7 +424,8 @@ int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_re
     uint8_t *w = static_cast<uint8_t *>(ws) + sizeof(WsHeader);
     p.qh = w;
     w += align256(rows * d * (dtype == RAT_F32 ? 4 : 2));
-    p.lse = reinterpret_cast<float *>(w);
+    p.lse = lse ? const_cast<float *>(lse) : reinterpret_cast<float *>(w);
+    p.lse_given = lse ? 1 : 0;
     w += align256(rows * 4);
     p.delta = reinterpret_cast<float *>(w);
     p.B = B; p.H = H; p.T = T; p.d = d; p.W = W; p.n_sink = n_sink;

@@ -66,3 +66,37 @@ def test_attention_backward_full_size_sampled_heads():
     x = synthetic.prefill_inputs(w)
     run(w.B, w.H, w.T, w.d, torch.bfloat16, D=w.D, W=w.W, rope_base=w.rope_base, x=x,
         heads=[(0, 0), (w.B - 1, w.H - 1)], seed=5)
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_forward_lse_and_backward_with_it(dtype, d):
+    # the forward's log-sum-exp (tensor-core kernel for bf16 d 128, CUDA-core otherwise) against
+    # the oracle's, and the backward fed with it equal to the backward that recomputes it
+    B, H, T = 1, 3, 333
+    w = synthetic.Workload("lse", B=B, H=H, d=d, T=T, dtype="f32" if dtype == torch.float32 else "bf16",
+                           seed=21)
+    x = synthetic.prefill_inputs(w)
+    dev = torch.device("cuda")
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    kw = dict(D_per_head=[1, 16, 64], W=0, rope_base=10000.0)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    rat.rat_dilated_attn_prefill(q, k, v, o, lse=lse, **kw)
+    qr = oracle.rope(f64(x["q"]), 0, 10000.0)
+    _, ref = oracle.dilated_attention(qr, f64(x["k"]), f64(x["v"]), W=0, D_per_head=[1, 16, 64],
+                                      return_lse=True)
+    tol_abs = 2e-2 if dtype == torch.bfloat16 else 1e-4
+    assert float(np.max(np.abs(f64(lse) - ref))) <= tol_abs * max(1.0, float(np.max(np.abs(ref))))
+    g = torch.Generator().manual_seed(22)
+    dO = torch.randn(q.shape, generator=g).to(dtype).to(dev)
+    ws = rat.Workspace(rat.rat_dilated_attn_backward_workspace_bytes(B, H, T, d,
+                                                                     0 if dtype == torch.float32 else 1))
+    outs = []
+    for given in (None, lse):
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        rat.rat_dilated_attn_backward(q, k, v, o, dO, dq, dk, dv, ws, lse=given, **kw)
+        outs.append((dq, dk, dv))
+    ref_b = oracle.dilated_attention_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(dO), **kw)
+    for got in outs:
+        for gg, r in zip(got, ref_b):
+            assert rel_err(gg, r) <= tol_for(dtype)
