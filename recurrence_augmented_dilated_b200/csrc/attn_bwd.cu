@@ -39,6 +39,8 @@ RAT_DEVICE void rope_lane(const AttnBwdParams &p, long long pos, int lane, float
     }
 }
 
+constexpr int kRows = 4;        // rows (keys or queries) whose loads are issued together
+
 }  // namespace
 
 template <typename E, int DH>
@@ -95,13 +97,13 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const __grid_constant_
 
     // pass 1: the softmax denominator (log2 units), unless the forward's is given
     float m = -INFINITY, l = 0.f;
-    for (int base = 0; base < (p.lse_given ? 0 : n); base += 4) {
-        float kx[4][CPL];
+    for (int base = 0; base < (p.lse_given ? 0 : n); base += kRows) {
+        float kx[kRows][CPL];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
+        for (int u = 0; u < kRows; ++u)
             if (base + u < n) RowIO<E, CPL>::load(kb + (size_t)key(base + u) * DH * EB, kx[u]);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRows; ++u) {
             if (base + u < n) {
                 float dot = 0.f;
 #pragma unroll
@@ -118,10 +120,10 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const __grid_constant_
     float dq[CPL];
 #pragma unroll
     for (int j = 0; j < CPL; ++j) dq[j] = 0.f;
-    for (int base = 0; base < n; base += 4) {
-        float kx[4][CPL], vx[4][CPL];
+    for (int base = 0; base < n; base += kRows) {
+        float kx[kRows][CPL], vx[kRows][CPL];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRows; ++u) {
             if (base + u < n) {
                 const size_t jr = (size_t)key(base + u) * DH * EB;
                 RowIO<E, CPL>::load(kb + jr, kx[u]);
@@ -129,7 +131,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dq_kernel(const __grid_constant_
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRows; ++u) {
             if (base + u < n) {
                 float sd = 0.f, pd = 0.f;
 #pragma unroll
@@ -178,10 +180,10 @@ __global__ void __launch_bounds__(256) attn_bwd_dkv_kernel(const __grid_constant
     float dk[CPL], dv[CPL];
 #pragma unroll
     for (int c = 0; c < CPL; ++c) { dk[c] = 0.f; dv[c] = 0.f; }
-    for (int base = 0; base < n; base += 4) {
-        float qx[4][CPL], gx[4][CPL], lse[4], dl[4];
+    for (int base = 0; base < n; base += kRows) {
+        float qx[kRows][CPL], gx[kRows][CPL], lse[kRows], dl[kRows];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRows; ++u) {
             if (base + u < n) {
                 const int t = j + base + u;             // both parts are contiguous from j
                 RowIO<E, CPL>::load(qb + (size_t)t * DH * EB, qx[u]);
@@ -191,7 +193,7 @@ __global__ void __launch_bounds__(256) attn_bwd_dkv_kernel(const __grid_constant
             }
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < kRows; ++u) {
             if (base + u < n) {
                 float sd = 0.f, pd = 0.f;
 #pragma unroll

@@ -51,8 +51,8 @@ constexpr int NS = 2;                 // K/V pipeline stages
 constexpr int kThreads = 192;         // warp 0: TMA, warp 1: MMA, warps 2-5: softmax / epilogue
 constexpr uint32_t QSUB = BM * 128;   // one [128 rows][64 bf16] 128B-swizzled sub-tile of Q / O
 constexpr int kMaxDil = 4;
-constexpr float kRescaleLog2 = 8.0f;
-constexpr uint32_t kRelBytes = 64 * 32 * 8;   // the RoPE table g_rope_rel  // move the running max only when it grows by > 2^8
+constexpr float kRescaleLog2 = 8.0f;             // move the running max only when it grows by > 2^8
+constexpr uint32_t kRelBytes = 64 * 32 * 8;       // the RoPE table g_rope_rel
 
 // Shared-memory / TMEM plan for key blocks of BN keys.
 template <int BN>
@@ -635,14 +635,15 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
 
 // ------------------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
+    // looked up once (a function-local static is initialised once, also under concurrent calls)
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void *ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
                 cudaSuccess && q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -743,7 +744,7 @@ int fill_params(Params &p, const AttnSm100Args &a) {
 template <int BN, bool SELF>
 int launch_tiles(const Params &p, int items, void *stream) {
     using C = Cfg<BN>;
-    static uint64_t attr_done = 0;
+    static std::atomic<uint64_t> attr_done{0};
     const int st = set_smem_attr(reinterpret_cast<const void *>(attn_sm100_kernel<BN, SELF>), C::SMEM_BYTES, &attr_done);
     if (st != RAT_OK) return st;
     attn_sm100_kernel<BN, SELF><<<(unsigned)items, kThreads, C::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(p);

@@ -1,6 +1,7 @@
 // internal.h -- declarations shared between the C ABI layer and the kernels (not installed).
 #pragma once
 
+#include <atomic>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -121,14 +122,15 @@ struct AttnSm100Args {
 int launch_attn_sm100(const AttnSm100Args &a, void *stream);
 
 // Opt kernel `fn` into `bytes` of dynamic shared memory on the current device, once per device
-// (bit `dev` of *done_mask records it).  Returns a rat_status.
-inline int set_smem_attr(const void *fn, uint32_t bytes, uint64_t *done_mask) {
+// (bit `dev` of *done_mask records it; the mask is atomic, so concurrent host threads may call
+// this -- at worst two of them both set the attribute).  Returns a rat_status.
+inline int set_smem_attr(const void *fn, uint32_t bytes, std::atomic<uint64_t> *done_mask) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RAT_ERR_CUDA;
-    if (*done_mask >> dev & 1) return RAT_OK;
+    if (done_mask->load(std::memory_order_acquire) >> dev & 1) return RAT_OK;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess)
         return RAT_ERR_CUDA;
-    *done_mask |= 1ull << dev;
+    done_mask->fetch_or(1ull << dev, std::memory_order_release);
     return RAT_OK;
 }
 

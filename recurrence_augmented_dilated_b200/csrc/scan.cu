@@ -445,7 +445,7 @@ template <typename E, int DH>
 static int launch_one(const RecurParams &p, void *stream) {
     using C = ScanCfg<E, DH>;
     auto kern = p.reset > 0 ? recur_kernel<E, DH, true> : recur_kernel<E, DH, false>;
-    static uint64_t attr_done[2] = {0, 0};
+    static std::atomic<uint64_t> attr_done[2] = {{0}, {0}};
     const int st = set_smem_attr(reinterpret_cast<const void *>(kern), C::SMEM, &attr_done[p.reset > 0]);
     if (st != RAT_OK) return st;
     const int sms = current_sm_count();

@@ -358,7 +358,7 @@ template <typename E, int DH>
 static int launch_one(const WindowParams &p, void *stream) {
     using C = WinCfg<E, DH>;
     auto kern = window_kernel<E, DH>;
-    static uint64_t attr_done = 0;
+    static std::atomic<uint64_t> attr_done{0};
     const int st = set_smem_attr(reinterpret_cast<const void *>(kern), C::SMEM, &attr_done);
     if (st != RAT_OK) return st;
     const int sms = current_sm_count();
