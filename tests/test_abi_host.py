@@ -106,6 +106,34 @@ def test_local_and_window_validation(L):
     assert L.rat_recur_prefill_window(*args(64, T=0)) == 0
 
 
+def test_empty_inputs_are_no_ops(L):
+    # T = 0: every entry point returns RAT_OK before touching a pointer or the GPU
+    P = ctypes.c_void_p
+    Dh = (ctypes.c_int32 * 2)(4, 16)
+    assert L.rat_dilated_attn_prefill(None, None, None, None, 1, 2, 0, 128, 1, 4, 0, None, 0, 0.0,
+                                      0.0, None) == 0
+    assert L.rat_dilated_attn_prefill_sinks(None, None, None, None, 1, 2, 0, 128, 1, 4, 0, Dh, 4, 0,
+                                            0.0, 0.0, None) == 0
+    assert L.rat_dilated_attn_prefill_topk(None, None, None, None, 1, 2, 0, 128, 1, 4, 0, None, 0, 8,
+                                           0, 0.0, 0.0, None) == 0
+    assert L.rat_dilated_attn_backward(*([None] * 8), 1, 2, 0, 128, 1, 4, 0, None, 0, None, 0, 0.0,
+                                       0.0, None, 0, None) == 0
+    assert L.rat_recur_backward(*([None] * 16), 1, 2, 0, 128, 1, 0, 0.0, None, 0, None) == 0
+    c = cache()
+    c.k_dil = c.v_dil = c.k_win = c.v_win = c.h_k = c.h_v = 256
+    assert L.rat_kv_compress(None, None, None, None, 0, ctypes.byref(c), None) == 0
+    assert c.pos == 0
+
+
+def test_option_limits(L):
+    P = ctypes.c_void_p
+    args = lambda top_k, n_sink: (P(256), P(256), P(256), P(256), 1, 1, 8, 128, 1, 4, 0, None,
+                                  n_sink, top_k, 0, 0.0, 0.0, None)
+    assert L.rat_dilated_attn_prefill_topk(*args(17, 0)) == -2      # at most 16 chunks
+    assert L.rat_dilated_attn_prefill_topk(*args(-1, 0)) == -1
+    assert L.rat_dilated_attn_prefill_topk(*args(2, -1)) == -1
+
+
 def test_recur_workspace_grows_with_chunks(L):
     a = rat.rat_recur_workspace_bytes(1, 1, 128, 128, 1)
     b = rat.rat_recur_workspace_bytes(1, 1, 129, 128, 1)
