@@ -13,7 +13,8 @@
 //   dq   : per query, the key set walked twice -- once for the softmax denominator (kept for
 //          the next launch), once for dq;
 //   dkv  : per key, the queries whose key set holds it walked once: the window t in
-//          [j, j + We - 1], and, for a chunk end (j mod D = D - 1), every t >= j + We.
+//          [j, j + We - 1], and, for a chunk end (j mod D = D - 1), every t >= j + We; the
+//          chunk ends are handed out first, so the long walks share CTAs.
 // Each (query, key) pair is recomputed in both gradient launches; p comes from the stored
 // denominator, so the two launches agree.  This is the plain CUDA-core path of the backward:
 // dot products are warp reductions, four rows' loads in flight per warp.
@@ -160,10 +161,20 @@ __global__ void __launch_bounds__(256) attn_bwd_dkv_kernel(const __grid_constant
     constexpr int CPL = DH / 32, EB = sizeof(E);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y, h = bh % p.H;
-    // key j; the oldest keys, which have the most queries, are in the first CTAs
-    const int j = blockIdx.x * 8 + warp;
-    if (j >= p.T) return;
+    // warps take the chunk ends first (every query older than their window holds them; the
+    // oldest, with the most queries, in the first CTAs), then the other keys (their window
+    // only), so that a CTA's warps have like amounts of work
+    const int kk = blockIdx.x * 8 + warp;
+    if (kk >= p.T) return;
     const int D = p.Dh[h];
+    const int n_ce = p.T / D;                              // chunk ends in the sequence
+    int j;
+    if (kk < n_ce) {
+        j = kk * D + D - 1;
+    } else {
+        const int m = kk - n_ce;                           // the m-th key that is not a chunk end
+        j = m + m / (D - 1);                               // (D > 1 here: with D = 1 all are)
+    }
     const int We = p.W > 1 ? p.W : 1;
     const size_t row = (size_t)bh * p.T;
     const size_t off = (row + j) * DH * EB + lane * CPL * EB;
