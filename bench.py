@@ -586,12 +586,14 @@ def run_decode_paged(w: synthetic.Workload, steps_timed: int, warmup: int, rank:
                                              rope_base=w.rope_base)
     torch.cuda.synchronize()
     stream = torch.cuda.current_stream()
+    prof = ProfiledRegion().__enter__()
     for _ in range(warmup):
         reset()
         gr.replay()
     torch.cuda.synchronize()
     st = rat.rat_sync_status(ws)
     if st != 0:
+        prof.__exit__()
         raise RuntimeError("paged decode device error " + rat.rat_status_string(st))
     if bufs["pos"].cpu().tolist() != [T + nsteps for T in lengths]:
         raise RuntimeError("paged decode positions did not advance")
@@ -606,6 +608,7 @@ def run_decode_paged(w: synthetic.Workload, steps_timed: int, warmup: int, rank:
             e1.record(stream)
             torch.cuda.synchronize()
             times.append(e0.elapsed_time(e1))
+    prof.__exit__()
     ms_total = max_over_ranks(sum(times) / len(times), world)
     ms_step = ms_total / nsteps
     rows = 0
@@ -650,14 +653,15 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     def step():
         rat.rat_recur_backward(k, v, a, kr, vr, dyk, dyv, dk, dv, da, ws, rope_base=w.rope_base)
 
-    for _ in range(warmup):
-        step()
-    torch.cuda.synchronize()
+    with ProfiledRegion():
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize()
     if rat.rat_sync_status(ws) != 0:
         raise RuntimeError("backward device error")
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(torch.cuda.current_device()) as clk:
+    with ClockSampler(torch.cuda.current_device()) as clk, ProfiledRegion():
         e0.record(stream)
         for _ in range(steps):
             step()
@@ -688,15 +692,17 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
         rat.rat_dilated_attn_backward(q, kr, vr, o, dO, dq, dkr, dvr, ws_a, D=w.D, W=w.W,
                                       D_per_head=Dph, rope_base=w.rope_base, lse=lse)
 
-    for _ in range(warmup):
-        astep()
-    torch.cuda.synchronize()
+    with ProfiledRegion():
+        for _ in range(warmup):
+            astep()
+        torch.cuda.synchronize()
     barrier(world)
-    e0.record(stream)
-    for _ in range(steps):
-        astep()
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with ProfiledRegion():
+        e0.record(stream)
+        for _ in range(steps):
+            astep()
+        e1.record(stream)
+        torch.cuda.synchronize()
     ams = max_over_ranks(e0.elapsed_time(e1) / steps, world)
     abytes = 8 * B * H * T * d * eb        # read q, k~, v~, o, dO; write dq, dk~, dv~
     pairs = sum(rat.rat_attended_keys(t, D_, w.W) for D_ in w.heads_D() for t in range(T)) * B
