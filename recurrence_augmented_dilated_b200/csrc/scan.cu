@@ -34,7 +34,12 @@
 // records RAT_ERR_TIMEOUT instead of hanging.  Flags carry a launch epoch, so the workspace is
 // never cleared between launches: the last CTA of a launch resets the tickets and bumps the
 // epoch.
-#include "common.cuh"
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <cstring>
+
+#include "tc.cuh"
 
 namespace rat {
 
@@ -430,6 +435,317 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
     }
 }
 
+// ---------------------------------------------------------------------------------------------
+// Channel-sliced form (bf16, d = 128, full-sequence recurrence).  The channels are independent,
+// so every (b, h) splits into two slices of 64 channels that scan separately: slice s holds
+// channels [32s, 32s + 32) and their rotate-half partners [64 + 32s, 96 + 32s).  At the same
+// bytes per chunk (48 KiB of a, k, v) a chunk then spans 128 rows, so each slice's look-back
+// chain advances half as often as the full-row chain of 64-row chunks, and the chain -- one L2
+// round trip per link under the streaming load -- stops setting the pace.
+//
+// A chunk of a slice arrives as one TMA box per tensor: the tensor viewed as
+// (32-channel column x, half y, row z) with y's stride d/2 channels, box (32, 2, 128), so a row
+// lands as 128 contiguous bytes (its 32 first-half channels, then their 32 partners).  Lane l of
+// a warp holds channels 2l, 2l+1 of that row (lanes 16-31 the partners of lanes 0-15), so each
+// warp reads a whole row per load without bank conflicts, and the RoPE partner of a lane is
+// lane l ^ 16 (one shuffle per row).  Each warp is one segment of 16 consecutive rows.
+struct SliceCfg {
+    static constexpr int DH = 128, SC = 64;       // channels per row, per slice
+    static constexpr int THREADS = 512, NPIPE = 2, PT = THREADS / NPIPE, PW = PT / 32;
+    static constexpr int TC = 128;                // rows per chunk
+    static constexpr int R = TC / PW;             // rows per warp (segment)
+    static constexpr int ROWB = SC * 2;           // bytes of one slice row in shared memory
+    static constexpr int TILEB = TC * ROWB;       // 16 KiB per tensor per chunk
+    static constexpr int STAGEB = 3 * TILEB;
+    static constexpr int SWB = PW * 3 * SC * 4;   // per-warp aggregates, then carries
+    static constexpr int PIPEB = 2 * STAGEB + SWB;
+    static constexpr int SMEM = NPIPE * PIPEB + 128;   // + alignment slack for the TMA boxes
+    static constexpr int LBW = 2;                 // predecessors read per look-back round
+    static_assert(R * PW == TC && PT >= SC, "one warp per segment, one thread per slice channel");
+};
+
+struct SliceParams {
+    RecurParams r;              // nchunks counts 128-row chunks here
+    CUtensorMap tm_a, tm_k, tm_v;
+};
+
+__global__ void __launch_bounds__(SliceCfg::THREADS, 1) recur_slice_kernel(const __grid_constant__ SliceParams sp) {
+    using C = SliceCfg;
+    const RecurParams &p = sp.r;
+    constexpr int R = C::R, SC = C::SC;
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ uint64_t bar[C::NPIPE][2];
+    __shared__ int s_ticket[C::NPIPE][2];
+    __shared__ uint32_t s_epoch;
+    __shared__ float s_theta_f[64], s_step_c[64], s_step_s[64];
+    __shared__ double s_theta[64];
+
+    const int tid = threadIdx.x;
+    const int pipe = tid / C::PT, pt = tid % C::PT;
+    const int pwarp = pt >> 5, lane = tid & 31;
+    const int half = lane >> 4, cl = lane & 15;                // partner half, pair in the half
+    const int barid = 1 + pipe;
+    uint8_t *smem_al = smem + ((128u - (smem_u32(smem) & 127u)) & 127u);
+    uint8_t *pbase = smem_al + pipe * C::PIPEB;
+    float *sw = reinterpret_cast<float *>(pbase + 2 * C::STAGEB);          // [PW][3][SC]
+    WsHeader *hdr = p.hdr;
+    const int items = 2 * p.BH;                                // (b, h, slice)
+    const int total = items * p.nchunks;
+
+    auto load_chunk = [&](int ticket, int st) {
+        const int c = ticket / items, item = ticket % items;
+        const int x = 32 * (item & 1), z = (item >> 1) * p.T + c * C::TC;
+        uint8_t *s = pbase + st * C::STAGEB;
+        mbar_arrive_expect_tx(&bar[pipe][st], 3 * C::TILEB);
+        tc::tma_load_3d(s, &sp.tm_a, x, 0, z, &bar[pipe][st]);
+        tc::tma_load_3d(s + C::TILEB, &sp.tm_k, x, 0, z, &bar[pipe][st]);
+        tc::tma_load_3d(s + 2 * C::TILEB, &sp.tm_v, x, 0, z, &bar[pipe][st]);
+    };
+    auto pipe_sync = [&]() { asm volatile("bar.sync %0, %1;" :: "r"(barid), "r"(C::PT) : "memory"); };
+    auto read_window = [&](int item, int j, int ch, uint64_t (&w)[C::LBW][5]) {
+#pragma unroll
+        for (int u = 0; u < C::LBW; ++u) {
+            const size_t jid = (size_t)item * p.nchunks + max(j - u, 0);
+            const uint64_t *pj = p.pre + jid * 2 * SC + ch;
+            const uint64_t *aj = p.agg + jid * 3 * SC + ch;
+            w[u][0] = ld_relaxed_gpu_u64(pj);
+            w[u][1] = ld_relaxed_gpu_u64(pj + SC);
+            w[u][2] = ld_relaxed_gpu_u64(aj);
+            w[u][3] = ld_relaxed_gpu_u64(aj + SC);
+            w[u][4] = ld_relaxed_gpu_u64(aj + 2 * SC);
+        }
+    };
+
+    if (tid < 64) {
+        s_theta_f[tid] = p.theta_f[tid];
+        s_theta[tid] = p.theta[tid];
+        s_step_c[tid] = p.step_cos[tid];
+        s_step_s[tid] = p.step_sin[tid];
+    }
+    if (tid == 0) {
+        s_epoch = *reinterpret_cast<volatile uint32_t *>(&hdr->epoch);
+        for (int q = 0; q < C::NPIPE; ++q) {
+            mbar_init(&bar[q][0], 1);
+            mbar_init(&bar[q][1], 1);
+        }
+        fence_mbar_init();
+        tc::prefetch_tmap(&sp.tm_a);
+        tc::prefetch_tmap(&sp.tm_k);
+        tc::prefetch_tmap(&sp.tm_v);
+    }
+    __syncthreads();
+    const uint32_t epoch_raw = s_epoch;
+    const uint32_t tag = (epoch_raw & 0x7fffffffu) | 0x80000000u;
+    if (pt == 0) {
+        const int t0k = (int)atomicAdd(&hdr->ticket, 1u);
+        s_ticket[pipe][0] = t0k;
+        if (t0k < total) load_chunk(t0k, 0);
+    }
+    pipe_sync();
+
+    for (int it = 0;; ++it) {
+        const int st = it & 1;
+        const int ticket = s_ticket[pipe][st];
+        if (ticket >= total) break;
+        if (pt == 0) {
+            const int nt = (int)atomicAdd(&hdr->ticket, 1u);
+            s_ticket[pipe][st ^ 1] = nt;
+            if (nt < total) load_chunk(nt, st ^ 1);
+        }
+        const int c = ticket / items, item = ticket % items;       // chunk-major order
+        const int bh = item >> 1, slice = item & 1;
+        const int t0 = c * C::TC;
+        const int rows = min(C::TC, p.T - t0);
+        const size_t chunk_id = (size_t)item * p.nchunks + c;
+        const size_t row0 = (size_t)bh * p.T + t0;
+        const bool publish = c != p.fault_chunk;
+        const uint8_t *sa = pbase + st * C::STAGEB, *sk = sa + C::TILEB, *sv = sa + 2 * C::TILEB;
+        uint64_t w[C::LBW][5];
+        if (pt < SC && c > 0) read_window(item, c - 1, pt, w);
+        mbar_wait_bounded(&bar[pipe][st], (it >> 1) & 1, hdr, 0x100u);
+
+        // ---- pass 1: this lane's two channels over the warp's R rows: gates (kept) and aggregate
+        const f2_t kOne2 = f2(1.f, 1.f), kZero2 = f2(0.f, 0.f);
+        f2_t G[R];
+        f2_t A = kOne2, Bk = kZero2, Bv = kZero2;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int r = pwarp * R + i;
+            const int off = (r < rows ? r : rows - 1) * C::ROWB + 4 * lane;
+            const f2_t xa = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sa + off));
+            const f2_t xk = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sk + off));
+            const f2_t xv = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sv + off));
+            G[i] = r < rows ? forget_gate2(xa) : kOne2;
+            const f2_t og = gate_complement2(G[i]);
+            A = f2_mul(A, G[i]);
+            Bk = f2_fma(G[i], Bk, f2_mul(og, xk));
+            Bv = f2_fma(G[i], Bv, f2_mul(og, xv));
+        }
+        {
+            float2 *s2 = reinterpret_cast<float2 *>(sw);
+            s2[((pwarp * 3 + 0) * SC) / 2 + lane] = make_float2(f2lo(A), f2hi(A));
+            s2[((pwarp * 3 + 1) * SC) / 2 + lane] = make_float2(f2lo(Bk), f2hi(Bk));
+            s2[((pwarp * 3 + 2) * SC) / 2 + lane] = make_float2(f2lo(Bv), f2hi(Bv));
+        }
+        pipe_sync();
+
+        // ---- one thread per slice channel: chunk aggregate (published), look-back for the
+        // state entering the chunk, inclusive state (published), carries entering each warp
+        if (pt < SC) {
+            const int ch = pt;                                     // slice channel 2l + u
+            const int gch = (ch < 32 ? 0 : 64) + 32 * slice + (ch & 31);   // channel of the row
+            float cA = 1.f, cK = 0.f, cV = 0.f;
+#pragma unroll
+            for (int wp = 0; wp < C::PW; ++wp) {
+                const float a = sw[(wp * 3 + 0) * SC + ch];
+                cK = fmaf(a, cK, sw[(wp * 3 + 1) * SC + ch]);
+                cV = fmaf(a, cV, sw[(wp * 3 + 2) * SC + ch]);
+                cA *= a;
+            }
+            if (c > 0 && publish) {
+                uint64_t *agg = p.agg + chunk_id * 3 * SC;
+                st_relaxed_gpu_u64(agg + ch, tagged(tag, cA));
+                st_relaxed_gpu_u64(agg + SC + ch, tagged(tag, cK));
+                st_relaxed_gpu_u64(agg + 2 * SC + ch, tagged(tag, cV));
+            }
+            float Hk = 0.f, Hv = 0.f;
+            if (c == 0) {
+                if (p.h0k) Hk = p.h0k[(size_t)bh * C::DH + gch];
+                if (p.h0v) Hv = p.h0v[(size_t)bh * C::DH + gch];
+            } else {
+                // the same walk as the full-row scan: LBW predecessors per round, an inclusive
+                // state ends it, an aggregate is composed in, a missing record ends the round
+                float xA = 1.f, xK = 0.f, xV = 0.f;
+                const uint64_t t_start = globaltimer_ns();
+                uint32_t spins = 0;
+                int j = c - 1;
+                for (bool first = true;; first = false) {
+                    if (!first) read_window(item, j, ch, w);
+                    bool done = false, stop = false;
+                    int passed = 0;
+#pragma unroll
+                    for (int u = 0; u < C::LBW; ++u) {
+                        if (done || stop || j - u < 0) continue;
+                        auto ok = [&](int e) { return (uint32_t)(w[u][e] >> 32) == tag; };
+                        auto val = [&](int e) { return __uint_as_float((uint32_t)w[u][e]); };
+                        if (ok(0) && ok(1)) {
+                            Hk = fmaf(xA, val(0), xK);
+                            Hv = fmaf(xA, val(1), xV);
+                            done = true;
+                        } else if (ok(2) && ok(3) && ok(4)) {
+                            xK = fmaf(xA, val(3), xK);
+                            xV = fmaf(xA, val(4), xV);
+                            xA *= val(2);
+                            ++passed;
+                        } else {
+                            stop = true;
+                        }
+                    }
+                    if (done) break;
+                    j -= passed;
+                    if (passed == 0) {
+                        if ((++spins & 7u) == 0u && globaltimer_ns() - t_start > p.wait_ns) {
+                            record_error(hdr, RAT_ERR_TIMEOUT, 0x200u);
+                            break;
+                        }
+                        __nanosleep(32);
+                    }
+                }
+            }
+            const float outK = fmaf(cA, Hk, cK), outV = fmaf(cA, Hv, cV);
+            if (publish) {
+                uint64_t *pre = p.pre + chunk_id * 2 * SC;
+                st_relaxed_gpu_u64(pre + ch, tagged(tag, outK));
+                st_relaxed_gpu_u64(pre + SC + ch, tagged(tag, outV));
+            }
+            if (c == p.nchunks - 1) {
+                if (p.hTk) p.hTk[(size_t)bh * C::DH + gch] = outK;
+                if (p.hTv) p.hTv[(size_t)bh * C::DH + gch] = outV;
+            }
+            float hK = Hk, hV = Hv;
+#pragma unroll
+            for (int wp = 0; wp < C::PW; ++wp) {
+                const float a = sw[(wp * 3 + 0) * SC + ch];
+                const float bk = sw[(wp * 3 + 1) * SC + ch];
+                const float bv = sw[(wp * 3 + 2) * SC + ch];
+                sw[(wp * 3 + 0) * SC + ch] = hK;
+                sw[(wp * 3 + 1) * SC + ch] = hV;
+                hK = fmaf(a, hK, bk);
+                hV = fmaf(a, hV, bv);
+            }
+        }
+        pipe_sync();
+
+        // ---- pass 2: rerun the warp's rows from its carry; write k~ (rotated) and v~
+        f2_t hk, hv;
+        {
+            const float2 *s2 = reinterpret_cast<const float2 *>(sw);
+            const float2 ck = s2[((pwarp * 3 + 0) * SC) / 2 + lane];
+            const float2 cv = s2[((pwarp * 3 + 1) * SC) / 2 + lane];
+            hk = f2(ck.x, ck.y);
+            hv = f2(cv.x, cv.y);
+        }
+        // RoPE of frequencies f = 32 slice + 2 cl (+1) at the warp's first row, advanced one
+        // position per row; a first-half lane takes x cos - x' sin, its partner x cos + x' sin
+        // (x' the other lane's value), so the sine carries the sign of the half.
+        f2_t rc = kOne2, rs = kZero2, sc = kOne2, ss = kZero2, nss = kZero2;
+        if (p.rope) {
+            const long long pos = p.pos0 + t0 + pwarp * R;
+            float c2[2], s2v[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const int f = 32 * slice + 2 * cl + u;
+                if (p.rope_f32) rope_cs_f32((int)pos, s_theta_f[f], c2[u], s2v[u]);
+                else rope_cs(pos, s_theta[f], c2[u], s2v[u]);
+            }
+            const float sg = half ? 1.f : -1.f;   // sin(-x) = -sin(x): exact
+            rc = f2(c2[0], c2[1]);
+            rs = f2(sg * s2v[0], sg * s2v[1]);
+            const int f0 = 32 * slice + 2 * cl;
+            sc = f2(s_step_c[f0], s_step_c[f0 + 1]);
+            ss = f2(s_step_s[f0], s_step_s[f0 + 1]);
+            nss = f2(-s_step_s[f0], -s_step_s[f0 + 1]);
+        }
+        const f2_t adv_c = half ? nss : ss, adv_s = half ? ss : nss;
+        uint8_t *yk = static_cast<uint8_t *>(p.yk) + 128 * half + 64 * slice + 4 * cl;
+        uint8_t *yv = static_cast<uint8_t *>(p.yv) + 128 * half + 64 * slice + 4 * cl;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            const int r = pwarp * R + i;
+            const int off = (r < rows ? r : rows - 1) * C::ROWB + 4 * lane;
+            const f2_t xk = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sk + off));
+            const f2_t xv = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sv + off));
+            const f2_t og = gate_complement2(G[i]);
+            hk = f2_fma(G[i], hk, f2_mul(og, xk));
+            hv = f2_fma(G[i], hv, f2_mul(og, xv));
+            f2_t ok = hk;
+            if (p.rope) {
+                const f2_t other = __shfl_xor_sync(0xffffffffu, hk, 16);
+                ok = f2_fma(other, rs, f2_mul(hk, rc));
+                // advance one position: (c + i s)(cos t + i sin t); rs keeps the half's sign
+                const f2_t nc = f2_fma(rc, sc, f2_mul(rs, adv_c));
+                rs = f2_fma(rs, sc, f2_mul(rc, adv_s));
+                rc = nc;
+            }
+            if (r < rows) {
+                const size_t go = (row0 + r) * (C::DH * 2);
+                *reinterpret_cast<uint32_t *>(yk + go) = f2_to_bf16x2(ok);
+                *reinterpret_cast<uint32_t *>(yv + go) = f2_to_bf16x2(hv);
+            }
+        }
+        pipe_sync();
+    }
+    if (pt == 0) {
+        __threadfence();
+        if (atomicAdd(&hdr->done, 1u) == gridDim.x * C::NPIPE - 1) {
+            hdr->ticket = 0;
+            hdr->done = 0;
+            __threadfence();
+            atomicExch(&hdr->epoch, epoch_raw + 1u);
+        }
+    }
+}
+
 int recur_chunk_rows(int d, int dtype) {
     const int eb = dtype == RAT_F32 ? 4 : 2;
     return 16384 / (d * eb);               // one 16 KiB tile per tensor
@@ -457,7 +773,61 @@ static int launch_one(const RecurParams &p, void *stream) {
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 
+static PFN_cuTensorMapEncodeTiled_v12000 scan_encode_fn() {
+    // looked up once (a function-local static is initialised once, also under concurrent calls)
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess && q == cudaDriverEntryPointSuccess)
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+        return nullptr;
+    }();
+    return fn;
+}
+
+// (32-channel column, half, row) view of a (rows, 128) bf16 tensor: x < 64 channels of a half,
+// y < 2 halves 64 channels apart, z < rows; box (32, 2, 128 rows), zero fill past the last row.
+static bool slice_map(CUtensorMap *m, const void *base, uint64_t rows) {
+    auto fn = scan_encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {64, 2, rows};
+    cuuint64_t strides[2] = {64 * 2, 128 * 2};
+    cuuint32_t box[3] = {32, 2, (cuuint32_t)SliceCfg::TC};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The channel-sliced scan; returns RAT_ERR_UNSUPPORTED when the tensor maps cannot be built
+// (the caller then runs the full-row scan).
+static int launch_slice(const RecurParams &p, void *stream) {
+    using C = SliceCfg;
+    SliceParams sp;
+    std::memset(&sp, 0, sizeof(sp));
+    sp.r = p;
+    sp.r.nchunks = (p.T + C::TC - 1) / C::TC;
+    const uint64_t rows = (uint64_t)p.BH * (uint64_t)p.T;
+    if (!slice_map(&sp.tm_a, p.a, rows) || !slice_map(&sp.tm_k, p.k, rows) || !slice_map(&sp.tm_v, p.v, rows))
+        return RAT_ERR_UNSUPPORTED;
+    static std::atomic<uint64_t> attr_done{0};
+    const int st = set_smem_attr(reinterpret_cast<const void *>(recur_slice_kernel), C::SMEM, &attr_done);
+    if (st != RAT_OK) return st;
+    const int sms = current_sm_count();
+    if (sms <= 0) return RAT_ERR_CUDA;
+    const long long total = 2ll * p.BH * sp.r.nchunks;
+    const unsigned grid = (unsigned)(total < sms ? total : sms);
+    recur_slice_kernel<<<grid, C::THREADS, C::SMEM, static_cast<cudaStream_t>(stream)>>>(sp);
+    return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
+}
+
 int launch_recur(const RecurParams &p, int dtype, void *stream) {
+    // bf16, d 128, full sequence, row coordinates within int32: the channel-sliced scan
+    if (dtype == RAT_BF16 && p.d == 128 && p.reset == 0 && (long long)p.BH * p.T < (1ll << 31) - SliceCfg::TC) {
+        const int st = launch_slice(p, stream);
+        if (st != RAT_ERR_UNSUPPORTED) return st;
+    }
     if (dtype == RAT_F32) {
         if (p.d == 64) return launch_one<float, 64>(p, stream);
         if (p.d == 128) return launch_one<float, 128>(p, stream);
