@@ -436,32 +436,35 @@ __global__ void __launch_bounds__(ScanCfg<E, DH>::THREADS, 1) recur_kernel(const
 }
 
 // ---------------------------------------------------------------------------------------------
-// Channel-sliced form (bf16, d = 128, full-sequence recurrence).  The channels are independent,
-// so every (b, h) splits into two slices of 64 channels that scan separately: slice s holds
-// channels [32s, 32s + 32) and their rotate-half partners [64 + 32s, 96 + 32s).  At the same
-// bytes per chunk (48 KiB of a, k, v) a chunk then spans 128 rows, so each slice's look-back
-// chain advances half as often as the full-row chain of 64-row chunks, and the chain -- one L2
-// round trip per link under the streaming load -- stops setting the pace.
+// Channel-sliced form (bf16, d = 128, full-sequence recurrence, T a multiple of 16).  The
+// channels are independent, so every (b, h) splits into two slices of 64 channels that scan
+// separately: slice s holds channels [32s, 32s + 32) and their rotate-half partners
+// [64 + 32s, 96 + 32s).  At the same bytes per chunk (48 KiB of a, k, v) a chunk then spans 128
+// rows, so each slice's look-back chain advances half as often as the full-row chain of 64-row
+// chunks, and the chain -- one L2 round trip per link under the streaming load -- stops setting
+// the pace.
 //
-// A chunk of a slice arrives as one TMA box per tensor: the tensor viewed as
-// (32-channel column x, half y, row z) with y's stride d/2 channels, box (32, 2, 128), so a row
-// lands as 128 contiguous bytes (its 32 first-half channels, then their 32 partners).  Lane l of
-// a warp holds channels 2l, 2l+1 of that row (lanes 16-31 the partners of lanes 0-15), so each
-// warp reads a whole row per load without bank conflicts, and the RoPE partner of a lane is
-// lane l ^ 16 (one shuffle per row).  Each warp is one segment of 16 consecutive rows.
+// Lanes: lane l of warp w holds channels 2c, 2c+1 (c = l mod 16) of the slice's first half and
+// their two partners, for the rows of segment 2w + l/16 (8 rows each, 16 segments per chunk),
+// so the RoPE rotation needs nothing from other lanes, as in the full-row scan.  Shared memory
+// layout: the chunk arrives as one TMA box per tensor from a 5-D view of the tensor,
+//     (channel x < 64, segment-in-warp u < 2, half y < 2, row-in-segment i < 8, 16-row group g)
+// at byte 2x + 2048u + 128y + 256i + 4096g, box (32, 2, 2, 8, 8); the box lands with u inside
+// y, so for each i the two half-warps of a warp read bytes 64 apart, and every load of a warp
+// covers all 32 banks once.
 struct SliceCfg {
     static constexpr int DH = 128, SC = 64;       // channels per row, per slice
     static constexpr int THREADS = 512, NPIPE = 2, PT = THREADS / NPIPE, PW = PT / 32;
     static constexpr int TC = 128;                // rows per chunk
-    static constexpr int R = TC / PW;             // rows per warp (segment)
-    static constexpr int ROWB = SC * 2;           // bytes of one slice row in shared memory
-    static constexpr int TILEB = TC * ROWB;       // 16 KiB per tensor per chunk
+    static constexpr int R = 8;                   // rows per segment
+    static constexpr int SEGS = TC / R;           // two per warp
+    static constexpr int TILEB = TC * SC * 2;     // 16 KiB per tensor per chunk
     static constexpr int STAGEB = 3 * TILEB;
     static constexpr int SWB = PW * 3 * SC * 4;   // per-warp aggregates, then carries
     static constexpr int PIPEB = 2 * STAGEB + SWB;
     static constexpr int SMEM = NPIPE * PIPEB + 128;   // + alignment slack for the TMA boxes
     static constexpr int LBW = 2;                 // predecessors read per look-back round
-    static_assert(R * PW == TC && PT >= SC, "one warp per segment, one thread per slice channel");
+    static_assert(SEGS == 2 * PW && PT >= SC, "two segments per warp, one thread per slice channel");
 };
 
 struct SliceParams {
@@ -469,10 +472,19 @@ struct SliceParams {
     CUtensorMap tm_a, tm_k, tm_v;
 };
 
+RAT_DEVICE void tma_load_5d(void *smem_dst, const CUtensorMap *map, int c0, int c1, int c2, int c3, int c4,
+                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        :: "r"(smem_u32(smem_dst)), "l"(map), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4), "r"(smem_u32(bar))
+        : "memory");
+}
+
 __global__ void __launch_bounds__(SliceCfg::THREADS, 1) recur_slice_kernel(const __grid_constant__ SliceParams sp) {
     using C = SliceCfg;
     const RecurParams &p = sp.r;
-    constexpr int R = C::R, SC = C::SC;
+    constexpr int R = C::R, SC = C::SC, NP = 2;
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ uint64_t bar[C::NPIPE][2];
     __shared__ int s_ticket[C::NPIPE][2];
@@ -483,7 +495,8 @@ __global__ void __launch_bounds__(SliceCfg::THREADS, 1) recur_slice_kernel(const
     const int tid = threadIdx.x;
     const int pipe = tid / C::PT, pt = tid % C::PT;
     const int pwarp = pt >> 5, lane = tid & 31;
-    const int half = lane >> 4, cl = lane & 15;                // partner half, pair in the half
+    const int segw = lane >> 4, cl = lane & 15;                // segment in the warp, pair in the half
+    const int seg = 2 * pwarp + segw;
     const int barid = 1 + pipe;
     uint8_t *smem_al = smem + ((128u - (smem_u32(smem) & 127u)) & 127u);
     uint8_t *pbase = smem_al + pipe * C::PIPEB;
@@ -491,15 +504,17 @@ __global__ void __launch_bounds__(SliceCfg::THREADS, 1) recur_slice_kernel(const
     WsHeader *hdr = p.hdr;
     const int items = 2 * p.BH;                                // (b, h, slice)
     const int total = items * p.nchunks;
+    // shared-memory byte offset of row r of the chunk, first-half pair of this lane
+    auto soff = [&](int r) { return 2048 * (r >> 4) + 256 * (r & 7) + 64 * ((r >> 3) & 1) + 4 * cl; };
 
     auto load_chunk = [&](int ticket, int st) {
         const int c = ticket / items, item = ticket % items;
-        const int x = 32 * (item & 1), z = (item >> 1) * p.T + c * C::TC;
+        const int g = ((item >> 1) * p.T + c * C::TC) / 16;
         uint8_t *s = pbase + st * C::STAGEB;
         mbar_arrive_expect_tx(&bar[pipe][st], 3 * C::TILEB);
-        tc::tma_load_3d(s, &sp.tm_a, x, 0, z, &bar[pipe][st]);
-        tc::tma_load_3d(s + C::TILEB, &sp.tm_k, x, 0, z, &bar[pipe][st]);
-        tc::tma_load_3d(s + 2 * C::TILEB, &sp.tm_v, x, 0, z, &bar[pipe][st]);
+        tma_load_5d(s, &sp.tm_a, 32 * (item & 1), 0, 0, 0, g, &bar[pipe][st]);
+        tma_load_5d(s + C::TILEB, &sp.tm_k, 32 * (item & 1), 0, 0, 0, g, &bar[pipe][st]);
+        tma_load_5d(s + 2 * C::TILEB, &sp.tm_v, 32 * (item & 1), 0, 0, 0, g, &bar[pipe][st]);
     };
     auto pipe_sync = [&]() { asm volatile("bar.sync %0, %1;" :: "r"(barid), "r"(C::PT) : "memory"); };
     auto read_window = [&](int item, int j, int ch, uint64_t (&w)[C::LBW][5]) {
@@ -564,35 +579,57 @@ __global__ void __launch_bounds__(SliceCfg::THREADS, 1) recur_slice_kernel(const
         if (pt < SC && c > 0) read_window(item, c - 1, pt, w);
         mbar_wait_bounded(&bar[pipe][st], (it >> 1) & 1, hdr, 0x100u);
 
-        // ---- pass 1: this lane's two channels over the warp's R rows: gates (kept) and aggregate
+        // ---- pass 1: gates of this lane's R rows (kept for pass 2) and their aggregate
         const f2_t kOne2 = f2(1.f, 1.f), kZero2 = f2(0.f, 0.f);
-        f2_t G[R];
-        f2_t A = kOne2, Bk = kZero2, Bv = kZero2;
+        f2_t G[R][NP];
+        f2_t A[NP], Bk[NP], Bv[NP];
+#pragma unroll
+        for (int q = 0; q < NP; ++q) { A[q] = kOne2; Bk[q] = kZero2; Bv[q] = kZero2; }
 #pragma unroll
         for (int i = 0; i < R; ++i) {
-            const int r = pwarp * R + i;
-            const int off = (r < rows ? r : rows - 1) * C::ROWB + 4 * lane;
-            const f2_t xa = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sa + off));
-            const f2_t xk = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sk + off));
-            const f2_t xv = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sv + off));
-            G[i] = r < rows ? forget_gate2(xa) : kOne2;
-            const f2_t og = gate_complement2(G[i]);
-            A = f2_mul(A, G[i]);
-            Bk = f2_fma(G[i], Bk, f2_mul(og, xk));
-            Bv = f2_fma(G[i], Bv, f2_mul(og, xv));
+            const int r = seg * R + i;
+            const int off = soff(r < rows ? r : rows - 1);         // rows past the end: identity step
+            f2_t xa[NP], xk[NP], xv[NP];
+            Lane<__nv_bfloat16>::template load<128>(sa + off - 4 * cl, cl, xa);
+            Lane<__nv_bfloat16>::template load<128>(sk + off - 4 * cl, cl, xk);
+            Lane<__nv_bfloat16>::template load<128>(sv + off - 4 * cl, cl, xv);
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                G[i][q] = r < rows ? forget_gate2(xa[q]) : kOne2;
+                const f2_t og = gate_complement2(G[i][q]);
+                A[q] = f2_mul(A[q], G[i][q]);
+                Bk[q] = f2_fma(G[i][q], Bk[q], f2_mul(og, xk[q]));
+                Bv[q] = f2_fma(G[i][q], Bv[q], f2_mul(og, xv[q]));
+            }
         }
-        {
-            float2 *s2 = reinterpret_cast<float2 *>(sw);
-            s2[((pwarp * 3 + 0) * SC) / 2 + lane] = make_float2(f2lo(A), f2hi(A));
-            s2[((pwarp * 3 + 1) * SC) / 2 + lane] = make_float2(f2lo(Bk), f2hi(Bk));
-            s2[((pwarp * 3 + 2) * SC) / 2 + lane] = make_float2(f2lo(Bv), f2hi(Bv));
+        // ---- the warp's second segment composes the first into its aggregate; the first
+        // segment's aggregate is the second's exclusive prefix
+        f2_t eA[NP], eK[NP], eV[NP];
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            eA[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(A[q]), 16), __shfl_up_sync(0xffffffffu, f2hi(A[q]), 16));
+            eK[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(Bk[q]), 16), __shfl_up_sync(0xffffffffu, f2hi(Bk[q]), 16));
+            eV[q] = f2(__shfl_up_sync(0xffffffffu, f2lo(Bv[q]), 16), __shfl_up_sync(0xffffffffu, f2hi(Bv[q]), 16));
+            if (segw == 0) { eA[q] = kOne2; eK[q] = kZero2; eV[q] = kZero2; }
+        }
+        if (segw == 1) {
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const f2_t wA = f2_mul(A[q], eA[q]);
+                const f2_t wK = f2_fma(A[q], eK[q], Bk[q]);
+                const f2_t wV = f2_fma(A[q], eV[q], Bv[q]);
+                float2 *s2 = reinterpret_cast<float2 *>(sw) + cl + 16 * q;   // slice channels 2cl (+32q)
+                s2[((pwarp * 3 + 0) * SC) / 2] = make_float2(f2lo(wA), f2hi(wA));
+                s2[((pwarp * 3 + 1) * SC) / 2] = make_float2(f2lo(wK), f2hi(wK));
+                s2[((pwarp * 3 + 2) * SC) / 2] = make_float2(f2lo(wV), f2hi(wV));
+            }
         }
         pipe_sync();
 
         // ---- one thread per slice channel: chunk aggregate (published), look-back for the
         // state entering the chunk, inclusive state (published), carries entering each warp
         if (pt < SC) {
-            const int ch = pt;                                     // slice channel 2l + u
+            const int ch = pt;                                     // slice channel
             const int gch = (ch < 32 ? 0 : 64) + 32 * slice + (ch & 31);   // channel of the row
             float cA = 1.f, cK = 0.f, cV = 0.f;
 #pragma unroll
@@ -676,21 +713,22 @@ __global__ void __launch_bounds__(SliceCfg::THREADS, 1) recur_slice_kernel(const
         }
         pipe_sync();
 
-        // ---- pass 2: rerun the warp's rows from its carry; write k~ (rotated) and v~
-        f2_t hk, hv;
-        {
-            const float2 *s2 = reinterpret_cast<const float2 *>(sw);
-            const float2 ck = s2[((pwarp * 3 + 0) * SC) / 2 + lane];
-            const float2 cv = s2[((pwarp * 3 + 1) * SC) / 2 + lane];
-            hk = f2(ck.x, ck.y);
-            hv = f2(cv.x, cv.y);
+        // ---- pass 2: rerun the segment from its carry with the kept gates; write k~ (rotated)
+        // and v~
+        f2_t hk[NP], hv[NP];
+#pragma unroll
+        for (int q = 0; q < NP; ++q) {
+            const float2 *s2 = reinterpret_cast<const float2 *>(sw) + cl + 16 * q;
+            const float2 ck = s2[((pwarp * 3 + 0) * SC) / 2];
+            const float2 cv = s2[((pwarp * 3 + 1) * SC) / 2];
+            hk[q] = f2_fma(eA[q], f2(ck.x, ck.y), eK[q]);
+            hv[q] = f2_fma(eA[q], f2(cv.x, cv.y), eV[q]);
         }
-        // RoPE of frequencies f = 32 slice + 2 cl (+1) at the warp's first row, advanced one
-        // position per row; a first-half lane takes x cos - x' sin, its partner x cos + x' sin
-        // (x' the other lane's value), so the sine carries the sign of the half.
+        // RoPE: frequencies 32 slice + 2 cl (+1) at the segment's first row, advanced one
+        // position per row; pair 0 (first half) takes x cos - x' sin, pair 1 x' cos + x sin
         f2_t rc = kOne2, rs = kZero2, sc = kOne2, ss = kZero2, nss = kZero2;
         if (p.rope) {
-            const long long pos = p.pos0 + t0 + pwarp * R;
+            const long long pos = p.pos0 + t0 + seg * R;
             float c2[2], s2v[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
@@ -698,39 +736,42 @@ __global__ void __launch_bounds__(SliceCfg::THREADS, 1) recur_slice_kernel(const
                 if (p.rope_f32) rope_cs_f32((int)pos, s_theta_f[f], c2[u], s2v[u]);
                 else rope_cs(pos, s_theta[f], c2[u], s2v[u]);
             }
-            const float sg = half ? 1.f : -1.f;   // sin(-x) = -sin(x): exact
             rc = f2(c2[0], c2[1]);
-            rs = f2(sg * s2v[0], sg * s2v[1]);
+            rs = f2(s2v[0], s2v[1]);
             const int f0 = 32 * slice + 2 * cl;
             sc = f2(s_step_c[f0], s_step_c[f0 + 1]);
             ss = f2(s_step_s[f0], s_step_s[f0 + 1]);
             nss = f2(-s_step_s[f0], -s_step_s[f0 + 1]);
         }
-        const f2_t adv_c = half ? nss : ss, adv_s = half ? ss : nss;
-        uint8_t *yk = static_cast<uint8_t *>(p.yk) + 128 * half + 64 * slice + 4 * cl;
-        uint8_t *yv = static_cast<uint8_t *>(p.yv) + 128 * half + 64 * slice + 4 * cl;
+        const f2_t kNegOne2 = f2(-1.f, -1.f);
+        uint8_t *yk = static_cast<uint8_t *>(p.yk) + 64 * slice;
+        uint8_t *yv = static_cast<uint8_t *>(p.yv) + 64 * slice;
 #pragma unroll
         for (int i = 0; i < R; ++i) {
-            const int r = pwarp * R + i;
-            const int off = (r < rows ? r : rows - 1) * C::ROWB + 4 * lane;
-            const f2_t xk = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sk + off));
-            const f2_t xv = f2_from_bf16x2(*reinterpret_cast<const uint32_t *>(sv + off));
-            const f2_t og = gate_complement2(G[i]);
-            hk = f2_fma(G[i], hk, f2_mul(og, xk));
-            hv = f2_fma(G[i], hv, f2_mul(og, xv));
-            f2_t ok = hk;
+            const int r = seg * R + i;
+            const int off = soff(r < rows ? r : rows - 1) - 4 * cl;
+            f2_t xk[NP], xv[NP];
+            Lane<__nv_bfloat16>::template load<128>(sk + off, cl, xk);
+            Lane<__nv_bfloat16>::template load<128>(sv + off, cl, xv);
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const f2_t og = gate_complement2(G[i][q]);
+                hk[q] = f2_fma(G[i][q], hk[q], f2_mul(og, xk[q]));
+                hv[q] = f2_fma(G[i][q], hv[q], f2_mul(og, xv[q]));
+            }
+            f2_t ok[NP] = {hk[0], hk[1]};
             if (p.rope) {
-                const f2_t other = __shfl_xor_sync(0xffffffffu, hk, 16);
-                ok = f2_fma(other, rs, f2_mul(hk, rc));
-                // advance one position: (c + i s)(cos t + i sin t); rs keeps the half's sign
-                const f2_t nc = f2_fma(rc, sc, f2_mul(rs, adv_c));
-                rs = f2_fma(rs, sc, f2_mul(rc, adv_s));
+                const f2_t nrs = f2_mul(rs, kNegOne2);
+                ok[0] = f2_fma(hk[1], nrs, f2_mul(hk[0], rc));
+                ok[1] = f2_fma(hk[0], rs, f2_mul(hk[1], rc));
+                const f2_t nc = f2_fma(rc, sc, f2_mul(rs, nss));
+                rs = f2_fma(rs, sc, f2_mul(rc, ss));
                 rc = nc;
             }
             if (r < rows) {
                 const size_t go = (row0 + r) * (C::DH * 2);
-                *reinterpret_cast<uint32_t *>(yk + go) = f2_to_bf16x2(ok);
-                *reinterpret_cast<uint32_t *>(yv + go) = f2_to_bf16x2(hv);
+                Lane<__nv_bfloat16>::template store<128>(yk + go, cl, ok);
+                Lane<__nv_bfloat16>::template store<128>(yv + go, cl, hv);
             }
         }
         pipe_sync();
@@ -786,16 +827,18 @@ static PFN_cuTensorMapEncodeTiled_v12000 scan_encode_fn() {
     return fn;
 }
 
-// (32-channel column, half, row) view of a (rows, 128) bf16 tensor: x < 64 channels of a half,
-// y < 2 halves 64 channels apart, z < rows; box (32, 2, 128 rows), zero fill past the last row.
+// 5-D view of a (rows, 128) bf16 tensor, rows a multiple of 16: channel x < 64 of a half,
+// segment-in-warp u < 2 (8 rows apart), half y < 2 (64 channels apart), row-in-segment i < 8,
+// 16-row group g; box (32, 2, 2, 8, 8) = one 128-row chunk of one slice.
 static bool slice_map(CUtensorMap *m, const void *base, uint64_t rows) {
     auto fn = scan_encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[3] = {64, 2, rows};
-    cuuint64_t strides[2] = {64 * 2, 128 * 2};
-    cuuint32_t box[3] = {32, 2, (cuuint32_t)SliceCfg::TC};
-    cuuint32_t estr[3] = {1, 1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+    constexpr uint64_t row = 128 * 2;
+    cuuint64_t dims[5] = {64, 2, 2, 8, rows / 16};
+    cuuint64_t strides[4] = {8 * row, 64 * 2, row, 16 * row};
+    cuuint32_t box[5] = {32, 2, 2, 8, (cuuint32_t)SliceCfg::TC / 16};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -823,8 +866,8 @@ static int launch_slice(const RecurParams &p, void *stream) {
 }
 
 int launch_recur(const RecurParams &p, int dtype, void *stream) {
-    // bf16, d 128, full sequence, row coordinates within int32: the channel-sliced scan
-    if (dtype == RAT_BF16 && p.d == 128 && p.reset == 0 && (long long)p.BH * p.T < (1ll << 31) - SliceCfg::TC) {
+    // bf16, d 128, full sequence, T a multiple of 16: the channel-sliced scan
+    if (dtype == RAT_BF16 && p.d == 128 && p.reset == 0 && p.T % 16 == 0) {
         const int st = launch_slice(p, stream);
         if (st != RAT_ERR_UNSUPPORTED) return st;
     }

@@ -45,6 +45,16 @@ def inputs(B, H, T, d, dtype, mu=2.0, sigma=1.0, seed=0):
     return synthetic.prefill_inputs(w)
 
 
+# bf16 d128 full-sequence scans with T a multiple of 16 run in 64-channel slices with 128-row
+# chunks; these lengths end in partial chunks (and, for the last (b, h), a box past the tensor)
+@pytest.mark.parametrize("T", [16, 48, 208, 1008, 4096 + 16])
+def test_sliced_scan_partial_chunks(T):
+    x = inputs(2, 3, T, 128, torch.bfloat16, seed=T + 7)
+    g = torch.Generator().manual_seed(T)
+    h0 = (torch.randn((2, 3, 128), generator=g), torch.randn((2, 3, 128), generator=g))
+    check(x["k"], x["v"], x["a"], rope_base=10000.0, pos0=37, h0=h0)
+
+
 def test_tiny_fp32_workload():
     w = synthetic.WORKLOADS["tiny_fp32"]
     x = synthetic.prefill_inputs(w)
