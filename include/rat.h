@@ -109,7 +109,10 @@ RAT_API int rat_sync_status(void *ws, void *stream);
  * Computes g = 1/(1+exp(-a)), 1-g, and h_t = g h_{t-1} + (1-g) x_t in float32 for every
  * channel.  Outputs may not alias inputs.  T = 0 is a no-op.  The scan carries state between
  * chunks of the sequence with a bounded-wait decoupled look-back; if that wait runs out the
- * device error word becomes RAT_ERR_TIMEOUT (see rat_sync_status).
+ * device error word becomes RAT_ERR_TIMEOUT (see rat_sync_status).  For bf16, d = 128 and T a
+ * multiple of 16 the channels of each (b, h) scan as two independent 64-channel slices
+ * (channels [32s, 32s+32) with their rotate-half partners); results are the same up to float32
+ * rounding order.
  * ---------------------------------------------------------------------------------------- */
 RAT_API size_t rat_recur_workspace_bytes(int B, int H, int T, int d, int dtype);
 
@@ -472,8 +475,9 @@ RAT_API int rat_dilated_decode_paged(const void *q, const void *k, const void *v
 
 /* Test hook for failure detection (no counterpart in the method): the next rat_recur_prefill
  * issued from the calling host thread withholds the look-back publication of chunk `chunk`
- * (chunk index >= 1 along the sequence, in every (b, h)) and bounds each look-back wait by
- * wait_limit_ns (1 ms .. 2 s).  Its successors' waits run out, the call's results are wrong,
+ * (chunk index >= 1 along the sequence, in every (b, h) and channel slice; a chunk is 128 rows
+ * of 64 channels for bf16, d = 128 and T a multiple of 16, else 16 KiB of each tensor's rows)
+ * and bounds each look-back wait by wait_limit_ns (1 ms .. 2 s).  Its successors' waits run out, the call's results are wrong,
  * and rat_sync_status() reports RAT_ERR_TIMEOUT; nothing hangs and the context stays usable.
  * Returns RAT_ERR_INVALID for out-of-range arguments. */
 RAT_API int rat_debug_inject_lookback_fault(int64_t chunk, int64_t wait_limit_ns);
