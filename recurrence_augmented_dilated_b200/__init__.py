@@ -162,7 +162,17 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _ptr(t: Optional[torch.Tensor]):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a tensor argument.  The library reads and writes every tensor as one
+    dense block of device memory, so a host tensor or a strided view is refused here (a host
+    address would be an illegal device access; a view would be read as if it were dense)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise RatError("tensor argument on %s (the library takes CUDA tensors)" % t.device, -1)
+    if not t.is_contiguous():
+        raise RatError("non-contiguous tensor argument (shape %s, strides %s)"
+                       % (tuple(t.shape), t.stride()), -1)
+    return ctypes.c_void_p(t.data_ptr())
 
 
 def _stream(stream=None):
@@ -284,7 +294,7 @@ def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,
     if D_per_head is not None:
         dph = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
     if lse is not None:
-        opt = AttnOptions(n_sink=int(n_sink), top_k=int(top_k), lse=lse.data_ptr())
+        opt = AttnOptions(n_sink=int(n_sink), top_k=int(top_k), lse=_ptr(lse).value)
         st = lib().rat_dilated_attn_prefill_ex(_ptr(q), _ptr(k_rec), _ptr(v_rec), _ptr(o), B, H, T,
                                                d, _dtype_code(q), int(D), int(W), dph, int(pos0),
                                                float(rope_base), float(scale), ctypes.byref(opt),

@@ -261,3 +261,16 @@ def test_paged_validation(L):
 def test_workspace_init_rejects_null(L):
     assert L.rat_workspace_init(None, 1024, None) == -5
     assert L.rat_sync_status(None, None) == -5
+
+
+def test_binding_refuses_host_tensors():
+    # the binding passes device addresses only: a host tensor is refused before any library call
+    import torch
+    k = torch.zeros((1, 1, 16, 128), dtype=torch.bfloat16)
+    with pytest.raises(rat.RatError) as e:
+        rat.rat_recur_prefill(k, k, k, k, k, ws=None)
+    assert e.value.status == -1
+    with pytest.raises(rat.RatError) as e:
+        rat.rat_dilated_attn_prefill(k, k, k, k, D=4)
+    assert e.value.status == -1
+    assert rat._ptr(None) is None
