@@ -54,8 +54,21 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+# device-code headers every kernel file includes
+KERNEL_HEADERS = ("common.cuh", "internal.h", "tc.cuh")
+
+
+def headers_sha():
+    h = hashlib.sha256()
+    for n in KERNEL_HEADERS:
+        with open(os.path.join(ROOT, "recurrence_augmented_dilated_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(kernel_file: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel is unchanged since."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernel is unchanged since: its
+    source file's hash, and (for entries that record it) the shared headers' hash, must match."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -64,6 +77,8 @@ def recorded_traffic(kernel_file: str, workload: str):
     e = table.get(kernel_file, {}).get(workload)
     src = os.path.join(ROOT, "recurrence_augmented_dilated_b200", "csrc", kernel_file)
     if not e or not os.path.exists(src) or e.get("source_sha") != file_sha(src):
+        return None
+    if "headers_sha" in e and e["headers_sha"] != headers_sha():
         return None
     return e.get("dram_bytes_per_launch")
 

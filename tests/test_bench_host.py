@@ -86,7 +86,15 @@ def test_recorded_traffic_follows_the_source_hash():
     for kernel_file, rows in table.items():
         for workload, e in rows.items():
             src = os.path.join(bench.ROOT, "recurrence_augmented_dilated_b200", "csrc", kernel_file)
-            want = e["dram_bytes_per_launch"] if e["source_sha"] == bench.file_sha(src) else None
+            same = e["source_sha"] == bench.file_sha(src) and \
+                e.get("headers_sha", bench.headers_sha()) == bench.headers_sha()
+            want = e["dram_bytes_per_launch"] if same else None
             assert bench.recorded_traffic(kernel_file, workload) == want
             assert os.path.exists(os.path.join(bench.ROOT, "profiles", e["capture"]))
     assert bench.recorded_traffic("scan.cu", "no_such_workload") is None
+
+
+def test_recorded_traffic_void_after_a_header_change(monkeypatch):
+    assert bench.recorded_traffic("scan.cu", "prefill_1p5b") is not None
+    monkeypatch.setattr(bench, "headers_sha", lambda: "0000000000000000")
+    assert bench.recorded_traffic("scan.cu", "prefill_1p5b") is None
