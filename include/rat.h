@@ -112,7 +112,9 @@ RAT_API int rat_sync_status(void *ws, void *stream);
  * device error word becomes RAT_ERR_TIMEOUT (see rat_sync_status).  For bf16, d = 128 and T a
  * multiple of 16 the channels of each (b, h) scan as two independent 64-channel slices
  * (channels [32s, 32s+32) with their rotate-half partners); results are the same up to float32
- * rounding order.
+ * rounding order.  Run-to-run reproducibility is to rounding, not to the bit: a chunk composes
+ * whichever predecessors' records are ready when it looks back, so the float32 carries (and
+ * through them a stored bf16 value) may differ in the last bit between two identical calls.
  * ---------------------------------------------------------------------------------------- */
 RAT_API size_t rat_recur_workspace_bytes(int B, int H, int T, int d, int dtype);
 
