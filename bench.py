@@ -2,15 +2,17 @@
 """Benchmark of the RAT+ dilated-inference hot path on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload prefill_1p5b] [--no-decode] [--all]
+                    [--workload hybrid_7p6b] [--only] [--no-decode]
 
 One step = one pass of the prefill path over one batch of the workload: the forget-gate
 recurrence over k and v (rat_recur_prefill), dilated attention (rat_dilated_attn_prefill) and
 the compressed-cache build (rat_kv_compress), on synthetic inputs already resident in HBM.
-`value` is prefill tokens/s over all ranks (B*T tokens per rank per step; weak scaling: every
-rank runs its own batch, no data-path collective).  Sub-objects report decode tokens/s on the
-decode workload (256 one-token steps against the compressed cache) and, with --all, the
-other prefill workloads.  Each kernel's average duration is measured with CUDA events on its
+`value` is prefill tokens/s over all ranks on the headline workload (the largest one, the
+7.6B-like hybrid head composition; B*T tokens per rank per step; weak scaling: every rank runs
+its own batch, no data-path collective).  The `workloads` object holds every other workload,
+each with its own kernels, roofline, clocks and CPU baseline: the 1.5B-like and 2.6B-like
+prefill, the tiny float32 layer, and decode (256 one-token steps against the compressed
+cache).  Each kernel's average duration is measured with CUDA events on its
 own stream inside the timed region and turned into a roofline fraction with the algorithmic
 bytes (or FLOPs) of one launch.
 
@@ -311,7 +313,22 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
     ms = e0.elapsed_time(e1) / steps
     ms_max = max_over_ranks(ms, world)
     kern = timer.mean_ms()
-    kern.update(side_timer.mean_ms())
+    span = side_timer.mean_ms()
+    # the append's own duration: timed alone on the main stream after the step loop (beside the
+    # attention its span also counts the time it waits for SM slots)
+    # (back to back between two events: one launch between events would also count the host's
+    # submission time of each call)
+    n_solo = max(8, steps)
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    cache.pos = 0
+    rat.rat_kv_compress(kr, vr, hk, hv, cache)
+    c0.record(stream)
+    for _ in range(n_solo):
+        cache.pos = 0
+        rat.rat_kv_compress(kr, vr, hk, hv, cache)
+    c1.record(stream)
+    torch.cuda.synchronize()
+    kern["compress"] = c0.elapsed_time(c1) / n_solo
     st = rat.rat_sync_status(ws)
     if st != 0:
         raise RuntimeError("device error " + rat.rat_status_string(st))
@@ -324,9 +341,16 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
         "gpu_launches_per_step": 3,
     }
     hbm = peaks["hbm_gbs"]
-    tc = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    # a step of a few ms timed over tens of steps is a burst, not a seconds-long loop under the
+    # power cap: the tensor-bound fraction is taken against the burst GEMM peak (the sustained
+    # one is reported beside it)
+    tc = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    tc_sus = peaks.get("bf16_tflops_sustained", tc)
+    step_kern = {n: t for n, t in kern.items() if n != "compress"}
     for name, t in kern.items():
-        e = {"ms": t, "share_of_kernel_time": t / sum(kern.values())}
+        e = {"ms": t}
+        if name in step_kern:
+            e["share_of_kernel_time"] = t / sum(step_kern.values())
         if name == "recur":
             e.update(bound="hbm", achieved=alg["recur_bytes"] / (t * 1e-3) / 1e9, peak=hbm, unit="GB/s")
         elif name == "attn":
@@ -337,12 +361,12 @@ def run_prefill(w: synthetic.Workload, steps: int, warmup: int, rank: int, world
             if alg["attn_flops"] / alg["attn_bytes"] < ridge or w.dtype == "f32":
                 e.update(bound="hbm", achieved=gbs, peak=hbm, unit="GB/s", tflops=tfs)
             else:
-                e.update(bound="tensor", achieved=tfs, peak=tc, unit="TFLOP/s", gbs=gbs)
+                e.update(bound="tensor", achieved=tfs, peak=tc, unit="TFLOP/s", gbs=gbs,
+                         peak_kind="burst", frac_of_sustained=tfs / tc_sus)
         elif name == "compress":
-            # launched beside the attention: the span runs from its launch until the attention
-            # leaves it SM slots, so it is not the kernel's own duration
+            # standalone duration; in the step it runs on a second stream beside the attention
             e.update(bound="hbm", achieved=alg["compress_bytes"] / (t * 1e-3) / 1e9, peak=hbm, unit="GB/s",
-                     overlapped_with="attn")
+                     overlapped_with="attn", span_beside_attn_ms=span.get("compress"))
         e["frac"] = e["achieved"] / e["peak"]
         e["of"] = peak_kind
         res["kernels"][name] = e
@@ -368,11 +392,25 @@ class _Null:
         return False
 
 
+def e2e_chunks(B: int, H: int, min_chunks: int = 4):
+    """(b, h0, h1) pieces of a (B, H, T, d) batch for the end-to-end pipeline: whole batch rows,
+    or, when there are fewer rows than min_chunks, groups of heads of one row (each piece
+    x[b:b+1, h0:h1] is one contiguous range)."""
+    per_row = 1
+    while B * per_row < min_chunks and per_row < H:
+        per_row *= 2
+    while H % per_row:
+        per_row -= 1
+    g = H // per_row
+    return [(b, i * g, (i + 1) * g) for b in range(B) for i in range(per_row)]
+
+
 def run_e2e(w, steps, warmup, x, dev, world):
-    """The layer step through the public API from host buffers: for each batch row, the H2D copy
-    of its q, k, v, a from pinned memory, the three calls, and the D2H copy of its output, on
-    three streams (copy in, compute, copy out) so that one row's copies overlap another row's
-    compute. Every copy of the step is inside the timed region."""
+    """The layer step through the public API from host buffers: for each piece of the batch (a
+    batch row, or a group of heads of one row), the H2D copy of its q, k, v, a from pinned
+    memory, the three calls, and the D2H copy of its output, on three streams (copy in, compute,
+    copy out) so that one piece's copies overlap another piece's compute. Every copy of the step
+    is inside the timed region."""
     import recurrence_augmented_dilated_b200 as rat
     names = ("q", "k", "v", "a")
     host = {n: x[n].pin_memory() for n in names}
@@ -380,45 +418,48 @@ def run_e2e(w, steps, warmup, x, dev, world):
     out_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
     B, H, T, d = o.shape
     dtc = rat.F32 if w.dtype == "f32" else rat.BF16
-    Dph = list(w.D_per_head) if w.D_per_head else None
-    # one cache and one scan workspace per batch row (calls on one row never overlap themselves)
-    caches = [rat.make_cache(1, H, d, w.W, T, dtc, w.heads_D()) for _ in range(B)]
-    ws = [rat.Workspace(rat.rat_recur_workspace_bytes(1, H, T, d, dtc)) for _ in range(B)]
+    Dh = w.heads_D()
+    pieces = e2e_chunks(B, H)
+    P = len(pieces)
+    # one cache and one scan workspace per piece (calls on one piece never overlap themselves)
+    caches = [rat.make_cache(1, h1 - h0, d, w.W, T, dtc, Dh[h0:h1]) for (_, h0, h1) in pieces]
+    ws = [rat.Workspace(rat.rat_recur_workspace_bytes(1, h1 - h0, T, d, dtc)) for (_, h0, h1) in pieces]
     s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    ev_in = [torch.cuda.Event() for _ in range(B)]
-    ev_comp = [torch.cuda.Event() for _ in range(B)]
-    ev_out = [torch.cuda.Event() for _ in range(B)]
+    ev_in = [torch.cuda.Event() for _ in range(P)]
+    ev_comp = [torch.cuda.Event() for _ in range(P)]
+    ev_out = [torch.cuda.Event() for _ in range(P)]
 
     def e2e_step():
-        for b in range(B):
-            r = slice(b, b + 1)
-            s_in.wait_event(ev_comp[b])          # the previous step's row b no longer needs its inputs
+        for i, (b, h0, h1) in enumerate(pieces):
+            r = (slice(b, b + 1), slice(h0, h1))
+            Dph = Dh[h0:h1] if w.D_per_head else None
+            s_in.wait_event(ev_comp[i])          # the previous step's piece i no longer needs its inputs
             with torch.cuda.stream(s_in):
                 for n in names:
                     dev[n][r].copy_(host[n][r], non_blocking=True)
-                ev_in[b].record(s_in)
-            s_comp.wait_event(ev_in[b])
-            s_comp.wait_event(ev_out[b])         # the previous step's row b output has been read
+                ev_in[i].record(s_in)
+            s_comp.wait_event(ev_in[i])
+            s_comp.wait_event(ev_out[i])         # the previous step's piece i output has been read
             with torch.cuda.stream(s_comp):
-                rat.rat_recur_prefill(dev["k"][r], dev["v"][r], dev["a"][r], kr[r], vr[r], ws[b],
+                rat.rat_recur_prefill(dev["k"][r], dev["v"][r], dev["a"][r], kr[r], vr[r], ws[i],
                                       hT_k=hk[r], hT_v=hv[r], rope_base=w.rope_base)
                 rat.rat_dilated_attn_prefill(dev["q"][r], kr[r], vr[r], o[r], D=w.D, W=w.W,
                                              D_per_head=Dph, rope_base=w.rope_base)
-                cache = caches[b][0]
+                cache = caches[i][0]
                 cache.pos = 0
                 rat.rat_kv_compress(kr[r], vr[r], hk[r], hv[r], cache)
-                ev_comp[b].record(s_comp)
-            s_out.wait_event(ev_comp[b])
+                ev_comp[i].record(s_comp)
+            s_out.wait_event(ev_comp[i])
             with torch.cuda.stream(s_out):
                 out_host[r].copy_(o[r], non_blocking=True)
-                ev_out[b].record(s_out)
+                ev_out[i].record(s_out)
 
     cur = torch.cuda.current_stream()
     for _ in range(max(1, warmup)):
         e2e_step()
     torch.cuda.synchronize()
-    for b in range(B):
-        if rat.rat_sync_status(ws[b]) != 0:
+    for i in range(P):
+        if rat.rat_sync_status(ws[i]) != 0:
             raise RuntimeError("device error in the end-to-end leg")
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -437,7 +478,8 @@ def run_e2e(w, steps, warmup, x, dev, world):
     d2h = out_host.numel() * out_host.element_size()
     return {"value": world * w.B * w.T / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "method": "per batch row: H2D, recurrence + attention + compress, D2H on three streams",
+            "method": "%d pieces (batch row x head group): H2D, recurrence + attention + compress, "
+                      "D2H on three streams" % P,
             "out": out_host}
 
 
@@ -736,16 +778,19 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
 # ----------------------------------------------------------------------------- oracle (CPU)
 def oracle_sample(w: synthetic.Workload, budget_s: float = 12.0):
     """Time the float64 oracle on whole (b, h) slices of w (recurrence + RoPE + attention over
-    every query row), as many slices as fit the budget (all of them when the workload fits);
-    returns (tokens/s scaled to the whole workload, threads, description, seconds)."""
+    every query row, or over evenly spaced rows when a slice does not fit the budget).  Heads
+    are sampled per dilation class (a hybrid's dense and dilated heads cost very different
+    amounts), each class's time scaled by its own slice count; returns (tokens/s scaled to the
+    whole workload, threads, description, seconds spent)."""
     import numpy as np
     import oracle
     cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     Dh = w.heads_D()
-    nsl = w.B * w.H
     x = synthetic.prefill_inputs(w)
-    # slices (b, h) b-major, heads interleaved by parity so a hybrid sample mixes dilations
-    order = sorted(range(nsl), key=lambda i: ((i % w.H) % 2, i))
+    classes = {}
+    for i in range(w.B * w.H):
+        classes.setdefault(Dh[i % w.H], []).append(i)
+    budget_c = budget_s / len(classes)
 
     def run(slices, rows, threads):
         b_idx = [i // w.H for i in slices]
@@ -757,49 +802,125 @@ def oracle_sample(w: synthetic.Workload, budget_s: float = 12.0):
                              W=w.W, rope_base=w.rope_base, rows=rows)
         return time.perf_counter() - t0
 
-    # probe one wave of slices in parallel at 32 and 96 rows: time = fixed (the recurrence over
-    # all T) + per row
-    nprobe = max(1, min(cores, nsl, 8))
-    wave = sorted(order[:nprobe])
-    t32 = run(wave, np.linspace(0, w.T - 1, 32).astype(np.int64), nprobe)
-    t96 = run(wave, np.linspace(0, w.T - 1, 96).astype(np.int64), nprobe)
-    per_row = max(t96 - t32, 1e-9) / 64
-    fixed = max(t32 - 32 * per_row, 0.0)
-    wave_full = fixed + per_row * w.T            # seconds for one wave of nprobe slices, all rows
-    waves = budget_s / max(wave_full, 1e-9)
-    rows = None
-    if waves >= 1:
-        nslices = min(nsl, max(nprobe, int(waves) * nprobe))
-    else:
-        nslices = nprobe
-        n = int((budget_s - fixed) / per_row) if budget_s > fixed else 32
-        rows = np.linspace(0, w.T - 1, min(w.T, max(32, n))).astype(np.int64)
+    total_s, spent, used, descs = 0.0, 0.0, 1, []
+    for D, members in sorted(classes.items()):
+        nsl = len(members)
+        # probe one wave of slices in parallel at 32 and 96 rows: time = fixed (the recurrence
+        # over all T) + per row
+        nprobe = max(1, min(cores, nsl, 8))
+        wave = members[:nprobe]
+        t32 = run(wave, np.linspace(0, w.T - 1, 32).astype(np.int64), nprobe)
+        t96 = run(wave, np.linspace(0, w.T - 1, 96).astype(np.int64), nprobe)
+        per_row = max(t96 - t32, 1e-9) / 64
+        fixed = max(t32 - 32 * per_row, 0.0)
+        wave_full = fixed + per_row * w.T        # one wave of nprobe slices, all rows
+        waves = budget_c / max(wave_full, 1e-9)
+        rows = None
+        if waves >= 1:
+            nslices = min(nsl, max(nprobe, int(waves) * nprobe))
+        else:
+            nslices = nprobe
+            n = int((budget_c - fixed) / per_row) if budget_c > fixed else 32
+            rows = np.linspace(0, w.T - 1, min(w.T, max(32, n))).astype(np.int64)
+        threads = max(1, min(cores, nslices))
+        used = max(used, threads)
+        slices = members[:nslices]
+        # a sample shorter than the budget (the whole class, when it fits) is repeated until
+        # about half the budget has been spent, and timed as the mean
+        reps, el = 0, 0.0
+        while reps == 0 or (el < 0.5 * budget_c and reps < 100):
+            el += run(slices, rows, threads)
+            reps += 1
+        spent += el + t32 + t96
+        frac_rows = 1.0 if rows is None else len(rows) / w.T
+        total_s += el / reps / frac_rows * nsl / nslices
+        descs.append("D=%d: %d of %d (b,h) slices, %s query rows, %d threads, mean of %d runs" % (
+            D, nslices, nsl, "all" if rows is None else "%d of %d" % (len(rows), w.T), threads, reps))
+    desc = "float64 oracle (recurrence + RoPE + attention); " + "; ".join(descs) + (
+        "; each dilation class scaled by its slice count" if len(classes) > 1 else "")
+    return w.B * w.T / total_s, used, desc, spent
+
+
+def oracle_decode_sample(w: synthetic.Workload, budget_s: float = 6.0, nslices: int = 8):
+    """Time the float64 decode oracle (state update, RoPE, attention over the whole history) on
+    nslices (b, h) slices of the decode workload: their contexts are consumed untimed, then
+    decode steps run until about the budget is spent; the per-step time is scaled to all
+    B*H slices.  Returns (tokens/s, threads, description, seconds)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    Dh = w.heads_D()
+    BH = w.B * w.H
+    picks = [(i * BH // nslices) for i in range(nslices)]
+    bh = [(i // w.H, i % w.H) for i in picks]
+    st = oracle.DecodeState([Dh[h] for _, h in bh], w.d, w.W, w.T + w.steps, rope_base=w.rope_base)
+    ctx = [synthetic.decode_context_slice(w, b, h) for b, h in bh]
+    st.prefill(*(torch.stack([c[i] for c in ctx]).double().numpy() for i in range(3)))
+    del ctx
+    tok = synthetic.decode_steps(w)
+    b_idx = [b for b, _ in bh]
+    h_idx = [h for _, h in bh]
+    tq, tk, tv, ta = (tok[n][:, b_idx, h_idx].double().numpy() for n in ("q", "k", "v", "a"))
     threads = max(1, min(cores, nslices))
-    slices = sorted(order[:nslices])
-    # a sample shorter than the budget (the whole workload, when it fits) is repeated until
-    # about half the budget has been spent, and timed as the mean
-    reps, el = 0, 0.0
-    while reps == 0 or (el < 0.5 * budget_s and reps < 100):
-        el += run(slices, rows, threads)
-        reps += 1
-    frac_rows = 1.0 if rows is None else len(rows) / w.T
-    full_s = el / reps / frac_rows * nsl / nslices
-    desc = "%d of %d (b,h) slices, %s query rows, float64, %d OpenMP threads, mean of %d runs" % (
-        nslices, nsl, "all" if rows is None else "%d of %d" % (len(rows), w.T), threads, reps)
-    return w.B * w.T / full_s, threads, desc, el
+    oracle.set_threads(threads)
+    n, el = 0, 0.0
+    while n < w.steps and (n < 8 or el < budget_s):
+        t0 = time.perf_counter()
+        st.step(tq[n], tk[n], tv[n], ta[n])
+        el += time.perf_counter() - t0
+        n += 1
+    step_full = el / n * BH / nslices
+    desc = ("float64 decode oracle on %d of %d (b,h) slices (full history kept), %d of %d steps "
+            "after the %d-position context, %d threads; scaled to all slices" % (
+                nslices, BH, n, w.steps, w.T, threads))
+    return w.B / step_full, threads, desc, el
 
 
 # ----------------------------------------------------------------------------- main
+OTHER_PREFILL = ("prefill_1p5b", "window_2p6b", "tiny_fp32")
+
+
+def dominant_roofline(kern, peak_kind):
+    """The roofline object of the step's dominant kernel (the cache append overlaps the
+    attention and is left out)."""
+    name = max((n for n in kern if not kern[n].get("overlapped_with")), key=lambda n: kern[n]["ms"])
+    k = kern[name]
+    roof = {"bound": k["bound"], "achieved": k["achieved"], "peak": k["peak"], "unit": k["unit"],
+            "frac": k["frac"], "of": peak_kind, "kernel": name, "traffic": k.get("traffic")}
+    if "peak_kind" in k:
+        roof["peak_kind"] = k["peak_kind"]
+        roof["frac_of_sustained"] = k["frac_of_sustained"]
+    return roof
+
+
+def attach_traffic(kern, w, variant="", window=0, n_sink=0, top_k=0):
+    src_of = {"recur": "window.cu" if window else "scan.cu",
+              "attn": "attn_simt.cu" if (top_k or (n_sink and w.dtype == "f32")) else "attn_sm100.cu",
+              "compress": "compress.cu"}
+    attn_variant = ("_top%d" % top_k if top_k else "") + ("_sinks%d" % n_sink if n_sink else "")
+    for n in kern:      # DRAM bytes per launch from the committed ncu capture (null if stale)
+        kern[n]["traffic"] = recorded_traffic(
+            src_of[n], w.name + (variant if n == "recur" else attn_variant if n == "attn" else ""))
+
+
+def workload_config(w):
+    return {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "D": w.D, "W": w.W,
+            "D_per_head": list(w.D_per_head) if w.D_per_head else None,
+            "rope_base": w.rope_base, "gates": [w.gate_mu, w.gate_sigma], "dtype": w.dtype}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="prefill_1p5b")
+    ap.add_argument("--workload", default="hybrid_7p6b",
+                    help="the headline prefill workload (top-level value and roofline)")
+    ap.add_argument("--only", action="store_true",
+                    help="time the headline workload alone (no other workloads, no decode)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--all", action="store_true", help="also time the other prefill workloads")
+    ap.add_argument("--all", action="store_true", help="(default) kept for older command lines")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--reset-every", type=int, default=0,
                     help="L > 0: the chunk-local recurrence (restart every L positions) in the "
@@ -819,6 +940,7 @@ def main():
                     help="keep warming up at least this long (clock sampling); 0 under a profiler")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    variant_leg = bool(args.reset_every or args.window or args.sinks or args.top_k)
 
     w = synthetic.WORKLOADS[args.workload]
     metric = "RAT+ layer prefill tokens/s and decode tokens/s at 1 B200; % HBM / tensor roofline"
@@ -838,8 +960,7 @@ def main():
                 "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": w.B * w.T / value * 1e3, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "D": w.D,
-                           "W": w.W, "rope_base": w.rope_base},
+                "config": workload_config(w),
                 "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                                  "sample": desc},
                 "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -853,72 +974,82 @@ def main():
     rank, world, local = dist_setup(args.gpus)
     import recurrence_augmented_dilated_b200 as rat
     rat.lib()       # fail loudly if the library is missing
+    cpu_here = rank == 0 and world == 1 and not args.no_cpu_baseline
 
     pre = run_prefill(w, args.steps, args.warmup, rank, world, peaks, peak_kind,
-                      with_e2e=(not args.no_e2e and args.reset_every == 0 and args.window == 0 and
-                                args.sinks == 0 and args.top_k == 0),
+                      with_e2e=(not args.no_e2e and not variant_leg),
                       min_warmup_s=args.min_warmup_s, reset_every=args.reset_every,
                       window=args.window, n_sink=args.sinks, top_k=args.top_k)
     kern = pre["kernels"]
-    src_of = {"recur": "window.cu" if args.window else "scan.cu",
-              "attn": "attn_simt.cu" if (args.sinks or args.top_k) else "attn_sm100.cu",
-              "compress": "compress.cu"}
     variant = ("_L%d" % args.reset_every if args.reset_every else
                "_window%d" % args.window if args.window else "")
-    for n in kern:      # DRAM bytes per launch from the committed ncu capture (null if stale)
-        kern[n]["traffic"] = recorded_traffic(src_of[n], w.name + (variant if n == "recur" else ""))
-    # the dominant kernel of the step (the cache append overlaps the attention)
-    dom_name = max((n for n in kern if not kern[n].get("overlapped_with")), key=lambda n: kern[n]["ms"])
-    dom = kern[dom_name]
-    roof = {"bound": dom["bound"], "achieved": dom["achieved"], "peak": dom["peak"],
-            "unit": dom["unit"], "frac": dom["frac"], "of": peak_kind, "kernel": dom_name,
-            "traffic": kern[dom_name]["traffic"]}
+    attach_traffic(kern, w, variant, args.window, args.sinks, args.top_k)
+    cfg = workload_config(w)
+    cfg.update({
+        "step": "%s + %s + rat_kv_compress (on a second stream, beside the attention)" % (
+            "rat_recur_prefill_window(Lw=%d)" % args.window if args.window else
+            "rat_recur_prefill_local(L=%d)" % args.reset_every if args.reset_every else
+            "rat_recur_prefill",
+            "rat_dilated_attn_prefill_topk(n_sink=%d, top_k=%d)" % (args.sinks, args.top_k)
+            if args.top_k else
+            "rat_dilated_attn_prefill_sinks(n_sink=%d)" % args.sinks if args.sinks else
+            "rat_dilated_attn_prefill"),
+        "l2": "inputs larger than L2 (q, k, v, a = %d MB per rank)" % (
+            4 * w.B * w.H * w.T * w.d * (2 if w.dtype == "bf16" else 4) // 2**20),
+        "parallelism": "replicas: dp%d over (batch) with no collective" % world})
     line = {
         "metric": metric, "value": pre["tokens_per_s"], "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": pre["ms_per_step"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f32", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "d": w.d, "D": w.D, "W": w.W,
-                   "D_per_head": list(w.D_per_head) if w.D_per_head else None,
-                   "rope_base": w.rope_base, "gates": [w.gate_mu, w.gate_sigma],
-                   "step": "%s + %s + rat_kv_compress (on a second stream, beside the attention)" % (
-                       "rat_recur_prefill_window(Lw=%d)" % args.window if args.window else
-                       "rat_recur_prefill_local(L=%d)" % args.reset_every if args.reset_every else
-                       "rat_recur_prefill",
-                       "rat_dilated_attn_prefill_topk(n_sink=%d, top_k=%d)" % (args.sinks, args.top_k)
-                       if args.top_k else
-                       "rat_dilated_attn_prefill_sinks(n_sink=%d)" % args.sinks if args.sinks else
-                       "rat_dilated_attn_prefill"),
-                   "l2": "inputs larger than L2 (q, k, v, a = %d MB per rank)" % (
-                       4 * w.B * w.H * w.T * w.d * (2 if w.dtype == "bf16" else 4) // 2**20),
-                   "parallelism": "replicas: dp%d over (batch) with no collective" % world},
-        "roofline": roof,
+        "config": cfg,
+        "roofline": dominant_roofline(kern, peak_kind),
         "kernels": kern,
         "clocks": pre["clocks"],
         "e2e": pre.get("e2e"),
         "gpu_launches": pre["gpu_launches_per_step"] * args.steps,
     }
-    if not args.no_decode:
+    if cpu_here:
+        v, cores, desc, el = oracle_sample(w)
+        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": el}
+
+    # every other workload, each with its own kernels, roofline, clocks and CPU baseline
+    others = {}
+    if not args.only and not variant_leg:
+        for name in OTHER_PREFILL:
+            if name == w.name:
+                continue
+            ow = synthetic.WORKLOADS[name]
+            r = run_prefill(ow, args.steps, args.warmup, rank, world, peaks, peak_kind,
+                            with_e2e=False, min_warmup_s=args.min_warmup_s)
+            attach_traffic(r["kernels"], ow)
+            sub = {"metric": "prefill tokens/s", "value": r["tokens_per_s"], "unit": "tokens/s",
+                   "ms_per_step": r["ms_per_step"], "config": workload_config(ow),
+                   "roofline": dominant_roofline(r["kernels"], peak_kind),
+                   "kernels": r["kernels"], "clocks": r["clocks"],
+                   "gpu_launches": r["gpu_launches_per_step"] * args.steps}
+            if cpu_here:
+                v, cores, desc, el = oracle_sample(ow, budget_s=6.0)
+                sub["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores,
+                                       "kind": "oracle", "sample": desc, "seconds": el}
+            others[name] = sub
+    if not args.no_decode and not args.only:
         dw = synthetic.WORKLOADS["decode_7p6b"]
-        line["decode"] = run_decode(dw, max(1, min(args.steps, 10)), 3, rank, world, peaks, peak_kind)
+        dec = run_decode(dw, max(1, min(args.steps, 10)), 3, rank, world, peaks, peak_kind)
+        if cpu_here:
+            v, cores, desc, el = oracle_decode_sample(dw)
+            dec["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                   "sample": desc, "seconds": el}
+        others["decode_7p6b"] = dec
+    if others:
+        line["workloads"] = others
     if args.backward:
         line["backward"] = run_backward(w, args.steps, args.warmup, world, peaks, peak_kind)
     if args.decode_paged:
         dw = synthetic.WORKLOADS["decode_7p6b"]
         line["decode_paged"] = run_decode_paged(dw, max(1, min(args.steps, 10)), 3, rank, world,
                                                 peaks, peak_kind)
-    if args.all:
-        line["other_workloads"] = []
-        for name in ("window_2p6b", "hybrid_7p6b", "tiny_fp32"):
-            r = run_prefill(synthetic.WORKLOADS[name], max(3, args.steps // 2), args.warmup, rank,
-                            world, peaks, peak_kind, with_e2e=False, min_warmup_s=args.min_warmup_s)
-            line["other_workloads"].append({"workload": name, "tokens_per_s": r["tokens_per_s"],
-                                            "ms_per_step": r["ms_per_step"], "kernels": r["kernels"],
-                                            "clocks": r["clocks"]})
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, desc, el = oracle_sample(w)
-        line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                                "sample": desc, "seconds": el}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
