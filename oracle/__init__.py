@@ -263,6 +263,20 @@ def dilated_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, rows=None,
     return (out, lse) if return_lse else out
 
 
+def attention_over_keys(q_t, k, v, keys, scale):
+    """Softmax attention of one query over an explicit list of key positions, each listed once:
+    o = sum_j softmax_j(scale * <q_t, k_j>) v_j over j in keys (the attention step of the RAT+
+    abstract and "RAT+ Deep Dive" section 3.1, with the key set given rather than derived).
+    Used where a key set comes from a selection with several admissible outcomes (top-k chunks
+    whose scores tie within rounding).  q_t (d,), k and v (T, d), keys a sequence of ints;
+    returns (d,) in float64."""
+    q_t, k, v = _f64(q_t), _f64(k), _f64(v)
+    idx = np.asarray(list(keys), dtype=np.int64)
+    s = scale * (k[idx] @ q_t)
+    p = np.exp(s - s.max())
+    return (p @ v[idx]) / p.sum()
+
+
 def topk_attention(q, k, v, D=1, W=0, D_per_head=None, scale=None, n_sink=0, top_k=0):
     """Dilated attention plus the top_k chunks (scored by their chunk-end keys) attended at
     every position ("RAT+ Deep Dive" section 4, dilation combined with top-k selection).

@@ -501,6 +501,34 @@ def test_topk_equals_masked_sdpa_with_argsort_selection(D, W, n_sink, top_k):
     np.testing.assert_allclose(got, ref.numpy(), rtol=1e-11, atol=1e-12)
 
 
+def test_attention_over_keys_equals_masked_sdpa():
+    # explicit key lists (random subsets, in shuffled order) against library attention under the
+    # matching boolean mask
+    T, d, scale = 50, 16, 0.3
+    q, k, v = (RNG.standard_normal((T, d)) for _ in range(3))
+    for t in (0, 7, 31, 49):
+        keys = RNG.permutation(t + 1)[:max(1, (t + 1) // 2)]
+        mask = np.zeros((1, T), dtype=bool)
+        mask[0, keys] = True
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q[t:t + 1]), torch.tensor(k), torch.tensor(v),
+            attn_mask=torch.tensor(mask), scale=scale).numpy()[0]
+        np.testing.assert_allclose(oracle.attention_over_keys(q[t], k, v, keys, scale), ref,
+                                   rtol=1e-12, atol=1e-13)
+
+
+def test_attention_over_the_key_set_is_the_dilated_attention():
+    T, d, D, W, n_sink = 90, 8, 6, 5, 2
+    q, k, v = (RNG.standard_normal((1, 1, T, d)) for _ in range(3))
+    scale = oracle.default_scale(d)
+    ref = oracle.dilated_attention(q, k, v, D=D, W=W, n_sink=n_sink)
+    for t in (0, 4, 5, 40, 89):
+        keys = [j for j in range(t + 1) if oracle.in_key_set(t, j, D, W, n_sink)]
+        np.testing.assert_allclose(oracle.attention_over_keys(q[0, 0, t], k[0, 0], v[0, 0], keys,
+                                                              scale), ref[0, 0, t],
+                                   rtol=1e-12, atol=1e-13)
+
+
 def test_attention_lse_is_the_log_partition():
     # log2 sum_j exp(s_j) over the key set, by a library logsumexp over the masked scores
     from scipy.special import logsumexp
