@@ -239,6 +239,12 @@ RAT_API int rat_recur_prefill_window(const void *k, const void *v, const void *g
  * Needs no workspace and never waits on other CTAs; its internal pipeline waits are bounded,
  * and an expired wait is recorded in a library-wide device error word that
  * rat_attn_sync_status() reads.
+ * RoPE on the tensor-core path reads a per-device table of the frequency set: the first call
+ * with a new rope_base (for a given d) writes it once and waits for that copy on the host
+ * before returning, so calls on any number of streams may follow without host syncs.  Up to 16
+ * distinct sets per device are kept for the life of the process; a 17th is refused with
+ * RAT_ERR_UNSUPPORTED, and so is the first call with a new set while `stream` is being
+ * captured into a CUDA graph (make one call outside the capture first).
  * ---------------------------------------------------------------------------------------- */
 RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o,
                              int B, int H, int T, int d, int dtype, int D, int W,
@@ -495,7 +501,10 @@ RAT_API int rat_debug_inject_lookback_fault(int64_t chunk, int64_t wait_limit_ns
  *   - Returns RAT_ERR_WORKSPACE when rat_decode_workspace_bytes(cache) exceeds 8 MiB (for d = 128
  *     that is roughly B * H * splits above 16,000).
  *   - The first call on each device looks up the array's device address (cudaGetSymbolAddress)
- *     with that device current; make that first call before any stream capture.
+ *     with that device current; make that first call before any stream capture.  The address
+ *     is kept per device index for the life of the process, in the primary context: it is not
+ *     looked up again after cudaDeviceReset, nor for a context the caller created itself, so
+ *     such callers must not use this entry point afterwards (or in that context).
  *   - Every call shares the one array, which keeps the previous call's contents; each call
  *     clears its header and tickets on `stream` first.  Calls that overlap on the GPU (other
  *     streams, other host threads) race on the array and must be serialised by the caller.

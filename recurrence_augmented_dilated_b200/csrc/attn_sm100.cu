@@ -39,8 +39,8 @@ __device__ unsigned g_attn_waiting; // bit s set: a wait at site s was in progre
 
 // (cos, sin)(l * theta_f) for l < 32 and the 64 RoPE frequencies, [f][l], formed on the host in
 // float64; the producer copies a launch's table next to Q.  kRelSlots tables per device, one per
-// distinct frequency set in use (replaced round-robin).
-constexpr int kRelSlots = 4;
+// distinct frequency set (RoPE base), each written once and never replaced.
+constexpr int kRelSlots = 16;
 __device__ float2 g_rope_rel[kRelSlots][64 * 32];
 
 namespace {
@@ -765,39 +765,53 @@ int launch_bn(const AttnSm100Args &a, const float2 *rel, void *stream) {
 
 int g_attn_block_keys = 0;   // 0: automatic; 64 or 128 forces the key-block width
 
-// The device table of a launch's RoPE frequencies: uploaded (stream-ordered) the first time a
-// frequency set is seen on this device, then reused.
+// The device table of a launch's RoPE frequencies.  The first call with a new frequency set
+// writes it into a free slot on a library stream and waits for that copy before the slot is
+// published, so a launch on any stream only ever reads a finished table; slots are never
+// overwritten (queued launches may read them at any time).  Beyond kRelSlots distinct sets the
+// call is refused (RAT_ERR_UNSUPPORTED), and a first use while `stream` is being captured is
+// refused too (the upload cannot be part of a graph).
 static int rope_rel_table(const double *theta, void *stream, const float2 **out) {
     struct Slot { double theta[64]; bool valid; };
     static std::mutex mu;
     static Slot slots[64][kRelSlots];
     static float2 *base[64];
-    static int next[64];
+    static cudaStream_t upload[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RAT_ERR_CUDA;
     std::lock_guard<std::mutex> lock(mu);
     if (!base[dev] && cudaGetSymbolAddress(reinterpret_cast<void **>(&base[dev]), g_rope_rel) != cudaSuccess)
         return RAT_ERR_CUDA;
+    int free_slot = -1;
     for (int i = 0; i < kRelSlots; ++i) {
-        if (slots[dev][i].valid && std::memcmp(slots[dev][i].theta, theta, sizeof(double) * 64) == 0) {
+        if (!slots[dev][i].valid) {
+            if (free_slot < 0) free_slot = i;
+            continue;
+        }
+        if (std::memcmp(slots[dev][i].theta, theta, sizeof(double) * 64) == 0) {
             *out = base[dev] + (size_t)i * 64 * 32;
             return RAT_OK;
         }
     }
-    const int i = next[dev];
-    next[dev] = (i + 1) % kRelSlots;
-    static float2 tab[64 * 32];      // guarded by mu; staged by the copy before it returns
+    if (free_slot < 0) return RAT_ERR_UNSUPPORTED;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cs) != cudaSuccess) return RAT_ERR_CUDA;
+    if (cs != cudaStreamCaptureStatusNone) return RAT_ERR_UNSUPPORTED;
+    if (!upload[dev] && cudaStreamCreateWithFlags(&upload[dev], cudaStreamNonBlocking) != cudaSuccess)
+        return RAT_ERR_CUDA;
+    static float2 tab[64 * 32];      // guarded by mu
     for (int f = 0; f < 64; ++f)
         for (int l = 0; l < 32; ++l) {
             const double ang = (double)l * theta[f];
             tab[f * 32 + l] = make_float2((float)std::cos(ang), (float)std::sin(ang));
         }
-    if (cudaMemcpyToSymbolAsync(g_rope_rel, tab, sizeof(tab), (size_t)i * sizeof(tab), cudaMemcpyHostToDevice,
-                                static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    if (cudaMemcpyToSymbolAsync(g_rope_rel, tab, sizeof(tab), (size_t)free_slot * sizeof(tab),
+                                cudaMemcpyHostToDevice, upload[dev]) != cudaSuccess ||
+        cudaStreamSynchronize(upload[dev]) != cudaSuccess)
         return RAT_ERR_CUDA;
-    std::memcpy(slots[dev][i].theta, theta, sizeof(double) * 64);
-    slots[dev][i].valid = true;
-    *out = base[dev] + (size_t)i * 64 * 32;
+    std::memcpy(slots[dev][free_slot].theta, theta, sizeof(double) * 64);
+    slots[dev][free_slot].valid = true;
+    *out = base[dev] + (size_t)free_slot * 64 * 32;
     return RAT_OK;
 }
 

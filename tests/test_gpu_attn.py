@@ -176,3 +176,30 @@ def test_repeated_launches_no_timeout_and_deterministic(name, block_keys):
     st = rat.rat_attn_sync_status()
     assert st == 0, hex(rat.lib().rat_attn_error_site())
     assert torch.equal(o, ref)
+
+
+def test_rope_tables_on_two_streams_without_host_syncs():
+    # six RoPE bases, first used inside launches interleaved over two streams with no host sync
+    # in between: each launch must read a finished table of its own base
+    B, H, T, d = 1, 2, 300, 128
+    bases = [500.0, 2500.0, 10000.0, 40000.0, 160000.0, 1.0e6]
+    q, k, v = qkv(B, H, T, d, torch.bfloat16, seed=91)
+    dev = torch.device("cuda")
+    qd, kd, vd = (x.to(dev) for x in (q, k, v))
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    for s in streams:
+        s.wait_stream(torch.cuda.current_stream())
+    outs = []
+    for rep in range(2):
+        for i, base in enumerate(bases):
+            s = streams[(i + rep) % 2]
+            o = torch.empty_like(qd)
+            with torch.cuda.stream(s):
+                rat.rat_dilated_attn_prefill(qd, kd, vd, o, D=8, W=4, rope_base=base, pos0=17,
+                                             stream=s)
+            outs.append((base, o))
+    torch.cuda.synchronize()
+    assert rat.rat_attn_sync_status() == 0
+    for base, o in outs:
+        ref = oracle.dilated_attention(oracle.rope(f64(q), 17, base), f64(k), f64(v), D=8, W=4)
+        assert rel_err(o, ref) <= TOL_BF16, base
