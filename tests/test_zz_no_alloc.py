@@ -30,18 +30,16 @@ def build_cache(w, T0, Tcap, rope_base):
     return cache, bufs
 
 
-@pytest.mark.parametrize("rope_base", [0.0, 10000.0])
-def test_noalloc_decode_matches_workspace_decode(rope_base):
-    w = synthetic.Workload("noalloc", B=2, H=3, d=128, T=0, W=8, D_per_head=(1, 4, 16),
-                           dtype="bf16", seed=77)
-    T0, steps = 150, 2
+def run_both(w, T0, steps, rope_base):
+    """steps decode calls in a row on each entry point over two copies of one cache; every
+    output and the caches they leave must agree."""
     ref_cache, ref_bufs = build_cache(w, T0, T0 + steps, rope_base)
     na_cache, na_bufs = build_cache(w, T0, T0 + steps, rope_base)
     ws = rat.Workspace(rat.rat_decode_workspace_bytes(ref_cache))
     tok = synthetic.decode_steps(w, steps)
     L = rat.lib()
     dev = torch.device("cuda")
-    for s in range(steps):          # two calls in a row on each entry point
+    for s in range(steps):
         args = [tok[n][s].reshape(w.B, w.H, 1, w.d).to(dev) for n in ("q", "k", "v", "a")]
         o_ref = torch.empty((w.B, w.H, 1, w.d), dtype=torch.bfloat16, device=dev)
         o_na = torch.full_like(o_ref, float("nan"))
@@ -57,6 +55,19 @@ def test_noalloc_decode_matches_workspace_decode(rope_base):
     assert na_cache.pos == ref_cache.pos == T0 + steps
     for n in ("h_k", "h_v", "k_dil", "v_dil", "k_win", "v_win"):
         assert rel_err(na_bufs[n], ref_bufs[n]) <= TOL_BF16, n
+
+
+@pytest.mark.parametrize("rope_base", [0.0, 10000.0])
+def test_noalloc_decode_matches_workspace_decode(rope_base):
+    # first a call over many slices and long contexts (many splits: the array fills far beyond
+    # what the next calls use), then two calls in a row on a small cache: stale partials and
+    # tickets of the large call must not leak into the small ones
+    big = synthetic.Workload("noalloc_big", B=8, H=16, d=128, T=0, W=8,
+                             D_per_head=tuple([1, 4] * 8), dtype="bf16", seed=78)
+    run_both(big, 4096, 1, rope_base)
+    w = synthetic.Workload("noalloc", B=2, H=3, d=128, T=0, W=8, D_per_head=(1, 4, 16),
+                           dtype="bf16", seed=77)
+    run_both(w, 150, 2, rope_base)
 
 
 def test_noalloc_rejects_oversized_scratch():
