@@ -765,8 +765,10 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     pairs = sum(rat.rat_attended_keys(t, D_, w.W) for D_ in w.heads_D() for t in range(T)) * B
     aflops = 10 * d * pairs                 # per pair: recomputed score, dp, dq, dk, dv
     a_ach = abytes / (ams * 1e-3) / 1e9
-    res["attention"] = {"step": "rat_dilated_attn_backward (3 CUDA-core launches, the forward's "
-                                "log-sum-exp given)", "ms": ams,
+    tc_path = w.dtype == "bf16" and w.d == 128
+    res["attention"] = {"step": "rat_dilated_attn_backward (%s, the forward's log-sum-exp given)" % (
+                            "prep on CUDA cores, dq and dk/dv launches on tcgen05 tensor cores"
+                            if tc_path else "3 CUDA-core launches"), "ms": ams,
                         "roofline": {"bound": "hbm", "achieved": a_ach, "peak": peaks["hbm_gbs"],
                                      "unit": "GB/s", "frac": a_ach / peaks["hbm_gbs"],
                                      "of": peak_kind, "algorithmic_bytes": abytes,

@@ -18,6 +18,8 @@
 // Each (query, key) pair is recomputed in both gradient launches; p comes from the stored
 // denominator, so the two launches agree.  This is the plain CUDA-core path of the backward:
 // dot products are warp reductions, four rows' loads in flight per warp.
+#include <cstring>
+
 #include "common.cuh"
 
 namespace rat {
@@ -244,8 +246,34 @@ static int launch_bwd(const AttnBwdParams &p, cudaStream_t s) {
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 
+// Tensor-core form: the prep kernel (q^, Delta), the forward's log-sum-exp when it was not
+// given (the forward attention runs once with its output in dq, which the dq launch then
+// overwrites), then the dq and dk/dv launches.
+static int launch_bwd_tc(const AttnBwdParams &p, cudaStream_t s) {
+    dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)(p.B * p.H));
+    attn_bwd_prep_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return RAT_ERR_CUDA;
+    if (!p.lse_given) {
+        AttnSm100Args a;
+        std::memset(&a, 0, sizeof(a));
+        a.q = p.q; a.k = p.k; a.v = p.v; a.o = p.dq;
+        a.B = p.B; a.H = p.H; a.T = p.T; a.d = p.d; a.W = p.W;
+        a.pos0 = p.pos0;
+        a.rope = p.rope;
+        a.scale_log2 = p.scale_log2;
+        a.Dh = p.Dh;
+        a.n_sink = 0;
+        a.lse = p.lse;
+        for (int c = 0; c < 64; ++c) a.theta[c] = p.theta[c];
+        const int st = launch_attn_sm100(a, s);
+        if (st != RAT_OK) return st;
+    }
+    return launch_attn_bwd_sm100(p, s);
+}
+
 int launch_attn_bwd(const AttnBwdParams &p, int dtype, void *stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (attn_bwd_sm100_supported(p, dtype)) return launch_bwd_tc(p, s);
     if (dtype == RAT_F32) {
         if (p.d == 64) return launch_bwd<float, 64>(p, s);
         if (p.d == 128) return launch_bwd<float, 128>(p, s);

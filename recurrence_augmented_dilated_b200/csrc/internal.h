@@ -186,9 +186,13 @@ struct AttnBwdParams {
     float scale, scale_log2;
     int Dh[kMaxHeads];
     double theta[64];
+    WsHeader *hdr;              // workspace header: device-side errors of the tensor-core kernels
 };
 size_t attn_bwd_workspace_bytes(int B, int H, int T, int d, int dtype);
 int launch_attn_bwd(const AttnBwdParams &p, int dtype, void *stream);
+// tensor-core form (bf16, d = 128, no sinks, at most four dilations > 1 in a launch)
+bool attn_bwd_sm100_supported(const AttnBwdParams &p, int dtype);
+int launch_attn_bwd_sm100(const AttnBwdParams &p, void *stream);
 
 struct DecodeParams {
     const void *q, *k, *v, *a;

@@ -421,6 +421,7 @@ int rat_dilated_attn_backward(const void *q, const void *k_rec, const void *v_re
     p.q = q; p.k = k_rec; p.v = v_rec; p.o = o; p.dO = dO;
     p.dq = dq; p.dk = dk_rec; p.dv = dv_rec;
     const size_t rows = (size_t)B * H * T;
+    p.hdr = static_cast<WsHeader *>(ws);
     uint8_t *w = static_cast<uint8_t *>(ws) + sizeof(WsHeader);
     p.qh = w;
     w += align256(rows * d * (dtype == RAT_F32 ? 4 : 2));

@@ -94,7 +94,20 @@ def test_recorded_traffic_follows_the_source_hash():
     assert bench.recorded_traffic("scan.cu", "no_such_workload") is None
 
 
-def test_recorded_traffic_void_after_a_header_change(monkeypatch):
-    assert bench.recorded_traffic("scan.cu", "prefill_1p5b") is not None
+def test_recorded_traffic_void_after_a_header_change(monkeypatch, tmp_path):
+    # a table entry taken on the current sources, in a copy of the tree: valid until a shared
+    # device header changes
+    import shutil
+    csrc = tmp_path / "recurrence_augmented_dilated_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    src = os.path.join(bench.ROOT, "recurrence_augmented_dilated_b200", "csrc")
+    for n in ("scan.cu",) + bench.KERNEL_HEADERS:
+        shutil.copy(os.path.join(src, n), csrc / n)
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    entry = {"dram_bytes_per_launch": 123, "source_sha": bench.file_sha(str(csrc / "scan.cu")),
+             "capture": "x.md", "headers_sha": bench.headers_sha()}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps({"scan.cu": {"w": entry}}))
+    assert bench.recorded_traffic("scan.cu", "w") == 123
     monkeypatch.setattr(bench, "headers_sha", lambda: "0000000000000000")
-    assert bench.recorded_traffic("scan.cu", "prefill_1p5b") is None
+    assert bench.recorded_traffic("scan.cu", "w") is None

@@ -100,3 +100,66 @@ def test_forward_lse_and_backward_with_it(dtype, d):
     for got in outs:
         for gg, r in zip(got, ref_b):
             assert rel_err(gg, r) <= tol_for(dtype)
+
+
+# bf16, d 128 without sinks runs on the tensor cores (dq and dk/dv launches): several query tiles
+# and key blocks with ragged tails, every key-set shape (dense, chunk ends only, chunk ends plus
+# a wide window, no chunk end inside the sequence, self key only), RoPE at an offset
+@pytest.mark.parametrize("T", [63, 64, 130, 1000])
+@pytest.mark.parametrize("D,W", [(1, 0), (3, 0), (8, 100), (600, 0), (16, 1)])
+def test_attention_backward_tensor_core_tiles(T, D, W):
+    run(1, 2, T, 128, torch.bfloat16, D=D, W=W, seed=T + D + W, rope_base=10000.0, pos0=7)
+
+
+def test_attention_backward_head_hybrid_lse_given():
+    # a dense head and four dilations in one launch, the forward's log-sum-exp passed in
+    B, H, T, d = 2, 6, 700, 128
+    Dh = [1, 2, 5, 64, 300, 1]
+    w = synthetic.Workload("hy", B=B, H=H, d=d, T=T, dtype="bf16", seed=31)
+    x = synthetic.prefill_inputs(w)
+    dev = torch.device("cuda")
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, T), dtype=torch.float32, device=dev)
+    rat.rat_dilated_attn_prefill(q, k, v, o, D_per_head=Dh, W=4, rope_base=500.0, lse=lse)
+    g = torch.Generator().manual_seed(32)
+    dO = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = rat.Workspace(rat.rat_dilated_attn_backward_workspace_bytes(B, H, T, d, 1))
+    rat.rat_dilated_attn_backward(q, k, v, o, dO.to(dev), dq, dk, dv, ws, D_per_head=Dh, W=4,
+                                  rope_base=500.0, lse=lse)
+    assert rat.rat_sync_status(ws) == 0
+    ref = oracle.dilated_attention_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(dO),
+                                            W=4, D_per_head=Dh, rope_base=500.0)
+    for got, r in zip((dq, dk, dv), ref):
+        assert rel_err(got, r) <= TOL_BF16
+
+
+def test_attention_backward_five_dilations_take_the_cuda_core_path():
+    # more than four distinct dilations in one call: the CUDA-core kernels, same results (the
+    # bf16 forward takes at most four, so o comes from the oracle, rounded to bf16)
+    B, H, T, d = 1, 5, 200, 128
+    Dh = [2, 3, 4, 5, 6]
+    w = synthetic.Workload("d5", B=B, H=H, d=d, T=T, dtype="bf16", seed=41)
+    x = synthetic.prefill_inputs(w)
+    dev = torch.device("cuda")
+    q, k, v = (x[n].to(dev) for n in ("q", "k", "v"))
+    o = torch.from_numpy(oracle.dilated_attention(f64(x["q"]), f64(x["k"]), f64(x["v"]), W=2,
+                                                  D_per_head=Dh)).to(torch.bfloat16).to(dev)
+    g = torch.Generator().manual_seed(42)
+    dO = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = rat.Workspace(rat.rat_dilated_attn_backward_workspace_bytes(B, H, T, d, 1))
+    rat.rat_dilated_attn_backward(q, k, v, o, dO.to(dev), dq, dk, dv, ws, D_per_head=Dh, W=2)
+    assert rat.rat_sync_status(ws) == 0
+    ref = oracle.dilated_attention_backward(f64(x["q"]), f64(x["k"]), f64(x["v"]), f64(dO), W=2,
+                                            D_per_head=Dh)
+    for got, r in zip((dq, dk, dv), ref):
+        assert rel_err(got, r) <= TOL_BF16
+
+
+def test_attention_backward_window_2p6b_sampled_heads():
+    # the window_2p6b workload (B 2, H 20, T 16384, D 64, W 128) at full size, two heads checked
+    w = synthetic.WORKLOADS["window_2p6b"]
+    x = synthetic.prefill_inputs(w)
+    run(w.B, w.H, w.T, w.d, torch.bfloat16, D=w.D, W=w.W, x=x, heads=[(0, 3), (1, 19)], seed=6)
