@@ -66,6 +66,10 @@ struct Cfg {
     // carveout, which leaves the rest of the SM's 256 KiB to L1
     static constexpr uint32_t OFF_BAR = OFF_V + NS * KTILE;
     static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
+    // top-k variant: a bitmap of the key blocks that hold some row's selected chunks
+    static constexpr uint32_t OFF_MAP = OFF_BAR + 256;
+    static constexpr uint32_t MAP_WORDS = 64;           // 2048 blocks: positions below 131072
+    static constexpr uint32_t SMEM_TOPK = OFF_MAP + MAP_WORDS * 4;
     static constexpr uint32_t COL_S1 = BN;              // S buffers at columns 0 and BN; the bf16
                                                         // P of a block overwrites the first BN/2
                                                         // columns of its S buffer
@@ -96,6 +100,7 @@ struct Params {
     int grp_nheads[kMaxHeads];
     int rope_f32;             // positions small enough for float32 angles (pos0 + T <= 2^13)
     int n_sink;               // attention sinks (n_sink < D of every dilated head, <= BN)
+    int top_k;                // top-k variant: chunks selected per row (1 .. 16)
     float *lse;               // [B*H][T] or null: log2 of each row's softmax denominator
     const float2 *rope_rel;   // device table [64 f][32 l] of (cos, sin)(l theta_f), see g_rope_rel
     float theta_f[64];
@@ -114,12 +119,12 @@ struct Plan {
     bool self_reg;    // We == 1 (dilated head): the self key is handled in registers, no window blocks
 };
 template <int BN>
-RAT_DEVICE Plan make_plan(int t0, int D, int W, int T, int n_sink) {
+RAT_DEVICE Plan make_plan(int t0, int D, int W, int T, int n_sink, bool regs_self = true) {
     Plan pl;
     pl.D = D;
     pl.We = W > 1 ? W : 1;
     pl.dense = D == 1;
-    pl.self_reg = !pl.dense && pl.We == 1;
+    pl.self_reg = regs_self && !pl.dense && pl.We == 1;
     pl.n_sink = n_sink;
     const int tmax = t0 + BM - 1;
     // a sink block when some query of the tile has a sink older than its window
@@ -164,6 +169,7 @@ struct Shared {
     // K and V of a stage have separate lifetimes: K is free once S has read it, V once PV has
     uint64_t q_full, q_ready, k_full[NS], v_full[NS], k_empty[NS], v_empty[NS];
     uint64_t s_full[2], p_full[2], o_ready[2], fin;
+    uint64_t sel_free[2], sel_ready;   // top-k variant: selection scores read, selection published
     uint32_t tmem;
     volatile int abort;
 };
@@ -207,13 +213,39 @@ RAT_DEVICE void rope_cs_fast(long long pos, double theta, float &c, float &s) {
     __sincosf((float)r, &s, &c);
 }
 
+// Index of the n-th (0-based) set bit of a bitmap of `words` 32-bit words; -1 if there is none.
+RAT_DEVICE int nth_set(const uint32_t *bm, int words, int n) {
+    for (int w = 0; w < words; ++w) {
+        uint32_t x = bm[w];
+        const int c = __popc(x);
+        if (n < c) {
+            for (; n > 0; --n) x &= x - 1;
+            return 32 * w + __ffs(x) - 1;
+        }
+        n -= c;
+    }
+    return -1;
+}
+RAT_DEVICE int count_set(const uint32_t *bm, int words) {
+    int n = 0;
+    for (int w = 0; w < words; ++w) n += __popc(bm[w]);
+    return n;
+}
+
 RAT_DEVICE uint32_t swz(uint32_t row, uint32_t chunk) {   // 128B swizzle inside a sub-tile
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
 }
 
 // SELF: the launch may have heads whose self key is kept in registers (W <= 1); launches with a
 // window (W > 1) compile without that code.
-template <int BN, bool SELF>
+// TOPK: top-k chunk selection combined with dilation ("RAT+ Deep Dive" section 4).  A selection
+// phase first runs S over the chunk-end blocks alone; each row keeps its 16 best chunks (by
+// chunk-end score, ties to the earlier chunk) in registers, and the 64-key blocks holding the
+// positions of every row's top_k chunks are marked in a shared bitmap.  The main loop then
+// visits, between the chunk-end and the window blocks, each marked block once, each row keeping
+// the columns of its own selected chunks (their chunk ends are keys already).  The self key
+// stays in the window blocks.
+template <int BN, bool SELF, bool TOPK = false>
 __global__ void __launch_bounds__(kThreads, Cfg<BN>::MIN_CTAS)
 attn_sm100_kernel(const __grid_constant__ Params p) {
     using C = Cfg<BN>;
@@ -238,9 +270,11 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
     const int b = (local % per_row) / p.grp_nheads[g];
     const int h = p.head_of[p.grp_head0[g] + (local % per_row) % p.grp_nheads[g]];
     const int bh = b * p.H + h;
-    const Plan pl = make_plan<BN>(t0, p.Dh[h], p.W, p.T, p.n_sink);
+    const Plan pl = make_plan<BN>(t0, p.Dh[h], p.W, p.T, p.n_sink, !TOPK);
     const bool self_reg = SELF && pl.self_reg;      // pl.self_reg implies W <= 1, hence SELF
-    const int nb = pl.ns + pl.nd + pl.nw;
+    const int nb = pl.ns + pl.nd + pl.nw;           // (+ the selected blocks, top-k variant)
+    const int nsel = TOPK ? pl.nd : 0;              // blocks of the selection phase
+    uint32_t *bmap = reinterpret_cast<uint32_t *>(smem + Cfg<BN>::OFF_MAP);
 
     if (threadIdx.x == 0) {
         mbar_init(&sh.q_full, 1);
@@ -259,6 +293,12 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         mbar_init(&sh.o_ready[0], 1);     // PV of even blocks
         mbar_init(&sh.o_ready[1], 1);     // PV of odd blocks
         mbar_init(&sh.fin, 1);
+        if (TOPK) {
+            mbar_init(&sh.sel_free[0], 128);
+            mbar_init(&sh.sel_free[1], 128);
+            mbar_init(&sh.sel_ready, 128);
+            for (uint32_t w = 0; w < C::MAP_WORDS; ++w) bmap[w] = 0u;
+        }
         sh.abort = 0;
         fence_mbar_init();
     }
@@ -285,25 +325,49 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             // stage frees up as soon as its S has completed
             // first key row of block j: the sinks at row 0, a dilated block in the compressed
             // view, a window block in the plain one
+            // (top-k variant: the ntk selected blocks sit between the chunk-end and the window
+            // blocks; they are known once the selection is published)
+            int ntk = 0;
             auto row_of = [&](int j) {
                 if (j < pl.ns) return 0;
                 j -= pl.ns;
-                return j < pl.nd ? BN * j : pl.ws + BN * (j - pl.nd);
+                if (j < pl.nd) return BN * j;
+                j -= pl.nd;
+                if (TOPK && j < ntk) return BN * nth_set(bmap, C::MAP_WORDS, j);
+                return pl.ws + BN * (j - ntk);
             };
             auto dil_blk = [&](int j) { return j >= pl.ns && j - pl.ns < pl.nd; };
+            // K loads are counted over both phases (g), V loads over the main loop only (j)
             int k_issued = 0, v_issued = 0;
-            for (int j = 0; j <= nb; ++j) {
-                if (j < nb) {
-                    const int s = j % NS;
-                    if (j >= NS && !wait_bar(sh, &sh.k_empty[s], ((j / NS) - 1) & 1, 1, j)) break;
-                    // with RoPE, stage 1 holds the softmax warps' rotation tables until Q is rotated
-                    if (j == 1 && p.rope && !wait_bar(sh, &sh.q_ready, 0, 10, j)) break;
-                    const CUtensorMap *tk = dil_blk(j) ? mk : &p.tm_k;
+            bool go = true;
+            if constexpr (TOPK) {
+                for (int g = 0; g < nsel; ++g) {          // selection phase: chunk-end K blocks
+                    const int s = g % NS;
+                    if (g >= NS && !wait_bar(sh, &sh.k_empty[s], ((g / NS) - 1) & 1, 1, g)) { go = false; break; }
+                    if (g == 1 && p.rope && !wait_bar(sh, &sh.q_ready, 0, 10, g)) { go = false; break; }
                     uint8_t *ks = smem + C::OFF_K + s * C::KTILE;
                     mbar_arrive_expect_tx(&sh.k_full[s], C::KTILE);
-                    tc::tma_load_3d(ks, tk, 0, row_of(j), bh, &sh.k_full[s]);
-                    tc::tma_load_3d(ks + C::KSUB, tk, 64, row_of(j), bh, &sh.k_full[s]);
-                    k_issued = j + 1;
+                    tc::tma_load_3d(ks, mk, 0, BN * g, bh, &sh.k_full[s]);
+                    tc::tma_load_3d(ks + C::KSUB, mk, 64, BN * g, bh, &sh.k_full[s]);
+                    k_issued = g + 1;
+                }
+                if (go && !wait_bar(sh, &sh.sel_ready, 0, 13, 0)) go = false;
+                if (go) ntk = count_set(bmap, C::MAP_WORDS);
+            }
+            const int nbt = nb + ntk;
+            for (int j = 0; go && j <= nbt; ++j) {
+                if (j < nbt) {
+                    const int g = nsel + j, s = g % NS;
+                    if (g >= NS && !wait_bar(sh, &sh.k_empty[s], ((g / NS) - 1) & 1, 1, j)) break;
+                    // with RoPE, stage 1 holds the softmax warps' rotation tables until Q is rotated
+                    if (g == 1 && p.rope && !wait_bar(sh, &sh.q_ready, 0, 10, j)) break;
+                    const CUtensorMap *tk = dil_blk(j) ? mk : &p.tm_k;
+                    uint8_t *ks = smem + C::OFF_K + s * C::KTILE;
+                    const int row = row_of(j);
+                    mbar_arrive_expect_tx(&sh.k_full[s], C::KTILE);
+                    tc::tma_load_3d(ks, tk, 0, row, bh, &sh.k_full[s]);
+                    tc::tma_load_3d(ks + C::KSUB, tk, 64, row, bh, &sh.k_full[s]);
+                    k_issued = g + 1;
                 }
                 if (j >= 1) {
                     const int jv = j - 1, s = jv % NS;
@@ -318,7 +382,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             }
             if (sh.abort) {
                 // let this CTA's own loads land before its shared memory goes away
-                for (int j = max(0, k_issued - NS); j < k_issued; ++j) wait_drain(&sh.k_full[j % NS], (j / NS) & 1);
+                for (int g = max(0, k_issued - NS); g < k_issued; ++g) wait_drain(&sh.k_full[g % NS], (g / NS) & 1);
                 for (int j = max(0, v_issued - NS); j < v_issued; ++j) wait_drain(&sh.v_full[j % NS], (j / NS) & 1);
                 wait_drain(&sh.q_full, 0);
             }
@@ -330,26 +394,45 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             constexpr uint32_t IDESC_QK = tc::idesc_bf16(BM, BN, 0);      // K^T: K-major B
             constexpr uint32_t IDESC_PV = tc::idesc_bf16(BM, DHEAD, 1);   // V: MN-major B
             const uint32_t sq = smem_u32(smem + C::OFF_Q);
+            // S(g) = Q K(g)^T into S buffer g & 1, from K stage g % NS
+            auto issue_s = [&](int g) {
+                const int s = g % NS, sb = g & 1;
+                const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::KTILE);
+                for (int kk = 0; kk < DHEAD / 16; ++kk) {
+                    // 16 channels of Q (A, K-major) and of K (B, K-major): d-half kk/4, +32 B per step
+                    const uint32_t qoff = (kk >> 2) * QSUB + (kk & 3) * 32;
+                    const uint32_t koff = (kk >> 2) * C::KSUB + (kk & 3) * 32;
+                    tc::mma_bf16_ss(tmem + sb * C::COL_S1, tc::smem_desc_sw128(sq + qoff, 16, 1024),
+                                    tc::smem_desc_sw128(sk + koff, 16, 1024), IDESC_QK, kk > 0);
+                }
+                tc::mma_commit(&sh.s_full[sb]);
+                tc::mma_commit(&sh.k_empty[s]);
+            };
             bool ok = wait_bar(sh, &sh.q_ready, 0, 2);
             tc::fence_after_sync();
-            for (int j = 0; ok && j <= nb; ++j) {
-                if (j < nb) {
-                    const int s = j % NS, sb = j & 1;
-                    if (!wait_bar(sh, &sh.k_full[s], (j / NS) & 1, 3, j)) break;
-                    // S buffer sb holds P(j-2) until PV(j-2) has read it: wait for that PV to
+            int ntk = 0;
+            if constexpr (TOPK) {
+                for (int g = 0; ok && g < nsel; ++g) {        // selection phase: S only
+                    if (!wait_bar(sh, &sh.k_full[g % NS], (g / NS) & 1, 3, g)) { ok = false; break; }
+                    // S buffer g & 1 is free once the softmax warps have read S(g-2)
+                    if (g >= 2 && !wait_bar(sh, &sh.sel_free[g & 1], ((g - 2) >> 1) & 1, 14, g)) { ok = false; break; }
+                    tc::fence_after_sync();
+                    issue_s(g);
+                }
+                // every selection-phase S has been read once the selection is published
+                if (ok) ok = wait_bar(sh, &sh.sel_ready, 0, 13);
+                if (ok) ntk = count_set(bmap, C::MAP_WORDS);
+            }
+            const int nbt = nb + ntk;
+            for (int j = 0; ok && j <= nbt; ++j) {
+                if (j < nbt) {
+                    const int g = nsel + j;
+                    if (!wait_bar(sh, &sh.k_full[g % NS], (g / NS) & 1, 3, j)) break;
+                    // S buffer g & 1 holds P(j-2) until PV(j-2) has read it: wait for that PV to
                     // complete (this thread issued it, so the barrier is at most one phase ahead)
                     if (j >= 2 && !wait_bar(sh, &sh.o_ready[(j - 2) & 1], ((j - 2) >> 1) & 1, 4, j)) break;
                     tc::fence_after_sync();
-                    const uint32_t sk = smem_u32(smem + C::OFF_K + s * C::KTILE);
-                    for (int kk = 0; kk < DHEAD / 16; ++kk) {
-                        // 16 channels of Q (A, K-major) and of K (B, K-major): d-half kk/4, +32 B per step
-                        const uint32_t qoff = (kk >> 2) * QSUB + (kk & 3) * 32;
-                        const uint32_t koff = (kk >> 2) * C::KSUB + (kk & 3) * 32;
-                        tc::mma_bf16_ss(tmem + sb * C::COL_S1, tc::smem_desc_sw128(sq + qoff, 16, 1024),
-                                        tc::smem_desc_sw128(sk + koff, 16, 1024), IDESC_QK, kk > 0);
-                    }
-                    tc::mma_commit(&sh.s_full[sb]);
-                    tc::mma_commit(&sh.k_empty[s]);
+                    issue_s(g);
                 }
                 if (j >= 1) {
                     const int jp = j - 1, s = jp % NS;
@@ -357,7 +440,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
                     if (!wait_bar(sh, &sh.v_full[s], (jp / NS) & 1, 12, jp)) break;
                     tc::fence_after_sync();
                     const uint32_t sv = smem_u32(smem + C::OFF_V + s * C::KTILE);
-                    const uint32_t pcol = (jp & 1) * C::COL_S1;     // P of block jp, in TMEM
+                    const uint32_t pcol = ((nsel + jp) & 1) * C::COL_S1;     // P of block jp, in TMEM
                     for (int kk = 0; kk < BN / 16; ++kk) {
                         // A = P[:, 16kk .. 16kk+15]: 8 TMEM columns of packed bf16 pairs
                         // B = V[16kk .. 16kk+15, :]  (MN-major: the two 64-channel atoms KSUB apart,
@@ -487,26 +570,95 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             w_self = 1.f;
         }
         float sv[BN];
+        // top-k variant: this row's selected chunks (indices, -1: none), best first
+        int sel[TOPK ? 16 : 1];
+        int ntk = 0;
+        if constexpr (TOPK) {
+            float best[16];
+#pragma unroll
+            for (int q = 0; q < 16; ++q) { best[q] = -INFINITY; sel[q] = -1; }
+            for (int g = 0; ok && g < nsel; ++g) {
+                const int sb = g & 1;
+                if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.s_full[sb], (g >> 1) & 1, 15, g))) { ok = false; break; }
+                tc::fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < BN / 32; ++c)
+                    tc::tmem_ld32(tl + sb * C::COL_S1 + 32 * c, reinterpret_cast<uint32_t *>(sv) + 32 * c);
+                tc::tmem_wait_ld();
+                tc::fence_before_sync();
+                mbar_arrive(&sh.sel_free[sb]);
+                // candidate chunk i = BN g + c: wholly older than the window (its end <= t - We);
+                // kept sorted, best first; an equal score does not displace an earlier chunk
+                int c_lo, c_hi;
+                block_range<BN>(pl, pl.ns + g, t, c_lo, c_hi);
+                if (t >= p.T) c_hi = -1;
+#pragma unroll
+                for (int c = 0; c < BN; ++c) {
+                    float v = sv[c];
+                    if (c > c_hi || !(v > best[15])) continue;
+                    int id = BN * g + c;
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) {
+                        if (v > best[q]) {
+                            const float tv = best[q];
+                            const int ti = sel[q];
+                            best[q] = v;
+                            sel[q] = id;
+                            v = tv;
+                            id = ti;
+                        }
+                    }
+                }
+            }
+            // the key blocks holding the positions (below each chunk end) of the row's top_k chunks
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                if (q >= p.top_k) sel[q] = -1;
+                if (sel[q] >= 0) {
+                    const int b0 = sel[q] * pl.D / BN, b1 = (sel[q] * pl.D + pl.D - 2) / BN;
+                    for (int b = b0; b <= b1; ++b) atomicOr(&bmap[b >> 5], 1u << (b & 31));
+                }
+            }
+            mbar_arrive(&sh.sel_ready);
+            if (ok) ok = __all_sync(0xffffffffu, wait_bar(sh, &sh.sel_ready, 0, 13));
+            if (ok) ntk = count_set(bmap, C::MAP_WORDS);
+        }
+        const int nbt = nb + ntk;
+        const int ndil = pl.ns + pl.nd;          // blocks before the selected ones
         int jdone = 0;
-        for (int j = 0; ok && j < nb; ++j) {
-            const int sb = j & 1;
-            if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.s_full[sb], (j >> 1) & 1, 7, j))) { ok = false; break; }
+        for (int j = 0; ok && j < nbt; ++j) {
+            const int sb = (nsel + j) & 1;
+            if (!__all_sync(0xffffffffu, wait_bar(sh, &sh.s_full[sb], ((nsel + j) >> 1) & 1, 7, j))) { ok = false; break; }
             tc::fence_after_sync();
 #pragma unroll
             for (int c = 0; c < BN / 32; ++c)
                 tc::tmem_ld32(tl + sb * C::COL_S1 + 32 * c, reinterpret_cast<uint32_t *>(sv) + 32 * c);
             tc::tmem_wait_ld();
 
-            int c_lo, c_hi;
-            block_range<BN>(pl, j, t, c_lo, c_hi);
             // row max of the raw scores (scale > 0 commutes with max), as an 8-way tree; keys
             // outside S(t) become -inf (only blocks that cut the key set need the mask)
             float m8[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) m8[u] = -INFINITY;
-            if (!(c_lo <= 0 && c_hi >= BN - 1)) {
+            if (TOPK && j >= ndil && j < ndil + ntk) {
+                // a selected block: the columns inside this row's selected chunks, ends excluded
+                const int base = BN * nth_set(bmap, C::MAP_WORDS, j - ndil);
+                unsigned long long keep = 0ull;
 #pragma unroll
-                for (int c = 0; c < BN; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
+                for (int q = 0; q < (TOPK ? 16 : 1); ++q) {
+                    if (sel[q] < 0) continue;
+                    const int lo = max(sel[q] * pl.D, base), hi = min(sel[q] * pl.D + pl.D - 2, base + BN - 1);
+                    if (lo <= hi) keep |= ((~0ull) >> (63 - (hi - lo))) << (lo - base);
+                }
+#pragma unroll
+                for (int c = 0; c < BN; ++c) sv[c] = (keep >> c) & 1ull ? sv[c] : -INFINITY;
+            } else {
+                int c_lo, c_hi;
+                block_range<BN>(pl, j >= ndil + ntk ? j - ntk : j, t, c_lo, c_hi);
+                if (!(c_lo <= 0 && c_hi >= BN - 1)) {
+#pragma unroll
+                    for (int c = 0; c < BN; ++c) sv[c] = (c >= c_lo && c <= c_hi) ? sv[c] : -INFINITY;
+                }
             }
 #pragma unroll
             for (int c = 0; c < BN; c += 2) m8[(c >> 1) & 7] = fmax3(m8[(c >> 1) & 7], sv[c], sv[c + 1]);
@@ -569,11 +721,11 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         }
         // ---- epilogue: (O + w_self v~_t) / l -> bf16 rows in the Q buffer (every S MMA, the only
         // reader of Q, has completed) -> TMA stores of this warp's 32 rows
-        bool have_o = ok && jdone == nb;
+        bool have_o = ok && jdone == nbt;
         uint4 vrow[16];           // v~ of the tile's rows (own array: keeps the k~ rows dead here)
         if (have_o && self_reg) load_rows(p.vg, vrow);      // in flight during the last PV
-        if (have_o && nb > 0)
-            have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready[(nb - 1) & 1], ((nb - 1) >> 1) & 1, 9, nb));
+        if (have_o && nbt > 0)
+            have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready[(nbt - 1) & 1], ((nbt - 1) >> 1) & 1, 9, nbt));
         if (have_o) {
             if (self_reg) {     // stage the self values in this warp's rows, 128B-swizzled
 #pragma unroll
@@ -588,7 +740,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
-                if (nb > 0) {
+                if (nbt > 0) {
                     tc::tmem_ld32(tl + C::COL_O + 32 * c, o);
                     tc::tmem_wait_ld();
                 } else {
@@ -731,6 +883,7 @@ int fill_params(Params &p, const AttnSm100Args &a) {
     p.rope = a.rope;
     p.rope_f32 = a.pos0 + (long long)a.T <= 8192 ? 1 : 0;
     p.n_sink = a.n_sink;
+    p.top_k = a.top_k;
     p.lse = a.lse;
     p.scale_log2 = a.scale_log2;
     for (int c = 0; c < 64; ++c) {
@@ -741,13 +894,14 @@ int fill_params(Params &p, const AttnSm100Args &a) {
     return items;
 }
 
-template <int BN, bool SELF>
+template <int BN, bool SELF, bool TOPK = false>
 int launch_tiles(const Params &p, int items, void *stream) {
     using C = Cfg<BN>;
+    constexpr uint32_t smem = TOPK ? C::SMEM_TOPK : C::SMEM_BYTES;
     static std::atomic<uint64_t> attr_done{0};
-    const int st = set_smem_attr(reinterpret_cast<const void *>(attn_sm100_kernel<BN, SELF>), C::SMEM_BYTES, &attr_done);
+    const int st = set_smem_attr(reinterpret_cast<const void *>(attn_sm100_kernel<BN, SELF, TOPK>), smem, &attr_done);
     if (st != RAT_OK) return st;
-    attn_sm100_kernel<BN, SELF><<<(unsigned)items, kThreads, C::SMEM_BYTES, static_cast<cudaStream_t>(stream)>>>(p);
+    attn_sm100_kernel<BN, SELF, TOPK><<<(unsigned)items, kThreads, smem, static_cast<cudaStream_t>(stream)>>>(p);
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 
@@ -757,6 +911,9 @@ int launch_bn(const AttnSm100Args &a, const float2 *rel, void *stream) {
     const int items = fill_params<BN>(p, a);
     if (items < 0) return items;
     p.rope_rel = rel;
+    if constexpr (BN == 64) {
+        if (a.top_k > 0) return launch_tiles<BN, false, true>(p, items, stream);
+    }
     return a.W <= 1 ? launch_tiles<BN, true>(p, items, stream) : launch_tiles<BN, false>(p, items, stream);
 }
 
@@ -822,7 +979,8 @@ int launch_attn_sm100(const AttnSm100Args &a, void *stream) {
         const int st = rope_rel_table(a.theta, stream, &rel);
         if (st != RAT_OK) return st;
     }
-    const int bn = g_attn_block_keys ? g_attn_block_keys : 64;
+    // (the top-k variant runs on 64-key blocks)
+    const int bn = a.top_k > 0 ? 64 : g_attn_block_keys ? g_attn_block_keys : 64;
     return bn == 64 ? launch_bn<64>(a, rel, stream) : launch_bn<128>(a, rel, stream);
 }
 

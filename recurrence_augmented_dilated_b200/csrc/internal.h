@@ -116,6 +116,7 @@ struct AttnSm100Args {
     float scale_log2;
     const int32_t *Dh;          // host [H]
     int n_sink;                 // attention sinks; the caller ensures n_sink < D (D > 1) and <= 64
+    int top_k;                  // > 0: top-k chunk selection (then n_sink == 0, T <= 65536)
     float *lse;                 // [B*H][T] or null: log2 of each row's softmax denominator
     double theta[64];
 };

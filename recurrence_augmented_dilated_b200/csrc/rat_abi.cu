@@ -323,7 +323,10 @@ int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, i
     bool sinks_fit = n_sink <= 64;
     for (int h = 0; h < H; ++h)
         if (Dh[h] > 1 && Dh[h] <= n_sink) sinks_fit = false;
-    if (dtype == RAT_BF16 && d == 128 && top_k == 0 && (n_sink == 0 || sinks_fit)) {
+    // top-k chunk selection runs there too when there are no sinks and the sequence's 64-key
+    // blocks fit the kernel's block bitmap
+    const bool topk_fits = top_k == 0 || (n_sink == 0 && T <= 65536);
+    if (dtype == RAT_BF16 && d == 128 && topk_fits && (n_sink == 0 || sinks_fit)) {
         AttnSm100Args a;
         std::memset(&a, 0, sizeof(a));
         a.q = q; a.k = k_rec; a.v = v_rec; a.o = o;
@@ -333,6 +336,7 @@ int attn_prefill(const void *q, const void *k_rec, const void *v_rec, void *o, i
         a.scale_log2 = scale_log2;
         a.Dh = Dh;
         a.n_sink = n_sink;
+        a.top_k = top_k;
         a.lse = lse;
         if (a.rope) rope_theta(rope_base, d, a.theta);
         return launch_attn_sm100(a, stream);
