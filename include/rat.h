@@ -272,9 +272,12 @@ RAT_API int rat_dilated_attn_prefill_sinks(const void *q, const void *k_rec, con
  * recurrence state that sums the chunk up), s_c = scale <q^_t, k~_{cD+D-1}>; every position of
  * the top_k best chunks (ties: the earlier chunk) joins S(t) and the sinks, each key once.
  *   Arguments as rat_dilated_attn_prefill_sinks, plus top_k in [0, 16] (RAT_ERR_UNSUPPORTED
- *   above 16).  Runs the CUDA-core kernel (float32 arithmetic) for both dtypes.  The selection
- *   is taken on float32 scores: where two chunk scores tie to within float32 rounding, either
- *   may be taken.  Prefill only: a decode step would need the uncompressed cache. */
+ *   above 16).  bf16 with d = 128, n_sink = 0 and T <= 65536 runs on the tensor cores: a
+ *   selection pass scores the chunk ends with q^ rounded to bf16 (the MMA operand), then the
+ *   key blocks holding the selected chunks join the attention with per-row masks.  Other calls
+ *   run the CUDA-core kernel (float32 arithmetic, q^ in float32).  Where two chunk scores tie
+ *   to within the rounding of the scoring precision, either may be taken.  Prefill only: a
+ *   decode step would need the uncompressed cache. */
 RAT_API int rat_dilated_attn_prefill_topk(const void *q, const void *k_rec, const void *v_rec,
                              void *o, int B, int H, int T, int d, int dtype, int D, int W,
                              const int32_t *D_per_head, int n_sink, int top_k, int64_t pos0,
@@ -324,8 +327,14 @@ RAT_API int rat_dilated_attn_prefill_ex(const void *q, const void *k_rec, const 
  *                        or NULL (the denominators are then recomputed: one more walk over
  *                        every key set)
  *   ws, ws_bytes       : workspace of at least rat_dilated_attn_backward_workspace_bytes
- * CUDA-core kernels with float32 accumulation: q^ is rounded to the dtype as the forward's
- * operand is, outputs are rounded once.  Three launches (prep, dq, dk~ and dv~); no device-side waits.
+ * bf16 with d = 128, n_sink = 0 and at most four distinct dilations > 1: a CUDA-core prep
+ * launch (q^ rounded to bf16 as the forward's operand, <dO_t, o_t>), then dq and dk~/dv~
+ * launches on the tensor cores (S, dP and S^T, dP^T products, dQ += dS K, dV += P^T dO,
+ * dK += dS^T q^; P and dS rounded to bf16 as MMA operands, float32 accumulation).  Without lse
+ * the forward runs once first to produce it (its output goes to dq, overwritten after).  Their
+ * pipeline waits are bounded; an expired one is recorded in the workspace header
+ * (rat_sync_status).  Other calls: three CUDA-core launches with float32 accumulation and no
+ * device-side waits.  Outputs are rounded once. 
  * ---------------------------------------------------------------------------------------- */
 RAT_API size_t rat_dilated_attn_backward_workspace_bytes(int B, int H, int T, int d, int dtype);
 
@@ -340,7 +349,8 @@ RAT_API int rat_dilated_attn_backward(const void *q, const void *k_rec, const vo
  * (wait site << 24) | (key block << 8) | phase parity; sites: 1 producer K-stage-free, 2 MMA
  * query-ready, 3 MMA K-stage-full, 4 MMA previous-PV, 5 MMA probabilities-ready, 6 softmax
  * query-loaded, 7 softmax scores-ready, 8 softmax rescale, 9 epilogue, 10 producer
- * query-rotated, 11 producer V-stage-free, 12 MMA V-stage-full.  0 if none. */
+ * query-rotated, 11 producer V-stage-free, 12 MMA V-stage-full; top-k selection: 13 selection
+ * published, 14 MMA selection-scores-read, 15 softmax selection-scores-ready.  0 if none. */
 RAT_API uint32_t rat_attn_error_site(void);
 
 /* Diagnostic: bit s set when a wait at site s (numbering as above) was still in progress when a

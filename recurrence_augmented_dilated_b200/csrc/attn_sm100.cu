@@ -11,17 +11,23 @@
 //   * the dilated stream -- the chunk ends i*D + D - 1, read through a TMA tensor map whose row
 //     stride is D rows of the recurrence output, so the gather costs nothing but a descriptor;
 //   * the window stream -- the contiguous band of positions the tile's windows cover.
-// Both are cut into blocks of 128 keys.  Per block:
+// Both are cut into blocks of BN keys (64 by default, two CTAs per SM; 128 selectable, one CTA
+// per SM).  Per block:
 //   S = Q K^T   (tcgen05.mma, bf16 operands from 128B-swizzled smem, f32 accumulator in TMEM,
 //                double-buffered so the next block's product overlaps this block's softmax);
 //   softmax     (one thread per query row reads its S row from TMEM, masks it to S(t), keeps a
 //                running max and sum; the max is only moved -- and O rescaled in TMEM -- when
 //                it grows by more than 2^8, which keeps the result exact and rescales rare);
-//   O += P V    (P written as bf16 into swizzled smem, V an MN-major smem operand).
-// Roles: warp 0 issues TMA loads (2-stage K/V ring), warp 1 allocates TMEM and issues the
-// MMAs, warps 2-5 do RoPE on Q (in smem), the softmax and the epilogue (O / l -> bf16 -> smem
-// -> TMA store).  Every mbarrier wait is bounded; on expiry the CTA records RAT_ERR_TIMEOUT in
-// a module error word, stops all roles, waits for its own async work and frees TMEM.
+//   O += P V    (P written back as bf16 into the first columns of its S buffer in TMEM and read
+//                from there as the A operand; V an MN-major smem operand).
+// With W <= 1 the self key stays out of the blocks: its k~ and v~ rows are read directly and it
+// joins the softmax and O in registers.  Attention sinks arrive as one more key block.  A
+// template variant adds top-k chunk selection (see attn_sm100_kernel).
+// Roles: warp 0 issues TMA loads (2-stage K and V rings with separate lifetimes), warp 1
+// allocates TMEM and issues the MMAs, warps 2-5 do RoPE on Q (in smem), the softmax and the
+// epilogue (O / l -> bf16 -> smem -> TMA store).  Every mbarrier wait is bounded; on expiry the
+// CTA records RAT_ERR_TIMEOUT in a module error word, stops all roles, waits for its own async
+// work and frees TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
