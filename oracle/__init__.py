@@ -56,6 +56,8 @@ def _load():
                                                   ctypes.c_double, _dp]
         lib.rat_oracle_recurrence_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp, _dp,
                                                        _dp, _dp]
+        lib.rat_oracle_recurrence_backward_reset.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp,
+                                                             _L, _L, _dp, _dp, _dp]
         lib.rat_oracle_rope.argtypes = [_L, _L, _L, _dp, _L, ctypes.c_double]
         lib.rat_oracle_in_key_set.argtypes = [_L, _L, _L, _L]
         lib.rat_oracle_in_key_set.restype = ctypes.c_int
@@ -170,10 +172,11 @@ def rope_transpose(y, pos0: int = 0, base: float = 10000.0):
     return np.concatenate([y1 * c + y2 * s, y2 * c - y1 * s], axis=-1)
 
 
-def recurrence_backward(x, a, dy, h0=None, dhT=None):
-    """Reverse-mode derivative of recurrence(x, a, h0) (the full-sequence form): returns
-    (dx, dg, dh0) for upstream gradients dy of the outputs and dhT of the final state; dg is
-    the gradient with respect to the gate value g = sigmoid(a)."""
+def recurrence_backward(x, a, dy, h0=None, dhT=None, pos0: int = 0, reset_every: int = 0):
+    """Reverse-mode derivative of recurrence(x, a, h0, pos0, reset_every): returns (dx, dg, dh0)
+    for upstream gradients dy of the outputs and dhT of the final state; dg is the gradient with
+    respect to the gate value g = sigmoid(a).  reset_every = L > 0 is the chunk-local form (the
+    state restarts before every absolute position pos0 + t that is a multiple of L)."""
     x, a, dy = _f64(x), _f64(a), _f64(dy)
     assert x.shape == a.shape == dy.shape
     T, d = x.shape[-2], x.shape[-1]
@@ -188,19 +191,24 @@ def recurrence_backward(x, a, dy, h0=None, dhT=None):
     if dhT is not None:
         dhT = _f64(dhT)
         dhTp = _ptr(dhT)
-    _load().rat_oracle_recurrence_backward(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(dy), dhTp,
-                                           _ptr(dx), _ptr(dg), _ptr(dh0))
+    if reset_every > 0:
+        _load().rat_oracle_recurrence_backward_reset(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(dy),
+                                                     dhTp, int(pos0), int(reset_every), _ptr(dx),
+                                                     _ptr(dg), _ptr(dh0))
+    else:
+        _load().rat_oracle_recurrence_backward(BH, T, d, _ptr(x), _ptr(a), h0p, _ptr(dy), dhTp,
+                                               _ptr(dx), _ptr(dg), _ptr(dh0))
     return dx, dg, dh0
 
 
 def recurrence_layer_backward(k, v, a, dk_rec, dv_rec, h0k=None, h0v=None, dhTk=None, dhTv=None,
-                              pos0: int = 0, rope_base: float = 0.0):
+                              pos0: int = 0, rope_base: float = 0.0, reset_every: int = 0):
     """Backward of the prefill recurrence step (k~ = RoPE(h^k), v~ = h^v, one gate for both):
     returns (dk, dv, da, dh0k, dh0v).  The gate is shared, so its gradient sums the k and v
-    parts, through dg/da = g (1 - g)."""
+    parts, through dg/da = g (1 - g).  reset_every = L > 0: the chunk-local form."""
     ek = rope_transpose(dk_rec, pos0, rope_base) if rope_base > 0 else _f64(dk_rec)
-    dk, dgk, dh0k = recurrence_backward(k, a, ek, h0k, dhTk)
-    dv, dgv, dh0v = recurrence_backward(v, a, dv_rec, h0v, dhTv)
+    dk, dgk, dh0k = recurrence_backward(k, a, ek, h0k, dhTk, pos0, reset_every)
+    dv, dgv, dh0v = recurrence_backward(v, a, dv_rec, h0v, dhTv, pos0, reset_every)
     a = _f64(a)
     with np.errstate(over="ignore"):        # saturated logits: exp -> inf gives g = 0 or 1
         g = 1.0 / (1.0 + np.exp(-a))

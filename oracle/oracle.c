@@ -176,6 +176,47 @@ void rat_oracle_recurrence_backward(long BH, long T, long d, const double *x, co
 }
 
 /*
+ * Backward of the chunk-local recurrence (RAT: the state restarts before every absolute
+ * position pos0 + t that is a multiple of L; "RAT+ Deep Dive" section 2.1), for one of x = k or
+ * x = v.  Forward: hs_t = 0 if (pos0 + t) mod L == 0, else h_{t-1} (h_{-1} = h0), then
+ * h_t = g_t hs_t + (1 - g_t) x_t.  Reverse-mode derivative: the total gradient of h_t is
+ *   mu_t = dy_t + [pos0 + t + 1 is not a block start] g_{t+1} mu_{t+1},  mu_{T-1} = dy_{T-1} + dhT,
+ * and  dL/dx_t = (1 - g_t) mu_t,  dL/dg_t = mu_t (hs_t - x_t),
+ *      dL/dh0 = [pos0 is not a block start] g_0 mu_0   (h0 reaches only rows before a restart).
+ * hs is recomputed by the forward loop; dg as in rat_oracle_recurrence_backward.
+ */
+void rat_oracle_recurrence_backward_reset(long BH, long T, long d, const double *x,
+                                          const double *a, const double *h0, const double *dy,
+                                          const double *dhT, long pos0, long L, double *dx,
+                                          double *dg, double *dh0)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        double *hs = (double *)malloc((size_t)(T + 1) * sizeof(double));  /* state entering t */
+        for (long c = 0; c < d; ++c) {
+            double h = h0 ? h0[bh * d + c] : 0.0;
+            for (long t = 0; t < T; ++t) {
+                long idx = (bh * T + t) * d + c;
+                if ((pos0 + t) % L == 0) h = 0.0;                /* a block starts at row t */
+                hs[t] = h;
+                h = forget_gate(a[idx]) * h + one_minus_gate(a[idx]) * x[idx];
+            }
+            double mu = dhT ? dhT[bh * d + c] : 0.0;         /* gradient arriving from t + 1 */
+            for (long t = T - 1; t >= 0; --t) {
+                long idx = (bh * T + t) * d + c;
+                mu += dy[idx];                               /* total dL/dh_t */
+                dx[idx] = one_minus_gate(a[idx]) * mu;
+                dg[idx] = mu * (hs[t] - x[idx]);
+                /* dL/dh_{t-1}: through h_t, unless the state was restarted at row t */
+                mu = (pos0 + t) % L == 0 ? 0.0 : mu * forget_gate(a[idx]);
+            }
+            if (dh0) dh0[bh * d + c] = mu;
+        }
+        free(hs);
+    }
+}
+
+/*
  * Rotary position embedding, rotate-half pairing, in place.                  [RoFormer]
  *   x : [BH][T][d];  position of row t is pos0 + t;  for c < d/2:
  *   theta_c = base^(-2c/d),  phi = (pos0 + t) * theta_c,

@@ -332,6 +332,109 @@ def test_backward_zero_gate_passes_the_gradient_through():
     assert np.all(da == 0.0) and np.all(dh0k == 0.0)
 
 
+# ---- backward of the chunk-local recurrence (the state restarts at multiples of L)
+def _torch_layer_reset(k, v, a, h0k, h0v, pos0, L, base):
+    """The chunk-local forward step written with torch float64 ops, for autograd."""
+    import torch
+    T, d = k.shape[-2], k.shape[-1]
+    g = torch.sigmoid(a)
+    hk, hv = h0k, h0v
+    yk, yv = [], []
+    for t in range(T):
+        if (pos0 + t) % L == 0:
+            hk, hv = torch.zeros_like(hk), torch.zeros_like(hv)
+        hk = g[..., t, :] * hk + (1 - g[..., t, :]) * k[..., t, :]
+        hv = g[..., t, :] * hv + (1 - g[..., t, :]) * v[..., t, :]
+        yk.append(hk)
+        yv.append(hv)
+    yk, yv = torch.stack(yk, -2), torch.stack(yv, -2)
+    if base > 0:
+        half = d // 2
+        theta = base ** (-2.0 * torch.arange(half, dtype=torch.float64) / d)
+        ang = (pos0 + torch.arange(T, dtype=torch.float64))[:, None] * theta[None, :]
+        c, s_ = torch.cos(ang), torch.sin(ang)
+        y1, y2 = yk[..., :half], yk[..., half:]
+        yk = torch.cat([y1 * c - y2 * s_, y2 * c + y1 * s_], -1)
+    return yk, yv, hk, hv
+
+
+@pytest.mark.parametrize("base,pos0,L", [(0.0, 0, 4), (10000.0, 37, 5), (0.0, 3, 1), (500.0, 1, 16)])
+def test_reset_backward_matches_autograd(base, pos0, L):
+    import torch
+    shp = (2, 11, 6)
+    k, v, a = (torch.tensor(RNG.standard_normal(shp), requires_grad=True) for _ in range(3))
+    h0k, h0v = (torch.tensor(RNG.standard_normal((2, 6)), requires_grad=True) for _ in range(2))
+    dyk, dyv = RNG.standard_normal(shp), RNG.standard_normal(shp)
+    dhk, dhv = RNG.standard_normal((2, 6)), RNG.standard_normal((2, 6))
+    yk, yv, hk, hv = _torch_layer_reset(k, v, a, h0k, h0v, pos0, L, base)
+    loss = ((yk * torch.tensor(dyk)).sum() + (yv * torch.tensor(dyv)).sum() +
+            (hk * torch.tensor(dhk)).sum() + (hv * torch.tensor(dhv)).sum())
+    loss.backward()
+    dk, dv, da, dh0k, dh0v = oracle.recurrence_layer_backward(
+        k.detach().numpy(), v.detach().numpy(), a.detach().numpy(), dyk, dyv,
+        h0k.detach().numpy(), h0v.detach().numpy(), dhk, dhv, pos0=pos0, rope_base=base,
+        reset_every=L)
+    for mine, ref in ((dk, k.grad), (dv, v.grad), (da, a.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12)
+    for mine, ref in ((dh0k, h0k.grad), (dh0v, h0v.grad)):
+        ref = ref.numpy() if ref is not None else np.zeros_like(mine)
+        np.testing.assert_allclose(mine, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_reset_backward_finite_differences():
+    # central differences of L = <dy, y> + <dhT, hT> through the oracle's chunk-local forward
+    T, d, pos0, Lb = 9, 3, 2, 4
+    x, a = RNG.standard_normal((1, T, d)), RNG.standard_normal((1, T, d))
+    h0, dy, dhT = RNG.standard_normal((1, d)), RNG.standard_normal((1, T, d)), RNG.standard_normal((1, d))
+
+    def L(x_, a_, h0_):
+        y, hT = oracle.recurrence(x_, a_, h0_, pos0=pos0, reset_every=Lb)
+        return float((y * dy).sum() + (hT * dhT).sum())
+
+    dx, dg, dh0 = oracle.recurrence_backward(x, a, dy, h0, dhT, pos0=pos0, reset_every=Lb)
+    g = 1.0 / (1.0 + np.exp(-a))
+    da = dg * g * (1 - g)
+    eps = 1e-6
+    for (t, c) in ((0, 0), (1, 2), (2, 1), (5, 0), (8, 2)):
+        for arr, grad in ((x, dx), (a, da)):
+            p_, m_ = arr.copy(), arr.copy()
+            p_[0, t, c] += eps
+            m_[0, t, c] -= eps
+            args_p = (p_, a, h0) if arr is x else (x, p_, h0)
+            args_m = (m_, a, h0) if arr is x else (x, m_, h0)
+            fd = (L(*args_p) - L(*args_m)) / (2 * eps)
+            assert abs(fd - grad[0, t, c]) <= 1e-7 * max(1.0, abs(fd)), (t, c, fd, grad[0, t, c])
+    for c in range(d):
+        p_, m_ = h0.copy(), h0.copy()
+        p_[0, c] += eps
+        m_[0, c] -= eps
+        fd = (L(x, a, p_) - L(x, a, m_)) / (2 * eps)
+        assert abs(fd - dh0[0, c]) <= 1e-7 * max(1.0, abs(fd))
+
+
+def test_reset_backward_without_a_block_start_is_the_full_backward():
+    # no multiple of L among pos0 .. pos0 + T - 1: the same bits as the full-sequence backward
+    x, a, dy = (RNG.standard_normal((2, 30, 4)) for _ in range(3))
+    h0, dhT = RNG.standard_normal((2, 4)), RNG.standard_normal((2, 4))
+    full = oracle.recurrence_backward(x, a, dy, h0, dhT)
+    loc = oracle.recurrence_backward(x, a, dy, h0, dhT, pos0=1, reset_every=100)
+    for f, l_ in zip(full, loc):
+        np.testing.assert_array_equal(f, l_)
+
+
+def test_reset_backward_every_position_keeps_only_the_input_term():
+    # L = 1: y_t = (1 - g_t) x_t, so dx = (1 - g) dy (+ dhT on the last row), dg = -dy x, dh0 = 0
+    x, a, dy = (RNG.standard_normal((2, 12, 3)) for _ in range(3))
+    dhT = RNG.standard_normal((2, 3))
+    dx, dg, dh0 = oracle.recurrence_backward(x, a, dy, None, dhT, pos0=5, reset_every=1)
+    mu = dy.copy()
+    mu[:, -1] += dhT
+    omg = 1.0 / (1.0 + np.exp(a))
+    np.testing.assert_allclose(dx, omg * mu, rtol=1e-14, atol=0)
+    np.testing.assert_allclose(dg, -mu * x, rtol=1e-14, atol=0)
+    assert np.all(dh0 == 0.0)
+
+
 def test_rope_transpose_inverts_rope():
     x = RNG.standard_normal((2, 11, 8))
     np.testing.assert_allclose(oracle.rope_transpose(oracle.rope(x, 123, 500.0), 123, 500.0), x,
