@@ -688,9 +688,11 @@ def run_decode_paged(w: synthetic.Workload, steps_timed: int, warmup: int, rank:
     }
 
 
-def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, peaks, peak_kind):
+def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, peaks, peak_kind,
+                 reset_every: int = 0):
     """Backward of the recurrence step on the prefill workload: the forward outputs and
-    upstream gradients are resident; each timed step is one rat_recur_backward call."""
+    upstream gradients are resident; each timed step is one rat_recur_backward call
+    (rat_recur_backward_local with reset_every = L > 0)."""
     import recurrence_augmented_dilated_b200 as rat
     dev = torch.device("cuda")
     x = synthetic.prefill_inputs(w)
@@ -699,7 +701,10 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     dtc = rat.F32 if w.dtype == "f32" else rat.BF16
     kr, vr = torch.empty_like(k), torch.empty_like(v)
     ws_f = rat.Workspace(rat.rat_recur_workspace_bytes(B, H, T, d, dtc))
-    rat.rat_recur_prefill(k, v, a, kr, vr, ws_f, rope_base=w.rope_base)
+    if reset_every > 0:
+        rat.rat_recur_prefill_local(k, v, a, kr, vr, ws_f, reset_every, rope_base=w.rope_base)
+    else:
+        rat.rat_recur_prefill(k, v, a, kr, vr, ws_f, rope_base=w.rope_base)
     g = torch.Generator(device=dev).manual_seed(w.seed + 77)
     dyk = torch.randn(k.shape, generator=g, device=dev).to(k.dtype)
     dyv = torch.randn(k.shape, generator=g, device=dev).to(k.dtype)
@@ -708,7 +713,8 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     stream = torch.cuda.current_stream()
 
     def step():
-        rat.rat_recur_backward(k, v, a, kr, vr, dyk, dyv, dk, dv, da, ws, rope_base=w.rope_base)
+        rat.rat_recur_backward(k, v, a, kr, vr, dyk, dyv, dk, dv, da, ws, rope_base=w.rope_base,
+                               reset_every=reset_every)
 
     with ProfiledRegion():
         for _ in range(warmup):
@@ -728,7 +734,9 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     eb = 2 if w.dtype == "bf16" else 4
     nbytes = 10 * B * H * T * d * eb       # read k, v, a, k~, v~, dk~, dv~; write dk, dv, da
     achieved = nbytes / (ms * 1e-3) / 1e9
-    res = {"workload": w.name, "step": "rat_recur_backward (3 launches)", "ms": ms,
+    res = {"workload": w.name, "ms": ms,
+           "step": ("rat_recur_backward_local(L=%d)" % reset_every if reset_every else
+                    "rat_recur_backward") + " (3 launches)",
            "tokens_per_s": world * B * T / (ms * 1e-3),
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "of": peak_kind,
@@ -1047,7 +1055,8 @@ def main():
     if others:
         line["workloads"] = others
     if args.backward:
-        line["backward"] = run_backward(w, args.steps, args.warmup, world, peaks, peak_kind)
+        line["backward"] = run_backward(w, args.steps, args.warmup, world, peaks, peak_kind,
+                                        reset_every=args.reset_every)
     if args.decode_paged:
         dw = synthetic.WORKLOADS["decode_7p6b"]
         line["decode_paged"] = run_decode_paged(dw, max(1, min(args.steps, 10)), 3, rank, world,

@@ -15,6 +15,7 @@
  *   rat_recur_prefill_window the same recurrence over a fixed window of the last Lw = 64
  *                            positions (RAT+'s L*).
  *   rat_recur_backward       gradients of rat_recur_prefill's step.
+ *   rat_recur_backward_local gradients of rat_recur_prefill_local's step.
  *   rat_dilated_attn_prefill causal attention of each query t over
  *                              S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D = D-1 },
  *                            We = max(W, 1), D per head; optional RoPE on q.
@@ -184,6 +185,22 @@ RAT_API int rat_recur_backward(const void *k, const void *v, const void *gate_lo
                        void *dgate_logit, float *dh0_k, float *dh0_v, int B, int H, int T,
                        int d, int dtype, int64_t pos0, float rope_base, void *ws,
                        size_t ws_bytes, void *stream);
+
+/* rat_recur_backward_local -- gradients of rat_recur_prefill_local's step (RAT's chunk-local
+ * recurrence, restarted before every absolute position pos0 + t with (pos0 + t) mod L = 0).
+ *   Arguments as rat_recur_backward, plus L >= 1 (RAT_ERR_INVALID otherwise), as given to the
+ *   forward.  Both recurrences are cut at block starts:
+ *     mu_t = e_t + [pos0 + t + 1 not a block start] g_{t+1} mu_{t+1},
+ *     dgate_t uses h_{t-1} = 0 at a block start,
+ *     dh0 = g_0 mu_0 when pos0 is not a block start, else 0 (h0 reaches only the rows before the
+ *     first start). */
+RAT_API int rat_recur_backward_local(const void *k, const void *v, const void *gate_logit,
+                             const float *h0_k, const float *h0_v, const void *k_rec,
+                             const void *v_rec, const void *dk_rec, const void *dv_rec,
+                             const float *dhT_k, const float *dhT_v, void *dk, void *dv,
+                             void *dgate_logit, float *dh0_k, float *dh0_v, int B, int H, int T,
+                             int d, int dtype, int64_t pos0, int64_t L, float rope_base, void *ws,
+                             size_t ws_bytes, void *stream);
 
 /* ------------------------------------------------------------------------------------------
  * rat_recur_prefill_window -- the fixed-window recurrence of RAT+: each state covers only the

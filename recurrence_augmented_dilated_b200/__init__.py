@@ -22,7 +22,8 @@ import torch
 __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_recur_prefill_local",
-    "rat_recur_prefill_window", "rat_recur_backward", "rat_recur_backward_workspace_bytes",
+    "rat_recur_prefill_window", "rat_recur_backward", "rat_recur_backward_local",
+    "rat_recur_backward_workspace_bytes",
     "rat_dilated_attn_backward", "rat_dilated_attn_backward_workspace_bytes",
     "rat_dilated_attn_prefill",
     "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
@@ -116,6 +117,8 @@ def lib():
         L.rat_recur_backward_workspace_bytes.restype = _sz
         L.rat_recur_backward_workspace_bytes.argtypes = [_i, _i, _i, _i]
         L.rat_recur_backward.argtypes = [_vp] * 16 + [_i, _i, _i, _i, _i, _i64, _f, _vp, _sz, _vp]
+        L.rat_recur_backward_local.argtypes = [_vp] * 16 + [_i, _i, _i, _i, _i, _i64, _i64, _f,
+                                                            _vp, _sz, _vp]
         L.rat_recur_prefill_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                _i, _i, _i, _i, _i, _i64, _i64, _f, _vp, _sz, _vp]
         L.rat_recur_prefill_local.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
@@ -253,16 +256,21 @@ def rat_recur_backward_workspace_bytes(B, H, T, d) -> int:
 
 def rat_recur_backward(k, v, gate_logit, k_rec, v_rec, dk_rec, dv_rec, dk, dv, dgate_logit,
                        ws: Workspace, h0_k=None, h0_v=None, dhT_k=None, dhT_v=None, dh0_k=None,
-                       dh0_v=None, pos0: int = 0, rope_base: float = 0.0, stream=None):
+                       dh0_v=None, pos0: int = 0, rope_base: float = 0.0, stream=None,
+                       reset_every: int = 0):
     """Gradients of the prefill recurrence step: dk, dv, dgate_logit (all (B, H, T, d)) and,
-    if given, dh0_k, dh0_v (float32 (B, H, d))."""
+    if given, dh0_k, dh0_v (float32 (B, H, d)).  reset_every = L > 0: the chunk-local form
+    (rat_recur_backward_local)."""
     B, H, T, d = k.shape
-    st = lib().rat_recur_backward(_ptr(k), _ptr(v), _ptr(gate_logit), _ptr(h0_k), _ptr(h0_v),
-                                  _ptr(k_rec), _ptr(v_rec), _ptr(dk_rec), _ptr(dv_rec),
-                                  _ptr(dhT_k), _ptr(dhT_v), _ptr(dk), _ptr(dv),
-                                  _ptr(dgate_logit), _ptr(dh0_k), _ptr(dh0_v), B, H, T, d,
-                                  _dtype_code(k), int(pos0), float(rope_base), ws.ptr, ws.nbytes,
-                                  _stream(stream))
+    args = [_ptr(k), _ptr(v), _ptr(gate_logit), _ptr(h0_k), _ptr(h0_v), _ptr(k_rec), _ptr(v_rec),
+            _ptr(dk_rec), _ptr(dv_rec), _ptr(dhT_k), _ptr(dhT_v), _ptr(dk), _ptr(dv),
+            _ptr(dgate_logit), _ptr(dh0_k), _ptr(dh0_v), B, H, T, d, _dtype_code(k), int(pos0)]
+    if reset_every > 0:
+        st = lib().rat_recur_backward_local(*args, int(reset_every), float(rope_base), ws.ptr,
+                                            ws.nbytes, _stream(stream))
+        _check("rat_recur_backward_local", st)
+        return
+    st = lib().rat_recur_backward(*args, float(rope_base), ws.ptr, ws.nbytes, _stream(stream))
     _check("rat_recur_backward", st)
 
 

@@ -81,6 +81,7 @@ struct RecurBwdParams {
     float theta_f[64];
     double theta[64];
     float step_cos[64], step_sin[64];
+    long long reset;                // > 0: the chunk-local form (state restarted at multiples)
 };
 size_t recur_bwd_workspace_bytes(int BH, int T, int d);
 int launch_recur_bwd(const RecurBwdParams &p, int dtype, void *stream);

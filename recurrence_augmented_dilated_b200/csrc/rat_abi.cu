@@ -185,6 +185,49 @@ int recur_prefill(const void *k, const void *v, const void *gate_logit, const fl
 }
 }  // namespace
 
+namespace {
+int recur_backward(const void *k, const void *v, const void *gate_logit, const float *h0_k,
+                   const float *h0_v, const void *k_rec, const void *v_rec, const void *dk_rec,
+                   const void *dv_rec, const float *dhT_k, const float *dhT_v, void *dk, void *dv,
+                   void *dgate_logit, float *dh0_k, float *dh0_v, int B, int H, int T, int d,
+                   int dtype, int64_t pos0, int64_t L, float rope_base, void *ws, size_t ws_bytes,
+                   void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || L < 0) return RAT_ERR_INVALID;
+    if (!supported_d(d)) return RAT_ERR_UNSUPPORTED;
+    if (pos0 < 0 || !std::isfinite(rope_base)) return RAT_ERR_INVALID;
+    if (T == 0) return RAT_OK;
+    const void *req[] = {k, v, gate_logit, k_rec, v_rec, dk_rec, dv_rec, dk, dv, dgate_logit};
+    for (const void *q : req)
+        if (!q || !aligned16(q)) return RAT_ERR_INVALID;
+    if ((long long)B * H * T > (1ll << 40)) return RAT_ERR_UNSUPPORTED;
+    const size_t need = recur_bwd_workspace_bytes(B * H, T, d);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RAT_ERR_WORKSPACE;
+    RecurBwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k; p.v = v; p.a = gate_logit; p.yk = k_rec; p.yv = v_rec; p.dyk = dk_rec; p.dyv = dv_rec;
+    p.h0k = h0_k; p.h0v = h0_v; p.dhTk = dhT_k; p.dhTv = dhT_v;
+    p.dk = dk; p.dv = dv; p.da = dgate_logit; p.dh0k = dh0_k; p.dh0v = dh0_v;
+    p.BH = B * H; p.T = T; p.d = d;
+    p.nch = (T + kBwdRows - 1) / kBwdRows;
+    p.pos0 = pos0;
+    p.reset = L;
+    p.rope = rope_base > 0.f ? 1 : 0;
+    uint8_t *w = static_cast<uint8_t *>(ws);
+    p.agg = reinterpret_cast<float *>(w + sizeof(WsHeader));
+    p.carry = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256((size_t)p.BH * p.nch * 3 * d * 4));
+    if (p.rope) {
+        rope_theta(rope_base, d, p.theta);
+        for (int c = 0; c < 64; ++c) {
+            p.theta_f[c] = (float)p.theta[c];
+            p.step_cos[c] = (float)std::cos(p.theta[c]);
+            p.step_sin[c] = (float)std::sin(p.theta[c]);
+        }
+        p.rope_f32 = (dtype == RAT_BF16 && pos0 + (int64_t)T <= 8192) ? 1 : 0;
+    }
+    return launch_recur_bwd(p, dtype, stream);
+}
+}  // namespace
+
 extern "C" {
 
 int rat_recur_prefill(const void *k, const void *v, const void *gate_logit, const float *h0_k,
@@ -206,38 +249,22 @@ int rat_recur_backward(const void *k, const void *v, const void *gate_logit, con
                        const float *dhT_v, void *dk, void *dv, void *dgate_logit, float *dh0_k,
                        float *dh0_v, int B, int H, int T, int d, int dtype, int64_t pos0,
                        float rope_base, void *ws, size_t ws_bytes, void *stream) {
-    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype)) return RAT_ERR_INVALID;
-    if (!supported_d(d)) return RAT_ERR_UNSUPPORTED;
-    if (pos0 < 0 || !std::isfinite(rope_base)) return RAT_ERR_INVALID;
-    if (T == 0) return RAT_OK;
-    const void *req[] = {k, v, gate_logit, k_rec, v_rec, dk_rec, dv_rec, dk, dv, dgate_logit};
-    for (const void *q : req)
-        if (!q || !aligned16(q)) return RAT_ERR_INVALID;
-    if ((long long)B * H * T > (1ll << 40)) return RAT_ERR_UNSUPPORTED;
-    const size_t need = recur_bwd_workspace_bytes(B * H, T, d);
-    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return RAT_ERR_WORKSPACE;
-    RecurBwdParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.k = k; p.v = v; p.a = gate_logit; p.yk = k_rec; p.yv = v_rec; p.dyk = dk_rec; p.dyv = dv_rec;
-    p.h0k = h0_k; p.h0v = h0_v; p.dhTk = dhT_k; p.dhTv = dhT_v;
-    p.dk = dk; p.dv = dv; p.da = dgate_logit; p.dh0k = dh0_k; p.dh0v = dh0_v;
-    p.BH = B * H; p.T = T; p.d = d;
-    p.nch = (T + kBwdRows - 1) / kBwdRows;
-    p.pos0 = pos0;
-    p.rope = rope_base > 0.f ? 1 : 0;
-    uint8_t *w = static_cast<uint8_t *>(ws);
-    p.agg = reinterpret_cast<float *>(w + sizeof(WsHeader));
-    p.carry = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256((size_t)p.BH * p.nch * 3 * d * 4));
-    if (p.rope) {
-        rope_theta(rope_base, d, p.theta);
-        for (int c = 0; c < 64; ++c) {
-            p.theta_f[c] = (float)p.theta[c];
-            p.step_cos[c] = (float)std::cos(p.theta[c]);
-            p.step_sin[c] = (float)std::sin(p.theta[c]);
-        }
-        p.rope_f32 = (dtype == RAT_BF16 && pos0 + (int64_t)T <= 8192) ? 1 : 0;
-    }
-    return launch_recur_bwd(p, dtype, stream);
+    return recur_backward(k, v, gate_logit, h0_k, h0_v, k_rec, v_rec, dk_rec, dv_rec, dhT_k,
+                          dhT_v, dk, dv, dgate_logit, dh0_k, dh0_v, B, H, T, d, dtype, pos0, 0,
+                          rope_base, ws, ws_bytes, stream);
+}
+
+int rat_recur_backward_local(const void *k, const void *v, const void *gate_logit,
+                             const float *h0_k, const float *h0_v, const void *k_rec,
+                             const void *v_rec, const void *dk_rec, const void *dv_rec,
+                             const float *dhT_k, const float *dhT_v, void *dk, void *dv,
+                             void *dgate_logit, float *dh0_k, float *dh0_v, int B, int H, int T,
+                             int d, int dtype, int64_t pos0, int64_t L, float rope_base, void *ws,
+                             size_t ws_bytes, void *stream) {
+    if (L < 1) return RAT_ERR_INVALID;
+    return recur_backward(k, v, gate_logit, h0_k, h0_v, k_rec, v_rec, dk_rec, dv_rec, dhT_k,
+                          dhT_v, dk, dv, dgate_logit, dh0_k, dh0_v, B, H, T, d, dtype, pos0, L,
+                          rope_base, ws, ws_bytes, stream);
 }
 
 int rat_recur_prefill_window(const void *k, const void *v, const void *gate_logit,

@@ -21,6 +21,12 @@
 // pairs (2l, 2l+1) and (2l + d/2, 2l+1 + d/2), the RoPE partners), loading U rows at a time.
 // No CTA waits for another.  HBM traffic: the reduce pass reads a, dk~, dv~ (3 N elements),
 // the output pass reads seven tensors and writes three (10 N), against the 10 N minimum.
+//
+// The chunk-local form (RESET; RAT's recurrence restarted before every absolute position that
+// is a multiple of L) cuts both recurrences at block starts: no gradient passes from a block
+// start t to t - 1 (the factor g_t of mu_{t-1} becomes 0, so a chunk map composed across a
+// start has A = 0), the state entering a block start is 0 in da, and h0 gets a gradient only
+// when row 0 is not a block start.
 #include "common.cuh"
 
 namespace rat {
@@ -61,6 +67,9 @@ RAT_DEVICE void rot_t(const f2_t *y, f2_t c, f2_t s, f2_t *x) {
     x[1] = f2_fma(y[0], ns, f2_mul(y[1], c));
 }
 
+// does a block of the chunk-local form start at row t?
+RAT_DEVICE bool block_start(const RecurBwdParams &p, long long t) { return (p.pos0 + t) % p.reset == 0; }
+
 // one step back in position: angle - theta
 RAT_DEVICE void step_back(f2_t &c, f2_t &s, f2_t sc, f2_t ss) {
     const f2_t ns = f2_mul(ss, f2(-1.f, -1.f));
@@ -71,7 +80,7 @@ RAT_DEVICE void step_back(f2_t &c, f2_t &s, f2_t sc, f2_t ss) {
 
 }  // namespace
 
-template <typename E, int DH>
+template <typename E, int DH, bool RESET>
 __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS) bwd_reduce_kernel(const __grid_constant__ RecurBwdParams p) {
     using C = BwdCfg<E, DH>;
     constexpr int NP = 2, U = C::UR;
@@ -92,6 +101,7 @@ __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS) bwd_reduce_kernel(cons
         Lane<E>::template load<C::HALFB>(ga + (size_t)(t1 + 1) * C::ROWB, cl, xa);
         gnext[0] = forget_gate2(xa[0]);
         gnext[1] = forget_gate2(xa[1]);
+        if (RESET && block_start(p, t1 + 1)) gnext[0] = gnext[1] = kZero2;   // nothing passes a start
     }
     f2_t rc = kOne2, rs = kZero2, sc = kOne2, ss = kZero2;
     if (p.rope) {
@@ -118,11 +128,12 @@ __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS) bwd_reduce_kernel(cons
                 step_back(rc, rs, sc, ss);
             }
 #pragma unroll
+            const bool start = RESET && block_start(p, tb - u);
             for (int q = 0; q < NP; ++q) {
                 A[q] = f2_mul(gnext[q], A[q]);
                 Bk[q] = f2_fma(gnext[q], Bk[q], ek[q]);
                 Bv[q] = f2_fma(gnext[q], Bv[q], yv[u][q]);
-                gnext[q] = forget_gate2(xa[u][q]);
+                gnext[q] = start ? kZero2 : forget_gate2(xa[u][q]);
             }
         }
     }
@@ -165,8 +176,11 @@ __global__ void __launch_bounds__(128) bwd_carry_kernel(const __grid_constant__ 
             cv = fmaf(a[u], cv, bv[u]);
         }
     }
-    // ck, cv are now mu_0: dh0 = g_0 mu_0
-    if (p.dh0k || p.dh0v) {
+    // ck, cv are now mu_0: dh0 = g_0 mu_0 (0 when row 0 starts a block: h0 is not used)
+    if (p.reset > 0 && p.pos0 % p.reset == 0) {
+        if (p.dh0k) p.dh0k[id] = 0.f;
+        if (p.dh0v) p.dh0v[id] = 0.f;
+    } else if (p.dh0k || p.dh0v) {
         float a0;
         const E *ar = static_cast<const E *>(p.a) + (size_t)bh * p.T * p.d + ch;
         if constexpr (sizeof(E) == 2) a0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(ar));
@@ -178,7 +192,7 @@ __global__ void __launch_bounds__(128) bwd_carry_kernel(const __grid_constant__ 
     }
 }
 
-template <typename E, int DH>
+template <typename E, int DH, bool RESET>
 __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS, 2) bwd_out_kernel(const __grid_constant__ RecurBwdParams p) {
     using C = BwdCfg<E, DH>;
     constexpr int NP = 2, U = C::U;
@@ -217,6 +231,7 @@ __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS, 2) bwd_out_kernel(cons
         Lane<E>::template load<C::HALFB>(ga + (size_t)(t1 + 1) * C::ROWB, cl, xa);
         gnext[0] = forget_gate2(xa[0]);
         gnext[1] = forget_gate2(xa[1]);
+        if (RESET && block_start(p, t1 + 1)) gnext[0] = gnext[1] = kZero2;
     }
     // rotation at t (for dk~_t) and at t - 1 (for k~_{t-1})
     f2_t rc = kOne2, rs = kZero2, pc = kOne2, ps = kZero2, sc = kOne2, ss = kZero2;
@@ -268,6 +283,11 @@ __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS, 2) bwd_out_kernel(cons
 #pragma unroll
                 for (int q = 0; q < NP; ++q) { hpk[q] = h0k[q]; hpv[q] = h0v[q]; }
             }
+            const bool start = RESET && block_start(p, t);
+            if (start) {                               // the state entering a block start is 0
+#pragma unroll
+                for (int q = 0; q < NP; ++q) { hpk[q] = kZero2; hpv[q] = kZero2; }
+            }
             f2_t ok[NP], ov[NP], oa[NP];
 #pragma unroll
             for (int q = 0; q < NP; ++q) {
@@ -280,7 +300,7 @@ __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS, 2) bwd_out_kernel(cons
                 const f2_t sk = f2_fma(xk[u][q], f2(-1.f, -1.f), hpk[q]);     // h_{t-1} - x_t
                 const f2_t sv = f2_fma(xv[u][q], f2(-1.f, -1.f), hpv[q]);
                 oa[q] = f2_mul(f2_mul(g, og), f2_fma(muk[q], sk, f2_mul(muv[q], sv)));
-                gnext[q] = g;
+                gnext[q] = start ? kZero2 : g;
             }
             const size_t o = (size_t)t * C::ROWB;
             Lane<E>::template store<C::HALFB>(odk + o, cl, ok);
@@ -301,10 +321,16 @@ static int launch_bwd_one(const RecurBwdParams &p, cudaStream_t s) {
     const long long streams = (long long)p.BH * p.nch;
     const long long grid = (streams + C::SPB - 1) / C::SPB;
     if (grid > 0x7fffffffll) return RAT_ERR_UNSUPPORTED;
-    bwd_reduce_kernel<E, DH><<<(unsigned)grid, C::THREADS, 0, s>>>(p);
     const long long n = (long long)p.BH * p.d;
-    bwd_carry_kernel<E><<<(unsigned)((n + 127) / 128), 128, 0, s>>>(p);
-    bwd_out_kernel<E, DH><<<(unsigned)grid, C::THREADS, 0, s>>>(p);
+    if (p.reset > 0) {
+        bwd_reduce_kernel<E, DH, true><<<(unsigned)grid, C::THREADS, 0, s>>>(p);
+        bwd_carry_kernel<E><<<(unsigned)((n + 127) / 128), 128, 0, s>>>(p);
+        bwd_out_kernel<E, DH, true><<<(unsigned)grid, C::THREADS, 0, s>>>(p);
+    } else {
+        bwd_reduce_kernel<E, DH, false><<<(unsigned)grid, C::THREADS, 0, s>>>(p);
+        bwd_carry_kernel<E><<<(unsigned)((n + 127) / 128), 128, 0, s>>>(p);
+        bwd_out_kernel<E, DH, false><<<(unsigned)grid, C::THREADS, 0, s>>>(p);
+    }
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 
