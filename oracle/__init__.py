@@ -372,10 +372,13 @@ class DecodeState:
 
     Keeping every position is the plain definition (the compressed cache is an optimisation
     of it); use it on a few (batch, head) slices.  Dbh gives each slice's dilation.
+    window_rec = Lw > 0 selects the fixed-window recurrence (recurrence_window): the state of
+    each new token is the recurrence restarted from zero Lw - 1 positions back, so the raw
+    inputs (k, v, a) of every position are kept too.
     """
 
     def __init__(self, Dbh, d: int, W: int, Tcap: int, rope_base: float = 0.0, scale=None,
-                 reset_every: int = 0, n_sink: int = 0):
+                 reset_every: int = 0, n_sink: int = 0, window_rec: int = 0):
         self.Dbh = np.ascontiguousarray(np.asarray(Dbh, dtype=np.int32))
         self.BH = len(self.Dbh)
         self.d, self.W, self.Tcap = d, int(W), int(Tcap)
@@ -388,11 +391,26 @@ class DecodeState:
         self.t = 0
         self.reset_every = int(reset_every)     # > 0: chunk-local recurrence (state zeroed at t % L == 0)
         self.n_sink = int(n_sink)               # attention sinks: the first n_sink positions
+        self.window_rec = int(window_rec)       # > 0: fixed-window recurrence over the last Lw positions
+        if self.window_rec > 0:
+            self.raw = np.zeros((3, self.BH, self.Tcap, d))     # k, v, a of every position
 
     def prefill(self, k, v, a):
         """Consume a context (BH, T, d) with the sequential recurrence and record history."""
         k, v, a = _f64(k), _f64(v), _f64(a)
         T = k.shape[-2]
+        if self.window_rec > 0:
+            Lw, t0 = self.window_rec, self.t
+            self.raw[0, :, t0:t0 + T], self.raw[1, :, t0:t0 + T], self.raw[2, :, t0:t0 + T] = k, v, a
+            lo = max(0, t0 - Lw)                  # history rows before the context, where present
+            yk = recurrence_window(self.raw[0, :, lo:t0 + T], self.raw[2, :, lo:t0 + T], Lw)[:, t0 - lo:]
+            yv = recurrence_window(self.raw[1, :, lo:t0 + T], self.raw[2, :, lo:t0 + T], Lw)[:, t0 - lo:]
+            if self.rope_base > 0:
+                yk = rope(yk, t0, self.rope_base)
+            self.khist[:, t0:t0 + T] = yk
+            self.vhist[:, t0:t0 + T] = yv
+            self.t += T
+            return
         yk, hk = recurrence(k, a, self.hk, pos0=self.t, reset_every=self.reset_every)
         yv, hv = recurrence(v, a, self.hv, pos0=self.t, reset_every=self.reset_every)
         if self.rope_base > 0:
@@ -408,6 +426,16 @@ class DecodeState:
         if self.reset_every > 0 and self.t % self.reset_every == 0:
             self.hk[:] = 0.0                    # a new block starts at this position
             self.hv[:] = 0.0
+        if self.window_rec > 0:
+            # the state entering the token: the recurrence from zero over the Lw - 1 positions
+            # before it (those that exist); the step below adds the token itself
+            t, Lw = self.t, self.window_rec
+            lo = max(0, t - Lw + 1)
+            zero = np.zeros((self.BH, self.d))
+            _, self.hk = recurrence(self.raw[0, :, lo:t], self.raw[2, :, lo:t], zero)
+            _, self.hv = recurrence(self.raw[1, :, lo:t], self.raw[2, :, lo:t], zero)
+            self.hk, self.hv = np.ascontiguousarray(self.hk), np.ascontiguousarray(self.hv)
+            self.raw[0, :, t], self.raw[1, :, t], self.raw[2, :, t] = k, v, a
         o = np.empty((self.BH, self.d))
         _load().rat_oracle_decode_step(self.BH, self.d, self.t, _ptr(self.Dbh, _ip), self.W,
                                        self.n_sink, self.scale, self.rope_base, _ptr(q), _ptr(k), _ptr(v),

@@ -825,3 +825,43 @@ def test_decode_equals_prefill_rows(rope_base, reset):
         np.testing.assert_allclose(o.reshape(B, H, d), ref["o"][:, :, t], rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(st.hk.reshape(B, H, d), ref["hT_k"], rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(st.hv.reshape(B, H, d), ref["hT_v"], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("rope_base,T0,Lw", [(0.0, 100, 64), (10000.0, 30, 64), (10000.0, 70, 8)])
+def test_window_decode_equals_prefill_rows(rope_base, T0, Lw):
+    # the fixed-window form: decoding token by token gives the attention rows of the joined
+    # sequence over the window recurrence's outputs (before and after the window fills)
+    B, H, steps, d, W = 1, 3, 50, 8, 3
+    Dh = [1, 4, 16]
+    T = T0 + steps
+    q, k, v = rand_qkv(B, H, T, d)
+    a = RNG.standard_normal((B, H, T, d)) + 2.0
+    yk = oracle.recurrence_window(k, a, Lw)
+    yv = oracle.recurrence_window(v, a, Lw)
+    qr = q
+    if rope_base > 0:
+        yk = oracle.rope(yk, 0, rope_base)
+        qr = oracle.rope(q, 0, rope_base)
+    ref = oracle.dilated_attention(qr, yk, yv, D_per_head=Dh, W=W)
+    st = oracle.DecodeState(np.tile(Dh, B), d, W, Tcap=T, rope_base=rope_base, window_rec=Lw)
+    st.prefill(k[:, :, :T0].reshape(B * H, T0, d), v[:, :, :T0].reshape(B * H, T0, d),
+               a[:, :, :T0].reshape(B * H, T0, d))
+    for s in range(steps):
+        t = T0 + s
+        o = st.step(q[:, :, t].reshape(B * H, d), k[:, :, t].reshape(B * H, d),
+                    v[:, :, t].reshape(B * H, d), a[:, :, t].reshape(B * H, d))
+        np.testing.assert_allclose(o.reshape(B, H, d), ref[:, :, t], rtol=1e-11, atol=1e-12)
+
+
+def test_window_decode_longer_than_the_sequence_is_the_full_recurrence():
+    # a window at least as long as every position's history: the full-recurrence decode
+    B, H, T0, steps, d, W = 1, 2, 20, 10, 8, 2
+    Dh = [1, 4]
+    q, k, v = rand_qkv(B, H, T0 + steps, d)
+    a = RNG.standard_normal((B, H, T0 + steps, d)) + 2.0
+    outs = []
+    for Lw in (0, 64):
+        st = oracle.DecodeState(np.tile(Dh, B), d, W, Tcap=T0 + steps, window_rec=Lw)
+        st.prefill(k[0, :, :T0], v[0, :, :T0], a[0, :, :T0])
+        outs.append([st.step(q[0, :, t], k[0, :, t], v[0, :, t], a[0, :, t]) for t in range(T0, T0 + steps)])
+    np.testing.assert_allclose(np.array(outs[1]), np.array(outs[0]), rtol=1e-12, atol=1e-13)
