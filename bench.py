@@ -484,28 +484,39 @@ def run_e2e(w, steps, warmup, x, dev, world):
 
 
 def run_decode(w: synthetic.Workload, steps_timed: int, warmup: int, rank: int, world: int, peaks,
-               peak_kind):
+               peak_kind, window_rec: int = 0):
     """Decode workload: context prefill + compress (untimed), then w.steps one-token steps per
-    timed repetition, captured in one CUDA graph and replayed."""
+    timed repetition, captured in one CUDA graph and replayed.  window_rec = 64: the
+    fixed-window recurrence (context by rat_recur_prefill_window with each chunk's history rows,
+    rat_kv_compress_window; every step reruns the recurrence over the raw ring)."""
     import recurrence_augmented_dilated_b200 as rat
     dev = torch.device("cuda")
     B, H, d, W, T0 = w.B, w.H, w.d, w.W, w.T
     nsteps = w.steps
     Tcap = T0 + nsteps
-    cache, bufs = rat.make_cache(B, H, d, W, Tcap, rat.BF16, w.heads_D())
+    cache, bufs = rat.make_cache(B, H, d, W, Tcap, rat.BF16, w.heads_D(), window_rec=window_rec)
     hk = torch.zeros((B, H, d), dtype=torch.float32, device=dev)
     hv = torch.zeros_like(hk)
     nchunks = (T0 + synthetic.CTX_CHUNK - 1) // synthetic.CTX_CHUNK
     ws_r = rat.Workspace(rat.rat_recur_workspace_bytes(B, H, synthetic.CTX_CHUNK, d, rat.BF16))
+    hist = {}
     for c in range(nchunks):
         k, v, a = synthetic.decode_context_block(w, c, device=dev, T=T0)
         kr, vr = torch.empty_like(k), torch.empty_like(v)
-        hk2, hv2 = torch.empty_like(hk), torch.empty_like(hv)
-        rat.rat_recur_prefill(k, v, a, kr, vr, ws_r, h0_k=hk, h0_v=hv, hT_k=hk2, hT_v=hv2,
-                              pos0=cache.pos, rope_base=w.rope_base)
-        rat.rat_kv_compress(kr, vr, hk2, hv2, cache)
-        hk, hv = hk2, hv2
+        if window_rec:
+            rat.rat_recur_prefill_window(k, v, a, kr, vr, ws_r, window_rec, pos0=cache.pos,
+                                         rope_base=w.rope_base, **hist)
+            rat.rat_kv_compress_window(kr, vr, k, v, a, cache)
+            hist = {n: x[:, :, -window_rec:].contiguous()
+                    for n, x in (("prev_k", k), ("prev_v", v), ("prev_gate_logit", a))}
+        else:
+            hk2, hv2 = torch.empty_like(hk), torch.empty_like(hv)
+            rat.rat_recur_prefill(k, v, a, kr, vr, ws_r, h0_k=hk, h0_v=hv, hT_k=hk2, hT_v=hv2,
+                                  pos0=cache.pos, rope_base=w.rope_base)
+            rat.rat_kv_compress(kr, vr, hk2, hv2, cache)
+            hk, hv = hk2, hv2
         del k, v, a, kr, vr
+    del hist
     del ws_r
     torch.cuda.synchronize()
     torch.cuda.empty_cache()      # only the cache and the step inputs stay on the device
@@ -514,7 +525,8 @@ def run_decode(w: synthetic.Workload, steps_timed: int, warmup: int, rank: int, 
     out = torch.empty((nsteps, B, H, 1, d), dtype=torch.bfloat16, device=dev)
     ws = rat.Workspace(rat.rat_decode_workspace_bytes(cache))
     # snapshot of the mutable cache state (state and ring), restored before every repetition
-    snap = {n: bufs[n].clone() for n in ("h_k", "h_v", "k_win", "v_win")}
+    snap = {n: bufs[n].clone() for n in ("h_k", "h_v", "k_win", "v_win") +
+            (("k_raw", "v_raw", "a_raw") if window_rec else ())}
     pos_ctx = cache.pos
 
     def reset():
@@ -561,6 +573,7 @@ def run_decode(w: synthetic.Workload, steps_timed: int, warmup: int, rank: int, 
     ms_total = max_over_ranks(sum(times) / len(times), world)
     ms_step = ms_total / nsteps
     # algorithmic bytes per step: K and V rows of every attended cache entry + the ring window
+    # (window form: + the raw k, v, a rows of the 63 positions before the token)
     eb = 2
     rows = 0
     for D in w.heads_D():
@@ -569,14 +582,18 @@ def run_decode(w: synthetic.Workload, steps_timed: int, warmup: int, rank: int, 
             rows += rat.rat_attended_keys(t, D, W) - 1      # the token itself comes from registers
     rows = rows * B / nsteps
     step_bytes = 2 * rows * d * eb
+    if window_rec:
+        step_bytes += 3 * (window_rec - 1) * B * H * d * eb
     achieved = step_bytes / (ms_step * 1e-3) / 1e9
     return {
-        "workload": w.name, "metric": "decode tokens/s", "unit": "tokens/s",
+        "workload": w.name + ("_window%d" % window_rec if window_rec else ""),
+        "metric": "decode tokens/s", "unit": "tokens/s",
         "value": world * B * nsteps / (ms_total / 1e3), "ms_per_token_step": ms_step,
         "steps_per_repetition": nsteps, "repetitions": steps_timed, "cuda_graph": True,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "of": peak_kind,
-                     "traffic": recorded_traffic("decode.cu", w.name)},
+                     "traffic": recorded_traffic("decode.cu", w.name + ("_window%d" % window_rec
+                                                                          if window_rec else ""))},
         "clocks": clk.summary(),
         "gpu_launches": nsteps * steps_timed,
     }
@@ -1046,7 +1063,8 @@ def main():
             others[name] = sub
     if not args.no_decode and not args.only:
         dw = synthetic.WORKLOADS["decode_7p6b"]
-        dec = run_decode(dw, max(1, min(args.steps, 10)), 3, rank, world, peaks, peak_kind)
+        dec = run_decode(dw, max(1, min(args.steps, 10)), 3, rank, world, peaks, peak_kind,
+                         window_rec=args.window if args.window == 64 else 0)
         if cpu_here:
             v, cores, desc, el = oracle_decode_sample(dw)
             dec["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",

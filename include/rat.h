@@ -409,11 +409,21 @@ typedef struct rat_kv_cache {
     int64_t reset_every;      /* recurrence block length L, or 0 (full sequence); >= 0     */
     int32_t n_sink;           /* attention sinks kept (first positions); 0 = none          */
     void *k_sink, *v_sink;    /* device [B][H][n_sink][d] of dtype, or NULL when n_sink == 0 */
+    int32_t window_rec;       /* 64: the fixed-window recurrence (L* = 64) decodes against
+                                 this cache (then reset_every = 0); 0: the full-sequence or
+                                 chunk-local recurrence                                    */
+    void *k_raw, *v_raw, *a_raw;  /* device [B][H][window_rec][d] of dtype: raw k, v and gate
+                                 logits of the last window_rec positions, position p in slot
+                                 p mod window_rec (rat_kv_raw_bytes each); NULL when 0      */
 } rat_kv_cache;
 
 /* Byte sizes of the buffers a cache with these fields needs (any output may be NULL). */
 RAT_API int rat_kv_cache_bytes(const rat_kv_cache *cache, size_t *dil_bytes, size_t *win_bytes,
                        size_t *state_bytes);
+
+/* Bytes of each of the three raw rings (k_raw, v_raw, a_raw) of a cache with window_rec > 0:
+ * B * H * window_rec * d * element size; 0 when window_rec is 0 or the cache is invalid. */
+RAT_API size_t rat_kv_raw_bytes(const rat_kv_cache *cache);
 
 /* rat_kv_compress -- append T positions of recurrence output to the cache.
  *   k_rec, v_rec : device (B, H, T, d) of cache->dtype: positions cache->pos .. cache->pos+T-1
@@ -421,9 +431,24 @@ RAT_API int rat_kv_cache_bytes(const rat_kv_cache *cache, size_t *dil_bytes, siz
  * Writes every position p with p mod D_h = D_h - 1 (and p / D_h < cap_h) to its dil entry, the
  * last min(W, T) positions to their ring slots and positions below n_sink to the sink rows;
  * copies the state; then advances
- * cache->pos by T on the host.  Bit-exact copies.  Requires cache->pos + T <= Tcap. */
+ * cache->pos by T on the host.  Bit-exact copies.  Requires cache->pos + T <= Tcap.  A cache with
+ * window_rec > 0 is refused (RAT_ERR_INVALID): it also needs the raw inputs, which
+ * rat_kv_compress_window takes. */
 RAT_API int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, const float *hT_v,
                     int T, rat_kv_cache *cache, void *stream);
+
+/* rat_kv_compress_window -- append T positions of the fixed-window recurrence (the outputs of
+ * rat_recur_prefill_window) to a cache with window_rec = 64 ("RAT+ Deep Dive" section 2.1,
+ * L* = 64).
+ *   k_rec, v_rec     : device (B, H, T, d) of cache->dtype, positions cache->pos .. pos + T - 1
+ *   k, v, gate_logit : device (B, H, T, d) of cache->dtype, the raw inputs of those positions
+ * Writes the chunk ends, ring and sink rows as rat_kv_compress does (the window form has no
+ * recurrence state to copy), and the raw rows of the last min(T, 64) positions to their raw
+ * ring slots; then advances cache->pos by T on the host.  Bit-exact copies.  RAT_ERR_INVALID for
+ * a cache without window_rec = 64 or cache->pos + T > Tcap. */
+RAT_API int rat_kv_compress_window(const void *k_rec, const void *v_rec, const void *k,
+                    const void *v, const void *gate_logit, int T, rat_kv_cache *cache,
+                    void *stream);
 
 /* ------------------------------------------------------------------------------------------
  * rat_dilated_decode -- one new token per sequence against the compressed cache.
@@ -432,7 +457,9 @@ RAT_API int rat_kv_compress(const void *k_rec, const void *v_rec, const float *h
  *   rope_base, scale    : as in prefill (rope_base must match the one used for the cache)
  *   ws, ws_bytes        : workspace of at least rat_decode_workspace_bytes(cache)
  * Per (b, h): state update h = g h + (1-g) x for k and v (h taken as 0 first when
- * cache->reset_every = L > 0 and t mod L = 0); k~_t = RoPE(h_k, t); append k~_t, v~_t
+ * cache->reset_every = L > 0 and t mod L = 0; with window_rec = 64, h is instead the
+ * recurrence rerun from zero over the raw rows of positions max(0, t-63) .. t-1, and the
+ * token's raw k, v, gate logit go to raw slot t mod 64); k~_t = RoPE(h_k, t); append k~_t, v~_t
  * to the dil cache if t mod D_h = D_h - 1, to ring slot t mod W and to the sink rows if
  * t < n_sink; then attention of RoPE(q, t) over the dil entries with position <= t - We, the
  * ring positions t-We < j < t, the sinks older than the window that are not chunk ends, and the

@@ -26,7 +26,8 @@ __all__ = [
     "rat_recur_backward_workspace_bytes",
     "rat_dilated_attn_backward", "rat_dilated_attn_backward_workspace_bytes",
     "rat_dilated_attn_prefill",
-    "rat_kv_cache_bytes", "rat_kv_compress", "rat_decode_workspace_bytes", "rat_dilated_decode",
+    "rat_kv_cache_bytes", "rat_kv_compress", "rat_kv_compress_window", "rat_kv_raw_bytes",
+    "rat_decode_workspace_bytes", "rat_dilated_decode",
     "rat_workspace_init", "rat_sync_status", "rat_attn_sync_status", "rat_set_attn_block_keys", "rat_attended_keys", "rat_status_string",
     "Workspace", "rat_dilated_decode_noalloc", "PagedKVCache", "make_paged_cache", "AttnOptions",
     "rat_paged_kv_compress", "rat_paged_decode_workspace_bytes", "rat_dilated_decode_paged",
@@ -57,6 +58,8 @@ class KVCache(ctypes.Structure):
         ("h_k", ctypes.c_void_p), ("h_v", ctypes.c_void_p),
         ("pos", ctypes.c_int64), ("reset_every", ctypes.c_int64),
         ("n_sink", ctypes.c_int32), ("k_sink", ctypes.c_void_p), ("v_sink", ctypes.c_void_p),
+        ("window_rec", ctypes.c_int32), ("k_raw", ctypes.c_void_p), ("v_raw", ctypes.c_void_p),
+        ("a_raw", ctypes.c_void_p),
     ]
 
 
@@ -128,6 +131,9 @@ def lib():
         L.rat_kv_cache_bytes.argtypes = [ctypes.POINTER(KVCache), ctypes.POINTER(_sz),
                                          ctypes.POINTER(_sz), ctypes.POINTER(_sz)]
         L.rat_kv_compress.argtypes = [_vp, _vp, _vp, _vp, _i, ctypes.POINTER(KVCache), _vp]
+        L.rat_kv_compress_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _i, ctypes.POINTER(KVCache), _vp]
+        L.rat_kv_raw_bytes.restype = _sz
+        L.rat_kv_raw_bytes.argtypes = [ctypes.POINTER(KVCache)]
         L.rat_decode_workspace_bytes.restype = _sz
         L.rat_decode_workspace_bytes.argtypes = [ctypes.POINTER(KVCache)]
         L.rat_dilated_decode.argtypes = [_vp, _vp, _vp, _vp, ctypes.POINTER(KVCache), _vp, _f, _f,
@@ -352,13 +358,14 @@ def rat_dilated_attn_backward(q, k_rec, v_rec, o, dO, dq, dk_rec, dv_rec, ws: Wo
 
 
 def make_cache(B, H, d, W, Tcap, dtype: int, D_per_head: Sequence[int], device="cuda",
-               reset_every: int = 0, n_sink: int = 0):
+               reset_every: int = 0, n_sink: int = 0, window_rec: int = 0):
     """Allocate (with torch) the buffers of a compressed cache and return (KVCache, buffers).
     reset_every = L > 0 selects the chunk-local recurrence for the decode steps; n_sink > 0
-    keeps the first n_sink positions as attention sinks."""
+    keeps the first n_sink positions as attention sinks; window_rec = 64 selects the
+    fixed-window recurrence (raw rings of the last 64 positions' k, v and gate logits)."""
     Dh = (ctypes.c_int32 * H)(*[int(x) for x in D_per_head])
     c = KVCache(B=B, H=H, d=d, W=W, Tcap=Tcap, dtype=dtype, D=Dh, reset_every=int(reset_every),
-                n_sink=int(n_sink))
+                n_sink=int(n_sink), window_rec=int(window_rec))
     dil, win, state = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
     _check("rat_kv_cache_bytes", lib().rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(dil),
                                                           ctypes.byref(win), ctypes.byref(state)))
@@ -376,12 +383,16 @@ def make_cache(B, H, d, W, Tcap, dtype: int, D_per_head: Sequence[int], device="
         "v_sink": torch.zeros((B, H, max(n_sink, 1), d), dtype=tdt, device=device),
         "D": Dh,
     }
+    for n in ("k_raw", "v_raw", "a_raw"):
+        bufs[n] = torch.zeros((B, H, max(window_rec, 1), d), dtype=tdt, device=device)
     c.k_dil, c.v_dil = bufs["k_dil"].data_ptr(), bufs["v_dil"].data_ptr()
     c.k_win = bufs["k_win"].data_ptr() if W > 0 else None
     c.v_win = bufs["v_win"].data_ptr() if W > 0 else None
     c.h_k, c.h_v = bufs["h_k"].data_ptr(), bufs["h_v"].data_ptr()
     c.k_sink = bufs["k_sink"].data_ptr() if n_sink > 0 else None
     c.v_sink = bufs["v_sink"].data_ptr() if n_sink > 0 else None
+    if window_rec > 0:
+        c.k_raw, c.v_raw, c.a_raw = (bufs[n].data_ptr() for n in ("k_raw", "v_raw", "a_raw"))
     c.pos = 0
     return c, bufs
 
@@ -398,6 +409,19 @@ def rat_kv_compress(k_rec, v_rec, hT_k, hT_v, cache: KVCache, stream=None):
     st = lib().rat_kv_compress(_ptr(k_rec), _ptr(v_rec), _ptr(hT_k), _ptr(hT_v), T,
                                ctypes.byref(cache), _stream(stream))
     _check("rat_kv_compress", st)
+
+
+def rat_kv_compress_window(k_rec, v_rec, k, v, gate_logit, cache: KVCache, stream=None):
+    """Append positions of the fixed-window recurrence (outputs and raw inputs) to a cache made
+    with window_rec = 64."""
+    T = k_rec.shape[2]
+    st = lib().rat_kv_compress_window(_ptr(k_rec), _ptr(v_rec), _ptr(k), _ptr(v), _ptr(gate_logit),
+                                      T, ctypes.byref(cache), _stream(stream))
+    _check("rat_kv_compress_window", st)
+
+
+def rat_kv_raw_bytes(cache: KVCache) -> int:
+    return int(lib().rat_kv_raw_bytes(ctypes.byref(cache)))
 
 
 def rat_decode_workspace_bytes(cache: KVCache) -> int:

@@ -14,7 +14,10 @@
 // slice are split over `splits` CTAs; each CTA keeps an online softmax per 16-lane group,
 // merges its groups and warps, and writes (max, sum, o) to the workspace; the last CTA of the
 // slice (atomic ticket, no waiting) merges the splits by log-sum-exp and resets the ticket.
-// Split 0 alone does steps 1-2 and adds the token itself to its softmax.
+// Split 0 alone does steps 1-2 and adds the token itself to its softmax.  With the fixed-window
+// recurrence ("RAT+ Deep Dive" section 2.1, L* = 64) step 1 reruns the recurrence from zero over
+// the raw rows of the 63 positions before t (a raw ring in the cache) instead of reading a
+// carried state, and the token's raw rows take the ring slot of position t - 64.
 // No CTA reads what another writes in the same launch: the new dil entry (position t) is never
 // older than the window, and the ring slot written held position t - W, outside the window.
 #include <mutex>
@@ -32,6 +35,10 @@ RAT_DEVICE void load8(const void *p, float *x) {      // 8 bf16 -> float
     x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
     x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
 }
+RAT_DEVICE void unpack8(uint4 u, float *x) {          // 8 bf16 -> float
+    x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+    x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
+}
 RAT_DEVICE uint4 pack8(const float *x) {
     return make_uint4(pack_bf16(x[0], x[1]), pack_bf16(x[2], x[3]), pack_bf16(x[4], x[5]),
                       pack_bf16(x[6], x[7]));
@@ -42,7 +49,8 @@ RAT_DEVICE uint4 pack8(const float *x) {
 // dilated entries live in pages of a pool found through a page table, and every sequence has
 // its own position (read from seq_pos, advanced by the last CTA of the sequence).
 // SINKS: the first n_sink positions are kept in sink rows and join every key set.
-template <int DH, bool PAGED, bool SINKS>
+// WINDOW: the fixed-window recurrence (raw rings; p.window_rec > 0).
+template <int DH, bool PAGED, bool SINKS, bool WINDOW>
 __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int LPR = DH / 8;                 // lanes per key row
     constexpr int GPW = 32 / LPR;               // key groups per warp
@@ -107,6 +115,56 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
     float m = -INFINITY, l = 0.f, o[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) o[j] = 0.f;
+
+    // fixed-window form, split 0: the affine map of the raw rows max(0, t - Lw + 1) .. t - 1 (the
+    // recurrence from zero over them), composed in kWarps * GPW segments, one per lane group with
+    // all its rows' loads in flight; warp 0 folds the segments in order below
+    constexpr int kSegs = kWarps * (32 / (DH / 8));
+    __shared__ float s_wa[WINDOW ? kSegs : 1][DH], s_wk[WINDOW ? kSegs : 1][DH], s_wv[WINDOW ? kSegs : 1][DH];
+    if (WINDOW && split == 0) {
+        const int seg = warp * GPW + grp;
+        const long long lo = max(0ll, t - p.window_rec + 1), n = t - lo;
+        const long long r0 = lo + n * seg / kSegs, r1 = lo + n * (seg + 1) / kSegs;
+        constexpr int kMaxSeg = (kWindowRows + kSegs - 1) / kSegs;      // rows per segment
+        uint4 ra[kMaxSeg], rk[kMaxSeg], rv[kMaxSeg];
+        const size_t ring = (size_t)bh * p.window_rec;
+#pragma unroll
+        for (int i = 0; i < kMaxSeg; ++i) {
+            if (r0 + i < r1) {
+                const size_t off = (ring + (size_t)((r0 + i) % p.window_rec)) * RB + cl * 16;
+                ra[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.araw) + off));
+                rk[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.kraw) + off));
+                rv[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.vraw) + off));
+            }
+        }
+        float A[8], K[8], V[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { A[j] = 1.f; K[j] = 0.f; V[j] = 0.f; }
+#pragma unroll
+        for (int i = 0; i < kMaxSeg; ++i) {
+            if (r0 + i < r1) {
+                float fa[8], fk[8], fv[8];
+                unpack8(ra[i], fa);
+                unpack8(rk[i], fk);
+                unpack8(rv[i], fv);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float g, omg;
+                    forget_gate(fa[j], g, omg);
+                    K[j] = fmaf(g, K[j], omg * fk[j]);
+                    V[j] = fmaf(g, V[j], omg * fv[j]);
+                    A[j] *= g;
+                }
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {      // both lanes of a pair hold the same group values
+            s_wa[seg][cl * 8 + j] = A[j];
+            s_wk[seg][cl * 8 + j] = K[j];
+            s_wv[seg][cl * 8 + j] = V[j];
+        }
+        __syncthreads();                   // split is uniform over the CTA
+    }
 
     // keys of this split: lane set s = warp*GPW + grp takes keys k_lo + s + m*kLanesets, KPI at a
     // time (their K and V rows in flight together, kept as packed bf16).  The loop runs on the
@@ -196,21 +254,45 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 
     // split 0: recurrence update, cache append, and the token itself as a key (group 0 of warp 0)
     if (split == 0 && warp == 0) {
+        const uint4 ku = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.k) + (size_t)bh * RB + cl * 16));
+        const uint4 vu = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.v) + (size_t)bh * RB + cl * 16));
+        const uint4 au = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.a) + (size_t)bh * RB + cl * 16));
         float kn[8], vn[8], an[8];
-        load8(static_cast<const uint8_t *>(p.k) + (size_t)bh * RB + cl * 16, kn);
-        load8(static_cast<const uint8_t *>(p.v) + (size_t)bh * RB + cl * 16, vn);
-        load8(static_cast<const uint8_t *>(p.a) + (size_t)bh * RB + cl * 16, an);
+        unpack8(ku, kn);
+        unpack8(vu, vn);
+        unpack8(au, an);
         float *hk = p.hk + (size_t)bh * DH + cl * 8;
         float *hv = p.hv + (size_t)bh * DH + cl * 8;
-        // chunk-local recurrence: the state is dropped before every position that starts a block
-        const bool fresh = p.reset > 0 && t % p.reset == 0;
+        // the state entering position t: the cache's (0 before a block start of the chunk-local
+        // recurrence), or, for the fixed-window form, the recurrence rerun from zero over the raw
+        // rows of positions max(0, t - Lw + 1) .. t - 1
+        float hsk[8], hsv[8];
+        if constexpr (WINDOW) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) { hsk[j] = 0.f; hsv[j] = 0.f; }
+            for (int sg = 0; sg < kSegs; ++sg) {       // the segments' maps, oldest first
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int c = cl * 8 + j;
+                    hsk[j] = fmaf(s_wa[sg][c], hsk[j], s_wk[sg][c]);
+                    hsv[j] = fmaf(s_wa[sg][c], hsv[j], s_wv[sg][c]);
+                }
+            }
+        } else {
+            const bool fresh = p.reset > 0 && t % p.reset == 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                hsk[j] = fresh ? 0.f : hk[j];
+                hsv[j] = fresh ? 0.f : hv[j];
+            }
+        }
         float sk[8], sv[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             float g, omg;
             forget_gate(an[j], g, omg);
-            sk[j] = fresh ? omg * kn[j] : fmaf(g, hk[j], omg * kn[j]);
-            sv[j] = fresh ? omg * vn[j] : fmaf(g, hv[j], omg * vn[j]);
+            sk[j] = fmaf(g, hsk[j], omg * kn[j]);
+            sv[j] = fmaf(g, hsv[j], omg * vn[j]);
         }
         float kt[8];
 #pragma unroll
@@ -247,6 +329,12 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
                 uint8_t *vs = static_cast<uint8_t *>(p.vsink) + ((size_t)bh * p.n_sink + (size_t)t) * RB;
                 *reinterpret_cast<uint4 *>(ks + cl * 16) = kpk;
                 *reinterpret_cast<uint4 *>(vs + cl * 16) = vpk;
+            }
+            if (WINDOW) {                    // the token's raw rows: slot t mod Lw held t - Lw
+                const size_t off = ((size_t)bh * p.window_rec + (size_t)(t % p.window_rec)) * RB + cl * 16;
+                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.kraw) + off) = ku;
+                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.vraw) + off) = vu;
+                *reinterpret_cast<uint4 *>(static_cast<uint8_t *>(p.araw) + off) = au;
             }
             if (p.W > 0) {
                 uint8_t *kw = static_cast<uint8_t *>(p.kwin) + ((size_t)bh * p.W + (size_t)(t % p.W)) * RB;
@@ -370,14 +458,20 @@ int launch_decode(const DecodeParams &p, int dtype, void *stream, bool paged) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool sinks = p.n_sink > 0;
     if (paged && sinks) return RAT_ERR_UNSUPPORTED;
+    const bool window = p.window_rec > 0;
+    if (paged && window) return RAT_ERR_UNSUPPORTED;
     if (p.d == 128) {
-        if (paged) decode_kernel<128, true, false><<<grid, kThreads, 0, s>>>(p);
-        else if (sinks) decode_kernel<128, false, true><<<grid, kThreads, 0, s>>>(p);
-        else decode_kernel<128, false, false><<<grid, kThreads, 0, s>>>(p);
+        if (paged) decode_kernel<128, true, false, false><<<grid, kThreads, 0, s>>>(p);
+        else if (window && sinks) decode_kernel<128, false, true, true><<<grid, kThreads, 0, s>>>(p);
+        else if (window) decode_kernel<128, false, false, true><<<grid, kThreads, 0, s>>>(p);
+        else if (sinks) decode_kernel<128, false, true, false><<<grid, kThreads, 0, s>>>(p);
+        else decode_kernel<128, false, false, false><<<grid, kThreads, 0, s>>>(p);
     } else if (p.d == 64) {
-        if (paged) decode_kernel<64, true, false><<<grid, kThreads, 0, s>>>(p);
-        else if (sinks) decode_kernel<64, false, true><<<grid, kThreads, 0, s>>>(p);
-        else decode_kernel<64, false, false><<<grid, kThreads, 0, s>>>(p);
+        if (paged) decode_kernel<64, true, false, false><<<grid, kThreads, 0, s>>>(p);
+        else if (window && sinks) decode_kernel<64, false, true, true><<<grid, kThreads, 0, s>>>(p);
+        else if (window) decode_kernel<64, false, false, true><<<grid, kThreads, 0, s>>>(p);
+        else if (sinks) decode_kernel<64, false, true, false><<<grid, kThreads, 0, s>>>(p);
+        else decode_kernel<64, false, false, false><<<grid, kThreads, 0, s>>>(p);
     } else {
         return RAT_ERR_UNSUPPORTED;
     }

@@ -199,6 +199,8 @@ int launch_attn_bwd_sm100(const AttnBwdParams &p, void *stream);
 struct DecodeParams {
     const void *q, *k, *v, *a;
     void *o;
+    int window_rec;             // > 0: the fixed-window recurrence over raw rings of window_rec rows
+    void *kraw, *vraw, *araw;   // [B*H][window_rec][d] raw k, v, gate logits, slot p mod window_rec
     void *kdil, *vdil, *kwin, *vwin;
     float *hk, *hv;
     int B, H, d, W, Tcap, splits;

@@ -4,6 +4,7 @@
 // work is enqueued on the caller's stream.  No entry point allocates device memory.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -38,9 +39,18 @@ bool valid_cache(const rat_kv_cache *c) {
     if (!c || c->B < 1 || c->H < 1 || c->H > kMaxHeads || !supported_d(c->d) || c->W < 0 ||
         c->Tcap < 1 || !valid_dtype(c->dtype) || !c->D || c->reset_every < 0 || c->n_sink < 0)
         return false;
+    // the fixed-window form (L* = 64) has no chunk-local restarts
+    if (c->window_rec != 0 && c->window_rec != kWindowRows) return false;
+    if (c->window_rec > 0 && c->reset_every != 0) return false;
     for (int h = 0; h < c->H; ++h)
         if (c->D[h] < 1) return false;
     return true;
+}
+
+// the raw rings of a cache with window_rec > 0 (none needed otherwise)
+bool raw_rings_ok(const rat_kv_cache *c) {
+    return c->window_rec == 0 || (c->k_raw && c->v_raw && c->a_raw && aligned16(c->k_raw) &&
+                                  aligned16(c->v_raw) && aligned16(c->a_raw));
 }
 
 bool valid_paged_cache(const rat_paged_kv_cache *c) {
@@ -495,7 +505,14 @@ int rat_kv_cache_bytes(const rat_kv_cache *c, size_t *dil_bytes, size_t *win_byt
     return RAT_OK;
 }
 
-int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, const float *hT_v,
+size_t rat_kv_raw_bytes(const rat_kv_cache *c) {
+    if (!valid_cache(c) || c->window_rec == 0) return 0;
+    return (size_t)c->B * c->H * c->window_rec * c->d * esize(c->dtype);
+}
+
+namespace {
+// the chunk ends, ring and sink rows of T positions (and the state when hT is given)
+int compress_common(const void *k_rec, const void *v_rec, const float *hT_k, const float *hT_v,
                     int T, rat_kv_cache *c, void *stream) {
     if (!valid_cache(c) || T < 0) return RAT_ERR_INVALID;
     if (c->pos < 0 || c->pos + T > c->Tcap) return RAT_ERR_INVALID;
@@ -518,9 +535,48 @@ int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, con
     p.ksink = c->k_sink; p.vsink = c->v_sink; p.n_sink = c->n_sink;
     for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
     p.total_cap = total_capacity(c->H, c->Tcap, c->D, p.off);
-    const int st = launch_compress(p, stream);
+    return launch_compress(p, stream);
+}
+}  // namespace
+
+int rat_kv_compress(const void *k_rec, const void *v_rec, const float *hT_k, const float *hT_v,
+                    int T, rat_kv_cache *c, void *stream) {
+    if (!valid_cache(c) || c->window_rec != 0) return RAT_ERR_INVALID;
+    const int st = compress_common(k_rec, v_rec, hT_k, hT_v, T, c, stream);
     if (st == RAT_OK) c->pos += T;
     return st;
+}
+
+int rat_kv_compress_window(const void *k_rec, const void *v_rec, const void *k, const void *v,
+                           const void *gate_logit, int T, rat_kv_cache *c, void *stream) {
+    if (!valid_cache(c) || c->window_rec == 0 || T < 0 || !raw_rings_ok(c)) return RAT_ERR_INVALID;
+    if (c->pos < 0 || c->pos + T > c->Tcap) return RAT_ERR_INVALID;
+    if (T == 0) return RAT_OK;
+    if (!k || !v || !gate_logit || !aligned16(k) || !aligned16(v) || !aligned16(gate_logit))
+        return RAT_ERR_INVALID;
+    int st = compress_common(k_rec, v_rec, nullptr, nullptr, T, c, stream);
+    if (st != RAT_OK) return st;
+    // raw rows of the last min(T, Lw) positions P .. pos+T-1 into slots p mod Lw: at most two
+    // runs of slots (before and after the wrap), each one strided copy over every (b, h) slice
+    const long long Lw = c->window_rec, end = c->pos + T, first = end - (T < Lw ? T : Lw);
+    const size_t row = (size_t)c->d * esize(c->dtype);
+    const void *src[3] = {k, v, gate_logit};
+    void *dst[3] = {c->k_raw, c->v_raw, c->a_raw};
+    const size_t slices = (size_t)c->B * c->H;
+    for (long long p0 = first; p0 < end;) {
+        const long long slot = p0 % Lw;
+        const long long n = std::min(end - p0, Lw - slot);        // up to the end of the ring
+        for (int i = 0; i < 3; ++i) {
+            const uint8_t *s = static_cast<const uint8_t *>(src[i]) + (size_t)(p0 - c->pos) * row;
+            uint8_t *d = static_cast<uint8_t *>(dst[i]) + (size_t)slot * row;
+            if (cudaMemcpy2DAsync(d, (size_t)Lw * row, s, (size_t)T * row, (size_t)n * row, slices,
+                                  cudaMemcpyDeviceToDevice, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+                return RAT_ERR_CUDA;
+        }
+        p0 += n;
+    }
+    c->pos += T;
+    return RAT_OK;
 }
 
 // ------------------------------------------------------------------------------ decode
@@ -613,7 +669,7 @@ int rat_dilated_decode_paged(const void *q, const void *k, const void *v, const 
 int rat_dilated_decode(const void *q, const void *k, const void *v, const void *gate_logit,
                        rat_kv_cache *c, void *o, float rope_base, float scale, void *ws,
                        size_t ws_bytes, void *stream) {
-    if (!valid_cache(c)) return RAT_ERR_INVALID;
+    if (!valid_cache(c) || !raw_rings_ok(c)) return RAT_ERR_INVALID;
     if (c->dtype != RAT_BF16) return RAT_ERR_UNSUPPORTED;
     if (!q || !k || !v || !gate_logit || !o) return RAT_ERR_INVALID;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(gate_logit) || !aligned16(o))
@@ -638,6 +694,8 @@ int rat_dilated_decode(const void *q, const void *k, const void *v, const void *
     p.t = c->pos;
     p.reset = c->reset_every;
     p.ksink = c->k_sink; p.vsink = c->v_sink; p.n_sink = c->n_sink;
+    p.window_rec = c->window_rec;
+    p.kraw = c->k_raw; p.vraw = c->v_raw; p.araw = c->a_raw;
     for (int h = 0; h < c->H; ++h) p.Dh[h] = c->D[h];
     p.total_cap = total_capacity(c->H, c->Tcap, c->D, p.off);
     p.rope = rope_base > 0.f ? 1 : 0;

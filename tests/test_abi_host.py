@@ -215,6 +215,38 @@ def test_cache_rejects_negative_block_length(L):
     assert L.rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(sz), None, None) == 0
 
 
+def test_window_cache_validation(L):
+    # the fixed-window form: window_rec 64 only, no chunk-local restarts, raw rings required by
+    # the calls that use them (not by the size helpers)
+    P = ctypes.c_void_p
+    c = cache()
+    c.window_rec = 64
+    assert rat.rat_kv_raw_bytes(c) == 2 * 2 * 64 * 128 * 2
+    sz = ctypes.c_size_t()
+    assert L.rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(sz), None, None) == 0
+    c.window_rec = 32
+    assert rat.rat_kv_raw_bytes(c) == 0
+    assert L.rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(sz), None, None) == -1
+    c.window_rec = 64
+    c.reset_every = 16
+    assert L.rat_kv_cache_bytes(ctypes.byref(c), ctypes.byref(sz), None, None) == -1
+    c.reset_every = 0
+    c.k_dil = c.v_dil = c.k_win = c.v_win = c.h_k = c.h_v = 256
+    # raw rings missing: refused by the window compress and by decode
+    assert L.rat_kv_compress_window(P(256), P(256), P(256), P(256), P(256), 10, ctypes.byref(c), None) == -1
+    ws = P(256 * 4096)
+    assert L.rat_dilated_decode(P(256), P(256), P(256), P(256), ctypes.byref(c), P(256), 0.0, 0.0,
+                                ws, 1 << 30, None) == -1
+    # the plain compress refuses a window cache even with its rings
+    c.k_raw = c.v_raw = c.a_raw = 256
+    assert L.rat_kv_compress(P(256), P(256), None, None, 10, ctypes.byref(c), None) == -1
+    # and the window compress refuses a cache without the window form
+    c2 = cache()
+    c2.k_dil = c2.v_dil = c2.k_win = c2.v_win = c2.h_k = c2.h_v = 256
+    assert L.rat_kv_compress_window(P(256), P(256), P(256), P(256), P(256), 10, ctypes.byref(c2), None) == -1
+    assert rat.rat_kv_raw_bytes(c2) == 0
+
+
 def paged(**kw):
     D = (ctypes.c_int32 * kw.get("H", 2))(*kw.get("Dlist", [1, 64]))
     c = rat.PagedKVCache(B=kw.get("B", 2), H=kw.get("H", 2), d=kw.get("d", 128), W=kw.get("W", 16),

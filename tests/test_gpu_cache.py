@@ -161,3 +161,71 @@ def test_decode_local_recurrence(L):
                            reset_every=L)
     assert err <= TOL_BF16, err
     assert herr <= TOL_F32, herr
+
+
+# ---- decode with the fixed-window recurrence (L* = 64): raw rings of the last 64 positions
+def run_window_decode(w, T0, steps, chunk, rope_base=0.0):
+    """GPU: the context prefilled in chunks by rat_recur_prefill_window (each chunk with the 64
+    raw rows before it as history) and appended by rat_kv_compress_window, then `steps` decode
+    tokens.  Oracle: DecodeState(window_rec=64) from the same raw inputs on every slice."""
+    B, H, d, W = w.B, w.H, w.d, w.W
+    Dh = w.heads_D()
+    Tcap = T0 + steps
+    dev = torch.device("cuda")
+    cache, bufs = rat.make_cache(B, H, d, W, Tcap, rat.BF16, Dh, window_rec=64)
+    for n in ("k_raw", "v_raw", "a_raw"):
+        bufs[n].fill_(POISON)
+    x = synthetic.prefill_inputs(w, T=T0)
+    ws = rat.Workspace(256)
+    for lo in range(0, T0, chunk):
+        hi = min(T0, lo + chunk)
+        k, v, a = (x[n][:, :, lo:hi].contiguous().to(dev) for n in ("k", "v", "a"))
+        kr, vr = torch.empty_like(k), torch.empty_like(v)
+        prev = {}
+        if lo >= 64:
+            prev = {n: x[m][:, :, lo - 64:lo].contiguous().to(dev)
+                    for n, m in (("prev_k", "k"), ("prev_v", "v"), ("prev_gate_logit", "a"))}
+        rat.rat_recur_prefill_window(k, v, a, kr, vr, ws, 64, pos0=lo, rope_base=rope_base, **prev)
+        rat.rat_kv_compress_window(kr, vr, k, v, a, cache)
+    assert rat.rat_sync_status(ws) == 0
+    assert cache.pos == T0
+    # the raw rings hold the last 64 raw rows, position p in slot p mod 64, bit for bit
+    for n, m in (("k_raw", "k"), ("v_raw", "v"), ("a_raw", "a")):
+        exp = torch.full((B, H, 64, d), POISON, dtype=torch.bfloat16)
+        for p in range(max(0, T0 - 64), T0):
+            exp[:, :, p % 64] = x[m][:, :, p]
+        assert torch.equal(bufs[n].cpu(), exp), n
+    tok = synthetic.decode_steps(w, steps)
+    wsd = rat.Workspace(rat.rat_decode_workspace_bytes(cache))
+    st = oracle.DecodeState([Dh[h] for b in range(B) for h in range(H)], d, W, Tcap,
+                            rope_base=rope_base, window_rec=64)
+    st.prefill(f64(x["k"]).reshape(B * H, T0, d), f64(x["v"]).reshape(B * H, T0, d),
+               f64(x["a"]).reshape(B * H, T0, d))
+    worst = 0.0
+    for s in range(steps):
+        o = torch.empty((B, H, 1, d), dtype=torch.bfloat16, device=dev)
+        args = [tok[n][s].reshape(B, H, 1, d).to(dev) for n in ("q", "k", "v", "a")]
+        rat.rat_dilated_decode(*args, cache, o, wsd, rope_base=rope_base)
+        ref = st.step(*(f64(tok[n][s]).reshape(B * H, d) for n in ("q", "k", "v", "a")))
+        worst = max(worst, rel_err(o.reshape(B * H, d), ref))
+    assert rat.rat_sync_status(wsd) == 0
+    assert cache.pos == Tcap
+    return worst
+
+
+@pytest.mark.parametrize("T0,chunk,rope_base", [(200, 200, 0.0), (300, 128, 10000.0), (40, 40, 10000.0)])
+def test_window_decode(T0, chunk, rope_base):
+    # contexts longer than the window (in one chunk and in three), and shorter than it (the
+    # window still filling during the decode steps)
+    w = synthetic.Workload("wdec", B=2, H=3, d=128, T=T0, W=8, D_per_head=(1, 4, 16),
+                           dtype="bf16", seed=T0 + chunk)
+    assert run_window_decode(w, T0, 70, chunk, rope_base) <= TOL_BF16
+
+
+def test_window_cache_refuses_the_plain_compress():
+    # a window cache must also receive the raw rows: rat_kv_compress refuses it
+    cache, _ = rat.make_cache(1, 1, 128, 4, 100, rat.BF16, [4], window_rec=64)
+    x = torch.zeros((1, 1, 10, 128), dtype=torch.bfloat16, device="cuda")
+    h = torch.zeros((1, 1, 128), device="cuda")
+    with pytest.raises(rat.RatError):
+        rat.rat_kv_compress(x, x, h, h, cache)
