@@ -205,8 +205,8 @@ RAT_API int rat_recur_backward_local(const void *k, const void *v, const void *g
 /* ------------------------------------------------------------------------------------------
  * rat_recur_prefill_window -- the fixed-window recurrence of RAT+: each state covers only the
  * last Lw positions.
- *   "RAT+ Deep Dive" section 2.1 (a fixed recurrence window L* = 64, looking back 64 tokens
- *   from the current one, computed in parallel in prefill).  Read as: the state at t is the
+ *   "RAT+ Deep Dive" section 2.1 (a fixed recurrence window L* = 64: each token's recurrence
+ *   reaches 64 positions back, and prefill computes it in parallel).  Read as: the state at t is the
  *   recurrence restarted from zero at t - Lw + 1,
  *     y_t = sum_{s = t-Lw+1}^{t} ( prod_{r = s+1}^{t} g_r ) (1 - g_s) x_s,   g = sigmoid(a),
  *   for x = k and x = v with the same gate, in float32; k~ = RoPE(y^k) when rope_base > 0.
@@ -270,7 +270,7 @@ RAT_API int rat_dilated_attn_prefill(const void *q, const void *k_rec, const voi
 
 /* rat_dilated_attn_prefill_sinks -- the same attention with attention sinks: the first n_sink
  * positions join every key set (StreamingLLM layers; "RAT+ Deep Dive" section 6, layer-wise
- * hybrid: "odd layers StreamingLLM").  Each key counts once (a sink already in the window or a
+ * hybrid, where the odd layers are StreamingLLM layers).  Each key counts once (a sink already in the window or a
  * chunk end is not repeated).  A StreamingLLM layer is D larger than any position (no chunk
  * ends), W its window, n_sink its sinks; sinks also combine with dilation.
  *   Arguments as rat_dilated_attn_prefill, plus n_sink >= 0 (0: exactly
@@ -283,8 +283,8 @@ RAT_API int rat_dilated_attn_prefill_sinks(const void *q, const void *k_rec, con
                              float rope_base, float scale, void *stream);
 
 /* rat_dilated_attn_prefill_topk -- the attention with top-k chunk selection combined with the
- * dilation ("RAT+ Deep Dive" section 4: "dilation provides global coverage while top-k increases
- * local density").  Read as: the blocks are the dilation's chunks [cD, cD + D - 1]; each chunk
+ * dilation ("RAT+ Deep Dive" section 4: dilation reaches the whole sequence, the selected blocks
+ * add dense local detail).  Read as: the blocks are the dilation's chunks [cD, cD + D - 1]; each chunk
  * wholly older than the window (cD + D - 1 <= t - We) is scored by its chunk-end key (the
  * recurrence state that sums the chunk up), s_c = scale <q^_t, k~_{cD+D-1}>; every position of
  * the top_k best chunks (ties: the earlier chunk) joins S(t) and the sinks, each key once.

@@ -19,9 +19,9 @@
  *                     chunk ends).
  *   [RoFormer]        rotary position embedding, cited by the RAT+ page; rotate-half pairing.
  *
- * The recurrence formula itself is lost from the blog's section 2.1 (only "forget-gate
- * mechanism ... g_l is an input-dependent forget gate, LSTM-like decaying memory" survives);
- * the form used here is the standard gated EMA  h_t = g_t * h_{t-1} + (1 - g_t) * x_t with
+ * The recurrence formula itself is lost from the blog's section 2.1: the text keeps only that
+ * the recurrence uses a forget gate which depends on the input and decays memory as an LSTM
+ * does; the form used here is the standard gated EMA  h_t = g_t * h_{t-1} + (1 - g_t) * x_t with
  * g_t = sigmoid(a_t), elementwise per channel, the same gate for keys and values.
  *
  * Readings taken where the pages are silent (each one is listed in the design notes):
@@ -74,9 +74,9 @@ void rat_oracle_recurrence(long BH, long T, long d, const double *x, const doubl
 }
 
 /*
- * Chunk-local recurrence of the predecessor RAT ("RAT+ Deep Dive" section 2.1: the original RAT
- * splits the sequence into blocks of size L and each token recurses only within its block; the
- * RAT paper's abstract: recurrence within each chunk).  Same step as above, but the state is
+ * Chunk-local recurrence of the predecessor RAT ("RAT+ Deep Dive" section 2.1: in the original
+ * RAT the recurrence of a token stays inside its own block of L positions; the RAT paper's
+ * abstract: recurrence within each chunk).  Same step as above, but the state is
  * set to zero before every absolute position p = pos0 + t with p mod L == 0 (L > 0), so each
  * block of L positions starts from an empty state.  h0 is the state before pos0 (dropped when
  * pos0 itself starts a block).
@@ -348,8 +348,8 @@ void rat_oracle_dilated_attention(long BH, long T, long d, const double *q, cons
 
 /*
  * Dilated attention with top-k chunk selection ("RAT+ Deep Dive" section 4: dilation combined
- * with top-k block selection, "dilation provides global coverage while top-k increases local
- * density").  Read as: the blocks are the dilation's chunks c = [cD, cD + D - 1]; a chunk wholly
+ * with top-k block selection, dilation reaching the whole sequence and the selected blocks adding
+ * dense local detail).  Read as: the blocks are the dilation's chunks c = [cD, cD + D - 1]; a chunk wholly
  * older than the window (cD + D - 1 <= t - We) is scored by its chunk-end key,
  * s_c = scale * <q_t, k_{cD+D-1}>; the top_k highest-scoring chunks (ties: the earlier chunk)
  * are attended at every position, on top of S(t) (and the sinks), each key once.

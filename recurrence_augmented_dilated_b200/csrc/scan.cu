@@ -1,7 +1,8 @@
 // scan.cu -- full-sequence forget-gate recurrence over keys and values (prefill).
 //
-// "RAT+ Deep Dive", section 2.1: every token's recurrence state accumulates information from
-// the start of the sequence (L = T) through a forget gate g = sigmoid(input-dependent logit),
+// "RAT+ Deep Dive", section 2.1: the recurrence of RAT+ runs over the whole sequence (L = T), so a
+// token's state sums up everything before it, decayed by a forget gate g = sigmoid(logit) that
+// depends on the input:
 //     h_t = g_t * h_{t-1} + (1 - g_t) * x_t,       x = k and x = v, same g, per channel,
 // and prefill computes it in parallel by an associative scan (section 7.3 table).  The map
 // h -> g h + (1-g) x is affine, so a run of steps composes to h -> A h + B with
