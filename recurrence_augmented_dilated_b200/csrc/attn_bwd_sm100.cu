@@ -28,6 +28,9 @@
 //                dV += P^T dO,  dK += dS^T Q^     (TS MMAs, both operands' tiles reused);
 //              epilogue: dk = scale dK, dv -> bf16 rows of the block's keys.
 // q^ = RoPE(q) (bf16, as the forward's operand) and Delta come from the CUDA-core prep kernel.
+// When the window is the self key alone (W <= 1), the key blocks of consecutive positions would
+// hold one attending query per key: a dilated head's dq tiles then take the self term per row
+// in their epilogue, and a CUDA-core kernel writes dk~, dv~ of the keys that are not chunk ends.
 // Roles per CTA (192 threads): warp 0 issues TMA loads, warp 1 allocates TMEM and issues the
 // MMAs (one elected thread), warps 2-5 do the elementwise work and the epilogue.  Every wait is
 // bounded: an expired one records RAT_ERR_TIMEOUT in the workspace header, and the CTA stops
@@ -79,6 +82,7 @@ struct Params {
     CUtensorMap tm_kd64[kMaxDil], tm_vd64[kMaxDil];     // chunk ends of one dilation: (d, T/D, B*H)
     CUtensorMap tm_kd128[kMaxDil], tm_vd128[kMaxDil];
     const float *lse, *delta;                      // [B*H][T]
+    const void *kg, *vg;                           // k~, v~ rows (self terms with W <= 1)
     void *dq, *dk, *dv;                            // outputs (B, H, T, d) bf16
     WsHeader *hdr;
     int B, H, T, W, ntiles;
@@ -180,6 +184,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
     const int We = p.W > 1 ? p.W : 1;
     // key blocks: nd of chunk ends (compressed indices BN*j ..), then nw window blocks from ws
     const int tmax = t0 + BM - 1;
+    // a dilated head whose window is the self key alone (W <= 1) takes the diagonal term per row
+    // in the epilogue instead of two window blocks that would each hold one key per row
+    const bool self_row = !dense && We == 1;
     int nd = 0, ws = 0, nw;
     if (dense) {
         nw = (min(tmax, p.T - 1) + 1 + BN - 1) / BN;
@@ -188,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
         ndk = min(ndk, p.T / D);
         nd = (ndk + BN - 1) / BN;
         ws = max(0, t0 - We + 1);
-        nw = (min(tmax, p.T - 1) + 1 - ws + BN - 1) / BN;
+        nw = self_row ? 0 : (min(tmax, p.T - 1) + 1 - ws + BN - 1) / BN;
     }
     const int nb = nd + nw;
 
@@ -337,12 +344,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
             tc::fence_before_sync();
             mbar_arrive(&sh.ds_full[s]);
         }
+        // the self term: dS_tt k~_t with p_tt = 2^(scale log2e <q^_t, k~_t> - lse_t) and
+        // dp_tt = <dO_t, v~_t>; q^_t and dO_t come from this tile's rows in shared memory
+        float ds_self = 0.f;
+        uint4 ks[16];
+        if (self_row && ok) {
+            const size_t ro = ((size_t)bh * p.T + (live ? t : 0)) * DHEAD * 2;
+            uint4 vs[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                ks[c] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.kg) + ro) + c);
+                vs[c] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.vg) + ro) + c);
+            }
+            ok = __all_sync(0xffffffffu, wait_bar(&sh.abort, p.hdr, &sh.qd_full, 0, 8));
+            float sd = 0.f, pd = 0.f;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {       // 16-byte chunk c: channels 8c .. 8c+7
+                const uint32_t off = (c >> 3) * SUB128 + r * 128u + ((((uint32_t)c & 7u) ^ ((uint32_t)r & 7u)) << 4);
+                const uint4 qq = *reinterpret_cast<const uint4 *>(smem + OFF_Q + off);
+                const uint4 gg = *reinterpret_cast<const uint4 *>(smem + OFF_G + off);
+                const uint32_t qu[4] = {qq.x, qq.y, qq.z, qq.w}, gu[4] = {gg.x, gg.y, gg.z, gg.w};
+                const uint32_t ku[4] = {ks[c].x, ks[c].y, ks[c].z, ks[c].w};
+                const uint32_t vu[4] = {vs[c].x, vs[c].y, vs[c].z, vs[c].w};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    sd = fmaf(bf16_lo(qu[i]), bf16_lo(ku[i]), sd);
+                    sd = fmaf(bf16_hi(qu[i]), bf16_hi(ku[i]), sd);
+                    pd = fmaf(bf16_lo(gu[i]), bf16_lo(vu[i]), pd);
+                    pd = fmaf(bf16_hi(gu[i]), bf16_hi(vu[i]), pd);
+                }
+            }
+            const float pr = live ? ex2_approx(fmaf(sd, p.scale_log2, -lse)) : 0.f;
+            ds_self = pr * (pd - dl);
+        }
         if (ok && nb > 0)
             ok = __all_sync(0xffffffffu, wait_bar(&sh.abort, p.hdr, &sh.dq_done[(nb - 1) & 1], ((nb - 1) >> 1) & 1, 7));
         if (ok) {
             tc::fence_after_sync();
             uint8_t *row = static_cast<uint8_t *>(p.dq) + ((size_t)bh * p.T + t) * DHEAD * 2;
-#pragma unroll 1
+#pragma unroll
             for (int c = 0; c < 2; ++c) {        // channels [32c, 32c+32) and their partners + 64
                 float lo[32], hi[32];
                 if (nb > 0) {
@@ -352,6 +392,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) lo[i] = hi[i] = 0.f;
+                }
+                if (self_row) {                      // + dS_tt k~_t on channels 32c+i and 64+32c+i
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const uint4 kl = ks[(32 * c + i) >> 3], kh = ks[(64 + 32 * c + i) >> 3];
+                        const uint32_t wl = ((i & 7) >> 1) == 0 ? kl.x : ((i & 7) >> 1) == 1 ? kl.y : ((i & 7) >> 1) == 2 ? kl.z : kl.w;
+                        const uint32_t wh = ((i & 7) >> 1) == 0 ? kh.x : ((i & 7) >> 1) == 1 ? kh.y : ((i & 7) >> 1) == 2 ? kh.z : kh.w;
+                        lo[i] = fmaf(ds_self, bf16_lo(wl), lo[i]);
+                        lo[i + 1] = fmaf(ds_self, bf16_hi(wl), lo[i + 1]);
+                        hi[i] = fmaf(ds_self, bf16_lo(wh), hi[i]);
+                        hi[i + 1] = fmaf(ds_self, bf16_hi(wh), hi[i + 1]);
+                    }
                 }
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
@@ -628,6 +680,45 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dkv_sm100_kernel(const _
     if (warp == 1) tc::tmem_dealloc(tmem, 512);
 }
 
+// ------------------------------------------------------------------------------ self keys
+// W <= 1: a key j that is not a chunk end is held by query j alone, so its gradients are one
+// pair's: p = 2^(scale log2e <q^_j, k~_j> - lse_j), ds = p (<dO_j, v~_j> - Delta_j),
+// dk~_j = scale ds q^_j, dv~_j = p dO_j.  One warp per row, four channels per lane.
+__global__ void __launch_bounds__(256) attn_bwd_self_kernel(const __grid_constant__ Params p,
+                                                            const void *qh, const void *k, const void *v,
+                                                            const void *dO) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bh = blockIdx.y, h = bh % p.H;
+    const int j = blockIdx.x * 8 + warp;
+    const int D = p.Dh[h];
+    if (j >= p.T || D == 1 || j % D == D - 1) return;
+    const size_t off = ((size_t)bh * p.T + j) * DHEAD * 2 + lane * 8;
+    auto ld4 = [&](const void *base, float *x) {
+        const uint2 u = __ldg(reinterpret_cast<const uint2 *>(static_cast<const uint8_t *>(base) + off));
+        x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+    };
+    float q[4], kk[4], vv[4], g[4];
+    ld4(qh, q);
+    ld4(k, kk);
+    ld4(v, vv);
+    ld4(dO, g);
+    float sd = 0.f, pd = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        sd = fmaf(q[i], kk[i], sd);
+        pd = fmaf(g[i], vv[i], pd);
+    }
+    sd = warp_sum(sd);
+    pd = warp_sum(pd);
+    const size_t r = (size_t)bh * p.T + j;
+    const float pr = ex2_approx(fmaf(sd, p.scale_log2, -p.lse[r]));
+    const float ds = pr * (pd - p.delta[r]) * p.scale;
+    *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.dk) + off) =
+        make_uint2(pack_bf16(ds * q[0], ds * q[1]), pack_bf16(ds * q[2], ds * q[3]));
+    *reinterpret_cast<uint2 *>(static_cast<uint8_t *>(p.dv) + off) =
+        make_uint2(pack_bf16(pr * g[0], pr * g[1]), pack_bf16(pr * g[2], pr * g[3]));
+}
+
 // ------------------------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 bwd_encode_fn() {
     static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
@@ -750,8 +841,10 @@ int launch_attn_bwd_sm100(const AttnBwdParams &a, void *stream) {
     for (int type = 0; type < 2; ++type)
         for (int gi = 0; gi < p.ngroups; ++gi) {
             const int D = a.Dh[order[p.grp_head0[gi]]];
+            // (with W <= 1 a key that is not a chunk end has only its own query: the per-row
+            // kernel below takes those keys)
             const int nblk = type == 0 ? (a.T / D + dkv::BM - 1) / dkv::BM
-                                       : (D > 1 ? (a.T + dkv::BM - 1) / dkv::BM : 0);
+                                       : (D > 1 && a.W > 1 ? (a.T + dkv::BM - 1) / dkv::BM : 0);
             if (nblk == 0) continue;
             p.sec_item0[p.nsec] = kitems;
             p.sec_grp[p.nsec] = gi;
@@ -763,6 +856,8 @@ int launch_attn_bwd_sm100(const AttnBwdParams &a, void *stream) {
     p.sec_item0[p.nsec] = kitems;
     p.lse = a.lse;
     p.delta = a.delta;
+    p.kg = a.k;
+    p.vg = a.v;
     p.dq = a.dq;
     p.dk = a.dk;
     p.dv = a.dv;
@@ -781,6 +876,12 @@ int launch_attn_bwd_sm100(const AttnBwdParams &a, void *stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (dq_items > 0) attn_bwd_dq_sm100_kernel<<<(unsigned)dq_items, kThreads, dqk::SMEM, s>>>(p);
     if (kitems > 0) attn_bwd_dkv_sm100_kernel<<<(unsigned)kitems, kThreads, dkv::SMEM, s>>>(p);
+    bool self_keys = false;
+    for (int h = 0; h < a.H; ++h) self_keys |= a.Dh[h] > 1;
+    if (self_keys && a.W <= 1) {
+        dim3 grid((unsigned)((a.T + 7) / 8), (unsigned)(a.B * a.H));
+        attn_bwd_self_kernel<<<grid, 256, 0, s>>>(p, a.qh, a.k, a.v, a.dO);
+    }
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
 }
 
