@@ -43,11 +43,12 @@ __device__ int g_attn_error;     // first device-side error of the attention ker
 __device__ unsigned g_attn_where; // where it happened: (site << 24) | (block << 8) | parity
 __device__ unsigned g_attn_waiting; // bit s set: a wait at site s was in progress when a CTA aborted
 
-// (cos, sin)(l * theta_f) for l < 32 and the 64 RoPE frequencies, [f][l], formed on the host in
+// (cos, sin)(l * theta_f) for l < 16 and the 64 RoPE frequencies, [f][l], formed on the host in
 // float64; the producer copies a launch's table next to Q.  kRelSlots tables per device, one per
 // distinct frequency set (RoPE base), each written once and never replaced.
 constexpr int kRelSlots = 16;
-__device__ float2 g_rope_rel[kRelSlots][64 * 32];
+constexpr int kRelL = 16;
+__device__ float2 g_rope_rel[kRelSlots][64 * kRelL];
 
 namespace {
 
@@ -58,7 +59,8 @@ constexpr int kThreads = 192;         // warp 0: TMA, warp 1: MMA, warps 2-5: so
 constexpr uint32_t QSUB = BM * 128;   // one [128 rows][64 bf16] 128B-swizzled sub-tile of Q / O
 constexpr int kMaxDil = 4;
 constexpr float kRescaleLog2 = 8.0f;             // move the running max only when it grows by > 2^8
-constexpr uint32_t kRelBytes = 64 * 32 * 8;       // the RoPE table g_rope_rel
+constexpr uint32_t kRelBytes = 64 * kRelL * 8;    // the RoPE table g_rope_rel
+constexpr int kBasStride = 65;                    // padded row of the per-tile base rotations
 
 // Shared-memory / TMEM plan for key blocks of BN keys.
 template <int BN>
@@ -108,7 +110,7 @@ struct Params {
     int n_sink;               // attention sinks (n_sink < D of every dilated head, <= BN)
     int top_k;                // top-k variant: chunks selected per row (1 .. 16)
     float *lse;               // [B*H][T] or null: log2 of each row's softmax denominator
-    const float2 *rope_rel;   // device table [64 f][32 l] of (cos, sin)(l theta_f), see g_rope_rel
+    const float2 *rope_rel;   // device table [64 f][16 l] of (cos, sin)(l theta_f), see g_rope_rel
     float theta_f[64];
     double theta[64];
 };
@@ -236,6 +238,15 @@ RAT_DEVICE int count_set(const uint32_t *bm, int words) {
     int n = 0;
     for (int w = 0; w < words; ++w) n += __popc(bm[w]);
     return n;
+}
+
+// 16 bytes global -> shared without passing through registers (completion: cp_async_wait_all)
+RAT_DEVICE void cp_async16(void *sdst, const void *gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(smem_u32(sdst)), "l"(gsrc) : "memory");
+}
+RAT_DEVICE void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 RAT_DEVICE uint32_t swz(uint32_t row, uint32_t chunk) {   // 128B swizzle inside a sub-tile
@@ -489,24 +500,24 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
         };
         uint4 xrow[16];
         if (self_reg) load_rows(p.kg, xrow);         // k~ of the tile's rows, in flight with Q
-        // rotate-half RoPE of the Q tile at positions pos0 + t.  Rotation of row 32w + l is
-        // rot(base_w) * rot(l): rot(l theta_f) for l < 32 arrives with Q (the launch's table, copied
-        // into the still-unused second K stage); while Q is in flight the softmax threads tabulate
-        // rot((pos0 + t0 + 32w) theta_f) in the second V stage; once Q has landed each thread
-        // rotates its own row.
-        const float2 *rel = reinterpret_cast<const float2 *>(smem + C::OFF_K + C::KTILE);  // [64 f][32 l]
-        float2 *bas = reinterpret_cast<float2 *>(smem + C::OFF_V + C::KTILE);              // [4 w][64 f]
+        // rotate-half RoPE of the Q tile at positions pos0 + t.  Rotation of row 16g + l is
+        // rot(base_g) * rot(l): rot(l theta_f) for l < 16 arrives with Q (the launch's table, copied
+        // into the still-unused second K stage); while Q is in flight each warp tabulates
+        // rot((pos0 + t0 + 16g) theta_f) for its own two row groups g in the second V stage; once Q
+        // has landed each thread rotates its own row.
+        const float2 *rel = reinterpret_cast<const float2 *>(smem + C::OFF_K + C::KTILE);  // [64 f][16 l]
+        float2 *bas = reinterpret_cast<float2 *>(smem + C::OFF_V + C::KTILE);              // [8 g][kBasStride]
         if (p.rope) {
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int e = r + 128 * k, w = e >> 6, f = e & 63;
-                const long long pos = p.pos0 + t0 + 32 * w;
+            for (int k = 0; k < 4; ++k) {
+                const int e = lane + 32 * k, g = 2 * q4 + (e >> 6), f = e & 63;
+                const long long pos = p.pos0 + t0 + 16 * g;
                 float cs, sn;
                 if (p.rope_f32) rope_cs_f32((int)pos, p.theta_f[f], cs, sn);
                 else rope_cs_fast(pos, p.theta[f], cs, sn);
-                bas[w * 64 + f] = make_float2(cs, sn);
+                bas[g * kBasStride + f] = make_float2(cs, sn);
             }
-            asm volatile("bar.sync 1, 128;" ::: "memory");     // reached by every softmax thread
+            __syncwarp();
         }
         // waits are made warp-uniform: tcgen05.ld/st below are warp-collective
         bool ok = __all_sync(0xffffffffu, wait_bar(sh, &sh.q_full, 0, 6));
@@ -523,7 +534,7 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
 #pragma unroll
                     for (int u = 0; u < 2; ++u) {
                         const int f = c * 8 + 2 * i + u;
-                        const float2 b = bas[q4 * 64 + f], rl = rel[f * 32 + lane];
+                        const float2 b = bas[(r >> 4) * kBasStride + f], rl = rel[f * kRelL + (r & 15)];
                         cs[u] = b.x * rl.x - b.y * rl.y;
                         sn[u] = b.y * rl.x + b.x * rl.y;
                     }
@@ -725,20 +736,25 @@ attn_sm100_kernel(const __grid_constant__ Params p) {
             mbar_arrive(&sh.p_full[j & 1]);
             jdone = j + 1;
         }
-        // ---- epilogue: (O + w_self v~_t) / l -> bf16 rows in the Q buffer (every S MMA, the only
-        // reader of Q, has completed) -> TMA stores of this warp's 32 rows
+        // ---- epilogue: (O + w_self v~_t) / l -> bf16 rows in the Q buffer -> TMA stores of this
+        // warp's 32 rows.  Every S product, the only reader of Q, has completed once the last S
+        // buffer was seen full, so the self values are copied straight into this warp's rows
+        // (128B-swizzled, no registers) while the last PV runs.
         bool have_o = ok && jdone == nbt;
-        uint4 vrow[16];           // v~ of the tile's rows (own array: keeps the k~ rows dead here)
-        if (have_o && self_reg) load_rows(p.vg, vrow);      // in flight during the last PV
+        if (have_o && self_reg) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(p.vg) + (size_t)bh * p.T * (DHEAD / 8) + xc;
+#pragma unroll
+            for (int k = 0; k < 16; ++k)       // rows past T repeat row T-1 (never stored)
+                cp_async16(sQ + (xc >> 3) * QSUB + swz(xr + 2 * k, xc & 7),
+                           src + (size_t)min(t0 + xr + 2 * k, p.T - 1) * (DHEAD / 8));
+        }
         if (have_o && nbt > 0)
             have_o = __all_sync(0xffffffffu, wait_bar(sh, &sh.o_ready[(nbt - 1) & 1], ((nbt - 1) >> 1) & 1, 9, nbt));
+        if (self_reg) {
+            cp_async_wait_all();
+            __syncwarp();
+        }
         if (have_o) {
-            if (self_reg) {     // stage the self values in this warp's rows, 128B-swizzled
-#pragma unroll
-                for (int k = 0; k < 16; ++k)
-                    *reinterpret_cast<uint4 *>(sQ + (xc >> 3) * QSUB + swz(xr + 2 * k, xc & 7)) = vrow[k];
-                __syncwarp();
-            }
             tc::fence_after_sync();
             const float inv = 1.0f / (l_run + w_self);
             // the row's softmax denominator, for the backward (m_run is in log2-scaled units)
@@ -952,7 +968,7 @@ static int rope_rel_table(const double *theta, void *stream, const float2 **out)
             continue;
         }
         if (std::memcmp(slots[dev][i].theta, theta, sizeof(double) * 64) == 0) {
-            *out = base[dev] + (size_t)i * 64 * 32;
+            *out = base[dev] + (size_t)i * 64 * kRelL;
             return RAT_OK;
         }
     }
@@ -962,11 +978,11 @@ static int rope_rel_table(const double *theta, void *stream, const float2 **out)
     if (cs != cudaStreamCaptureStatusNone) return RAT_ERR_UNSUPPORTED;
     if (!upload[dev] && cudaStreamCreateWithFlags(&upload[dev], cudaStreamNonBlocking) != cudaSuccess)
         return RAT_ERR_CUDA;
-    static float2 tab[64 * 32];      // guarded by mu
+    static float2 tab[64 * kRelL];      // guarded by mu
     for (int f = 0; f < 64; ++f)
-        for (int l = 0; l < 32; ++l) {
+        for (int l = 0; l < kRelL; ++l) {
             const double ang = (double)l * theta[f];
-            tab[f * 32 + l] = make_float2((float)std::cos(ang), (float)std::sin(ang));
+            tab[f * kRelL + l] = make_float2((float)std::cos(ang), (float)std::sin(ang));
         }
     if (cudaMemcpyToSymbolAsync(g_rope_rel, tab, sizeof(tab), (size_t)free_slot * sizeof(tab),
                                 cudaMemcpyHostToDevice, upload[dev]) != cudaSuccess ||
@@ -974,7 +990,7 @@ static int rope_rel_table(const double *theta, void *stream, const float2 **out)
         return RAT_ERR_CUDA;
     std::memcpy(slots[dev][free_slot].theta, theta, sizeof(double) * 64);
     slots[dev][free_slot].valid = true;
-    *out = base[dev] + (size_t)free_slot * 64 * 32;
+    *out = base[dev] + (size_t)free_slot * 64 * kRelL;
     return RAT_OK;
 }
 

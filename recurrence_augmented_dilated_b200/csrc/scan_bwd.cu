@@ -127,8 +127,8 @@ __global__ void __launch_bounds__(BwdCfg<E, DH>::THREADS) bwd_reduce_kernel(cons
                 rot_t(yk[u], rc, rs, ek);
                 step_back(rc, rs, sc, ss);
             }
-#pragma unroll
             const bool start = RESET && block_start(p, tb - u);
+#pragma unroll
             for (int q = 0; q < NP; ++q) {
                 A[q] = f2_mul(gnext[q], A[q]);
                 Bk[q] = f2_fma(gnext[q], Bk[q], ek[q]);
