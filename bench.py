@@ -753,12 +753,12 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     achieved = nbytes / (ms * 1e-3) / 1e9
     res = {"workload": w.name, "ms": ms,
            "step": ("rat_recur_backward_local(L=%d)" % reset_every if reset_every else
-                    "rat_recur_backward") + " (3 launches)",
+                    "rat_recur_backward") + " (1 launch: scan from the end, decoupled look-back)",
            "tokens_per_s": world * B * T / (ms * 1e-3),
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "of": peak_kind,
                         "algorithmic_bytes": nbytes},
-           "clocks": clk.summary(), "gpu_launches": 3 * steps}
+           "clocks": clk.summary(), "gpu_launches": steps}
     # attention backward on the same shapes: q, k~, v~, o, dO resident
     q = x["q"].to(dev)
     o = torch.empty_like(q)

@@ -174,7 +174,10 @@ RAT_API int rat_recur_prefill_local(const void *k, const void *v, const void *ga
  *   ws, ws_bytes     : workspace of at least rat_recur_backward_workspace_bytes(B, H, T, d)
  * float32 arithmetic; bf16 outputs rounded once.  h_{t-1} is taken from the stored (rounded)
  * forward outputs, as a memory-saving training step would.  Outputs may not alias inputs.
- * T = 0 is a no-op.  Three launches (chunk reduce, carry, output); no device-side waits.
+ * T = 0 is a no-op.  One launch: a scan from the end of the sequence whose chunks combine by a
+ * decoupled look-back with bounded waits (a wait that runs out records RAT_ERR_TIMEOUT in the
+ * workspace, read by rat_sync_status()).  The workspace follows the prefill rules (zeroed once
+ * by rat_workspace_init, one call at a time); RAT_ERR_UNSUPPORTED when B*H*ceil(T/32) >= 2^31.
  * ---------------------------------------------------------------------------------------- */
 RAT_API size_t rat_recur_backward_workspace_bytes(int B, int H, int T, int d);
 
@@ -535,13 +538,16 @@ RAT_API int rat_dilated_decode_paged(const void *q, const void *k, const void *v
                              float rope_base, float scale, void *ws, size_t ws_bytes,
                              void *stream);
 
-/* Test hook for failure detection (no counterpart in the method): the next rat_recur_prefill
- * issued from the calling host thread withholds the look-back publication of chunk `chunk`
- * (chunk index >= 1 along the sequence, in every (b, h) and channel slice; a chunk is 128 rows
- * of 64 channels for bf16, d = 128 and T a multiple of 16, else 16 KiB of each tensor's rows)
- * and bounds each look-back wait by wait_limit_ns (1 ms .. 2 s).  Its successors' waits run out, the call's results are wrong,
- * and rat_sync_status() reports RAT_ERR_TIMEOUT; nothing hangs and the context stays usable.
- * Returns RAT_ERR_INVALID for out-of-range arguments. */
+/* Test hook for failure detection (no counterpart in the method): the next rat_recur_prefill,
+ * rat_recur_prefill_local, rat_recur_backward or rat_recur_backward_local issued from the calling
+ * host thread withholds the look-back publication of chunk `chunk` (chunk index >= 1 along the
+ * sequence, in every (b, h) and channel slice; a prefill chunk is 128 rows of 64 channels for
+ * bf16, d = 128 and T a multiple of 16, else 16 KiB of each tensor's rows; a backward chunk is
+ * 64 rows for bf16 and 32 for float32) and bounds each look-back wait by wait_limit_ns
+ * (1 ms .. 2 s).  The chunks that wait for it (after it for the prefill, before it for the
+ * backward) run out of time, the call's results are wrong, and rat_sync_status() reports
+ * RAT_ERR_TIMEOUT; nothing hangs and the context stays usable.  Returns RAT_ERR_INVALID for
+ * out-of-range arguments. */
 RAT_API int rat_debug_inject_lookback_fault(int64_t chunk, int64_t wait_limit_ns);
 
 /* rat_dilated_decode_noalloc -- the same decode step, for callers that cannot allocate.

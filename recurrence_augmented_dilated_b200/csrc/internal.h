@@ -64,7 +64,6 @@ struct WindowParams {
 int launch_window(const WindowParams &p, int dtype, void *stream);
 
 // backward of the recurrence step (reduce, carry and output launches over 64-row chunks)
-constexpr int kBwdRows = 64;
 struct RecurBwdParams {
     const void *k, *v, *a;          // forward inputs
     const void *yk, *yv;            // forward outputs k~ (rotated), v~
@@ -73,8 +72,10 @@ struct RecurBwdParams {
     const float *dhTk, *dhTv;       // gradient of the final state, or null
     void *dk, *dv, *da;             // outputs
     float *dh0k, *dh0v;             // gradient of the initial state, or null
-    float *agg;                     // [BH][nch][3][d]  A, Bk, Bv of each chunk (reverse map)
-    float *carry;                   // [BH][nch][2][d]  gradient entering each chunk from the right
+    WsHeader *hdr;
+    // look-back records, one 64-bit word per value: (launch tag << 32) | float bits
+    uint64_t *agg;                  // [BH * nch][3][d]  map (A, Bk, Bv) of each chunk
+    uint64_t *pre;                  // [BH * nch][2][d]  carry leaving each chunk to the left
     int BH, T, d, nch;
     long long pos0;
     int rope, rope_f32;
@@ -82,7 +83,10 @@ struct RecurBwdParams {
     double theta[64];
     float step_cos[64], step_sin[64];
     long long reset;                // > 0: the chunk-local form (state restarted at multiples)
+    long long fault_chunk;          // test hook: chunk index that never publishes (-1: none)
+    unsigned long long wait_ns;     // bound of each look-back wait
 };
+int recur_bwd_chunk_rows(int d, int dtype);
 size_t recur_bwd_workspace_bytes(int BH, int T, int d);
 int launch_recur_bwd(const RecurBwdParams &p, int dtype, void *stream);
 

@@ -218,13 +218,19 @@ int recur_backward(const void *k, const void *v, const void *gate_logit, const f
     p.h0k = h0_k; p.h0v = h0_v; p.dhTk = dhT_k; p.dhTv = dhT_v;
     p.dk = dk; p.dv = dv; p.da = dgate_logit; p.dh0k = dh0_k; p.dh0v = dh0_v;
     p.BH = B * H; p.T = T; p.d = d;
-    p.nch = (T + kBwdRows - 1) / kBwdRows;
+    const int tc = recur_bwd_chunk_rows(d, dtype);
+    if ((long long)B * H * ((T + tc - 1) / tc) > 0x7fffffffll) return RAT_ERR_UNSUPPORTED;
+    p.nch = (T + tc - 1) / tc;
     p.pos0 = pos0;
     p.reset = L;
     p.rope = rope_base > 0.f ? 1 : 0;
     uint8_t *w = static_cast<uint8_t *>(ws);
-    p.agg = reinterpret_cast<float *>(w + sizeof(WsHeader));
-    p.carry = reinterpret_cast<float *>(w + sizeof(WsHeader) + align256((size_t)p.BH * p.nch * 3 * d * 4));
+    p.hdr = reinterpret_cast<WsHeader *>(w);
+    p.agg = reinterpret_cast<uint64_t *>(w + sizeof(WsHeader));
+    p.pre = reinterpret_cast<uint64_t *>(w + sizeof(WsHeader) + align256((size_t)p.BH * p.nch * 3 * d * 8));
+    p.fault_chunk = g_fault_chunk;
+    p.wait_ns = g_fault_chunk >= 0 ? g_fault_wait_ns : kWaitLimitNs;
+    g_fault_chunk = -1;
     if (p.rope) {
         rope_theta(rope_base, d, p.theta);
         for (int c = 0; c < 64; ++c) {

@@ -144,3 +144,38 @@ def test_local_backward_full_size_sampled_heads():
     x = synthetic.prefill_inputs(w)
     dyk, dyv = grads(w.B, w.H, w.T, w.d, torch.bfloat16, seed=19)
     check(x, dyk, dyv, rope_base=w.rope_base, heads=[(0, 0), (3, 15)], reset_every=16)
+
+
+def test_backward_workspace_reused_across_calls():
+    # one workspace, several calls of both forms and both dtypes: the look-back records carry a
+    # per-launch tag, so no call reads another's records (every result matches the oracle)
+    B, H, T, d = 1, 2, 700, 128
+    for i, (dtype, L) in enumerate([(torch.bfloat16, 0), (torch.float32, 16), (torch.bfloat16, 5),
+                                    (torch.float32, 0), (torch.bfloat16, 0)]):
+        x = inputs(B, H, T, d, dtype, seed=40 + i)
+        dyk, dyv = grads(B, H, T, d, dtype, seed=50 + i)
+        check(x, dyk, dyv, rope_base=10000.0, reset_every=L)
+
+
+def test_backward_lookback_timeout_is_reported():
+    # failure detection: one chunk withholds its publication (test hook); the chunks before it
+    # wait for it until their bound runs out, the workspace reports RAT_ERR_TIMEOUT, nothing hangs
+    # and the next call on the same workspace is correct again
+    L = rat.lib()
+    B, H, T, d = 1, 2, 1024, 128
+    x = inputs(B, H, T, d, torch.bfloat16, seed=31)
+    dyk, dyv = grads(B, H, T, d, torch.bfloat16, seed=32)
+    dev = torch.device("cuda")
+    k, v, a = (x[n].to(dev) for n in ("k", "v", "a"))
+    kr, vr, _, _ = gpu_recur(k, v, a)
+    dk, dv, da = torch.empty_like(k), torch.empty_like(v), torch.empty_like(a)
+    ws = rat.Workspace(rat.rat_recur_backward_workspace_bytes(B, H, T, d))
+    L.rat_debug_inject_lookback_fault(5, 20_000_000)      # chunk 5, 20 ms waits, next call only
+    rat.rat_recur_backward(k, v, a, kr, vr, dyk.to(dev), dyv.to(dev), dk, dv, da, ws)
+    assert rat.rat_sync_status(ws) == -4
+    rat.rat_recur_backward(k, v, a, kr, vr, dyk.to(dev), dyv.to(dev), dk, dv, da, ws)
+    assert rat.rat_sync_status(ws) == 0
+    ref = oracle.recurrence_layer_backward(f64(x["k"]), f64(x["v"]), f64(x["a"]), f64(dyk), f64(dyv),
+                                           None, None, None, None)
+    for g, r in zip((dk, dv, da), ref[:3]):
+        assert rel_err(g, r) <= TOL_BF16
