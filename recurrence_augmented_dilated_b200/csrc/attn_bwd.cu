@@ -46,25 +46,58 @@ constexpr int kRows = 4;        // rows (keys or queries) whose loads are issued
 
 }  // namespace
 
+// q^ = RoPE(q) and Delta_t = dO_t . o_t.  One warp walks kPrepRows consecutive rows; lane l holds
+// channels l*CPL .. l*CPL+CPL-1 (the rotate-half partner of channel c < d/2 sits in lane l ^ 16).
+// The lane's angles are formed once at the warp's first row and advanced one position per row
+// by a complex multiply with (cos theta, sin theta).
+constexpr int kPrepRows = 16;
+
 template <typename E, int DH>
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const __grid_constant__ AttnBwdParams p) {
-    constexpr int CPL = DH / 32, EB = sizeof(E);
+    constexpr int CPL = DH / 32, EB = sizeof(E), ROWB = DH * EB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = blockIdx.y;
-    const int t = blockIdx.x * 8 + warp;
-    if (t >= p.T) return;
-    const size_t off = ((size_t)bh * p.T + t) * DH * EB + lane * CPL * EB;
-    float q[CPL], o[CPL], g[CPL];
-    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.q) + off, q);
-    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.o) + off, o);
-    RowIO<E, CPL>::load(static_cast<const uint8_t *>(p.dO) + off, g);
-    if (p.rope) rope_lane<DH>(p, p.pos0 + t, lane, 1.f, q);
-    RowIO<E, CPL>::store(static_cast<uint8_t *>(p.qh) + off, q);
-    float dot = 0.f;
+    const int t0 = (blockIdx.x * 8 + warp) * kPrepRows;
+    if (t0 >= p.T) return;
+    const int nr = min(kPrepRows, p.T - t0);
+    const size_t off = ((size_t)bh * p.T + t0) * ROWB + lane * CPL * EB;
+    const uint8_t *gq = static_cast<const uint8_t *>(p.q) + off;
+    const uint8_t *go = static_cast<const uint8_t *>(p.o) + off;
+    const uint8_t *gg = static_cast<const uint8_t *>(p.dO) + off;
+    uint8_t *gh = static_cast<uint8_t *>(p.qh) + off;
+    float cs[CPL], sn[CPL], sc[CPL], ss[CPL];
+    if (p.rope) {
 #pragma unroll
-    for (int j = 0; j < CPL; ++j) dot = fmaf(g[j], o[j], dot);
-    dot = warp_sum(dot);
-    if (lane == 0) p.delta[(size_t)bh * p.T + t] = dot;
+        for (int j = 0; j < CPL; ++j) {
+            const double th = p.theta[(lane * CPL + j) % (DH / 2)];
+            rope_cs(p.pos0 + t0, th, cs[j], sn[j]);
+            rope_cs(1, th, sc[j], ss[j]);
+        }
+    }
+    const bool first_half = lane < 16;
+#pragma unroll 4
+    for (int r = 0; r < nr; ++r) {
+        float q[CPL], o[CPL], g[CPL];
+        RowIO<E, CPL>::load(gq + (size_t)r * ROWB, q);
+        RowIO<E, CPL>::load(go + (size_t)r * ROWB, o);
+        RowIO<E, CPL>::load(gg + (size_t)r * ROWB, g);
+        if (p.rope) {
+#pragma unroll
+            for (int j = 0; j < CPL; ++j) {
+                const float partner = __shfl_xor_sync(0xffffffffu, q[j], 16);
+                q[j] = first_half ? q[j] * cs[j] - partner * sn[j] : q[j] * cs[j] + partner * sn[j];
+                const float nc = cs[j] * sc[j] - sn[j] * ss[j];     // one position on
+                sn[j] = sn[j] * sc[j] + cs[j] * ss[j];
+                cs[j] = nc;
+            }
+        }
+        RowIO<E, CPL>::store(gh + (size_t)r * ROWB, q);
+        float dot = 0.f;
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) dot = fmaf(g[j], o[j], dot);
+        dot = warp_sum(dot);
+        if (lane == 0) p.delta[(size_t)bh * p.T + t0 + r] = dot;
+    }
 }
 
 template <typename E, int DH>
@@ -240,7 +273,8 @@ size_t attn_bwd_workspace_bytes(int B, int H, int T, int d, int dtype) {
 template <typename E, int DH>
 static int launch_bwd(const AttnBwdParams &p, cudaStream_t s) {
     dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)(p.B * p.H));
-    attn_bwd_prep_kernel<E, DH><<<grid, 256, 0, s>>>(p);
+    const dim3 pgrid((unsigned)((p.T + 8 * kPrepRows - 1) / (8 * kPrepRows)), (unsigned)(p.B * p.H));
+    attn_bwd_prep_kernel<E, DH><<<pgrid, 256, 0, s>>>(p);
     attn_bwd_dq_kernel<E, DH><<<grid, 256, 0, s>>>(p);
     attn_bwd_dkv_kernel<E, DH><<<grid, 256, 0, s>>>(p);
     return cudaGetLastError() == cudaSuccess ? RAT_OK : RAT_ERR_CUDA;
@@ -250,8 +284,8 @@ static int launch_bwd(const AttnBwdParams &p, cudaStream_t s) {
 // given (the forward attention runs once with its output in dq, which the dq launch then
 // overwrites), then the dq and dk/dv launches.
 static int launch_bwd_tc(const AttnBwdParams &p, cudaStream_t s) {
-    dim3 grid((unsigned)((p.T + 7) / 8), (unsigned)(p.B * p.H));
-    attn_bwd_prep_kernel<__nv_bfloat16, 128><<<grid, 256, 0, s>>>(p);
+    const dim3 pgrid((unsigned)((p.T + 8 * kPrepRows - 1) / (8 * kPrepRows)), (unsigned)(p.B * p.H));
+    attn_bwd_prep_kernel<__nv_bfloat16, 128><<<pgrid, 256, 0, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return RAT_ERR_CUDA;
     if (!p.lse_given) {
         AttnSm100Args a;
