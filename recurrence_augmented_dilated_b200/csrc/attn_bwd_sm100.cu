@@ -51,16 +51,26 @@ constexpr int kMaxDil = 4;
 constexpr uint32_t SUB128 = 128 * 128;   // [128 rows][64 bf16] 128B-swizzled sub-tile
 constexpr uint32_t SUB64 = 64 * 128;     // [64 rows][64 bf16]
 
-// ---- dq kernel: 128 queries x blocks of 64 keys
+// ---- dq kernel: 128 queries x blocks of BN keys.  BN = 64: S[2], dP[2] and dQ take 384 TMEM
+// columns (512 allocated), one CTA per SM; BN = 32: 256 columns and 96 KiB of shared memory,
+// two CTAs per SM, for launches whose tiles are short (every head dilated).
+template <int BN_>
+struct DqCfg {
+    static constexpr int BM = 128, BN = BN_;
+    static constexpr uint32_t SUBK = BN * 128;           // [BN rows][64 bf16] 128B-swizzled sub-tile
+    static constexpr uint32_t OFF_Q = 0;                 // q^ tile, two d-halves
+    static constexpr uint32_t OFF_G = OFF_Q + 2 * SUB128;   // dO tile
+    static constexpr uint32_t OFF_K = OFF_G + 2 * SUB128;   // two stages of a K block (two d-halves each)
+    static constexpr uint32_t OFF_V = OFF_K + 2 * 2 * SUBK;
+    static constexpr uint32_t OFF_BAR = OFF_V + 2 * 2 * SUBK;
+    static constexpr uint32_t SMEM = OFF_BAR + 256;
+    static constexpr uint32_t COL_S = 0, COL_P = 2 * BN, COL_Q = 4 * BN;   // S[2], dP[2], dQ
+    static constexpr uint32_t TMEM_COLS = BN == 64 ? 512 : 256;
+    static constexpr int MIN_CTAS = BN == 64 ? 1 : 2;
+    static_assert(BN == 32 || BN == 64, "key blocks of 32 or 64");
+};
 namespace dqk {
-constexpr int BM = 128, BN = 64;
-constexpr uint32_t OFF_Q = 0;                       // q^ tile, two d-halves
-constexpr uint32_t OFF_G = OFF_Q + 2 * SUB128;      // dO tile
-constexpr uint32_t OFF_K = OFF_G + 2 * SUB128;      // two stages of a K block (two d-halves each)
-constexpr uint32_t OFF_V = OFF_K + 2 * 2 * SUB64;
-constexpr uint32_t OFF_BAR = OFF_V + 2 * 2 * SUB64;
-constexpr uint32_t SMEM = OFF_BAR + 256;
-constexpr uint32_t COL_S = 0, COL_P = 2 * BN, COL_Q = 4 * BN;   // S[2], dP[2], dQ
+constexpr int BM = 128;
 }  // namespace dqk
 
 // ---- dkv kernel: 128 keys x tiles of 64 queries
@@ -78,8 +88,8 @@ constexpr uint32_t COL_S = 0, COL_P = 2 * BN, COL_V = 4 * BN, COL_K = 4 * BN + D
 struct Params {
     CUtensorMap tm_qh128, tm_g128;                 // q^, dO: (d, T, B*H), box (64, 128, 1)
     CUtensorMap tm_qh64, tm_g64;                   // box (64, 64, 1)
-    CUtensorMap tm_k64, tm_v64, tm_k128, tm_v128;  // k~, v~ rows, boxes of 64 / 128 rows
-    CUtensorMap tm_kd64[kMaxDil], tm_vd64[kMaxDil];     // chunk ends of one dilation: (d, T/D, B*H)
+    CUtensorMap tm_kq, tm_vq, tm_k128, tm_v128;    // k~, v~ rows, boxes of the dq launch's BN / 128 rows
+    CUtensorMap tm_kdq[kMaxDil], tm_vdq[kMaxDil];       // chunk ends of one dilation: (d, T/D, B*H)
     CUtensorMap tm_kd128[kMaxDil], tm_vd128[kMaxDil];
     const float *lse, *delta;                      // [B*H][T]
     const void *kg, *vg;                           // k~, v~ rows (self terms with W <= 1)
@@ -158,8 +168,13 @@ struct BarsQ {
 static_assert(sizeof(BarsQ) <= 256, "barriers fit the reserved bytes");
 
 // ------------------------------------------------------------------------------ dq kernel
-__global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __grid_constant__ Params p) {
-    using namespace dqk;
+template <int BN_>
+__global__ void __launch_bounds__(kThreads, DqCfg<BN_>::MIN_CTAS) attn_bwd_dq_sm100_kernel(const __grid_constant__ Params p) {
+    using C = DqCfg<BN_>;
+    constexpr int BM = C::BM, BN = C::BN;
+    constexpr uint32_t SUBK = C::SUBK, OFF_Q = C::OFF_Q, OFF_G = C::OFF_G, OFF_K = C::OFF_K,
+                       OFF_V = C::OFF_V, OFF_BAR = C::OFF_BAR, COL_S = C::COL_S, COL_P = C::COL_P,
+                       COL_Q = C::COL_Q;
     extern __shared__ __align__(1024) uint8_t smem[];
     if (smem_u32(smem) & 1023u) {     // CTA-uniform, before any barrier, TMA or TMEM use
         if (threadIdx.x == 0) record_error(p.hdr, RAT_ERR_UNSUPPORTED, 0x4ffu);
@@ -212,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
         sh.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tc::tmem_alloc(&sh.tmem, 512);
+    if (warp == 1) tc::tmem_alloc(&sh.tmem, C::TMEM_COLS);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -221,8 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            const CUtensorMap *mk = dense ? &p.tm_k64 : &p.tm_kd64[max(p.dslot[h], 0)];
-            const CUtensorMap *mv = dense ? &p.tm_v64 : &p.tm_vd64[max(p.dslot[h], 0)];
+            const CUtensorMap *mk = dense ? &p.tm_kq : &p.tm_kdq[max(p.dslot[h], 0)];
+            const CUtensorMap *mv = dense ? &p.tm_vq : &p.tm_vdq[max(p.dslot[h], 0)];
             tc::prefetch_tmap(&p.tm_qh128);
             tc::prefetch_tmap(&p.tm_g128);
             mbar_arrive_expect_tx(&sh.qd_full, 4 * SUB128);
@@ -235,14 +250,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
                 const int s = j & 1;
                 if (j >= 2 && !wait_bar(&sh.abort, p.hdr, &sh.kv_empty[s], ((j >> 1) - 1) & 1, 1)) break;
                 const bool dil = j < nd;
-                const CUtensorMap *tk = dil ? mk : &p.tm_k64, *tv = dil ? mv : &p.tm_v64;
+                const CUtensorMap *tk = dil ? mk : &p.tm_kq, *tv = dil ? mv : &p.tm_vq;
                 const int row = dil ? BN * j : ws + BN * (j - nd);
-                uint8_t *ks = smem + OFF_K + s * 2 * SUB64, *vs = smem + OFF_V + s * 2 * SUB64;
-                mbar_arrive_expect_tx(&sh.kv_full[s], 4 * SUB64);
+                uint8_t *ks = smem + OFF_K + s * 2 * SUBK, *vs = smem + OFF_V + s * 2 * SUBK;
+                mbar_arrive_expect_tx(&sh.kv_full[s], 4 * SUBK);
                 tc::tma_load_3d(ks, tk, 0, row, bh, &sh.kv_full[s]);
-                tc::tma_load_3d(ks + SUB64, tk, 64, row, bh, &sh.kv_full[s]);
+                tc::tma_load_3d(ks + SUBK, tk, 64, row, bh, &sh.kv_full[s]);
                 tc::tma_load_3d(vs, tv, 0, row, bh, &sh.kv_full[s]);
-                tc::tma_load_3d(vs + SUB64, tv, 64, row, bh, &sh.kv_full[s]);
+                tc::tma_load_3d(vs + SUBK, tv, 64, row, bh, &sh.kv_full[s]);
                 issued = j + 1;
             }
             if (sh.abort) {       // let this CTA's own loads land before its shared memory goes away
@@ -266,11 +281,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
                     // buffers s hold dS(j-2) until its dQ MMA has read it
                     if (j >= 2 && !wait_bar(&sh.abort, p.hdr, &sh.dq_done[s], ((j - 2) >> 1) & 1, 4)) break;
                     tc::fence_after_sync();
-                    const uint32_t sk = smem_u32(smem + OFF_K + s * 2 * SUB64);
-                    const uint32_t sv = smem_u32(smem + OFF_V + s * 2 * SUB64);
+                    const uint32_t sk = smem_u32(smem + OFF_K + s * 2 * SUBK);
+                    const uint32_t sv = smem_u32(smem + OFF_V + s * 2 * SUBK);
                     for (int kk = 0; kk < DHEAD / 16; ++kk) {
                         const uint32_t ao = (kk >> 2) * SUB128 + (kk & 3) * 32;
-                        const uint32_t bo = (kk >> 2) * SUB64 + (kk & 3) * 32;
+                        const uint32_t bo = (kk >> 2) * SUBK + (kk & 3) * 32;
                         tc::mma_bf16_ss(tmem + COL_S + s * BN, tc::smem_desc_sw128(sq + ao, 16, 1024),
                                         tc::smem_desc_sw128(sk + bo, 16, 1024), IDESC_S, kk > 0);
                         tc::mma_bf16_ss(tmem + COL_P + s * BN, tc::smem_desc_sw128(sg + ao, 16, 1024),
@@ -282,11 +297,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
                     const int jp = j - 1, s = jp & 1;
                     if (!wait_bar(&sh.abort, p.hdr, &sh.ds_full[s], (jp >> 1) & 1, 5)) break;
                     tc::fence_after_sync();
-                    const uint32_t sk = smem_u32(smem + OFF_K + s * 2 * SUB64);
+                    const uint32_t sk = smem_u32(smem + OFF_K + s * 2 * SUBK);
                     for (int kk = 0; kk < BN / 16; ++kk)
                         // A = dS[:, 16kk ..]: 8 TMEM columns of packed bf16 pairs; B = K[16kk .., :]
                         tc::mma_bf16_ts(tmem + COL_Q, tmem + COL_S + s * BN + kk * 8,
-                                        tc::smem_desc_sw128(sk + kk * 16 * 128, SUB64, 1024), IDESC_Q,
+                                        tc::smem_desc_sw128(sk + kk * 16 * 128, SUBK, 1024), IDESC_Q,
                                         (jp > 0 || kk > 0) ? 1u : 0u);
                     tc::mma_commit(&sh.dq_done[s]);
                     tc::mma_commit(&sh.kv_empty[s]);
@@ -311,10 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
             if (!__all_sync(0xffffffffu, wait_bar(&sh.abort, p.hdr, &sh.sdp_full[s], (j >> 1) & 1, 6))) { ok = false; break; }
             tc::fence_after_sync();
             float sv[BN], pv[BN];
-            tc::tmem_ld32(tl + COL_S + s * BN, reinterpret_cast<uint32_t *>(sv));
-            tc::tmem_ld32(tl + COL_S + s * BN + 32, reinterpret_cast<uint32_t *>(sv) + 32);
-            tc::tmem_ld32(tl + COL_P + s * BN, reinterpret_cast<uint32_t *>(pv));
-            tc::tmem_ld32(tl + COL_P + s * BN + 32, reinterpret_cast<uint32_t *>(pv) + 32);
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c) {
+                tc::tmem_ld32(tl + COL_S + s * BN + 32 * c, reinterpret_cast<uint32_t *>(sv) + 32 * c);
+                tc::tmem_ld32(tl + COL_P + s * BN + 32 * c, reinterpret_cast<uint32_t *>(pv) + 32 * c);
+            }
             tc::tmem_wait_ld();
             // columns of block j this row attends to
             int c_lo, c_hi;
@@ -327,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
                 c_lo = dense ? 0 : t - We + 1 - base;
             }
             if (!live) c_hi = -1;
-            uint32_t pk[32];
+            uint32_t pk[BN / 2];
 #pragma unroll
             for (int i = 0; i < BN / 2; ++i) {
                 float d2[2];
@@ -339,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
                 }
                 pk[i] = pack_bf16(d2[0], d2[1]);
             }
-            tc::tmem_st32(tl + COL_S + s * BN, pk);
+            if constexpr (BN == 64) tc::tmem_st32(tl + COL_S + s * BN, pk);
+            else tc::tmem_st16(tl + COL_S + s * BN, pk);
             tc::tmem_wait_st();
             tc::fence_before_sync();
             mbar_arrive(&sh.ds_full[s]);
@@ -429,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_bwd_dq_sm100_kernel(const __
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 1) tc::tmem_dealloc(tmem, 512);
+    if (warp == 1) tc::tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 struct BarsK {
@@ -772,9 +789,13 @@ int launch_attn_bwd_sm100(const AttnBwdParams &a, void *stream) {
     std::memset(&p, 0, sizeof(p));
     const uint64_t BH = (uint64_t)a.B * a.H, T = (uint64_t)a.T;
     const uint64_t row = DHEAD * 2, slice = T * row;
+    // dq key blocks: 32 keys (two CTAs per SM) when every head is dilated, else 64
+    bool dense = false;
+    for (int h = 0; h < a.H; ++h) dense |= a.Dh[h] == 1;
+    const uint32_t bnq = dense ? 64 : 32;
     if (!bwd_map(&p.tm_qh128, a.qh, T, BH, row, slice, 128) || !bwd_map(&p.tm_g128, a.dO, T, BH, row, slice, 128) ||
         !bwd_map(&p.tm_qh64, a.qh, T, BH, row, slice, 64) || !bwd_map(&p.tm_g64, a.dO, T, BH, row, slice, 64) ||
-        !bwd_map(&p.tm_k64, a.k, T, BH, row, slice, 64) || !bwd_map(&p.tm_v64, a.v, T, BH, row, slice, 64) ||
+        !bwd_map(&p.tm_kq, a.k, T, BH, row, slice, bnq) || !bwd_map(&p.tm_vq, a.v, T, BH, row, slice, bnq) ||
         !bwd_map(&p.tm_k128, a.k, T, BH, row, slice, 128) || !bwd_map(&p.tm_v128, a.v, T, BH, row, slice, 128))
         return RAT_ERR_CUDA;
     int dvals[kMaxDil], nd = 0;
@@ -795,14 +816,14 @@ int launch_attn_bwd_sm100(const AttnBwdParams &a, void *stream) {
             if (cap > 0) {
                 const uint8_t *kb = static_cast<const uint8_t *>(a.k) + off;
                 const uint8_t *vb = static_cast<const uint8_t *>(a.v) + off;
-                if (!bwd_map(&p.tm_kd64[slot], kb, cap, BH, (uint64_t)D * row, slice, 64) ||
-                    !bwd_map(&p.tm_vd64[slot], vb, cap, BH, (uint64_t)D * row, slice, 64) ||
+                if (!bwd_map(&p.tm_kdq[slot], kb, cap, BH, (uint64_t)D * row, slice, bnq) ||
+                    !bwd_map(&p.tm_vdq[slot], vb, cap, BH, (uint64_t)D * row, slice, bnq) ||
                     !bwd_map(&p.tm_kd128[slot], kb, cap, BH, (uint64_t)D * row, slice, 128) ||
                     !bwd_map(&p.tm_vd128[slot], vb, cap, BH, (uint64_t)D * row, slice, 128))
                     return RAT_ERR_CUDA;
             } else {   // no chunk end inside the sequence: no block reads these maps
-                p.tm_kd64[slot] = p.tm_k64;
-                p.tm_vd64[slot] = p.tm_v64;
+                p.tm_kdq[slot] = p.tm_kq;
+                p.tm_vdq[slot] = p.tm_vq;
                 p.tm_kd128[slot] = p.tm_k128;
                 p.tm_vd128[slot] = p.tm_v128;
             }
@@ -868,13 +889,18 @@ int launch_attn_bwd_sm100(const AttnBwdParams &a, void *stream) {
     p.scale_log2 = a.scale_log2;
     for (int c = 0; c < 64; ++c) p.theta[c] = a.theta[c];
 
-    static std::atomic<uint64_t> attr_q{0}, attr_k{0};
-    int st = set_smem_attr(reinterpret_cast<const void *>(attn_bwd_dq_sm100_kernel), dqk::SMEM, &attr_q);
+    static std::atomic<uint64_t> attr_q64{0}, attr_q32{0}, attr_k{0};
+    int st = bnq == 64
+                 ? set_smem_attr(reinterpret_cast<const void *>(attn_bwd_dq_sm100_kernel<64>), DqCfg<64>::SMEM, &attr_q64)
+                 : set_smem_attr(reinterpret_cast<const void *>(attn_bwd_dq_sm100_kernel<32>), DqCfg<32>::SMEM, &attr_q32);
     if (st != RAT_OK) return st;
     st = set_smem_attr(reinterpret_cast<const void *>(attn_bwd_dkv_sm100_kernel), dkv::SMEM, &attr_k);
     if (st != RAT_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (dq_items > 0) attn_bwd_dq_sm100_kernel<<<(unsigned)dq_items, kThreads, dqk::SMEM, s>>>(p);
+    if (dq_items > 0) {
+        if (bnq == 64) attn_bwd_dq_sm100_kernel<64><<<(unsigned)dq_items, kThreads, DqCfg<64>::SMEM, s>>>(p);
+        else attn_bwd_dq_sm100_kernel<32><<<(unsigned)dq_items, kThreads, DqCfg<32>::SMEM, s>>>(p);
+    }
     if (kitems > 0) attn_bwd_dkv_sm100_kernel<<<(unsigned)kitems, kThreads, dkv::SMEM, s>>>(p);
     bool self_keys = false;
     for (int h = 0; h < a.H; ++h) self_keys |= a.Dh[h] > 1;
