@@ -163,3 +163,15 @@ def test_attention_backward_window_2p6b_sampled_heads():
     w = synthetic.WORKLOADS["window_2p6b"]
     x = synthetic.prefill_inputs(w)
     run(w.B, w.H, w.T, w.d, torch.bfloat16, D=w.D, W=w.W, x=x, heads=[(0, 3), (1, 19)], seed=6)
+
+
+# chunk-end key blocks whose query walks span many 64-query tiles (T > 1024), with ragged last
+# tiles, blocks whose first key lies deep in the sequence, a window beside the chunk ends, and a
+# launch that mixes a dense head (64-key dq blocks) with dilated ones
+@pytest.mark.parametrize("T,D,W", [(1025, 16, 0), (2500, 37, 3), (3000, 200, 70)])
+def test_attention_backward_long_walks(T, D, W):
+    run(1, 2, T, 128, torch.bfloat16, D=D, W=W, seed=T + D, rope_base=10000.0, pos0=11)
+
+
+def test_attention_backward_long_walks_head_hybrid():
+    run(1, 3, 2100, 128, torch.bfloat16, D_per_head=[1, 16, 64], W=4, seed=99)
