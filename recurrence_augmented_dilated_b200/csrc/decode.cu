@@ -49,9 +49,11 @@ RAT_DEVICE uint4 pack8(const float *x) {
 // dilated entries live in pages of a pool found through a page table, and every sequence has
 // its own position (read from seq_pos, advanced by the last CTA of the sequence).
 // SINKS: the first n_sink positions are kept in sink rows and join every key set.
-// WINDOW: the fixed-window recurrence (raw rings; p.window_rec > 0).
+// WINDOW: the fixed-window recurrence (raw rings; p.window_rec > 0).  Its split 0 also reruns
+// the recurrence over the raw ring, a few rows at a time.  Every instantiation is held to the
+// CTAs per SM of the uniform form (five; six for the paged form).
 template <int DH, bool PAGED, bool SINKS, bool WINDOW>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant__ DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, PAGED ? 6 : 5) decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int LPR = DH / 8;                 // lanes per key row
     constexpr int GPW = 32 / LPR;               // key groups per warp
     constexpr int RB = DH * 2;                  // row bytes (bf16)
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
 
     // fixed-window form, split 0: the affine map of the raw rows max(0, t - Lw + 1) .. t - 1 (the
     // recurrence from zero over them), composed in kWarps * GPW segments, one per lane group with
-    // all its rows' loads in flight; warp 0 folds the segments in order below
+    // kBatch rows' loads in flight at a time; warp 0 folds the segments in order below
     constexpr int kSegs = kWarps * (32 / (DH / 8));
     __shared__ float s_wa[WINDOW ? kSegs : 1][DH], s_wk[WINDOW ? kSegs : 1][DH], s_wv[WINDOW ? kSegs : 1][DH];
     if (WINDOW && split == 0) {
@@ -126,34 +128,38 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const __grid_constant_
         const long long lo = max(0ll, t - p.window_rec + 1), n = t - lo;
         const long long r0 = lo + n * seg / kSegs, r1 = lo + n * (seg + 1) / kSegs;
         constexpr int kMaxSeg = (kWindowRows + kSegs - 1) / kSegs;      // rows per segment
-        uint4 ra[kMaxSeg], rk[kMaxSeg], rv[kMaxSeg];
+        constexpr int kBatch = 2;            // rows whose loads are in flight together (registers)
         const size_t ring = (size_t)bh * p.window_rec;
-#pragma unroll
-        for (int i = 0; i < kMaxSeg; ++i) {
-            if (r0 + i < r1) {
-                const size_t off = (ring + (size_t)((r0 + i) % p.window_rec)) * RB + cl * 16;
-                ra[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.araw) + off));
-                rk[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.kraw) + off));
-                rv[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.vraw) + off));
-            }
-        }
         float A[8], K[8], V[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) { A[j] = 1.f; K[j] = 0.f; V[j] = 0.f; }
 #pragma unroll
-        for (int i = 0; i < kMaxSeg; ++i) {
-            if (r0 + i < r1) {
-                float fa[8], fk[8], fv[8];
-                unpack8(ra[i], fa);
-                unpack8(rk[i], fk);
-                unpack8(rv[i], fv);
+        for (int i0 = 0; i0 < kMaxSeg; i0 += kBatch) {
+            uint4 ra[kBatch], rk[kBatch], rv[kBatch];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    float g, omg;
-                    forget_gate(fa[j], g, omg);
-                    K[j] = fmaf(g, K[j], omg * fk[j]);
-                    V[j] = fmaf(g, V[j], omg * fv[j]);
-                    A[j] *= g;
+            for (int i = 0; i < kBatch; ++i) {
+                if (r0 + i0 + i < r1) {
+                    const size_t off = (ring + (size_t)((r0 + i0 + i) % p.window_rec)) * RB + cl * 16;
+                    ra[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.araw) + off));
+                    rk[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.kraw) + off));
+                    rv[i] = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(p.vraw) + off));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kBatch; ++i) {
+                if (r0 + i0 + i < r1) {
+                    float fa[8], fk[8], fv[8];
+                    unpack8(ra[i], fa);
+                    unpack8(rk[i], fk);
+                    unpack8(rv[i], fv);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        float g, omg;
+                        forget_gate(fa[j], g, omg);
+                        K[j] = fmaf(g, K[j], omg * fk[j]);
+                        V[j] = fmaf(g, V[j], omg * fv[j]);
+                        A[j] *= g;
+                    }
                 }
             }
         }
