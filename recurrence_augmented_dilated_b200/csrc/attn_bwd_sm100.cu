@@ -10,10 +10,11 @@
 // and dq = RoPE^T(dq^).  p_tj = 2^(scale log2e <q^_t, k~_j> - lse_t) from the forward's
 // log2-sum-exp, so no running maximum is kept.  Every contraction runs on the tensor cores:
 //
-//   dq kernel  (one CTA per 128-query tile, like the forward): per block of 64 keys (the
+//   dq kernel  (one CTA per 128-query tile, like the forward): per block of BN keys (the
 //              chunk ends through the strided tensor map, then the window band, the whole
-//              prefix for a dense head)
-//                S = Q^ K^T and dP = dO V^T   (SS MMAs, 128 x 64 each, into TMEM),
+//              prefix for a dense head; BN = 32 when every head is dilated, so that two CTAs
+//              share an SM, else 64)
+//                S = Q^ K^T and dP = dO V^T   (SS MMAs, 128 x BN each, into TMEM),
 //                dS = P o (dP - Delta)        (softmax warps, one TMEM lane = query row each;
 //                                              written back into TMEM as bf16),
 //                dQ += dS K                   (TS MMA: dS from TMEM, K as the MN-major operand);

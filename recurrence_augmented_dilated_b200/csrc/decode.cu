@@ -17,7 +17,8 @@
 // Split 0 alone does steps 1-2 and adds the token itself to its softmax.  With the fixed-window
 // recurrence ("RAT+ Deep Dive" section 2.1, L* = 64) step 1 reruns the recurrence from zero over
 // the raw rows of the 63 positions before t (a raw ring in the cache) instead of reading a
-// carried state, and the token's raw rows take the ring slot of position t - 64.
+// carried state, and the token's raw rows take the ring slot of position t - 64; that pass loads
+// two rows at a time so the form keeps the uniform form's registers and CTAs per SM.
 // No CTA reads what another writes in the same launch: the new dil entry (position t) is never
 // older than the window, and the ring slot written held position t - W, outside the window.
 #include <mutex>
