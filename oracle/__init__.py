@@ -58,6 +58,8 @@ def _load():
                                                        _dp, _dp]
         lib.rat_oracle_recurrence_backward_reset.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _dp,
                                                              _L, _L, _dp, _dp, _dp]
+        lib.rat_oracle_recurrence_window_backward.argtypes = [_L, _L, _L, _dp, _dp, _dp, _dp, _L,
+                                                              _dp, _dp, _dp, _dp, _dp]
         lib.rat_oracle_rope.argtypes = [_L, _L, _L, _dp, _L, ctypes.c_double]
         lib.rat_oracle_in_key_set.argtypes = [_L, _L, _L, _L]
         lib.rat_oracle_in_key_set.restype = ctypes.c_int
@@ -214,6 +216,51 @@ def recurrence_layer_backward(k, v, a, dk_rec, dv_rec, h0k=None, h0v=None, dhTk=
         g = 1.0 / (1.0 + np.exp(-a))
         omg = 1.0 / (1.0 + np.exp(a))
     return dk, dv, g * omg * (dgk + dgv), dh0k, dh0v
+
+
+def recurrence_window_backward(x, a, dy, Lw: int = 64, prev_x=None, prev_a=None):
+    """Reverse-mode derivative of recurrence_window(x, a, Lw, prev_x, prev_a): returns
+    (dx, dg, dprev_x, dprev_g) for upstream gradients dy of the outputs; dg is the gradient with
+    respect to the gate value g = sigmoid(a); dprev_x, dprev_g are the gradients of the history
+    rows (None without them)."""
+    x, a, dy = _f64(x), _f64(a), _f64(dy)
+    assert x.shape == a.shape == dy.shape and int(Lw) >= 1
+    T, d = x.shape[-2], x.shape[-1]
+    BH = int(np.prod(x.shape[:-2])) if x.ndim > 2 else 1
+    dx, dg = np.empty_like(x), np.empty_like(x)
+    px = pa = dpx = dpg = None
+    dprev_x = dprev_g = None
+    if prev_x is not None:
+        prev_x, prev_a = _f64(prev_x), _f64(prev_a)
+        assert prev_x.shape == x.shape[:-2] + (int(Lw), d) and prev_a.shape == prev_x.shape
+        px, pa = _ptr(prev_x), _ptr(prev_a)
+        dprev_x, dprev_g = np.empty_like(prev_x), np.empty_like(prev_x)
+        dpx, dpg = _ptr(dprev_x), _ptr(dprev_g)
+    _load().rat_oracle_recurrence_window_backward(BH, T, d, _ptr(x), _ptr(a), px, pa, int(Lw),
+                                                  _ptr(dy), _ptr(dx), _ptr(dg), dpx, dpg)
+    return dx, dg, dprev_x, dprev_g
+
+
+def recurrence_window_layer_backward(k, v, a, dk_rec, dv_rec, Lw: int = 64, prev_k=None,
+                                     prev_v=None, prev_a=None, pos0: int = 0,
+                                     rope_base: float = 0.0):
+    """Backward of the fixed-window prefill step (k~ = RoPE(y^k), v~ = y^v, one gate for both):
+    returns (dk, dv, da, dprev_k, dprev_v, dprev_a), the last three None without history rows.
+    The gate is shared, so its gradient sums the k and v parts, through dg/da = g (1 - g)."""
+    ek = rope_transpose(dk_rec, pos0, rope_base) if rope_base > 0 else _f64(dk_rec)
+    dk, dgk, dpk, dpgk = recurrence_window_backward(k, a, ek, Lw, prev_k, prev_a)
+    dv, dgv, dpv, dpgv = recurrence_window_backward(v, a, dv_rec, Lw, prev_v, prev_a)
+
+    def dlogit(logit, dgate):
+        logit = _f64(logit)
+        with np.errstate(over="ignore"):    # saturated logits: exp -> inf gives g = 0 or 1
+            g = 1.0 / (1.0 + np.exp(-logit))
+            omg = 1.0 / (1.0 + np.exp(logit))
+        return g * omg * dgate
+
+    da = dlogit(a, dgk + dgv)
+    dpa = dlogit(prev_a, dpgk + dpgv) if prev_k is not None else None
+    return dk, dv, da, dpk, dpv, dpa
 
 
 def in_key_set(t: int, j: int, D: int, W: int, n_sink: int = 0) -> bool:

@@ -176,6 +176,84 @@ void rat_oracle_recurrence_backward(long BH, long T, long d, const double *x, co
 }
 
 /*
+ * Backward of the fixed-window recurrence (rat_oracle_recurrence_window: y_t is the recurrence
+ * restarted from zero at t - Lw + 1), for one of x = k or x = v.  Each output y_t is its own
+ * restarted recurrence over the window W(t) = [max(t - Lw + 1, lo), t] (lo = -Lw with history
+ * rows, else 0), so by the rule of rat_oracle_recurrence_backward applied to that recurrence alone,
+ * with upstream gradient dy_t at its last row and nothing else,
+ *   nu = dy_t at s = t,   then for s = t, t-1, ..., start:
+ *     dL/dx_s += (1 - g_s) nu,   dL/dg_s += nu (h^t_{s-1} - x_s),   nu <- g_s nu,
+ * where h^t is the restarted state (h^t_{start-1} = 0), recomputed for every t.  The sums over t
+ * are the gradients; O(T Lw^2) per channel.  dprev_x / dprev_g ([BH][Lw][d], or NULL) receive
+ * the gradients of the history rows prev_x / prev_a (given only with them).
+ */
+void rat_oracle_recurrence_window_backward(long BH, long T, long d, const double *x,
+                                           const double *a, const double *prev_x,
+                                           const double *prev_a, long Lw, const double *dy,
+                                           double *dx, double *dg, double *dprev_x,
+                                           double *dprev_g)
+{
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        double *hs = (double *)malloc((size_t)(Lw + 1) * sizeof(double));  /* hs[i] = state before row start+i */
+        double *xs = (double *)malloc((size_t)Lw * sizeof(double));
+        double *gs = (double *)malloc((size_t)Lw * sizeof(double));
+        double *os = (double *)malloc((size_t)Lw * sizeof(double));
+        for (long c = 0; c < d; ++c) {
+            for (long t = 0; t < T; ++t) {
+                dx[(bh * T + t) * d + c] = 0.0;
+                dg[(bh * T + t) * d + c] = 0.0;
+            }
+            if (dprev_x)
+                for (long i = 0; i < Lw; ++i) {
+                    dprev_x[(bh * Lw + i) * d + c] = 0.0;
+                    dprev_g[(bh * Lw + i) * d + c] = 0.0;
+                }
+            for (long t = 0; t < T; ++t) {
+                long start = t - Lw + 1;
+                long lo = prev_x ? -Lw : 0;
+                if (start < lo) start = lo;
+                long n = t - start + 1;
+                /* the window's inputs, oldest first, and its restarted forward states */
+                hs[0] = 0.0;
+                for (long i = 0; i < n; ++i) {
+                    long s = start + i;
+                    double xv, av;
+                    if (s >= 0) {
+                        xv = x[(bh * T + s) * d + c];
+                        av = a[(bh * T + s) * d + c];
+                    } else {
+                        xv = prev_x[(bh * Lw + (Lw + s)) * d + c];
+                        av = prev_a[(bh * Lw + (Lw + s)) * d + c];
+                    }
+                    xs[i] = xv;
+                    gs[i] = forget_gate(av);
+                    os[i] = one_minus_gate(av);
+                    hs[i + 1] = gs[i] * hs[i] + os[i] * xv;
+                }
+                double nu = dy[(bh * T + t) * d + c];         /* dL/dh^t_s, from s = t down */
+                for (long i = n - 1; i >= 0; --i) {
+                    long s = start + i;
+                    double ddx = os[i] * nu, ddg = nu * (hs[i] - xs[i]);
+                    if (s >= 0) {
+                        dx[(bh * T + s) * d + c] += ddx;
+                        dg[(bh * T + s) * d + c] += ddg;
+                    } else if (dprev_x) {
+                        dprev_x[(bh * Lw + (Lw + s)) * d + c] += ddx;
+                        dprev_g[(bh * Lw + (Lw + s)) * d + c] += ddg;
+                    }
+                    nu *= gs[i];
+                }
+            }
+        }
+        free(hs);
+        free(xs);
+        free(gs);
+        free(os);
+    }
+}
+
+/*
  * Backward of the chunk-local recurrence (RAT: the state restarts before every absolute
  * position pos0 + t that is a multiple of L; "RAT+ Deep Dive" section 2.1), for one of x = k or
  * x = v.  Forward: hs_t = 0 if (pos0 + t) mod L == 0, else h_{t-1} (h_{-1} = h0), then

@@ -435,6 +435,121 @@ def test_reset_backward_every_position_keeps_only_the_input_term():
     assert np.all(dh0 == 0.0)
 
 
+# ---- backward of the fixed-window recurrence (state restarted from zero at t - Lw + 1)
+def _torch_layer_window(k, v, a, pk, pv, pa, Lw, pos0, base):
+    """The window forward step with torch float64 ops, for autograd: each output row runs its
+    own restarted loop over the window (history rows joined in front when given)."""
+    import torch
+    T, d = k.shape[-2], k.shape[-1]
+    if pk is not None:
+        k, v, a = (torch.cat([p_, x_], -2) for p_, x_ in ((pk, k), (pv, v), (pa, a)))
+        off = Lw
+    else:
+        off = 0
+    g = torch.sigmoid(a)
+    yk, yv = [], []
+    for t in range(T):
+        tt = t + off
+        hk = torch.zeros_like(k[..., 0, :])
+        hv = torch.zeros_like(v[..., 0, :])
+        for s in range(max(tt - Lw + 1, 0), tt + 1):
+            hk = g[..., s, :] * hk + (1 - g[..., s, :]) * k[..., s, :]
+            hv = g[..., s, :] * hv + (1 - g[..., s, :]) * v[..., s, :]
+        yk.append(hk)
+        yv.append(hv)
+    yk, yv = torch.stack(yk, -2), torch.stack(yv, -2)
+    if base > 0:
+        half = d // 2
+        theta = base ** (-2.0 * torch.arange(half, dtype=torch.float64) / d)
+        ang = (pos0 + torch.arange(T, dtype=torch.float64))[:, None] * theta[None, :]
+        c, s_ = torch.cos(ang), torch.sin(ang)
+        y1, y2 = yk[..., :half], yk[..., half:]
+        yk = torch.cat([y1 * c - y2 * s_, y2 * c + y1 * s_], -1)
+    return yk, yv
+
+
+@pytest.mark.parametrize("base,pos0,Lw,hist", [(0.0, 0, 4, False), (10000.0, 37, 5, True),
+                                               (0.0, 0, 1, True), (500.0, 3, 16, False),
+                                               (0.0, 0, 6, True)])
+def test_window_backward_matches_autograd(base, pos0, Lw, hist):
+    import torch
+    shp = (2, 13, 6)
+    k, v, a = (torch.tensor(RNG.standard_normal(shp), requires_grad=True) for _ in range(3))
+    pk = pv = pa = None
+    if hist:
+        pk, pv, pa = (torch.tensor(RNG.standard_normal((2, Lw, 6)), requires_grad=True)
+                      for _ in range(3))
+    dyk, dyv = RNG.standard_normal(shp), RNG.standard_normal(shp)
+    yk, yv = _torch_layer_window(k, v, a, pk, pv, pa, Lw, pos0, base)
+    ((yk * torch.tensor(dyk)).sum() + (yv * torch.tensor(dyv)).sum()).backward()
+    np_ = (lambda t: None if t is None else t.detach().numpy())
+    dk, dv, da, dpk, dpv, dpa = oracle.recurrence_window_layer_backward(
+        np_(k), np_(v), np_(a), dyk, dyv, Lw, np_(pk), np_(pv), np_(pa), pos0=pos0, rope_base=base)
+    pairs = [(dk, k.grad), (dv, v.grad), (da, a.grad)]
+    if hist:
+        pairs += [(dpk, pk.grad), (dpv, pv.grad), (dpa, pa.grad)]
+    else:
+        assert dpk is None and dpv is None and dpa is None
+    for mine, ref in pairs:
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_window_backward_finite_differences():
+    # central differences of L = <dy, y> through the oracle's own window forward, history included
+    T, d, Lw = 11, 3, 4
+    x, a = RNG.standard_normal((1, T, d)), RNG.standard_normal((1, T, d))
+    px, pa = RNG.standard_normal((1, Lw, d)), RNG.standard_normal((1, Lw, d))
+    dy = RNG.standard_normal((1, T, d))
+
+    def L(x_, a_, px_, pa_):
+        return float((oracle.recurrence_window(x_, a_, Lw, px_, pa_) * dy).sum())
+
+    dx, dg, dpx, dpg = oracle.recurrence_window_backward(x, a, dy, Lw, px, pa)
+    sig = lambda z: 1.0 / (1.0 + np.exp(-z))
+    da, dpa = dg * sig(a) * (1 - sig(a)), dpg * sig(pa) * (1 - sig(pa))
+    eps = 1e-6
+    cases = [(x, dx, 0), (a, da, 1), (px, dpx, 2), (pa, dpa, 3)]
+    for arr, grad, slot in cases:
+        for (t, c) in ((0, 0), (1, 2), (arr.shape[1] - 1, 1), (arr.shape[1] // 2, 0)):
+            p_, m_ = arr.copy(), arr.copy()
+            p_[0, t, c] += eps
+            m_[0, t, c] -= eps
+            base_args = [x, a, px, pa]
+            ap, am = list(base_args), list(base_args)
+            ap[slot], am[slot] = p_, m_
+            fd = (L(*ap) - L(*am)) / (2 * eps)
+            assert abs(fd - grad[0, t, c]) <= 1e-7 * max(1.0, abs(fd)), (slot, t, c, fd, grad[0, t, c])
+    # the oldest history row is outside every window of rows 0 .. T-1
+    assert np.all(dpx[:, 0] == 0.0) and np.all(dpg[:, 0] == 0.0)
+
+
+def test_window_backward_longer_than_the_sequence_is_the_full_backward():
+    # Lw >= T and no history: every window starts at row 0, the full-sequence recurrence from 0
+    x, a, dy = (RNG.standard_normal((2, 20, 4)) for _ in range(3))
+    dx, dg, _, _ = oracle.recurrence_window_backward(x, a, dy, Lw=20)
+    fx, fg, _ = oracle.recurrence_backward(x, a, dy)
+    np.testing.assert_allclose(dx, fx, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(dg, fg, rtol=1e-12, atol=1e-14)
+
+
+def test_window_backward_of_one_keeps_only_the_input_term():
+    # Lw = 1: y_t = (1 - g_t) x_t, so dx = (1 - g) dy and dg = -x dy
+    x, a, dy = (RNG.standard_normal((2, 12, 3)) for _ in range(3))
+    dx, dg, _, _ = oracle.recurrence_window_backward(x, a, dy, Lw=1)
+    np.testing.assert_allclose(dx, dy / (1.0 + np.exp(a)), rtol=1e-14, atol=0)
+    np.testing.assert_allclose(dg, -x * dy, rtol=1e-14, atol=0)
+
+
+def test_window_backward_is_the_adjoint_of_the_linear_map():
+    # at fixed gates the window map x -> y is linear: <dy, y(x)> = <dx(dy), x> (+ history part)
+    x, a, dy = (RNG.standard_normal((3, 70, 4)) for _ in range(3))
+    px, pa = RNG.standard_normal((3, 8, 4)), RNG.standard_normal((3, 8, 4))
+    y = oracle.recurrence_window(x, a, 8, px, pa)
+    dx, _, dpx, _ = oracle.recurrence_window_backward(x, a, dy, 8, px, pa)
+    lhs, rhs = float((dy * y).sum()), float((dx * x).sum() + (dpx * px).sum())
+    assert abs(lhs - rhs) <= 1e-12 * max(abs(lhs), 1.0)
+
+
 def test_rope_transpose_inverts_rope():
     x = RNG.standard_normal((2, 11, 8))
     np.testing.assert_allclose(oracle.rope_transpose(oracle.rope(x, 123, 500.0), 123, 500.0), x,
