@@ -706,10 +706,11 @@ def run_decode_paged(w: synthetic.Workload, steps_timed: int, warmup: int, rank:
 
 
 def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, peaks, peak_kind,
-                 reset_every: int = 0):
+                 reset_every: int = 0, window: int = 0):
     """Backward of the recurrence step on the prefill workload: the forward outputs and
     upstream gradients are resident; each timed step is one rat_recur_backward call
-    (rat_recur_backward_local with reset_every = L > 0)."""
+    (rat_recur_backward_local with reset_every = L > 0, rat_recur_backward_window with
+    window = 64, which reads the forward inputs only)."""
     import recurrence_augmented_dilated_b200 as rat
     dev = torch.device("cuda")
     x = synthetic.prefill_inputs(w)
@@ -718,7 +719,9 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     dtc = rat.F32 if w.dtype == "f32" else rat.BF16
     kr, vr = torch.empty_like(k), torch.empty_like(v)
     ws_f = rat.Workspace(rat.rat_recur_workspace_bytes(B, H, T, d, dtc))
-    if reset_every > 0:
+    if window:
+        rat.rat_recur_prefill_window(k, v, a, kr, vr, ws_f, window, rope_base=w.rope_base)
+    elif reset_every > 0:
         rat.rat_recur_prefill_local(k, v, a, kr, vr, ws_f, reset_every, rope_base=w.rope_base)
     else:
         rat.rat_recur_prefill(k, v, a, kr, vr, ws_f, rope_base=w.rope_base)
@@ -730,8 +733,12 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
     stream = torch.cuda.current_stream()
 
     def step():
-        rat.rat_recur_backward(k, v, a, kr, vr, dyk, dyv, dk, dv, da, ws, rope_base=w.rope_base,
-                               reset_every=reset_every)
+        if window:
+            rat.rat_recur_backward_window(k, v, a, dyk, dyv, dk, dv, da, window,
+                                          rope_base=w.rope_base)
+        else:
+            rat.rat_recur_backward(k, v, a, kr, vr, dyk, dyv, dk, dv, da, ws,
+                                   rope_base=w.rope_base, reset_every=reset_every)
 
     with ProfiledRegion():
         for _ in range(warmup):
@@ -749,11 +756,14 @@ def run_backward(w: synthetic.Workload, steps: int, warmup: int, world: int, pea
         torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
     eb = 2 if w.dtype == "bf16" else 4
-    nbytes = 10 * B * H * T * d * eb       # read k, v, a, k~, v~, dk~, dv~; write dk, dv, da
+    # read k, v, a, k~, v~ (not the window form), dk~, dv~; write dk, dv, da
+    nbytes = (8 if window else 10) * B * H * T * d * eb
     achieved = nbytes / (ms * 1e-3) / 1e9
     res = {"workload": w.name, "ms": ms,
-           "step": ("rat_recur_backward_local(L=%d)" % reset_every if reset_every else
-                    "rat_recur_backward") + " (1 launch: scan from the end, decoupled look-back)",
+           "step": ("rat_recur_backward_window(Lw=%d) (1 launch: blocks of Lw rows, no waits)" % window
+                    if window else
+                    ("rat_recur_backward_local(L=%d)" % reset_every if reset_every else
+                     "rat_recur_backward") + " (1 launch: scan from the end, decoupled look-back)"),
            "tokens_per_s": world * B * T / (ms * 1e-3),
            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "of": peak_kind,
@@ -1074,7 +1084,8 @@ def main():
         line["workloads"] = others
     if args.backward:
         line["backward"] = run_backward(w, args.steps, args.warmup, world, peaks, peak_kind,
-                                        reset_every=args.reset_every)
+                                        reset_every=args.reset_every,
+                                        window=args.window if args.window == 64 else 0)
     if args.decode_paged:
         dw = synthetic.WORKLOADS["decode_7p6b"]
         line["decode_paged"] = run_decode_paged(dw, max(1, min(args.steps, 10)), 3, rank, world,

@@ -16,6 +16,7 @@
  *                            positions (RAT+'s L*).
  *   rat_recur_backward       gradients of rat_recur_prefill's step.
  *   rat_recur_backward_local gradients of rat_recur_prefill_local's step.
+ *   rat_recur_backward_window gradients of rat_recur_prefill_window's step.
  *   rat_dilated_attn_prefill causal attention of each query t over
  *                              S(t) = { t-We < j <= t }  U  { j <= t-We : j mod D = D-1 },
  *                            We = max(W, 1), D per head; optional RoPE on q.
@@ -234,6 +235,39 @@ RAT_API int rat_recur_prefill_window(const void *k, const void *v, const void *g
                              void *k_rec, void *v_rec, int B, int H, int T, int d, int dtype,
                              int64_t pos0, int64_t Lw, float rope_base,
                              void *ws, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------
+ * rat_recur_backward_window -- gradients of rat_recur_prefill_window's step (the fixed-window
+ * recurrence, "RAT+ Deep Dive" section 2.1, L* = 64), for training in that form.
+ *   Each output y_t is the recurrence restarted from zero at t - Lw + 1, so the gradient sums,
+ *   over the Lw outputs whose windows hold a row, the reverse pass of each restarted recurrence:
+ *     dL/dx_s = (1 - g_s) sum_{t=s}^{s+Lw-1} e_t prod_{r=s+1}^{t} g_r,
+ *     dL/dg_s = sum_{t=s}^{s+Lw-1} e_t prod_{r=s+1}^{t} g_r (h^t_{s-1} - x_s),
+ *   h^t the state restarted at t - Lw + 1 (h^t_{t-Lw} = 0), e^k_t = RoPE_t^T(dk~_t),
+ *   e^v_t = dv~_t, dgate_logit = g (1 - g) (dg^k + dg^v).  Computed in blocks of Lw rows with
+ *   products of one block's gates only (no division by a gate, no subtraction of older states).
+ *
+ *   k, v, gate_logit : device, (B, H, T, d) of dtype          the forward inputs
+ *   prev_k, prev_v, prev_gate_logit
+ *                    : device, (B, H, Lw, d) of dtype, or all three NULL: the forward's history
+ *                      rows
+ *   dk_rec, dv_rec   : device, (B, H, T, d) of dtype          upstream gradients of k~, v~
+ *   dk, dv, dgate_logit : device, (B, H, T, d) of dtype       outputs
+ *   dprev_k, dprev_v, dprev_gate_logit
+ *                    : device, (B, H, Lw, d) of dtype, or all three NULL: gradients of the history
+ *                      rows (only with them; the oldest row gets 0, no window of rows 0.. holds it)
+ *   pos0, Lw, rope_base : as given to the forward (Lw = 64, RAT_ERR_UNSUPPORTED otherwise)
+ * float32 arithmetic; bf16 outputs rounded once.  The forward outputs are not needed (the block
+ * states are recomputed from the inputs).  Outputs may not alias inputs.  T = 0 is a no-op.  One
+ * launch; no CTA waits for another, so the call needs no workspace and records no device error.
+ * ---------------------------------------------------------------------------------------- */
+RAT_API int rat_recur_backward_window(const void *k, const void *v, const void *gate_logit,
+                              const void *prev_k, const void *prev_v,
+                              const void *prev_gate_logit, const void *dk_rec,
+                              const void *dv_rec, void *dk, void *dv, void *dgate_logit,
+                              void *dprev_k, void *dprev_v, void *dprev_gate_logit, int B, int H,
+                              int T, int d, int dtype, int64_t pos0, int64_t Lw, float rope_base,
+                              void *stream);
 
 /* ------------------------------------------------------------------------------------------
  * rat_dilated_attn_prefill -- causal dilated attention with an optional local window and a

@@ -23,6 +23,7 @@ __all__ = [
     "RatError", "lib", "library_path", "F32", "BF16", "KVCache",
     "rat_recur_workspace_bytes", "rat_recur_prefill", "rat_recur_prefill_local",
     "rat_recur_prefill_window", "rat_recur_backward", "rat_recur_backward_local",
+    "rat_recur_backward_window",
     "rat_recur_backward_workspace_bytes",
     "rat_dilated_attn_backward", "rat_dilated_attn_backward_workspace_bytes",
     "rat_dilated_attn_prefill",
@@ -124,6 +125,8 @@ def lib():
                                                             _vp, _sz, _vp]
         L.rat_recur_prefill_window.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                _i, _i, _i, _i, _i, _i64, _i64, _f, _vp, _sz, _vp]
+        L.rat_recur_backward_window.argtypes = [_vp] * 14 + [_i, _i, _i, _i, _i, _i64, _i64, _f,
+                                                             _vp]
         L.rat_recur_prefill_local.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                               _i, _i, _i, _i, _i, _i64, _i64, _f, _vp, _sz, _vp]
         L.rat_dilated_attn_prefill.argtypes = [_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i,
@@ -292,6 +295,22 @@ def rat_recur_prefill_window(k, v, gate_logit, k_rec, v_rec, ws: Workspace, Lw: 
                                         int(Lw), float(rope_base), ws.ptr, ws.nbytes,
                                         _stream(stream))
     _check("rat_recur_prefill_window", st)
+
+
+def rat_recur_backward_window(k, v, gate_logit, dk_rec, dv_rec, dk, dv, dgate_logit,
+                              Lw: int = 64, prev_k=None, prev_v=None, prev_gate_logit=None,
+                              dprev_k=None, dprev_v=None, dprev_gate_logit=None, pos0: int = 0,
+                              rope_base: float = 0.0, stream=None):
+    """Gradients of the fixed-window recurrence step: dk, dv, dgate_logit (all (B, H, T, d))
+    and, with history rows, optionally dprev_k, dprev_v, dprev_gate_logit ((B, H, Lw, d))."""
+    B, H, T, d = k.shape
+    st = lib().rat_recur_backward_window(_ptr(k), _ptr(v), _ptr(gate_logit), _ptr(prev_k),
+                                         _ptr(prev_v), _ptr(prev_gate_logit), _ptr(dk_rec),
+                                         _ptr(dv_rec), _ptr(dk), _ptr(dv), _ptr(dgate_logit),
+                                         _ptr(dprev_k), _ptr(dprev_v), _ptr(dprev_gate_logit),
+                                         B, H, T, d, _dtype_code(k), int(pos0), int(Lw),
+                                         float(rope_base), _stream(stream))
+    _check("rat_recur_backward_window", st)
 
 
 def rat_dilated_attn_prefill(q, k_rec, v_rec, o, D: int = 1, W: int = 0,

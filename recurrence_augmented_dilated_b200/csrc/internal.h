@@ -63,6 +63,23 @@ struct WindowParams {
 };
 int launch_window(const WindowParams &p, int dtype, void *stream);
 
+// backward of the fixed-window recurrence (one launch, no waits between CTAs)
+struct WindowBwdParams {
+    const void *k, *v, *a;          // forward inputs
+    const void *pk, *pv, *pa;       // [BH][kWindowRows][d] history rows, or all null
+    const void *dyk, *dyv;          // upstream gradients of k~, v~
+    void *dk, *dv, *da;             // outputs
+    void *dpk, *dpv, *dpa;          // gradients of the history rows, or all null
+    int BH, T, d, nblk;             // nblk = ceil(T / kWindowRows)
+    long long pos0;
+    int rope, rope_f32;
+    float theta_f[64];
+    double theta[64];
+    float step_cos[64], step_sin[64];
+    float step64_cos[64], step64_sin[64];   // rotation by kWindowRows positions
+};
+int launch_window_bwd(const WindowBwdParams &p, int dtype, void *stream);
+
 // backward of the recurrence step (reduce, carry and output launches over 64-row chunks)
 struct RecurBwdParams {
     const void *k, *v, *a;          // forward inputs

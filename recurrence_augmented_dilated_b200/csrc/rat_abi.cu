@@ -324,6 +324,54 @@ int rat_recur_prefill_window(const void *k, const void *v, const void *gate_logi
     return launch_window(p, dtype, stream);
 }
 
+int rat_recur_backward_window(const void *k, const void *v, const void *gate_logit,
+                              const void *prev_k, const void *prev_v,
+                              const void *prev_gate_logit, const void *dk_rec,
+                              const void *dv_rec, void *dk, void *dv, void *dgate_logit,
+                              void *dprev_k, void *dprev_v, void *dprev_gate_logit, int B, int H,
+                              int T, int d, int dtype, int64_t pos0, int64_t Lw, float rope_base,
+                              void *stream) {
+    if (B < 1 || H < 1 || T < 0 || !valid_dtype(dtype) || Lw < 1) return RAT_ERR_INVALID;
+    if (!supported_d(d) || Lw != kWindowRows) return RAT_ERR_UNSUPPORTED;
+    if (pos0 < 0 || !std::isfinite(rope_base)) return RAT_ERR_INVALID;
+    const int nprev = (prev_k != nullptr) + (prev_v != nullptr) + (prev_gate_logit != nullptr);
+    const int ndprev = (dprev_k != nullptr) + (dprev_v != nullptr) + (dprev_gate_logit != nullptr);
+    if ((nprev != 0 && nprev != 3) || (ndprev != 0 && ndprev != 3) || (ndprev && !nprev))
+        return RAT_ERR_INVALID;
+    if (T == 0) return RAT_OK;
+    if (!k || !v || !gate_logit || !dk_rec || !dv_rec || !dk || !dv || !dgate_logit)
+        return RAT_ERR_INVALID;
+    const void *ptrs[] = {k, v, gate_logit, dk_rec, dv_rec, dk, dv, dgate_logit, prev_k, prev_v,
+                          prev_gate_logit, dprev_k, dprev_v, dprev_gate_logit};
+    for (const void *q : ptrs)
+        if (q && !aligned16(q)) return RAT_ERR_INVALID;
+    if ((long long)B * H * T > (1ll << 40) || (long long)B * H * (d / 32) * (T / kWindowRows + 2) >= (1ll << 31))
+        return RAT_ERR_UNSUPPORTED;
+    WindowBwdParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.k = k; p.v = v; p.a = gate_logit;
+    p.pk = prev_k; p.pv = prev_v; p.pa = prev_gate_logit;
+    p.dyk = dk_rec; p.dyv = dv_rec;
+    p.dk = dk; p.dv = dv; p.da = dgate_logit;
+    p.dpk = dprev_k; p.dpv = dprev_v; p.dpa = dprev_gate_logit;
+    p.BH = B * H; p.T = T; p.d = d;
+    p.nblk = (T + kWindowRows - 1) / kWindowRows;
+    p.pos0 = pos0;
+    p.rope = rope_base > 0.f ? 1 : 0;
+    if (p.rope) {
+        rope_theta(rope_base, d, p.theta);
+        for (int c = 0; c < 64; ++c) {
+            p.theta_f[c] = (float)p.theta[c];
+            p.step_cos[c] = (float)std::cos(p.theta[c]);
+            p.step_sin[c] = (float)std::sin(p.theta[c]);
+            p.step64_cos[c] = (float)std::cos(kWindowRows * p.theta[c]);
+            p.step64_sin[c] = (float)std::sin(kWindowRows * p.theta[c]);
+        }
+        p.rope_f32 = (dtype == RAT_BF16 && pos0 + (int64_t)T <= 8192) ? 1 : 0;
+    }
+    return launch_window_bwd(p, dtype, stream);
+}
+
 int rat_recur_prefill_local(const void *k, const void *v, const void *gate_logit,
                             const float *h0_k, const float *h0_v, void *k_rec, void *v_rec,
                             float *hT_k, float *hT_v, int B, int H, int T, int d, int dtype,

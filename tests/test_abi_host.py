@@ -106,6 +106,29 @@ def test_local_and_window_validation(L):
     assert L.rat_recur_prefill_window(*args(64, T=0)) == 0
 
 
+def test_window_backward_validation(L):
+    P = ctypes.c_void_p
+    three = (P(256), P(512), P(768))
+    bargs = lambda Lw=64, prev=(None, None, None), dprev=(None, None, None), T=8, d=128, dt=1, \
+        pos0=0, out=P(1024): (P(256), P(256), P(256), *prev, P(256), P(256), out, P(256), P(256),
+                              *dprev, 1, 1, T, d, dt, pos0, Lw, 0.0, None)
+    assert L.rat_recur_backward_window(*bargs(Lw=0)) == -1
+    assert L.rat_recur_backward_window(*bargs(Lw=32)) == -2
+    assert L.rat_recur_backward_window(*bargs(d=96)) == -2
+    assert L.rat_recur_backward_window(*bargs(dt=7)) == -1
+    assert L.rat_recur_backward_window(*bargs(pos0=-1)) == -1
+    # history rows and their gradients: all three or none; gradients only with the rows
+    assert L.rat_recur_backward_window(*bargs(prev=(P(256), None, None))) == -1
+    assert L.rat_recur_backward_window(*bargs(dprev=three)) == -1
+    assert L.rat_recur_backward_window(*bargs(prev=three, dprev=(P(256), P(256), None))) == -1
+    # misaligned or missing output
+    assert L.rat_recur_backward_window(*bargs(out=P(1032))) == -1
+    assert L.rat_recur_backward_window(*bargs(out=None)) == -1
+    assert L.rat_recur_backward_window(*bargs(prev=three, dprev=(P(256), P(264), P(256)))) == -1
+    # T == 0 is a no-op (no pointer is read)
+    assert L.rat_recur_backward_window(*bargs(T=0, out=None)) == 0
+
+
 def test_empty_inputs_are_no_ops(L):
     # T = 0: every entry point returns RAT_OK before touching a pointer or the GPU
     P = ctypes.c_void_p
