@@ -85,6 +85,20 @@ def test_window_backward_history_rows_and_rope(dtype, want_dprev, T, pos0):
             assert torch.count_nonzero(t[:, :, 0]).item() == 0
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("d", [64, 128])
+def test_window_backward_history_gradients_many_ranges(dtype, d):
+    # B 3 x H 5 x (blocks -1 .. 20) x slices: more items than CTAs, so ranges start inside a
+    # (b, h), on its history block and right after it; no RoPE, and RoPE at positions past the
+    # float32-angle bound
+    for pos0, base in ((0, 0.0), (9000, 10000.0)):
+        x = inputs(3, 5, 1300, d, dtype, seed=40 + d + pos0)
+        p = inputs(3, 5, 64, d, dtype, seed=41 + d + pos0)
+        dyk, dyv = grads(3, 5, 1300, d, dtype, seed=42 + d + pos0)
+        check(x, dyk, dyv, prev=(p["k"], p["v"], p["a"]), want_dprev=True, pos0=pos0,
+              rope_base=base)
+
+
 def test_window_backward_two_calls_equal_one():
     # a sequence cut in two, the second call given the last 64 rows of the first as history:
     # the second call's history gradients add to the first call's last 64 rows
