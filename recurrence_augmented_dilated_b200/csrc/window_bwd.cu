@@ -32,14 +32,16 @@
 // from one extra block at its start, and Lam of a range's last block from the next block's a,
 // dk~, dv~.  No CTA waits for another.
 //
-// Per block, 32 segments of 2 rows; a lane holds two channel pairs of a row pair (a pair and its
+// Per block, 16 segments of 4 rows; a lane holds two channel pairs of its rows (a pair and its
 // RoPE partner), so the transposed rotation of dk~ needs nothing from other lanes:
 //   1. each lane forms its segment's aggregates: the next block's gate product and its sum of
 //      e P (for Lam), this block's gate product, local F, Y driven by the segment's own part of
 //      Lam, and the local reverse sums of mu and rho;
-//   2. one thread per channel walks the 32 segments forwards (Lam, P, F, Y entering each
-//      segment, and E), another backwards (D, mu, rho entering from the right);
-//   3. each lane finishes its rows: dk, dv, da, and U of this block for the next one.
+//   2. four walks over the 16 segments, one thread per channel each: forwards for k and for v
+//      (Lam, P, F, Y entering each segment, and E), backwards for k and for v (D and the mu, rho
+//      carries entering from the right);
+//   3. each lane finishes its rows: dk, dv, da, and U of this block for the next one (kept in
+//      registers, like the next block's gates, which the look-ahead forms once for both uses).
 // Data movement: per block the slices of a, dk~, dv~ and of k, v arrive by cp.async in two
 // rings (three and two stages), issued three and two blocks ahead; the next block's a, dk~, dv~
 // serve as this block's look-ahead and then as the next block's own data.  HBM traffic: five
