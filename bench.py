@@ -965,7 +965,9 @@ def main():
     ap.add_argument("--decode-paged", action="store_true",
                     help="also time ragged decode (context lengths T/2 .. T) on a paged cache")
     ap.add_argument("--backward", action="store_true",
-                    help="also time the backward of the recurrence step on the workload")
+                    help="also time the backward of the recurrence step on the workload (of the "
+                         "chunk-local form with --reset-every, of the window form with "
+                         "--window 64) and of the attention")
     ap.add_argument("--sinks", type=int, default=0,
                     help="n > 0: the first n positions join every key set (attention sinks)")
     ap.add_argument("--top-k", type=int, default=0,
