@@ -51,9 +51,9 @@ struct WinCfg {
     static constexpr int HALFB = ROWB / 2;
     static constexpr int TILEB = LW * ROWB;             // one tensor of one block
     static constexpr int STAGEB = 3 * TILEB;            // a, k, v
-    // [SEGS + 1][3][DH] aggregates -> exclusive prefixes (+ block total), [SEGS][DH] suffix
-    // gate products
-    static constexpr int XB = (SEGS + 1) * 3 * DH * 4 + SEGS * DH * 4;
+    // [SEGS + 1][3][DH] aggregates -> exclusive prefixes of Bk, Bv (+ block totals), [SEGS][DH]
+    // suffix gate products, [SEGS][DH] prefix gate products
+    static constexpr int XB = (SEGS + 1) * 3 * DH * 4 + 2 * SEGS * DH * 4;
     static constexpr int FIT = (200 * 1024 - XB) / STAGEB;
     static constexpr int NST = FIT >= 3 ? 3 : (FIT >= 1 ? FIT : 1);   // stages in the ring
     static constexpr int SMEM = NST * STAGEB + XB;
@@ -122,6 +122,7 @@ window_kernel(const __grid_constant__ WindowParams p) {
     const int chq[NP] = {2 * cl, 2 * cl + HALF};                // first channel of each pair
     float *X = reinterpret_cast<float *>(smem + C::NST * C::STAGEB);   // [SEGS + 1][3][DH]
     float *S = X + (C::SEGS + 1) * 3 * DH;                            // [SEGS][DH]
+    float *Pt = S + C::SEGS * DH;                                     // [SEGS][DH]
     const long long total = (long long)p.BH * p.nblk;
     const long long f0 = total * blockIdx.x / gridDim.x;
     const long long f1 = total * (blockIdx.x + 1) / gridDim.x;
@@ -218,49 +219,48 @@ window_kernel(const __grid_constant__ WindowParams p) {
         }
         __syncthreads();
 
-        // ---- one thread per channel: product of the gates of the segments after s into S,
-        // exclusive prefixes (segments before s) over X in place, the block total in X[SEGS]
-        if (tid < DH) {
-            const int ch = tid;
+        // ---- three walks over the segments, one thread per channel each: the product of the
+        // gates of the segments after s into S; the gates before s into Pt with the exclusive
+        // prefix of Bk over X in place; the exclusive prefix of Bv; block totals in X[SEGS]
+        // (A is only read, so the walks run side by side)
+        if (tid < 3 * DH) {
+            const int w = tid / DH, ch = tid % DH;
             constexpr int GS = DH == 128 ? 8 : 4;      // segments loaded ahead of the chain
-            float sA = 1.f;
+            if (w == 2) {
+                float sA = 1.f;
 #pragma unroll 1
-            for (int g0 = C::SEGS - GS; g0 >= 0; g0 -= GS) {
-                float xa[GS];
+                for (int g0 = C::SEGS - GS; g0 >= 0; g0 -= GS) {
+                    float xa[GS];
 #pragma unroll
-                for (int u = 0; u < GS; ++u) xa[u] = X[(g0 + u) * 3 * DH + ch];
+                    for (int u = 0; u < GS; ++u) xa[u] = X[(g0 + u) * 3 * DH + ch];
 #pragma unroll
-                for (int u = GS - 1; u >= 0; --u) {
-                    S[(g0 + u) * DH + ch] = sA;
-                    sA *= xa[u];
+                    for (int u = GS - 1; u >= 0; --u) {
+                        S[(g0 + u) * DH + ch] = sA;
+                        sA *= xa[u];
+                    }
                 }
-            }
-            float pA = 1.f, pK = 0.f, pV = 0.f;
+            } else {
+                const int off = w ? 2 * DH : DH;       // Bk or Bv
+                float pA = 1.f, pB = 0.f;
 #pragma unroll 1
-            for (int g0 = 0; g0 < C::SEGS; g0 += GS) {
-                float xa[GS], xk[GS], xv[GS];
+                for (int g0 = 0; g0 < C::SEGS; g0 += GS) {
+                    float xa[GS], xb[GS];
 #pragma unroll
-                for (int u = 0; u < GS; ++u) {
-                    const float *x = X + (g0 + u) * 3 * DH + ch;
-                    xa[u] = x[0];
-                    xk[u] = x[DH];
-                    xv[u] = x[2 * DH];
-                }
+                    for (int u = 0; u < GS; ++u) {
+                        const float *x = X + (g0 + u) * 3 * DH + ch;
+                        xa[u] = x[0];
+                        xb[u] = x[off];
+                    }
 #pragma unroll
-                for (int u = 0; u < GS; ++u) {
-                    float *x = X + (g0 + u) * 3 * DH + ch;
-                    x[0] = pA;
-                    x[DH] = pK;
-                    x[2 * DH] = pV;
-                    pK = fmaf(xa[u], pK, xk[u]);
-                    pV = fmaf(xa[u], pV, xv[u]);
-                    pA *= xa[u];
+                    for (int u = 0; u < GS; ++u) {
+                        if (w == 0) Pt[(g0 + u) * DH + ch] = pA;
+                        X[(g0 + u) * 3 * DH + ch + off] = pB;
+                        pB = fmaf(xa[u], pB, xb[u]);
+                        pA *= xa[u];
+                    }
                 }
+                X[C::SEGS * 3 * DH + ch + off] = pB;
             }
-            float *x = X + C::SEGS * 3 * DH + ch;
-            x[0] = pA;
-            x[DH] = pK;
-            x[2 * DH] = pV;
         }
         __syncthreads();
 
@@ -281,7 +281,7 @@ window_kernel(const __grid_constant__ WindowParams p) {
 #pragma unroll
         for (int q = 0; q < NP; ++q) {
             const float *x = X + seg * 3 * DH + chq[q];
-            Pp[q] = f2(x[0], x[1]);
+            Pp[q] = f2(Pt[seg * DH + chq[q]], Pt[seg * DH + chq[q] + 1]);
             Fk[q] = f2(x[DH], x[DH + 1]);
             Fv[q] = f2(x[2 * DH], x[2 * DH + 1]);
             const float *e = X + C::SEGS * 3 * DH + chq[q];
